@@ -1,0 +1,72 @@
+"""Dense-masked formulation of the MoE layer, in NumPy float64, for tiny shapes.
+
+TEST INFRASTRUCTURE (see ``oracle/__init__.py``).
+
+A second, structurally different algorithm used to pin the C oracle: the
+weights are dequantised in full, *every* expert is applied to *every* token
+with batched ``einsum`` contractions, and the routing enters only as a dense
+[T, E] weight matrix that is zero outside each token's selected experts.  The
+C oracle instead routes first and evaluates only the selected experts, one
+token at a time.  Both follow the formulas stated in ``moe_oracle.c``'s header
+(sigmoid+bias router of the Colibri-Nano model card "Architecture" and the
+colibri README "What's implemented"; per-row int4 with f32 scales of the
+nanocolibri-engine README "Converting a checkpoint yourself").
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import _np, bf16_bits_to_f64
+
+
+def decode_int4(packed: np.ndarray) -> np.ndarray:
+    """Packed bytes [..., n/2] -> int codes [..., n] (low nibble = even element)."""
+    p = packed.astype(np.int16)
+    lo = p & 0xF
+    hi = (p >> 4) & 0xF
+    codes = np.empty(packed.shape[:-1] + (2 * packed.shape[-1],), np.int16)
+    codes[..., 0::2] = np.where(lo >= 8, lo - 16, lo)
+    codes[..., 1::2] = np.where(hi >= 8, hi - 16, hi)
+    return codes
+
+
+def _sigmoid(z):
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def routing_matrix(x: np.ndarray, W: np.ndarray, bias: np.ndarray, K: int, scale: float):
+    """Dense routing weights R [T,E]: R[t,e] = w[t,k] if e = e_k, else 0."""
+    s = _sigmoid(x @ W.T.astype(np.float64))
+    key = s + bias.astype(np.float64)[None, :]
+    key = np.where(np.isnan(key), -np.inf, key)
+    T, E = s.shape
+    R = np.zeros((T, E))
+    for t in range(T):
+        order = np.argsort(-key[t], kind="stable")  # equal keys keep index order
+        sel = order[:K]
+        R[t, sel] = scale * s[t, sel] / s[t, sel].sum()
+    return R
+
+
+def moe_dense(x, layer: dict, shape, residual: bool = False):
+    """Layer output [T,H] in float64.  x: bf16 [T,H] (torch) or bf16 bits."""
+    xf = bf16_bits_to_f64(x)
+    E, K, I, Is = shape.E, shape.K, shape.I, shape.Is
+    R = routing_matrix(xf, _np(layer["router_w"], np.float64), _np(layer["router_bias"], np.float64),
+                       K, shape.routed_scaling)
+    W13 = decode_int4(_np(layer["w13"], np.uint8)) * _np(layer["s13"], np.float64)[..., None]
+    W2 = decode_int4(_np(layer["w2"], np.uint8)) * _np(layer["s2"], np.float64)[..., None]
+    G = np.einsum("th,eih->tei", xf, W13[:, :I])
+    U = np.einsum("th,eih->tei", xf, W13[:, I:])
+    Hh = G * _sigmoid(G) * U
+    Y = np.einsum("tei,eji->tej", Hh, W2)
+    out = np.einsum("te,tej->tj", R, Y)
+    if Is > 0:
+        S13 = decode_int4(_np(layer["sh_w13"], np.uint8)) * _np(layer["sh_s13"], np.float64)[:, None]
+        S2 = decode_int4(_np(layer["sh_w2"], np.uint8)) * _np(layer["sh_s2"], np.float64)[:, None]
+        g = xf @ S13[:Is].T
+        u = xf @ S13[Is:].T
+        out = out + (g * _sigmoid(g) * u) @ S2.T
+    if residual:
+        out = out + xf
+    return out, R
