@@ -1,0 +1,511 @@
+#!/usr/bin/env python3
+"""Benchmark of the int4 expert-FFN MoE layer forward (sigmoid+bias router,
+top-k, int4 SwiGLU experts, shared expert, weighted combine) on B200.
+
+Default workload: the Nano decode stack -- 23 stacked MoE layers (hidden 1024,
+64 experts, top-2, routed intermediate 512, shared intermediate 2048), each
+layer adding its input (x_{l+1} = x_l + MoE_l(x_l)), at T=64 tokens, with the
+decode sweep T in {1,4,16,64} reported beside it.  One step = one pass of the
+whole layer stack over one batch of synthetic tokens.  The metric counts one
+token passing through one MoE layer as one token (tokens/s = T*layers/s).
+
+Timing: W warm-up steps, then exactly K timed steps bracketed by a barrier
+and a device synchronize; each step is timed with CUDA events on the stream
+that runs it, and L2 is flushed (a 256 MiB write) between steps, outside the
+timed events.  Four different input batches rotate, so the routing changes
+from step to step.  The step is replayed as a CUDA graph of the library's
+C-ABI calls.  A second, instrumented pass records the library's per-stage
+events to time each kernel; the roofline uses that per-kernel time.
+
+--impl reference times the CPU oracle (plain C, double precision, one core)
+on a bounded sample of the same workload.
+
+Multi-GPU (torchrun, N>1): independent replicas, one per GPU, no collective on
+the data path (the layer has no exchange step); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "MoE-layer tokens/s; achieved HBM GB/s (decode) and TFLOPS (prefill) vs roofline"
+UNIT = "tokens/s"
+FLUSH_BYTES = 256 << 20
+N_BATCHES = 4
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="nano_decode_stack", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=None, help="T (default: the workload's largest)")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the per-T sweep of the decode stack")
+    ap.add_argument("--no-graph", action="store_true", help="launch the C-ABI calls directly")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------- peaks
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- work accounting
+
+def step_bytes_flops(shape, T, uniq_per_layer):
+    """Algorithmic bytes and flops of one pass over the layers.
+
+    bytes: router W + bias, shared-expert weights + scales, every touched
+    routed expert's weights + scales, x in and out (bf16).  Scratch excluded.
+    flops: 2*T*E*H + 6*T*K*H*I + 6*T*H*Is per layer."""
+    lb = workloads.layer_weight_bytes(shape)
+    H, E, K, I, Is = shape.H, shape.E, shape.K, shape.I, shape.Is
+    nbytes = 0
+    for u in uniq_per_layer:
+        nbytes += lb["router"] + lb["shared"] + u * lb["expert"] + 2 * T * H * 2
+    flops = len(uniq_per_layer) * (2 * T * E * H + 6 * T * K * H * I + 6 * T * H * Is)
+    return nbytes, flops
+
+
+def gate_up_bytes(shape, T, uniq):
+    """Algorithmic bytes of one gate/up launch: the w13 codes + scales of every
+    touched routed expert and of the shared expert, x read once, h written."""
+    H, K, I, Is = shape.H, shape.K, shape.I, shape.Is
+    per_expert = 2 * I * H // 2 + 2 * I * 4
+    shared = (2 * Is * H // 2 + 2 * Is * 4) if Is else 0
+    return uniq * per_expert + shared + T * H * 2 + T * K * I * 2 + T * Is * 2
+
+
+def down_bytes(shape, T, uniq):
+    H, K, I, Is = shape.H, shape.K, shape.I, shape.Is
+    per_expert = H * I // 2 + H * 4
+    shared = (H * Is // 2 + H * 4) if Is else 0
+    return uniq * per_expert + shared + T * K * I * 2 + T * Is * 2 + (T * K + (T if Is else 0)) * H * 4
+
+
+# --------------------------------------------------------------------------- our arm
+
+class Stack:
+    """Device weights of the workload's layers and the buffers of one T."""
+
+    def __init__(self, moe, wl, T, device, layers=None):
+        self.moe, self.wl, self.T, self.device = moe, wl, T, device
+        self.shape = wl.shape
+        self.layers = layers if layers is not None else [
+            workloads.make_layer(wl.shape, wl.wid, l, device, wl.bias_mode) for l in range(wl.layers)]
+        self.xs = [workloads.make_x(wl.shape, T, wl.wid, batch=b, device=device) for b in range(N_BATCHES)]
+        self.acts = [torch.empty((T, wl.shape.H), dtype=torch.bfloat16, device=device) for _ in range(wl.layers)]
+        self.ws = moe.new_workspace(wl.shape, T, device)
+        self.flags = moe.MOE_ADD_RESIDUAL if wl.residual else 0
+
+    def run(self, b, stage_events=None, x=None):
+        inp = self.xs[b] if x is None else x
+        for l, layer in enumerate(self.layers):
+            ev = None if stage_events is None else stage_events[l]
+            self.moe.layer_forward(inp, layer, self.shape, out=self.acts[l], workspace=self.ws,
+                                   flags=self.flags, stage_events=ev)
+            inp = self.acts[l]
+        return inp
+
+    def routing_unique(self):
+        """Touched routed experts per (batch, layer), from the library's top-k output."""
+        K = self.shape.K
+        idx = torch.empty((self.T, K), dtype=torch.int32, device=self.device)
+        out = []
+        for b in range(N_BATCHES):
+            inp, per = self.xs[b], []
+            for l, layer in enumerate(self.layers):
+                self.moe.layer_forward(inp, layer, self.shape, out=self.acts[l], workspace=self.ws,
+                                       flags=self.flags, topk_idx=idx)
+                per.append(int(torch.unique(idx).numel()))
+                inp = self.acts[l]
+            out.append(per)
+        torch.cuda.synchronize()
+        return out
+
+
+def make_events(n):
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in evs:
+        e.record()
+    return evs
+
+
+def timed_steps(stack, steps, warmup, use_graph, flush, instrumented=False, dist_barrier=None):
+    """Returns (per-step ms list, per-stage ms sums per step, launches per step)."""
+    L = len(stack.layers)
+    stage_ev = [make_events(8) for _ in range(L)] if instrumented else None
+    torch.cuda.synchronize()
+    graphs = None
+    if use_graph:
+        graphs = []
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for b in range(N_BATCHES):  # eager warm-up before capture
+                stack.run(b, stage_ev)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        for b in range(N_BATCHES):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                stack.run(b, stage_ev)
+            graphs.append(g)
+        torch.cuda.synchronize()
+
+    def one(b):
+        if graphs is not None:
+            graphs[b].replay()
+        else:
+            stack.run(b, stage_ev)
+
+    for i in range(warmup):
+        flush.zero_()
+        one(i % N_BATCHES)
+    torch.cuda.synchronize()
+    if dist_barrier:
+        dist_barrier()
+    torch.cuda.synchronize()
+    st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    step_ms, stage_ms = [], []
+    for i in range(steps):
+        flush.zero_()
+        st[i].record()
+        one(i % N_BATCHES)
+        en[i].record()
+        if instrumented:
+            en[i].synchronize()
+            stage_ms.append([sum(stage_ev[l][2 * s].elapsed_time(stage_ev[l][2 * s + 1]) for l in range(L))
+                             for s in range(4)])
+    torch.cuda.synchronize()
+    if dist_barrier:
+        dist_barrier()
+    torch.cuda.synchronize()
+    step_ms = [st[i].elapsed_time(en[i]) for i in range(steps)]
+    del graphs
+    return step_ms, stage_ms
+
+
+def e2e_steps(stack, steps, warmup, flush, dist_barrier=None):
+    """Same step through the public API with host buffers: pinned host x ->
+    device, the layer stack (graph of C-ABI calls), device -> pinned host out."""
+    T, H = stack.T, stack.shape.H
+    host_x = [stack.xs[b].cpu().pin_memory() for b in range(N_BATCHES)]
+    host_out = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(stack.xs[0])
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        stack.run(0, x=x_dev)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        out_dev = stack.run(0, x=x_dev)
+    torch.cuda.synchronize()
+
+    def one(b):
+        x_dev.copy_(host_x[b], non_blocking=True)
+        g.replay()
+        host_out.copy_(out_dev, non_blocking=True)
+
+    for i in range(warmup):
+        flush.zero_()
+        one(i % N_BATCHES)
+    torch.cuda.synchronize()
+    if dist_barrier:
+        dist_barrier()
+    st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        st[i].record()
+        one(i % N_BATCHES)
+        en[i].record()
+    torch.cuda.synchronize()
+    if dist_barrier:
+        dist_barrier()
+    ms = [st[i].elapsed_time(en[i]) for i in range(steps)]
+    del g
+    return ms, T * H * 2, T * H * 2
+
+
+def cpu_baseline_sample(stack, budget_s=20.0):
+    """The oracle (single-threaded C, f64) on a bounded sample of the step:
+    the first tokens of batch 0 through every layer, each layer fed the GPU's
+    bf16 input of that layer.  Returns tokens/s (token-layers) and the sample."""
+    import oracle
+    shape = stack.shape
+    with torch.no_grad():
+        inputs = [stack.xs[0]]
+        stack.run(0)
+        inputs += stack.acts[:-1]
+        inputs = [t.cpu() for t in inputs]
+    layers_cpu = [{k: v.cpu() for k, v in layer.items()} for layer in stack.layers]
+    n_tok = stack.T
+    # calibrate on one token of layer 0, then size the sample to the budget
+    t0 = time.perf_counter()
+    oracle.moe_tokens(inputs[0], layers_cpu[0], shape, residual=stack.wl.residual, tokens=[0])
+    per = max(time.perf_counter() - t0, 1e-4)
+    n_tok = int(max(1, min(stack.T, budget_s / (per * len(layers_cpu)))))
+    toks = list(range(n_tok))
+    t0 = time.perf_counter()
+    for l, layer in enumerate(layers_cpu):
+        oracle.moe_tokens(inputs[l], layer, shape, residual=stack.wl.residual, tokens=toks)
+    dt = time.perf_counter() - t0
+    return n_tok * len(layers_cpu) / dt, f"{n_tok} of {stack.T} tokens of one batch through all {len(layers_cpu)} layers ({dt:.1f} s)"
+
+
+def run_ours(args, rank, world, device, dist):
+    import int4_expert_ffn_sigmoid_b200 as moe
+    wl = workloads.WORKLOADS[args.workload]
+    T = args.tokens or max(wl.tokens)
+    peaks = measured_peaks()
+    barrier = (lambda: dist.barrier()) if world > 1 else None
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    use_graph = not args.no_graph
+
+    stack = Stack(moe, wl, T, device)
+    uniq = stack.routing_unique()
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        step_ms, _ = timed_steps(stack, args.steps, args.warmup, use_graph, flush, dist_barrier=barrier)
+    clocks = clk.summary()
+    _, stage_ms = timed_steps(stack, args.steps, 2, use_graph, flush, instrumented=True)
+    e2e_ms, h2d, d2h = e2e_steps(stack, args.steps, args.warmup, flush, dist_barrier=barrier)
+
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms, sum(e2e_ms)], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_total = float(t[0]), float(t[1])
+    else:
+        e2e_total = sum(e2e_ms)
+    L = wl.layers
+    tokens_per_step = T * L
+    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+    e2e_value = world * tokens_per_step * args.steps / (e2e_total / 1e3)
+
+    # work accounting (batch i % 4 at step i)
+    step_b, step_f = [], []
+    for i in range(args.steps):
+        b, f = step_bytes_flops(wl.shape, T, uniq[i % N_BATCHES])
+        step_b.append(b)
+        step_f.append(f)
+    ms_mean = total_ms / args.steps
+    step_gbs = statistics.mean(step_b) / (ms_mean / 1e3) / 1e9
+    step_tflops = statistics.mean(step_f) / (ms_mean / 1e3) / 1e12
+
+    # dominant kernel (largest per-step stage time) and its roofline
+    stage_mean = [statistics.mean(s[k] for s in stage_ms) for k in range(4)]
+    names = moe.STAGE_NAMES
+    dom = int(np.argmax(stage_mean))
+    launches = args.steps * L
+    if dom == 1:
+        alg = statistics.mean(sum(gate_up_bytes(wl.shape, T, u) for u in uniq[i % N_BATCHES]) for i in range(args.steps))
+    elif dom == 2:
+        alg = statistics.mean(sum(down_bytes(wl.shape, T, u) for u in uniq[i % N_BATCHES]) for i in range(args.steps))
+    else:
+        alg = None
+    per_launch_us = stage_mean[dom] / L * 1e3
+    roofline = None
+    if alg is not None:
+        achieved = alg / L / (per_launch_us / 1e6) / 1e9
+        roofline = {"bound": "hbm", "kernel": f"experts_{'w13' if dom == 1 else 'w2'}_kernel",
+                    "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                    "alg_bytes_per_launch": int(alg / L), "avg_launch_us": round(per_launch_us, 3),
+                    "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy)"}
+
+    sweep = {}
+    if wl.name == "nano_decode_stack" and not args.no_sweep:
+        for Ts in wl.tokens:
+            st = stack if Ts == T else Stack(moe, wl, Ts, device, layers=stack.layers)
+            u = st.routing_unique()
+            ms, _ = timed_steps(st, max(5, args.steps // 2), 3, use_graph, flush)
+            b = statistics.mean(step_bytes_flops(wl.shape, Ts, u[i % N_BATCHES])[0] for i in range(len(ms)))
+            m = statistics.mean(ms)
+            sweep[str(Ts)] = {"tokens_per_s": round(Ts * L / (m / 1e3), 1), "ms_per_step": round(m, 4),
+                              "step_gbs": round(b / (m / 1e3) / 1e9, 1),
+                              "step_hbm_frac": round(b / (m / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+            if st is not stack:
+                del st
+                torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample = cpu_baseline_sample(stack)
+        cpu = {"value": round(v, 2), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
+
+    kernels_per_layer = 4 if T <= moe.decode_max_tokens() else 5
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "layers": L, "T": T, "H": wl.shape.H, "E": wl.shape.E,
+                   "K": wl.shape.K, "I": wl.shape.I, "Is": wl.shape.Is, "tokens_counted": "T*layers per step",
+                   "l2": "flushed between steps (256 MiB write, outside the timed events)",
+                   "inputs": f"{N_BATCHES} rotating batches", "cuda_graph": use_graph,
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "step_hbm": {"achieved_gbs": round(step_gbs, 1), "frac": round(step_gbs / peaks["hbm_gbs"], 4),
+                     "alg_bytes_per_step": int(statistics.mean(step_b)), "tflops": round(step_tflops, 3)},
+        "stages_us_per_step": {names[k]: round(stage_mean[k] * 1e3, 2) for k in range(4)},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": kernels_per_layer * launches,
+        "clocks": clocks,
+        "sweep": sweep or None,
+    }
+    return line
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm: each step is a bounded sample of
+    the workload (the first tokens of a batch through every layer, the oracle
+    chaining its own outputs rounded to bf16 as the next layer's input)."""
+    import oracle
+    if rank != 0:
+        return None
+    wl = workloads.WORKLOADS[args.workload]
+    T = args.tokens or max(wl.tokens)
+    layers = [workloads.make_layer(wl.shape, wl.wid, l, "cpu", wl.bias_mode) for l in range(wl.layers)]
+    xs = [workloads.make_x(wl.shape, T, wl.wid, batch=b, device="cpu") for b in range(N_BATCHES)]
+    n_tok = min(T, 4)
+
+    def step(i):
+        x = xs[i % N_BATCHES][:n_tok].contiguous()
+        for layer in layers:
+            r = oracle.moe_tokens(x, layer, wl.shape, residual=wl.residual)
+            x = torch.from_numpy(r["out"]).to(torch.bfloat16)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    value = n_tok * wl.layers * args.steps / dt
+    sample = f"{n_tok} of {T} tokens per step through all {wl.layers} layers"
+    return {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "layers": wl.layers, "T": T, "tokens_counted": "T*layers per step"},
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    dist = None
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    try:
+        line = run_ours(args, rank, world, device, dist)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,157 @@
+/*
+ * moe_int4.h -- C ABI of the B200 (sm_100a) forward pass of one
+ * Mixture-of-Experts FFN layer with int4 experts and a sigmoid+bias router.
+ *
+ * The layer (Colibri-Nano model card, "Architecture"; colibri README in the
+ * project listing, "What's implemented"; nanocolibri-engine README,
+ * "Converting a checkpoint yourself"):
+ *
+ *   L[t,e] = sum_h x[t,h] W[e,h]            router logits (f32 weights)
+ *   s[t,e] = sigmoid(L[t,e])                 score
+ *   S_t    = the K experts with the largest s[t,e] + bias[e]
+ *            (the bias only decides the selection; ties go to the lower
+ *            expert index; a NaN key counts as -infinity)
+ *   w[t,k] = routed_scaling * s[t,e_k] / sum_{j in S_t} s[t,j]
+ *   FFN_e(x) = W2_e (silu(Wg_e x) * (Wu_e x)),  silu(z) = z sigmoid(z)
+ *   out[t] = sum_k w[t,k] FFN_{e_k}(x_t) + FFN_shared(x_t)  [+ x_t]
+ *
+ * The shared expert has weight 1 and is not multiplied by routed_scaling.
+ * Routed tokens are bucketed by expert ("batch-union": each expert touched by
+ * the batch is read once and applied to all its tokens) before the expert
+ * FFNs run.
+ *
+ * Weight format ("per-row symmetric with f32 scales"): every matrix is stored
+ * row-major with one row per OUTPUT feature.  A row of n int4 codes takes n/2
+ * bytes: byte j holds element 2j in bits 0..3 and element 2j+1 in bits 4..7,
+ * each a 4-bit two's-complement code c in [-8, 7].  The dequantised weight is
+ * c * scale[row] with one f32 scale per row.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers to caller-owned, contiguous,
+ *    row-major memory on the current CUDA device.  Pointers must be 16-byte
+ *    aligned.  The library never allocates or frees device memory.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *    stream-ordered and asynchronous: the return value reports argument
+ *    errors and launch errors only, unless MOE_DEBUG_CHECK is set.
+ *  - Calls are reentrant provided concurrent calls use distinct workspaces
+ *    and outputs.  `out` must not alias `x`.
+ */
+#ifndef MOE_INT4_H
+#define MOE_INT4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+/* Status codes. */
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG 1  /* NULL pointer, bad struct_size, T < 0, K > E, misaligned pointer */
+#define MOE_ERR_UNSUPPORTED 2  /* shape outside the supported set (see moe_cfg_t) */
+#define MOE_ERR_WORKSPACE 3    /* workspace NULL or smaller than moe_layer_workspace_bytes() */
+#define MOE_ERR_CUDA 4         /* a CUDA runtime call or kernel launch failed */
+#define MOE_ERR_DEVICE_CHECK 5 /* MOE_DEBUG_CHECK: a kernel's range check failed */
+
+/* Flags of moe_cfg_t.flags. */
+#define MOE_ADD_RESIDUAL (1u << 0)  /* out = x + MoE(x) (one layer of a residual stack) */
+#define MOE_DEBUG_CHECK (1u << 1)   /* synchronise the stream and report device range checks */
+#define MOE_FORCE_DECODE (1u << 2)  /* use the small-batch (weight-streaming) kernels at any T */
+#define MOE_FORCE_PREFILL (1u << 3) /* use the large-batch (grouped GEMM) kernels at any T */
+
+/* The always-resident shared expert (intermediate size Is).
+ *   w13: uint8 [2*Is][H/2]  rows 0..Is-1 gate, rows Is..2*Is-1 up
+ *   s13: f32   [2*Is]       one scale per w13 row
+ *   w2 : uint8 [H][Is/2]
+ *   s2 : f32   [H] */
+typedef struct moe_shared_weights {
+    const uint8_t* w13;
+    const float* s13;
+    const uint8_t* w2;
+    const float* s2;
+} moe_shared_weights_t;
+
+/* Stages of one forward call, for the optional per-stage event hook. */
+#define MOE_STAGE_ROUTE 0   /* router, selection, bucketing */
+#define MOE_STAGE_GATE_UP 1 /* expert gate/up projections + SwiGLU (routed and shared) */
+#define MOE_STAGE_DOWN 2    /* expert down projections (routed and shared) */
+#define MOE_STAGE_COMBINE 3 /* weighted combine (+ shared expert, + residual) */
+#define MOE_NUM_STAGES 4
+
+/* Layer configuration.
+ *   struct_size    : sizeof(moe_cfg_t) (ABI versioning).
+ *   H              : hidden size; multiple of 128, at most 16384.
+ *   E              : routed experts, 1..256.
+ *   K              : experts per token, 1..8 and K <= E.
+ *   I              : routed intermediate size; multiple of 128, at most 8192.
+ *   Is             : shared intermediate size; 0 (no shared expert) or a
+ *                    multiple of 128, at most 8192.
+ *   routed_scaling : factor on the normalised routing weights (finite, > 0).
+ *   flags          : MOE_* flags above.
+ *   workspace      : device scratch of at least moe_layer_workspace_bytes()
+ *                    bytes, 256-byte aligned; its contents need no
+ *                    initialisation and are overwritten by every call.
+ *   topk_idx_out   : optional device int32 [T][K]: selected experts, in
+ *                    decreasing order of s + bias (NULL = not written).
+ *   topk_w_out     : optional device f32 [T][K]: their routing weights.
+ *   stage_events   : optional array of 2*MOE_NUM_STAGES cudaEvent_t handles
+ *                    (created by the caller, e.g. with cudaEventCreate);
+ *                    events [2s] and [2s+1] are recorded on `stream` before
+ *                    and after stage s.  NULL = no recording. */
+typedef struct moe_cfg {
+    uint32_t struct_size;
+    int32_t H, E, K, I, Is;
+    float routed_scaling;
+    uint32_t flags;
+    void* workspace;
+    size_t workspace_bytes;
+    int32_t* topk_idx_out;
+    float* topk_w_out;
+    void* const* stage_events;
+} moe_cfg_t;
+
+/* Bytes of workspace moe_layer_forward needs for T tokens under `cfg`
+ * (workspace, workspace_bytes and the output pointers are ignored).
+ * Returns 0 if cfg is NULL or the shape is invalid or unsupported. */
+size_t moe_layer_workspace_bytes(const moe_cfg_t* cfg, int32_t T);
+
+/* Forward pass of one MoE layer for T tokens.
+ *   x          : bf16 [T][H]
+ *   router_w   : f32  [E][H]
+ *   router_bias: f32  [E]
+ *   packed_w13 : uint8 [E][2I][H/2]  per expert: rows 0..I-1 gate, I..2I-1 up
+ *   scales13   : f32  [E][2I]
+ *   packed_w2  : uint8 [E][H][I/2]
+ *   scales2    : f32  [E][H]
+ *   shared_w   : the shared expert (required when cfg->Is > 0, else ignored)
+ *   out        : bf16 [T][H]  (written; one round-to-nearest-even of the f32 sum)
+ *   T          : tokens, 0..2^20 (T = 0 returns MOE_OK and launches nothing)
+ *   cfg, stream: see above.
+ * The routing weights and every expert contribution are accumulated in f32;
+ * the gate/up intermediate is kept in fp16 or f32, never bf16.
+ * Returns MOE_OK or an MOE_ERR_* code; on an error nothing is launched
+ * (except MOE_ERR_CUDA / MOE_ERR_DEVICE_CHECK, raised after launching). */
+int moe_layer_forward(const void* x, const float* router_w, const float* router_bias,
+                      const uint8_t* packed_w13, const float* scales13,
+                      const uint8_t* packed_w2, const float* scales2,
+                      const moe_shared_weights_t* shared_w, void* out, int32_t T,
+                      const moe_cfg_t* cfg, void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moe_status_str(int status);
+
+/* MOE_ABI_VERSION of the loaded library. */
+int moe_abi_version(void);
+
+/* Largest T for which moe_layer_forward takes the small-batch
+ * (weight-streaming) path when neither MOE_FORCE_* flag is set. */
+int32_t moe_decode_max_tokens(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_INT4_H */

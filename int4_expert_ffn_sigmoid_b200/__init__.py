@@ -1,0 +1,209 @@
+"""B200 (sm_100a) forward pass of one int4 expert-FFN MoE layer with a
+sigmoid+bias router: the Python binding of ``libmoe_int4.so``.
+
+This module only marshals arguments: every step of the layer (router,
+selection, bucketing, expert FFNs, shared expert, combine) runs in the
+library's CUDA kernels.  torch provides device memory and streams.  There is
+no fallback: if the library is missing, importing the binding raises.
+
+The C ABI is declared in ``include/moe_int4.h``; the names here mirror it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "MoeError", "moe_cfg_t", "moe_shared_weights_t", "lib", "EXPORTED_SYMBOLS",
+    "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK", "MOE_FORCE_DECODE", "MOE_FORCE_PREFILL",
+    "workspace_bytes", "layer_forward", "MoELayer", "decode_max_tokens", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_int4.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_WORKSPACE = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_DEVICE_CHECK = 5
+
+MOE_ADD_RESIDUAL = 1 << 0
+MOE_DEBUG_CHECK = 1 << 1
+MOE_FORCE_DECODE = 1 << 2
+MOE_FORCE_PREFILL = 1 << 3
+
+MOE_STAGE_ROUTE, MOE_STAGE_GATE_UP, MOE_STAGE_DOWN, MOE_STAGE_COMBINE = range(4)
+MOE_NUM_STAGES = 4
+STAGE_NAMES = ("route", "gate_up", "down", "combine")
+
+# Every function declared in include/moe_int4.h.
+EXPORTED_SYMBOLS = ("moe_layer_workspace_bytes", "moe_layer_forward", "moe_status_str",
+                    "moe_abi_version", "moe_decode_max_tokens")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str = "moe_layer_forward"):
+        self.status = status
+        super().__init__(f"{what} failed: {status_str(status)} ({status})")
+
+
+class moe_cfg_t(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("H", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("K", ctypes.c_int32), ("I", ctypes.c_int32), ("Is", ctypes.c_int32),
+                ("routed_scaling", ctypes.c_float), ("flags", ctypes.c_uint32),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("topk_idx_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p),
+                ("stage_events", ctypes.c_void_p)]
+
+
+class moe_shared_weights_t(ctypes.Structure):
+    _fields_ = [("w13", ctypes.c_void_p), ("s13", ctypes.c_void_p),
+                ("w2", ctypes.c_void_p), ("s2", ctypes.c_void_p)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m int4_expert_ffn_sigmoid_b200._build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp = ctypes.c_void_p
+    L.moe_layer_workspace_bytes.argtypes = [ctypes.POINTER(moe_cfg_t), ctypes.c_int32]
+    L.moe_layer_workspace_bytes.restype = ctypes.c_size_t
+    L.moe_layer_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(moe_shared_weights_t),
+                                    vp, ctypes.c_int32, ctypes.POINTER(moe_cfg_t), vp]
+    L.moe_layer_forward.restype = ctypes.c_int
+    L.moe_status_str.argtypes = [ctypes.c_int]
+    L.moe_status_str.restype = ctypes.c_char_p
+    L.moe_abi_version.argtypes = []
+    L.moe_abi_version.restype = ctypes.c_int
+    L.moe_decode_max_tokens.argtypes = []
+    L.moe_decode_max_tokens.restype = ctypes.c_int32
+    if L.moe_abi_version() != 1:
+        raise ImportError("libmoe_int4.so ABI version mismatch")
+    return L
+
+
+lib = _load()
+
+
+def status_str(status: int) -> str:
+    return lib.moe_status_str(int(status)).decode()
+
+
+def decode_max_tokens() -> int:
+    return int(lib.moe_decode_max_tokens())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def make_cfg(shape, flags: int = 0, workspace: Optional[torch.Tensor] = None,
+             topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+             stage_events=None) -> moe_cfg_t:
+    c = moe_cfg_t()
+    c.struct_size = ctypes.sizeof(moe_cfg_t)
+    c.H, c.E, c.K, c.I, c.Is = shape.H, shape.E, shape.K, shape.I, shape.Is
+    c.routed_scaling = float(shape.routed_scaling)
+    c.flags = int(flags)
+    if workspace is not None:
+        c.workspace = workspace.data_ptr()
+        c.workspace_bytes = workspace.numel() * workspace.element_size()
+    c.topk_idx_out = None if topk_idx is None else topk_idx.data_ptr()
+    c.topk_w_out = None if topk_w is None else topk_w.data_ptr()
+    if stage_events is not None:
+        if len(stage_events) != 2 * MOE_NUM_STAGES:
+            raise ValueError(f"stage_events needs {2 * MOE_NUM_STAGES} events")
+        arr = (ctypes.c_void_p * len(stage_events))(*[int(e.cuda_event) for e in stage_events])
+        c._events_keepalive = arr
+        c.stage_events = ctypes.cast(arr, ctypes.c_void_p).value
+    return c
+
+
+def workspace_bytes(shape, T: int, flags: int = 0) -> int:
+    c = make_cfg(shape, flags)
+    return int(lib.moe_layer_workspace_bytes(ctypes.byref(c), int(T)))
+
+
+def new_workspace(shape, T: int, device, flags: int = 0) -> torch.Tensor:
+    n = workspace_bytes(shape, T, flags)
+    if n == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED, "moe_layer_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _check_dev(name, t, dtype, shape=None):
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor, got {t.dtype} on {t.device}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def layer_forward(x: torch.Tensor, layer: dict, shape, out: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, flags: int = 0,
+                  topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None, stage_events=None) -> torch.Tensor:
+    """Call ``moe_layer_forward`` on torch tensors (see include/moe_int4.h).
+
+    ``layer`` holds router_w, router_bias, w13, s13, w2, s2 and, when
+    shape.Is > 0, sh_w13, sh_s13, sh_w2, sh_s2 (the layout of
+    ``workloads.make_layer``).  Returns ``out`` (bf16 [T, H]).  ``stage_events``:
+    optional sequence of 2*MOE_NUM_STAGES ``torch.cuda.Event`` already recorded
+    once (so that they exist); the library records them around each stage."""
+    T = x.shape[0]
+    H, E, I, Is = shape.H, shape.E, shape.I, shape.Is
+    _check_dev("x", x, torch.bfloat16, (T, H))
+    _check_dev("router_w", layer["router_w"], torch.float32, (E, H))
+    _check_dev("router_bias", layer["router_bias"], torch.float32, (E,))
+    _check_dev("w13", layer["w13"], torch.uint8, (E, 2 * I, H // 2))
+    _check_dev("s13", layer["s13"], torch.float32, (E, 2 * I))
+    _check_dev("w2", layer["w2"], torch.uint8, (E, H, I // 2))
+    _check_dev("s2", layer["s2"], torch.float32, (E, H))
+    sh = moe_shared_weights_t()
+    if Is > 0:
+        _check_dev("sh_w13", layer["sh_w13"], torch.uint8, (2 * Is, H // 2))
+        _check_dev("sh_s13", layer["sh_s13"], torch.float32, (2 * Is,))
+        _check_dev("sh_w2", layer["sh_w2"], torch.uint8, (H, Is // 2))
+        _check_dev("sh_s2", layer["sh_s2"], torch.float32, (H,))
+        sh.w13, sh.s13 = layer["sh_w13"].data_ptr(), layer["sh_s13"].data_ptr()
+        sh.w2, sh.s2 = layer["sh_w2"].data_ptr(), layer["sh_s2"].data_ptr()
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    _check_dev("out", out, torch.bfloat16, (T, H))
+    if workspace is None:
+        workspace = new_workspace(shape, T, x.device, flags)
+    if topk_idx is not None:
+        _check_dev("topk_idx", topk_idx, torch.int32, (T, shape.K))
+    if topk_w is not None:
+        _check_dev("topk_w", topk_w, torch.float32, (T, shape.K))
+    cfg = make_cfg(shape, flags, workspace, topk_idx, topk_w, stage_events)
+    s = stream if stream is not None else torch.cuda.current_stream(x.device)
+    st = lib.moe_layer_forward(_ptr(x), _ptr(layer["router_w"]), _ptr(layer["router_bias"]),
+                               _ptr(layer["w13"]), _ptr(layer["s13"]), _ptr(layer["w2"]),
+                               _ptr(layer["s2"]), ctypes.byref(sh), _ptr(out), int(T),
+                               ctypes.byref(cfg), ctypes.c_void_p(s.cuda_stream))
+    if st != MOE_OK:
+        raise MoeError(st)
+    return out
+
+
+class MoELayer:
+    """One layer's device weights plus a workspace sized for up to ``max_tokens``."""
+
+    def __init__(self, layer: dict, shape, max_tokens: int, device=None):
+        self.layer = layer
+        self.shape = shape
+        self.device = torch.device(device) if device is not None else layer["w13"].device
+        self.max_tokens = int(max_tokens)
+        self.workspace = new_workspace(shape, self.max_tokens, self.device)
+
+    def __call__(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, residual: bool = False,
+                 flags: int = 0, topk_idx=None, topk_w=None, stage_events=None) -> torch.Tensor:
+        if x.shape[0] > self.max_tokens:
+            raise ValueError(f"T={x.shape[0]} exceeds max_tokens={self.max_tokens}")
+        f = flags | (MOE_ADD_RESIDUAL if residual else 0)
+        return layer_forward(x, self.layer, self.shape, out=out, workspace=self.workspace, flags=f,
+                             topk_idx=topk_idx, topk_w=topk_w, stage_events=stage_events)

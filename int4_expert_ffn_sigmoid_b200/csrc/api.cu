@@ -1,0 +1,208 @@
+// C ABI of the int4 MoE layer forward: argument validation, workspace
+// layout, kernel sequence.  See include/moe_int4.h for the contract.
+#include <math.h>
+#include <string.h>
+
+#include "moe_common.cuh"
+#include "moe_int4.h"
+#include "moe_launch.h"
+
+namespace {
+
+using namespace moe;
+
+constexpr unsigned kKnownFlags = MOE_ADD_RESIDUAL | MOE_DEBUG_CHECK | MOE_FORCE_DECODE | MOE_FORCE_PREFILL;
+constexpr int32_t kMaxTokens = 1 << 20;
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct WsLayout {
+    size_t ctrl, idx, wts, logits, counts, offsets, bucket_e, bucket_n, bucket_off, ts13, ts2;
+    size_t tok_of_slot, slot_of, hist, h_r, h_s, y, total;
+};
+
+WsLayout ws_layout(const moe_cfg_t& c, int32_t T) {
+    WsLayout L{};
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t r = o;
+        o = align256(o + bytes);
+        return r;
+    };
+    const size_t TK = (size_t)T * c.K, E = (size_t)c.E;
+    L.ctrl = take(sizeof(Ctrl));
+    L.idx = take(TK * 4);
+    L.wts = take(TK * 4);
+    L.logits = take((size_t)(T < kDecodeMaxTokens ? T : kDecodeMaxTokens) * E * 4);
+    L.counts = take(E * 4);
+    L.offsets = take(E * 4);
+    L.bucket_e = take((E + 1) * 4);
+    L.bucket_n = take((E + 1) * 4);
+    L.bucket_off = take((E + 1) * 4);
+    L.ts13 = take((E + 2) * 4);
+    L.ts2 = take((E + 2) * 4);
+    L.tok_of_slot = take(TK * 4);
+    L.slot_of = take(TK * 4);
+    L.hist = take((size_t)kRouterMaxBlocks * E * 4);
+    L.h_r = take(TK * (size_t)c.I * 2);
+    L.h_s = take((size_t)T * (size_t)c.Is * 2);
+    L.y = take((TK + (c.Is > 0 ? (size_t)T : 0)) * (size_t)c.H * 4);
+    L.total = o;
+    return L;
+}
+
+int validate_cfg(const moe_cfg_t* c) {
+    if (!c || c->struct_size != sizeof(moe_cfg_t)) return MOE_ERR_INVALID_ARG;
+    if (c->H <= 0 || c->E <= 0 || c->K <= 0 || c->I <= 0 || c->Is < 0 || c->K > c->E) return MOE_ERR_INVALID_ARG;
+    if (!(c->routed_scaling > 0.0f) || !isfinite(c->routed_scaling)) return MOE_ERR_INVALID_ARG;
+    if (c->flags & ~kKnownFlags) return MOE_ERR_INVALID_ARG;
+    if ((c->flags & MOE_FORCE_DECODE) && (c->flags & MOE_FORCE_PREFILL)) return MOE_ERR_INVALID_ARG;
+    if (c->H % 128 || c->H > 16384) return MOE_ERR_UNSUPPORTED;
+    if (c->E > kMaxE || c->K > kMaxK) return MOE_ERR_UNSUPPORTED;
+    if (c->I % 128 || c->I > 8192) return MOE_ERR_UNSUPPORTED;
+    if (c->Is % 128 || c->Is > 8192) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+inline bool aligned(const void* ptr, size_t a) { return ((uintptr_t)ptr % a) == 0; }
+
+int sm_count() {
+    static int cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+}  // namespace
+
+extern "C" {
+
+int moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+int32_t moe_decode_max_tokens(void) { return kDecodeMaxTokens; }
+
+const char* moe_status_str(int status) {
+    switch (status) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK";
+        default: return "MOE_ERR_UNKNOWN";
+    }
+}
+
+size_t moe_layer_workspace_bytes(const moe_cfg_t* cfg, int32_t T) {
+    if (validate_cfg(cfg) != MOE_OK || T < 0 || T > kMaxTokens) return 0;
+    return ws_layout(*cfg, T).total;
+}
+
+int moe_layer_forward(const void* x, const float* router_w, const float* router_bias,
+                      const uint8_t* packed_w13, const float* scales13, const uint8_t* packed_w2,
+                      const float* scales2, const moe_shared_weights_t* shared_w, void* out, int32_t T,
+                      const moe_cfg_t* cfg, void* stream) {
+    int st = validate_cfg(cfg);
+    if (st != MOE_OK) return st;
+    if (T < 0 || T > kMaxTokens) return MOE_ERR_INVALID_ARG;
+    if (!x || !router_w || !router_bias || !packed_w13 || !scales13 || !packed_w2 || !scales2 || !out)
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->Is > 0 && (!shared_w || !shared_w->w13 || !shared_w->s13 || !shared_w->w2 || !shared_w->s2))
+        return MOE_ERR_INVALID_ARG;
+    const void* ptrs[] = {x, router_w, router_bias, packed_w13, scales13, packed_w2, scales2, out,
+                          cfg->Is > 0 ? shared_w->w13 : nullptr, cfg->Is > 0 ? shared_w->s13 : nullptr,
+                          cfg->Is > 0 ? shared_w->w2 : nullptr, cfg->Is > 0 ? shared_w->s2 : nullptr,
+                          cfg->topk_idx_out, cfg->topk_w_out};
+    for (const void* ptr : ptrs)
+        if (ptr && !aligned(ptr, 16)) return MOE_ERR_INVALID_ARG;
+    const size_t xbytes = (size_t)T * cfg->H * 2;
+    const uintptr_t xa = (uintptr_t)x, oa = (uintptr_t)out;
+    if (T > 0 && xa < oa + xbytes && oa < xa + xbytes) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(*cfg, T);
+    if (!cfg->workspace || cfg->workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+    if (!aligned(cfg->workspace, 256)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+
+    char* ws = static_cast<char*>(cfg->workspace);
+    Params p;
+    memset(&p, 0, sizeof p);
+    p.T = T; p.H = cfg->H; p.E = cfg->E; p.K = cfg->K; p.I = cfg->I; p.Is = cfg->Is;
+    p.scale = cfg->routed_scaling;
+    p.flags = cfg->flags;
+    p.x = static_cast<const __nv_bfloat16*>(x);
+    p.rw = router_w; p.rb = router_bias;
+    p.w13 = packed_w13; p.s13 = scales13; p.w2 = packed_w2; p.s2 = scales2;
+    if (cfg->Is > 0) {
+        p.sh_w13 = shared_w->w13; p.sh_s13 = shared_w->s13; p.sh_w2 = shared_w->w2; p.sh_s2 = shared_w->s2;
+    }
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.topk_idx_out = cfg->topk_idx_out;
+    p.topk_w_out = cfg->topk_w_out;
+    p.ctrl = reinterpret_cast<Ctrl*>(ws + L.ctrl);
+    p.idx = reinterpret_cast<int32_t*>(ws + L.idx);
+    p.wts = reinterpret_cast<float*>(ws + L.wts);
+    p.logits = reinterpret_cast<float*>(ws + L.logits);
+    p.counts = reinterpret_cast<int32_t*>(ws + L.counts);
+    p.offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+    p.bucket_e = reinterpret_cast<int32_t*>(ws + L.bucket_e);
+    p.bucket_n = reinterpret_cast<int32_t*>(ws + L.bucket_n);
+    p.bucket_off = reinterpret_cast<int32_t*>(ws + L.bucket_off);
+    p.ts13 = reinterpret_cast<int32_t*>(ws + L.ts13);
+    p.ts2 = reinterpret_cast<int32_t*>(ws + L.ts2);
+    p.tok_of_slot = reinterpret_cast<int32_t*>(ws + L.tok_of_slot);
+    p.slot_of = reinterpret_cast<int32_t*>(ws + L.slot_of);
+    p.hist = reinterpret_cast<int32_t*>(ws + L.hist);
+    p.h_r = reinterpret_cast<__half*>(ws + L.h_r);
+    p.h_s = reinterpret_cast<__half*>(ws + L.h_s);
+    p.y = reinterpret_cast<float*>(ws + L.y);
+    const int ntiles = cdiv(T, kRouterTileTokens);
+    p.router_blocks = ntiles < kRouterMaxBlocks ? ntiles : kRouterMaxBlocks;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool small_router = T <= kDecodeMaxTokens;
+    const long long TK = (long long)T * cfg->K;
+    const long long routed_buckets = (cfg->E < TK ? cfg->E : TK) + cdiv(TK, kChunkTokens);
+    const long long shared_chunks = cfg->Is > 0 ? cdiv(T, kChunkTokens) : 0;
+    const long long warps13 = (long long)(cfg->I / 8) * routed_buckets + (long long)(cfg->Is / 8) * shared_chunks;
+    const long long warps2 = (long long)(cfg->H / 16) * (routed_buckets + shared_chunks);
+    const int cap = sm_count() * 8;
+    const int grid13 = (int)(cdiv(warps13, 8) < cap ? cdiv(warps13, 8) : cap);
+    const int grid2 = (int)(cdiv(warps2, 8) < cap ? cdiv(warps2, 8) : cap);
+
+    void* const* ev = cfg->stage_events;
+    auto mark = [&](int idx) -> cudaError_t {
+        return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[idx]), s) : cudaSuccess;
+    };
+    cudaError_t err = mark(2 * MOE_STAGE_ROUTE);
+    if (err == cudaSuccess) err = cudaMemsetAsync(p.ctrl, 0, sizeof(Ctrl), s);
+    if (err == cudaSuccess) err = launch_router(p, small_router, s);
+    if (err == cudaSuccess) err = mark(2 * MOE_STAGE_ROUTE + 1);
+    if (err == cudaSuccess) err = mark(2 * MOE_STAGE_GATE_UP);
+    if (err == cudaSuccess) err = launch_experts_w13(p, grid13, s);
+    if (err == cudaSuccess) err = mark(2 * MOE_STAGE_GATE_UP + 1);
+    if (err == cudaSuccess) err = mark(2 * MOE_STAGE_DOWN);
+    if (err == cudaSuccess) err = launch_experts_w2(p, grid2, s);
+    if (err == cudaSuccess) err = mark(2 * MOE_STAGE_DOWN + 1);
+    if (err == cudaSuccess) err = mark(2 * MOE_STAGE_COMBINE);
+    if (err == cudaSuccess) err = launch_combine(p, s);
+    if (err == cudaSuccess) err = mark(2 * MOE_STAGE_COMBINE + 1);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    if (cfg->flags & MOE_DEBUG_CHECK) {
+        unsigned status = 0;
+        err = cudaMemcpyAsync(&status, &p.ctrl->status, sizeof status, cudaMemcpyDeviceToHost, s);
+        if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+        if (err != cudaSuccess) return MOE_ERR_CUDA;
+        if (status != 0) return MOE_ERR_DEVICE_CHECK;
+    }
+    return MOE_OK;
+}
+
+}  // extern "C"

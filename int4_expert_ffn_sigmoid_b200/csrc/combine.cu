@@ -1,0 +1,51 @@
+// Weighted combine: out[t] = sum_k w[t,k] y[slot(t,k)] + y_shared[t] (+ x[t]),
+// summed in f32 (k ascending, then the shared expert, then the residual) and
+// rounded once to bf16 (round to nearest even).
+//
+// Method: colibri README (project listing), "What's implemented" (shared
+// expert; routed experts weighted by the sigmoid router); Colibri-Nano model
+// card, "Architecture" (the always-resident shared expert is added for every
+// token).
+#include "moe_common.cuh"
+#include "moe_launch.h"
+
+namespace moe {
+
+__global__ void __launch_bounds__(256) combine_kernel(Params p) {
+    const int t = blockIdx.x;
+    const int j = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
+    if (j >= p.H) return;
+    const int K = p.K, H = p.H;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    for (int k = 0; k < K; ++k) {
+        const int s = __ldg(p.slot_of + (size_t)t * K + k);
+        const float w = __ldg(p.wts + (size_t)t * K + k);
+        const float4 v = __ldg(reinterpret_cast<const float4*>(p.y + (size_t)s * H + j));
+        a0 = fmaf(w, v.x, a0);
+        a1 = fmaf(w, v.y, a1);
+        a2 = fmaf(w, v.z, a2);
+        a3 = fmaf(w, v.w, a3);
+    }
+    if (p.Is > 0) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(p.y + ((size_t)p.T * K + t) * H + j));
+        a0 += v.x; a1 += v.y; a2 += v.z; a3 += v.w;
+    }
+    if (p.flags & 1u) {  // MOE_ADD_RESIDUAL
+        const uint2 xv = __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)t * H + j));
+        a0 += bf16lo(xv.x); a1 += bf16hi(xv.x); a2 += bf16lo(xv.y); a3 += bf16hi(xv.y);
+    }
+    __nv_bfloat162 o01 = __floats2bfloat162_rn(a0, a1);
+    __nv_bfloat162 o23 = __floats2bfloat162_rn(a2, a3);
+    uint2 ov;
+    ov.x = *reinterpret_cast<uint32_t*>(&o01);
+    ov.y = *reinterpret_cast<uint32_t*>(&o23);
+    *reinterpret_cast<uint2*>(p.out + (size_t)t * H + j) = ov;
+}
+
+cudaError_t launch_combine(const Params& p, cudaStream_t stream) {
+    dim3 grid(p.T, (p.H + 1023) / 1024);
+    combine_kernel<<<grid, 256, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,19 @@
+// Host-side launch entry points of the kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "moe_common.cuh"
+
+namespace moe {
+
+// Router + bucketing.  small_path: T <= kDecodeMaxTokens.
+cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream);
+// Expert gate/up + SwiGLU (weight-streaming mma.sync kernel).
+cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream);
+// Expert down projection (weight-streaming mma.sync kernel).
+cudaError_t launch_experts_w2(const Params& p, int grid, cudaStream_t stream);
+// Weighted combine + shared expert (+ residual) -> bf16 out.
+cudaError_t launch_combine(const Params& p, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,87 @@
+"""Comparison of the CUDA path with the CPU oracle (helpers for GPU tests).
+
+Bars (the layer's stated acceptance criteria):
+  * selected experts identical to the oracle's, except for "ties": tokens
+    whose oracle margin (K-th minus (K+1)-th selection key) is below 1e-6.
+    For a tie the GPU's choice must lie in the tie set: every selected expert's
+    oracle key >= the oracle's K-th key - 1e-6, no repeats;
+  * routing weights within 1e-6 relative of the oracle's;
+  * layer output: per-token relative L2 error ||out - ref|| / ||ref|| <= 2e-3,
+    with out the GPU's bf16 output widened exactly and ref the oracle's f64
+    result evaluated with the GPU's selection (identical to the oracle's own
+    selection except at ties).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+
+TIE_MARGIN = 1e-6
+W_RTOL = 1e-6
+OUT_TOL = 2e-3
+
+
+def to_cpu_layer(layer: dict) -> dict:
+    return {k: v.detach().cpu() for k, v in layer.items()}
+
+
+def check_routing(idx_gpu: np.ndarray, w_gpu: np.ndarray, ref: dict, bias: np.ndarray, K: int):
+    """Returns (tie token indices, max weight rel error over non-tie tokens)."""
+    T = idx_gpu.shape[0]
+    margin = ref["margin"]
+    keys = ref["scores"] + bias.astype(np.float64)[None, :]
+    ties = np.nonzero(margin < TIE_MARGIN)[0]
+    non = np.ones(T, bool)
+    non[ties] = False
+    bad = np.nonzero(non & np.any(idx_gpu != ref["idx"], axis=1))[0]
+    assert bad.size == 0, (f"{bad.size} non-tie tokens select different experts; first {bad[:5]}: "
+                           f"gpu {idx_gpu[bad[:3]]} oracle {ref['idx'][bad[:3]]} margin {margin[bad[:3]]}")
+    for t in ties:
+        sel = idx_gpu[t]
+        assert len(set(sel.tolist())) == K, (t, sel)
+        kth = np.sort(keys[t])[::-1][K - 1]
+        assert np.all(keys[t, sel] >= kth - TIE_MARGIN), (t, sel, keys[t, sel], kth)
+    werr = 0.0
+    if non.any():
+        werr = float(np.max(np.abs(w_gpu[non] - ref["weights"][non]) / np.abs(ref["weights"][non])))
+        assert werr <= W_RTOL, f"routing weight relative error {werr:.3e} > {W_RTOL}"
+    return ties, werr
+
+
+def rel_l2(out_gpu: torch.Tensor, ref: np.ndarray) -> np.ndarray:
+    o = out_gpu.detach().float().cpu().numpy().astype(np.float64)
+    num = np.linalg.norm(o - ref, axis=1)
+    den = np.linalg.norm(ref, axis=1)
+    return num / np.maximum(den, 1e-300)
+
+
+def compare_layer(x: torch.Tensor, out: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, layer_cpu: dict,
+                  shape, residual: bool, sample=None) -> dict:
+    """Full comparison.  Routing is checked on every token; outputs on
+    ``sample`` (token indices; default all)."""
+    xc = x.detach().cpu()
+    ref_r = oracle.route(xc, layer_cpu["router_w"], layer_cpu["router_bias"], shape.K, shape.routed_scaling)
+    idx_g = idx.detach().cpu().numpy()
+    w_g = w.detach().cpu().numpy().astype(np.float64)
+    ties, werr = check_routing(idx_g, w_g, ref_r, layer_cpu["router_bias"].numpy(), shape.K)
+    T = x.shape[0]
+    tok = np.arange(T) if sample is None else np.unique(np.asarray(sample, np.int64))
+    ref = oracle.moe_tokens(xc, layer_cpu, shape, residual=residual, tokens=tok.astype(np.int32),
+                            idx_override=idx_g[tok])
+    err = rel_l2(out[torch.from_numpy(tok).to(out.device)], ref["out"])
+    assert np.all(np.isfinite(err)), "non-finite output"
+    worst = int(tok[int(np.argmax(err))])
+    assert err.max() <= OUT_TOL, f"per-token rel L2 {err.max():.3e} > {OUT_TOL} at token {worst}"
+    return dict(ties=len(ties), max_rel_l2=float(err.max()), mean_rel_l2=float(err.mean()),
+                max_w_rel=werr, tokens_checked=len(tok))
+
+
+def sample_tokens(T: int, n: int = 32, seed: int = 0, extra=()) -> np.ndarray:
+    """First and last few tokens (ragged tail) plus a seeded random draw."""
+    rng = np.random.default_rng(seed)
+    head = np.arange(min(T, 4))
+    tail = np.arange(max(0, T - 4), T)
+    mid = rng.choice(T, size=min(T, n), replace=False)
+    return np.unique(np.concatenate([head, tail, mid, np.asarray(extra, np.int64)]))

@@ -1,0 +1,125 @@
+"""The C-ABI library without a GPU: it loads, exports every function that
+include/moe_int4.h declares, and its host-side validation returns the
+documented status codes before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_int4.h")
+
+
+@pytest.fixture(scope="module")
+def moe():
+    from int4_expert_ffn_sigmoid_b200 import _build
+    _build.build()
+    import int4_expert_ffn_sigmoid_b200 as m
+    return m
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(moe_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_exports_every_declared_function(moe):
+    names = _declared_functions()
+    assert set(names) == set(moe.EXPORTED_SYMBOLS), names
+    for n in names:
+        assert hasattr(moe.lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", moe.LIB_PATH], capture_output=True, text=True).stdout
+    for n in names:
+        assert re.search(rf"\bT {n}$", out, flags=re.M), n
+
+
+def test_struct_layout_matches_c(moe, tmp_path):
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "moe_int4.h"\n'
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(moe_cfg_t),"
+        " offsetof(moe_cfg_t, routed_scaling), offsetof(moe_cfg_t, flags),"
+        " offsetof(moe_cfg_t, workspace), offsetof(moe_cfg_t, workspace_bytes),"
+        " offsetof(moe_cfg_t, topk_w_out), sizeof(moe_shared_weights_t)); return 0;}\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)])
+    c_vals = [int(v) for v in subprocess.check_output([str(exe)]).split()]
+    cfg = moe.moe_cfg_t
+    py_vals = [ctypes.sizeof(cfg), cfg.routed_scaling.offset, cfg.flags.offset, cfg.workspace.offset,
+               cfg.workspace_bytes.offset, cfg.topk_w_out.offset, ctypes.sizeof(moe.moe_shared_weights_t)]
+    assert c_vals == py_vals
+
+
+def test_version_and_strings(moe):
+    assert moe.lib.moe_abi_version() == 1
+    assert moe.status_str(0) == "MOE_OK"
+    assert moe.status_str(3) == "MOE_ERR_WORKSPACE"
+    assert moe.status_str(99) == "MOE_ERR_UNKNOWN"
+    assert moe.decode_max_tokens() == 64
+
+
+def _shape(**kw):
+    import workloads
+    base = dict(H=1024, E=64, K=2, I=512, Is=2048, routed_scaling=1.0)
+    base.update(kw)
+    return workloads.LayerShape(**base)
+
+
+def test_workspace_query(moe):
+    a = moe.workspace_bytes(_shape(), 16)
+    b = moe.workspace_bytes(_shape(), 4096)
+    assert 0 < a < b
+    assert a % 256 == 0
+    assert moe.workspace_bytes(_shape(H=1000), 16) == 0      # H not a multiple of 128
+    assert moe.workspace_bytes(_shape(K=65, E=64), 16) == 0  # K > E
+    assert moe.workspace_bytes(_shape(E=300), 16) == 0       # E > 256
+    assert moe.workspace_bytes(_shape(), -1) == 0
+    assert moe.workspace_bytes(_shape(Is=0), 16) < a         # no shared-expert scratch
+
+
+# Fake device pointers: validation runs before any dereference or CUDA call.
+FAKE = 1 << 20
+
+
+def _call(moe, shape, T=0, ws_bytes=1 << 30, flags=0, x=FAKE, out=FAKE * 64, shared=True,
+          cfg_patch=None, ws=FAKE * 256):
+    cfg = moe.make_cfg(shape, flags)
+    cfg.workspace = ws
+    cfg.workspace_bytes = ws_bytes
+    if cfg_patch:
+        cfg_patch(cfg)
+    sh = moe.moe_shared_weights_t(FAKE, FAKE, FAKE, FAKE) if shared else None
+    vp = ctypes.c_void_p
+    return moe.lib.moe_layer_forward(vp(x), vp(FAKE), vp(FAKE), vp(FAKE), vp(FAKE), vp(FAKE), vp(FAKE),
+                                     ctypes.byref(sh) if sh is not None else None, vp(out), T,
+                                     ctypes.byref(cfg), None)
+
+
+def test_forward_validation_codes(moe):
+    s = _shape()
+    assert _call(moe, s) == 0                                           # T = 0: no-op
+    assert _call(moe, s, T=-1) == moe.MOE_ERR_INVALID_ARG
+    assert _call(moe, s, x=0) == moe.MOE_ERR_INVALID_ARG                # NULL x
+    assert _call(moe, s, x=FAKE + 4) == moe.MOE_ERR_INVALID_ARG         # misaligned
+    assert _call(moe, s, shared=False) == moe.MOE_ERR_INVALID_ARG       # Is > 0 needs shared
+    assert _call(moe, _shape(Is=0), shared=False) == 0
+    assert _call(moe, s, T=4, out=FAKE) == moe.MOE_ERR_INVALID_ARG      # out aliases x
+    assert _call(moe, s, T=4, ws_bytes=100) == moe.MOE_ERR_WORKSPACE
+    assert _call(moe, s, T=4, ws=0) == moe.MOE_ERR_WORKSPACE
+    assert _call(moe, s, ws=FAKE * 256 + 16) == moe.MOE_ERR_INVALID_ARG  # workspace alignment
+    assert _call(moe, _shape(H=1000)) == moe.MOE_ERR_UNSUPPORTED
+    assert _call(moe, _shape(I=200)) == moe.MOE_ERR_UNSUPPORTED
+    assert _call(moe, _shape(K=9, E=64)) == moe.MOE_ERR_UNSUPPORTED
+    assert _call(moe, _shape(K=5, E=4)) == moe.MOE_ERR_INVALID_ARG
+    assert _call(moe, _shape(routed_scaling=0.0)) == moe.MOE_ERR_INVALID_ARG
+    assert _call(moe, s, flags=1 << 7) == moe.MOE_ERR_INVALID_ARG
+    assert _call(moe, s, flags=moe.MOE_FORCE_DECODE | moe.MOE_FORCE_PREFILL) == moe.MOE_ERR_INVALID_ARG
+
+    def bad_size(c):
+        c.struct_size = 12
+    assert _call(moe, s, cfg_patch=bad_size) == moe.MOE_ERR_INVALID_ARG
+    assert moe.lib.moe_layer_forward(None, None, None, None, None, None, None, None, None, 0, None,
+                                     None) == moe.MOE_ERR_INVALID_ARG

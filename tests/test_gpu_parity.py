@@ -1,0 +1,191 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Every workload of the layer is covered: the Nano layer at T=16, the 23-layer
+Nano decode stack at T in {1,4,16,64} (compared layer by layer, the oracle fed
+the GPU's bf16 input of that layer), Nano prefill at T=4096, Zipf-skewed
+routing at T=16384, and the 256-expert top-8 layer at T in {1,32,512}.  Large
+cases check routing on every token and outputs on sampled tokens.  Edge cases:
+ragged T, raw int4 codes (code -8), no shared expert, K=1, K=E, E not a
+multiple of 32, exact ties, NaN bias, maximum H, batch independence and token
+permutation (bit-exact).
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from tests._parity import OUT_TOL, compare_layer, sample_tokens, to_cpu_layer
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def moe(cuda_device):
+    import int4_expert_ffn_sigmoid_b200 as m
+    return m
+
+
+def run(moe, x, layer, shape, residual=False, flags=0):
+    T = x.shape[0]
+    idx = torch.empty((T, shape.K), dtype=torch.int32, device=x.device)
+    w = torch.empty((T, shape.K), dtype=torch.float32, device=x.device)
+    f = flags | (moe.MOE_ADD_RESIDUAL if residual else 0) | moe.MOE_DEBUG_CHECK
+    out = moe.layer_forward(x, layer, shape, flags=f, topk_idx=idx, topk_w=w)
+    torch.cuda.synchronize()
+    return out, idx, w
+
+
+def check(moe, x, layer, shape, residual=False, sample=None, flags=0, layer_cpu=None):
+    out, idx, w = run(moe, x, layer, shape, residual, flags)
+    r = compare_layer(x, out, idx, w, layer_cpu or to_cpu_layer(layer), shape, residual, sample)
+    print(f"T={x.shape[0]} {r}")
+    return out, idx, w, r
+
+
+def test_nano_layer_t16(moe, cuda_device):
+    wl = workloads.WORKLOADS["nano_layer_t16"]
+    layer = workloads.make_layer(wl.shape, wl.wid, 0, cuda_device, wl.bias_mode)
+    x = workloads.make_x(wl.shape, 16, wl.wid, device=cuda_device)
+    check(moe, x, layer, wl.shape)
+
+
+@pytest.mark.parametrize("T", [1, 4, 16, 64])
+def test_nano_decode_stack(moe, cuda_device, T):
+    wl = workloads.WORKLOADS["nano_decode_stack"]
+    x = workloads.make_x(wl.shape, T, wl.wid, device=cuda_device)
+    x0 = x.clone()
+    for l in range(wl.layers):
+        layer = workloads.make_layer(wl.shape, wl.wid, l, cuda_device, wl.bias_mode)
+        x, _, _, r = check(moe, x, layer, wl.shape, residual=True)
+        del layer
+    assert torch.isfinite(x.float()).all()
+    assert not torch.equal(x, x0)
+
+
+def test_nano_prefill_t4096(moe, cuda_device):
+    wl = workloads.WORKLOADS["nano_prefill_t4096"]
+    layer = workloads.make_layer(wl.shape, wl.wid, 0, cuda_device, wl.bias_mode)
+    x = workloads.make_x(wl.shape, 4096, wl.wid, device=cuda_device)
+    _, idx, _, _ = check(moe, x, layer, wl.shape, sample=sample_tokens(4096, 40, 1))
+    loads = torch.bincount(idx.flatten().long(), minlength=64)
+    assert int(loads.min()) > 0            # zero bias: every expert receives tokens
+
+
+def test_nano_zipf_t16384(moe, cuda_device):
+    wl = workloads.WORKLOADS["nano_zipf_t16384"]
+    layer = workloads.make_layer(wl.shape, wl.wid, 0, cuda_device, wl.bias_mode)
+    x = workloads.make_x(wl.shape, 16384, wl.wid, device=cuda_device)
+    out, idx, w = run(moe, x, layer, wl.shape)
+    idx_np = idx.cpu().numpy()
+    loads = np.bincount(idx_np.reshape(-1), minlength=64)
+    hot = np.nonzero(idx_np == np.argmax(loads))[0][:3]
+    cold = np.nonzero(idx_np == np.argmin(loads))[0][:3]
+    r = compare_layer(x, out, idx, w, to_cpu_layer(layer), wl.shape, False,
+                      sample_tokens(16384, 32, 2, extra=np.concatenate([hot, cold])))
+    print("zipf loads", sorted(loads.tolist(), reverse=True)[:5], "...", sorted(loads.tolist())[:3], r)
+    assert loads.max() > 2000 and loads.min() < 200
+
+
+@pytest.mark.parametrize("T,n", [(1, 1), (32, 8), (512, 10)])
+def test_large_layer(moe, cuda_device, T, n):
+    wl = workloads.WORKLOADS["large_layer"]
+    layer = workloads.make_layer(wl.shape, wl.wid, 0, cuda_device, wl.bias_mode)
+    x = workloads.make_x(wl.shape, T, wl.wid, device=cuda_device)
+    check(moe, x, layer, wl.shape, sample=sample_tokens(T, n, 3))
+
+
+# --- edge cases on small shapes -------------------------------------------------
+
+SMALL = [
+    dict(H=128, E=40, K=3, I=128, Is=128, scale=1.3),
+    dict(H=256, E=8, K=8, I=256, Is=0, scale=1.0),     # K = E, no shared expert
+    dict(H=384, E=33, K=1, I=128, Is=256, scale=2.5),  # K = 1, E not a multiple of 32
+    dict(H=128, E=256, K=8, I=128, Is=128, scale=2.5),
+]
+
+
+@pytest.mark.parametrize("case", range(len(SMALL)))
+@pytest.mark.parametrize("T", [1, 3, 17, 64, 65, 300])
+@pytest.mark.parametrize("raw", [False, True])
+def test_small_shapes(moe, cuda_device, case, T, raw):
+    c = SMALL[case]
+    shape = workloads.LayerShape(c["H"], c["E"], c["K"], c["I"], c["Is"], c["scale"])
+    layer = workloads.make_layer(shape, 200 + case, 0, cuda_device, "uniform", raw_codes=raw)
+    if raw:  # larger router weights so raw-code experts still see a spread of scores
+        layer["router_w"].mul_(5)
+    x = workloads.make_x(shape, T, 200 + case, device=cuda_device)
+    check(moe, x, layer, shape, residual=(T % 2 == 1))
+
+
+def test_force_flags_same_result(moe, cuda_device):
+    c = SMALL[0]
+    shape = workloads.LayerShape(c["H"], c["E"], c["K"], c["I"], c["Is"], c["scale"])
+    layer = workloads.make_layer(shape, 210, 0, cuda_device)
+    x = workloads.make_x(shape, 40, 210, device=cuda_device)
+    a, _, _ = run(moe, x, layer, shape)
+    b, _, _ = run(moe, x, layer, shape, flags=moe.MOE_FORCE_DECODE)
+    c_, _, _ = run(moe, x, layer, shape, flags=moe.MOE_FORCE_PREFILL)
+    check(moe, x, layer, shape, flags=moe.MOE_FORCE_PREFILL)
+    assert torch.equal(a, b)
+    assert (a.float() - c_.float()).abs().max() <= 1e-2 * a.float().abs().max()
+
+
+def test_max_hidden(moe, cuda_device):
+    shape = workloads.LayerShape(H=16384, E=8, K=2, I=128, Is=128, routed_scaling=1.0)
+    layer = workloads.make_layer(shape, 220, 0, cuda_device)
+    x = workloads.make_x(shape, 5, 220, device=cuda_device)
+    check(moe, x, layer, shape)
+
+
+def test_exact_ties_lower_index(moe, cuda_device):
+    shape = workloads.LayerShape(H=128, E=8, K=2, I=128, Is=0, routed_scaling=1.0)
+    layer = workloads.make_layer(shape, 230, 0, cuda_device)
+    layer["router_w"][5] = layer["router_w"][1]
+    layer["router_w"][6] = layer["router_w"][1]
+    layer["router_bias"][:] = -1.0
+    layer["router_bias"][[1, 5, 6]] = 0.5
+    x = workloads.make_x(shape, 20, 230, device=cuda_device)
+    out, idx, w = run(moe, x, layer, shape)
+    assert idx[:, 0].eq(1).all() and idx[:, 1].eq(5).all()
+    torch.testing.assert_close(w, torch.full_like(w, 0.5), rtol=1e-6, atol=0)
+
+
+def test_nan_bias_never_selected(moe, cuda_device):
+    shape = workloads.LayerShape(H=128, E=8, K=3, I=128, Is=128, routed_scaling=1.0)
+    layer = workloads.make_layer(shape, 240, 0, cuda_device)
+    layer["router_bias"][2] = float("nan")
+    layer["router_bias"][4] = 10.0
+    x = workloads.make_x(shape, 9, 240, device=cuda_device)
+    out, idx, _, _ = check(moe, x, layer, shape)
+    assert not idx.eq(2).any() and idx[:, 0].eq(4).all()
+
+
+def test_batch_independence_and_permutation(moe, cuda_device):
+    wl = workloads.WORKLOADS["nano_layer_t16"]
+    layer = workloads.make_layer(wl.shape, wl.wid, 0, cuda_device, wl.bias_mode)
+    for T in (16, 200):
+        x = workloads.make_x(wl.shape, T, wl.wid, batch=5, device=cuda_device)
+        out, _, _ = run(moe, x, layer, wl.shape)
+        perm = torch.randperm(T, generator=torch.Generator().manual_seed(T)).to(cuda_device)
+        outp, _, _ = run(moe, x[perm].contiguous(), layer, wl.shape)
+        assert torch.equal(outp, out[perm])
+        for t in (0, T // 2, T - 1):
+            o1, _, _ = run(moe, x[t:t + 1].contiguous(), layer, wl.shape)
+            assert torch.equal(o1[0], out[t])
+
+
+def test_workspace_reuse_and_stream(moe, cuda_device):
+    """Two calls on one workspace, the second on a side stream, are independent."""
+    wl = workloads.WORKLOADS["nano_layer_t16"]
+    layer = workloads.make_layer(wl.shape, wl.wid, 0, cuda_device, wl.bias_mode)
+    m = moe.MoELayer(layer, wl.shape, 300)
+    xa = workloads.make_x(wl.shape, 300, wl.wid, batch=1, device=cuda_device)
+    xb = workloads.make_x(wl.shape, 7, wl.wid, batch=2, device=cuda_device)
+    ra = m(xa).clone()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        rb = m(xb)
+    s.synchronize()
+    assert torch.equal(m(xa), ra)
+    assert torch.equal(rb, moe.layer_forward(xb, layer, wl.shape))
