@@ -216,9 +216,17 @@ def make_events(n):
 
 
 def timed_steps(stack, steps, warmup, use_graph, flush, instrumented=False, dist_barrier=None):
-    """Returns (per-step ms list, per-stage ms sums per step, launches per step)."""
+    """Returns (per-step ms list, per-stage ms sums per step).
+
+    instrumented=True: the library records its per-stage events around every
+    kernel.  Events recorded inside a captured graph cannot be timed, so this
+    pass launches the C-ABI calls directly, behind a GPU sleep long enough for
+    the whole step to be queued first: the stage brackets then hold device
+    time only, not host launch latency."""
     L = len(stack.layers)
     stage_ev = [make_events(8) for _ in range(L)] if instrumented else None
+    if instrumented:
+        use_graph = False
     torch.cuda.synchronize()
     graphs = None
     if use_graph:
@@ -255,6 +263,8 @@ def timed_steps(stack, steps, warmup, use_graph, flush, instrumented=False, dist
     step_ms, stage_ms = [], []
     for i in range(steps):
         flush.zero_()
+        if instrumented:
+            torch.cuda._sleep(20_000_000)
         st[i].record()
         one(i % N_BATCHES)
         en[i].record()

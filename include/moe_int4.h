@@ -61,6 +61,8 @@ extern "C" {
 #define MOE_DEBUG_CHECK (1u << 1)   /* synchronise the stream and report device range checks */
 #define MOE_FORCE_DECODE (1u << 2)  /* use the small-batch (weight-streaming) kernels at any T */
 #define MOE_FORCE_PREFILL (1u << 3) /* use the large-batch (grouped GEMM) kernels at any T */
+#define MOE_OUT_F32 (1u << 4)       /* out is f32 [T][H] (the f32 sum, no bf16 rounding): for
+                                       checking the arithmetic apart from the output rounding */
 
 /* The always-resident shared expert (intermediate size Is).
  *   w13: uint8 [2*Is][H/2]  rows 0..Is-1 gate, rows Is..2*Is-1 up
@@ -127,11 +129,13 @@ size_t moe_layer_workspace_bytes(const moe_cfg_t* cfg, int32_t T);
  *   packed_w2  : uint8 [E][H][I/2]
  *   scales2    : f32  [E][H]
  *   shared_w   : the shared expert (required when cfg->Is > 0, else ignored)
- *   out        : bf16 [T][H]  (written; one round-to-nearest-even of the f32 sum)
+ *   out        : bf16 [T][H]  (written; one round-to-nearest-even of the f32 sum),
+ *                or f32 [T][H] under MOE_OUT_F32
  *   T          : tokens, 0..2^20 (T = 0 returns MOE_OK and launches nothing)
  *   cfg, stream: see above.
  * The routing weights and every expert contribution are accumulated in f32;
- * the gate/up intermediate is kept in fp16 or f32, never bf16.
+ * the SwiGLU intermediate h is kept in fp16 as h * 2^-8 (so |h| up to 1.6e7),
+ * never in bf16.
  * Returns MOE_OK or an MOE_ERR_* code; on an error nothing is launched
  * (except MOE_ERR_CUDA / MOE_ERR_DEVICE_CHECK, raised after launching). */
 int moe_layer_forward(const void* x, const float* router_w, const float* router_bias,

@@ -18,7 +18,7 @@ import torch
 
 __all__ = [
     "MoeError", "moe_cfg_t", "moe_shared_weights_t", "lib", "EXPORTED_SYMBOLS",
-    "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK", "MOE_FORCE_DECODE", "MOE_FORCE_PREFILL",
+    "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK", "MOE_FORCE_DECODE", "MOE_FORCE_PREFILL", "MOE_OUT_F32",
     "workspace_bytes", "layer_forward", "MoELayer", "decode_max_tokens", "LIB_PATH",
 ]
 
@@ -35,6 +35,7 @@ MOE_ADD_RESIDUAL = 1 << 0
 MOE_DEBUG_CHECK = 1 << 1
 MOE_FORCE_DECODE = 1 << 2
 MOE_FORCE_PREFILL = 1 << 3
+MOE_OUT_F32 = 1 << 4
 
 MOE_STAGE_ROUTE, MOE_STAGE_GATE_UP, MOE_STAGE_DOWN, MOE_STAGE_COMBINE = range(4)
 MOE_NUM_STAGES = 4
@@ -170,9 +171,10 @@ def layer_forward(x: torch.Tensor, layer: dict, shape, out: Optional[torch.Tenso
         _check_dev("sh_s2", layer["sh_s2"], torch.float32, (H,))
         sh.w13, sh.s13 = layer["sh_w13"].data_ptr(), layer["sh_s13"].data_ptr()
         sh.w2, sh.s2 = layer["sh_w2"].data_ptr(), layer["sh_s2"].data_ptr()
+    odt = torch.float32 if flags & MOE_OUT_F32 else torch.bfloat16
     if out is None:
-        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
-    _check_dev("out", out, torch.bfloat16, (T, H))
+        out = torch.empty((T, H), dtype=odt, device=x.device)
+    _check_dev("out", out, odt, (T, H))
     if workspace is None:
         workspace = new_workspace(shape, T, x.device, flags)
     if topk_idx is not None:

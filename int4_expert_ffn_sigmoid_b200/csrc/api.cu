@@ -6,19 +6,21 @@
 #include "moe_common.cuh"
 #include "moe_int4.h"
 #include "moe_launch.h"
+#include "moe_tc.h"
 
 namespace {
 
 using namespace moe;
 
-constexpr unsigned kKnownFlags = MOE_ADD_RESIDUAL | MOE_DEBUG_CHECK | MOE_FORCE_DECODE | MOE_FORCE_PREFILL;
+constexpr unsigned kKnownFlags =
+    MOE_ADD_RESIDUAL | MOE_DEBUG_CHECK | MOE_FORCE_DECODE | MOE_FORCE_PREFILL | MOE_OUT_F32;
 constexpr int32_t kMaxTokens = 1 << 20;
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct WsLayout {
-    size_t ctrl, idx, wts, logits, counts, offsets, bucket_e, bucket_n, bucket_off, ts13, ts2;
-    size_t tok_of_slot, slot_of, hist, h_r, h_s, y, total;
+    size_t ctrl, idx, wts, logits, counts, offsets, bucket_e, bucket_n, bucket_off, ts13, ts2, tcs1, tcs2;
+    size_t tok_of_slot, slot_of, hist, h_r, h_s, hexp, y, x_perm, total;
 };
 
 WsLayout ws_layout(const moe_cfg_t& c, int32_t T) {
@@ -41,12 +43,16 @@ WsLayout ws_layout(const moe_cfg_t& c, int32_t T) {
     L.bucket_off = take((E + 1) * 4);
     L.ts13 = take((E + 2) * 4);
     L.ts2 = take((E + 2) * 4);
+    L.tcs1 = take((E + 2) * 4);
+    L.tcs2 = take((E + 2) * 4);
     L.tok_of_slot = take(TK * 4);
     L.slot_of = take(TK * 4);
     L.hist = take((size_t)kRouterMaxBlocks * E * 4);
     L.h_r = take(TK * (size_t)c.I * 2);
     L.h_s = take((size_t)T * (size_t)c.Is * 2);
+    L.hexp = take((size_t)T * 4);
     L.y = take((TK + (c.Is > 0 ? (size_t)T : 0)) * (size_t)c.H * 4);
+    L.x_perm = take(TK * (size_t)c.H * 2);
     L.total = o;
     return L;
 }
@@ -124,8 +130,9 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
     for (const void* ptr : ptrs)
         if (ptr && !aligned(ptr, 16)) return MOE_ERR_INVALID_ARG;
     const size_t xbytes = (size_t)T * cfg->H * 2;
+    const size_t obytes = xbytes * ((cfg->flags & MOE_OUT_F32) ? 2 : 1);
     const uintptr_t xa = (uintptr_t)x, oa = (uintptr_t)out;
-    if (T > 0 && xa < oa + xbytes && oa < xa + xbytes) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && xa < oa + obytes && oa < xa + xbytes) return MOE_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(*cfg, T);
     if (!cfg->workspace || cfg->workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
     if (!aligned(cfg->workspace, 256)) return MOE_ERR_INVALID_ARG;
@@ -157,25 +164,34 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
     p.bucket_off = reinterpret_cast<int32_t*>(ws + L.bucket_off);
     p.ts13 = reinterpret_cast<int32_t*>(ws + L.ts13);
     p.ts2 = reinterpret_cast<int32_t*>(ws + L.ts2);
+    p.tcs1 = reinterpret_cast<int32_t*>(ws + L.tcs1);
+    p.tcs2 = reinterpret_cast<int32_t*>(ws + L.tcs2);
     p.tok_of_slot = reinterpret_cast<int32_t*>(ws + L.tok_of_slot);
     p.slot_of = reinterpret_cast<int32_t*>(ws + L.slot_of);
     p.hist = reinterpret_cast<int32_t*>(ws + L.hist);
     p.h_r = reinterpret_cast<__half*>(ws + L.h_r);
     p.h_s = reinterpret_cast<__half*>(ws + L.h_s);
+    p.hexp = reinterpret_cast<int32_t*>(ws + L.hexp);
     p.y = reinterpret_cast<float*>(ws + L.y);
     const int ntiles = cdiv(T, kRouterTileTokens);
     p.router_blocks = ntiles < kRouterMaxBlocks ? ntiles : kRouterMaxBlocks;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const bool small_router = T <= kDecodeMaxTokens;
+    const bool force_prefill = (cfg->flags & MOE_FORCE_PREFILL) != 0;
+    const bool small_router = T <= kDecodeMaxTokens && !force_prefill;
+    // Tensor-core grouped GEMMs for large batches; GEMM-2 tiles 256 output
+    // columns, so they need H % 256 == 0 (otherwise the mma.sync kernels run).
+    const bool use_tc = !small_router && !(cfg->flags & MOE_FORCE_DECODE) && cfg->H % 256 == 0;
+    p.x_perm = use_tc ? reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm) : nullptr;
     const long long TK = (long long)T * cfg->K;
     const long long routed_buckets = (cfg->E < TK ? cfg->E : TK) + cdiv(TK, kChunkTokens);
     const long long shared_chunks = cfg->Is > 0 ? cdiv(T, kChunkTokens) : 0;
-    const long long warps13 = (long long)(cfg->I / 8) * routed_buckets + (long long)(cfg->Is / 8) * shared_chunks;
-    const long long warps2 = (long long)(cfg->H / 16) * (routed_buckets + shared_chunks);
-    const int cap = sm_count() * 8;
-    const int grid13 = (int)(cdiv(warps13, 8) < cap ? cdiv(warps13, 8) : cap);
-    const int grid2 = (int)(cdiv(warps2, 8) < cap ? cdiv(warps2, 8) : cap);
+    // upper bounds of the weight-streaming kernels' CTA tasks
+    const long long tasks13 = (long long)(cfg->I / 64) * routed_buckets + (long long)(cfg->Is / 64) * shared_chunks;
+    const long long tasks2 = (long long)(cfg->H / 128) * (routed_buckets + shared_chunks);
+    const long long cap13 = experts_resident_ctas(0), cap2 = experts_resident_ctas(1);
+    const int grid13 = (int)(tasks13 < cap13 ? tasks13 : cap13);
+    const int grid2 = (int)(tasks2 < cap2 ? tasks2 : cap2);
 
     void* const* ev = cfg->stage_events;
     auto mark = [&](int idx) -> cudaError_t {
@@ -185,11 +201,21 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
     if (err == cudaSuccess) err = cudaMemsetAsync(p.ctrl, 0, sizeof(Ctrl), s);
     if (err == cudaSuccess) err = launch_router(p, small_router, s);
     if (err == cudaSuccess) err = mark(2 * MOE_STAGE_ROUTE + 1);
+    int tc_grid1 = 0, tc_grid2 = 0;
+    if (use_tc) {
+        const long long mt_routed = (cfg->E < TK ? cfg->E : TK) + cdiv(TK, 128);
+        const long long mt_shared = cfg->Is > 0 ? cdiv(T, 128) : 0;
+        const long long t1 = mt_routed * (cfg->I / 128) + mt_shared * (cfg->Is / 128);
+        const long long t2 = (mt_routed + mt_shared) * (cfg->H / 256);
+        const int sms = sm_count();
+        tc_grid1 = (int)(t1 < sms ? t1 : sms);
+        tc_grid2 = (int)(t2 < sms ? t2 : sms);
+    }
     if (err == cudaSuccess) err = mark(2 * MOE_STAGE_GATE_UP);
-    if (err == cudaSuccess) err = launch_experts_w13(p, grid13, s);
+    if (err == cudaSuccess) err = use_tc ? launch_tc_gemm(p, 1, tc_grid1, s) : launch_experts_w13(p, grid13, s);
     if (err == cudaSuccess) err = mark(2 * MOE_STAGE_GATE_UP + 1);
     if (err == cudaSuccess) err = mark(2 * MOE_STAGE_DOWN);
-    if (err == cudaSuccess) err = launch_experts_w2(p, grid2, s);
+    if (err == cudaSuccess) err = use_tc ? launch_tc_gemm(p, 2, tc_grid2, s) : launch_experts_w2(p, grid2, s);
     if (err == cudaSuccess) err = mark(2 * MOE_STAGE_DOWN + 1);
     if (err == cudaSuccess) err = mark(2 * MOE_STAGE_COMBINE);
     if (err == cudaSuccess) err = launch_combine(p, s);

@@ -11,8 +11,8 @@ namespace moe {
 
 // Largest T that takes the weight-streaming (small-batch) path by default.
 constexpr int kDecodeMaxTokens = 64;
-// Tokens of one bucket handled by one expert-kernel task (8 mma n-tiles of 8).
-constexpr int kChunkTokens = 64;
+// Tokens of one bucket handled by one expert-kernel task (2 mma n-tiles of 8).
+constexpr int kChunkTokens = 16;
 // Large-batch router: tokens per tile and the cap on router CTAs.
 constexpr int kRouterTileTokens = 16;
 constexpr int kRouterMaxBlocks = 296;
@@ -21,6 +21,14 @@ constexpr int kDecodeRouterTok = 8;
 constexpr int kDecodeRouterExp = 8;
 constexpr int kMaxK = 8;
 constexpr int kMaxE = 256;
+// The SwiGLU intermediate h of token t is stored in fp16 as h * 2^-k_t, with
+// k_t = 8 + floor(log2(mean_h x[t,h]^2)) clamped to [kHExpMin, kHExpMax]:
+// h grows like |x|^2, so the stored value stays in fp16's normal range
+// whatever the input scale.  The factor is exact and undone in the down
+// projection's epilogue.
+constexpr int kHExpBase = 8;
+constexpr int kHExpMin = -40;
+constexpr int kHExpMax = 60;
 
 // Device status bits (set by range checks, read back under MOE_DEBUG_CHECK).
 enum : unsigned {
@@ -28,6 +36,7 @@ enum : unsigned {
     ST_BAD_SLOT = 2u,    // a slot outside [0, T*K)
     ST_BAD_COUNT = 4u,   // bucket counts do not sum to T*K
     ST_BAD_TASK = 8u,    // a task resolved to a bucket outside the list
+    ST_TIMEOUT = 16u,    // a bounded pipeline wait of the tensor-core kernel gave up
 };
 
 // First 256 bytes of the workspace.  Zeroed at the start of every call.
@@ -37,7 +46,13 @@ struct Ctrl {
     int n_buckets;      // non-empty routed buckets + the shared bucket
     int tasks13;        // gate/up tasks over all buckets
     int tasks2;         // down tasks over all buckets
-    int pad[59];
+    int tc_tiles1;      // tensor-core GEMM-1 tiles over the routed buckets
+    int tc_tiles2;      // tensor-core GEMM-2 tiles over the routed buckets
+    int claim13;        // next gate/up task to claim (weight-streaming kernel)
+    int claim2;         // next down task to claim
+    unsigned blk_done[kDecodeMaxTokens / 8];  // small-batch router: CTAs done per token block
+    unsigned sel_done;  // small-batch router: token blocks whose selection is done
+    int pad[46];
 };
 static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
 
@@ -75,53 +90,47 @@ struct Params {
     int32_t* bucket_off;  // [E+1]
     int32_t* ts13;        // [E+2] exclusive prefix of gate/up tasks per bucket
     int32_t* ts2;         // [E+2] exclusive prefix of down tasks per bucket
+    int32_t* tcs1;        // [E+2] exclusive prefix of tensor-core GEMM-1 tiles (routed buckets)
+    int32_t* tcs2;        // [E+2] exclusive prefix of tensor-core GEMM-2 tiles (routed buckets)
+    __nv_bfloat16* x_perm;  // [T*K][H] tokens gathered in slot order (tensor-core path), or null
     int32_t* tok_of_slot; // [T*K]
     int32_t* slot_of;     // [T*K] slot of (t, k)
     int32_t* hist;        // [router blocks][E]
     __half* h_r;          // [T*K][I]  routed SwiGLU intermediate
     __half* h_s;          // [T][Is]   shared SwiGLU intermediate
+    int32_t* hexp;        // [T] per-token exponent k_t of the h storage scale
     float* y;             // [T*K + T][H] expert outputs (already row-scaled)
     int router_blocks;
 };
 
 // ---------------------------------------------------------------------------
-// int4 -> 16-bit float conversion by the exponent-bias ("magic number")
-// technique of Kim et al., "Who Says Elephants Can't Run" (2022): the 4-bit
-// code, made unsigned by flipping its sign bit (c + 8), is OR-ed into the low
-// mantissa bits of a 16-bit float whose value is 2^m (ulp 1), giving 2^m + c + 8
-// exactly; subtracting 2^m + 8 leaves c exactly.  bf16: 2^7 = 0x4300;
-// fp16: 2^10 = 0x6400.  Output pair s holds (nibble s, nibble s+4) of the
-// 32-bit word, low half first; callers pair activations the same way.
+// int4 -> 16-bit float by the exponent-bias ("magic number") technique of
+// Kim et al., "Who Says Elephants Can't Run" (2022): the 4-bit code c, made
+// unsigned by flipping its sign bit (c + 8), is OR-ed into the low mantissa
+// bits of a 16-bit float equal to 2^m with ulp 1, which gives exactly
+// 2^m + 8 + c.  The weight-streaming kernels feed these *biased* values to the
+// tensor cores and remove the bias from the f32 result (bias * sum of the
+// activations), which saves the subtraction.  bf16: 2^7 = 0x4300 (bias 136);
+// fp16: 2^10 = 0x6400 (bias 1032).  Output pair j holds elements (2j, 2j+1)
+// of the word, low half first (natural order).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void int4x8_to_bf16x2(uint32_t w, uint32_t (&o)[4]) {
-    const uint32_t v = w ^ 0x88888888u;
-    const __nv_bfloat162 bias = __halves2bfloat162(__ushort_as_bfloat16(0x4308), __ushort_as_bfloat16(0x4308));
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        uint32_t t = ((v >> (4 * s)) & 0x000F000Fu) | 0x43004300u;
-        __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&t), bias);
-        o[s] = *reinterpret_cast<uint32_t*>(&r);
-    }
-}
+constexpr uint32_t kMagicBf16 = 0x43004300u;
+constexpr uint32_t kMagicF16 = 0x64006400u;
+constexpr float kBiasBf16 = 136.0f;
+constexpr float kBiasF16 = 1032.0f;
+constexpr uint32_t kOnesBf16 = 0x3F803F80u;
+constexpr uint32_t kOnesF16 = 0x3C003C00u;
 
-__device__ __forceinline__ void int4x8_to_f16x2(uint32_t w, uint32_t (&o)[4]) {
+template <uint32_t kMagic>
+__device__ __forceinline__ void int4x8_biased(uint32_t w, uint32_t (&o)[4]) {
     const uint32_t v = w ^ 0x88888888u;
-    const __half2 bias = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        uint32_t t = ((v >> (4 * s)) & 0x000F000Fu) | 0x64006400u;
-        __half2 r = __hsub2(*reinterpret_cast<__half2*>(&t), bias);
-        o[s] = *reinterpret_cast<uint32_t*>(&r);
-    }
-}
-
-// Eight consecutive 16-bit activations (a uint4) -> the four pairs
-// (e0,e4), (e1,e5), (e2,e6), (e3,e7), matching int4x8_to_*x2.
-__device__ __forceinline__ void pair8(const uint4& v, uint32_t (&o)[4]) {
-    o[0] = __byte_perm(v.x, v.z, 0x5410);
-    o[1] = __byte_perm(v.x, v.z, 0x7632);
-    o[2] = __byte_perm(v.y, v.w, 0x5410);
-    o[3] = __byte_perm(v.y, v.w, 0x7632);
+    const uint32_t v4 = v >> 4;
+    // half 0 <- low nibble of byte j of v (element 2j); half 1 <- low nibble
+    // of byte j of v >> 4 (element 2j + 1)
+    o[0] = (__byte_perm(v, v4, 0x0400) & 0x000F000Fu) | kMagic;
+    o[1] = (__byte_perm(v, v4, 0x0501) & 0x000F000Fu) | kMagic;
+    o[2] = (__byte_perm(v, v4, 0x0602) & 0x000F000Fu) | kMagic;
+    o[3] = (__byte_perm(v, v4, 0x0703) & 0x000F000Fu) | kMagic;
 }
 
 // Streamed weights: read once, keep out of L1.

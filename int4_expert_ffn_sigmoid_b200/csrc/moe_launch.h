@@ -13,6 +13,9 @@ cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream)
 cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream);
 // Expert down projection (weight-streaming mma.sync kernel).
 cudaError_t launch_experts_w2(const Params& p, int grid, cudaStream_t stream);
+// CTAs of the weight-streaming kernel `which` (0: gate/up, 1: down) that fit
+// on the device at once (the persistent grid size).
+int experts_resident_ctas(int which);
 // Weighted combine + shared expert (+ residual) -> bf16 out.
 cudaError_t launch_combine(const Params& p, cudaStream_t stream);
 

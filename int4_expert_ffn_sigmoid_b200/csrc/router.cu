@@ -35,6 +35,25 @@ __device__ __forceinline__ float warp_sum_tree(float v) {
     return v;
 }
 
+// Exponent k_t of the token's h storage scale 2^-k_t (one warp):
+// k_t = 8 + floor(log2(mean_h x[t,h]^2)), the mean square summed in the same
+// lane order as the router logits.
+__device__ __forceinline__ void token_hexp(const Params& p, int t, int lane) {
+    const __nv_bfloat16* xr = p.x + (size_t)t * p.H;
+    float acc = 0.f;
+    for (int i = 0; i < p.H / 128; ++i) {
+        const uint2 xv = __ldg(reinterpret_cast<const uint2*>(xr + i * 128 + lane * 4));
+        const float a = bf16lo(xv.x), b = bf16hi(xv.x), c = bf16lo(xv.y), d = bf16hi(xv.y);
+        acc = fmaf(a, a, acc);
+        acc = fmaf(b, b, acc);
+        acc = fmaf(c, c, acc);
+        acc = fmaf(d, d, acc);
+    }
+    const float ms = warp_sum_tree(acc) / (float)p.H;
+    const int e = (ms > 0.f && isfinite(ms)) ? ilogbf(ms) : 0;
+    if (lane == 0) p.hexp[t] = min(max(kHExpBase + e, kHExpMin), kHExpMax);
+}
+
 // Top-K of one token (one warp).  Lane l holds experts l, l+32, ...  The key
 // is sigmoid(L) + bias (NaN -> -inf); ties go to the lower expert index.  The
 // weight of the k-th pick is scale * s_k / (s_0 + ... + s_{K-1}).
@@ -150,37 +169,53 @@ __device__ void finalize_buckets(const Params& p, const int* s_cnt, int* s_off) 
     __syncthreads();
     if (warp == 0) {
         const int nb = s_nb;
-        int base13 = 0, base2 = 0;
+        int base13 = 0, base2 = 0, baset1 = 0, baset2 = 0;
         for (int b0 = 0; b0 < nb; b0 += 32) {
             const int b = b0 + lane;
-            int n13 = 0, n2 = 0;
+            int n13 = 0, n2 = 0, nt1 = 0, nt2 = 0;
             if (b < nb) {
                 const int e = p.bucket_e[b];
                 const int irow = (e == E) ? p.Is : p.I;
-                const int ch = chunks_of(p.bucket_n[b]);
-                n13 = (irow / 8) * ch;
-                n2 = (p.H / 16) * ch;
+                const int n = p.bucket_n[b];
+                const int ch = chunks_of(n);
+                n13 = (irow / 64) * ch;   // CTA tasks: 64 gate/up rows x 64 tokens
+                n2 = (p.H / 128) * ch;    // CTA tasks: 128 down rows x 64 tokens
+                if (e != E) {  // tensor-core tiles: 128 tokens x 128 features / 256 columns
+                    const int mt = (n + 127) / 128;
+                    nt1 = mt * (p.I / 128);
+                    nt2 = mt * (p.H / 256);
+                }
             }
-            int i13 = n13, i2 = n2;
+            int i13 = n13, i2 = n2, it1 = nt1, it2 = nt2;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int a = __shfl_up_sync(0xffffffffu, i13, o);
                 const int c2 = __shfl_up_sync(0xffffffffu, i2, o);
-                if (lane >= o) { i13 += a; i2 += c2; }
+                const int d1 = __shfl_up_sync(0xffffffffu, it1, o);
+                const int d2 = __shfl_up_sync(0xffffffffu, it2, o);
+                if (lane >= o) { i13 += a; i2 += c2; it1 += d1; it2 += d2; }
             }
             if (b < nb) {
                 p.ts13[b] = base13 + i13 - n13;
                 p.ts2[b] = base2 + i2 - n2;
+                p.tcs1[b] = baset1 + it1 - nt1;
+                p.tcs2[b] = baset2 + it2 - nt2;
             }
             base13 += __shfl_sync(0xffffffffu, i13, 31);
             base2 += __shfl_sync(0xffffffffu, i2, 31);
+            baset1 += __shfl_sync(0xffffffffu, it1, 31);
+            baset2 += __shfl_sync(0xffffffffu, it2, 31);
         }
         if (lane == 0) {
             p.ts13[nb] = base13;
             p.ts2[nb] = base2;
+            p.tcs1[nb] = baset1;
+            p.tcs2[nb] = baset2;
             p.ctrl->n_buckets = nb;
             p.ctrl->tasks13 = base13;
             p.ctrl->tasks2 = base2;
+            p.ctrl->tc_tiles1 = baset1;
+            p.ctrl->tc_tiles2 = baset2;
         }
     }
     __syncthreads();
@@ -189,27 +224,39 @@ __device__ void finalize_buckets(const Params& p, const int* s_cnt, int* s_off) 
 // ---------------------------------------------------------------------------
 // Small batch (T <= kDecodeMaxTokens): grid (ceil(T/8), ceil(E/8)); warp w of
 // CTA (bx, by) computes the logits of expert 8*by + w for tokens 8*bx ...
-// 8*bx + 7.  The last CTA to finish selects, counts, scans and scatters.
+// 8*bx + 7.  The last CTA of each token block selects that block's tokens
+// (one warp per token); the last of those counts, scans and scatters.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) router_small_kernel(Params p) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int t0 = blockIdx.x * kDecodeRouterTok;
     const int e = blockIdx.y * kDecodeRouterExp + warp;
     const int nt = min(kDecodeRouterTok, p.T - t0);
+    if (blockIdx.y == 0 && warp < nt) token_hexp(p, t0 + warp, lane);
     if (e < p.E) {
         float acc[kDecodeRouterTok];
 #pragma unroll
         for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = 0.f;
         const float4* W = reinterpret_cast<const float4*>(p.rw + (size_t)e * p.H);
-        const int nblk = p.H / 128;
-        for (int i = 0; i < nblk; ++i) {
-            const float4 wv = __ldg(W + i * 32 + lane);
+        const int nblk = p.H / 128;  // processed 4 blocks per batch of loads
+        for (int i0 = 0; i0 < nblk; i0 += 4) {
+            float4 wv[4];
+            uint2 xv[4][kDecodeRouterTok];
 #pragma unroll
-            for (int tt = 0; tt < kDecodeRouterTok; ++tt) {
-                if (tt < nt) {
-                    const uint2 xv = __ldg(reinterpret_cast<const uint2*>(
-                        p.x + (size_t)(t0 + tt) * p.H + i * 128 + lane * 4));
-                    acc[tt] = dot_step(acc[tt], xv, wv);
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u;
+                wv[u] = i < nblk ? __ldg(W + i * 32 + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int tt = 0; tt < kDecodeRouterTok; ++tt)
+                    xv[u][tt] = (i < nblk && tt < nt)
+                                    ? __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)(t0 + tt) * p.H + i * 128 + lane * 4))
+                                    : make_uint2(0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (i0 + u < nblk) {
+#pragma unroll
+                    for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = dot_step(acc[tt], xv[u][tt], wv[u]);
                 }
             }
         }
@@ -220,36 +267,43 @@ __global__ void __launch_bounds__(256) router_small_kernel(Params p) {
         }
     }
 
+    // ---- last CTA of this token block: selection of its tokens
     __shared__ int s_last;
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) {
-        const unsigned n = gridDim.x * gridDim.y;
-        s_last = (atomicAdd(&p.ctrl->done, 1u) == n - 1);
-    }
+    if (threadIdx.x == 0) s_last = (atomicAdd(&p.ctrl->blk_done[blockIdx.x], 1u) == gridDim.y - 1);
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    __shared__ float s_lg[kDecodeRouterTok * kMaxE];
+    for (int i = threadIdx.x; i < nt * p.E; i += blockDim.x) s_lg[i] = __ldcg(p.logits + (size_t)t0 * p.E + i);
+    __syncthreads();
+    if (warp < nt) {
+        const int sel = select_token<false>(p, t0 + warp, s_lg + warp * p.E, lane);
+        if (lane < p.K && (sel < 0 || sel >= p.E)) atomicOr(&p.ctrl->status, ST_BAD_EXPERT);
+    }
 
+    // ---- last token block: counts, scan, bucket and task lists, slots
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(&p.ctrl->sel_done, 1u) == gridDim.x - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
     __shared__ int s_idx[kDecodeMaxTokens * kMaxK];
     __shared__ int s_cnt[kMaxE];
     __shared__ int s_off[kMaxE];
+    const int TK = p.T * p.K;
     for (int i = threadIdx.x; i < p.E; i += blockDim.x) s_cnt[i] = 0;
     __syncthreads();
-    for (int t = warp; t < p.T; t += 8) {
-        int sel = select_token<true>(p, t, p.logits + (size_t)t * p.E, lane);
-        if (lane < p.K) {
-            if (sel < 0 || sel >= p.E) {
-                atomicOr(&p.ctrl->status, ST_BAD_EXPERT);
-                sel = 0;
-            }
-            s_idx[t * p.K + lane] = sel;
-            atomicAdd(&s_cnt[sel], 1);
-        }
+    for (int i = threadIdx.x; i < TK; i += blockDim.x) {
+        int ex = __ldcg(p.idx + i);
+        if (ex < 0 || ex >= p.E) ex = 0;  // reported above; keep every index in range
+        s_idx[i] = ex;
+        atomicAdd(&s_cnt[ex], 1);
     }
     __syncthreads();
     finalize_buckets(p, s_cnt, s_off);
-    const int TK = p.T * p.K;
     for (int i = threadIdx.x; i < TK; i += blockDim.x) {
         const int ex = s_idx[i];
         int rank = 0;
@@ -263,7 +317,6 @@ __global__ void __launch_bounds__(256) router_small_kernel(Params p) {
         p.slot_of[i] = slot;
         p.tok_of_slot[slot] = i / p.K;
     }
-    if (threadIdx.x == 0) p.ctrl->done = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -284,6 +337,7 @@ __global__ void __launch_bounds__(256) router_large_kernel(Params p) {
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int t0 = tile * kRouterTileTokens;
         const int nt = min(kRouterTileTokens, p.T - t0);
+        for (int tt = warp; tt < nt; tt += 8) token_hexp(p, t0 + tt, lane);
         for (int e0 = warp; e0 < E; e0 += 16) {
             const int e1 = e0 + 8;
             const bool has1 = e1 < E;
@@ -387,6 +441,16 @@ __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
             p.tok_of_slot[slot] = t0 + i / K;
         }
         __syncthreads();
+        if (p.x_perm) {  // copy each token row to its slots (one warp per slot)
+            const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+            for (int i = warp; i < n; i += blockDim.x / 32) {
+                if (s_idx[i] < 0) continue;
+                const int slot = p.slot_of[(size_t)t0 * K + i];
+                const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)(t0 + i / K) * p.H);
+                uint4* dst = reinterpret_cast<uint4*>(p.x_perm + (size_t)slot * p.H);
+                for (int c = lane; c < p.H / 8; c += 32) dst[c] = __ldg(src + c);
+            }
+        }
         for (int e = threadIdx.x; e < E; e += blockDim.x) {
             int c = 0;
             for (int j = 0; j < n; ++j) c += (s_idx[j] == e);

@@ -10,6 +10,16 @@ Bars (the layer's stated acceptance criteria):
     with out the GPU's bf16 output widened exactly and ref the oracle's f64
     result evaluated with the GPU's selection (identical to the oracle's own
     selection except at ties).
+
+Two further bars, derived from the arithmetic, for shapes whose rows are too
+short for the 2e-3 bar to leave room above the bf16 output rounding (that
+rounding alone averages ~1.7e-3 and varies more when a token has few elements):
+  * OUT_F32_TOL: the f32 output mode (no output rounding) against the exact
+    result.  The kernels' own error is dominated by the fp16 intermediate h
+    (unit roundoff 2^-11 = 4.9e-4, i.e. ~2.8e-4 RMS relative), so 1e-3 is met
+    with margin and any wrong term (relative error O(1)) fails it;
+  * and, bit for bit, the bf16 output equals round-to-nearest-even of the f32
+    output of the same call (the output rounding is the only difference).
 """
 from __future__ import annotations
 
@@ -21,6 +31,7 @@ import oracle
 TIE_MARGIN = 1e-6
 W_RTOL = 1e-6
 OUT_TOL = 2e-3
+OUT_F32_TOL = 1e-3
 
 
 def to_cpu_layer(layer: dict) -> dict:
@@ -50,17 +61,24 @@ def check_routing(idx_gpu: np.ndarray, w_gpu: np.ndarray, ref: dict, bias: np.nd
     return ties, werr
 
 
-def rel_l2(out_gpu: torch.Tensor, ref: np.ndarray) -> np.ndarray:
+def rel_l2(out_gpu: torch.Tensor, ref: np.ndarray, against=None) -> np.ndarray:
+    """||out - against|| / ||ref|| per token (against defaults to ref)."""
     o = out_gpu.detach().float().cpu().numpy().astype(np.float64)
-    num = np.linalg.norm(o - ref, axis=1)
+    a = ref if against is None else against
+    num = np.linalg.norm(o - a, axis=1)
     den = np.linalg.norm(ref, axis=1)
     return num / np.maximum(den, 1e-300)
 
 
+def bf16_round(ref: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(ref).to(torch.bfloat16).double().numpy()
+
+
 def compare_layer(x: torch.Tensor, out: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, layer_cpu: dict,
-                  shape, residual: bool, sample=None) -> dict:
+                  shape, residual: bool, sample=None, tol: float = OUT_TOL, rounded: bool = False) -> dict:
     """Full comparison.  Routing is checked on every token; outputs on
-    ``sample`` (token indices; default all)."""
+    ``sample`` (token indices; default all).  ``rounded``: compare with the
+    correctly rounded bf16 result instead of the exact one."""
     xc = x.detach().cpu()
     ref_r = oracle.route(xc, layer_cpu["router_w"], layer_cpu["router_bias"], shape.K, shape.routed_scaling)
     idx_g = idx.detach().cpu().numpy()
@@ -70,10 +88,11 @@ def compare_layer(x: torch.Tensor, out: torch.Tensor, idx: torch.Tensor, w: torc
     tok = np.arange(T) if sample is None else np.unique(np.asarray(sample, np.int64))
     ref = oracle.moe_tokens(xc, layer_cpu, shape, residual=residual, tokens=tok.astype(np.int32),
                             idx_override=idx_g[tok])
-    err = rel_l2(out[torch.from_numpy(tok).to(out.device)], ref["out"])
+    o = out[torch.from_numpy(tok).to(out.device)]
+    err = rel_l2(o, ref["out"], bf16_round(ref["out"]) if rounded else None)
     assert np.all(np.isfinite(err)), "non-finite output"
     worst = int(tok[int(np.argmax(err))])
-    assert err.max() <= OUT_TOL, f"per-token rel L2 {err.max():.3e} > {OUT_TOL} at token {worst}"
+    assert err.max() <= tol, f"per-token rel L2 {err.max():.3e} > {tol} at token {worst}"
     return dict(ties=len(ties), max_rel_l2=float(err.max()), mean_rel_l2=float(err.mean()),
                 max_w_rel=werr, tokens_checked=len(tok))
 
