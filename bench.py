@@ -151,20 +151,28 @@ def step_bytes_flops(shape, T, uniq_per_layer):
     return nbytes, flops
 
 
-def gate_up_bytes(shape, T, uniq):
-    """Algorithmic bytes of one gate/up launch: the w13 codes + scales of every
-    touched routed expert and of the shared expert, x read once, h written."""
-    H, K, I, Is = shape.H, shape.K, shape.I, shape.Is
-    per_expert = 2 * I * H // 2 + 2 * I * 4
-    shared = (2 * Is * H // 2 + 2 * Is * 4) if Is else 0
-    return uniq * per_expert + shared + T * H * 2 + T * K * I * 2 + T * Is * 2
+def stage_work(stage, shape, T, uniq):
+    """Algorithmic (bytes, flops) of one launch of a layer stage.
 
-
-def down_bytes(shape, T, uniq):
+    gate_up: the w13 codes + scales of every touched routed expert and of the
+    shared expert, the activations read once, h written; 2 flop per MAC of
+    gate and up.  down: the w2 codes + scales, h read, y (f32) written.  Only
+    real tokens count (no tile padding), scratch traffic beyond that is not
+    algorithmic."""
     H, K, I, Is = shape.H, shape.K, shape.I, shape.Is
-    per_expert = H * I // 2 + H * 4
-    shared = (H * Is // 2 + H * 4) if Is else 0
-    return uniq * per_expert + shared + T * K * I * 2 + T * Is * 2 + (T * K + (T if Is else 0)) * H * 4
+    if stage == "gate_up":
+        per_expert = 2 * I * H // 2 + 2 * I * 4
+        shared = (2 * Is * H // 2 + 2 * Is * 4) if Is else 0
+        nbytes = uniq * per_expert + shared + T * H * 2 + T * K * I * 2 + T * Is * 2
+        flops = 4 * T * K * H * I + 4 * T * H * Is
+    elif stage == "down":
+        per_expert = H * I // 2 + H * 4
+        shared = (H * Is // 2 + H * 4) if Is else 0
+        nbytes = uniq * per_expert + shared + T * K * I * 2 + T * Is * 2 + (T * K + (T if Is else 0)) * H * 4
+        flops = 2 * T * K * H * I + 2 * T * H * Is
+    else:
+        raise ValueError(stage)
+    return nbytes, flops
 
 
 # --------------------------------------------------------------------------- our arm
@@ -392,23 +400,27 @@ def run_ours(args, rank, world, device, dist):
     # dominant kernel (largest per-step stage time) and its roofline
     stage_mean = [statistics.mean(s[k] for s in stage_ms) for k in range(4)]
     names = moe.STAGE_NAMES
-    dom = int(np.argmax(stage_mean))
-    launches = args.steps * L
-    if dom == 1:
-        alg = statistics.mean(sum(gate_up_bytes(wl.shape, T, u) for u in uniq[i % N_BATCHES]) for i in range(args.steps))
-    elif dom == 2:
-        alg = statistics.mean(sum(down_bytes(wl.shape, T, u) for u in uniq[i % N_BATCHES]) for i in range(args.steps))
+    dom = 1 if stage_mean[1] >= stage_mean[2] else 2  # the dominant expert kernel
+    tc_path = T > moe.decode_max_tokens() and wl.shape.H % 256 == 0
+    kname = (("grouped_gemm_kernel<1>" if dom == 1 else "grouped_gemm_kernel<2>") if tc_path
+             else ("experts_w13_kernel" if dom == 1 else "experts_w2_kernel"))
+    work = [[stage_work(names[dom], wl.shape, T, u) for u in uniq[i % N_BATCHES]] for i in range(args.steps)]
+    alg_b = statistics.mean(sum(w[0] for w in ws) for ws in work) / L
+    alg_f = statistics.mean(sum(w[1] for w in ws) for ws in work) / L
+    per_launch_s = stage_mean[dom] / L / 1e3
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if alg_f / alg_b >= ridge:
+        achieved = alg_f / per_launch_s / 1e12
+        roofline = {"bound": "tensor", "kernel": kname, "achieved": round(achieved, 2),
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                    "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json bf16_tflops, burst)"}
     else:
-        alg = None
-    per_launch_us = stage_mean[dom] / L * 1e3
-    roofline = None
-    if alg is not None:
-        achieved = alg / L / (per_launch_us / 1e6) / 1e9
-        roofline = {"bound": "hbm", "kernel": f"experts_{'w13' if dom == 1 else 'w2'}_kernel",
-                    "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
-                    "alg_bytes_per_launch": int(alg / L), "avg_launch_us": round(per_launch_us, 3),
+        achieved = alg_b / per_launch_s / 1e9
+        roofline = {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                     "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy)"}
+    roofline.update({"traffic": None, "alg_bytes_per_launch": int(alg_b), "alg_flops_per_launch": int(alg_f),
+                     "avg_launch_us": round(per_launch_s * 1e6, 3)})
 
     sweep = {}
     if wl.name == "nano_decode_stack" and not args.no_sweep:
@@ -431,6 +443,7 @@ def run_ours(args, rank, world, device, dist):
         cpu = {"value": round(v, 2), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
 
     kernels_per_layer = 4 if T <= moe.decode_max_tokens() else 5
+    launches = args.steps * L
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,

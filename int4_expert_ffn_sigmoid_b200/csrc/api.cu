@@ -189,7 +189,8 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
     // upper bounds of the weight-streaming kernels' CTA tasks
     const long long tasks13 = (long long)(cfg->I / 64) * routed_buckets + (long long)(cfg->Is / 64) * shared_chunks;
     const long long tasks2 = (long long)(cfg->H / 128) * (routed_buckets + shared_chunks);
-    const long long cap13 = experts_resident_ctas(0), cap2 = experts_resident_ctas(1);
+    const long long cap13 = experts_resident_ctas(0, cfg->H);
+    const long long cap2 = experts_resident_ctas(1, cfg->I > cfg->Is ? cfg->I : cfg->Is);
     const int grid13 = (int)(tasks13 < cap13 ? tasks13 : cap13);
     const int grid2 = (int)(tasks2 < cap2 ? tasks2 : cap2);
 
@@ -198,7 +199,6 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
         return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[idx]), s) : cudaSuccess;
     };
     cudaError_t err = mark(2 * MOE_STAGE_ROUTE);
-    if (err == cudaSuccess) err = cudaMemsetAsync(p.ctrl, 0, sizeof(Ctrl), s);
     if (err == cudaSuccess) err = launch_router(p, small_router, s);
     if (err == cudaSuccess) err = mark(2 * MOE_STAGE_ROUTE + 1);
     int tc_grid1 = 0, tc_grid2 = 0;

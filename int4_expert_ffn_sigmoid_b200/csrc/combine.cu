@@ -14,6 +14,8 @@ namespace moe {
 __global__ void __launch_bounds__(256) combine_kernel(Params p) {
     const int t = blockIdx.x;
     const int j = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
+    pdl_wait();
+    pdl_release();
     if (j >= p.H) return;
     const int K = p.K, H = p.H;
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
@@ -47,9 +49,7 @@ __global__ void __launch_bounds__(256) combine_kernel(Params p) {
 }
 
 cudaError_t launch_combine(const Params& p, cudaStream_t stream) {
-    dim3 grid(p.T, (p.H + 1023) / 1024);
-    combine_kernel<<<grid, 256, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, dim3(p.T, (p.H + 1023) / 1024), dim3(256), 0, stream, p);
 }
 
 }  // namespace moe

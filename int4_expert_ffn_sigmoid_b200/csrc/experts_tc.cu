@@ -14,12 +14,14 @@
 // N) x 64 reduction elements per pipeline stage.  GEMM-1's 256 columns are 128
 // gate rows and the 128 up rows of the same features, so one thread of the
 // epilogue holds gate and up of one (token, feature) pair.
-// Roles (320 threads):
+// Roles (448 threads):
 //   warp 0      TMA producer (activation tile, raw int4 weight tile) and TMEM owner
 //   warp 1      MMA issuer (one thread, tcgen05.mma kind::f16, M=128 N=256 K=16)
-//   warps 2-5   dequantisers: raw int4 -> exact 16-bit integers in the 128-byte
-//               swizzled K-major layout of the B operand (row scale applied later)
-//   warps 6-9   epilogue: tcgen05.ld of the accumulator, scales, SwiGLU, stores
+//   warps 2-9   dequantisers, one B row per thread: raw int4 -> exact 16-bit
+//               integers in the 128-byte swizzled K-major layout of the B
+//               operand (the row scale is applied in the epilogue)
+//   warps 10-13 epilogue: tcgen05.ld of the accumulator, scales (staged in
+//               shared memory per tile), SwiGLU, stores
 // Every mbarrier wait is bounded (clock64); on timeout the CTA records
 // ST_TIMEOUT in the status word, drains what it issued and exits.
 #include <cuda.h>
@@ -37,11 +39,12 @@ constexpr int A_BYTES = BM * BK * 2;    // 16 KiB, bf16/fp16 activations
 constexpr int B_BYTES = BN * BK * 2;    // 32 KiB, dequantised weights
 constexpr int RAW_BYTES = BN * BK / 2;  // 8 KiB, packed int4 weights
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RAW_BYTES;
-constexpr int NUM_THREADS = 320;
+constexpr int NUM_THREADS = 448;
+constexpr int DEQ_WARPS = 8;
 constexpr int TMEM_COLS = 512;          // two 256-column accumulators
 constexpr long long kTimeoutCycles = 4000000000LL;
 constexpr long long kDrainCycles = 200000000LL;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1280;
 
 struct Shared {
     uint64_t full_tma[STAGES];
@@ -52,7 +55,13 @@ struct Shared {
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
+    float ep_scale[BN];  // the current tile's row scales (epilogue)
+    int ep_ok[4];        // per epilogue warp: its accumulator wait succeeded
 };
+static_assert(sizeof(Shared) <= 1280, "shared control block");
+
+// Barrier among the 4 epilogue warps only.
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -242,7 +251,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&sh->full_tma[s], 1);
-            mbar_init(&sh->full_deq[s], 4);
+            mbar_init(&sh->full_deq[s], DEQ_WARPS);
             mbar_init(&sh->empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -263,6 +272,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
+    pdl_wait();  // barriers and TMEM were set up while the previous kernel finished
+    pdl_release();
     const int ntiles = total_tiles(a);
 
     if (warp == 0) {
@@ -348,9 +359,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
                 mbar_wait(&sh->drain, 0, sh, kDrainCycles);
             }
         }
-    } else if (warp < 6) {
-        // ---------------- dequantisers (128 threads) ----------------
-        const int dt = threadIdx.x - 64;  // 0..127
+    } else if (warp < 2 + DEQ_WARPS) {
+        // ---------------- dequantisers (one B row per thread) ----------------
+        const int r = threadIdx.x - 64;  // B row = output column of the tile
         int s = 0;
         uint32_t ph = 0;
         bool ok = true;
@@ -362,9 +373,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
                 if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
                 const uint8_t* raw = raw_tile(s);
                 uint8_t* bt = b_tile(s);
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int r = dt + h * 128;  // B row (output column of the tile)
+                {
                     const uint4 q0 = *reinterpret_cast<const uint4*>(raw + r * 32);
                     const uint4 q1 = *reinterpret_cast<const uint4*>(raw + r * 32 + 16);
                     const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
@@ -388,20 +397,36 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
         const int m = quarter * 32 + lane;  // token row of the tile
         uint32_t acc_ph[2] = {0, 0};
         int buf = 0;
+        const int et = threadIdx.x - 64 - 32 * DEQ_WARPS;  // 0..127
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
             const Tile t = decode_tile(a, tile);
+            const bool valid = m < t.n_valid;
+            // this tile's row scales and this thread's token, loaded while the
+            // tensor cores still work on the tile
+            const int irow = t.shared ? a.Is : a.I;
+            epi_bar();  // every epilogue warp is done with the previous tile's scales
+            if (GEMM == 1) {
+                const float* sc = t.shared ? a.s_s : a.s_r + (size_t)t.e * 2 * a.I;
+                sh->ep_scale[et] = __ldg(sc + t.col0 + et);
+                sh->ep_scale[BN / 2 + et] = __ldg(sc + irow + t.col0 + et);
+            } else {
+                const float* sc = t.shared ? a.s_s : a.s_r + (size_t)t.e * a.H;
+                sh->ep_scale[et] = __ldg(sc + t.col0 + et);
+                sh->ep_scale[BN / 2 + et] = __ldg(sc + t.col0 + BN / 2 + et);
+            }
+            const int tok = valid ? (t.shared ? t.slot0 + m : __ldg(a.tok_of_slot + t.slot0 + m)) : 0;
+            const int hx = __ldg(a.hexp + tok);
             int got = 0;
             if (lane == 0) got = mbar_wait(&sh->acc_full[buf], acc_ph[buf], sh);
-            if (!__shfl_sync(0xffffffffu, got, 0)) break;
+            if (lane == 0) sh->ep_ok[quarter] = got;
+            epi_bar();  // scales visible; every warp's wait outcome known
+            if (!(sh->ep_ok[0] && sh->ep_ok[1] && sh->ep_ok[2] && sh->ep_ok[3])) break;
             tc_fence_after();
             const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;
-            const bool valid = m < t.n_valid;
+            const float* scs = sh->ep_scale;
             if (GEMM == 1) {
-                const int irow = t.shared ? a.Is : a.I;
-                const float* sc = t.shared ? a.s_s : a.s_r + (size_t)t.e * 2 * a.I;
                 __half* hrow = (t.shared ? a.h_s : a.h_r) + (size_t)(t.slot0 + m) * irow + t.col0;
-                const int tok = valid ? (t.shared ? t.slot0 + m : __ldg(a.tok_of_slot + t.slot0 + m)) : 0;
-                const float hsc = ldexpf(1.0f, -__ldg(a.hexp + tok));
+                const float hsc = ldexpf(1.0f, -hx);
 #pragma unroll 1
                 for (int c0 = 0; c0 < BN / 2; c0 += 16) {
                     uint32_t g[16], u[16];
@@ -410,11 +435,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
                     uint32_t packed[8];
 #pragma unroll
                     for (int i = 0; i < 16; i += 2) {
-                        const int j = t.col0 + c0 + i;
-                        const float g0 = __uint_as_float(g[i]) * __ldg(sc + j);
-                        const float g1 = __uint_as_float(g[i + 1]) * __ldg(sc + j + 1);
-                        const float u0 = __uint_as_float(u[i]) * __ldg(sc + irow + j);
-                        const float u1 = __uint_as_float(u[i + 1]) * __ldg(sc + irow + j + 1);
+                        const int j = c0 + i;
+                        const float g0 = __uint_as_float(g[i]) * scs[j];
+                        const float g1 = __uint_as_float(g[i + 1]) * scs[j + 1];
+                        const float u0 = __uint_as_float(u[i]) * scs[BN / 2 + j];
+                        const float u1 = __uint_as_float(u[i + 1]) * scs[BN / 2 + j + 1];
                         __half2 hv = __floats2half2_rn(silu_mul(g0, u0) * hsc, silu_mul(g1, u1) * hsc);
                         packed[i >> 1] = *reinterpret_cast<uint32_t*>(&hv);
                     }
@@ -425,11 +450,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
                     }
                 }
             } else {
-                const float* sc = t.shared ? a.s_s : a.s_r + (size_t)t.e * a.H;
                 const size_t slot = t.shared ? (size_t)a.T * a.K + t.slot0 + m : (size_t)(t.slot0 + m);
                 float* yrow = a.y + slot * a.H + t.col0;
-                const int tok = valid ? (t.shared ? t.slot0 + m : __ldg(a.tok_of_slot + t.slot0 + m)) : 0;
-                const float inv = ldexpf(1.0f, __ldg(a.hexp + tok));
+                const float inv = ldexpf(1.0f, hx);
 #pragma unroll 1
                 for (int c0 = 0; c0 < BN; c0 += 16) {
                     uint32_t v[16];
@@ -438,11 +461,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
                         float4* dst = reinterpret_cast<float4*>(yrow + c0);
 #pragma unroll
                         for (int i = 0; i < 16; i += 4) {
-                            const int j = t.col0 + c0 + i;
-                            dst[i >> 2] = make_float4(__uint_as_float(v[i]) * (__ldg(sc + j) * inv),
-                                                      __uint_as_float(v[i + 1]) * (__ldg(sc + j + 1) * inv),
-                                                      __uint_as_float(v[i + 2]) * (__ldg(sc + j + 2) * inv),
-                                                      __uint_as_float(v[i + 3]) * (__ldg(sc + j + 3) * inv));
+                            const int j = c0 + i;
+                            dst[i >> 2] = make_float4(__uint_as_float(v[i]) * (scs[j] * inv),
+                                                      __uint_as_float(v[i + 1]) * (scs[j + 1] * inv),
+                                                      __uint_as_float(v[i + 2]) * (scs[j + 2] * inv),
+                                                      __uint_as_float(v[i + 3]) * (scs[j + 3] * inv));
                         }
                     }
                 }
@@ -558,10 +581,10 @@ cudaError_t launch_tc_gemm(const Params& p, int gemm, int grid, cudaStream_t str
     }
     if (!ok) return cudaErrorInvalidValue;
     if (gemm == 1)
-        tc::grouped_gemm_kernel<1><<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, stream>>>(mA_r, mA_s, mB_r, mB_s, a);
-    else
-        tc::grouped_gemm_kernel<2><<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, stream>>>(mA_r, mA_s, mB_r, mB_s, a);
-    return cudaGetLastError();
+        return launch_pdl(tc::grouped_gemm_kernel<1>, dim3(grid), dim3(tc::NUM_THREADS), tc::SMEM_BYTES, stream, mA_r,
+                          mA_s, mB_r, mB_s, a);
+    return launch_pdl(tc::grouped_gemm_kernel<2>, dim3(grid), dim3(tc::NUM_THREADS), tc::SMEM_BYTES, stream, mA_r,
+                      mA_s, mB_r, mB_s, a);
 }
 
 }  // namespace moe

@@ -14,7 +14,7 @@ constexpr int kDecodeMaxTokens = 64;
 // Tokens of one bucket handled by one expert-kernel task (2 mma n-tiles of 8).
 constexpr int kChunkTokens = 16;
 // Large-batch router: tokens per tile and the cap on router CTAs.
-constexpr int kRouterTileTokens = 16;
+constexpr int kRouterTileTokens = 32;
 constexpr int kRouterMaxBlocks = 296;
 // Small-batch router: tokens and experts per CTA (one warp per expert).
 constexpr int kDecodeRouterTok = 8;
@@ -39,10 +39,11 @@ enum : unsigned {
     ST_TIMEOUT = 16u,    // a bounded pipeline wait of the tensor-core kernel gave up
 };
 
-// First 256 bytes of the workspace.  Zeroed at the start of every call.
+// First 256 bytes of the workspace.  The first kernel of every call zeroes
+// status, claim13 and claim2; every other field is written before it is read
+// within the call, so the workspace needs no initialisation.
 struct Ctrl {
     unsigned status;
-    unsigned done;      // last-CTA-done ticket of the router
     int n_buckets;      // non-empty routed buckets + the shared bucket
     int tasks13;        // gate/up tasks over all buckets
     int tasks2;         // down tasks over all buckets
@@ -50,10 +51,44 @@ struct Ctrl {
     int tc_tiles2;      // tensor-core GEMM-2 tiles over the routed buckets
     int claim13;        // next gate/up task to claim (weight-streaming kernel)
     int claim2;         // next down task to claim
-    unsigned blk_done[kDecodeMaxTokens / 8];  // small-batch router: CTAs done per token block
-    unsigned sel_done;  // small-batch router: token blocks whose selection is done
-    int pad[46];
+    int pad[56];
 };
+
+// Programmatic dependent launch: every kernel of a call is launched so that
+// it may start while its predecessor in the stream finishes.  pdl_wait()
+// blocks until the predecessor grid has completed and its writes are
+// visible; nothing produced by an earlier kernel is touched before it.
+// pdl_release() lets the next kernel launch (it still waits for this grid's
+// completion before reading anything).  Both are no-ops when the kernel was
+// launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Warms L2 with bytes [0, n) of p, spread over the grid (128-byte lines).
+__device__ __forceinline__ void prefetch_l2_slice(const void* p, size_t n) {
+    const size_t lines = (n + 127) / 128;
+    const size_t per = (lines + gridDim.x - 1) / gridDim.x;
+    const size_t first = (size_t)blockIdx.x * per;
+    for (size_t l = first + threadIdx.x; l < first + per && l < lines; l += blockDim.x)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const char*>(p) + l * 128));
+}
+
+// Launches `kernel` with programmatic stream serialization allowed.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
 
 // Everything a kernel needs: shape, inputs, outputs and workspace views.
@@ -108,29 +143,30 @@ struct Params {
 // Kim et al., "Who Says Elephants Can't Run" (2022): the 4-bit code c, made
 // unsigned by flipping its sign bit (c + 8), is OR-ed into the low mantissa
 // bits of a 16-bit float equal to 2^m with ulp 1, which gives exactly
-// 2^m + 8 + c.  The weight-streaming kernels feed these *biased* values to the
-// tensor cores and remove the bias from the f32 result (bias * sum of the
-// activations), which saves the subtraction.  bf16: 2^7 = 0x4300 (bias 136);
-// fp16: 2^10 = 0x6400 (bias 1032).  Output pair j holds elements (2j, 2j+1)
-// of the word, low half first (natural order).
+// 2^m + 8 + c; subtracting 2^m + 8 leaves c exactly.  bf16: 2^7 = 0x4300;
+// fp16: 2^10 = 0x6400.  Output pair j holds elements (2j, 2j+1) of the 32-bit
+// word, low half first (natural order).
 // ---------------------------------------------------------------------------
-constexpr uint32_t kMagicBf16 = 0x43004300u;
-constexpr uint32_t kMagicF16 = 0x64006400u;
-constexpr float kBiasBf16 = 136.0f;
-constexpr float kBiasF16 = 1032.0f;
-constexpr uint32_t kOnesBf16 = 0x3F803F80u;
-constexpr uint32_t kOnesF16 = 0x3C003C00u;
-
-template <uint32_t kMagic>
-__device__ __forceinline__ void int4x8_biased(uint32_t w, uint32_t (&o)[4]) {
+template <bool kBf16>
+__device__ __forceinline__ void int4x8_to_16(uint32_t w, uint32_t (&o)[4]) {
     const uint32_t v = w ^ 0x88888888u;
     const uint32_t v4 = v >> 4;
-    // half 0 <- low nibble of byte j of v (element 2j); half 1 <- low nibble
-    // of byte j of v >> 4 (element 2j + 1)
-    o[0] = (__byte_perm(v, v4, 0x0400) & 0x000F000Fu) | kMagic;
-    o[1] = (__byte_perm(v, v4, 0x0501) & 0x000F000Fu) | kMagic;
-    o[2] = (__byte_perm(v, v4, 0x0602) & 0x000F000Fu) | kMagic;
-    o[3] = (__byte_perm(v, v4, 0x0703) & 0x000F000Fu) | kMagic;
+    constexpr uint32_t kMagic = kBf16 ? 0x43004300u : 0x64006400u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        // half 0 <- low nibble of byte j of v (element 2j); half 1 <- low
+        // nibble of byte j of v >> 4 (element 2j + 1)
+        uint32_t t = (__byte_perm(v, v4, j | ((4 + j) << 8)) & 0x000F000Fu) | kMagic;
+        if (kBf16) {
+            const __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&t),
+                                             __halves2bfloat162(__ushort_as_bfloat16(0x4308), __ushort_as_bfloat16(0x4308)));
+            o[j] = *reinterpret_cast<const uint32_t*>(&r);
+        } else {
+            const __half2 r = __hsub2(*reinterpret_cast<__half2*>(&t),
+                                      __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408)));
+            o[j] = *reinterpret_cast<const uint32_t*>(&r);
+        }
+    }
 }
 
 // Streamed weights: read once, keep out of L1.

@@ -35,23 +35,40 @@ __device__ __forceinline__ float warp_sum_tree(float v) {
     return v;
 }
 
-// Exponent k_t of the token's h storage scale 2^-k_t (one warp):
-// k_t = 8 + floor(log2(mean_h x[t,h]^2)), the mean square summed in the same
-// lane order as the router logits.
-__device__ __forceinline__ void token_hexp(const Params& p, int t, int lane) {
-    const __nv_bfloat16* xr = p.x + (size_t)t * p.H;
-    float acc = 0.f;
-    for (int i = 0; i < p.H / 128; ++i) {
-        const uint2 xv = __ldg(reinterpret_cast<const uint2*>(xr + i * 128 + lane * 4));
-        const float a = bf16lo(xv.x), b = bf16hi(xv.x), c = bf16lo(xv.y), d = bf16hi(xv.y);
-        acc = fmaf(a, a, acc);
-        acc = fmaf(b, b, acc);
-        acc = fmaf(c, c, acc);
-        acc = fmaf(d, d, acc);
-    }
-    const float ms = warp_sum_tree(acc) / (float)p.H;
+__device__ __forceinline__ float sq_step(float acc, uint2 xv) {
+    const float a = bf16lo(xv.x), b = bf16hi(xv.x), c = bf16lo(xv.y), d = bf16hi(xv.y);
+    acc = fmaf(a, a, acc);
+    acc = fmaf(b, b, acc);
+    acc = fmaf(c, c, acc);
+    acc = fmaf(d, d, acc);
+    return acc;
+}
+
+// k_t = 8 + floor(log2(mean_h x[t,h]^2)), clamped: the exponent of the
+// token's h storage scale 2^-k_t.  `lane_sq` is the lane's share of the sum of
+// squares in the router's lane order (see dot_step).
+__device__ __forceinline__ void store_hexp(const Params& p, int t, float lane_sq, int lane) {
+    const float ms = warp_sum_tree(lane_sq) / (float)p.H;
     const int e = (ms > 0.f && isfinite(ms)) ? ilogbf(ms) : 0;
     if (lane == 0) p.hexp[t] = min(max(kHExpBase + e, kHExpMin), kHExpMax);
+}
+
+// k_t of one token (one warp), loads issued four 128-blocks at a time.
+__device__ __forceinline__ void token_hexp(const Params& p, int t, int lane) {
+    const __nv_bfloat16* xr = p.x + (size_t)t * p.H;
+    const int nblk = p.H / 128;
+    float acc = 0.f;
+    for (int i0 = 0; i0 < nblk; i0 += 4) {
+        uint2 xv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            xv[u] = i0 + u < nblk ? __ldg(reinterpret_cast<const uint2*>(xr + (i0 + u) * 128 + lane * 4))
+                                  : make_uint2(0u, 0u);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (i0 + u < nblk) acc = sq_step(acc, xv[u]);
+    }
+    store_hexp(p, t, acc, lane);
 }
 
 // Top-K of one token (one warp).  Lane l holds experts l, l+32, ...  The key
@@ -221,22 +238,41 @@ __device__ void finalize_buckets(const Params& p, const int* s_cnt, int* s_off) 
     __syncthreads();
 }
 
+// Zeroes the per-call control words (first kernel of a call, one thread,
+// after pdl_wait: every kernel of the previous call has completed).
+__device__ __forceinline__ void reset_ctrl(const Params& p) {
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+        p.ctrl->status = 0;
+        p.ctrl->claim13 = 0;
+        p.ctrl->claim2 = 0;
+    }
+}
+
 // ---------------------------------------------------------------------------
-// Small batch (T <= kDecodeMaxTokens): grid (ceil(T/8), ceil(E/8)); warp w of
-// CTA (bx, by) computes the logits of expert 8*by + w for tokens 8*bx ...
-// 8*bx + 7.  The last CTA of each token block selects that block's tokens
-// (one warp per token); the last of those counts, scans and scatters.
+// Small batch (T <= kDecodeMaxTokens), two kernels.
+// router_logits_kernel: grid (ceil(T/8), ceil(E/8)); warp w of CTA (bx, by)
+// computes the logits of expert 8*by + w for tokens 8*bx ... 8*bx + 7 (warp 0
+// of the first expert column also the tokens' h-scale exponents).
+// router_select_kernel: one CTA selects every token (one warp per token),
+// counts, scans and scatters.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) router_small_kernel(Params p) {
+__global__ void __launch_bounds__(256) router_logits_kernel(Params p) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int t0 = blockIdx.x * kDecodeRouterTok;
     const int e = blockIdx.y * kDecodeRouterExp + warp;
     const int nt = min(kDecodeRouterTok, p.T - t0);
-    if (blockIdx.y == 0 && warp < nt) token_hexp(p, t0 + warp, lane);
+    if (e < p.E) {  // the router weights do not depend on the previous kernel
+        const char* wrow = reinterpret_cast<const char*>(p.rw + (size_t)e * p.H);
+        for (int l = lane; l < p.H * 4 / 128; l += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(wrow + l * 128));
+    }
+    pdl_wait();
+    reset_ctrl(p);
+    pdl_release();
+    const bool do_sq = blockIdx.y == 0 && warp == 0;
     if (e < p.E) {
-        float acc[kDecodeRouterTok];
+        float acc[kDecodeRouterTok], sq[kDecodeRouterTok];
 #pragma unroll
-        for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = 0.f;
+        for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = sq[tt] = 0.f;
         const float4* W = reinterpret_cast<const float4*>(p.rw + (size_t)e * p.H);
         const int nblk = p.H / 128;  // processed 4 blocks per batch of loads
         for (int i0 = 0; i0 < nblk; i0 += 4) {
@@ -256,7 +292,10 @@ __global__ void __launch_bounds__(256) router_small_kernel(Params p) {
             for (int u = 0; u < 4; ++u) {
                 if (i0 + u < nblk) {
 #pragma unroll
-                    for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = dot_step(acc[tt], xv[u][tt], wv[u]);
+                    for (int tt = 0; tt < kDecodeRouterTok; ++tt) {
+                        acc[tt] = dot_step(acc[tt], xv[u][tt], wv[u]);
+                        if (do_sq) sq[tt] = sq_step(sq[tt], xv[u][tt]);
+                    }
                 }
             }
         }
@@ -264,46 +303,34 @@ __global__ void __launch_bounds__(256) router_small_kernel(Params p) {
         for (int tt = 0; tt < kDecodeRouterTok; ++tt) {
             const float v = warp_sum_tree(acc[tt]);
             if (lane == 0 && tt < nt) p.logits[(size_t)(t0 + tt) * p.E + e] = v;
+            if (do_sq && tt < nt) store_hexp(p, t0 + tt, sq[tt], lane);
         }
     }
+}
 
-    // ---- last CTA of this token block: selection of its tokens
-    __shared__ int s_last;
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) s_last = (atomicAdd(&p.ctrl->blk_done[blockIdx.x], 1u) == gridDim.y - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    __shared__ float s_lg[kDecodeRouterTok * kMaxE];
-    for (int i = threadIdx.x; i < nt * p.E; i += blockDim.x) s_lg[i] = __ldcg(p.logits + (size_t)t0 * p.E + i);
-    __syncthreads();
-    if (warp < nt) {
-        const int sel = select_token<false>(p, t0 + warp, s_lg + warp * p.E, lane);
-        if (lane < p.K && (sel < 0 || sel >= p.E)) atomicOr(&p.ctrl->status, ST_BAD_EXPERT);
-    }
-
-    // ---- last token block: counts, scan, bucket and task lists, slots
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) s_last = (atomicAdd(&p.ctrl->sel_done, 1u) == gridDim.x - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
+__global__ void __launch_bounds__(1024) router_select_kernel(Params p) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     __shared__ int s_idx[kDecodeMaxTokens * kMaxK];
     __shared__ int s_cnt[kMaxE];
     __shared__ int s_off[kMaxE];
-    const int TK = p.T * p.K;
+    pdl_wait();
+    pdl_release();
     for (int i = threadIdx.x; i < p.E; i += blockDim.x) s_cnt[i] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < TK; i += blockDim.x) {
-        int ex = __ldcg(p.idx + i);
-        if (ex < 0 || ex >= p.E) ex = 0;  // reported above; keep every index in range
-        s_idx[i] = ex;
-        atomicAdd(&s_cnt[ex], 1);
+    for (int t = warp; t < p.T; t += blockDim.x / 32) {
+        int sel = select_token<true>(p, t, p.logits + (size_t)t * p.E, lane);
+        if (lane < p.K) {
+            if (sel < 0 || sel >= p.E) {
+                atomicOr(&p.ctrl->status, ST_BAD_EXPERT);
+                sel = 0;
+            }
+            s_idx[t * p.K + lane] = sel;
+            atomicAdd(&s_cnt[sel], 1);
+        }
     }
     __syncthreads();
     finalize_buckets(p, s_cnt, s_off);
+    const int TK = p.T * p.K;
     for (int i = threadIdx.x; i < TK; i += blockDim.x) {
         const int ex = s_idx[i];
         int rank = 0;
@@ -320,96 +347,209 @@ __global__ void __launch_bounds__(256) router_small_kernel(Params p) {
 }
 
 // ---------------------------------------------------------------------------
-// Large batch: router_blocks CTAs walk tiles of 16 tokens (tile = block,
-// block + grid, ...).  Each tile's logits stay in shared memory; one warp per
-// token selects; every CTA records its per-expert slot counts in hist.  The
-// last CTA sums them, scans and builds the bucket and task lists.
+// Large batch, three kernels.
+// router_large_kernel: router_blocks CTAs walk tiles of 16 tokens (tile =
+// block, block + grid, ...); each tile's logits stay in shared memory, one
+// warp per token selects, and every CTA records its per-expert slot counts.
+// router_finalize_kernel: one CTA sums the counts, scans and builds the
+// bucket and task lists.  scatter_large_kernel: slots (and, for the
+// tensor-core path, the gathered activation rows).
 // ---------------------------------------------------------------------------
+// Tensor-core router logits for a tile of kRouterTileTokens tokens and every
+// expert.  x is exactly bf16; each f32 router weight w is split exactly into
+// three bf16 terms w = hi + mid + lo (hi = bf16(w), mid = bf16(w - hi),
+// lo = bf16(w - hi - mid); together they hold w's 24-bit mantissa), and
+// x.w = x.lo + x.mid + x.hi is accumulated in f32 by mma.sync m16n8k16
+// (A = tokens, B = experts).  Every 16-wide k step is accumulated from zero
+// by the tensor cores (16 products per instruction) and added to the running
+// f32 sum with ordinary IEEE adds, so the logits carry f32 rounding only.  The activations are staged in shared memory
+// with cp.async (chunks of kRouterKC along the hidden dimension, double-
+// buffered) and read with ldmatrix.
+constexpr int kRouterKC = 128;                // hidden elements per staged chunk (H % 128 == 0)
+constexpr int kRouterXS = kRouterKC + 8;      // padded row (bf16 elements)
+constexpr int kRouterMT = kRouterTileTokens / 16;
+
+__device__ __forceinline__ void split3(float w, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(m);
+    hi = __bfloat16_as_ushort(h);
+    mid = __bfloat16_as_ushort(m);
+    lo = __bfloat16_as_ushort(__float2bfloat16_rn(r2));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* smem_row) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_row))));
+}
+
 __global__ void __launch_bounds__(256) router_large_kernel(Params p) {
-    __shared__ float s_logit[kRouterTileTokens][kMaxE];
+    // the staged activations and, after the k loop, the tile's logits share one buffer
+    constexpr int kXBytes = 2 * kRouterTileTokens * kRouterXS * 2;
+    constexpr int kLBytes = kRouterTileTokens * kMaxE * 4;
+    __shared__ __align__(16) uint8_t s_buf[kXBytes > kLBytes ? kXBytes : kLBytes];
     __shared__ int s_cnt[kMaxE];
-    __shared__ int s_off[kMaxE];
+    auto s_x = reinterpret_cast<uint16_t (*)[kRouterTileTokens][kRouterXS]>(s_buf);
+    auto s_logit = reinterpret_cast<float (*)[kMaxE]>(s_buf);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, q = lane & 3;
     const int E = p.E, H = p.H;
+    const int n_ntiles = (E + 7) / 8;
+    pdl_wait();
+    reset_ctrl(p);
+    pdl_release();
     for (int i = threadIdx.x; i < E; i += blockDim.x) s_cnt[i] = 0;
     __syncthreads();
-    const int ntiles = (p.T + kRouterTileTokens - 1) / kRouterTileTokens;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int ntiles_tok = (p.T + kRouterTileTokens - 1) / kRouterTileTokens;
+    const int nchunks = H / kRouterKC;
+    for (int tile = blockIdx.x; tile < ntiles_tok; tile += gridDim.x) {
         const int t0 = tile * kRouterTileTokens;
         const int nt = min(kRouterTileTokens, p.T - t0);
         for (int tt = warp; tt < nt; tt += 8) token_hexp(p, t0 + tt, lane);
-        for (int e0 = warp; e0 < E; e0 += 16) {
-            const int e1 = e0 + 8;
-            const bool has1 = e1 < E;
-            float a0[kRouterTileTokens], a1[kRouterTileTokens];
+
+        auto stage_chunk = [&](int c, int buf) {
+            for (int i = threadIdx.x; i < kRouterTileTokens * (kRouterKC / 8); i += blockDim.x) {
+                const int r = i / (kRouterKC / 8), part = i % (kRouterKC / 8);
+                uint16_t* dst = &s_x[buf][r][part * 8];
+                if (r < nt) {
+                    const void* src = p.x + (size_t)(t0 + r) * H + c * kRouterKC + part * 8;
+                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                                 "l"(src)
+                                 : "memory");
+                } else {
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        };
+
+        // this warp's expert n-tiles: warp, warp + 8, ... (at most kMaxE / 64)
+        float acc[kMaxE / 64][kRouterMT][4];
 #pragma unroll
-            for (int tt = 0; tt < kRouterTileTokens; ++tt) { a0[tt] = 0.f; a1[tt] = 0.f; }
-            const float4* W0 = reinterpret_cast<const float4*>(p.rw + (size_t)e0 * H);
-            const float4* W1 = reinterpret_cast<const float4*>(p.rw + (size_t)(has1 ? e1 : e0) * H);
-            for (int i = 0; i < H / 128; ++i) {
-                const float4 w0 = __ldg(W0 + i * 32 + lane);
-                const float4 w1 = __ldg(W1 + i * 32 + lane);
+        for (int j = 0; j < kMaxE / 64; ++j)
 #pragma unroll
-                for (int tt = 0; tt < kRouterTileTokens; ++tt) {
-                    if (tt < nt) {
-                        const uint2 xv = __ldg(reinterpret_cast<const uint2*>(
-                            p.x + (size_t)(t0 + tt) * H + i * 128 + lane * 4));
-                        a0[tt] = dot_step(a0[tt], xv, w0);
-                        a1[tt] = dot_step(a1[tt], xv, w1);
+            for (int m = 0; m < kRouterMT; ++m) acc[j][m][0] = acc[j][m][1] = acc[j][m][2] = acc[j][m][3] = 0.f;
+
+        __syncthreads();  // s_x is free (previous tile done)
+        stage_chunk(0, 0);
+        for (int c = 0; c < nchunks; ++c) {
+            if (c + 1 < nchunks) stage_chunk(c + 1, (c + 1) & 1);
+            else asm volatile("cp.async.commit_group;" ::: "memory");
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+            __syncthreads();
+            const uint16_t (*xs)[kRouterXS] = s_x[c & 1];
+#pragma unroll
+            for (int j = 0; j < kMaxE / 64; ++j) {
+                const int ntile = warp + 8 * j;
+                if (ntile < n_ntiles) {
+                    const int e = ntile * 8 + g;
+                    const float* wrow = p.rw + (size_t)min(e, E - 1) * H + c * kRouterKC;
+                    for (int ks = 0; ks < kRouterKC / 16; ks += 2) {
+                        // B fragments of two k steps: w[k + 2q, +1] and w[k + 2q + 8, +9]
+                        float2 wv[2][2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            wv[u][0] = __ldg(reinterpret_cast<const float2*>(wrow + (ks + u) * 16 + 2 * q));
+                            wv[u][1] = __ldg(reinterpret_cast<const float2*>(wrow + (ks + u) * 16 + 2 * q + 8));
+                        }
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            uint32_t bh[2], bm[2], bl[2];
+#pragma unroll
+                            for (int v = 0; v < 2; ++v) {
+                                const float w0 = e < E ? wv[u][v].x : 0.f, w1 = e < E ? wv[u][v].y : 0.f;
+                                uint16_t h0, m0, l0, h1, m1, l1;
+                                split3(w0, h0, m0, l0);
+                                split3(w1, h1, m1, l1);
+                                bh[v] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                                bm[v] = (uint32_t)m0 | ((uint32_t)m1 << 16);
+                                bl[v] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+                            }
+#pragma unroll
+                            for (int m = 0; m < kRouterMT; ++m) {
+                                uint32_t a[4];
+                                ldmatrix_x4(a, &xs[m * 16 + (lane & 15)][(ks + u) * 16 + (lane >> 4) * 8]);
+                                float t[4] = {0.f, 0.f, 0.f, 0.f};
+                                mma_bf16(t, a, bl[0], bl[1]);
+                                mma_bf16(t, a, bm[0], bm[1]);
+                                mma_bf16(t, a, bh[0], bh[1]);
+#pragma unroll
+                                for (int v = 0; v < 4; ++v) acc[j][m][v] += t[v];
+                            }
+                        }
                     }
                 }
             }
+            __syncthreads();  // chunk c's readers are done before it is overwritten
+        }
 #pragma unroll
-            for (int tt = 0; tt < kRouterTileTokens; ++tt) {
-                const float v0 = warp_sum_tree(a0[tt]);
-                const float v1 = warp_sum_tree(a1[tt]);
-                if (lane == 0 && tt < nt) {
-                    s_logit[tt][e0] = v0;
-                    if (has1) s_logit[tt][e1] = v1;
+        for (int j = 0; j < kMaxE / 64; ++j) {
+            const int ntile = warp + 8 * j;
+            if (ntile < n_ntiles) {
+                const int e = ntile * 8 + 2 * q;
+#pragma unroll
+                for (int m = 0; m < kRouterMT; ++m) {
+                    const int r = m * 16 + g;
+                    if (e < E) { s_logit[r][e] = acc[j][m][0]; s_logit[r + 8][e] = acc[j][m][2]; }
+                    if (e + 1 < E) { s_logit[r][e + 1] = acc[j][m][1]; s_logit[r + 8][e + 1] = acc[j][m][3]; }
                 }
             }
         }
         __syncthreads();
         for (int tt = warp; tt < nt; tt += 8) {
             const int sel = select_token<false>(p, t0 + tt, s_logit[tt], lane);
-            if (lane < p.K) {
-                if (sel >= 0 && sel < E) atomicAdd(&s_cnt[sel], 1);
-                else atomicOr(&p.ctrl->status, ST_BAD_EXPERT);
-            }
+            // an index outside [0, E) cannot occur; it is counted nowhere and
+            // reported by the scatter kernel's range check
+            if (lane < p.K && sel >= 0 && sel < E) atomicAdd(&s_cnt[sel], 1);
         }
-        __syncthreads();
     }
+    __syncthreads();
     for (int i = threadIdx.x; i < E; i += blockDim.x) p.hist[(size_t)blockIdx.x * E + i] = s_cnt[i];
+}
 
-    __shared__ int s_last;
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) s_last = (atomicAdd(&p.ctrl->done, 1u) == gridDim.x - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int c = 0;
-        for (int b = 0; b < (int)gridDim.x; ++b) c += __ldcg(p.hist + (size_t)b * E + e);
-        s_cnt[e] = c;
+__global__ void __launch_bounds__(1024) router_finalize_kernel(Params p) {
+    __shared__ int s_cnt[kMaxE];
+    __shared__ int s_off[kMaxE];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+    const int E = p.E, nblk = p.router_blocks;
+    pdl_wait();
+    pdl_release();
+    // hist[b][e] -> exclusive prefix over b (per expert), one warp per expert
+    for (int e = warp; e < E; e += nwarp) {
+        int run = 0;
+        for (int b0 = 0; b0 < nblk; b0 += 32) {
+            const int b = b0 + lane;
+            const int v = b < nblk ? p.hist[(size_t)b * E + e] : 0;
+            int inc = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += u;
+            }
+            if (b < nblk) p.hist[(size_t)b * E + e] = run + inc - v;
+            run += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) s_cnt[e] = run;
     }
     __syncthreads();
     finalize_buckets(p, s_cnt, s_off);
-    if (threadIdx.x == 0) p.ctrl->done = 0;
+    // base of every (router CTA, expert) = bucket start + earlier CTAs' slots
+    for (int i = threadIdx.x; i < nblk * E; i += blockDim.x) p.hist[i] += s_off[i % E];
 }
 
-// Large batch, second pass: CTA c walks the same tiles as router CTA c and
-// assigns slots in (tile, token, k) order, after the slots of CTAs 0..c-1.
+// CTA c walks the same tiles as router CTA c and assigns slots in (tile,
+// token, k) order, after the slots of CTAs 0..c-1.
 __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
     __shared__ int s_base[kMaxE];
     __shared__ int s_idx[kRouterTileTokens * kMaxK];
     const int E = p.E, K = p.K;
     const int TK = p.T * K;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int b = p.offsets[e];
-        for (int c = 0; c < (int)blockIdx.x; ++c) b += p.hist[(size_t)c * E + e];
-        s_base[e] = b;
-    }
+    pdl_wait();
+    pdl_release();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_base[e] = p.hist[(size_t)blockIdx.x * E + e];
     __syncthreads();
     const int ntiles = (p.T + kRouterTileTokens - 1) / kRouterTileTokens;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -461,16 +601,17 @@ __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
 }
 
 cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream) {
+    cudaError_t err;
     if (small_path) {
         dim3 grid((p.T + kDecodeRouterTok - 1) / kDecodeRouterTok, (p.E + kDecodeRouterExp - 1) / kDecodeRouterExp);
-        router_small_kernel<<<grid, 256, 0, stream>>>(p);
-        return cudaGetLastError();
+        err = launch_pdl(router_logits_kernel, grid, dim3(256), 0, stream, p);
+        if (err == cudaSuccess) err = launch_pdl(router_select_kernel, dim3(1), dim3(1024), 0, stream, p);
+        return err;
     }
-    router_large_kernel<<<p.router_blocks, 256, 0, stream>>>(p);
-    cudaError_t err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
-    scatter_large_kernel<<<p.router_blocks, 256, 0, stream>>>(p);
-    return cudaGetLastError();
+    err = launch_pdl(router_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
+    if (err == cudaSuccess) err = launch_pdl(router_finalize_kernel, dim3(1), dim3(1024), 0, stream, p);
+    if (err == cudaSuccess) err = launch_pdl(scatter_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
+    return err;
 }
 
 }  // namespace moe
