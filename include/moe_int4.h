@@ -144,6 +144,41 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
                       const moe_shared_weights_t* shared_w, void* out, int32_t T,
                       const moe_cfg_t* cfg, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * For callers that cannot allocate device memory.
+ *
+ * moe_layer_forward needs a caller-provided workspace.  Some callers cannot
+ * call cudaMalloc or any other allocator: a plug-in running inside a host
+ * framework that owns all device memory through its own pool, for example,
+ * or code that must not allocate while one of its streams is being captured.
+ * moe_layer_forward_static_ws serves them.  The paper has no counterpart of
+ * this entry point; it exists for integration only.
+ *
+ * It takes the same arguments as moe_layer_forward and computes the same
+ * result with the same kernels, but ignores cfg->workspace and
+ * cfg->workspace_bytes.  Its scratch memory is one array of
+ * MOE_STATIC_WORKSPACE_BYTES (32 MiB) that the library itself holds in device
+ * memory, on every GPU that loads it, until the process exits.
+ *  - A call whose moe_layer_workspace_bytes(cfg, T) exceeds that size returns
+ *    MOE_ERR_WORKSPACE and launches nothing.
+ *  - It allocates nothing and calls no allocating routine.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current.  Make that first call
+ *    before any stream capture begins.
+ *  - Every call on a device shares the one array, and the array keeps the
+ *    last call's contents.  Calls that may run at the same time on the GPU
+ *    (on different streams, with nothing ordering them) race on it and must
+ *    not be issued; calls ordered on one stream are fine.  No part of the
+ *    array has to start at zero: each call sets what it uses.
+ * ------------------------------------------------------------------------- */
+#define MOE_STATIC_WORKSPACE_BYTES ((size_t)32 << 20)
+
+int moe_layer_forward_static_ws(const void* x, const float* router_w, const float* router_bias,
+                                const uint8_t* packed_w13, const float* scales13,
+                                const uint8_t* packed_w2, const float* scales2,
+                                const moe_shared_weights_t* shared_w, void* out, int32_t T,
+                                const moe_cfg_t* cfg, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* moe_status_str(int status);
 

@@ -43,7 +43,11 @@ STAGE_NAMES = ("route", "gate_up", "down", "combine")
 
 # Every function declared in include/moe_int4.h.
 EXPORTED_SYMBOLS = ("moe_layer_workspace_bytes", "moe_layer_forward", "moe_status_str",
-                    "moe_abi_version", "moe_decode_max_tokens")
+                    "moe_abi_version", "moe_decode_max_tokens", "moe_layer_forward_static_ws")
+
+# Scratch capacity of moe_layer_forward_static_ws (the entry point for callers
+# that cannot allocate device memory).
+MOE_STATIC_WORKSPACE_BYTES = 32 << 20
 
 
 class MoeError(RuntimeError):
@@ -68,7 +72,7 @@ class moe_shared_weights_t(ctypes.Structure):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is not built; run `python -m int4_expert_ffn_sigmoid_b200._build`")
+        raise ImportError(f"{LIB_PATH} is not built; run `python int4_expert_ffn_sigmoid_b200/_build.py`")
     L = ctypes.CDLL(LIB_PATH)
     vp = ctypes.c_void_p
     L.moe_layer_workspace_bytes.argtypes = [ctypes.POINTER(moe_cfg_t), ctypes.c_int32]
@@ -76,6 +80,8 @@ def _load() -> ctypes.CDLL:
     L.moe_layer_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(moe_shared_weights_t),
                                     vp, ctypes.c_int32, ctypes.POINTER(moe_cfg_t), vp]
     L.moe_layer_forward.restype = ctypes.c_int
+    L.moe_layer_forward_static_ws.argtypes = L.moe_layer_forward.argtypes
+    L.moe_layer_forward_static_ws.restype = ctypes.c_int
     L.moe_status_str.argtypes = [ctypes.c_int]
     L.moe_status_str.restype = ctypes.c_char_p
     L.moe_abi_version.argtypes = []

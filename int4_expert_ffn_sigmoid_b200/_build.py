@@ -1,7 +1,8 @@
 """Build the CUDA library ``libmoe_int4.so`` in-tree for sm_100a with nvcc.
 
-Usage: ``python -m int4_expert_ffn_sigmoid_b200._build [--force] [--verbose]``
-(``--verbose`` prints ptxas register / spill / shared-memory reports).
+Usage: ``python int4_expert_ffn_sigmoid_b200/_build.py [--force] [--verbose]``
+(``--verbose`` prints ptxas register / spill / shared-memory reports).  Run it
+by path: importing the package loads the library this script builds.
 """
 from __future__ import annotations
 
@@ -37,9 +38,21 @@ def _deps():
     return files
 
 
+STAMP = os.path.join(BUILD, "sources.txt")
+
+
+def _source_list() -> str:
+    return "\n".join(os.path.basename(f) for f in sources())
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    """The library exists, is newer than every source and header, and was
+    built from the current set of source files."""
+    if not os.path.exists(LIB) or not os.path.exists(STAMP):
         return False
+    with open(STAMP) as f:
+        if f.read() != _source_list():
+            return False
     t = os.path.getmtime(LIB)
     return all(os.path.getmtime(f) <= t for f in _deps())
 
@@ -73,6 +86,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(_source_list())
     return LIB
 
 

@@ -14,8 +14,8 @@ HEADER = os.path.join(ROOT, "include", "moe_int4.h")
 
 @pytest.fixture(scope="module")
 def moe():
-    from int4_expert_ffn_sigmoid_b200 import _build
-    _build.build()
+    import __graft_entry__
+    __graft_entry__._load_build_module().build()
     import int4_expert_ffn_sigmoid_b200 as m
     return m
 
