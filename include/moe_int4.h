@@ -116,7 +116,10 @@ typedef struct moe_cfg {
 } moe_cfg_t;
 
 /* Bytes of workspace moe_layer_forward needs for T tokens under `cfg`
- * (workspace, workspace_bytes and the output pointers are ignored).
+ * (workspace, workspace_bytes and the output pointers are ignored; flags are
+ * not: the size depends on the kernel sequence that T and the flags select,
+ * so a workspace for up to N tokens must hold the largest of the sizes for
+ * T = N and T = min(N, moe_decode_max_tokens())).
  * Returns 0 if cfg is NULL or the shape is invalid or unsupported. */
 size_t moe_layer_workspace_bytes(const moe_cfg_t* cfg, int32_t T);
 
@@ -133,9 +136,21 @@ size_t moe_layer_workspace_bytes(const moe_cfg_t* cfg, int32_t T);
  *                or f32 [T][H] under MOE_OUT_F32
  *   T          : tokens, 0..2^20 (T = 0 returns MOE_OK and launches nothing)
  *   cfg, stream: see above.
- * The routing weights and every expert contribution are accumulated in f32;
- * the SwiGLU intermediate h is kept in fp16 as h * 2^-8 (so |h| up to 1.6e7),
- * never in bf16.
+ * Arithmetic.  Router logits, scores and routing weights are f32.  Two
+ * kernel sequences compute the experts:
+ *  - small batches (T <= moe_decode_max_tokens(), unless MOE_FORCE_PREFILL),
+ *    and larger ones when H is not a multiple of 256 or under
+ *    MOE_FORCE_DECODE: weight-streaming kernels.  An activation row (x of a
+ *    token, or a 512-wide slice of its SwiGLU intermediate h) is written as
+ *    s * (q0 + q1/256) with int8 q0, q1 and a power of two s from the row's
+ *    largest magnitude, so each element is represented to within 2^-15 of
+ *    that magnitude (rows whose largest magnitude is below 2^-113 become
+ *    zero; a row holding NaN or infinity gives NaN outputs).  Weight codes
+ *    times activation parts accumulate exactly in int32; h is kept in f32.
+ *  - otherwise: tensor-core kernels with bf16 x, f32 accumulation, and h
+ *    kept in fp16 as h * 2^-k_t with a per-token power of two 2^-k_t that
+ *    keeps it in fp16's normal range.
+ * Expert outputs and their weighted sum are f32 until the output rounding.
  * Returns MOE_OK or an MOE_ERR_* code; on an error nothing is launched
  * (except MOE_ERR_CUDA / MOE_ERR_DEVICE_CHECK, raised after launching). */
 int moe_layer_forward(const void* x, const float* router_w, const float* router_bias,

@@ -136,7 +136,10 @@ def workspace_bytes(shape, T: int, flags: int = 0) -> int:
 
 
 def new_workspace(shape, T: int, device, flags: int = 0) -> torch.Tensor:
-    n = workspace_bytes(shape, T, flags)
+    """A workspace for any call of up to T tokens under `flags` (the sizes of
+    the two kernel sequences differ, so both sides of the small-batch limit
+    are asked)."""
+    n = max(workspace_bytes(shape, T, flags), workspace_bytes(shape, min(T, decode_max_tokens()), flags))
     if n == 0:
         raise MoeError(MOE_ERR_UNSUPPORTED, "moe_layer_workspace_bytes")
     return torch.empty(n, dtype=torch.uint8, device=device)

@@ -18,9 +18,24 @@ constexpr int32_t kMaxTokens = 1 << 20;
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// Kernel sequence of a call: the small-batch router + weight-streaming
+// experts; the large router + tensor-core grouped GEMMs; or the large router
+// + weight-streaming experts (H not a multiple of 256, or MOE_FORCE_DECODE).
+enum class Path { kSmall, kTensorCore, kLargeStreaming };
+
+Path choose_path(const moe_cfg_t& c, int32_t T) {
+    if (T <= kDecodeMaxTokens && !(c.flags & MOE_FORCE_PREFILL)) return Path::kSmall;
+    // GEMM-2 of the tensor-core path tiles 256 output columns
+    if (!(c.flags & MOE_FORCE_DECODE) && c.H % 256 == 0) return Path::kTensorCore;
+    return Path::kLargeStreaming;
+}
+
 struct WsLayout {
-    size_t ctrl, idx, wts, logits, counts, offsets, bucket_e, bucket_n, bucket_off, ts13, ts2, tcs1, tcs2;
-    size_t tok_of_slot, slot_of, hist, h_r, h_s, hexp, y, x_perm, total;
+    size_t ctrl, idx, wts, counts, offsets, bucket_e, bucket_n, bucket_off, ts13, ts2, tcs1, tcs2;
+    size_t tok_of_slot, slot_of, hist, rank, hexp, y;
+    size_t h_r, h_s, x_perm;                            // tensor-core path
+    size_t xq, xs, h32_r, h32_s, hmax_r, hmax_s;        // weight-streaming paths
+    size_t total;
 };
 
 WsLayout ws_layout(const moe_cfg_t& c, int32_t T) {
@@ -31,11 +46,11 @@ WsLayout ws_layout(const moe_cfg_t& c, int32_t T) {
         o = align256(o + bytes);
         return r;
     };
-    const size_t TK = (size_t)T * c.K, E = (size_t)c.E;
+    const Path path = choose_path(c, T);
+    const size_t TK = (size_t)T * c.K, E = (size_t)c.E, H = (size_t)c.H;
     L.ctrl = take(sizeof(Ctrl));
     L.idx = take(TK * 4);
     L.wts = take(TK * 4);
-    L.logits = take((size_t)(T < kDecodeMaxTokens ? T : kDecodeMaxTokens) * E * 4);
     L.counts = take(E * 4);
     L.offsets = take(E * 4);
     L.bucket_e = take((E + 1) * 4);
@@ -48,11 +63,23 @@ WsLayout ws_layout(const moe_cfg_t& c, int32_t T) {
     L.tok_of_slot = take(TK * 4);
     L.slot_of = take(TK * 4);
     L.hist = take((size_t)kRouterMaxBlocks * E * 4);
-    L.h_r = take(TK * (size_t)c.I * 2);
-    L.h_s = take((size_t)T * (size_t)c.Is * 2);
+    L.rank = take(TK * 4);
     L.hexp = take((size_t)T * 4);
-    L.y = take((TK + (c.Is > 0 ? (size_t)T : 0)) * (size_t)c.H * 4);
-    L.x_perm = take(TK * (size_t)c.H * 2);
+    const size_t shared_rows = c.Is > 0 ? (size_t)T : 0;
+    if (path == Path::kTensorCore) {
+        L.h_r = take(TK * (size_t)c.I * 2);
+        L.h_s = take((size_t)T * (size_t)c.Is * 2);
+        L.x_perm = take(TK * H * 2);
+        L.y = take((TK + shared_rows) * H * 4);
+    } else {
+        L.xq = take((size_t)T * 2 * H);
+        L.xs = take((size_t)T * 4);
+        L.h32_r = take(TK * (size_t)c.I * 4);
+        L.h32_s = take((size_t)T * (size_t)c.Is * 4);
+        L.hmax_r = take(TK * (size_t)(c.I / 64) * 4);
+        L.hmax_s = take((size_t)T * (size_t)(c.Is / 64) * 4);
+        L.y = take((TK * slices_of(c.I) + shared_rows * slices_of(c.Is)) * H * 4);
+    }
     L.total = o;
     return L;
 }
@@ -139,6 +166,9 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
     if (T == 0) return MOE_OK;
 
     char* ws = static_cast<char*>(cfg->workspace);
+    const Path path = choose_path(*cfg, T);
+    const bool small = path == Path::kSmall, use_tc = path == Path::kTensorCore;
+    auto at = [&](size_t off) { return static_cast<void*>(ws + off); };
     Params p;
     memset(&p, 0, sizeof p);
     p.T = T; p.H = cfg->H; p.E = cfg->E; p.K = cfg->K; p.I = cfg->I; p.Is = cfg->Is;
@@ -153,53 +183,65 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
     p.out = static_cast<__nv_bfloat16*>(out);
     p.topk_idx_out = cfg->topk_idx_out;
     p.topk_w_out = cfg->topk_w_out;
-    p.ctrl = reinterpret_cast<Ctrl*>(ws + L.ctrl);
-    p.idx = reinterpret_cast<int32_t*>(ws + L.idx);
-    p.wts = reinterpret_cast<float*>(ws + L.wts);
-    p.logits = reinterpret_cast<float*>(ws + L.logits);
-    p.counts = reinterpret_cast<int32_t*>(ws + L.counts);
-    p.offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
-    p.bucket_e = reinterpret_cast<int32_t*>(ws + L.bucket_e);
-    p.bucket_n = reinterpret_cast<int32_t*>(ws + L.bucket_n);
-    p.bucket_off = reinterpret_cast<int32_t*>(ws + L.bucket_off);
-    p.ts13 = reinterpret_cast<int32_t*>(ws + L.ts13);
-    p.ts2 = reinterpret_cast<int32_t*>(ws + L.ts2);
-    p.tcs1 = reinterpret_cast<int32_t*>(ws + L.tcs1);
-    p.tcs2 = reinterpret_cast<int32_t*>(ws + L.tcs2);
-    p.tok_of_slot = reinterpret_cast<int32_t*>(ws + L.tok_of_slot);
-    p.slot_of = reinterpret_cast<int32_t*>(ws + L.slot_of);
-    p.hist = reinterpret_cast<int32_t*>(ws + L.hist);
-    p.h_r = reinterpret_cast<__half*>(ws + L.h_r);
-    p.h_s = reinterpret_cast<__half*>(ws + L.h_s);
-    p.hexp = reinterpret_cast<int32_t*>(ws + L.hexp);
-    p.y = reinterpret_cast<float*>(ws + L.y);
+    p.ctrl = static_cast<Ctrl*>(at(L.ctrl));
+    p.idx = static_cast<int32_t*>(at(L.idx));
+    p.wts = static_cast<float*>(at(L.wts));
+    p.counts = static_cast<int32_t*>(at(L.counts));
+    p.offsets = static_cast<int32_t*>(at(L.offsets));
+    p.bucket_e = static_cast<int32_t*>(at(L.bucket_e));
+    p.bucket_n = static_cast<int32_t*>(at(L.bucket_n));
+    p.bucket_off = static_cast<int32_t*>(at(L.bucket_off));
+    p.ts13 = static_cast<int32_t*>(at(L.ts13));
+    p.ts2 = static_cast<int32_t*>(at(L.ts2));
+    p.tcs1 = static_cast<int32_t*>(at(L.tcs1));
+    p.tcs2 = static_cast<int32_t*>(at(L.tcs2));
+    p.tok_of_slot = static_cast<int32_t*>(at(L.tok_of_slot));
+    p.slot_of = static_cast<int32_t*>(at(L.slot_of));
+    p.hist = static_cast<int32_t*>(at(L.hist));
+    p.rank = static_cast<int32_t*>(at(L.rank));
+    p.hexp = static_cast<int32_t*>(at(L.hexp));
+    p.y = static_cast<float*>(at(L.y));
+    if (use_tc) {
+        p.h_r = static_cast<__half*>(at(L.h_r));
+        p.h_s = static_cast<__half*>(at(L.h_s));
+        p.x_perm = static_cast<__nv_bfloat16*>(at(L.x_perm));
+        p.nsl_r = p.nsl_s = 1;
+    } else {
+        p.xq = static_cast<int8_t*>(at(L.xq));
+        p.xs = static_cast<float*>(at(L.xs));
+        p.h32_r = static_cast<float*>(at(L.h32_r));
+        p.h32_s = static_cast<float*>(at(L.h32_s));
+        p.hmax_r = static_cast<float*>(at(L.hmax_r));
+        p.hmax_s = static_cast<float*>(at(L.hmax_s));
+        p.nsl_r = slices_of(cfg->I);
+        p.nsl_s = slices_of(cfg->Is);
+    }
+    p.decode_groups = small ? cdiv(T, kDecodeRouterTok) : 0;
     const int ntiles = cdiv(T, kRouterTileTokens);
     p.router_blocks = ntiles < kRouterMaxBlocks ? ntiles : kRouterMaxBlocks;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const bool force_prefill = (cfg->flags & MOE_FORCE_PREFILL) != 0;
-    const bool small_router = T <= kDecodeMaxTokens && !force_prefill;
-    // Tensor-core grouped GEMMs for large batches; GEMM-2 tiles 256 output
-    // columns, so they need H % 256 == 0 (otherwise the mma.sync kernels run).
-    const bool use_tc = !small_router && !(cfg->flags & MOE_FORCE_DECODE) && cfg->H % 256 == 0;
-    p.x_perm = use_tc ? reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm) : nullptr;
     const long long TK = (long long)T * cfg->K;
     const long long routed_buckets = (cfg->E < TK ? cfg->E : TK) + cdiv(TK, kChunkTokens);
     const long long shared_chunks = cfg->Is > 0 ? cdiv(T, kChunkTokens) : 0;
     // upper bounds of the weight-streaming kernels' CTA tasks
     const long long tasks13 = (long long)(cfg->I / 64) * routed_buckets + (long long)(cfg->Is / 64) * shared_chunks;
-    const long long tasks2 = (long long)(cfg->H / 128) * (routed_buckets + shared_chunks);
-    const long long cap13 = experts_resident_ctas(0, cfg->H);
-    const long long cap2 = experts_resident_ctas(1, cfg->I > cfg->Is ? cfg->I : cfg->Is);
-    const int grid13 = (int)(tasks13 < cap13 ? tasks13 : cap13);
-    const int grid2 = (int)(tasks2 < cap2 ? tasks2 : cap2);
+    const long long tasks2 = (long long)(cfg->H / 128) *
+                             (routed_buckets * slices_of(cfg->I) + shared_chunks * slices_of(cfg->Is));
+    int grid13 = 0, grid2 = 0;
+    if (!use_tc) {
+        const long long cap13 = experts_resident_ctas(0, cfg->H, small);
+        const long long cap2 = experts_resident_ctas(1, cfg->H, small);
+        grid13 = (int)(tasks13 < cap13 ? tasks13 : cap13);
+        grid2 = (int)(tasks2 < cap2 ? tasks2 : cap2);
+    }
 
     void* const* ev = cfg->stage_events;
     auto mark = [&](int idx) -> cudaError_t {
         return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[idx]), s) : cudaSuccess;
     };
     cudaError_t err = mark(2 * MOE_STAGE_ROUTE);
-    if (err == cudaSuccess) err = launch_router(p, small_router, s);
+    if (err == cudaSuccess) err = launch_router(p, small, s);
     if (err == cudaSuccess) err = mark(2 * MOE_STAGE_ROUTE + 1);
     int tc_grid1 = 0, tc_grid2 = 0;
     if (use_tc) {

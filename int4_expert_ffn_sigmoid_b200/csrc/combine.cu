@@ -1,6 +1,8 @@
 // Weighted combine: out[t] = sum_k w[t,k] y[slot(t,k)] + y_shared[t] (+ x[t]),
 // summed in f32 (k ascending, then the shared expert, then the residual) and
-// rounded once to bf16 (round to nearest even).
+// rounded once to bf16 (round to nearest even).  An expert output that the
+// weight-streaming down projection wrote as partial rows, one per slice of
+// its reduction, is first summed over the slices (ascending).
 //
 // Method: colibri README (project listing), "What's implemented" (shared
 // expert; routed experts weighted by the sigmoid router); Colibri-Nano model
@@ -18,18 +20,28 @@ __global__ void __launch_bounds__(256) combine_kernel(Params p) {
     pdl_release();
     if (j >= p.H) return;
     const int K = p.K, H = p.H;
+    const size_t TK = (size_t)p.T * K;
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     for (int k = 0; k < K; ++k) {
-        const int s = __ldg(p.slot_of + (size_t)t * K + k);
-        const float w = __ldg(p.wts + (size_t)t * K + k);
-        const float4 v = __ldg(reinterpret_cast<const float4*>(p.y + (size_t)s * H + j));
+        const int s = __ldcg(p.slot_of + (size_t)t * K + k);
+        const float w = __ldcg(p.wts + (size_t)t * K + k);
+        float4 v = __ldcg(reinterpret_cast<const float4*>(p.y + (size_t)s * H + j));
+        for (int sl = 1; sl < p.nsl_r; ++sl) {
+            const float4 u = __ldcg(reinterpret_cast<const float4*>(p.y + (sl * TK + s) * H + j));
+            v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+        }
         a0 = fmaf(w, v.x, a0);
         a1 = fmaf(w, v.y, a1);
         a2 = fmaf(w, v.z, a2);
         a3 = fmaf(w, v.w, a3);
     }
     if (p.Is > 0) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(p.y + ((size_t)p.T * K + t) * H + j));
+        const float* ys = p.y + TK * p.nsl_r * H;
+        float4 v = __ldcg(reinterpret_cast<const float4*>(ys + (size_t)t * H + j));
+        for (int sl = 1; sl < p.nsl_s; ++sl) {
+            const float4 u = __ldcg(reinterpret_cast<const float4*>(ys + ((size_t)sl * p.T + t) * H + j));
+            v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+        }
         a0 += v.x; a1 += v.y; a2 += v.z; a3 += v.w;
     }
     if (p.flags & 1u) {  // MOE_ADD_RESIDUAL

@@ -7,31 +7,47 @@
 // nanocolibri-engine README, "Converting a checkpoint yourself": per-row
 // symmetric int4, f32 row scales.
 //
-// Design.  One CTA (8 warps) owns one task = (bucket, chunk of up to 16 of the
-// bucket's tokens, block of rows: 64 gate rows + the same 64 up rows, or 128
-// down rows) and walks the reduction dimension in 128-wide k blocks.  The
-// grid is persistent; CTA c takes tasks c, c + grid, ... counted from the
-// heaviest end of the task list (the shared expert's tasks come last in it).
-// The bucket and task tables are copied to shared memory once per CTA.
+// Design.  One CTA (8 warps) owns one task and walks the reduction dimension
+// in 128-wide k blocks.  Gate/up task = (bucket, chunk of up to 16 of its
+// tokens, 64 gate rows + the same 64 up rows); down task = (bucket, chunk,
+// 512-wide slice of the intermediate dimension, 128 down rows).  The grid is
+// persistent; CTA c takes tasks c, c + grid, ... counted from the heaviest
+// end of the task list (the shared expert's tasks are at that end).
 //  - Weights go HBM -> registers: every thread streams 16 contiguous bytes
 //    (32 codes) of two rows per k block with non-allocating 128-bit loads,
-//    kept 4 k blocks ahead in a register ring.  They never touch shared
-//    memory.
-//  - The chunk's activations (x rows, or h rows for the down projection) are
-//    staged in shared memory with cp.async: the whole reduction range at once
-//    when it fits (one barrier per task), else through a 4-deep ring of
-//    128-wide slices.  Rows are padded by 16 bytes so that the per-thread
-//    16-byte fragment reads are conflict-free.
-//  - Codes are unpacked to exact 16-bit integers in natural order and feed
-//    mma.sync m16n8k16 with the tokens as the n dimension; thread q's 16-byte
-//    chunk is exactly its A fragments over two k steps, and the matching
-//    activation chunk is exactly its B fragments.  The four 32-bit words of a
-//    chunk accumulate into four independent accumulator sets (summed at the
-//    end), so consecutive mma never wait on each other.  The row scale is
-//    applied to the f32 result (it factors out of the row's dot product).
+//    kept 4 k blocks ahead in a register ring; they never touch shared memory.
+//  - The codes become int8 operands 16*c with three logic operations per
+//    eight weights (lo8 / hi8), and feed mma.sync m16n8k32 (s8 x s8 -> s32).
+//    Thread q's 16-byte chunk of a row is exactly its A fragments of four
+//    mma k steps: word m gives the even elements (lo8) and the odd ones (hi8)
+//    of one k step.
+//  - Activations are two int8 parts per token (v ~= s (q0 + q1/256), see
+//    quant2); the two parts of token j are mma columns 2j and 2j+1, so a
+//    thread's accumulators hold both parts of the same (row, token) and the
+//    products accumulate exactly in int32.  The chunk's activation rows are
+//    staged in shared memory, padded by 16 bytes so that the per-thread
+//    16-byte fragment reads are conflict-free: the gate/up kernel copies the
+//    router's quantized x (cp.async, whole rows; for H <= 1024 into a second
+//    buffer while the previous task computes; for H > 2048 through a 4-deep
+//    ring of 128-wide slices); the down kernel prefetches the next task's f32
+//    slice of h and its per-64-row maxima of |h| (from the gate/up epilogue)
+//    while the current task computes, then quantizes it with one scale per
+//    (token, slice).
+//  - Latency: the weight ring runs on across task boundaries (the last
+//    blocks of a task are replaced by the first blocks of the CTA's next
+//    task), and a CTA whose first task belongs to the shared expert fills its
+//    ring before the router has finished.
 //  - Gate/up: the 16 mma rows are 8 gate rows and the same 8 up rows, so each
 //    thread ends with gate and up of the same (row, token) and applies SwiGLU
-//    in registers.
+//    in registers; h is stored in f32.  Row and activation scales are applied
+//    to the integer result (they factor out of the row's dot product).
+//  - Down: every slice writes its own partial output row; the combine adds
+//    the slices.
+//  - Small-batch path: each gate/up CTA derives the bucket list, its task
+//    list and the token of every slot from the router's per-group pick counts
+//    and ranks in its prologue; its CTA 0 also writes them to the workspace
+//    for the down kernel and the combine (on the large-batch path the large
+//    router writes them).
 #include "moe_common.cuh"
 #include "moe_launch.h"
 
@@ -39,15 +55,17 @@ namespace moe {
 
 namespace {
 
-constexpr int kRows13 = 64;  // gate (and up) rows per CTA task
-constexpr int kRows2 = 128;  // down rows per CTA task
-constexpr int kRing = 4;     // weight k blocks in flight per thread
-constexpr int kXRing = 4;    // staged activation slices (ring mode)
-constexpr int kPad = 8;      // 16-bit elements of padding per staged row
-constexpr int kTiles = kChunkTokens / 8;
-constexpr int kTab = kMaxE + 2;  // entries of each shared-memory table
-
-// Activation staging capacity of the whole-range mode (elements per row).
+constexpr int kRows13 = 64;   // gate (and up) rows per gate/up task
+constexpr int kRows2 = 128;   // down rows per down task
+constexpr int kRing = 4;      // weight k blocks in flight per thread
+constexpr int kXRing = 4;     // staged activation slices (ring mode)
+constexpr int kPadB = 16;     // bytes of padding per staged row
+constexpr int kStageRows = 2 * kChunkTokens;  // two int8 rows (parts) per token
+constexpr int kTab = kMaxE + 2;               // entries of each table
+constexpr int kMaxSlots = kDecodeMaxTokens * kMaxK;
+// Gate/up activation staging: two whole-row buffers up to kDoubleMaxK, one
+// up to kWholeMaxK, a ring of slices beyond.
+constexpr int kDoubleMaxK = 1024;
 constexpr int kWholeMaxK = 2048;
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
@@ -58,26 +76,196 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
+                 "l"(gmem)
+                 : "memory");
+}
 
-// Shared-memory copy of the bucket and task lists of one kernel.
 struct Tables {
     int n_buckets, ntask;
     int e[kTab], n[kTab], off[kTab], ts[kTab];
 };
 
-__device__ __forceinline__ void load_tables(const Params& p, const int32_t* ts, int ntask_field, Tables& tb) {
-    const int nb = p.ctrl->n_buckets;
-    for (int i = threadIdx.x; i <= nb; i += blockDim.x) {
-        tb.ts[i] = ts[i];
+// Per-CTA shared state, ahead of the staging areas.
+struct Shm {
+    Tables tb;
+    int tok[kMaxSlots];                           // small-batch path: token of each routed slot
+    float xsr[2][kChunkTokens];                   // gate/up: activation scale of each token (per buffer)
+    float hmr[kChunkTokens][kSliceK / kRows13];   // down: the slice's per-64-row maxima of |h|
+    float xsc[kChunkTokens];                      // down: activation scale / 16 of each token
+    QScale qs[kChunkTokens];                      // down: activation scale of each token
+    float hm[8][kChunkTokens];                    // gate/up: per-warp max |h| of each token
+};
+constexpr size_t kShmBytes = (sizeof(Shm) + 127) & ~size_t(127);
+// scratch of the small-batch table build, in the staging area
+constexpr size_t kBuildBytes = (size_t)(kDecodeGroups + 2) * kMaxE * 4;
+
+constexpr size_t max_sz(size_t a, size_t b) { return a > b ? a : b; }
+// gate/up staging modes: 0 two whole-row buffers, 1 one whole-row buffer, 2 ring of slices
+constexpr size_t kSmem13[3] = {
+    kShmBytes + max_sz(kBuildBytes, (size_t)2 * kStageRows * (kDoubleMaxK + kPadB)),
+    kShmBytes + max_sz(kBuildBytes, (size_t)kStageRows * (kWholeMaxK + kPadB)),
+    kShmBytes + max_sz(kBuildBytes, (size_t)kStageRows * (kXRing * 128 + kPadB))};
+// down: int8 staging of one slice + the next task's f32 slice
+constexpr int kStride2 = kSliceK + kPadB;
+constexpr size_t kRaw2Off = (size_t)kStageRows * kStride2;
+constexpr size_t kSmem2 = kShmBytes + kRaw2Off + (size_t)kChunkTokens * kSliceK * 4;
+
+// Tables written to the workspace (by the large router, or by CTA 0 of the
+// small-batch gate/up kernel for the down kernel).
+__device__ __forceinline__ void load_tables(const Params& p, const int32_t* ts, const int* ntask, Tables& tb) {
+    const int nb = __ldcg(&p.ctrl->n_buckets);
+    for (int i = threadIdx.x; i <= nb && i < kTab; i += blockDim.x) {
+        tb.ts[i] = __ldcg(ts + i);
         if (i < nb) {
-            tb.e[i] = p.bucket_e[i];
-            tb.n[i] = p.bucket_n[i];
-            tb.off[i] = p.bucket_off[i];
+            tb.e[i] = __ldcg(p.bucket_e + i);
+            tb.n[i] = __ldcg(p.bucket_n + i);
+            tb.off[i] = __ldcg(p.bucket_off + i);
         }
     }
     if (threadIdx.x == 0) {
-        tb.n_buckets = nb;
-        tb.ntask = ntask_field;
+        tb.n_buckets = nb < kTab ? nb : 0;
+        tb.ntask = nb < kTab ? __ldcg(ntask) : 0;
+        if (nb >= kTab) atomicOr(&p.ctrl->status, ST_BAD_COUNT);
+    }
+    __syncthreads();
+}
+
+// Small-batch path, gate/up kernel: the bucket list, the gate/up task prefix
+// and the token of every routed slot, from the router's per-group pick
+// counts (hist), picks (idx) and ranks.  The slot of pick (t, k) of expert e
+// is offset[e] + (picks of e in the groups before t's) + rank[t, k].  CTA 0
+// also writes the bucket list, the down-task prefix, slot_of and tok_of_slot
+// to the workspace.
+__device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
+    int* s_base = scratch;  // [kDecodeGroups][kMaxE]
+    int* s_cnt = scratch + kDecodeGroups * kMaxE;
+    int* s_off = s_cnt + kMaxE;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int E = p.E, K = p.K, T = p.T, TK = T * K, G = p.decode_groups;
+    const bool writer = blockIdx.x == 0;
+    Tables& tb = sh.tb;
+    int my_e[2], my_rank[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int i = tid + 256 * u;
+        my_e[u] = i < TK ? __ldcg(p.idx + i) : -1;
+        my_rank[u] = i < TK ? __ldcg(p.rank + i) : 0;
+    }
+    if (tid < E) {
+        int h[kDecodeGroups];
+#pragma unroll
+        for (int g = 0; g < kDecodeGroups; ++g) h[g] = g < G ? __ldcg(p.hist + (size_t)g * E + tid) : 0;
+        int run = 0;
+#pragma unroll
+        for (int g = 0; g < kDecodeGroups; ++g) {
+            s_base[g * kMaxE + tid] = run;
+            run += h[g];
+        }
+        s_cnt[tid] = run;
+    }
+    for (int i = tid; i < kMaxSlots; i += blockDim.x) sh.tok[i] = -1;
+    __syncthreads();
+    if (warp == 0) {
+        // lane l owns experts 8l .. 8l+7: counts, non-empty buckets, gate/up
+        // and down tasks, scanned across the warp in one pass
+        constexpr int kPer = kMaxE / 32;
+        const int R13 = p.I / kRows13, R2 = (p.H / kRows2) * slices_of(p.I);
+        int c[kPer];
+        int v[4] = {0, 0, 0, 0};  // slots, buckets, gate/up tasks, down tasks
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int e = lane * kPer + j;
+            c[j] = e < E ? s_cnt[e] : 0;
+            v[0] += c[j];
+            v[1] += c[j] > 0;
+            v[2] += R13 * chunks_of(c[j]);
+            v[3] += R2 * chunks_of(c[j]);
+        }
+        int inc[4] = {v[0], v[1], v[2], v[3]};
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int a = __shfl_up_sync(0xffffffffu, inc[i], o);
+                if (lane >= o) inc[i] += a;
+            }
+        int off = inc[0] - v[0], b = inc[1] - v[1], b13 = inc[2] - v[2], b2 = inc[3] - v[3];
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int e = lane * kPer + j;
+            if (e < E) {
+                s_off[e] = off;
+                if (c[j] > 0) {
+                    tb.e[b] = e;
+                    tb.n[b] = c[j];
+                    tb.off[b] = off;
+                    tb.ts[b] = b13;
+                    if (writer) {
+                        p.bucket_e[b] = e;
+                        p.bucket_n[b] = c[j];
+                        p.bucket_off[b] = off;
+                        p.ts2[b] = b2;
+                    }
+                    ++b;
+                }
+                off += c[j];
+                b13 += R13 * chunks_of(c[j]);
+                b2 += R2 * chunks_of(c[j]);
+            }
+        }
+        const int total = __shfl_sync(0xffffffffu, inc[0], 31);
+        int nb = __shfl_sync(0xffffffffu, inc[1], 31);
+        int t13 = __shfl_sync(0xffffffffu, inc[2], 31), t2 = __shfl_sync(0xffffffffu, inc[3], 31);
+        __syncwarp();
+        if (lane == 0) {
+            if (total != TK) {  // inconsistent counts: flag them and run no routed task
+                atomicOr(&p.ctrl->status, ST_BAD_COUNT);
+                nb = t13 = t2 = 0;
+            }
+            if (p.Is > 0) {  // the shared expert: last bucket, slots TK .. TK+T-1
+                tb.e[nb] = E;
+                tb.n[nb] = T;
+                tb.off[nb] = TK;
+                tb.ts[nb] = t13;
+                if (writer) {
+                    p.bucket_e[nb] = E;
+                    p.bucket_n[nb] = T;
+                    p.bucket_off[nb] = TK;
+                    p.ts2[nb] = t2;
+                }
+                t13 += (p.Is / kRows13) * chunks_of(T);
+                t2 += (p.H / kRows2) * slices_of(p.Is) * chunks_of(T);
+                ++nb;
+            }
+            tb.ts[nb] = t13;
+            tb.n_buckets = nb;
+            tb.ntask = t13;
+            if (writer) {
+                p.ts2[nb] = t2;
+                p.ctrl->n_buckets = nb;
+                p.ctrl->tasks2 = t2;
+            }
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int i = tid + 256 * u;
+        if (i >= TK) continue;
+        const int e = my_e[u], t = i / K;
+        int slot = -1;
+        if (e >= 0 && e < E) slot = s_off[e] + s_base[(t / kDecodeRouterTok) * kMaxE + e] + my_rank[u];
+        else atomicOr(&p.ctrl->status, ST_BAD_EXPERT);
+        if (slot < 0 || slot >= TK) {
+            atomicOr(&p.ctrl->status, ST_BAD_SLOT);
+            slot = -1;
+        } else {
+            sh.tok[slot] = t;
+            if (writer) p.tok_of_slot[slot] = t;
+        }
+        if (writer) p.slot_of[i] = slot < 0 ? 0 : slot;
     }
     __syncthreads();
 }
@@ -91,267 +279,483 @@ __device__ __forceinline__ int find_bucket(const Tables& tb, int task) {
     return lo;
 }
 
-// Stage k blocks [kb_lo, kb_hi) of the chunk's rows (row j at xs + j*stride).
-// Ring mode keeps slice kb at column (kb % kXRing) * 128, whole mode at kb * 128.
-template <bool kWhole>
-__device__ __forceinline__ void stage(uint16_t* xs, int stride, const uint16_t* const* rows, int n, int kb_lo,
-                                      int kb_hi) {
-    const int per_row = (kb_hi - kb_lo) * 16;  // 16-byte chunks per row
-    for (int c = threadIdx.x; c < n * per_row; c += blockDim.x) {
-        const int j = c / per_row, r = c - j * per_row;
-        const int kb = kb_lo + (r >> 4), part = r & 15;
-        const uint16_t* src = rows[j];
-        const int col = (kWhole ? kb : kb % kXRing) * 128 + part * 8;
-        if (src) cp_async16(xs + j * stride + col, src + kb * 128 + part * 8);
-    }
+// Token of slot s of a bucket starting at slot `off`.
+template <bool kSmall>
+__device__ __forceinline__ int slot_token(const Params& p, const Shm& sh, bool shared, int off, int s) {
+    if (shared) return s;
+    if (kSmall) return off + s < kMaxSlots ? sh.tok[off + s] : -1;
+    return __ldcg(p.tok_of_slot + off + s);
 }
 
-// One k block: unpack this thread's 16 bytes of rows a and b, multiply with
-// the staged activations of every n-tile.
-template <bool kBf16>
-__device__ __forceinline__ void kblock(const uint4& wa, const uint4& wb, const uint16_t* xs, int stride, int col0,
-                                       int ntiles, float (&part)[4][kTiles][4]) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+// One k block: this thread's 16 bytes of weight rows a (mma row g) and b (mma
+// row g + 8) against NT n-tiles of staged activations; xrow points at staged
+// row g, byte q*32 of the k block, and n-tile i is 8*i rows further.
+template <int NT, int kSets>
+__device__ __forceinline__ void kblock8(const uint4& wa, const uint4& wb, const uint8_t* xrow, int tile_stride,
+                                        int (&part)[kSets][NT][4]) {
     const uint32_t aw[4] = {wa.x, wa.y, wa.z, wa.w};
     const uint32_t bw[4] = {wb.x, wb.y, wb.z, wb.w};
+    uint32_t A[4][4];
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        uint32_t PA[4], PB[4];
-        int4x8_to_16<kBf16>(aw[w], PA);
-        int4x8_to_16<kBf16>(bw[w], PB);
-        const uint32_t s0[4] = {PA[0], PB[0], PA[1], PB[1]};
-        const uint32_t s1[4] = {PA[2], PB[2], PA[3], PB[3]};
+    for (int m = 0; m < 4; ++m) {
+        A[m][0] = lo8(aw[m]);
+        A[m][1] = lo8(bw[m]);
+        A[m][2] = hi8(aw[m]);
+        A[m][3] = hi8(bw[m]);
+    }
 #pragma unroll
-        for (int i = 0; i < kTiles; ++i) {
-            if (i < ntiles) {
-                const uint4 xv = *reinterpret_cast<const uint4*>(xs + (8 * i + g) * stride + col0 + q * 32 + w * 8);
-                if (kBf16) {
-                    mma_bf16(part[w][i], s0, xv.x, xv.y);
-                    mma_bf16(part[w][i], s1, xv.z, xv.w);
-                } else {
-                    mma_f16(part[w][i], s0, xv.x, xv.y);
-                    mma_f16(part[w][i], s1, xv.z, xv.w);
-                }
-            }
-        }
+    for (int i = 0; i < NT; ++i) {
+        const uint4 b01 = *reinterpret_cast<const uint4*>(xrow + i * tile_stride);
+        const uint4 b23 = *reinterpret_cast<const uint4*>(xrow + i * tile_stride + 16);
+        mma_s8(part[0][i], A[0], b01.x, b01.y);
+        mma_s8(part[kSets - 1][i], A[1], b01.z, b01.w);
+        mma_s8(part[0][i], A[2], b23.x, b23.y);
+        mma_s8(part[kSets - 1][i], A[3], b23.z, b23.w);
     }
 }
 
-// Main loop of both projections: this thread streams 16 bytes of rows ra
-// (mma row g) and rb (mma row g + 8) per k block; on return acc[i] holds
-// weights x activations of n-tile i.
-template <bool kBf16, bool kWhole>
-__device__ __forceinline__ void stream_rows(const uint8_t* ra, const uint8_t* rb, int nkb, uint16_t* xs, int stride,
-                                            const uint16_t* const* rows, int nc, int ntiles,
-                                            float (&acc)[kTiles][4]) {
-    float part[4][kTiles][4];
-#pragma unroll
-    for (int w = 0; w < 4; ++w)
-#pragma unroll
-        for (int i = 0; i < kTiles; ++i) part[w][i][0] = part[w][i][1] = part[w][i][2] = part[w][i][3] = 0.f;
-    uint4 ring_a[kRing], ring_b[kRing];
+// This thread's weight stream of one task: 16 bytes of rows a (mma row g)
+// and b (mma row g + 8) per k block, nkb blocks 64 bytes apart (nkb = 0: no
+// task).
+struct WStream {
+    const uint8_t* ra;
+    const uint8_t* rb;
+    int nkb;
+};
+
+// Register ring of weight blocks in flight (block kb of a task in slot
+// kb % kRing).
+struct Ring {
+    uint4 a[kRing], b[kRing];
+};
+
+__device__ __forceinline__ void prime(Ring& r, const WStream& s) {
 #pragma unroll
     for (int i = 0; i < kRing; ++i) {
-        ring_a[i] = i < nkb ? ld_stream_v4(ra + i * 64) : make_uint4(0, 0, 0, 0);
-        ring_b[i] = i < nkb ? ld_stream_v4(rb + i * 64) : make_uint4(0, 0, 0, 0);
+        r.a[i] = i < s.nkb ? ld_stream_v4(s.ra + i * 64) : make_uint4(0, 0, 0, 0);
+        r.b[i] = i < s.nkb ? ld_stream_v4(s.rb + i * 64) : make_uint4(0, 0, 0, 0);
     }
-    if (kWhole) {
-        stage<true>(xs, stride, rows, nc, 0, nkb);
-        cp_async_commit();
-        cp_async_wait<0>();
-        __syncthreads();
-    } else {
+}
+
+// Main loop of both projections.  On entry the ring holds the first blocks
+// of `cur` and (whole modes) every k block of its activations is staged and
+// visible at byte 128*kb of its rows.  Ring mode: stage_slice(kb) issues the
+// cp.async of block kb into slot kb % kXRing, driven from here.  While the
+// last blocks of `cur` are consumed, the freed ring slots are refilled with
+// the first blocks of `nxt` (when cur.nkb is a multiple of kRing, so that
+// they land in their own slots); returns whether it did.
+template <int NT, bool kRingMode, typename StageSlice>
+__device__ __forceinline__ bool stream8(Ring& ring, const WStream& cur, const WStream& nxt, const uint8_t* xs,
+                                        int stride, StageSlice&& stage_slice, int (&acc)[NT][4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int nkb = cur.nkb;
+    const bool cont = nxt.nkb > 0 && nkb % kRing == 0;
+    // two accumulator sets break the chain of dependent mma when there is one tile
+    constexpr int kSets = NT == 1 ? 2 : 1;
+    int part[kSets][NT][4];
+#pragma unroll
+    for (int s = 0; s < kSets; ++s)
+#pragma unroll
+        for (int i = 0; i < NT; ++i) part[s][i][0] = part[s][i][1] = part[s][i][2] = part[s][i][3] = 0;
+    if (kRingMode) {
 #pragma unroll
         for (int i = 0; i < kXRing - 1; ++i) {
-            if (i < nkb) stage<false>(xs, stride, rows, nc, i, i + 1);
+            if (i < nkb) stage_slice(i);
             cp_async_commit();
         }
     }
+    const uint8_t* xrow = xs + g * stride + q * 32;
     for (int kb0 = 0; kb0 < nkb; kb0 += kRing) {
 #pragma unroll
         for (int rr = 0; rr < kRing; ++rr) {
             const int kb = kb0 + rr;
             if (kb < nkb) {
-                if (!kWhole) {
+                if (kRingMode) {
                     cp_async_wait<kXRing - 2>();
-                    __syncthreads();  // slice kb visible to all; slice kb-1's readers are done
-                    if (kb + kXRing - 1 < nkb) stage<false>(xs, stride, rows, nc, kb + kXRing - 1, kb + kXRing);
+                    __syncthreads();  // block kb visible to all; block kb-1's readers are done
+                    if (kb + kXRing - 1 < nkb) stage_slice(kb + kXRing - 1);
                     cp_async_commit();
                 }
-                const uint4 wa = ring_a[rr], wb = ring_b[rr];
-                if (kb + kRing < nkb) {
-                    ring_a[rr] = ld_stream_v4(ra + (kb + kRing) * 64);
-                    ring_b[rr] = ld_stream_v4(rb + (kb + kRing) * 64);
+                const uint4 wa = ring.a[rr], wb = ring.b[rr];
+                const int nb = kb + kRing;
+                if (nb < nkb) {
+                    ring.a[rr] = ld_stream_v4(cur.ra + nb * 64);
+                    ring.b[rr] = ld_stream_v4(cur.rb + nb * 64);
+                } else if (cont && nb - nkb < nxt.nkb) {
+                    ring.a[rr] = ld_stream_v4(nxt.ra + (nb - nkb) * 64);
+                    ring.b[rr] = ld_stream_v4(nxt.rb + (nb - nkb) * 64);
                 }
-                kblock<kBf16>(wa, wb, xs, stride, (kWhole ? kb : kb % kXRing) * 128, ntiles, part);
+                kblock8<NT, kSets>(wa, wb, xrow + (kRingMode ? kb % kXRing : kb) * 128, 8 * stride, part);
             }
         }
     }
 #pragma unroll
-    for (int i = 0; i < kTiles; ++i)
+    for (int i = 0; i < NT; ++i)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[i][c] = (part[0][i][c] + part[1][i][c]) + (part[2][i][c] + part[3][i][c]);
+        for (int c = 0; c < 4; ++c) acc[i][c] = part[0][i][c] + part[kSets - 1][i][c] * (kSets - 1);
+    return cont;
 }
 
-// Per-task data of the epilogue, loaded before the main loop: the h-scale
-// exponent of each token column this thread owns.
-__device__ __forceinline__ void load_hexp(const Params& p, bool shared, int off, int tok0, int n,
-                                          int (&hx)[2 * kTiles]) {
-    const int q = (threadIdx.x & 31) & 3;
-#pragma unroll
-    for (int i = 0; i < kTiles; ++i)
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const int s = tok0 + 8 * i + 2 * q + cc;
-            int t = -1;
-            if (s < n) t = shared ? s : __ldg(p.tok_of_slot + off + s);
-            hx[2 * i + cc] = (t >= 0 && t < p.T) ? __ldg(p.hexp + t) : 0;
-        }
+// Both int8 parts of mma columns 2j, 2j+1 -> the value in units of the
+// activation scale times 16.
+__device__ __forceinline__ float join(int c0, int c1) { return (float)c0 + (float)c1 * (1.0f / 256.0f); }
+
+// One gate/up task as this thread sees it.
+struct Task13 {
+    WStream w;  // gate row r0 + g and up row r0 + g
+    bool ok;    // false: no task, or a table entry out of range
+    bool shared;
+    int e, off, irow, rbk, tok0, nc, r0;
+};
+
+// Gate/up task `local` of bucket (e, n, off).
+__device__ __forceinline__ Task13 make13(const Params& p, int e, int n, int off, int local) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, q = lane & 3;
+    Task13 t;
+    t.ok = !(e < 0 || e > p.E || (e == p.E && p.Is == 0));
+    t.shared = e == p.E;
+    t.e = e;
+    t.off = off;
+    t.irow = t.shared ? p.Is : p.I;
+    const int R = t.irow / kRows13;
+    const int c = local / R;
+    t.rbk = local - c * R;
+    t.tok0 = c * kChunkTokens;
+    t.nc = min(kChunkTokens, n - t.tok0);
+    t.r0 = t.rbk * kRows13 + warp * 8;
+    const int row_bytes = p.H / 2;
+    const uint8_t* W = t.shared ? p.sh_w13 : p.w13 + (size_t)(t.ok ? e : 0) * 2 * p.I * row_bytes;
+    t.w.ra = W + (size_t)(t.r0 + g) * row_bytes + q * 16;
+    t.w.rb = W + (size_t)(t.irow + t.r0 + g) * row_bytes + q * 16;
+    t.w.nkb = t.ok ? p.H / 128 : 0;
+    return t;
 }
 
-constexpr size_t kTabBytes = (sizeof(Tables) + 15) & ~size_t(15);
+__device__ __forceinline__ Task13 task13_at(const Params& p, const Tables& tb, int lin) {
+    if (lin >= tb.ntask) {
+        Task13 t{};
+        return t;
+    }
+    const int task = tb.ntask - 1 - lin;
+    const int b = find_bucket(tb, task);
+    return make13(p, tb.e[b], tb.n[b], tb.off[b], task - tb.ts[b]);
+}
 
-template <bool kWhole>
-__global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
-    extern __shared__ __align__(16) uint8_t dsm[];
-    Tables& tb = *reinterpret_cast<Tables*>(dsm);
-    uint16_t* xs = reinterpret_cast<uint16_t*>(dsm + kTabBytes);
-    __shared__ const uint16_t* rows[kChunkTokens];
+// Issues the cp.async of task t's activation rows (both parts of each token)
+// into `buf` and of its tokens' activation scales into xsr, as one group.
+template <bool kSmall>
+__device__ __forceinline__ void stage13(const Params& p, const Shm& sh, const Task13& t, uint8_t* buf, int stride,
+                                        float* xsr) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, q = lane & 3;
-    const int H = p.H, E = p.E;
-    const int row_bytes = H / 2;
-    const int nkb = H / 128;
-    const int stride = (kWhole ? H : kXRing * 128) + kPad;
-    // the shared expert's weights are needed whatever the routing: warm L2
-    // while the router finishes
+    const int H = p.H;
+    for (int r = warp; r < 2 * t.nc; r += 8) {
+        const int tok = slot_token<kSmall>(p, sh, t.shared, t.off, t.tok0 + (r >> 1));
+        if (tok < 0 || tok >= p.T) continue;
+        const int8_t* src = p.xq + (size_t)tok * 2 * H + (r & 1) * H;
+        for (int c16 = lane; c16 < H / 16; c16 += 32) cp_async16(buf + r * stride + c16 * 16, src + c16 * 16);
+    }
+    if (threadIdx.x < t.nc) {
+        const int tok = slot_token<kSmall>(p, sh, t.shared, t.off, t.tok0 + threadIdx.x);
+        if (tok >= 0 && tok < p.T) {
+            cp_async4(xsr + threadIdx.x, p.xs + tok);
+        } else {
+            xsr[threadIdx.x] = 0.f;
+            atomicOr(&p.ctrl->status, ST_BAD_SLOT);
+        }
+    }
+    cp_async_commit();
+}
+
+template <int NT, bool kRingMode, typename StageSlice>
+__device__ __forceinline__ bool run13(Ring& ring, const Task13& tk, const WStream& nx, float gs, float us,
+                                      const Params& p, const uint8_t* xs, int stride, Shm& sh, const float* xsr,
+                                      StageSlice&& stage_slice) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, q = lane & 3;
+    int acc[NT][4];
+    const bool cont = stream8<NT, kRingMode>(ring, tk.w, nx, xs, stride, stage_slice, acc);
+    const int slot0 = (tk.shared ? 0 : tk.off) + tk.tok0;
+    float* hrow0 = (tk.shared ? p.h32_s : p.h32_r) + (size_t)slot0 * tk.irow + tk.r0 + g;
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+        const int j = 4 * i + q;
+        float hm = 0.f;
+        if (j < tk.nc) {
+            const float xsc = xsr[j] * 0.0625f;
+            const float gv = join(acc[i][0], acc[i][1]) * (gs * xsc);
+            const float uv = join(acc[i][2], acc[i][3]) * (us * xsc);
+            const float h = silu_mul(gv, uv);
+            hrow0[(size_t)j * tk.irow] = h;
+            hm = fabsf(h);
+        }
+        hm = nanmax(hm, __shfl_xor_sync(0xffffffffu, hm, 4));
+        hm = nanmax(hm, __shfl_xor_sync(0xffffffffu, hm, 8));
+        hm = nanmax(hm, __shfl_xor_sync(0xffffffffu, hm, 16));
+        if (g == 0 && j < tk.nc) sh.hm[warp][j] = hm;
+    }
+    __syncthreads();  // also: every warp is past its main loop
+    if (threadIdx.x < tk.nc) {
+        const int j = threadIdx.x;
+        const int nrb = tk.irow / kRows13;
+        float m = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) m = nanmax(m, sh.hm[w][j]);
+        (tk.shared ? p.hmax_s : p.hmax_r)[(size_t)(slot0 + j) * nrb + tk.rbk] = m;
+    }
+    return cont;
+}
+
+// kMode: 0 two whole-row staging buffers (the next task's activations load
+// while the current task computes), 1 one whole-row buffer, 2 ring of slices.
+template <int kMode, bool kSmall>
+__global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
+    extern __shared__ __align__(128) uint8_t dsm[];
+    Shm& sh = *reinterpret_cast<Shm*>(dsm);
+    uint8_t* xs = dsm + kShmBytes;
+    const int g = (threadIdx.x & 31) >> 2;
+    const int H = p.H;
+    const int stride = (kMode == 2 ? kXRing * 128 : H) + kPadB;
+    const int bufbytes = kStageRows * stride;
+    Ring ring;
+    // The shared expert's tasks come first in every CTA's order and do not
+    // depend on the routing: a CTA whose first task is one starts its weight
+    // stream before the router has finished; the rest of the shared expert
+    // is warmed in L2.
+    const int ns = p.Is > 0 ? (p.Is / kRows13) * chunks_of(p.T) : 0;
+    bool primed = false;
+    const uint8_t* primed_ra = nullptr;
+    if ((int)blockIdx.x < ns) {
+        const Task13 t = make13(p, p.E, p.T, p.T * p.K, ns - 1 - (int)blockIdx.x);
+        prime(ring, t.w);
+        primed = true;
+        primed_ra = t.w.ra;
+    }
     if (p.Is > 0) prefetch_l2_slice(p.sh_w13, (size_t)p.Is * p.H);
     pdl_wait();
     pdl_release();
-    load_tables(p, p.ts13, p.ctrl->tasks13, tb);
+    if (kSmall) build_tables_small(p, sh, reinterpret_cast<int*>(xs));
+    else load_tables(p, p.ts13, &p.ctrl->tasks13, sh.tb);
+    const Tables& tb = sh.tb;
+    Task13 cur = task13_at(p, tb, blockIdx.x);
+    if (primed && cur.w.ra != primed_ra) primed = false;
+    if (kMode != 2 && cur.ok) stage13<kSmall>(p, sh, cur, xs, stride, sh.xsr[0]);
+    const float* S = cur.shared ? p.sh_s13 : p.s13 + (size_t)cur.e * 2 * p.I;
+    float gs = cur.ok ? __ldg(S + cur.r0 + g) : 0.f, us = cur.ok ? __ldg(S + cur.irow + cur.r0 + g) : 0.f;
+    int buf = 0;
     for (int lin = blockIdx.x; lin < tb.ntask; lin += gridDim.x) {
-        const int task = tb.ntask - 1 - lin;
-        const int b = find_bucket(tb, task);
-        const int e = tb.e[b], n = tb.n[b], off = tb.off[b];
-        if (e < 0 || e > E || (e == E && p.Is == 0)) {
+        const Task13 nx = task13_at(p, tb, lin + gridDim.x);
+        if (!cur.ok) {  // a table entry out of range: flag it and stop
             if (threadIdx.x == 0) atomicOr(&p.ctrl->status, ST_BAD_TASK);
-            continue;
+            break;
         }
-        const bool shared = (e == E);
-        const int irow = shared ? p.Is : p.I;
-        const int R = irow / kRows13;
-        const int local = task - tb.ts[b];
-        const int c = local / R, rbk = local - c * R;
-        const int tok0 = c * kChunkTokens;
-        const int nc = min(kChunkTokens, n - tok0);
-        const int ntiles = (nc + 7) >> 3;
-        const int r0 = rbk * kRows13 + warp * 8;
-        const uint8_t* W = shared ? p.sh_w13 : p.w13 + (size_t)e * 2 * p.I * row_bytes;
-        const float* S = shared ? p.sh_s13 : p.s13 + (size_t)e * 2 * p.I;
-        const uint8_t* grow = W + (size_t)(r0 + g) * row_bytes + q * 16;
-        const uint8_t* urow = W + (size_t)(irow + r0 + g) * row_bytes + q * 16;
-
-        __syncthreads();  // the previous task is done with rows[] and xs
-        for (int j = threadIdx.x; j < nc; j += blockDim.x) {
-            const int t = shared ? tok0 + j : __ldg(p.tok_of_slot + off + tok0 + j);
-            const bool ok = t >= 0 && t < p.T;
-            if (!ok) atomicOr(&p.ctrl->status, ST_BAD_SLOT);
-            rows[j] = ok ? reinterpret_cast<const uint16_t*>(p.x + (size_t)t * H) : nullptr;
+        if (!primed) prime(ring, cur.w);
+        if (kMode == 2 && threadIdx.x < cur.nc) {  // ring mode: the scales only (slices are staged in the loop)
+            const int tok = slot_token<kSmall>(p, sh, cur.shared, cur.off, cur.tok0 + threadIdx.x);
+            if (tok >= 0 && tok < p.T) cp_async4(sh.xsr[0] + threadIdx.x, p.xs + tok);
+            else sh.xsr[0][threadIdx.x] = 0.f;
         }
-        int hx[2 * kTiles];
-        load_hexp(p, shared, off, tok0, n, hx);
-        const float gs = __ldg(S + r0 + g), us = __ldg(S + irow + r0 + g);
-        __syncthreads();
-        float acc[kTiles][4];
-        stream_rows<true, kWhole>(grow, urow, nkb, xs, stride, rows, nc, ntiles, acc);
-
-        __half* hb = shared ? p.h_s : p.h_r;
-        const size_t hbase = shared ? 0 : (size_t)off;
-#pragma unroll
-        for (int i = 0; i < kTiles; ++i) {
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int s = tok0 + 8 * i + 2 * q + cc;
-                if (i < ntiles && s < n) {
-                    const float sc = ldexpf(1.0f, -hx[2 * i + cc]);
-                    const float gv = acc[i][cc] * gs, uv = acc[i][2 + cc] * us;
-                    hb[(hbase + s) * irow + r0 + g] = __float2half_rn(silu_mul(gv, uv) * sc);
-                }
+        if (kMode != 2) cp_async_wait<0>();
+        __syncthreads();  // cur's activations are visible; the previous task is done with every buffer
+        if (kMode == 0 && nx.ok) stage13<kSmall>(p, sh, nx, xs + (buf ^ 1) * bufbytes, stride, sh.xsr[buf ^ 1]);
+        float gs_n = 0.f, us_n = 0.f;
+        if (nx.ok) {
+            const float* Sn = nx.shared ? p.sh_s13 : p.s13 + (size_t)nx.e * 2 * p.I;
+            gs_n = __ldg(Sn + nx.r0 + g);
+            us_n = __ldg(Sn + nx.irow + nx.r0 + g);
+        }
+        const int nc = cur.nc;
+        const Task13& c = cur;
+        auto stage_slice = [&](int kb) {
+            const int r = threadIdx.x >> 3, part = threadIdx.x & 7;
+            if (r < 2 * nc) {
+                const int tok = slot_token<kSmall>(p, sh, c.shared, c.off, c.tok0 + (r >> 1));
+                if (tok >= 0 && tok < p.T)
+                    cp_async16(xs + r * stride + (kb % kXRing) * 128 + part * 16,
+                               p.xq + (size_t)tok * 2 * H + (r & 1) * H + kb * 128 + part * 16);
             }
+        };
+        const uint8_t* xb = xs + (kMode == 0 ? buf * bufbytes : 0);
+        const float* xsr = sh.xsr[kMode == 0 ? buf : 0];
+        switch ((2 * nc + 7) >> 3) {
+            case 1: primed = run13<1, kMode == 2>(ring, cur, nx.w, gs, us, p, xb, stride, sh, xsr, stage_slice); break;
+            case 2: primed = run13<2, kMode == 2>(ring, cur, nx.w, gs, us, p, xb, stride, sh, xsr, stage_slice); break;
+            case 3: primed = run13<3, kMode == 2>(ring, cur, nx.w, gs, us, p, xb, stride, sh, xsr, stage_slice); break;
+            default: primed = run13<4, kMode == 2>(ring, cur, nx.w, gs, us, p, xb, stride, sh, xsr, stage_slice); break;
         }
+        if (kMode == 1 && nx.ok) stage13<kSmall>(p, sh, nx, xs, stride, sh.xsr[0]);
+        cur = nx;
+        gs = gs_n;
+        us = us_n;
+        if (kMode == 0) buf ^= 1;
     }
 }
 
-template <bool kWhole>
+// One down task as this thread sees it.
+struct Task2 {
+    WStream w;  // down rows j0 + g and j0 + g + 8, from the slice's first k block
+    bool ok, shared;
+    int e, off, irow, sl, k0, klen, tok0, nc, j0;
+};
+
+// Down task `local` of bucket (e, n, off).
+__device__ __forceinline__ Task2 make2(const Params& p, int e, int n, int off, int local) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, q = lane & 3;
+    Task2 t;
+    t.ok = !(e < 0 || e > p.E || (e == p.E && p.Is == 0));
+    t.shared = e == p.E;
+    t.e = e;
+    t.off = off;
+    t.irow = t.shared ? p.Is : p.I;
+    const int R = p.H / kRows2, nsl = slices_of(t.irow);
+    const int rbk = local % R, rest = local / R;
+    t.sl = rest % nsl;
+    const int c = rest / nsl;
+    t.k0 = t.sl * kSliceK;
+    t.klen = min(kSliceK, t.irow - t.k0);
+    t.tok0 = c * kChunkTokens;
+    t.nc = min(kChunkTokens, n - t.tok0);
+    t.j0 = rbk * kRows2 + warp * 16;
+    const int row_bytes = t.irow / 2;
+    const uint8_t* W = t.shared ? p.sh_w2 : p.w2 + (size_t)(t.ok ? e : 0) * p.H * row_bytes;
+    t.w.ra = W + (size_t)(t.j0 + g) * row_bytes + t.k0 / 2 + q * 16;
+    t.w.rb = W + (size_t)(t.j0 + g + 8) * row_bytes + t.k0 / 2 + q * 16;
+    t.w.nkb = t.ok ? t.klen / 128 : 0;
+    return t;
+}
+
+__device__ __forceinline__ Task2 task2_at(const Params& p, const Tables& tb, int lin) {
+    if (lin >= tb.ntask) {
+        Task2 t{};
+        return t;
+    }
+    const int task = tb.ntask - 1 - lin;
+    const int b = find_bucket(tb, task);
+    return make2(p, tb.e[b], tb.n[b], tb.off[b], task - tb.ts[b]);
+}
+
+// Issues the cp.async of task t's f32 slice of h (raw[j][k], k < klen) and of
+// its per-64-row maxima of |h| (sh.hmr), as one group.
+__device__ __forceinline__ void fetch2(const Params& p, Shm& sh, const Task2& t, float* raw) {
+    const float* hb = t.shared ? p.h32_s : p.h32_r;
+    const float* hmb = t.shared ? p.hmax_s : p.hmax_r;
+    const int nrb = t.irow / kRows13;
+    const int slot0 = (t.shared ? 0 : t.off) + t.tok0;
+    const int per = t.klen / 4;  // 16-byte chunks per token
+    for (int c = threadIdx.x; c < t.nc * per; c += blockDim.x) {
+        const int j = c / per, k4 = c - j * per;
+        cp_async16(raw + j * kSliceK + k4 * 4, hb + (size_t)(slot0 + j) * t.irow + t.k0 + k4 * 4);
+    }
+    const int nb = t.klen / kRows13;
+    for (int c = threadIdx.x; c < t.nc * nb; c += blockDim.x) {
+        const int j = c / nb, r = c - j * nb;
+        cp_async4(&sh.hmr[j][r], hmb + (size_t)(slot0 + j) * nrb + t.k0 / kRows13 + r);
+    }
+    cp_async_commit();
+}
+
+template <int NT>
+__device__ __forceinline__ bool run2(Ring& ring, const Task2& tk, const WStream& nx, float s_lo, float s_hi,
+                                     const Params& p, const uint8_t* xs, const Shm& sh) {
+    const int g = (threadIdx.x & 31) >> 2, q = (threadIdx.x & 31) & 3;
+    int acc[NT][4];
+    const bool cont = stream8<NT, false>(ring, tk.w, nx, xs, kStride2, [](int) {}, acc);
+    const size_t TK = (size_t)p.T * p.K;
+    const size_t yrow0 = tk.shared ? TK * p.nsl_r + (size_t)tk.sl * p.T + tk.tok0 : (size_t)tk.sl * TK + tk.off + tk.tok0;
+    float* y0 = p.y + yrow0 * p.H + tk.j0 + g;
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+        const int j = 4 * i + q;
+        if (j < tk.nc) {
+            const float xsc = sh.xsc[j];
+            float* yr = y0 + (size_t)j * p.H;
+            yr[0] = join(acc[i][0], acc[i][1]) * (s_lo * xsc);
+            yr[8] = join(acc[i][2], acc[i][3]) * (s_hi * xsc);
+        }
+    }
+    return cont;
+}
+
 __global__ void __launch_bounds__(256, 2) experts_w2_kernel(Params p) {
-    extern __shared__ __align__(16) uint8_t dsm[];
-    Tables& tb = *reinterpret_cast<Tables*>(dsm);
-    uint16_t* hs = reinterpret_cast<uint16_t*>(dsm + kTabBytes);
-    __shared__ const uint16_t* rows[kChunkTokens];
+    extern __shared__ __align__(128) uint8_t dsm[];
+    Shm& sh = *reinterpret_cast<Shm*>(dsm);
+    uint8_t* xs = dsm + kShmBytes;
+    float* raw = reinterpret_cast<float*>(xs + kRaw2Off);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, q = lane & 3;
-    const int H = p.H, E = p.E;
-    const int R = H / kRows2;
-    const int stride = (kWhole ? max(p.I, p.Is) : kXRing * 128) + kPad;
+    const int g = lane >> 2;
+    Ring ring;
+    const int ns = p.Is > 0 ? (p.H / kRows2) * chunks_of(p.T) * slices_of(p.Is) : 0;
+    bool primed = false;
+    const uint8_t* primed_ra = nullptr;
+    if ((int)blockIdx.x < ns) {
+        const Task2 t = make2(p, p.E, p.T, p.T * p.K, ns - 1 - (int)blockIdx.x);
+        prime(ring, t.w);
+        primed = true;
+        primed_ra = t.w.ra;
+    }
     if (p.Is > 0) prefetch_l2_slice(p.sh_w2, (size_t)p.H * p.Is / 2);
     pdl_wait();
     pdl_release();
-    load_tables(p, p.ts2, p.ctrl->tasks2, tb);
+    load_tables(p, p.ts2, &p.ctrl->tasks2, sh.tb);
+    const Tables& tb = sh.tb;
+    Task2 cur = task2_at(p, tb, blockIdx.x);
+    if (primed && cur.w.ra != primed_ra) primed = false;
+    if (cur.ok) fetch2(p, sh, cur, raw);
+    const float* S = cur.shared ? p.sh_s2 : p.s2 + (size_t)cur.e * p.H;
+    float s_lo = cur.ok ? __ldg(S + cur.j0 + g) : 0.f, s_hi = cur.ok ? __ldg(S + cur.j0 + g + 8) : 0.f;
     for (int lin = blockIdx.x; lin < tb.ntask; lin += gridDim.x) {
-        const int task = tb.ntask - 1 - lin;
-        const int b = find_bucket(tb, task);
-        const int e = tb.e[b], n = tb.n[b], off = tb.off[b];
-        if (e < 0 || e > E || (e == E && p.Is == 0)) {
+        const Task2 nx = task2_at(p, tb, lin + gridDim.x);
+        if (!cur.ok) {  // a table entry out of range: flag it and stop
             if (threadIdx.x == 0) atomicOr(&p.ctrl->status, ST_BAD_TASK);
-            continue;
+            break;
         }
-        const bool shared = (e == E);
-        const int irow = shared ? p.Is : p.I;
-        const int row_bytes = irow / 2;
-        const int nkb = irow / 128;
-        const int local = task - tb.ts[b];
-        const int c = local / R, rbk = local - c * R;
-        const int tok0 = c * kChunkTokens;
-        const int nc = min(kChunkTokens, n - tok0);
-        const int ntiles = (nc + 7) >> 3;
-        const int j0 = rbk * kRows2 + warp * 16;
-        const uint8_t* W = shared ? p.sh_w2 : p.w2 + (size_t)e * H * row_bytes;
-        const float* S = shared ? p.sh_s2 : p.s2 + (size_t)e * H;
-        const uint8_t* lrow = W + (size_t)(j0 + g) * row_bytes + q * 16;
-        const uint8_t* hrow8 = W + (size_t)(j0 + g + 8) * row_bytes + q * 16;
-        const __half* hb = shared ? p.h_s : p.h_r;
-        const size_t hbase = shared ? 0 : (size_t)off;
-
+        if (!primed) prime(ring, cur.w);
+        const int nc = cur.nc, klen = cur.klen;
+        cp_async_wait<0>();
+        __syncthreads();  // cur's h slice and maxima are visible; the previous task is done with xs
+        if (threadIdx.x < nc) {
+            const int j = threadIdx.x;
+            float m = 0.f;
+            for (int r = 0; r < klen / kRows13; ++r) m = nanmax(m, sh.hmr[j][r]);
+            const QScale qs = qscale(m);
+            sh.qs[j] = qs;
+            sh.xsc[j] = qs.s * 0.0625f;
+        }
         __syncthreads();
-        for (int j = threadIdx.x; j < nc; j += blockDim.x)
-            rows[j] = reinterpret_cast<const uint16_t*>(hb + (hbase + tok0 + j) * irow);
-        int hx[2 * kTiles];
-        load_hexp(p, shared, off, tok0, n, hx);
-        const float sl = __ldg(S + j0 + g), sh = __ldg(S + j0 + g + 8);
-        __syncthreads();
-        float acc[kTiles][4];
-        stream_rows<false, kWhole>(lrow, hrow8, nkb, hs, stride, rows, nc, ntiles, acc);
-
-#pragma unroll
-        for (int i = 0; i < kTiles; ++i) {
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int s = tok0 + 8 * i + 2 * q + cc;
-                if (i < ntiles && s < n) {
-                    const float inv = ldexpf(1.0f, hx[2 * i + cc]);
-                    const size_t ys = shared ? (size_t)p.T * p.K + s : (size_t)off + s;
-                    float* yr = p.y + ys * H + j0 + g;
-                    yr[0] = acc[i][cc] * (sl * inv);
-                    yr[8] = acc[i][2 + cc] * (sh * inv);
-                }
+        for (int j = warp; j < nc; j += 8) {
+            const QScale qs = sh.qs[j];
+            const float* src = raw + j * kSliceK;
+            for (int gi = lane; gi < klen / 8; gi += 32) {
+                const float4 a = *reinterpret_cast<const float4*>(src + 8 * gi);
+                const float4 b2 = *reinterpret_cast<const float4*>(src + 8 * gi + 4);
+                const float f[8] = {a.x, a.y, a.z, a.w, b2.x, b2.y, b2.z, b2.w};
+                uint2 p0, p1;
+                quant2x8(f, qs, p0, p1);
+                *reinterpret_cast<uint2*>(xs + (2 * j) * kStride2 + 8 * gi) = p0;
+                *reinterpret_cast<uint2*>(xs + (2 * j + 1) * kStride2 + 8 * gi) = p1;
             }
         }
+        __syncthreads();  // staged; raw and hmr are free for the next task
+        if (nx.ok) fetch2(p, sh, nx, raw);
+        float s_lo_n = 0.f, s_hi_n = 0.f;
+        if (nx.ok) {
+            const float* Sn = nx.shared ? p.sh_s2 : p.s2 + (size_t)nx.e * p.H;
+            s_lo_n = __ldg(Sn + nx.j0 + g);
+            s_hi_n = __ldg(Sn + nx.j0 + g + 8);
+        }
+        switch ((2 * nc + 7) >> 3) {
+            case 1: primed = run2<1>(ring, cur, nx.w, s_lo, s_hi, p, xs, sh); break;
+            case 2: primed = run2<2>(ring, cur, nx.w, s_lo, s_hi, p, xs, sh); break;
+            case 3: primed = run2<3>(ring, cur, nx.w, s_lo, s_hi, p, xs, sh); break;
+            default: primed = run2<4>(ring, cur, nx.w, s_lo, s_hi, p, xs, sh); break;
+        }
+        cur = nx;
+        s_lo = s_lo_n;
+        s_hi = s_hi_n;
     }
 }
 
 template <typename Kern>
 int resident(Kern kern, size_t smem, int which) {
-    static int cache[4][64];
+    static int cache[8][64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
     int& c = cache[which][dev];
@@ -365,30 +769,39 @@ int resident(Kern kern, size_t smem, int which) {
     return c;
 }
 
-constexpr size_t kWholeSmem = kTabBytes + (size_t)kChunkTokens * (kWholeMaxK + kPad) * 2;
-constexpr size_t kRingSmem = kTabBytes + (size_t)kChunkTokens * (kXRing * 128 + kPad) * 2;
-
 }  // namespace
 
 // Persistent grid of the weight-streaming kernels: the CTAs that fit at once
-// (which: 0 gate/up, 1 down; kdim: its longest reduction range).
-int experts_resident_ctas(int which, int kdim) {
-    const bool whole = kdim <= kWholeMaxK;
-    if (which == 0)
-        return whole ? resident(experts_w13_kernel<true>, kWholeSmem, 0)
-                     : resident(experts_w13_kernel<false>, kRingSmem, 1);
-    return whole ? resident(experts_w2_kernel<true>, kWholeSmem, 2) : resident(experts_w2_kernel<false>, kRingSmem, 3);
+// (which: 0 gate/up, 1 down).  Also sets the kernels' shared-memory limits.
+int experts_resident_ctas(int which, int H, bool small) {
+    if (which == 1) return resident(experts_w2_kernel, kSmem2, 6);
+    const int mode = H <= kDoubleMaxK ? 0 : H <= kWholeMaxK ? 1 : 2;
+    switch (mode * 2 + (small ? 1 : 0)) {
+        case 0: return resident(experts_w13_kernel<0, false>, kSmem13[0], 0);
+        case 1: return resident(experts_w13_kernel<0, true>, kSmem13[0], 1);
+        case 2: return resident(experts_w13_kernel<1, false>, kSmem13[1], 2);
+        case 3: return resident(experts_w13_kernel<1, true>, kSmem13[1], 3);
+        case 4: return resident(experts_w13_kernel<2, false>, kSmem13[2], 4);
+        default: return resident(experts_w13_kernel<2, true>, kSmem13[2], 5);
+    }
 }
 
 cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
-    if (p.H <= kWholeMaxK) return launch_pdl(experts_w13_kernel<true>, dim3(grid), dim3(256), kWholeSmem, stream, p);
-    return launch_pdl(experts_w13_kernel<false>, dim3(grid), dim3(256), kRingSmem, stream, p);
+    const bool small = p.decode_groups > 0;
+    const int mode = p.H <= kDoubleMaxK ? 0 : p.H <= kWholeMaxK ? 1 : 2;
+    const dim3 g(grid), b(256);
+    switch (mode * 2 + (small ? 1 : 0)) {
+        case 0: return launch_pdl(experts_w13_kernel<0, false>, g, b, kSmem13[0], stream, p);
+        case 1: return launch_pdl(experts_w13_kernel<0, true>, g, b, kSmem13[0], stream, p);
+        case 2: return launch_pdl(experts_w13_kernel<1, false>, g, b, kSmem13[1], stream, p);
+        case 3: return launch_pdl(experts_w13_kernel<1, true>, g, b, kSmem13[1], stream, p);
+        case 4: return launch_pdl(experts_w13_kernel<2, false>, g, b, kSmem13[2], stream, p);
+        default: return launch_pdl(experts_w13_kernel<2, true>, g, b, kSmem13[2], stream, p);
+    }
 }
 
 cudaError_t launch_experts_w2(const Params& p, int grid, cudaStream_t stream) {
-    if (max(p.I, p.Is) <= kWholeMaxK)
-        return launch_pdl(experts_w2_kernel<true>, dim3(grid), dim3(256), kWholeSmem, stream, p);
-    return launch_pdl(experts_w2_kernel<false>, dim3(grid), dim3(256), kRingSmem, stream, p);
+    return launch_pdl(experts_w2_kernel, dim3(grid), dim3(256), kSmem2, stream, p);
 }
 
 }  // namespace moe

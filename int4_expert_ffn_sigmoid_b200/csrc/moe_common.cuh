@@ -11,14 +11,23 @@ namespace moe {
 
 // Largest T that takes the weight-streaming (small-batch) path by default.
 constexpr int kDecodeMaxTokens = 64;
-// Tokens of one bucket handled by one expert-kernel task (2 mma n-tiles of 8).
+// Tokens of one bucket handled by one weight-streaming task: each token
+// takes two int8 columns (its two activation parts), so 16 tokens fill four
+// mma n-tiles of 8 columns.
 constexpr int kChunkTokens = 16;
+// Reduction slice of the weight-streaming down projection: its activations
+// are quantized per (token, slice) and every slice writes its own partial
+// output row, summed by the combine.
+constexpr int kSliceK = 512;
 // Large-batch router: tokens per tile and the cap on router CTAs.
 constexpr int kRouterTileTokens = 32;
 constexpr int kRouterMaxBlocks = 296;
-// Small-batch router: tokens and experts per CTA (one warp per expert).
+// Small-batch router: a cluster of kDecodeRouterCtas CTAs per group of
+// kDecodeRouterTok tokens; CTA r of the cluster computes the logits of the
+// r-th eighth of the experts.
 constexpr int kDecodeRouterTok = 8;
-constexpr int kDecodeRouterExp = 8;
+constexpr int kDecodeRouterCtas = 8;
+constexpr int kDecodeGroups = (64 + kDecodeRouterTok - 1) / kDecodeRouterTok;
 constexpr int kMaxK = 8;
 constexpr int kMaxE = 256;
 // The SwiGLU intermediate h of token t is stored in fp16 as h * 2^-k_t, with
@@ -117,7 +126,6 @@ struct Params {
     Ctrl* ctrl;
     int32_t* idx;         // [T*K] selected experts
     float* wts;           // [T*K] routing weights
-    float* logits;        // [T*E] (small-batch router)
     int32_t* counts;      // [E]
     int32_t* offsets;     // [E]   first slot of each expert's bucket
     int32_t* bucket_e;    // [E+1]
@@ -134,8 +142,18 @@ struct Params {
     __half* h_r;          // [T*K][I]  routed SwiGLU intermediate
     __half* h_s;          // [T][Is]   shared SwiGLU intermediate
     int32_t* hexp;        // [T] per-token exponent k_t of the h storage scale
-    float* y;             // [T*K + T][H] expert outputs (already row-scaled)
+    float* y;             // expert outputs (already row-scaled): [nsl_r][T*K][H] then [nsl_s][T][H]
     int router_blocks;
+    // weight-streaming (int8 mma) path
+    int8_t* xq;           // [T][2][H] two-part int8 activations (see quant2), or null
+    float* xs;            // [T] part-0 scale of xq (part 1: xs / 256); NaN for a non-finite row
+    int32_t* rank;        // [T*K] small-batch router: rank of (t, k) among its token group's picks of the expert
+    float* h32_r;         // [T*K][I]  routed SwiGLU intermediate (f32)
+    float* h32_s;         // [T][Is]   shared SwiGLU intermediate (f32)
+    float* hmax_r;        // [T*K][I/64] max |h| of each 64-row block
+    float* hmax_s;        // [T][Is/64]
+    int nsl_r, nsl_s;     // slices of the down projection's reduction (routed, shared)
+    int decode_groups;    // token groups of the small-batch router (0: tables come from the large router)
 };
 
 // ---------------------------------------------------------------------------
@@ -205,6 +223,89 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
 }
 
 // Bucket geometry of the expert kernels.
-__device__ __forceinline__ int chunks_of(int n) { return (n + kChunkTokens - 1) / kChunkTokens; }
+__device__ __host__ __forceinline__ int chunks_of(int n) { return (n + kChunkTokens - 1) / kChunkTokens; }
+__device__ __host__ __forceinline__ int slices_of(int k) { return (k + kSliceK - 1) / kSliceK; }
+
+// ---------------------------------------------------------------------------
+// int8 operands of the weight-streaming kernels.
+//
+// Weights: the int4 code c (two's complement nibble) becomes the int8 value
+// 16*c by moving the nibble to the high half of a byte: for a 32-bit word of
+// eight codes (element 2j in the low nibble of byte j, 2j+1 in the high one),
+//   lo8(w) = (w << 4) & 0xF0F0F0F0  -> byte j = 16 * c[2j]
+//   hi8(w) =  w       & 0xF0F0F0F0  -> byte j = 16 * c[2j+1]
+// (three logic operations per eight weights; exact).
+//
+// Activations: a row v (a token's x, or a slice of its SwiGLU intermediate)
+// is written as v ~= s * (q0 + q1 / 256) with int8 q0, q1 in [-127, 127] and a
+// power of two s chosen from max|v| so that |v| / s <= 127: q0 = rint(v / s),
+// then q1 = rint(256 (v - s q0) / s), the residual being exact.  The error is
+// at most s / 512 per element (max|v| / 2^15 at worst, usually less), and
+// the products with the 16*c weights accumulate exactly in int32.  Within
+// every group of eight consecutive elements the bytes are stored in the order
+// (0, 2, 4, 6, 1, 3, 5, 7), matching lo8 / hi8 of the weights, so that one
+// 8-byte read holds the two mma k-halves of one weight word.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t lo8(uint32_t w) { return (w << 4) & 0xF0F0F0F0u; }
+__device__ __forceinline__ uint32_t hi8(uint32_t w) { return w & 0xF0F0F0F0u; }
+
+// max that keeps a NaN once it has seen one
+__device__ __forceinline__ float nanmax(float m, float a) { return (a > m || a != a) ? a : m; }
+
+struct QScale {
+    float s, inv, inv256;  // s = 2^e; NaN s marks a non-finite row (its q are 0)
+};
+
+// Scale of a row whose largest magnitude is amax.  Magnitudes below 2^-113
+// (e clamped at -119) quantize to zero.
+__device__ __forceinline__ QScale qscale(float amax) {
+    QScale r;
+    if (!(amax <= 3.402823466e38f)) {  // NaN or infinite
+        r.s = __int_as_float(0x7fc00000);
+        r.inv = r.inv256 = 0.f;
+        return r;
+    }
+    int e = 0;
+    if (amax > 0.f) {
+        e = ilogbf(amax) - 6;  // amax / 2^e in [64, 128)
+        if (amax > 127.f * __int_as_float((min(max(e, -126), 127) + 127) << 23)) ++e;
+        e = min(max(e, -119), 126);
+    }
+    r.s = __int_as_float((e + 127) << 23);
+    r.inv = __int_as_float((127 - e) << 23);
+    r.inv256 = __int_as_float((135 - e) << 23);
+    return r;
+}
+
+// The two int8 parts of v under scale qs.
+__device__ __forceinline__ void quant2(float v, const QScale& qs, int& q0, int& q1) {
+    const float a = rintf(v * qs.inv);
+    const float r = fmaf(-a, qs.s, v);
+    const float b = fminf(fmaxf(rintf(r * qs.inv256), -127.f), 127.f);
+    q0 = (int)a;
+    q1 = (int)b;
+}
+
+// Eight consecutive elements -> the two 8-byte groups (part 0, part 1) in the
+// (0, 2, 4, 6, 1, 3, 5, 7) byte order.
+__device__ __forceinline__ void quant2x8(const float (&v)[8], const QScale& qs, uint2& p0, uint2& p1) {
+    int a[8], b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) quant2(v[i], qs, a[i], b[i]);
+    auto pack = [](int e0, int e1, int e2, int e3) {
+        return (uint32_t)(e0 & 0xff) | ((uint32_t)(e1 & 0xff) << 8) | ((uint32_t)(e2 & 0xff) << 16) |
+               ((uint32_t)(e3 & 0xff) << 24);
+    };
+    p0 = make_uint2(pack(a[0], a[2], a[4], a[6]), pack(a[1], a[3], a[5], a[7]));
+    p1 = make_uint2(pack(b[0], b[2], b[4], b[6]), pack(b[1], b[3], b[5], b[7]));
+}
+
+// D(16x8, s32) += A(16x32, s8) * B(32x8, s8), A row-major, B column-major.
+__device__ __forceinline__ void mma_s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 
 }  // namespace moe

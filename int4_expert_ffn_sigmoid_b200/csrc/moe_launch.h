@@ -13,10 +13,11 @@ cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream)
 cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream);
 // Expert down projection (weight-streaming mma.sync kernel).
 cudaError_t launch_experts_w2(const Params& p, int grid, cudaStream_t stream);
-// CTAs of the weight-streaming kernel `which` (0: gate/up, 1: down; kdim: its
-// longest reduction range) that fit on the device at once (the persistent
-// grid size).  Also sets the kernel's shared-memory attribute.
-int experts_resident_ctas(int which, int kdim);
+// CTAs of the weight-streaming kernel `which` (0: gate/up, 1: down) that fit
+// on the device at once (the persistent grid size) for hidden size H, with
+// the small-batch (small) or large-batch bucket tables.  Also sets the
+// kernel's shared-memory attribute.
+int experts_resident_ctas(int which, int H, bool small);
 // Weighted combine + shared expert (+ residual) -> bf16 out.
 cudaError_t launch_combine(const Params& p, cudaStream_t stream);
 

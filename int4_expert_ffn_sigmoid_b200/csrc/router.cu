@@ -8,11 +8,15 @@
 // batch-union MoE: every expert touched by the batch is read once for all of
 // its tokens).
 //
-// Every logit is computed with one fixed arithmetic order whatever the batch
-// size: lane l of a warp accumulates, with fused multiply-adds, the elements
-// 128*i + 4*l + j (i ascending, then j = 0..3), and the 32 lane partials are
-// summed by an xor-butterfly (16, 8, 4, 2, 1).  A token therefore gets the
-// same bits from the small-batch and the large-batch router.
+// Each router computes a logit with one fixed arithmetic order that does not
+// depend on the other tokens of the batch, so a token gets the same routing
+// whatever it is batched with (within one path).  The small-batch router
+// accumulates, in lane l of a warp, the elements 128*i + 4*l + j (i ascending,
+// then j = 0..3) with fused multiply-adds and sums the 32 lane partials by an
+// xor-butterfly (16, 8, 4, 2, 1); the large-batch router is described above
+// router_large_kernel.
+#include <cooperative_groups.h>
+
 #include "moe_common.cuh"
 #include "moe_launch.h"
 
@@ -71,12 +75,13 @@ __device__ __forceinline__ void token_hexp(const Params& p, int t, int lane) {
     store_hexp(p, t, acc, lane);
 }
 
-// Top-K of one token (one warp).  Lane l holds experts l, l+32, ...  The key
-// is sigmoid(L) + bias (NaN -> -inf); ties go to the lower expert index.  The
-// weight of the k-th pick is scale * s_k / (s_0 + ... + s_{K-1}).
-// Returns, on lanes k < K, the k-th selected expert (else -1).
-template <bool kGlobalLogits>
-__device__ int select_token(const Params& p, int t, const float* lg, int lane) {
+// Top-K of one token (one warp).  Lane l holds the logits L[j] of experts
+// l + 32 j (entries of experts >= E are ignored).  The key is sigmoid(L) +
+// bias (NaN -> -inf); ties go to the lower expert index.  The weight of the
+// k-th pick is scale * s_k / (s_0 + ... + s_{K-1}).  Writes idx / wts (and
+// the optional user outputs) of token t; returns, on lanes k < K, the k-th
+// selected expert (else -1).
+__device__ int select_from_logits(const Params& p, int t, const float (&L)[kMaxE / 32], const float* bias, int lane) {
     const int E = p.E, K = p.K;
     float key[kMaxE / 32], sc[kMaxE / 32];
 #pragma unroll
@@ -85,9 +90,8 @@ __device__ int select_token(const Params& p, int t, const float* lg, int lane) {
         key[j] = -INFINITY;
         sc[j] = 0.f;
         if (e < E) {
-            const float L = kGlobalLogits ? __ldcg(lg + e) : lg[e];
-            const float s = 1.0f / (1.0f + expf(-L));
-            const float kk = s + __ldg(p.rb + e);
+            const float s = 1.0f / (1.0f + expf(-L[j]));
+            const float kk = s + bias[e];
             key[j] = isnan(kk) ? -INFINITY : kk;
             sc[j] = s;
         }
@@ -127,6 +131,51 @@ __device__ int select_token(const Params& p, int t, const float* lg, int lane) {
         if (p.topk_w_out) p.topk_w_out[o] = w;
     }
     return lane < K ? my_e : -1;
+}
+
+// select_from_logits with the token's logits in shared memory.
+__device__ int select_token(const Params& p, int t, const float* lg, int lane) {
+    float L[kMaxE / 32];
+#pragma unroll
+    for (int j = 0; j < kMaxE / 32; ++j) {
+        const int e = lane + 32 * j;
+        L[j] = e < p.E ? lg[e] : 0.f;
+    }
+    return select_from_logits(p, t, L, p.rb, lane);
+}
+
+// Writes xq (both int8 parts, see quant2) and xs of token t (one warp) from
+// its bf16 row xrow (global or shared memory).
+__device__ void quantize_x_row(const Params& p, int t, const __nv_bfloat16* xrow, int lane) {
+    const uint4* xr = reinterpret_cast<const uint4*>(xrow);
+    const int ng = p.H / 8;
+    float m = 0.f;
+    for (int gi = lane; gi < ng; gi += 32) {
+        const uint4 v = xr[gi];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m = nanmax(nanmax(m, fabsf(bf16lo(w[i]))), fabsf(bf16hi(w[i])));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = nanmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const QScale qs = qscale(m);
+    uint2* q0 = reinterpret_cast<uint2*>(p.xq + (size_t)t * 2 * p.H);
+    uint2* q1 = reinterpret_cast<uint2*>(p.xq + (size_t)t * 2 * p.H + p.H);
+    for (int gi = lane; gi < ng; gi += 32) {
+        const uint4 v = xr[gi];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float f[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = bf16lo(w[i]);
+            f[2 * i + 1] = bf16hi(w[i]);
+        }
+        uint2 a, b;
+        quant2x8(f, qs, a, b);
+        q0[gi] = a;
+        q1[gi] = b;
+    }
+    if (lane == 0) p.xs[t] = qs.s;
 }
 
 // Bucket list and task prefixes from the per-expert slot counts (one CTA of
@@ -195,8 +244,8 @@ __device__ void finalize_buckets(const Params& p, const int* s_cnt, int* s_off) 
                 const int irow = (e == E) ? p.Is : p.I;
                 const int n = p.bucket_n[b];
                 const int ch = chunks_of(n);
-                n13 = (irow / 64) * ch;   // CTA tasks: 64 gate/up rows x 64 tokens
-                n2 = (p.H / 128) * ch;    // CTA tasks: 128 down rows x 64 tokens
+                n13 = (irow / 64) * ch;                    // tasks: 64 gate/up rows x a token chunk
+                n2 = (p.H / 128) * ch * slices_of(irow);   // tasks: 128 down rows x a chunk x a slice
                 if (e != E) {  // tensor-core tiles: 128 tokens x 128 features / 256 columns
                     const int mt = (n + 127) / 128;
                     nt1 = mt * (p.I / 128);
@@ -249,33 +298,93 @@ __device__ __forceinline__ void reset_ctrl(const Params& p) {
 }
 
 // ---------------------------------------------------------------------------
-// Small batch (T <= kDecodeMaxTokens), two kernels.
-// router_logits_kernel: grid (ceil(T/8), ceil(E/8)); warp w of CTA (bx, by)
-// computes the logits of expert 8*by + w for tokens 8*bx ... 8*bx + 7 (warp 0
-// of the first expert column also the tokens' h-scale exponents).
-// router_select_kernel: one CTA selects every token (one warp per token),
-// counts, scans and scatters.
+// Small batch (T <= kDecodeMaxTokens): one kernel, a cluster of
+// kDecodeRouterCtas CTAs per group of kDecodeRouterTok tokens (grid
+// (groups, kDecodeRouterCtas)).  CTA r computes the logits of the experts
+// [r*epc, (r+1)*epc), epc = ceil(E / kDecodeRouterCtas), for the group's
+// tokens into its shared memory (the group's activations are staged there
+// with one round of cp.async); after a cluster barrier CTA 0 reads every
+// token's logits through distributed shared memory, selects (one warp per
+// token), and writes the group's per-expert pick counts (hist[group][e]) and
+// the rank of every pick among the group's picks of the same expert, in
+// (token, k) order.  The other CTAs quantize the group's activations (xq,
+// xs) from their shared copy.  The expert kernels derive the buckets and slots from hist, idx and
+// rank themselves: the slot of pick (t, k) of expert e is offset[e] + (picks
+// of e in earlier groups) + rank, i.e. buckets list their tokens in (t, k)
+// order.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) router_logits_kernel(Params p) {
+// The group's activations are staged in shared memory up to this hidden size.
+constexpr int kRouterXMaxH = 2048;
+
+__global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(256) router_decode_kernel(Params p) {
+    namespace cg = cooperative_groups;
+    constexpr int kEpcMax = kMaxE / kDecodeRouterCtas;
+    __shared__ __align__(16) __nv_bfloat16 s_x[kDecodeRouterTok][kRouterXMaxH];
+    __shared__ float s_logit[kDecodeRouterTok][kEpcMax];
+    __shared__ float s_bias[kMaxE];
+    __shared__ int s_pick[kDecodeRouterTok * kMaxK];
+    cg::cluster_group cluster = cg::this_cluster();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int r = blockIdx.y;  // rank in the cluster
     const int t0 = blockIdx.x * kDecodeRouterTok;
-    const int e = blockIdx.y * kDecodeRouterExp + warp;
     const int nt = min(kDecodeRouterTok, p.T - t0);
-    if (e < p.E) {  // the router weights do not depend on the previous kernel
-        const char* wrow = reinterpret_cast<const char*>(p.rw + (size_t)e * p.H);
-        for (int l = lane; l < p.H * 4 / 128; l += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(wrow + l * 128));
+    const int E = p.E, H = p.H, K = p.K;
+    const int nblk = H / 128;
+    const int epc = (E + kDecodeRouterCtas - 1) / kDecodeRouterCtas;
+    const int e_lo = r * epc, e_hi = min(E, e_lo + epc);
+    const bool staged = H <= kRouterXMaxH;
+    // Nothing below depends on the previous kernel until pdl_wait: the bias,
+    // the first 8 blocks of this warp's first router row (registers) and the
+    // rest of the CTA's rows (L2).
+    if (r == 0)
+        for (int e = threadIdx.x; e < E; e += blockDim.x) s_bias[e] = __ldg(p.rb + e);
+    float4 wpre[8];
+    {
+        const int e = e_lo + warp;
+        const float4* W = reinterpret_cast<const float4*>(p.rw + (size_t)min(e, E - 1) * H);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) wpre[i] = (e < e_hi && i < nblk) ? __ldg(W + i * 32 + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int e = e_lo + warp; e < e_hi; e += 8) {
+        const char* wrow = reinterpret_cast<const char*>(p.rw + (size_t)e * H);
+        for (int l = lane; l < H * 4 / 128; l += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(wrow + l * 128));
     }
     pdl_wait();
     reset_ctrl(p);
     pdl_release();
-    const bool do_sq = blockIdx.y == 0 && warp == 0;
-    if (e < p.E) {
-        float acc[kDecodeRouterTok], sq[kDecodeRouterTok];
+    if (staged) {
+        const int per = H / 8;  // 16-byte chunks per row
+        for (int c = threadIdx.x; c < nt * per; c += blockDim.x) {
+            const int tt = c / per, k = c - tt * per;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(
+                             __cvta_generic_to_shared(&s_x[tt][k * 8]))),
+                         "l"(p.x + (size_t)(t0 + tt) * H + k * 8)
+                         : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();
+    }
+    auto xblock = [&](int tt, int i) -> uint2 {
+        if (tt >= nt) return make_uint2(0u, 0u);
+        if (staged) return *reinterpret_cast<const uint2*>(&s_x[tt][i * 128 + lane * 4]);
+        return __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)(t0 + tt) * H + i * 128 + lane * 4));
+    };
+    for (int e = e_lo + warp, j = 0; e < e_hi; e += 8, ++j) {
+        float acc[kDecodeRouterTok];
 #pragma unroll
-        for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = sq[tt] = 0.f;
-        const float4* W = reinterpret_cast<const float4*>(p.rw + (size_t)e * p.H);
-        const int nblk = p.H / 128;  // processed 4 blocks per batch of loads
-        for (int i0 = 0; i0 < nblk; i0 += 4) {
+        for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = 0.f;
+        const float4* W = reinterpret_cast<const float4*>(p.rw + (size_t)e * H);
+        int i_first = 0;
+        if (j == 0) {  // the prefetched blocks
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (i < nblk)
+#pragma unroll
+                    for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = dot_step(acc[tt], xblock(tt, i), wpre[i]);
+            i_first = 8;
+        }
+        for (int i0 = i_first; i0 < nblk; i0 += 4) {
             float4 wv[4];
             uint2 xv[4][kDecodeRouterTok];
 #pragma unroll
@@ -283,67 +392,56 @@ __global__ void __launch_bounds__(256) router_logits_kernel(Params p) {
                 const int i = i0 + u;
                 wv[u] = i < nblk ? __ldg(W + i * 32 + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int tt = 0; tt < kDecodeRouterTok; ++tt)
-                    xv[u][tt] = (i < nblk && tt < nt)
-                                    ? __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)(t0 + tt) * p.H + i * 128 + lane * 4))
-                                    : make_uint2(0u, 0u);
+                for (int tt = 0; tt < kDecodeRouterTok; ++tt) xv[u][tt] = i < nblk ? xblock(tt, i) : make_uint2(0u, 0u);
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (i0 + u < nblk) {
+            for (int u = 0; u < 4; ++u)
+                if (i0 + u < nblk)
 #pragma unroll
-                    for (int tt = 0; tt < kDecodeRouterTok; ++tt) {
-                        acc[tt] = dot_step(acc[tt], xv[u][tt], wv[u]);
-                        if (do_sq) sq[tt] = sq_step(sq[tt], xv[u][tt]);
-                    }
-                }
-            }
+                    for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = dot_step(acc[tt], xv[u][tt], wv[u]);
         }
 #pragma unroll
         for (int tt = 0; tt < kDecodeRouterTok; ++tt) {
             const float v = warp_sum_tree(acc[tt]);
-            if (lane == 0 && tt < nt) p.logits[(size_t)(t0 + tt) * p.E + e] = v;
-            if (do_sq && tt < nt) store_hexp(p, t0 + tt, sq[tt], lane);
+            if (lane == 0) s_logit[tt][e - e_lo] = v;
         }
     }
-}
-
-__global__ void __launch_bounds__(1024) router_select_kernel(Params p) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    __shared__ int s_idx[kDecodeMaxTokens * kMaxK];
-    __shared__ int s_cnt[kMaxE];
-    __shared__ int s_off[kMaxE];
-    pdl_wait();
-    pdl_release();
-    for (int i = threadIdx.x; i < p.E; i += blockDim.x) s_cnt[i] = 0;
-    __syncthreads();
-    for (int t = warp; t < p.T; t += blockDim.x / 32) {
-        int sel = select_token<true>(p, t, p.logits + (size_t)t * p.E, lane);
-        if (lane < p.K) {
-            if (sel < 0 || sel >= p.E) {
-                atomicOr(&p.ctrl->status, ST_BAD_EXPERT);
-                sel = 0;
+    cluster.sync();  // every logit of the group is in some CTA's shared memory
+    if (r == 0) {
+        if (warp < nt) {
+            float L[kMaxE / 32];
+#pragma unroll
+            for (int jj = 0; jj < kMaxE / 32; ++jj) {
+                const int e = lane + 32 * jj;
+                L[jj] = 0.f;
+                if (e < E) {
+                    const int src = e / epc;
+                    L[jj] = *cluster.map_shared_rank(&s_logit[warp][e - src * epc], src);
+                }
             }
-            s_idx[t * p.K + lane] = sel;
-            atomicAdd(&s_cnt[sel], 1);
+            const int sel = select_from_logits(p, t0 + warp, L, s_bias, lane);
+            if (lane < K) s_pick[warp * K + lane] = sel;
         }
-    }
-    __syncthreads();
-    finalize_buckets(p, s_cnt, s_off);
-    const int TK = p.T * p.K;
-    for (int i = threadIdx.x; i < TK; i += blockDim.x) {
-        const int ex = s_idx[i];
-        int rank = 0;
-        for (int j = 0; j < i; ++j) rank += (s_idx[j] == ex);
-        const int slot = s_off[ex] + rank;
-        if (slot < 0 || slot >= TK) {
-            atomicOr(&p.ctrl->status, ST_BAD_SLOT);
-            p.slot_of[i] = 0;
-            continue;
+        __syncthreads();
+        const int n = nt * K;
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            const int e = s_pick[i];
+            int rk = 0;
+            for (int jj = 0; jj < i; ++jj) rk += (s_pick[jj] == e);
+            p.rank[(size_t)t0 * K + i] = rk;
         }
-        p.slot_of[i] = slot;
-        p.tok_of_slot[slot] = i / p.K;
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            int c = 0;
+            for (int jj = 0; jj < n; ++jj) c += (s_pick[jj] == e);
+            p.hist[(size_t)blockIdx.x * E + e] = c;
+        }
+    } else {
+        // token tt of the group is quantized by CTA max(tt, 1), warp (tt == 0)
+        for (int tt = 0; tt < nt; ++tt)
+            if (r == max(tt, 1) && warp == (tt == 0 ? 1 : 0))
+                quantize_x_row(p, t0 + tt, staged ? &s_x[tt][0] : p.x + (size_t)(t0 + tt) * H, lane);
     }
+    cluster.sync();  // the remote reads of CTA 0 are done before any CTA exits
 }
 
 // ---------------------------------------------------------------------------
@@ -352,8 +450,9 @@ __global__ void __launch_bounds__(1024) router_select_kernel(Params p) {
 // block, block + grid, ...); each tile's logits stay in shared memory, one
 // warp per token selects, and every CTA records its per-expert slot counts.
 // router_finalize_kernel: one CTA sums the counts, scans and builds the
-// bucket and task lists.  scatter_large_kernel: slots (and, for the
-// tensor-core path, the gathered activation rows).
+// bucket and task lists.  scatter_large_kernel: slots, and the gathered
+// activation rows of the tensor-core path or the int8 activations of the
+// weight-streaming kernels.
 // ---------------------------------------------------------------------------
 // Tensor-core router logits for a tile of kRouterTileTokens tokens and every
 // expert.  x is exactly bf16; each f32 router weight w is split exactly into
@@ -500,7 +599,7 @@ __global__ void __launch_bounds__(256) router_large_kernel(Params p) {
         }
         __syncthreads();
         for (int tt = warp; tt < nt; tt += 8) {
-            const int sel = select_token<false>(p, t0 + tt, s_logit[tt], lane);
+            const int sel = select_token(p, t0 + tt, s_logit[tt], lane);
             // an index outside [0, E) cannot occur; it is counted nowhere and
             // reported by the scatter kernel's range check
             if (lane < p.K && sel >= 0 && sel < E) atomicAdd(&s_cnt[sel], 1);
@@ -591,6 +690,11 @@ __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
                 for (int c = lane; c < p.H / 8; c += 32) dst[c] = __ldg(src + c);
             }
         }
+        if (p.xq) {  // int8 activations of the weight-streaming kernels (one warp per token)
+            const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+            for (int tt = warp; tt < n / K; tt += blockDim.x / 32)
+                quantize_x_row(p, t0 + tt, p.x + (size_t)(t0 + tt) * p.H, lane);
+        }
         for (int e = threadIdx.x; e < E; e += blockDim.x) {
             int c = 0;
             for (int j = 0; j < n; ++j) c += (s_idx[j] == e);
@@ -602,12 +706,8 @@ __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
 
 cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream) {
     cudaError_t err;
-    if (small_path) {
-        dim3 grid((p.T + kDecodeRouterTok - 1) / kDecodeRouterTok, (p.E + kDecodeRouterExp - 1) / kDecodeRouterExp);
-        err = launch_pdl(router_logits_kernel, grid, dim3(256), 0, stream, p);
-        if (err == cudaSuccess) err = launch_pdl(router_select_kernel, dim3(1), dim3(1024), 0, stream, p);
-        return err;
-    }
+    if (small_path)
+        return launch_pdl(router_decode_kernel, dim3(p.decode_groups, kDecodeRouterCtas), dim3(256), 0, stream, p);
     err = launch_pdl(router_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
     if (err == cudaSuccess) err = launch_pdl(router_finalize_kernel, dim3(1), dim3(1024), 0, stream, p);
     if (err == cudaSuccess) err = launch_pdl(scatter_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
