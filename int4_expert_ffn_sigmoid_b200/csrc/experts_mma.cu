@@ -55,8 +55,8 @@ namespace moe {
 
 namespace {
 
-constexpr int kRows13 = 64;   // gate (and up) rows per gate/up task
-constexpr int kRows2 = 128;   // down rows per down task
+constexpr int kRows13 = kTaskRows13;  // gate (and up) rows per gate/up task
+constexpr int kRows2 = kTaskRows2;    // down rows per down task
 constexpr int kRing = 4;      // weight k blocks in flight per thread
 constexpr int kXRing = 4;     // staged activation slices (ring mode)
 constexpr int kPadB = 16;     // bytes of padding per staged row
@@ -88,9 +88,16 @@ struct Tables {
 };
 
 // Per-CTA shared state, ahead of the staging areas.
+// One task of the CTA's task sequence, decoded once (see precompute_tasks).
+struct TaskDesc {
+    int e, off, rbk, sl, tok0, nc;  // e < 0: no task
+};
+constexpr int kMaxCtaTasks = 32;
+
 struct Shm {
     Tables tb;
-    int tok[kMaxSlots];                           // small-batch path: token of each routed slot
+    TaskDesc td[kMaxCtaTasks];                    // the first tasks of this CTA, in its order
+    int tok[kMaxSlots];                           // token of each routed slot (T*K <= kMaxSlots)
     float xsr[2][kChunkTokens];                   // gate/up: activation scale of each token (per buffer)
     float hmr[kChunkTokens][kSliceK / kRows13];   // down: the slice's per-64-row maxima of |h|
     float xsc[kChunkTokens];                      // down: activation scale / 16 of each token
@@ -98,23 +105,26 @@ struct Shm {
     float hm[8][kChunkTokens];                    // gate/up: per-warp max |h| of each token
 };
 constexpr size_t kShmBytes = (sizeof(Shm) + 127) & ~size_t(127);
+
+// gate/up staging modes: 0 two whole-row buffers, 1 one whole-row buffer, 2 ring of slices
 // scratch of the small-batch table build, in the staging area
 constexpr size_t kBuildBytes = (size_t)(kDecodeGroups + 2) * kMaxE * 4;
-
-constexpr size_t max_sz(size_t a, size_t b) { return a > b ? a : b; }
-// gate/up staging modes: 0 two whole-row buffers, 1 one whole-row buffer, 2 ring of slices
-constexpr size_t kSmem13[3] = {
-    kShmBytes + max_sz(kBuildBytes, (size_t)2 * kStageRows * (kDoubleMaxK + kPadB)),
-    kShmBytes + max_sz(kBuildBytes, (size_t)kStageRows * (kWholeMaxK + kPadB)),
-    kShmBytes + max_sz(kBuildBytes, (size_t)kStageRows * (kXRing * 128 + kPadB))};
+static_assert(kBuildBytes <= (size_t)kStageRows * (kXRing * 128 + kPadB), "table build scratch fits the staging area");
+constexpr size_t kSmem13[3] = {kShmBytes + (size_t)2 * kStageRows * (kDoubleMaxK + kPadB),
+                               kShmBytes + (size_t)kStageRows * (kWholeMaxK + kPadB),
+                               kShmBytes + (size_t)kStageRows * (kXRing * 128 + kPadB)};
 // down: int8 staging of one slice + the next task's f32 slice
 constexpr int kStride2 = kSliceK + kPadB;
 constexpr size_t kRaw2Off = (size_t)kStageRows * kStride2;
 constexpr size_t kSmem2 = kShmBytes + kRaw2Off + (size_t)kChunkTokens * kSliceK * 4;
 
-// Tables written to the workspace (by the large router, or by CTA 0 of the
-// small-batch gate/up kernel for the down kernel).
-__device__ __forceinline__ void load_tables(const Params& p, const int32_t* ts, const int* ntask, Tables& tb) {
+// The bucket list and task prefix that the router wrote to the workspace,
+// and (for at most kMaxSlots routed slots) the token of every slot.
+__device__ __forceinline__ void load_tables(const Params& p, const int32_t* ts, const int* ntask, Tables& tb,
+                                            int* tok) {
+    const int TK = p.T * p.K;
+    if (tok && TK <= kMaxSlots)
+        for (int i = threadIdx.x; i < TK; i += blockDim.x) tok[i] = __ldcg(p.tok_of_slot + i);
     const int nb = __ldcg(&p.ctrl->n_buckets);
     for (int i = threadIdx.x; i <= nb && i < kTab; i += blockDim.x) {
         tb.ts[i] = __ldcg(ts + i);
@@ -171,7 +181,7 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
         // lane l owns experts 8l .. 8l+7: counts, non-empty buckets, gate/up
         // and down tasks, scanned across the warp in one pass
         constexpr int kPer = kMaxE / 32;
-        const int R13 = p.I / kRows13, R2 = (p.H / kRows2) * slices_of(p.I);
+        const int R13 = p.I / kTaskRows13, R2 = (p.H / kTaskRows2) * slices_of(p.I);
         int c[kPer];
         int v[4] = {0, 0, 0, 0};  // slots, buckets, gate/up tasks, down tasks
 #pragma unroll
@@ -235,8 +245,8 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
                     p.bucket_off[nb] = TK;
                     p.ts2[nb] = t2;
                 }
-                t13 += (p.Is / kRows13) * chunks_of(T);
-                t2 += (p.H / kRows2) * slices_of(p.Is) * chunks_of(T);
+                t13 += (p.Is / kTaskRows13) * chunks_of(T);
+                t2 += (p.H / kTaskRows2) * slices_of(p.Is) * chunks_of(T);
                 ++nb;
             }
             tb.ts[nb] = t13;
@@ -270,6 +280,7 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
     __syncthreads();
 }
 
+
 __device__ __forceinline__ int find_bucket(const Tables& tb, int task) {
     int lo = 0, hi = tb.n_buckets;  // ts[lo] <= task < ts[hi]
     while (hi - lo > 1) {
@@ -279,11 +290,11 @@ __device__ __forceinline__ int find_bucket(const Tables& tb, int task) {
     return lo;
 }
 
-// Token of slot s of a bucket starting at slot `off`.
-template <bool kSmall>
+// Token of slot s of a bucket starting at slot `off` (from shared memory
+// when load_tables copied the slot tokens there).
 __device__ __forceinline__ int slot_token(const Params& p, const Shm& sh, bool shared, int off, int s) {
     if (shared) return s;
-    if (kSmall) return off + s < kMaxSlots ? sh.tok[off + s] : -1;
+    if (p.T * p.K <= kMaxSlots) return off + s < kMaxSlots ? sh.tok[off + s] : -1;
     return __ldcg(p.tok_of_slot + off + s);
 }
 
@@ -431,31 +442,94 @@ __device__ __forceinline__ Task13 make13(const Params& p, int e, int n, int off,
     return t;
 }
 
-__device__ __forceinline__ Task13 task13_at(const Params& p, const Tables& tb, int lin) {
-    if (lin >= tb.ntask) {
-        Task13 t{};
-        return t;
-    }
+// The r-th task of CTA c in snake order over the heaviest-first task list:
+// even rounds go up the CTAs, odd rounds come back down, so that a CTA whose
+// first task was one of the heaviest gets one of the lightest next.
+__device__ __forceinline__ int snake(int c, int r) {
+    return (r & 1) ? (r + 1) * (int)gridDim.x - 1 - c : r * (int)gridDim.x + c;
+}
+
+// Task `lin` of the heaviest-first list: its bucket and coordinates.  kind
+// 0: gate/up (rows, chunk), 1: down (rows, slice, chunk).
+__device__ __forceinline__ TaskDesc decode_task(const Params& p, const Tables& tb, int kind, int lin) {
+    TaskDesc d;
+    d.e = -1;
+    d.off = d.rbk = d.sl = d.tok0 = d.nc = 0;
+    if (lin >= tb.ntask) return d;
     const int task = tb.ntask - 1 - lin;
     const int b = find_bucket(tb, task);
-    return make13(p, tb.e[b], tb.n[b], tb.off[b], task - tb.ts[b]);
+    const int e = tb.e[b], n = tb.n[b], local = task - tb.ts[b];
+    const int irow = e == p.E ? p.Is : p.I;
+    int c;
+    if (kind == 0) {
+        const int R = irow / kRows13;
+        c = local / R;
+        d.rbk = local - c * R;
+    } else {
+        const int R = p.H / kRows2, nsl = slices_of(irow);
+        const int rest = local / R;
+        d.rbk = local - rest * R;
+        c = rest / nsl;
+        d.sl = rest - c * nsl;
+    }
+    d.e = e;
+    d.off = tb.off[b];
+    d.tok0 = c * kChunkTokens;
+    d.nc = min(kChunkTokens, n - d.tok0);
+    return d;
+}
+
+// Decodes the CTA's first kMaxCtaTasks tasks (in snake order) into shared
+// memory, so that the task loop does not repeat the search and divisions.
+__device__ __forceinline__ void precompute_tasks(const Params& p, Shm& sh, int kind) {
+    if (threadIdx.x < kMaxCtaTasks) sh.td[threadIdx.x] = decode_task(p, sh.tb, kind, snake(blockIdx.x, threadIdx.x));
+    __syncthreads();
+}
+
+__device__ __forceinline__ TaskDesc task_desc(const Params& p, const Shm& sh, int kind, int r) {
+    return r < kMaxCtaTasks ? sh.td[r] : decode_task(p, sh.tb, kind, snake(blockIdx.x, r));
+}
+
+// Gate/up task from its descriptor (no task: ok = false).
+__device__ __forceinline__ Task13 task13_from(const Params& p, const TaskDesc& d) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, q = lane & 3;
+    Task13 t{};
+    if (d.e < 0) return t;
+    t.ok = !(d.e > p.E || (d.e == p.E && p.Is == 0));
+    t.shared = d.e == p.E;
+    t.e = d.e;
+    t.off = d.off;
+    t.irow = t.shared ? p.Is : p.I;
+    t.rbk = d.rbk;
+    t.tok0 = d.tok0;
+    t.nc = d.nc;
+    t.r0 = d.rbk * kRows13 + warp * 8;
+    const int row_bytes = p.H / 2;
+    const uint8_t* W = t.shared ? p.sh_w13 : p.w13 + (size_t)(t.ok ? d.e : 0) * 2 * p.I * row_bytes;
+    t.w.ra = W + (size_t)(t.r0 + g) * row_bytes + q * 16;
+    t.w.rb = W + (size_t)(t.irow + t.r0 + g) * row_bytes + q * 16;
+    t.w.nkb = t.ok ? p.H / 128 : 0;
+    return t;
+}
+
+__device__ __forceinline__ Task13 task13_r(const Params& p, const Shm& sh, int r) {
+    return task13_from(p, task_desc(p, sh, 0, r));
 }
 
 // Issues the cp.async of task t's activation rows (both parts of each token)
 // into `buf` and of its tokens' activation scales into xsr, as one group.
-template <bool kSmall>
 __device__ __forceinline__ void stage13(const Params& p, const Shm& sh, const Task13& t, uint8_t* buf, int stride,
                                         float* xsr) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int H = p.H;
     for (int r = warp; r < 2 * t.nc; r += 8) {
-        const int tok = slot_token<kSmall>(p, sh, t.shared, t.off, t.tok0 + (r >> 1));
+        const int tok = slot_token(p, sh, t.shared, t.off, t.tok0 + (r >> 1));
         if (tok < 0 || tok >= p.T) continue;
         const int8_t* src = p.xq + (size_t)tok * 2 * H + (r & 1) * H;
         for (int c16 = lane; c16 < H / 16; c16 += 32) cp_async16(buf + r * stride + c16 * 16, src + c16 * 16);
     }
     if (threadIdx.x < t.nc) {
-        const int tok = slot_token<kSmall>(p, sh, t.shared, t.off, t.tok0 + threadIdx.x);
+        const int tok = slot_token(p, sh, t.shared, t.off, t.tok0 + threadIdx.x);
         if (tok >= 0 && tok < p.T) {
             cp_async4(xsr + threadIdx.x, p.xs + tok);
         } else {
@@ -506,7 +580,7 @@ __device__ __forceinline__ bool run13(Ring& ring, const Task13& tk, const WStrea
 
 // kMode: 0 two whole-row staging buffers (the next task's activations load
 // while the current task computes), 1 one whole-row buffer, 2 ring of slices.
-template <int kMode, bool kSmall>
+template <int kMode>
 __global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
     extern __shared__ __align__(128) uint8_t dsm[];
     Shm& sh = *reinterpret_cast<Shm*>(dsm);
@@ -532,30 +606,32 @@ __global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
     if (p.Is > 0) prefetch_l2_slice(p.sh_w13, (size_t)p.Is * p.H);
     pdl_wait();
     pdl_release();
-    if (kSmall) build_tables_small(p, sh, reinterpret_cast<int*>(xs));
-    else load_tables(p, p.ts13, &p.ctrl->tasks13, sh.tb);
+    if (p.decode_groups > 0) build_tables_small(p, sh, reinterpret_cast<int*>(xs));
+    else load_tables(p, p.ts13, &p.ctrl->tasks13, sh.tb, sh.tok);
+    precompute_tasks(p, sh, 0);
     const Tables& tb = sh.tb;
-    Task13 cur = task13_at(p, tb, blockIdx.x);
+    Task13 cur = task13_r(p, sh, 0);
     if (primed && cur.w.ra != primed_ra) primed = false;
-    if (kMode != 2 && cur.ok) stage13<kSmall>(p, sh, cur, xs, stride, sh.xsr[0]);
+    // activations first: they are L2 hits that should not queue behind the weight stream
+    if (kMode != 2 && cur.ok) stage13(p, sh, cur, xs, stride, sh.xsr[0]);
     const float* S = cur.shared ? p.sh_s13 : p.s13 + (size_t)cur.e * 2 * p.I;
     float gs = cur.ok ? __ldg(S + cur.r0 + g) : 0.f, us = cur.ok ? __ldg(S + cur.irow + cur.r0 + g) : 0.f;
     int buf = 0;
-    for (int lin = blockIdx.x; lin < tb.ntask; lin += gridDim.x) {
-        const Task13 nx = task13_at(p, tb, lin + gridDim.x);
+    for (int r = 0, lin = blockIdx.x; lin < tb.ntask; lin = snake(blockIdx.x, ++r)) {
+        const Task13 nx = task13_r(p, sh, r + 1);
         if (!cur.ok) {  // a table entry out of range: flag it and stop
             if (threadIdx.x == 0) atomicOr(&p.ctrl->status, ST_BAD_TASK);
             break;
         }
         if (!primed) prime(ring, cur.w);
         if (kMode == 2 && threadIdx.x < cur.nc) {  // ring mode: the scales only (slices are staged in the loop)
-            const int tok = slot_token<kSmall>(p, sh, cur.shared, cur.off, cur.tok0 + threadIdx.x);
+            const int tok = slot_token(p, sh, cur.shared, cur.off, cur.tok0 + threadIdx.x);
             if (tok >= 0 && tok < p.T) cp_async4(sh.xsr[0] + threadIdx.x, p.xs + tok);
             else sh.xsr[0][threadIdx.x] = 0.f;
         }
         if (kMode != 2) cp_async_wait<0>();
         __syncthreads();  // cur's activations are visible; the previous task is done with every buffer
-        if (kMode == 0 && nx.ok) stage13<kSmall>(p, sh, nx, xs + (buf ^ 1) * bufbytes, stride, sh.xsr[buf ^ 1]);
+        if (kMode == 0 && nx.ok) stage13(p, sh, nx, xs + (buf ^ 1) * bufbytes, stride, sh.xsr[buf ^ 1]);
         float gs_n = 0.f, us_n = 0.f;
         if (nx.ok) {
             const float* Sn = nx.shared ? p.sh_s13 : p.s13 + (size_t)nx.e * 2 * p.I;
@@ -567,7 +643,7 @@ __global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
         auto stage_slice = [&](int kb) {
             const int r = threadIdx.x >> 3, part = threadIdx.x & 7;
             if (r < 2 * nc) {
-                const int tok = slot_token<kSmall>(p, sh, c.shared, c.off, c.tok0 + (r >> 1));
+                const int tok = slot_token(p, sh, c.shared, c.off, c.tok0 + (r >> 1));
                 if (tok >= 0 && tok < p.T)
                     cp_async16(xs + r * stride + (kb % kXRing) * 128 + part * 16,
                                p.xq + (size_t)tok * 2 * H + (r & 1) * H + kb * 128 + part * 16);
@@ -581,12 +657,231 @@ __global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
             case 3: primed = run13<3, kMode == 2>(ring, cur, nx.w, gs, us, p, xb, stride, sh, xsr, stage_slice); break;
             default: primed = run13<4, kMode == 2>(ring, cur, nx.w, gs, us, p, xb, stride, sh, xsr, stage_slice); break;
         }
-        if (kMode == 1 && nx.ok) stage13<kSmall>(p, sh, nx, xs, stride, sh.xsr[0]);
+        if (kMode == 1 && nx.ok) stage13(p, sh, nx, xs, stride, sh.xsr[0]);
         cur = nx;
         gs = gs_n;
         us = us_n;
         if (kMode == 0) buf ^= 1;
     }
+}
+
+// ---------------------------------------------------------------------------
+// Gate/up for H <= kBulkMaxK: one CTA per SM.  Each warp's 8 gate rows and 8
+// up rows of a task are two contiguous blocks of the weight matrix; the
+// warp's lane 0 fetches them with two bulk copies (cp.async.bulk, completion
+// counted on an mbarrier) into the warp's own two-slot ring in shared memory,
+// two tasks ahead, so that every SM keeps 128 KB of weights in flight, and
+// the warp reads its fragments from there.  Activations are staged per task
+// as in the kernel above (two cp.async buffers).  Every wait is bounded: on
+// a timeout the CTA flags ST_TIMEOUT, stops issuing, and still waits (again
+// bounded) for the copies it issued before it exits.
+// ---------------------------------------------------------------------------
+constexpr int kBulkMaxK = 1024;
+constexpr int kBulkSlots = 2;
+constexpr size_t kBulkWarpSlot = 16 * (kBulkMaxK / 2);  // 8 gate + 8 up rows
+constexpr size_t kBulkBarBytes = 128;
+constexpr size_t kSmem13Bulk = kShmBytes + kBulkBarBytes + 8 * kBulkSlots * kBulkWarpSlot +
+                               (size_t)2 * kStageRows * (kBulkMaxK + kPadB);
+constexpr long long kBulkWaitCycles = 4000000000LL;  // ~2 s
+
+__device__ __forceinline__ void bar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar))),
+                 "r"(count)
+                 : "memory");
+}
+__device__ __forceinline__ void bar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(bar))),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool bar_try(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar))), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for phase `parity` of bar.
+__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, long long limit) {
+    if (bar_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!bar_try(bar, parity))
+        if (clock64() - t0 > limit) return false;
+    return true;
+}
+// bytes (a multiple of 16, both addresses 16-byte aligned) global -> shared,
+// completion counted on bar.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src), "r"(bytes), "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar)))
+                 : "memory");
+}
+
+// Lane 0 of the calling warp issues the warp's 8 gate + 8 up rows of task t
+// into `slot`.
+__device__ __forceinline__ void issue13(const Params& p, const Task13& t, uint8_t* slot, uint64_t* bar) {
+    if ((threadIdx.x & 31) != 0 || !t.ok) return;
+    const size_t rb = (size_t)p.H / 2;
+    const uint8_t* W = t.shared ? p.sh_w13 : p.w13 + (size_t)t.e * 2 * p.I * rb;
+    const int r0 = t.r0;  // this warp's first row (r0 is per warp)
+    bar_expect_tx(bar, (uint32_t)(16 * rb));
+    bulk_g2s(slot, W + (size_t)r0 * rb, (uint32_t)(8 * rb), bar);
+    bulk_g2s(slot + 8 * rb, W + (size_t)(t.irow + r0) * rb, (uint32_t)(8 * rb), bar);
+}
+
+template <int NT>
+__device__ __forceinline__ void run13b(const Task13& tk, const uint8_t* wslot, float gs, float us, const Params& p,
+                                       const uint8_t* xs, int stride, Shm& sh, const float* xsr) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, q = lane & 3;
+    const int rb = p.H / 2, nkb = p.H / 128;
+    constexpr int kSets = NT == 1 ? 2 : 1;
+    int part[kSets][NT][4];
+#pragma unroll
+    for (int s = 0; s < kSets; ++s)
+#pragma unroll
+        for (int i = 0; i < NT; ++i) part[s][i][0] = part[s][i][1] = part[s][i][2] = part[s][i][3] = 0;
+    const uint8_t* ga = wslot + g * rb + q * 16;
+    const uint8_t* ua = wslot + (8 + g) * rb + q * 16;
+    const uint8_t* xrow = xs + g * stride + q * 32;
+#pragma unroll 2
+    for (int kb = 0; kb < nkb; ++kb) {
+        const uint4 wa = *reinterpret_cast<const uint4*>(ga + kb * 64);
+        const uint4 wb = *reinterpret_cast<const uint4*>(ua + kb * 64);
+        kblock8<NT, kSets>(wa, wb, xrow + kb * 128, 8 * stride, part);
+    }
+    int acc[NT][4];
+#pragma unroll
+    for (int i = 0; i < NT; ++i)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[i][c] = part[0][i][c] + part[kSets - 1][i][c] * (kSets - 1);
+    const int slot0 = (tk.shared ? 0 : tk.off) + tk.tok0;
+    float* hrow0 = (tk.shared ? p.h32_s : p.h32_r) + (size_t)slot0 * tk.irow + tk.r0 + g;
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+        const int j = 4 * i + q;
+        float hm = 0.f;
+        if (j < tk.nc) {
+            const float xsc = xsr[j] * 0.0625f;
+            const float gv = join(acc[i][0], acc[i][1]) * (gs * xsc);
+            const float uv = join(acc[i][2], acc[i][3]) * (us * xsc);
+            const float h = silu_mul(gv, uv);
+            hrow0[(size_t)j * tk.irow] = h;
+            hm = fabsf(h);
+        }
+        hm = nanmax(hm, __shfl_xor_sync(0xffffffffu, hm, 4));
+        hm = nanmax(hm, __shfl_xor_sync(0xffffffffu, hm, 8));
+        hm = nanmax(hm, __shfl_xor_sync(0xffffffffu, hm, 16));
+        if (g == 0 && j < tk.nc) sh.hm[warp][j] = hm;
+    }
+    __syncthreads();
+    if (threadIdx.x < tk.nc) {
+        const int j = threadIdx.x;
+        const int nrb = tk.irow / kRows13;
+        float m = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) m = nanmax(m, sh.hm[w][j]);
+        (tk.shared ? p.hmax_s : p.hmax_r)[(size_t)(slot0 + j) * nrb + tk.rbk] = m;
+    }
+}
+
+__global__ void __launch_bounds__(256, 1) experts_w13_bulk_kernel(Params p) {
+    extern __shared__ __align__(128) uint8_t dsm[];
+    Shm& sh = *reinterpret_cast<Shm*>(dsm);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(dsm + kShmBytes);  // [warp][slot]
+    uint8_t* wring = dsm + kShmBytes + kBulkBarBytes;
+    uint8_t* xs = wring + 8 * kBulkSlots * kBulkWarpSlot;
+    const int warp = threadIdx.x >> 5, g = (threadIdx.x & 31) >> 2;
+    const int H = p.H;
+    const int stride = H + kPadB;
+    const int bufbytes = kStageRows * stride;
+    const size_t wslot_bytes = (size_t)16 * (H / 2);
+    auto slot_ptr = [&](int s) { return wring + ((size_t)warp * kBulkSlots + s) * kBulkWarpSlot; };
+    auto bar_of = [&](int s) { return bars + warp * kBulkSlots + s; };
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 8 * kBulkSlots; ++i) bar_init(bars + i, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    (void)wslot_bytes;
+    // A CTA whose first task belongs to the shared expert fetches its weights
+    // before the router has finished.
+    const int ns = p.Is > 0 ? (p.Is / kRows13) * chunks_of(p.T) : 0;
+    bool pre = false;
+    const uint8_t* pre_ra = nullptr;
+    if ((int)blockIdx.x < ns) {
+        const Task13 t = make13(p, p.E, p.T, p.T * p.K, ns - 1 - (int)blockIdx.x);
+        issue13(p, t, slot_ptr(0), bar_of(0));
+        pre = true;
+        pre_ra = t.w.ra;
+    }
+    if (p.Is > 0) prefetch_l2_slice(p.sh_w13, (size_t)p.Is * p.H);
+    pdl_wait();
+    pdl_release();
+    if (p.decode_groups > 0) build_tables_small(p, sh, reinterpret_cast<int*>(xs));
+    else load_tables(p, p.ts13, &p.ctrl->tasks13, sh.tb, sh.tok);
+    precompute_tasks(p, sh, 0);
+    Task13 cur = task13_r(p, sh, 0);
+    bool abort = false;
+    if (pre && cur.w.ra != pre_ra) {  // cannot happen with consistent tables
+        if (threadIdx.x == 0) atomicOr(&p.ctrl->status, ST_BAD_TASK);
+        abort = true;
+    }
+    bool issued[kBulkSlots] = {pre, false};
+    uint32_t ph[kBulkSlots] = {0u, 0u};
+    if (!abort) {
+        if (!pre && cur.ok) { issue13(p, cur, slot_ptr(0), bar_of(0)); issued[0] = true; }
+        const Task13 t1 = task13_r(p, sh, 1);
+        if (t1.ok) { issue13(p, t1, slot_ptr(1), bar_of(1)); issued[1] = true; }
+        // activations first in the memory queues of this SM's first task
+        if (cur.ok) stage13(p, sh, cur, xs, stride, sh.xsr[0]);
+    }
+    const float* S = cur.shared ? p.sh_s13 : p.s13 + (size_t)cur.e * 2 * p.I;
+    float gs = cur.ok ? __ldg(S + cur.r0 + g) : 0.f, us = cur.ok ? __ldg(S + cur.irow + cur.r0 + g) : 0.f;
+    for (int r = 0; !abort && cur.ok; ++r) {
+        const int s = r & 1;
+        const Task13 nx = task13_r(p, sh, r + 1);
+        cp_async_wait<0>();
+        __syncthreads();  // cur's activations are visible; the previous task is done with the other buffer
+        if (nx.ok) stage13(p, sh, nx, xs + (s ^ 1) * bufbytes, stride, sh.xsr[s ^ 1]);
+        float gs_n = 0.f, us_n = 0.f;
+        if (nx.ok) {
+            const float* Sn = nx.shared ? p.sh_s13 : p.s13 + (size_t)nx.e * 2 * p.I;
+            gs_n = __ldg(Sn + nx.r0 + g);
+            us_n = __ldg(Sn + nx.irow + nx.r0 + g);
+        }
+        // this warp's weights of cur (slot s); a timeout flags the CTA, whose
+        // warps then stop issuing and leave the loop together below
+        const bool got = bar_wait(bar_of(s), ph[s], kBulkWaitCycles);
+        if (got) ph[s] ^= 1u, issued[s] = false;
+        if (!got && (threadIdx.x & 31) == 0) atomicOr(&p.ctrl->status, ST_TIMEOUT);
+        if (__syncthreads_or(!got)) {
+            abort = true;
+            break;
+        }
+        const uint8_t* wslot = slot_ptr(s);
+        const uint8_t* xb = xs + s * bufbytes;
+        const float* xsr = sh.xsr[s];
+        switch ((2 * cur.nc + 7) >> 3) {
+            case 1: run13b<1>(cur, wslot, gs, us, p, xb, stride, sh, xsr); break;
+            case 2: run13b<2>(cur, wslot, gs, us, p, xb, stride, sh, xsr); break;
+            case 3: run13b<3>(cur, wslot, gs, us, p, xb, stride, sh, xsr); break;
+            default: run13b<4>(cur, wslot, gs, us, p, xb, stride, sh, xsr); break;
+        }
+        // the slot is free (the epilogue's barrier follows every warp's reads): refill it two tasks ahead
+        const Task13 t2 = task13_r(p, sh, r + 2);
+        if (t2.ok) { issue13(p, t2, slot_ptr(s), bar_of(s)); issued[s] = true; }
+        cur = nx;
+        gs = gs_n;
+        us = us_n;
+    }
+    // every copy this warp issued has landed before the CTA's shared memory goes away
+    for (int s = 0; s < kBulkSlots; ++s)
+        if (issued[s]) bar_wait(bar_of(s), ph[s], kBulkWaitCycles);
+    cp_async_wait<0>();
 }
 
 // One down task as this thread sees it.
@@ -622,14 +917,32 @@ __device__ __forceinline__ Task2 make2(const Params& p, int e, int n, int off, i
     return t;
 }
 
-__device__ __forceinline__ Task2 task2_at(const Params& p, const Tables& tb, int lin) {
-    if (lin >= tb.ntask) {
-        Task2 t{};
-        return t;
-    }
-    const int task = tb.ntask - 1 - lin;
-    const int b = find_bucket(tb, task);
-    return make2(p, tb.e[b], tb.n[b], tb.off[b], task - tb.ts[b]);
+// Down task from its descriptor (no task: ok = false).
+__device__ __forceinline__ Task2 task2_from(const Params& p, const TaskDesc& d) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, q = lane & 3;
+    Task2 t{};
+    if (d.e < 0) return t;
+    t.ok = !(d.e > p.E || (d.e == p.E && p.Is == 0));
+    t.shared = d.e == p.E;
+    t.e = d.e;
+    t.off = d.off;
+    t.irow = t.shared ? p.Is : p.I;
+    t.sl = d.sl;
+    t.k0 = d.sl * kSliceK;
+    t.klen = min(kSliceK, t.irow - t.k0);
+    t.tok0 = d.tok0;
+    t.nc = d.nc;
+    t.j0 = d.rbk * kRows2 + warp * 16;
+    const int row_bytes = t.irow / 2;
+    const uint8_t* W = t.shared ? p.sh_w2 : p.w2 + (size_t)(t.ok ? d.e : 0) * p.H * row_bytes;
+    t.w.ra = W + (size_t)(t.j0 + g) * row_bytes + t.k0 / 2 + q * 16;
+    t.w.rb = W + (size_t)(t.j0 + g + 8) * row_bytes + t.k0 / 2 + q * 16;
+    t.w.nkb = t.ok ? t.klen / 128 : 0;
+    return t;
+}
+
+__device__ __forceinline__ Task2 task2_r(const Params& p, const Shm& sh, int r) {
+    return task2_from(p, task_desc(p, sh, 1, r));
 }
 
 // Issues the cp.async of task t's f32 slice of h (raw[j][k], k < klen) and of
@@ -694,15 +1007,16 @@ __global__ void __launch_bounds__(256, 2) experts_w2_kernel(Params p) {
     if (p.Is > 0) prefetch_l2_slice(p.sh_w2, (size_t)p.H * p.Is / 2);
     pdl_wait();
     pdl_release();
-    load_tables(p, p.ts2, &p.ctrl->tasks2, sh.tb);
+    load_tables(p, p.ts2, &p.ctrl->tasks2, sh.tb, nullptr);
+    precompute_tasks(p, sh, 1);
     const Tables& tb = sh.tb;
-    Task2 cur = task2_at(p, tb, blockIdx.x);
+    Task2 cur = task2_r(p, sh, 0);
     if (primed && cur.w.ra != primed_ra) primed = false;
     if (cur.ok) fetch2(p, sh, cur, raw);
     const float* S = cur.shared ? p.sh_s2 : p.s2 + (size_t)cur.e * p.H;
     float s_lo = cur.ok ? __ldg(S + cur.j0 + g) : 0.f, s_hi = cur.ok ? __ldg(S + cur.j0 + g + 8) : 0.f;
-    for (int lin = blockIdx.x; lin < tb.ntask; lin += gridDim.x) {
-        const Task2 nx = task2_at(p, tb, lin + gridDim.x);
+    for (int r = 0, lin = blockIdx.x; lin < tb.ntask; lin = snake(blockIdx.x, ++r)) {
+        const Task2 nx = task2_r(p, sh, r + 1);
         if (!cur.ok) {  // a table entry out of range: flag it and stop
             if (threadIdx.x == 0) atomicOr(&p.ctrl->status, ST_BAD_TASK);
             break;
@@ -756,6 +1070,7 @@ __global__ void __launch_bounds__(256, 2) experts_w2_kernel(Params p) {
 template <typename Kern>
 int resident(Kern kern, size_t smem, int which) {
     static int cache[8][64];
+    static_assert(kSmem13Bulk <= 227 * 1024, "bulk gate/up shared memory");
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
     int& c = cache[which][dev];
@@ -773,30 +1088,25 @@ int resident(Kern kern, size_t smem, int which) {
 
 // Persistent grid of the weight-streaming kernels: the CTAs that fit at once
 // (which: 0 gate/up, 1 down).  Also sets the kernels' shared-memory limits.
-int experts_resident_ctas(int which, int H, bool small) {
-    if (which == 1) return resident(experts_w2_kernel, kSmem2, 6);
+int experts_resident_ctas(int which, int H) {
+    if (which == 1) return resident(experts_w2_kernel, kSmem2, 3);
+    if (H <= kBulkMaxK) return resident(experts_w13_bulk_kernel, kSmem13Bulk, 4);
     const int mode = H <= kDoubleMaxK ? 0 : H <= kWholeMaxK ? 1 : 2;
-    switch (mode * 2 + (small ? 1 : 0)) {
-        case 0: return resident(experts_w13_kernel<0, false>, kSmem13[0], 0);
-        case 1: return resident(experts_w13_kernel<0, true>, kSmem13[0], 1);
-        case 2: return resident(experts_w13_kernel<1, false>, kSmem13[1], 2);
-        case 3: return resident(experts_w13_kernel<1, true>, kSmem13[1], 3);
-        case 4: return resident(experts_w13_kernel<2, false>, kSmem13[2], 4);
-        default: return resident(experts_w13_kernel<2, true>, kSmem13[2], 5);
+    switch (mode) {
+        case 0: return resident(experts_w13_kernel<0>, kSmem13[0], 0);
+        case 1: return resident(experts_w13_kernel<1>, kSmem13[1], 1);
+        default: return resident(experts_w13_kernel<2>, kSmem13[2], 2);
     }
 }
 
 cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
-    const bool small = p.decode_groups > 0;
-    const int mode = p.H <= kDoubleMaxK ? 0 : p.H <= kWholeMaxK ? 1 : 2;
     const dim3 g(grid), b(256);
-    switch (mode * 2 + (small ? 1 : 0)) {
-        case 0: return launch_pdl(experts_w13_kernel<0, false>, g, b, kSmem13[0], stream, p);
-        case 1: return launch_pdl(experts_w13_kernel<0, true>, g, b, kSmem13[0], stream, p);
-        case 2: return launch_pdl(experts_w13_kernel<1, false>, g, b, kSmem13[1], stream, p);
-        case 3: return launch_pdl(experts_w13_kernel<1, true>, g, b, kSmem13[1], stream, p);
-        case 4: return launch_pdl(experts_w13_kernel<2, false>, g, b, kSmem13[2], stream, p);
-        default: return launch_pdl(experts_w13_kernel<2, true>, g, b, kSmem13[2], stream, p);
+    if (p.H <= kBulkMaxK) return launch_pdl(experts_w13_bulk_kernel, g, b, kSmem13Bulk, stream, p);
+    const int mode = p.H <= kDoubleMaxK ? 0 : p.H <= kWholeMaxK ? 1 : 2;
+    switch (mode) {
+        case 0: return launch_pdl(experts_w13_kernel<0>, g, b, kSmem13[0], stream, p);
+        case 1: return launch_pdl(experts_w13_kernel<1>, g, b, kSmem13[1], stream, p);
+        default: return launch_pdl(experts_w13_kernel<2>, g, b, kSmem13[2], stream, p);
     }
 }
 

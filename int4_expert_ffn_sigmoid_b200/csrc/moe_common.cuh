@@ -11,6 +11,9 @@ namespace moe {
 
 // Largest T that takes the weight-streaming (small-batch) path by default.
 constexpr int kDecodeMaxTokens = 64;
+// Rows of one weight-streaming task: gate/up (each with its up row), down.
+constexpr int kTaskRows13 = 64;
+constexpr int kTaskRows2 = 128;
 // Tokens of one bucket handled by one weight-streaming task: each token
 // takes two int8 columns (its two activation parts), so 16 tokens fill four
 // mma n-tiles of 8 columns.
@@ -49,8 +52,8 @@ enum : unsigned {
 };
 
 // First 256 bytes of the workspace.  The first kernel of every call zeroes
-// status, claim13 and claim2; every other field is written before it is read
-// within the call, so the workspace needs no initialisation.
+// status; every other field is written before it is read within the call,
+// so the workspace needs no initialisation.
 struct Ctrl {
     unsigned status;
     int n_buckets;      // non-empty routed buckets + the shared bucket
@@ -58,9 +61,7 @@ struct Ctrl {
     int tasks2;         // down tasks over all buckets
     int tc_tiles1;      // tensor-core GEMM-1 tiles over the routed buckets
     int tc_tiles2;      // tensor-core GEMM-2 tiles over the routed buckets
-    int claim13;        // next gate/up task to claim (weight-streaming kernel)
-    int claim2;         // next down task to claim
-    int pad[56];
+    int pad[58];
 };
 
 // Programmatic dependent launch: every kernel of a call is launched so that
@@ -218,8 +219,11 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
+// silu(g) * u = g * sigmoid(g) * u, with the fast exponential and divide
+// intrinsics (a few ulp; for g below about -88 the exponential overflows to
+// infinity and the result is a signed zero, the correct limit).
 __device__ __forceinline__ float silu_mul(float g, float u) {
-    return g / (1.0f + expf(-g)) * u;
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
 // Bucket geometry of the expert kernels.

@@ -14,10 +14,9 @@ cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream);
 // Expert down projection (weight-streaming mma.sync kernel).
 cudaError_t launch_experts_w2(const Params& p, int grid, cudaStream_t stream);
 // CTAs of the weight-streaming kernel `which` (0: gate/up, 1: down) that fit
-// on the device at once (the persistent grid size) for hidden size H, with
-// the small-batch (small) or large-batch bucket tables.  Also sets the
-// kernel's shared-memory attribute.
-int experts_resident_ctas(int which, int H, bool small);
+// on the device at once (the persistent grid size) for hidden size H.  Also
+// sets the kernel's shared-memory attribute.
+int experts_resident_ctas(int which, int H);
 // Weighted combine + shared expert (+ residual) -> bf16 out.
 cudaError_t launch_combine(const Params& p, cudaStream_t stream);
 

@@ -244,8 +244,8 @@ __device__ void finalize_buckets(const Params& p, const int* s_cnt, int* s_off) 
                 const int irow = (e == E) ? p.Is : p.I;
                 const int n = p.bucket_n[b];
                 const int ch = chunks_of(n);
-                n13 = (irow / 64) * ch;                    // tasks: 64 gate/up rows x a token chunk
-                n2 = (p.H / 128) * ch * slices_of(irow);   // tasks: 128 down rows x a chunk x a slice
+                n13 = (irow / kTaskRows13) * ch;                    // gate/up rows x a token chunk
+                n2 = (p.H / kTaskRows2) * ch * slices_of(irow);     // down rows x a chunk x a slice
                 if (e != E) {  // tensor-core tiles: 128 tokens x 128 features / 256 columns
                     const int mt = (n + 127) / 128;
                     nt1 = mt * (p.I / 128);
@@ -287,14 +287,10 @@ __device__ void finalize_buckets(const Params& p, const int* s_cnt, int* s_off) 
     __syncthreads();
 }
 
-// Zeroes the per-call control words (first kernel of a call, one thread,
+// Zeroes the per-call status word (first kernel of a call, one thread,
 // after pdl_wait: every kernel of the previous call has completed).
 __device__ __forceinline__ void reset_ctrl(const Params& p) {
-    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
-        p.ctrl->status = 0;
-        p.ctrl->claim13 = 0;
-        p.ctrl->claim2 = 0;
-    }
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) p.ctrl->status = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -308,7 +304,8 @@ __device__ __forceinline__ void reset_ctrl(const Params& p) {
 // token), and writes the group's per-expert pick counts (hist[group][e]) and
 // the rank of every pick among the group's picks of the same expert, in
 // (token, k) order.  The other CTAs quantize the group's activations (xq,
-// xs) from their shared copy.  The expert kernels derive the buckets and slots from hist, idx and
+// xs) from their shared copy.  The gate/up kernel derives the bucket and
+// task tables from hist, idx and rank.  The expert kernels derive the buckets and slots from hist, idx and
 // rank themselves: the slot of pick (t, k) of expert e is offset[e] + (picks
 // of e in earlier groups) + rank, i.e. buckets list their tokens in (t, k)
 // order.

@@ -53,6 +53,16 @@ def test_struct_layout_matches_c(moe, tmp_path):
     assert c_vals == py_vals
 
 
+def test_header_constants_match_binding(moe):
+    text = open(HEADER).read()
+    for name in ("MOE_STATIC_WORKSPACE_BYTES", "MOE_OUT_F32", "MOE_FORCE_DECODE",
+                 "MOE_FORCE_PREFILL", "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK"):
+        m = re.search(rf"#define {name} (.+)", text)
+        assert m, name
+        expr = m.group(1).split("/*")[0].replace("(size_t)", "").replace("u", "")
+        assert eval(expr) == getattr(moe, name), name
+
+
 def test_version_and_strings(moe):
     assert moe.lib.moe_abi_version() == 1
     assert moe.status_str(0) == "MOE_OK"
