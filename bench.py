@@ -402,8 +402,9 @@ def run_ours(args, rank, world, device, dist):
     names = moe.STAGE_NAMES
     dom = 1 if stage_mean[1] >= stage_mean[2] else 2  # the dominant expert kernel
     tc_path = T > moe.decode_max_tokens() and wl.shape.H % 256 == 0
+    w13_name = "experts_w13_bulk_kernel" if wl.shape.H <= 1024 else "experts_w13_kernel"
     kname = (("grouped_gemm_kernel<1>" if dom == 1 else "grouped_gemm_kernel<2>") if tc_path
-             else ("experts_w13_kernel" if dom == 1 else "experts_w2_kernel"))
+             else (w13_name if dom == 1 else "experts_w2_kernel"))
     work = [[stage_work(names[dom], wl.shape, T, u) for u in uniq[i % N_BATCHES]] for i in range(args.steps)]
     alg_b = statistics.mean(sum(w[0] for w in ws) for ws in work) / L
     alg_f = statistics.mean(sum(w[1] for w in ws) for ws in work) / L
