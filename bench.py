@@ -358,6 +358,22 @@ def cpu_baseline_sample(stack, budget_s=20.0):
     return n_tok * len(layers_cpu) / dt, f"{n_tok} of {stack.T} tokens of one batch through all {len(layers_cpu)} layers ({dt:.1f} s)"
 
 
+def max_over_ranks(values, dist, device):
+    """Element-wise maximum of `values` over all ranks (the slowest rank's
+    times); the values themselves for a single process (dist None)."""
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_throughput(world, tokens_per_step, steps, total_ms):
+    """Whole-job tokens/s: every rank ran `steps` steps of `tokens_per_step`
+    tokens, and the job took the slowest rank's `total_ms`."""
+    return world * tokens_per_step * steps / (total_ms / 1e3)
+
+
 def run_ours(args, rank, world, device, dist):
     import int4_expert_ffn_sigmoid_b200 as moe
     wl = workloads.WORKLOADS[args.workload]
@@ -375,17 +391,11 @@ def run_ours(args, rank, world, device, dist):
     _, stage_ms = timed_steps(stack, args.steps, 2, use_graph, flush, instrumented=True)
     e2e_ms, h2d, d2h = e2e_steps(stack, args.steps, args.warmup, flush, dist_barrier=barrier)
 
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms, sum(e2e_ms)], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_total = float(t[0]), float(t[1])
-    else:
-        e2e_total = sum(e2e_ms)
+    total_ms, e2e_total = max_over_ranks([sum(step_ms), sum(e2e_ms)], dist if world > 1 else None, device)
     L = wl.layers
     tokens_per_step = T * L
-    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
-    e2e_value = world * tokens_per_step * args.steps / (e2e_total / 1e3)
+    value = job_throughput(world, tokens_per_step, args.steps, total_ms)
+    e2e_value = job_throughput(world, tokens_per_step, args.steps, e2e_total)
 
     # work accounting (batch i % 4 at step i)
     step_b, step_f = [], []
@@ -443,7 +453,9 @@ def run_ours(args, rank, world, device, dist):
         v, sample = cpu_baseline_sample(stack)
         cpu = {"value": round(v, 2), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
 
-    kernels_per_layer = 4 if T <= moe.decode_max_tokens() else 5
+    # small batch: router, gate/up, down, combine; large batch: router, finalize,
+    # scatter, gate/up, down, combine
+    kernels_per_layer = 4 if T <= moe.decode_max_tokens() else 6
     launches = args.steps * L
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
