@@ -158,8 +158,8 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
     Tables& tb = sh.tb;
     int my_e[2], my_rank[2];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const int i = tid + 256 * u;
+    for (int u = 0; u < 2; ++u) {  // threads 0..255 cover the T*K <= 512 picks
+        const int i = tid < 256 ? tid + 256 * u : TK;
         my_e[u] = i < TK ? __ldcg(p.idx + i) : -1;
         my_rank[u] = i < TK ? __ldcg(p.rank + i) : 0;
     }
@@ -262,7 +262,7 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
     __syncthreads();
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-        const int i = tid + 256 * u;
+        const int i = tid < 256 ? tid + 256 * u : TK;
         if (i >= TK) continue;
         const int e = my_e[u], t = i / K;
         int slot = -1;
@@ -522,7 +522,7 @@ __device__ __forceinline__ void stage13(const Params& p, const Shm& sh, const Ta
                                         float* xsr) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int H = p.H;
-    for (int r = warp; r < 2 * t.nc; r += 8) {
+    for (int r = warp; r < 2 * t.nc; r += blockDim.x / 32) {
         const int tok = slot_token(p, sh, t.shared, t.off, t.tok0 + (r >> 1));
         if (tok < 0 || tok >= p.T) continue;
         const int8_t* src = p.xq + (size_t)tok * 2 * H + (r & 1) * H;
@@ -1068,7 +1068,7 @@ __global__ void __launch_bounds__(256, 2) experts_w2_kernel(Params p) {
 }
 
 template <typename Kern>
-int resident(Kern kern, size_t smem, int which) {
+int resident(Kern kern, size_t smem, int which, int threads = 256) {
     static int cache[8][64];
     static_assert(kSmem13Bulk <= 227 * 1024, "bulk gate/up shared memory");
     int dev = 0;
@@ -1077,7 +1077,7 @@ int resident(Kern kern, size_t smem, int which) {
     if (c == 0) {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         int per_sm = 0, sms = 0;
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         c = (per_sm > 0 ? per_sm : 1) * (sms > 0 ? sms : 148);
     }
