@@ -11,7 +11,9 @@
 // README, "Converting a checkpoint yourself": per-row symmetric int4, f32 scales.
 //
 // Tile: 128 tokens (MMA M, one TMEM lane per token) x 256 output columns (MMA
-// N) x 64 reduction elements per pipeline stage.  GEMM-1's 256 columns are 128
+// N) x 64 reduction elements per pipeline stage.  Two rings: TMA stages hold
+// the activation and raw int4 tiles of 6 k blocks; 2 slots hold the
+// dequantised B operand between the dequantisers and the MMA.  GEMM-1's 256 columns are 128
 // gate rows and the 128 up rows of the same features, so one thread of the
 // epilogue holds gate and up of one (token, feature) pair.
 // Roles (448 threads):
@@ -34,22 +36,29 @@ namespace moe {
 namespace tc {
 
 constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int STAGES = 4;
+// Two rings: TMA stages (activation tile + raw int4 tile) run TSTAGES k
+// blocks ahead to cover load latency; the dequantised B operand needs only
+// BSTAGES slots between the dequantisers and the MMA.
+constexpr int TSTAGES = 6;
+constexpr int BSTAGES = 2;
 constexpr int A_BYTES = BM * BK * 2;    // 16 KiB, bf16/fp16 activations
 constexpr int B_BYTES = BN * BK * 2;    // 32 KiB, dequantised weights
 constexpr int RAW_BYTES = BN * BK / 2;  // 8 KiB, packed int4 weights
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RAW_BYTES;
-constexpr int NUM_THREADS = 448;
+constexpr int TSTAGE_BYTES = A_BYTES + RAW_BYTES;
+constexpr int RING_BYTES = TSTAGES * TSTAGE_BYTES + BSTAGES * B_BYTES;
 constexpr int DEQ_WARPS = 8;
+constexpr int NUM_THREADS = 64 + 32 * DEQ_WARPS + 128;
 constexpr int TMEM_COLS = 512;          // two 256-column accumulators
 constexpr long long kTimeoutCycles = 4000000000LL;
 constexpr long long kDrainCycles = 200000000LL;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1280;
+constexpr int SMEM_BYTES = RING_BYTES + 1024 + 1280;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of the grouped GEMM");
 
 struct Shared {
-    uint64_t full_tma[STAGES];
-    uint64_t full_deq[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full_tma[TSTAGES];  // activation + raw tiles landed (TMA transaction count)
+    uint64_t empty_t[TSTAGES];   // MMA done with the activation tile, dequantisers with the raw tile
+    uint64_t full_deq[BSTAGES];  // B operand dequantised (one arrival per dequant warp)
+    uint64_t empty_b[BSTAGES];   // MMA done with the B operand
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
@@ -242,17 +251,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
                     const TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Shared* sh = reinterpret_cast<Shared*>(smem + STAGES * STAGE_BYTES);
-    auto a_tile = [&](int s) { return smem + s * STAGE_BYTES; };
-    auto b_tile = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
-    auto raw_tile = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES + B_BYTES; };
+    Shared* sh = reinterpret_cast<Shared*>(smem + RING_BYTES);
+    auto a_tile = [&](int s) { return smem + s * TSTAGE_BYTES; };
+    auto raw_tile = [&](int s) { return smem + s * TSTAGE_BYTES + A_BYTES; };
+    auto b_tile = [&](int s) { return smem + TSTAGES * TSTAGE_BYTES + s * B_BYTES; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < TSTAGES; ++s) {
             mbar_init(&sh->full_tma[s], 1);
+            mbar_init(&sh->empty_t[s], 1 + DEQ_WARPS);
+        }
+        for (int s = 0; s < BSTAGES; ++s) {
             mbar_init(&sh->full_deq[s], DEQ_WARPS);
-            mbar_init(&sh->empty[s], 1);
+            mbar_init(&sh->empty_b[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sh->acc_full[b], 1);
@@ -285,9 +297,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB_s)) : "memory");
             int s = 0;
             uint32_t ph = 0;
-            uint32_t issued_par[STAGES];
-            bool issued[STAGES];
-            for (int i = 0; i < STAGES; ++i) issued[i] = false, issued_par[i] = 0;
+            uint32_t issued_par[TSTAGES];
+            bool issued[TSTAGES];
+            for (int i = 0; i < TSTAGES; ++i) issued[i] = false, issued_par[i] = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
                 const Tile t = decode_tile(a, tile);
@@ -305,26 +317,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
                     brow1 = base + t.col0 + BN / 2;
                 }
                 for (int kb = 0; kb < t.nkb; ++kb) {
-                    if (!mbar_wait(&sh->empty[s], ph ^ 1u, sh)) { ok = false; break; }
+                    if (!mbar_wait(&sh->empty_t[s], ph ^ 1u, sh)) { ok = false; break; }
                     mbar_expect_tx(&sh->full_tma[s], A_BYTES + RAW_BYTES);
                     tma_load_2d(a_tile(s), mA, &sh->full_tma[s], kb * BK, t.a_row);
                     tma_load_2d(raw_tile(s), mB, &sh->full_tma[s], kb * (BK / 2), brow0);
                     tma_load_2d(raw_tile(s) + RAW_BYTES / 2, mB, &sh->full_tma[s], kb * (BK / 2), brow1);
                     issued[s] = true;
                     issued_par[s] = ph;
-                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                    if (++s == TSTAGES) { s = 0; ph ^= 1u; }
                 }
             }
             // make sure no copy is still landing when the CTA leaves
-            for (int i = 0; i < STAGES; ++i)
+            for (int i = 0; i < TSTAGES; ++i)
                 if (issued[i]) mbar_wait(&sh->full_tma[i], issued_par[i], sh, kDrainCycles);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_f16(GEMM == 1 ? 1 : 0, BM, BN);
-            int s = 0;
-            uint32_t ph = 0;
+            int s = 0, sb = 0;
+            uint32_t ph = 0, phb = 0;
             uint32_t acc_ph[2] = {0, 0};
             int buf = 0;
             bool ok = true, any = false;
@@ -334,20 +346,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
                 tc_fence_after();
                 const uint32_t d = tmem + buf * BN;
                 for (int kb = 0; kb < t.nkb; ++kb) {
-                    if (!mbar_wait(&sh->full_tma[s], ph, sh) || !mbar_wait(&sh->full_deq[s], ph, sh)) {
+                    if (!mbar_wait(&sh->full_tma[s], ph, sh) || !mbar_wait(&sh->full_deq[sb], phb, sh)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t aaddr = smem_u32(a_tile(s)), baddr = smem_u32(b_tile(s));
+                    const uint32_t aaddr = smem_u32(a_tile(s)), baddr = smem_u32(b_tile(sb));
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         mma_f16_ss(d, smem_desc_sw128(aaddr + kk * 32), smem_desc_sw128(baddr + kk * 32), idesc,
                                    (kb | kk) != 0);
                     }
                     any = true;
-                    mma_commit(&sh->empty[s]);
-                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                    mma_commit(&sh->empty_t[s]);
+                    mma_commit(&sh->empty_b[sb]);
+                    if (++s == TSTAGES) { s = 0; ph ^= 1u; }
+                    if (++sb == BSTAGES) { sb = 0; phb ^= 1u; }
                 }
                 if (!ok) break;
                 mma_commit(&sh->acc_full[buf]);
@@ -362,17 +376,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
     } else if (warp < 2 + DEQ_WARPS) {
         // ---------------- dequantisers (one B row per thread) ----------------
         const int r = threadIdx.x - 64;  // B row = output column of the tile
-        int s = 0;
-        uint32_t ph = 0;
+        int s = 0, sb = 0;
+        uint32_t ph = 0, phb = 0;
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
             const Tile t = decode_tile(a, tile);
             for (int kb = 0; kb < t.nkb; ++kb) {
                 int got = 0;
-                if (lane == 0) got = mbar_wait(&sh->full_tma[s], ph, sh);
+                if (lane == 0) got = mbar_wait(&sh->full_tma[s], ph, sh) && mbar_wait(&sh->empty_b[sb], phb ^ 1u, sh);
                 if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
                 const uint8_t* raw = raw_tile(s);
-                uint8_t* bt = b_tile(s);
+                uint8_t* bt = b_tile(sb);
                 {
                     const uint4 q0 = *reinterpret_cast<const uint4*>(raw + r * 32);
                     const uint4 q1 = *reinterpret_cast<const uint4*>(raw + r * 32 + 16);
@@ -387,8 +401,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sh->full_deq[s]);
-                if (++s == STAGES) { s = 0; ph ^= 1u; }
+                if (lane == 0) {
+                    mbar_arrive(&sh->full_deq[sb]);
+                    mbar_arrive(&sh->empty_t[s]);  // this warp is done with the raw tile
+                }
+                if (++s == TSTAGES) { s = 0; ph ^= 1u; }
+                if (++sb == BSTAGES) { sb = 0; phb ^= 1u; }
             }
         }
     } else {
