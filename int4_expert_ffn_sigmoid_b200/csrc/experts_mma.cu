@@ -110,9 +110,12 @@ constexpr size_t kShmBytes = (sizeof(Shm) + 127) & ~size_t(127);
 // scratch of the small-batch table build, in the staging area
 constexpr size_t kBuildBytes = (size_t)(kDecodeGroups + 2) * kMaxE * 4;
 static_assert(kBuildBytes <= (size_t)kStageRows * (kXRing * 128 + kPadB), "table build scratch fits the staging area");
+// Mode 2 stages whole rows too when a task's rows fit in this many bytes.
+constexpr size_t kRingWholeBytes = 100 * 1024;
 constexpr size_t kSmem13[3] = {kShmBytes + (size_t)2 * kStageRows * (kDoubleMaxK + kPadB),
                                kShmBytes + (size_t)kStageRows * (kWholeMaxK + kPadB),
-                               kShmBytes + (size_t)kStageRows * (kXRing * 128 + kPadB)};
+                               kShmBytes + kRingWholeBytes};
+static_assert(kRingWholeBytes >= (size_t)kStageRows * (kXRing * 128 + kPadB), "ring staging fits");
 // down: int8 staging of one slice + the next task's f32 slice
 constexpr int kStride2 = kSliceK + kPadB;
 constexpr size_t kRaw2Off = (size_t)kStageRows * kStride2;
@@ -579,7 +582,9 @@ __device__ __forceinline__ bool run13(Ring& ring, const Task13& tk, const WStrea
 }
 
 // kMode: 0 two whole-row staging buffers (the next task's activations load
-// while the current task computes), 1 one whole-row buffer, 2 ring of slices.
+// while the current task computes), 1 one whole-row buffer, 2 (large H) one
+// whole-row buffer for tasks whose rows fit in kRingWholeBytes, else a ring of
+// 128-wide slices.
 template <int kMode>
 __global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
     extern __shared__ __align__(128) uint8_t dsm[];
@@ -624,7 +629,13 @@ __global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
             break;
         }
         if (!primed) prime(ring, cur.w);
-        if (kMode == 2 && threadIdx.x < cur.nc) {  // ring mode: the scales only (slices are staged in the loop)
+        // large H: whole rows when every row the mma tiles read (8 per n-tile) fits,
+        // else slices staged in the main loop
+        const bool whole2 = kMode == 2 && (size_t)8 * ((2 * cur.nc + 7) >> 3) * (H + kPadB) <= kRingWholeBytes;
+        if (whole2) {
+            stage13(p, sh, cur, xs, H + kPadB, sh.xsr[0]);
+            cp_async_wait<0>();
+        } else if (kMode == 2 && threadIdx.x < cur.nc) {  // the scales only
             const int tok = slot_token(p, sh, cur.shared, cur.off, cur.tok0 + threadIdx.x);
             if (tok >= 0 && tok < p.T) cp_async4(sh.xsr[0] + threadIdx.x, p.xs + tok);
             else sh.xsr[0][threadIdx.x] = 0.f;
@@ -651,11 +662,20 @@ __global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
         };
         const uint8_t* xb = xs + (kMode == 0 ? buf * bufbytes : 0);
         const float* xsr = sh.xsr[kMode == 0 ? buf : 0];
-        switch ((2 * nc + 7) >> 3) {
-            case 1: primed = run13<1, kMode == 2>(ring, cur, nx.w, gs, us, p, xb, stride, sh, xsr, stage_slice); break;
-            case 2: primed = run13<2, kMode == 2>(ring, cur, nx.w, gs, us, p, xb, stride, sh, xsr, stage_slice); break;
-            case 3: primed = run13<3, kMode == 2>(ring, cur, nx.w, gs, us, p, xb, stride, sh, xsr, stage_slice); break;
-            default: primed = run13<4, kMode == 2>(ring, cur, nx.w, gs, us, p, xb, stride, sh, xsr, stage_slice); break;
+        if (kMode == 2 && whole2) {
+            switch ((2 * nc + 7) >> 3) {
+                case 1: primed = run13<1, false>(ring, cur, nx.w, gs, us, p, xb, H + kPadB, sh, xsr, stage_slice); break;
+                case 2: primed = run13<2, false>(ring, cur, nx.w, gs, us, p, xb, H + kPadB, sh, xsr, stage_slice); break;
+                case 3: primed = run13<3, false>(ring, cur, nx.w, gs, us, p, xb, H + kPadB, sh, xsr, stage_slice); break;
+                default: primed = run13<4, false>(ring, cur, nx.w, gs, us, p, xb, H + kPadB, sh, xsr, stage_slice); break;
+            }
+        } else {
+            switch ((2 * nc + 7) >> 3) {
+                case 1: primed = run13<1, kMode == 2>(ring, cur, nx.w, gs, us, p, xb, stride, sh, xsr, stage_slice); break;
+                case 2: primed = run13<2, kMode == 2>(ring, cur, nx.w, gs, us, p, xb, stride, sh, xsr, stage_slice); break;
+                case 3: primed = run13<3, kMode == 2>(ring, cur, nx.w, gs, us, p, xb, stride, sh, xsr, stage_slice); break;
+                default: primed = run13<4, kMode == 2>(ring, cur, nx.w, gs, us, p, xb, stride, sh, xsr, stage_slice); break;
+            }
         }
         if (kMode == 1 && nx.ok) stage13(p, sh, nx, xs, stride, sh.xsr[0]);
         cur = nx;

@@ -310,13 +310,20 @@ __device__ __forceinline__ void reset_ctrl(const Params& p) {
 // of e in earlier groups) + rank, i.e. buckets list their tokens in (t, k)
 // order.
 // ---------------------------------------------------------------------------
-// The group's activations are staged in shared memory up to this hidden size.
-constexpr int kRouterXMaxH = 2048;
+// The group's activations are staged in (dynamic) shared memory up to this
+// hidden size.
+constexpr int kRouterXMaxH = 12288;
+constexpr int kRouterWarps = 16;
+constexpr int kRouterBatch = 8;  // router-weight blocks per batch of loads
+size_t router_decode_smem(int H) {
+    return H <= kRouterXMaxH ? (size_t)kDecodeRouterTok * H * sizeof(__nv_bfloat16) : 0;
+}
 
-__global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(256) router_decode_kernel(Params p) {
+__global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(32 * kRouterWarps, 1)
+    router_decode_kernel(Params p) {
     namespace cg = cooperative_groups;
     constexpr int kEpcMax = kMaxE / kDecodeRouterCtas;
-    __shared__ __align__(16) __nv_bfloat16 s_x[kDecodeRouterTok][kRouterXMaxH];
+    extern __shared__ __align__(16) __nv_bfloat16 s_xd[];  // [kDecodeRouterTok][H] when staged
     __shared__ float s_logit[kDecodeRouterTok][kEpcMax];
     __shared__ float s_bias[kMaxE];
     __shared__ int s_pick[kDecodeRouterTok * kMaxK];
@@ -331,18 +338,19 @@ __global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(256)
     const int e_lo = r * epc, e_hi = min(E, e_lo + epc);
     const bool staged = H <= kRouterXMaxH;
     // Nothing below depends on the previous kernel until pdl_wait: the bias,
-    // the first 8 blocks of this warp's first router row (registers) and the
+    // the first batch of this warp's first router row (registers) and the
     // rest of the CTA's rows (L2).
     if (r == 0)
         for (int e = threadIdx.x; e < E; e += blockDim.x) s_bias[e] = __ldg(p.rb + e);
-    float4 wpre[8];
+    float4 wpre[kRouterBatch];
     {
         const int e = e_lo + warp;
         const float4* W = reinterpret_cast<const float4*>(p.rw + (size_t)min(e, E - 1) * H);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) wpre[i] = (e < e_hi && i < nblk) ? __ldg(W + i * 32 + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < kRouterBatch; ++i)
+            wpre[i] = (e < e_hi && i < nblk) ? __ldg(W + i * 32 + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    for (int e = e_lo + warp; e < e_hi; e += 8) {
+    for (int e = e_lo + warp; e < e_hi; e += kRouterWarps) {
         const char* wrow = reinterpret_cast<const char*>(p.rw + (size_t)e * H);
         for (int l = lane; l < H * 4 / 128; l += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(wrow + l * 128));
     }
@@ -354,7 +362,7 @@ __global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(256)
         for (int c = threadIdx.x; c < nt * per; c += blockDim.x) {
             const int tt = c / per, k = c - tt * per;
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(
-                             __cvta_generic_to_shared(&s_x[tt][k * 8]))),
+                             __cvta_generic_to_shared(s_xd + (size_t)tt * H + k * 8))),
                          "l"(p.x + (size_t)(t0 + tt) * H + k * 8)
                          : "memory");
         }
@@ -364,38 +372,32 @@ __global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(256)
     }
     auto xblock = [&](int tt, int i) -> uint2 {
         if (tt >= nt) return make_uint2(0u, 0u);
-        if (staged) return *reinterpret_cast<const uint2*>(&s_x[tt][i * 128 + lane * 4]);
+        if (staged) return *reinterpret_cast<const uint2*>(s_xd + (size_t)tt * H + i * 128 + lane * 4);
         return __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)(t0 + tt) * H + i * 128 + lane * 4));
     };
-    for (int e = e_lo + warp, j = 0; e < e_hi; e += 8, ++j) {
+    for (int e = e_lo + warp, j = 0; e < e_hi; e += kRouterWarps, ++j) {
         float acc[kDecodeRouterTok];
 #pragma unroll
         for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = 0.f;
         const float4* W = reinterpret_cast<const float4*>(p.rw + (size_t)e * H);
-        int i_first = 0;
-        if (j == 0) {  // the prefetched blocks
+        // batches of kRouterBatch blocks; the next batch is in flight while this one is used
+        float4 cur[kRouterBatch], nxt[kRouterBatch];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (i < nblk)
+        for (int u = 0; u < kRouterBatch; ++u)
+            cur[u] = j == 0 ? wpre[u] : (u < nblk ? __ldg(W + u * 32 + lane) : make_float4(0.f, 0.f, 0.f, 0.f));
+        for (int i0 = 0; i0 < nblk; i0 += kRouterBatch) {
 #pragma unroll
-                    for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = dot_step(acc[tt], xblock(tt, i), wpre[i]);
-            i_first = 8;
-        }
-        for (int i0 = i_first; i0 < nblk; i0 += 4) {
-            float4 wv[4];
-            uint2 xv[4][kDecodeRouterTok];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i = i0 + u;
-                wv[u] = i < nblk ? __ldg(W + i * 32 + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int tt = 0; tt < kDecodeRouterTok; ++tt) xv[u][tt] = i < nblk ? xblock(tt, i) : make_uint2(0u, 0u);
+            for (int u = 0; u < kRouterBatch; ++u) {
+                const int i = i0 + kRouterBatch + u;
+                nxt[u] = i < nblk ? __ldg(W + i * 32 + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < kRouterBatch; ++u)
                 if (i0 + u < nblk)
 #pragma unroll
-                    for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = dot_step(acc[tt], xv[u][tt], wv[u]);
+                    for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = dot_step(acc[tt], xblock(tt, i0 + u), cur[u]);
+#pragma unroll
+            for (int u = 0; u < kRouterBatch; ++u) cur[u] = nxt[u];
         }
 #pragma unroll
         for (int tt = 0; tt < kDecodeRouterTok; ++tt) {
@@ -436,7 +438,7 @@ __global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(256)
         // token tt of the group is quantized by CTA max(tt, 1), warp (tt == 0)
         for (int tt = 0; tt < nt; ++tt)
             if (r == max(tt, 1) && warp == (tt == 0 ? 1 : 0))
-                quantize_x_row(p, t0 + tt, staged ? &s_x[tt][0] : p.x + (size_t)(t0 + tt) * H, lane);
+                quantize_x_row(p, t0 + tt, staged ? s_xd + (size_t)tt * H : p.x + (size_t)(t0 + tt) * H, lane);
     }
     cluster.sync();  // the remote reads of CTA 0 are done before any CTA exits
 }
@@ -703,8 +705,19 @@ __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
 
 cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream) {
     cudaError_t err;
-    if (small_path)
-        return launch_pdl(router_decode_kernel, dim3(p.decode_groups, kDecodeRouterCtas), dim3(256), 0, stream, p);
+    if (small_path) {
+        const size_t smem = router_decode_smem(p.H);
+        static int attr_set[64];
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 && !attr_set[dev]) {
+            const cudaError_t e = cudaFuncSetAttribute(router_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)router_decode_smem(kRouterXMaxH));
+            if (e != cudaSuccess) return e;
+            attr_set[dev] = 1;
+        }
+        return launch_pdl(router_decode_kernel, dim3(p.decode_groups, kDecodeRouterCtas), dim3(32 * kRouterWarps),
+                          smem, stream, p);
+    }
     err = launch_pdl(router_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
     if (err == cudaSuccess) err = launch_pdl(router_finalize_kernel, dim3(1), dim3(1024), 0, stream, p);
     if (err == cudaSuccess) err = launch_pdl(scatter_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
