@@ -217,6 +217,15 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
         p.nsl_s = slices_of(cfg->Is);
     }
     p.decode_groups = small ? cdiv(T, kDecodeRouterTok) : 0;
+    // down tasks of large hidden sizes cover several 128-row groups, so that a
+    // task streams enough weight bytes to outweigh its per-task costs
+    {
+        const int groups = cfg->H / kTaskRows2, want = cfg->H / 1024 > 1 ? cfg->H / 1024 : 1;
+        int rg = 1;
+        for (int c : {8, 6, 4, 3, 2})
+            if (c <= want && groups % c == 0) { rg = c; break; }
+        p.rows2 = kTaskRows2 * rg;
+    }
     const int ntiles = cdiv(T, kRouterTileTokens);
     p.router_blocks = ntiles < kRouterMaxBlocks ? ntiles : kRouterMaxBlocks;
 
@@ -226,7 +235,7 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
     const long long shared_chunks = cfg->Is > 0 ? cdiv(T, kChunkTokens) : 0;
     // upper bounds of the weight-streaming kernels' CTA tasks
     const long long tasks13 = (long long)(cfg->I / 64) * routed_buckets + (long long)(cfg->Is / 64) * shared_chunks;
-    const long long tasks2 = (long long)(cfg->H / 128) *
+    const long long tasks2 = (long long)(cfg->H / p.rows2) *
                              (routed_buckets * slices_of(cfg->I) + shared_chunks * slices_of(cfg->Is));
     int grid13 = 0, grid2 = 0;
     if (!use_tc) {

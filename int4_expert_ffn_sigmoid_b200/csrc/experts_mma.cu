@@ -119,7 +119,8 @@ static_assert(kRingWholeBytes >= (size_t)kStageRows * (kXRing * 128 + kPadB), "r
 // down: int8 staging of one slice + the next task's f32 slice
 constexpr int kStride2 = kSliceK + kPadB;
 constexpr size_t kRaw2Off = (size_t)kStageRows * kStride2;
-constexpr size_t kSmem2 = kShmBytes + kRaw2Off + (size_t)kChunkTokens * kSliceK * 4;
+constexpr size_t kRs2Off = kRaw2Off + (size_t)kChunkTokens * kSliceK * 4;  // row scales [2][kMaxRows2]
+constexpr size_t kSmem2 = kShmBytes + kRs2Off + (size_t)2 * kMaxRows2 * 4;
 
 // The bucket list and task prefix that the router wrote to the workspace,
 // and (for at most kMaxSlots routed slots) the token of every slot.
@@ -184,7 +185,7 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
         // lane l owns experts 8l .. 8l+7: counts, non-empty buckets, gate/up
         // and down tasks, scanned across the warp in one pass
         constexpr int kPer = kMaxE / 32;
-        const int R13 = p.I / kTaskRows13, R2 = (p.H / kTaskRows2) * slices_of(p.I);
+        const int R13 = p.I / kTaskRows13, R2 = (p.H / p.rows2) * slices_of(p.I);
         int c[kPer];
         int v[4] = {0, 0, 0, 0};  // slots, buckets, gate/up tasks, down tasks
 #pragma unroll
@@ -249,7 +250,7 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
                     p.ts2[nb] = t2;
                 }
                 t13 += (p.Is / kTaskRows13) * chunks_of(T);
-                t2 += (p.H / kTaskRows2) * slices_of(p.Is) * chunks_of(T);
+                t2 += (p.H / p.rows2) * slices_of(p.Is) * chunks_of(T);
                 ++nb;
             }
             tb.ts[nb] = t13;
@@ -469,7 +470,7 @@ __device__ __forceinline__ TaskDesc decode_task(const Params& p, const Tables& t
         c = local / R;
         d.rbk = local - c * R;
     } else {
-        const int R = p.H / kRows2, nsl = slices_of(irow);
+        const int R = p.H / p.rows2, nsl = slices_of(irow);
         const int rest = local / R;
         d.rbk = local - rest * R;
         c = rest / nsl;
@@ -904,11 +905,12 @@ __global__ void __launch_bounds__(256, 1) experts_w13_bulk_kernel(Params p) {
     cp_async_wait<0>();
 }
 
-// One down task as this thread sees it.
+// One down task as this thread sees it: ng row groups of 128 rows starting
+// at row0; in group m this thread streams rows row0 + 128 m + j0 + g and + 8.
 struct Task2 {
-    WStream w;  // down rows j0 + g and j0 + g + 8, from the slice's first k block
+    WStream w;  // this thread's rows of group 0, from the slice's first k block
     bool ok, shared;
-    int e, off, irow, sl, k0, klen, tok0, nc, j0;
+    int e, off, irow, sl, k0, klen, tok0, nc, j0, row0, ng;
 };
 
 // Down task `local` of bucket (e, n, off).
@@ -920,7 +922,7 @@ __device__ __forceinline__ Task2 make2(const Params& p, int e, int n, int off, i
     t.e = e;
     t.off = off;
     t.irow = t.shared ? p.Is : p.I;
-    const int R = p.H / kRows2, nsl = slices_of(t.irow);
+    const int R = p.H / p.rows2, nsl = slices_of(t.irow);
     const int rbk = local % R, rest = local / R;
     t.sl = rest % nsl;
     const int c = rest / nsl;
@@ -928,11 +930,13 @@ __device__ __forceinline__ Task2 make2(const Params& p, int e, int n, int off, i
     t.klen = min(kSliceK, t.irow - t.k0);
     t.tok0 = c * kChunkTokens;
     t.nc = min(kChunkTokens, n - t.tok0);
-    t.j0 = rbk * kRows2 + warp * 16;
+    t.row0 = rbk * p.rows2;
+    t.ng = p.rows2 / kRows2;
+    t.j0 = warp * 16;
     const int row_bytes = t.irow / 2;
     const uint8_t* W = t.shared ? p.sh_w2 : p.w2 + (size_t)(t.ok ? e : 0) * p.H * row_bytes;
-    t.w.ra = W + (size_t)(t.j0 + g) * row_bytes + t.k0 / 2 + q * 16;
-    t.w.rb = W + (size_t)(t.j0 + g + 8) * row_bytes + t.k0 / 2 + q * 16;
+    t.w.ra = W + (size_t)(t.row0 + t.j0 + g) * row_bytes + t.k0 / 2 + q * 16;
+    t.w.rb = W + (size_t)(t.row0 + t.j0 + g + 8) * row_bytes + t.k0 / 2 + q * 16;
     t.w.nkb = t.ok ? t.klen / 128 : 0;
     return t;
 }
@@ -952,11 +956,13 @@ __device__ __forceinline__ Task2 task2_from(const Params& p, const TaskDesc& d) 
     t.klen = min(kSliceK, t.irow - t.k0);
     t.tok0 = d.tok0;
     t.nc = d.nc;
-    t.j0 = d.rbk * kRows2 + warp * 16;
+    t.row0 = d.rbk * p.rows2;
+    t.ng = p.rows2 / kRows2;
+    t.j0 = warp * 16;
     const int row_bytes = t.irow / 2;
     const uint8_t* W = t.shared ? p.sh_w2 : p.w2 + (size_t)(t.ok ? d.e : 0) * p.H * row_bytes;
-    t.w.ra = W + (size_t)(t.j0 + g) * row_bytes + t.k0 / 2 + q * 16;
-    t.w.rb = W + (size_t)(t.j0 + g + 8) * row_bytes + t.k0 / 2 + q * 16;
+    t.w.ra = W + (size_t)(t.row0 + t.j0 + g) * row_bytes + t.k0 / 2 + q * 16;
+    t.w.rb = W + (size_t)(t.row0 + t.j0 + g + 8) * row_bytes + t.k0 / 2 + q * 16;
     t.w.nkb = t.ok ? t.klen / 128 : 0;
     return t;
 }
@@ -965,9 +971,12 @@ __device__ __forceinline__ Task2 task2_r(const Params& p, const Shm& sh, int r) 
     return task2_from(p, task_desc(p, sh, 1, r));
 }
 
-// Issues the cp.async of task t's f32 slice of h (raw[j][k], k < klen) and of
-// its per-64-row maxima of |h| (sh.hmr), as one group.
-__device__ __forceinline__ void fetch2(const Params& p, Shm& sh, const Task2& t, float* raw) {
+// Issues the cp.async of task t's f32 slice of h (raw[j][k], k < klen), of
+// its per-64-row maxima of |h| (sh.hmr) and of its row scales (rs), as one
+// group.
+__device__ __forceinline__ void fetch2(const Params& p, Shm& sh, const Task2& t, float* raw, float* rs) {
+    const float* S = (t.shared ? p.sh_s2 : p.s2 + (size_t)t.e * p.H) + t.row0;
+    for (int c = threadIdx.x; c < p.rows2 / 4; c += blockDim.x) cp_async16(rs + 4 * c, S + 4 * c);
     const float* hb = t.shared ? p.h32_s : p.h32_r;
     const float* hmb = t.shared ? p.hmax_s : p.hmax_r;
     const int nrb = t.irow / kRows13;
@@ -986,22 +995,38 @@ __device__ __forceinline__ void fetch2(const Params& p, Shm& sh, const Task2& t,
 }
 
 template <int NT>
-__device__ __forceinline__ bool run2(Ring& ring, const Task2& tk, const WStream& nx, float s_lo, float s_hi,
-                                     const Params& p, const uint8_t* xs, const Shm& sh) {
+__device__ __forceinline__ bool run2(Ring& ring, const Task2& tk, const WStream& nx, const float* rs, const Params& p,
+                                     const uint8_t* xs, const Shm& sh) {
     const int g = (threadIdx.x & 31) >> 2, q = (threadIdx.x & 31) & 3;
-    int acc[NT][4];
-    const bool cont = stream8<NT, false>(ring, tk.w, nx, xs, kStride2, [](int) {}, acc);
     const size_t TK = (size_t)p.T * p.K;
     const size_t yrow0 = tk.shared ? TK * p.nsl_r + (size_t)tk.sl * p.T + tk.tok0 : (size_t)tk.sl * TK + tk.off + tk.tok0;
-    float* y0 = p.y + yrow0 * p.H + tk.j0 + g;
+    const size_t group_bytes = (size_t)kRows2 * (tk.irow / 2);
+    bool cont = false;
+    for (int m = 0; m < tk.ng; ++m) {
+        WStream cur = tk.w;
+        cur.ra += m * group_bytes;
+        cur.rb += m * group_bytes;
+        WStream nxt = nx;
+        if (m + 1 < tk.ng) {
+            nxt = tk.w;
+            nxt.ra += (m + 1) * group_bytes;
+            nxt.rb += (m + 1) * group_bytes;
+        }
+        int acc[NT][4];
+        cont = stream8<NT, false>(ring, cur, nxt, xs, kStride2, [](int) {}, acc);
+        if (!cont && m + 1 < tk.ng) prime(ring, nxt);
+        const int jr = m * kRows2 + tk.j0 + g;  // row of this thread within the task
+        const float s_lo = rs[jr], s_hi = rs[jr + 8];
+        float* y0 = p.y + yrow0 * p.H + tk.row0 + jr;
 #pragma unroll
-    for (int i = 0; i < NT; ++i) {
-        const int j = 4 * i + q;
-        if (j < tk.nc) {
-            const float xsc = sh.xsc[j];
-            float* yr = y0 + (size_t)j * p.H;
-            yr[0] = join(acc[i][0], acc[i][1]) * (s_lo * xsc);
-            yr[8] = join(acc[i][2], acc[i][3]) * (s_hi * xsc);
+        for (int i = 0; i < NT; ++i) {
+            const int j = 4 * i + q;
+            if (j < tk.nc) {
+                const float xsc = sh.xsc[j];
+                float* yr = y0 + (size_t)j * p.H;
+                yr[0] = join(acc[i][0], acc[i][1]) * (s_lo * xsc);
+                yr[8] = join(acc[i][2], acc[i][3]) * (s_hi * xsc);
+            }
         }
     }
     return cont;
@@ -1012,10 +1037,10 @@ __global__ void __launch_bounds__(256, 2) experts_w2_kernel(Params p) {
     Shm& sh = *reinterpret_cast<Shm*>(dsm);
     uint8_t* xs = dsm + kShmBytes;
     float* raw = reinterpret_cast<float*>(xs + kRaw2Off);
+    float* rs2 = reinterpret_cast<float*>(xs + kRs2Off);  // [task parity][row of the task]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2;
     Ring ring;
-    const int ns = p.Is > 0 ? (p.H / kRows2) * chunks_of(p.T) * slices_of(p.Is) : 0;
+    const int ns = p.Is > 0 ? (p.H / p.rows2) * chunks_of(p.T) * slices_of(p.Is) : 0;
     bool primed = false;
     const uint8_t* primed_ra = nullptr;
     if ((int)blockIdx.x < ns) {
@@ -1032,9 +1057,7 @@ __global__ void __launch_bounds__(256, 2) experts_w2_kernel(Params p) {
     const Tables& tb = sh.tb;
     Task2 cur = task2_r(p, sh, 0);
     if (primed && cur.w.ra != primed_ra) primed = false;
-    if (cur.ok) fetch2(p, sh, cur, raw);
-    const float* S = cur.shared ? p.sh_s2 : p.s2 + (size_t)cur.e * p.H;
-    float s_lo = cur.ok ? __ldg(S + cur.j0 + g) : 0.f, s_hi = cur.ok ? __ldg(S + cur.j0 + g + 8) : 0.f;
+    if (cur.ok) fetch2(p, sh, cur, raw, rs2);
     for (int r = 0, lin = blockIdx.x; lin < tb.ntask; lin = snake(blockIdx.x, ++r)) {
         const Task2 nx = task2_r(p, sh, r + 1);
         if (!cur.ok) {  // a table entry out of range: flag it and stop
@@ -1068,22 +1091,15 @@ __global__ void __launch_bounds__(256, 2) experts_w2_kernel(Params p) {
             }
         }
         __syncthreads();  // staged; raw and hmr are free for the next task
-        if (nx.ok) fetch2(p, sh, nx, raw);
-        float s_lo_n = 0.f, s_hi_n = 0.f;
-        if (nx.ok) {
-            const float* Sn = nx.shared ? p.sh_s2 : p.s2 + (size_t)nx.e * p.H;
-            s_lo_n = __ldg(Sn + nx.j0 + g);
-            s_hi_n = __ldg(Sn + nx.j0 + g + 8);
-        }
+        if (nx.ok) fetch2(p, sh, nx, raw, rs2 + ((r + 1) & 1) * kMaxRows2);
+        const float* rs = rs2 + (r & 1) * kMaxRows2;
         switch ((2 * nc + 7) >> 3) {
-            case 1: primed = run2<1>(ring, cur, nx.w, s_lo, s_hi, p, xs, sh); break;
-            case 2: primed = run2<2>(ring, cur, nx.w, s_lo, s_hi, p, xs, sh); break;
-            case 3: primed = run2<3>(ring, cur, nx.w, s_lo, s_hi, p, xs, sh); break;
-            default: primed = run2<4>(ring, cur, nx.w, s_lo, s_hi, p, xs, sh); break;
+            case 1: primed = run2<1>(ring, cur, nx.w, rs, p, xs, sh); break;
+            case 2: primed = run2<2>(ring, cur, nx.w, rs, p, xs, sh); break;
+            case 3: primed = run2<3>(ring, cur, nx.w, rs, p, xs, sh); break;
+            default: primed = run2<4>(ring, cur, nx.w, rs, p, xs, sh); break;
         }
         cur = nx;
-        s_lo = s_lo_n;
-        s_hi = s_hi_n;
     }
 }
 

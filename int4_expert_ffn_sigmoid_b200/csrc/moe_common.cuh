@@ -11,9 +11,11 @@ namespace moe {
 
 // Largest T that takes the weight-streaming (small-batch) path by default.
 constexpr int kDecodeMaxTokens = 64;
-// Rows of one weight-streaming task: gate/up (each with its up row), down.
+// Rows of one weight-streaming task: gate/up (each with its up row); one
+// row group of a down task (a down task has Params::rows2 rows, a multiple).
 constexpr int kTaskRows13 = 64;
 constexpr int kTaskRows2 = 128;
+constexpr int kMaxRows2 = 1024;
 // Tokens of one bucket handled by one weight-streaming task: each token
 // takes two int8 columns (its two activation parts), so 16 tokens fill four
 // mma n-tiles of 8 columns.
@@ -154,6 +156,7 @@ struct Params {
     float* hmax_r;        // [T*K][I/64] max |h| of each 64-row block
     float* hmax_s;        // [T][Is/64]
     int nsl_r, nsl_s;     // slices of the down projection's reduction (routed, shared)
+    int rows2;            // output rows of one down task (kTaskRows2 times 1..8, dividing H)
     int decode_groups;    // token groups of the small-batch router (0: tables come from the large router)
 };
 
