@@ -453,9 +453,7 @@ def run_ours(args, rank, world, device, dist):
         v, sample = cpu_baseline_sample(stack)
         cpu = {"value": round(v, 2), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
 
-    # small batch: router, gate/up, down, combine; large batch: router, finalize,
-    # scatter, gate/up, down, combine
-    kernels_per_layer = 4 if T <= moe.decode_max_tokens() else 6
+    kernels_per_layer = moe.kernel_launches(wl.shape, T)
     launches = args.steps * L
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -204,6 +204,11 @@ int moe_abi_version(void);
  * (weight-streaming) path when neither MOE_FORCE_* flag is set. */
 int32_t moe_decode_max_tokens(void);
 
+/* Number of kernels one moe_layer_forward call launches for T tokens under
+ * cfg (the stage events are not kernels).  Returns 0 if T = 0 or the call
+ * would be rejected for cfg or T (the pointers in cfg are not looked at). */
+int32_t moe_layer_kernel_launches(const moe_cfg_t* cfg, int32_t T);
+
 #ifdef __cplusplus
 }
 #endif

@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "MoeError", "moe_cfg_t", "moe_shared_weights_t", "lib", "EXPORTED_SYMBOLS",
     "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK", "MOE_FORCE_DECODE", "MOE_FORCE_PREFILL", "MOE_OUT_F32",
-    "workspace_bytes", "layer_forward", "MoELayer", "decode_max_tokens", "LIB_PATH",
+    "workspace_bytes", "layer_forward", "MoELayer", "decode_max_tokens", "kernel_launches", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_int4.so")
@@ -43,7 +43,8 @@ STAGE_NAMES = ("route", "gate_up", "down", "combine")
 
 # Every function declared in include/moe_int4.h.
 EXPORTED_SYMBOLS = ("moe_layer_workspace_bytes", "moe_layer_forward", "moe_status_str",
-                    "moe_abi_version", "moe_decode_max_tokens", "moe_layer_forward_static_ws")
+                    "moe_abi_version", "moe_decode_max_tokens", "moe_layer_forward_static_ws",
+                    "moe_layer_kernel_launches")
 
 # Scratch capacity of moe_layer_forward_static_ws (the entry point for callers
 # that cannot allocate device memory).
@@ -88,6 +89,8 @@ def _load() -> ctypes.CDLL:
     L.moe_abi_version.restype = ctypes.c_int
     L.moe_decode_max_tokens.argtypes = []
     L.moe_decode_max_tokens.restype = ctypes.c_int32
+    L.moe_layer_kernel_launches.argtypes = [ctypes.POINTER(moe_cfg_t), ctypes.c_int32]
+    L.moe_layer_kernel_launches.restype = ctypes.c_int32
     if L.moe_abi_version() != 1:
         raise ImportError("libmoe_int4.so ABI version mismatch")
     return L
@@ -128,6 +131,12 @@ def make_cfg(shape, flags: int = 0, workspace: Optional[torch.Tensor] = None,
         c._events_keepalive = arr
         c.stage_events = ctypes.cast(arr, ctypes.c_void_p).value
     return c
+
+
+def kernel_launches(shape, T: int, flags: int = 0) -> int:
+    """Kernels one layer_forward call launches for T tokens (0: invalid)."""
+    c = make_cfg(shape, flags)
+    return int(lib.moe_layer_kernel_launches(ctypes.byref(c), int(T)))
 
 
 def workspace_bytes(shape, T: int, flags: int = 0) -> int:

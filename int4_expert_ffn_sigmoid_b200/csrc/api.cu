@@ -32,7 +32,7 @@ Path choose_path(const moe_cfg_t& c, int32_t T) {
 
 struct WsLayout {
     size_t ctrl, idx, wts, counts, offsets, bucket_e, bucket_n, bucket_off, ts13, ts2, tcs1, tcs2;
-    size_t tok_of_slot, slot_of, hist, rank, hexp, y;
+    size_t tok_of_slot, slot_of, hist, rank, hexp, y, lpart;
     size_t h_r, h_s, x_perm;                            // tensor-core path
     size_t xq, xs, h32_r, h32_s, hmax_r, hmax_s;        // weight-streaming paths
     size_t total;
@@ -65,6 +65,7 @@ WsLayout ws_layout(const moe_cfg_t& c, int32_t T) {
     L.hist = take((size_t)kRouterMaxBlocks * E * 4);
     L.rank = take(TK * 4);
     L.hexp = take((size_t)T * 4);
+    L.lpart = take((size_t)router_split_slices(c.E, c.H, path == Path::kSmall) * T * E * 4);
     const size_t shared_rows = c.Is > 0 ? (size_t)T : 0;
     if (path == Path::kTensorCore) {
         L.h_r = take(TK * (size_t)c.I * 2);
@@ -121,6 +122,14 @@ extern "C" {
 int moe_abi_version(void) { return MOE_ABI_VERSION; }
 
 int32_t moe_decode_max_tokens(void) { return kDecodeMaxTokens; }
+
+int32_t moe_layer_kernel_launches(const moe_cfg_t* cfg, int32_t T) {
+    if (validate_cfg(cfg) != MOE_OK || T <= 0 || T > kMaxTokens) return 0;
+    // small batch: [router logits,] cluster router, gate/up, down, combine;
+    // otherwise: router, finalize, scatter, gate/up, down, combine
+    if (choose_path(*cfg, T) == Path::kSmall) return router_split_slices(cfg->E, cfg->H, true) > 0 ? 5 : 4;
+    return 6;
+}
 
 const char* moe_status_str(int status) {
     switch (status) {
@@ -217,6 +226,8 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
         p.nsl_s = slices_of(cfg->Is);
     }
     p.decode_groups = small ? cdiv(T, kDecodeRouterTok) : 0;
+    p.lslices = router_split_slices(cfg->E, cfg->H, small);
+    p.lpart = p.lslices > 0 ? static_cast<float*>(at(L.lpart)) : nullptr;
     // down tasks of large hidden sizes cover several 128-row groups, so that a
     // task streams enough weight bytes to outweigh its per-task costs
     {

@@ -158,6 +158,8 @@ struct Params {
     int nsl_r, nsl_s;     // slices of the down projection's reduction (routed, shared)
     int rows2;            // output rows of one down task (kTaskRows2 times 1..8, dividing H)
     int decode_groups;    // token groups of the small-batch router (0: tables come from the large router)
+    float* lpart;         // [lslices][T][E] partial router logits of the split small-batch router
+    int lslices;          // hidden-dimension slices of lpart (0: the small-batch router computes its logits)
 };
 
 // ---------------------------------------------------------------------------

@@ -9,6 +9,9 @@ namespace moe {
 
 // Router + bucketing.  small_path: T <= kDecodeMaxTokens.
 cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream);
+// Hidden-dimension slices of the split small-batch router's partial logits
+// (0: the cluster router computes the logits itself).
+int router_split_slices(int E, int H, bool small_path);
 // Expert gate/up + SwiGLU (weight-streaming mma.sync kernel).
 cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream);
 // Expert down projection (weight-streaming mma.sync kernel).

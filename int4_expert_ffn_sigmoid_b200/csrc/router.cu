@@ -315,9 +315,85 @@ __device__ __forceinline__ void reset_ctrl(const Params& p) {
 constexpr int kRouterXMaxH = 12288;
 constexpr int kRouterWarps = 16;
 constexpr int kRouterBatch = 8;  // router-weight blocks per batch of loads
+// Router weights of at least this many bytes (E * H * 4) are read by a
+// separate logits kernel spread over many SMs (router_logits_kernel) instead
+// of by the clusters' 8 CTAs per token group.
+constexpr size_t kRouterSplitBytes = (size_t)2 << 20;
+constexpr int kLogitSliceBlocks = 3;   // 128-element blocks of the hidden dimension per slice
+constexpr int kLogitCtaExperts = 32;   // experts per CTA (4 per warp)
+
+int router_split_slices(int E, int H, bool small_path) {
+    if (!small_path || (size_t)E * H * 4 < kRouterSplitBytes) return 0;
+    return (H / 128 + kLogitSliceBlocks - 1) / kLogitSliceBlocks;
+}
+
 size_t router_decode_smem(int H) {
     return H <= kRouterXMaxH ? (size_t)kDecodeRouterTok * H * sizeof(__nv_bfloat16) : 0;
 }
+
+// Split small-batch router, first kernel: CTA (s, b) computes, for every
+// token, the partial logits over hidden slice s (blocks s*kLogitSliceBlocks
+// onwards, 128 elements each) of experts [32 b, 32 b + 32): warp w takes
+// experts 32 b + 4 w .. + 3 and holds their weights of the slice in
+// registers (loaded before waiting on the previous kernel); the tokens'
+// activations of the slice are staged in shared memory.  Lane l accumulates
+// the elements 128 i + 4 l + j of the slice (i ascending, then j) and the
+// lanes are summed by the xor-butterfly; the cluster kernel adds the slices
+// in ascending order.  The logit of a token therefore does not depend on the
+// other tokens of the batch.
+__global__ void __launch_bounds__(256) router_logits_kernel(Params p) {
+    extern __shared__ __align__(16) __nv_bfloat16 s_xl[];  // [T][kLogitSliceBlocks * 128]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int E = p.E, H = p.H, T = p.T;
+    const int s = blockIdx.x;
+    const int b0 = s * kLogitSliceBlocks, nb = min(kLogitSliceBlocks, H / 128 - b0);
+    const int e0 = blockIdx.y * kLogitCtaExperts + warp * 4;
+    constexpr int kW = kLogitSliceBlocks * 128;
+    float4 w[4][kLogitSliceBlocks];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int i = 0; i < kLogitSliceBlocks; ++i)
+            w[u][i] = (e0 + u < E && i < nb)
+                          ? __ldg(reinterpret_cast<const float4*>(p.rw + (size_t)(e0 + u) * H + (b0 + i) * 128) + lane)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    pdl_wait();
+    pdl_release();
+    const int per = nb * 16;  // 16-byte chunks of a token's slice
+    for (int c = threadIdx.x; c < T * per; c += blockDim.x) {
+        const int t = c / per, k = c - t * per;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(
+                         __cvta_generic_to_shared(s_xl + (size_t)t * kW + k * 8))),
+                     "l"(p.x + (size_t)t * H + b0 * 128 + k * 8)
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    if (e0 >= E) return;
+    for (int t = 0; t < T; ++t) {
+        uint2 xv[kLogitSliceBlocks];
+#pragma unroll
+        for (int i = 0; i < kLogitSliceBlocks; ++i)
+            xv[i] = i < nb ? *reinterpret_cast<const uint2*>(s_xl + (size_t)t * kW + i * 128 + lane * 4)
+                           : make_uint2(0u, 0u);
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < kLogitSliceBlocks; ++i)
+                if (i < nb) acc = dot_step(acc, xv[i], w[u][i]);
+            v[u] = warp_sum_tree(acc);
+        }
+        if (lane < 4 && e0 + lane < E) {
+            const float r = lane == 0 ? v[0] : lane == 1 ? v[1] : lane == 2 ? v[2] : v[3];
+            p.lpart[((size_t)s * T + t) * E + e0 + lane] = r;
+        }
+    }
+}
+
+size_t router_logits_smem(int T) { return (size_t)T * kLogitSliceBlocks * 128 * sizeof(__nv_bfloat16); }
 
 __global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(32 * kRouterWarps, 1)
     router_decode_kernel(Params p) {
@@ -337,20 +413,21 @@ __global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(32 *
     const int epc = (E + kDecodeRouterCtas - 1) / kDecodeRouterCtas;
     const int e_lo = r * epc, e_hi = min(E, e_lo + epc);
     const bool staged = H <= kRouterXMaxH;
+    const bool split = p.lslices > 0;  // the logits kernel ran first
     // Nothing below depends on the previous kernel until pdl_wait: the bias,
     // the first batch of this warp's first router row (registers) and the
     // rest of the CTA's rows (L2).
     if (r == 0)
         for (int e = threadIdx.x; e < E; e += blockDim.x) s_bias[e] = __ldg(p.rb + e);
     float4 wpre[kRouterBatch];
-    {
+    if (!split) {
         const int e = e_lo + warp;
         const float4* W = reinterpret_cast<const float4*>(p.rw + (size_t)min(e, E - 1) * H);
 #pragma unroll
         for (int i = 0; i < kRouterBatch; ++i)
             wpre[i] = (e < e_hi && i < nblk) ? __ldg(W + i * 32 + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    for (int e = e_lo + warp; e < e_hi; e += kRouterWarps) {
+    for (int e = e_lo + warp; !split && e < e_hi; e += kRouterWarps) {
         const char* wrow = reinterpret_cast<const char*>(p.rw + (size_t)e * H);
         for (int l = lane; l < H * 4 / 128; l += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(wrow + l * 128));
     }
@@ -375,7 +452,17 @@ __global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(32 *
         if (staged) return *reinterpret_cast<const uint2*>(s_xd + (size_t)tt * H + i * 128 + lane * 4);
         return __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)(t0 + tt) * H + i * 128 + lane * 4));
     };
-    for (int e = e_lo + warp, j = 0; e < e_hi; e += kRouterWarps, ++j) {
+    if (split) {  // this CTA's experts: the sum of the slices' partial logits, slice 0 first
+        const int ne = e_hi - e_lo;
+        for (int i = threadIdx.x; i < nt * ne; i += blockDim.x) {
+            const int tt = i / ne, e = e_lo + (i - tt * ne);
+            const float* src = p.lpart + (size_t)(t0 + tt) * E + e;
+            float v = 0.f;
+            for (int sl = 0; sl < p.lslices; ++sl) v += __ldcg(src + (size_t)sl * p.T * E);
+            s_logit[tt][e - e_lo] = v;
+        }
+    }
+    for (int e = e_lo + warp, j = 0; !split && e < e_hi; e += kRouterWarps, ++j) {
         float acc[kDecodeRouterTok];
 #pragma unroll
         for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = 0.f;
@@ -714,6 +801,11 @@ cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream)
                                                        (int)router_decode_smem(kRouterXMaxH));
             if (e != cudaSuccess) return e;
             attr_set[dev] = 1;
+        }
+        if (p.lslices > 0) {
+            const cudaError_t e = launch_pdl(router_logits_kernel, dim3(p.lslices, (p.E + kLogitCtaExperts - 1) / kLogitCtaExperts),
+                                             dim3(256), router_logits_smem(p.T), stream, p);
+            if (e != cudaSuccess) return e;
         }
         return launch_pdl(router_decode_kernel, dim3(p.decode_groups, kDecodeRouterCtas), dim3(32 * kRouterWarps),
                           smem, stream, p);

@@ -159,6 +159,22 @@ def test_max_hidden(moe, cuda_device):
         check(moe, x, layer, shape, layer_cpu=cpu)
 
 
+def test_split_router(moe, cuda_device):
+    """Router weights of 2 MB or more take the split small-batch router (a
+    logits kernel over slices of the hidden dimension, then the cluster
+    selection): a ragged last slice (22 blocks of 128 in slices of 3), E not a
+    multiple of 32, and a token's result independent of the rest of the batch."""
+    shape = workloads.LayerShape(H=2816, E=200, K=6, I=128, Is=128, routed_scaling=2.5)
+    assert moe.kernel_launches(shape, 9) == 5
+    layer = workloads.make_layer(shape, 250, 0, cuda_device)
+    cpu = to_cpu_layer(layer)
+    x = workloads.make_x(shape, 64, 250, device=cuda_device)
+    out, _, _, _ = check(moe, x, layer, shape, layer_cpu=cpu)
+    for t0, sub in ((0, 1), (5, 9), (40, 24)):
+        o1, _, _ = run(moe, x[t0:t0 + sub].contiguous(), layer, shape)
+        assert torch.equal(o1, out[t0:t0 + sub])
+
+
 def test_large_intermediate_values(moe, cuda_device):
     """Inputs around +-300 drive the SwiGLU intermediate to ~1e5 (beyond fp16's
     65504 unless it is stored scaled); outputs stay finite and match."""
