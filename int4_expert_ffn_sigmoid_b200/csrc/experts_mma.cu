@@ -48,8 +48,11 @@
 //    and ranks in its prologue; its CTA 0 also writes them to the workspace
 //    for the down kernel and the combine (on the large-batch path the large
 //    router writes them).
+#include <cuda.h>
+
 #include "moe_common.cuh"
 #include "moe_launch.h"
+#include "moe_tc.h"
 
 namespace moe {
 
@@ -905,6 +908,266 @@ __global__ void __launch_bounds__(256, 1) experts_w13_bulk_kernel(Params p) {
     cp_async_wait<0>();
 }
 
+// ---------------------------------------------------------------------------
+// Gate/up for H > kBulkMaxK with H a multiple of 256: one CTA per SM, a
+// producer warp and 8 consumer warps around a ring of kTmaStages stages.  A
+// stage is one 256-wide k chunk of a task: its 64 gate rows and 64 up rows
+// (two TMA tile loads of 64 rows x 128 bytes with the 128-byte swizzle) and
+// the chunk's activations (both int8 parts of each of the task's tokens,
+// 256 bytes each), which the producer lanes copy with cp.async and whose
+// completion counts on the same mbarrier as the tile loads.  The consumers
+// read their mma fragments from the stage and release it; the producer runs
+// ahead across task boundaries, so the weight stream does not pause between
+// tasks, and a CTA whose first task belongs to the shared expert issues that
+// task's first stages of weights before the router has finished.  Every wait
+// is bounded: a timeout flags ST_TIMEOUT and sets the CTA's abort flag, after
+// which nobody waits any more, the tasks run to their end on whatever the
+// stages hold, and the producer waits (bounded) for its last copies before
+// it exits.
+// ---------------------------------------------------------------------------
+constexpr int kTmaStages = 8;
+constexpr int kTmaChunk = 256;                                 // k elements per stage
+constexpr int kTmaRowBytes = kTmaChunk / 2;                    // 128 bytes of codes per row and stage
+constexpr int kTmaWBytes = 2 * kRows13 * kTmaRowBytes;         // gate + up tiles: 16 KB
+constexpr int kTmaXStride = kTmaChunk + kPadB;                 // staged activation row
+constexpr int kTmaXBytes = kStageRows * kTmaXStride;
+constexpr int kTmaThreads = 288;                               // 8 consumer warps + the producer warp
+constexpr size_t kTmaMiscBytes = 256 + 2 * 8 * kChunkTokens * 4;  // barriers, flag, per-warp maxima
+constexpr size_t kSmem13Tma = kShmBytes + kTmaMiscBytes + 1024 /* alignment */ +
+                              (size_t)kTmaStages * (kTmaWBytes + kTmaXBytes);
+static_assert(kSmem13Tma <= 227 * 1024, "TMA gate/up shared memory");
+static_assert((size_t)kTmaStages * kTmaXBytes >= kBuildBytes, "table build scratch fits the activation ring");
+
+__device__ __forceinline__ void bar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar)))
+                 : "memory");
+}
+// Arrives on bar once every cp.async this thread issued so far has landed.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(bar)))
+                 : "memory");
+}
+__device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar))), "r"(x), "r"(y)
+        : "memory");
+}
+// The weights of k chunk c of a task whose gate rows start at row rg and up
+// rows at ru of `map`: expect the bytes, then the two tile loads.
+__device__ __forceinline__ void issue_w13_chunk(const CUtensorMap* map, uint64_t* bar, uint8_t* dst, int c, int rg,
+                                                int ru) {
+    bar_expect_tx(bar, kTmaWBytes);
+    tma_tile(dst, map, bar, c * kTmaRowBytes, rg);
+    tma_tile(dst + kTmaWBytes / 2, map, bar, c * kTmaRowBytes, ru);
+}
+
+// Consumer main loop of one task: nch stages from stage counter n on.
+template <int NT>
+__device__ __forceinline__ void consume13(int nch, uint32_t& n, uint64_t* full, uint64_t* empty, const uint8_t* wring,
+                                          const uint8_t* xring, volatile int* abort, unsigned* status,
+                                          int (&acc)[NT][4]) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, q = lane & 3;
+    constexpr int kSets = NT == 1 ? 2 : 1;
+    int part[kSets][NT][4];
+#pragma unroll
+    for (int s = 0; s < kSets; ++s)
+#pragma unroll
+        for (int i = 0; i < NT; ++i) part[s][i][0] = part[s][i][1] = part[s][i][2] = part[s][i][3] = 0;
+    // row warp*8 + g of a 1024-byte aligned tile: its 16-byte chunk j sits at j ^ g
+    const int wrow = (warp * 8 + g) * kTmaRowBytes;
+    for (int c = 0; c < nch; ++c, ++n) {
+        const int s = n % kTmaStages;
+        if (!*abort && !bar_wait(full + s, (n / kTmaStages) & 1, kBulkWaitCycles)) {
+            *abort = 1;
+            if (lane == 0) atomicOr(status, ST_TIMEOUT);
+        }
+        const uint8_t* wt = wring + (size_t)s * kTmaWBytes + wrow;
+        const uint8_t* xt = xring + (size_t)s * kTmaXBytes + g * kTmaXStride + q * 32;
+#pragma unroll
+        for (int kb = 0; kb < kTmaChunk / 128; ++kb) {
+            const int off = ((kb * 4 + q) ^ g) << 4;
+            const uint4 wa = *reinterpret_cast<const uint4*>(wt + off);
+            const uint4 wb = *reinterpret_cast<const uint4*>(wt + kTmaWBytes / 2 + off);
+            kblock8<NT, kSets>(wa, wb, xt + kb * 128, 8 * kTmaXStride, part);
+        }
+        __syncwarp();
+        if (lane == 0) bar_arrive(empty + s);
+    }
+#pragma unroll
+    for (int i = 0; i < NT; ++i)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[i][c] = part[0][i][c] + part[kSets - 1][i][c] * (kSets - 1);
+}
+
+__global__ void __launch_bounds__(kTmaThreads, 1)
+    experts_w13_tma_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_s, Params p) {
+    extern __shared__ __align__(128) uint8_t dsm[];
+    Shm& sh = *reinterpret_cast<Shm*>(dsm);
+    uint64_t* full = reinterpret_cast<uint64_t*>(dsm + kShmBytes);
+    uint64_t* empty = full + kTmaStages;
+    volatile int* abort = reinterpret_cast<volatile int*>(empty + kTmaStages);
+    float(*hm2)[8][kChunkTokens] = reinterpret_cast<float(*)[8][kChunkTokens]>(dsm + kShmBytes + 256);
+    const uint32_t base_s = static_cast<uint32_t>(__cvta_generic_to_shared(dsm));
+    const uint32_t ring_s = (base_s + (uint32_t)(kShmBytes + kTmaMiscBytes) + 1023u) & ~1023u;
+    uint8_t* wring = dsm + (ring_s - base_s);
+    uint8_t* xring = wring + (size_t)kTmaStages * kTmaWBytes;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const bool producer = warp == 8;
+    const int H = p.H, nch = H / kTmaChunk;
+    unsigned* status = &p.ctrl->status;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kTmaStages; ++i) {
+            bar_init(full + i, 1 + 32);  // the tile loads' arrival + one cp.async arrival per producer lane
+            bar_init(empty + i, 8);      // one arrival per consumer warp
+        }
+        *abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    // the shared expert's first task of this CTA, if its first task is one
+    const int ns = p.Is > 0 ? (p.Is / kRows13) * chunks_of(p.T) : 0;
+    const bool pre = (int)blockIdx.x < ns;
+    const int npre = pre ? min(kTmaStages, nch) : 0;
+    int pre_rbk = 0, pre_tok0 = 0;
+    if (pre) {
+        const int R = p.Is / kRows13, local = ns - 1 - (int)blockIdx.x;
+        pre_rbk = local % R;
+        pre_tok0 = (local / R) * kChunkTokens;
+        if (producer && lane == 0)
+            for (int c = 0; c < npre; ++c)
+                issue_w13_chunk(&tm_s, full + c, wring + (size_t)c * kTmaWBytes, c, pre_rbk * kRows13,
+                                p.Is + pre_rbk * kRows13);
+    }
+    if (p.Is > 0) prefetch_l2_slice(p.sh_w13, (size_t)p.Is * p.H);
+    pdl_wait();
+    pdl_release();
+    if (p.decode_groups > 0) build_tables_small(p, sh, reinterpret_cast<int*>(xring));
+    else load_tables(p, p.ts13, &p.ctrl->tasks13, sh.tb, sh.tok);
+    precompute_tasks(p, sh, 0);
+    if (threadIdx.x == 0 && pre) {  // cannot fail with consistent tables
+        const TaskDesc d = sh.td[0];
+        if (!(d.e == p.E && d.rbk == pre_rbk && d.tok0 == pre_tok0 && sh.tb.ntask > (int)blockIdx.x)) {
+            *abort = 1;
+            atomicOr(status, ST_BAD_TASK);
+        }
+    }
+    __syncthreads();
+    const int ntask = sh.tb.ntask;
+    if (!producer && *abort) return;
+    if (producer) {
+        uint32_t n = 0;
+        int last_round[kTmaStages];
+#pragma unroll
+        for (int s = 0; s < kTmaStages; ++s) last_round[s] = s < npre ? 0 : -1;
+        for (int r = 0; !*abort && snake(blockIdx.x, r) < ntask; ++r) {
+            const TaskDesc d = task_desc(p, sh, 0, r);
+            if (d.e < 0 || d.e > p.E || (d.e == p.E && p.Is == 0)) break;  // the consumers flag it
+            const bool shared = d.e == p.E;
+            const int irow = shared ? p.Is : p.I;
+            const int rg = (shared ? 0 : d.e * 2 * p.I) + d.rbk * kRows13, ru = rg + irow;
+            // lane l < 2 nc copies activation row l (part l & 1 of the chunk's token l >> 1)
+            const int8_t* src = nullptr;
+            if (lane < 2 * d.nc) {
+                const int tok = slot_token(p, sh, shared, d.off, d.tok0 + (lane >> 1));
+                if (tok >= 0 && tok < p.T) src = p.xq + (size_t)tok * 2 * H + (lane & 1) * H;
+            }
+            for (int c = 0; c < nch; ++c, ++n) {
+                const int s = n % kTmaStages;
+                const int round = (int)(n / kTmaStages);
+                const bool issued = r == 0 && c < npre;  // weights issued before the wait
+                if (round > 0) {
+                    bool ok = *abort == 0 && bar_wait(empty + s, (round - 1) & 1, kBulkWaitCycles);
+                    if (__any_sync(0xffffffffu, !ok)) {
+                        if (lane == 0 && !*abort) atomicOr(status, ST_TIMEOUT);
+                        *abort = 1;
+                        break;
+                    }
+                }
+                if (lane == 0 && !issued)
+                    issue_w13_chunk(shared ? &tm_s : &tm_r, full + s, wring + (size_t)s * kTmaWBytes, c, rg, ru);
+                if (src) {
+                    uint8_t* dst = xring + (size_t)s * kTmaXBytes + lane * kTmaXStride;
+#pragma unroll
+                    for (int j = 0; j < kTmaChunk / 16; ++j) cp_async16(dst + j * 16, src + c * kTmaChunk + j * 16);
+                }
+                cp_async_arrive(full + s);
+                last_round[s] = round;
+            }
+        }
+        // stages issued before an abort that nobody consumed: their arrivals
+        // (pre-issued weights) and their copies land before the CTA exits
+        if (*abort) {
+            for (int s = 0; s < npre; ++s)
+                if (last_round[s] == 0 && n <= (uint32_t)s) cp_async_arrive(full + s);
+            for (int s = 0; s < kTmaStages; ++s)
+                if (last_round[s] >= 0) bar_wait(full + s, last_round[s] & 1, kBulkWaitCycles);
+        }
+        cp_async_wait<0>();
+        return;
+    }
+    // consumers
+    uint32_t n = 0;
+    for (int r = 0; snake(blockIdx.x, r) < ntask; ++r) {
+        const Task13 t = task13_r(p, sh, r);
+        if (!t.ok) {
+            if (threadIdx.x == 0) atomicOr(status, ST_BAD_TASK);
+            break;
+        }
+        const float* S = t.shared ? p.sh_s13 : p.s13 + (size_t)t.e * 2 * p.I;
+        const float gs = __ldg(S + t.r0 + g), us = __ldg(S + t.irow + t.r0 + g);
+        const int NTt = (2 * t.nc + 7) >> 3;
+        float xsc[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int j = 4 * i + q;
+            xsc[i] = 0.f;
+            if (i < NTt && j < t.nc) {
+                const int tok = slot_token(p, sh, t.shared, t.off, t.tok0 + j);
+                xsc[i] = (tok >= 0 && tok < p.T) ? __ldcg(p.xs + tok) * 0.0625f : 0.f;
+            }
+        }
+        int acc[4][4];
+        switch (NTt) {
+            case 1: consume13<1>(nch, n, full, empty, wring, xring, abort, status, reinterpret_cast<int(&)[1][4]>(acc)); break;
+            case 2: consume13<2>(nch, n, full, empty, wring, xring, abort, status, reinterpret_cast<int(&)[2][4]>(acc)); break;
+            case 3: consume13<3>(nch, n, full, empty, wring, xring, abort, status, reinterpret_cast<int(&)[3][4]>(acc)); break;
+            default: consume13<4>(nch, n, full, empty, wring, xring, abort, status, acc); break;
+        }
+        const int slot0 = (t.shared ? 0 : t.off) + t.tok0;
+        float* hrow0 = (t.shared ? p.h32_s : p.h32_r) + (size_t)slot0 * t.irow + t.r0 + g;
+        float(*hm)[kChunkTokens] = hm2[r & 1];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (i >= NTt) break;
+            const int j = 4 * i + q;
+            float hmv = 0.f;
+            if (j < t.nc) {
+                const float gv = join(acc[i][0], acc[i][1]) * (gs * xsc[i]);
+                const float uv = join(acc[i][2], acc[i][3]) * (us * xsc[i]);
+                const float h = silu_mul(gv, uv);
+                hrow0[(size_t)j * t.irow] = h;
+                hmv = fabsf(h);
+            }
+            hmv = nanmax(hmv, __shfl_xor_sync(0xffffffffu, hmv, 4));
+            hmv = nanmax(hmv, __shfl_xor_sync(0xffffffffu, hmv, 8));
+            hmv = nanmax(hmv, __shfl_xor_sync(0xffffffffu, hmv, 16));
+            if (g == 0 && j < t.nc) hm[warp][j] = hmv;
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");  // the consumer warps' maxima are in
+        if (threadIdx.x < t.nc) {
+            const int j = threadIdx.x;
+            const int nrb = t.irow / kRows13;
+            float m = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) m = nanmax(m, hm[w][j]);
+            (t.shared ? p.hmax_s : p.hmax_r)[(size_t)(slot0 + j) * nrb + t.rbk] = m;
+        }
+    }
+}
+
 // One down task as this thread sees it: ng row groups of 128 rows starting
 // at row0; in group m this thread streams rows row0 + 128 m + j0 + g and + 8.
 struct Task2 {
@@ -1127,6 +1390,7 @@ int resident(Kern kern, size_t smem, int which, int threads = 256) {
 int experts_resident_ctas(int which, int H) {
     if (which == 1) return resident(experts_w2_kernel, kSmem2, 3);
     if (H <= kBulkMaxK) return resident(experts_w13_bulk_kernel, kSmem13Bulk, 4);
+    if (H % kTmaChunk == 0) return resident(experts_w13_tma_kernel, kSmem13Tma, 5, kTmaThreads);
     const int mode = H <= kDoubleMaxK ? 0 : H <= kWholeMaxK ? 1 : 2;
     switch (mode) {
         case 0: return resident(experts_w13_kernel<0>, kSmem13[0], 0);
@@ -1138,6 +1402,19 @@ int experts_resident_ctas(int which, int H) {
 cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
     const dim3 g(grid), b(256);
     if (p.H <= kBulkMaxK) return launch_pdl(experts_w13_bulk_kernel, g, b, kSmem13Bulk, stream, p);
+    if (p.H % kTmaChunk == 0) {
+        // routed gate/up rows [E*2I][H/2] and the shared expert's [2Is][H/2],
+        // tiles of 64 rows x 128 bytes (any valid map when there is no shared expert)
+        CUtensorMap tm_r, tm_s;
+        const bool ok =
+            encode_tensor_map_2d(&tm_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.w13, p.H / 2, (uint64_t)p.E * 2 * p.I,
+                                 kTmaRowBytes, kRows13, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_tensor_map_2d(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.Is > 0 ? (const void*)p.sh_w13 : (const void*)p.w13,
+                                 p.H / 2, p.Is > 0 ? 2 * (uint64_t)p.Is : 2 * (uint64_t)kRows13, kTmaRowBytes, kRows13,
+                                 CU_TENSOR_MAP_SWIZZLE_128B);
+        if (!ok) return cudaErrorInvalidValue;
+        return launch_pdl(experts_w13_tma_kernel, g, dim3(kTmaThreads), kSmem13Tma, stream, tm_r, tm_s, p);
+    }
     const int mode = p.H <= kDoubleMaxK ? 0 : p.H <= kWholeMaxK ? 1 : 2;
     switch (mode) {
         case 0: return launch_pdl(experts_w13_kernel<0>, g, b, kSmem13[0], stream, p);

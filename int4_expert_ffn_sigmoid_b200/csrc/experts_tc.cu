@@ -542,6 +542,11 @@ int g_smem_set[64];
 
 }  // namespace
 
+bool encode_tensor_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t inner,
+                          uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+    return get_encode() && make_map(m, dt, esize, base, inner, rows, box_inner, box_rows, sw);
+}
+
 int tc_smem_bytes() { return tc::SMEM_BYTES; }
 
 cudaError_t launch_tc_gemm(const Params& p, int gemm, int grid, cudaStream_t stream) {

@@ -34,6 +34,12 @@ typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_
                                     const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                     CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// A 2-D tensor map over a row-major [rows][inner] matrix of esize-byte
+// elements (box box_inner x box_rows); false if the driver entry point is
+// missing or rejects the arguments.
+bool encode_tensor_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t inner,
+                          uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw);
+
 // Launch GEMM-1 (gemm = 1) or GEMM-2 (gemm = 2) of the large-batch path.
 cudaError_t launch_tc_gemm(const Params& p, int gemm, int grid, cudaStream_t stream);
 int tc_smem_bytes();

@@ -175,6 +175,19 @@ def test_split_router(moe, cuda_device):
         assert torch.equal(o1, out[t0:t0 + sub])
 
 
+@pytest.mark.parametrize("H", [1152, 2176, 2304])
+def test_gate_up_staging_variants(moe, cuda_device, H):
+    """Hidden sizes above 1024 that are not multiples of 256 take the
+    gate/up kernels with register-ring weights (whole-row activations up to
+    2048, slices beyond); multiples of 256 take the TMA-ring kernel."""
+    shape = workloads.LayerShape(H=H, E=16, K=3, I=256, Is=128, routed_scaling=1.5)
+    layer = workloads.make_layer(shape, 260, 0, cuda_device)
+    cpu = to_cpu_layer(layer)
+    for T in (5, 40):
+        x = workloads.make_x(shape, T, 260, device=cuda_device)
+        check(moe, x, layer, shape, layer_cpu=cpu, residual=True)
+
+
 def test_large_intermediate_values(moe, cuda_device):
     """Inputs around +-300 drive the SwiGLU intermediate to ~1e5 (beyond fp16's
     65504 unless it is stored scaled); outputs stay finite and match."""
