@@ -250,8 +250,9 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
                              (routed_buckets * slices_of(cfg->I) + shared_chunks * slices_of(cfg->Is));
     int grid13 = 0, grid2 = 0;
     if (!use_tc) {
-        const long long cap13 = experts_resident_ctas(0, cfg->H);
-        const long long cap2 = experts_resident_ctas(1, cfg->H);
+        const bool w2_tma = experts_w2_tma(cfg->H, cfg->I, cfg->Is);
+        const long long cap13 = experts_resident_ctas(0, cfg->H, w2_tma);
+        const long long cap2 = experts_resident_ctas(1, cfg->H, w2_tma);
         grid13 = (int)(tasks13 < cap13 ? tasks13 : cap13);
         grid2 = (int)(tasks2 < cap2 ? tasks2 : cap2);
     }

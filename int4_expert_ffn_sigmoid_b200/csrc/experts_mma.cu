@@ -1366,6 +1366,254 @@ __global__ void __launch_bounds__(256, 2) experts_w2_kernel(Params p) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// Down projection with a TMA weight ring (large H; I and Is multiples of 256):
+// one CTA per SM, a producer warp and 8 consumer warps, as the TMA gate/up
+// kernel.  A stage is one 256-wide k chunk of one 128-row group of the task
+// (one TMA tile load of 128 rows x 128 bytes, 128-byte swizzle).  The
+// consumers prefetch the next task's f32 h slice, maxima and row scales with
+// cp.async and quantize the current task's slice in shared memory while the
+// producer keeps the ring full.
+// ---------------------------------------------------------------------------
+constexpr int kW2Bytes = kRows2 * kTmaRowBytes;  // one stage: 16 KB
+constexpr size_t kW2MiscBytes = 256;
+constexpr size_t kW2XOff = (size_t)kTmaStages * kW2Bytes;           // from the ring's start
+constexpr size_t kW2RawOff = kW2XOff + (size_t)kStageRows * kStride2;
+constexpr size_t kW2RsOff = kW2RawOff + (size_t)kChunkTokens * kSliceK * 4;
+constexpr size_t kSmem2Tma = kShmBytes + kW2MiscBytes + 1024 /* alignment */ + kW2RsOff + (size_t)2 * kMaxRows2 * 4;
+static_assert(kSmem2Tma <= 227 * 1024, "TMA down shared memory");
+
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// fetch2 for the 256 consumer threads.
+__device__ __forceinline__ void fetch2c(const Params& p, Shm& sh, const Task2& t, float* raw, float* rs) {
+    const int tid = threadIdx.x;
+    const float* S = (t.shared ? p.sh_s2 : p.s2 + (size_t)t.e * p.H) + t.row0;
+    for (int c = tid; c < p.rows2 / 4; c += 256) cp_async16(rs + 4 * c, S + 4 * c);
+    const float* hb = t.shared ? p.h32_s : p.h32_r;
+    const float* hmb = t.shared ? p.hmax_s : p.hmax_r;
+    const int nrb = t.irow / kRows13;
+    const int slot0 = (t.shared ? 0 : t.off) + t.tok0;
+    const int per = t.klen / 4;
+    for (int c = tid; c < t.nc * per; c += 256) {
+        const int j = c / per, k4 = c - j * per;
+        cp_async16(raw + j * kSliceK + k4 * 4, hb + (size_t)(slot0 + j) * t.irow + t.k0 + k4 * 4);
+    }
+    const int nb = t.klen / kRows13;
+    for (int c = tid; c < t.nc * nb; c += 256) {
+        const int j = c / nb, r = c - j * nb;
+        cp_async4(&sh.hmr[j][r], hmb + (size_t)(slot0 + j) * nrb + t.k0 / kRows13 + r);
+    }
+    cp_async_commit();
+}
+
+template <int NT>
+__device__ __forceinline__ void consume2(const Task2& tk, uint32_t& n, uint64_t* full, uint64_t* empty,
+                                         const uint8_t* wring, const uint8_t* xs, const float* rs, const Params& p,
+                                         const Shm& sh, volatile int* abort, unsigned* status) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, q = lane & 3;
+    constexpr int kSets = NT == 1 ? 2 : 1;
+    const size_t TK = (size_t)p.T * p.K;
+    const size_t yrow0 = tk.shared ? TK * p.nsl_r + (size_t)tk.sl * p.T + tk.tok0 : (size_t)tk.sl * TK + tk.off + tk.tok0;
+    const int nkc = tk.klen / kTmaChunk;
+    // rows warp*16 + g and + 8 of a 1024-byte aligned tile: 16-byte chunk j sits at j ^ g
+    const int wa_row = (warp * 16 + g) * kTmaRowBytes, wb_row = wa_row + 8 * kTmaRowBytes;
+    for (int m = 0; m < tk.ng; ++m) {
+        int part[kSets][NT][4];
+#pragma unroll
+        for (int s = 0; s < kSets; ++s)
+#pragma unroll
+            for (int i = 0; i < NT; ++i) part[s][i][0] = part[s][i][1] = part[s][i][2] = part[s][i][3] = 0;
+        for (int c = 0; c < nkc; ++c, ++n) {
+            const int s = n % kTmaStages;
+            if (!*abort && !bar_wait(full + s, (n / kTmaStages) & 1, kBulkWaitCycles)) {
+                *abort = 1;
+                if (lane == 0) atomicOr(status, ST_TIMEOUT);
+            }
+            const uint8_t* wt = wring + (size_t)s * kW2Bytes;
+            const uint8_t* xt = xs + g * kStride2 + q * 32 + c * kTmaChunk;
+#pragma unroll
+            for (int kb = 0; kb < kTmaChunk / 128; ++kb) {
+                const int off = ((kb * 4 + q) ^ g) << 4;
+                const uint4 wa = *reinterpret_cast<const uint4*>(wt + wa_row + off);
+                const uint4 wb = *reinterpret_cast<const uint4*>(wt + wb_row + off);
+                kblock8<NT, kSets>(wa, wb, xt + kb * 128, 8 * kStride2, part);
+            }
+            __syncwarp();
+            if (lane == 0) bar_arrive(empty + s);
+        }
+        const int jr = m * kRows2 + warp * 16 + g;  // row of this thread within the task
+        const float s_lo = rs[jr], s_hi = rs[jr + 8];
+        float* y0 = p.y + yrow0 * p.H + tk.row0 + jr;
+#pragma unroll
+        for (int i = 0; i < NT; ++i) {
+            const int j = 4 * i + q;
+            if (j < tk.nc) {
+                const int a0 = part[0][i][0] + part[kSets - 1][i][0] * (kSets - 1);
+                const int a1 = part[0][i][1] + part[kSets - 1][i][1] * (kSets - 1);
+                const int a2 = part[0][i][2] + part[kSets - 1][i][2] * (kSets - 1);
+                const int a3 = part[0][i][3] + part[kSets - 1][i][3] * (kSets - 1);
+                const float xsc = sh.xsc[j];
+                float* yr = y0 + (size_t)j * p.H;
+                yr[0] = join(a0, a1) * (s_lo * xsc);
+                yr[8] = join(a2, a3) * (s_hi * xsc);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kTmaThreads, 1)
+    experts_w2_tma_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_s, Params p) {
+    extern __shared__ __align__(128) uint8_t dsm[];
+    Shm& sh = *reinterpret_cast<Shm*>(dsm);
+    uint64_t* full = reinterpret_cast<uint64_t*>(dsm + kShmBytes);
+    uint64_t* empty = full + kTmaStages;
+    volatile int* abort = reinterpret_cast<volatile int*>(empty + kTmaStages);
+    const uint32_t base_s = static_cast<uint32_t>(__cvta_generic_to_shared(dsm));
+    const uint32_t ring_s = (base_s + (uint32_t)(kShmBytes + kW2MiscBytes) + 1023u) & ~1023u;
+    uint8_t* wring = dsm + (ring_s - base_s);
+    uint8_t* xs = wring + kW2XOff;
+    float* raw = reinterpret_cast<float*>(wring + kW2RawOff);
+    float* rs2 = reinterpret_cast<float*>(wring + kW2RsOff);  // [task parity][row of the task]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool producer = warp == 8;
+    unsigned* status = &p.ctrl->status;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kTmaStages; ++i) {
+            bar_init(full + i, 1);   // the tile load's arrival
+            bar_init(empty + i, 8);  // one arrival per consumer warp
+        }
+        *abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    const int R = p.H / p.rows2, ng = p.rows2 / kRows2;
+    // the shared expert's first task of this CTA, if its first task is one
+    const int nsl_s = p.Is > 0 ? slices_of(p.Is) : 0;
+    const int ns = p.Is > 0 ? R * chunks_of(p.T) * nsl_s : 0;
+    const bool pre = (int)blockIdx.x < ns;
+    int pre_rbk = 0, pre_sl = 0, pre_tok0 = 0, npre = 0;
+    if (pre) {
+        const int local = ns - 1 - (int)blockIdx.x, rest = local / R;
+        pre_rbk = local % R;
+        pre_sl = rest % nsl_s;
+        pre_tok0 = (rest / nsl_s) * kChunkTokens;
+        const int k0 = pre_sl * kSliceK, nkc = min(kSliceK, p.Is - k0) / kTmaChunk;
+        npre = min(kTmaStages, ng * nkc);
+        if (producer && lane == 0)
+            for (int i = 0; i < npre; ++i) {
+                const int m = i / nkc, c = i - m * nkc;
+                bar_expect_tx(full + i, kW2Bytes);
+                tma_tile(wring + (size_t)i * kW2Bytes, &tm_s, full + i, (k0 + c * kTmaChunk) / 2,
+                         pre_rbk * p.rows2 + m * kRows2);
+            }
+    }
+    if (p.Is > 0) prefetch_l2_slice(p.sh_w2, (size_t)p.H * p.Is / 2);
+    pdl_wait();
+    pdl_release();
+    load_tables(p, p.ts2, &p.ctrl->tasks2, sh.tb, nullptr);
+    precompute_tasks(p, sh, 1);
+    if (threadIdx.x == 0 && pre) {  // cannot fail with consistent tables
+        const TaskDesc d = sh.td[0];
+        if (!(d.e == p.E && d.rbk == pre_rbk && d.sl == pre_sl && d.tok0 == pre_tok0 &&
+              sh.tb.ntask > (int)blockIdx.x)) {
+            *abort = 1;
+            atomicOr(status, ST_BAD_TASK);
+        }
+    }
+    __syncthreads();
+    const int ntask = sh.tb.ntask;
+    if (!producer && *abort) return;
+    if (producer) {
+        uint32_t n = 0;
+        int last_round[kTmaStages];
+#pragma unroll
+        for (int s = 0; s < kTmaStages; ++s) last_round[s] = s < npre ? 0 : -1;
+        for (int r = 0; !*abort && snake(blockIdx.x, r) < ntask; ++r) {
+            const TaskDesc d = task_desc(p, sh, 1, r);
+            if (d.e < 0 || d.e > p.E || (d.e == p.E && p.Is == 0)) break;  // the consumers flag it
+            const bool shared = d.e == p.E;
+            const int irow = shared ? p.Is : p.I;
+            const int k0 = d.sl * kSliceK, nkc = min(kSliceK, irow - k0) / kTmaChunk;
+            const int row0 = (shared ? 0 : d.e * p.H) + d.rbk * p.rows2;
+            const CUtensorMap* map = shared ? &tm_s : &tm_r;
+            bool stop = false;
+            for (int m = 0; m < ng && !stop; ++m)
+                for (int c = 0; c < nkc; ++c, ++n) {
+                    const int s = n % kTmaStages;
+                    const int round = (int)(n / kTmaStages);
+                    if (round > 0) {
+                        const bool ok = *abort == 0 && bar_wait(empty + s, (round - 1) & 1, kBulkWaitCycles);
+                        if (__any_sync(0xffffffffu, !ok)) {
+                            if (lane == 0 && !*abort) atomicOr(status, ST_TIMEOUT);
+                            *abort = 1;
+                            stop = true;
+                            break;
+                        }
+                    }
+                    if (lane == 0 && !(r == 0 && (int)n < npre)) {
+                        bar_expect_tx(full + s, kW2Bytes);
+                        tma_tile(wring + (size_t)s * kW2Bytes, map, full + s, (k0 + c * kTmaChunk) / 2, row0 + m * kRows2);
+                    }
+                    last_round[s] = round;
+                }
+        }
+        // copies nobody will consume land before the CTA exits
+        if (*abort && lane == 0)
+            for (int s = 0; s < kTmaStages; ++s)
+                if (last_round[s] >= 0) bar_wait(full + s, last_round[s] & 1, kBulkWaitCycles);
+        __syncwarp();
+        return;
+    }
+    // consumers
+    uint32_t n = 0;
+    Task2 cur = task2_r(p, sh, 0);
+    if (cur.ok) fetch2c(p, sh, cur, raw, rs2);
+    for (int r = 0; snake(blockIdx.x, r) < ntask; ++r) {
+        const Task2 nx = task2_r(p, sh, r + 1);
+        if (!cur.ok) {
+            if (threadIdx.x == 0) atomicOr(status, ST_BAD_TASK);
+            break;
+        }
+        const int nc = cur.nc, klen = cur.klen;
+        cp_async_wait<0>();
+        consumers_sync();  // cur's h slice and maxima are visible; the previous task is done with xs
+        if (threadIdx.x < nc) {
+            const int j = threadIdx.x;
+            float m = 0.f;
+            for (int b = 0; b < klen / kRows13; ++b) m = nanmax(m, sh.hmr[j][b]);
+            const QScale qs = qscale(m);
+            sh.qs[j] = qs;
+            sh.xsc[j] = qs.s * 0.0625f;
+        }
+        consumers_sync();
+        for (int j = warp; j < nc; j += 8) {
+            const QScale qs = sh.qs[j];
+            const float* src = raw + j * kSliceK;
+            for (int gi = lane; gi < klen / 8; gi += 32) {
+                const float4 a = *reinterpret_cast<const float4*>(src + 8 * gi);
+                const float4 b2 = *reinterpret_cast<const float4*>(src + 8 * gi + 4);
+                const float f[8] = {a.x, a.y, a.z, a.w, b2.x, b2.y, b2.z, b2.w};
+                uint2 p0, p1;
+                quant2x8(f, qs, p0, p1);
+                *reinterpret_cast<uint2*>(xs + (2 * j) * kStride2 + 8 * gi) = p0;
+                *reinterpret_cast<uint2*>(xs + (2 * j + 1) * kStride2 + 8 * gi) = p1;
+            }
+        }
+        consumers_sync();  // staged; raw and hmr are free for the next task
+        if (nx.ok) fetch2c(p, sh, nx, raw, rs2 + ((r + 1) & 1) * kMaxRows2);
+        const float* rs = rs2 + (r & 1) * kMaxRows2;
+        switch ((2 * nc + 7) >> 3) {
+            case 1: consume2<1>(cur, n, full, empty, wring, xs, rs, p, sh, abort, status); break;
+            case 2: consume2<2>(cur, n, full, empty, wring, xs, rs, p, sh, abort, status); break;
+            case 3: consume2<3>(cur, n, full, empty, wring, xs, rs, p, sh, abort, status); break;
+            default: consume2<4>(cur, n, full, empty, wring, xs, rs, p, sh, abort, status); break;
+        }
+        cur = nx;
+    }
+    cp_async_wait<0>();
+}
+
 template <typename Kern>
 int resident(Kern kern, size_t smem, int which, int threads = 256) {
     static int cache[8][64];
@@ -1387,8 +1635,9 @@ int resident(Kern kern, size_t smem, int which, int threads = 256) {
 
 // Persistent grid of the weight-streaming kernels: the CTAs that fit at once
 // (which: 0 gate/up, 1 down).  Also sets the kernels' shared-memory limits.
-int experts_resident_ctas(int which, int H) {
-    if (which == 1) return resident(experts_w2_kernel, kSmem2, 3);
+int experts_resident_ctas(int which, int H, bool w2_tma) {
+    if (which == 1) return w2_tma ? resident(experts_w2_tma_kernel, kSmem2Tma, 6, kTmaThreads)
+                                  : resident(experts_w2_kernel, kSmem2, 3);
     if (H <= kBulkMaxK) return resident(experts_w13_bulk_kernel, kSmem13Bulk, 4);
     if (H % kTmaChunk == 0) return resident(experts_w13_tma_kernel, kSmem13Tma, 5, kTmaThreads);
     const int mode = H <= kDoubleMaxK ? 0 : H <= kWholeMaxK ? 1 : 2;
@@ -1423,7 +1672,21 @@ cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
     }
 }
 
+bool experts_w2_tma(int H, int I, int Is) { return H > kBulkMaxK && I % kTmaChunk == 0 && Is % kTmaChunk == 0; }
+
 cudaError_t launch_experts_w2(const Params& p, int grid, cudaStream_t stream) {
+    if (experts_w2_tma(p.H, p.I, p.Is)) {
+        // routed down rows [E*H][I/2] and the shared expert's [H][Is/2], tiles
+        // of 128 rows x 128 bytes (any valid map when there is no shared expert)
+        CUtensorMap tm_r, tm_s;
+        const bool ok =
+            encode_tensor_map_2d(&tm_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.w2, p.I / 2, (uint64_t)p.E * p.H,
+                                 kTmaRowBytes, kRows2, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_tensor_map_2d(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.Is > 0 ? (const void*)p.sh_w2 : (const void*)p.w2,
+                                 p.Is > 0 ? p.Is / 2 : p.I / 2, p.H, kTmaRowBytes, kRows2, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (!ok) return cudaErrorInvalidValue;
+        return launch_pdl(experts_w2_tma_kernel, dim3(grid), dim3(kTmaThreads), kSmem2Tma, stream, tm_r, tm_s, p);
+    }
     return launch_pdl(experts_w2_kernel, dim3(grid), dim3(256), kSmem2, stream, p);
 }
 

@@ -176,16 +176,20 @@ def test_split_router(moe, cuda_device):
 
 
 @pytest.mark.parametrize("H", [1152, 2176, 2304])
-def test_gate_up_staging_variants(moe, cuda_device, H):
-    """Hidden sizes above 1024 that are not multiples of 256 take the
-    gate/up kernels with register-ring weights (whole-row activations up to
-    2048, slices beyond); multiples of 256 take the TMA-ring kernel."""
-    shape = workloads.LayerShape(H=H, E=16, K=3, I=256, Is=128, routed_scaling=1.5)
+def test_streaming_kernel_variants(moe, cuda_device, H):
+    """Hidden sizes above 1024: gate/up takes the register-ring kernels when H
+    is not a multiple of 256 (whole-row activations up to 2048, slices beyond)
+    and the TMA-ring kernel otherwise; the down projection takes its TMA-ring
+    kernel (I and Is multiples of 256; a 768-wide I gives slices of 512 and
+    256).  T = 100 runs the large-batch router with the weight-streaming
+    kernels (H not a multiple of 256, or MOE_FORCE_DECODE)."""
+    shape = workloads.LayerShape(H=H, E=16, K=3, I=768, Is=256, routed_scaling=1.5)
     layer = workloads.make_layer(shape, 260, 0, cuda_device)
     cpu = to_cpu_layer(layer)
-    for T in (5, 40):
+    for T in (5, 40, 100):
         x = workloads.make_x(shape, T, 260, device=cuda_device)
-        check(moe, x, layer, shape, layer_cpu=cpu, residual=True)
+        flags = moe.MOE_FORCE_DECODE if T > 64 else 0
+        check(moe, x, layer, shape, layer_cpu=cpu, residual=True, flags=flags)
 
 
 def test_large_intermediate_values(moe, cuda_device):
