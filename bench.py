@@ -358,6 +358,19 @@ def cpu_baseline_sample(stack, budget_s=20.0):
     return n_tok * len(layers_cpu) / dt, f"{n_tok} of {stack.T} tokens of one batch through all {len(layers_cpu)} layers ({dt:.1f} s)"
 
 
+def streaming_kernel_names(shape):
+    """Gate/up and down kernels of the weight-streaming path for this shape
+    (the library's selection: TMA-ring kernels from H = 1024 on when H, I and
+    Is are multiples of 256; bulk-copy gate/up below; register-ring kernels
+    otherwise)."""
+    if shape.H >= 1024 and shape.H % 256 == 0:
+        w13 = "experts_w13_tma_kernel"
+    else:
+        w13 = "experts_w13_bulk_kernel" if shape.H <= 1024 else "experts_w13_kernel"
+    tma2 = shape.H >= 1024 and shape.I % 256 == 0 and shape.Is % 256 == 0
+    return w13, "experts_w2_tma_kernel" if tma2 else "experts_w2_kernel"
+
+
 def max_over_ranks(values, dist, device):
     """Element-wise maximum of `values` over all ranks (the slowest rank's
     times); the values themselves for a single process (dist None)."""
@@ -412,9 +425,9 @@ def run_ours(args, rank, world, device, dist):
     names = moe.STAGE_NAMES
     dom = 1 if stage_mean[1] >= stage_mean[2] else 2  # the dominant expert kernel
     tc_path = T > moe.decode_max_tokens() and wl.shape.H % 256 == 0
-    w13_name = "experts_w13_bulk_kernel" if wl.shape.H <= 1024 else "experts_w13_kernel"
+    w13_name, w2_name = streaming_kernel_names(wl.shape)
     kname = (("grouped_gemm_kernel<1>" if dom == 1 else "grouped_gemm_kernel<2>") if tc_path
-             else (w13_name if dom == 1 else "experts_w2_kernel"))
+             else (w13_name if dom == 1 else w2_name))
     work = [[stage_work(names[dom], wl.shape, T, u) for u in uniq[i % N_BATCHES]] for i in range(args.steps)]
     alg_b = statistics.mean(sum(w[0] for w in ws) for ws in work) / L
     alg_f = statistics.mean(sum(w[1] for w in ws) for ws in work) / L

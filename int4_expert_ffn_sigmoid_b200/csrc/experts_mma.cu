@@ -1614,6 +1614,11 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     cp_async_wait<0>();
 }
 
+// The TMA-ring kernels serve hidden sizes from kTmaMinH on (measured faster
+// than the bulk-copy gate/up and the register-ring down kernel there).
+constexpr int kTmaMinH = 1024;
+bool w13_tma(int H) { return H >= kTmaMinH && H % kTmaChunk == 0; }
+
 template <typename Kern>
 int resident(Kern kern, size_t smem, int which, int threads = 256) {
     static int cache[8][64];
@@ -1638,8 +1643,8 @@ int resident(Kern kern, size_t smem, int which, int threads = 256) {
 int experts_resident_ctas(int which, int H, bool w2_tma) {
     if (which == 1) return w2_tma ? resident(experts_w2_tma_kernel, kSmem2Tma, 6, kTmaThreads)
                                   : resident(experts_w2_kernel, kSmem2, 3);
+    if (w13_tma(H)) return resident(experts_w13_tma_kernel, kSmem13Tma, 5, kTmaThreads);
     if (H <= kBulkMaxK) return resident(experts_w13_bulk_kernel, kSmem13Bulk, 4);
-    if (H % kTmaChunk == 0) return resident(experts_w13_tma_kernel, kSmem13Tma, 5, kTmaThreads);
     const int mode = H <= kDoubleMaxK ? 0 : H <= kWholeMaxK ? 1 : 2;
     switch (mode) {
         case 0: return resident(experts_w13_kernel<0>, kSmem13[0], 0);
@@ -1650,8 +1655,7 @@ int experts_resident_ctas(int which, int H, bool w2_tma) {
 
 cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
     const dim3 g(grid), b(256);
-    if (p.H <= kBulkMaxK) return launch_pdl(experts_w13_bulk_kernel, g, b, kSmem13Bulk, stream, p);
-    if (p.H % kTmaChunk == 0) {
+    if (w13_tma(p.H)) {
         // routed gate/up rows [E*2I][H/2] and the shared expert's [2Is][H/2],
         // tiles of 64 rows x 128 bytes (any valid map when there is no shared expert)
         CUtensorMap tm_r, tm_s;
@@ -1664,6 +1668,7 @@ cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
         if (!ok) return cudaErrorInvalidValue;
         return launch_pdl(experts_w13_tma_kernel, g, dim3(kTmaThreads), kSmem13Tma, stream, tm_r, tm_s, p);
     }
+    if (p.H <= kBulkMaxK) return launch_pdl(experts_w13_bulk_kernel, g, b, kSmem13Bulk, stream, p);
     const int mode = p.H <= kDoubleMaxK ? 0 : p.H <= kWholeMaxK ? 1 : 2;
     switch (mode) {
         case 0: return launch_pdl(experts_w13_kernel<0>, g, b, kSmem13[0], stream, p);
@@ -1672,7 +1677,7 @@ cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
     }
 }
 
-bool experts_w2_tma(int H, int I, int Is) { return H > kBulkMaxK && I % kTmaChunk == 0 && Is % kTmaChunk == 0; }
+bool experts_w2_tma(int H, int I, int Is) { return H >= kTmaMinH && I % kTmaChunk == 0 && Is % kTmaChunk == 0; }
 
 cudaError_t launch_experts_w2(const Params& p, int grid, cudaStream_t stream) {
     if (experts_w2_tma(p.H, p.I, p.Is)) {

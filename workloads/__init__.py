@@ -34,7 +34,7 @@ from typing import Dict, Iterable, List, Optional
 import torch
 
 __all__ = [
-    "LayerShape", "NANO", "LARGE", "Workload", "WORKLOADS",
+    "LayerShape", "NANO", "LARGE", "LARGE_E32", "Workload", "WORKLOADS",
     "quantize_rows_int4", "pack_int4", "random_int4_codes",
     "make_layer", "make_x", "zipf_bias_path", "load_zipf_bias",
     "layer_weight_bytes", "expert_bytes",
@@ -63,6 +63,8 @@ NANO = LayerShape(H=1024, E=64, K=2, I=512, Is=2048, routed_scaling=1.0)
 # Layer shaped like the 744B streaming engine's: hidden 6144, 256 experts,
 # top-8, intermediate 2048 (routed and shared), scaling factor 2.5.
 LARGE = LayerShape(H=6144, E=256, K=8, I=2048, Is=2048, routed_scaling=2.5)
+# The same expert shapes with 32 experts (profiling stand-in).
+LARGE_E32 = LayerShape(H=6144, E=32, K=8, I=2048, Is=2048, routed_scaling=2.5)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -97,6 +99,10 @@ WORKLOADS: Dict[str, Workload] = {
                  "one Nano MoE layer, T=16384, Zipf(1.2) expert popularity via router bias"),
         Workload("large_layer", 4, LARGE, 1, (1, 32, 512), "uniform", False,
                  "one 6144-hidden 256-expert top-8 layer, T in {1,32,512}"),
+        Workload("large_layer_e32", 5, LARGE_E32, 1, (4,), "uniform", False,
+                 "the large layer's expert shapes with 32 experts (about 0.6 GB of weights), T=4: "
+                 "about one token per touched expert, as in the large layer at T=32; sized for "
+                 "profiler captures of its kernels"),
     ]
 }
 
