@@ -358,6 +358,30 @@ def cpu_baseline_sample(stack, budget_s=20.0):
     return n_tok * len(layers_cpu) / dt, f"{n_tok} of {stack.T} tokens of one batch through all {len(layers_cpu)} layers ({dt:.1f} s)"
 
 
+def captured_traffic(workload: str, T: int, kernel: str):
+    """DRAM bytes per launch of `kernel` on this workload and T from the
+    committed ncu capture (profiles/traffic.json), or None when there is none
+    or the kernel's sources have changed since it was taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            entries = json.load(f)["entries"]
+    except (OSError, ValueError, KeyError):
+        return None
+    for e in entries:
+        if (e["workload"], e["T"], e["kernel"]) != (workload, T, kernel):
+            continue
+        h = hashlib.sha256()
+        try:
+            for src in e["sources"]:
+                with open(os.path.join(ROOT, src), "rb") as f:
+                    h.update(f.read())
+        except OSError:
+            return None
+        return int(e["read"]) + int(e["write"]) if h.hexdigest() == e["sha256"] else None
+    return None
+
+
 def streaming_kernel_names(shape):
     """Gate/up and down kernels of the weight-streaming path for this shape
     (the library's selection: TMA-ring kernels from H = 1024 on when H, I and
@@ -443,7 +467,7 @@ def run_ours(args, rank, world, device, dist):
         roofline = {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                     "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy)"}
-    roofline.update({"traffic": None, "alg_bytes_per_launch": int(alg_b), "alg_flops_per_launch": int(alg_f),
+    roofline.update({"traffic": captured_traffic(wl.name, T, kname), "alg_bytes_per_launch": int(alg_b), "alg_flops_per_launch": int(alg_f),
                      "avg_launch_us": round(per_launch_s * 1e6, 3)})
 
     sweep = {}

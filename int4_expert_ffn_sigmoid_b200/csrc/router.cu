@@ -315,15 +315,18 @@ __device__ __forceinline__ void reset_ctrl(const Params& p) {
 constexpr int kRouterXMaxH = 12288;
 constexpr int kRouterWarps = 16;
 constexpr int kRouterBatch = 8;  // router-weight blocks per batch of loads
-// Router weights of at least this many bytes (E * H * 4) are read by a
-// separate logits kernel spread over many SMs (router_logits_kernel) instead
-// of by the clusters' 8 CTAs per token group.
-constexpr size_t kRouterSplitBytes = (size_t)2 << 20;
+// When a warp of the cluster router would stream more than this many bytes of
+// router weights (its ceil(epc / kRouterWarps) rows of H f32 each), the
+// logits are computed by a separate kernel spread over many SMs
+// (router_logits_kernel) instead of by the clusters' 8 CTAs per token group.
+constexpr size_t kRouterWarpMaxBytes = 8192;
 constexpr int kLogitSliceBlocks = 3;   // 128-element blocks of the hidden dimension per slice
 constexpr int kLogitCtaExperts = 32;   // experts per CTA (4 per warp)
 
 int router_split_slices(int E, int H, bool small_path) {
-    if (!small_path || (size_t)E * H * 4 < kRouterSplitBytes) return 0;
+    const int epc = (E + kDecodeRouterCtas - 1) / kDecodeRouterCtas;
+    const size_t warp_bytes = (size_t)((epc + kRouterWarps - 1) / kRouterWarps) * H * 4;
+    if (!small_path || warp_bytes <= kRouterWarpMaxBytes) return 0;
     return (H / 128 + kLogitSliceBlocks - 1) / kLogitSliceBlocks;
 }
 

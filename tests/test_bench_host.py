@@ -64,3 +64,32 @@ def test_reference_arm_line(monkeypatch):
     assert line["impl"] == "reference" and line["unit"] == bench.UNIT and line["metric"] == bench.METRIC
     assert line["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+
+
+def test_captured_traffic_lookup():
+    """roofline.traffic comes from the committed capture table only for a
+    listed (workload, T, kernel) whose sources hash to the recorded value."""
+    import hashlib
+    import json
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        entries = json.load(f)["entries"]
+    assert entries
+    for e in entries:
+        h = hashlib.sha256()
+        for src in e["sources"]:
+            with open(os.path.join(bench.ROOT, src), "rb") as f:
+                h.update(f.read())
+        got = bench.captured_traffic(e["workload"], e["T"], e["kernel"])
+        assert got == (e["read"] + e["write"] if h.hexdigest() == e["sha256"] else None)
+    assert bench.captured_traffic("nano_decode_stack", 64, "no_such_kernel") is None
+    assert bench.captured_traffic("no_such_workload", 64, entries[0]["kernel"]) is None
+
+
+def test_streaming_kernel_names_follow_the_library_selection():
+    import workloads
+    assert bench.streaming_kernel_names(workloads.NANO) == ("experts_w13_tma_kernel", "experts_w2_tma_kernel")
+    assert bench.streaming_kernel_names(workloads.LARGE) == ("experts_w13_tma_kernel", "experts_w2_tma_kernel")
+    small = workloads.LayerShape(H=384, E=8, K=2, I=128, Is=128, routed_scaling=1.0)
+    assert bench.streaming_kernel_names(small) == ("experts_w13_bulk_kernel", "experts_w2_kernel")
+    odd = workloads.LayerShape(H=1152, E=8, K=2, I=768, Is=256, routed_scaling=1.0)
+    assert bench.streaming_kernel_names(odd) == ("experts_w13_kernel", "experts_w2_tma_kernel")
