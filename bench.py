@@ -448,7 +448,7 @@ def run_ours(args, rank, world, device, dist):
     stage_mean = [statistics.mean(s[k] for s in stage_ms) for k in range(4)]
     names = moe.STAGE_NAMES
     dom = 1 if stage_mean[1] >= stage_mean[2] else 2  # the dominant expert kernel
-    tc_path = T > moe.decode_max_tokens() and wl.shape.H % 256 == 0
+    tc_path = moe.layer_path(wl.shape, T) == moe.MOE_PATH_TENSOR_CORE
     w13_name, w2_name = streaming_kernel_names(wl.shape)
     kname = (("grouped_gemm_kernel<1>" if dom == 1 else "grouped_gemm_kernel<2>") if tc_path
              else (w13_name if dom == 1 else w2_name))

@@ -60,7 +60,7 @@ extern "C" {
 #define MOE_ADD_RESIDUAL (1u << 0)  /* out = x + MoE(x) (one layer of a residual stack) */
 #define MOE_DEBUG_CHECK (1u << 1)   /* synchronise the stream and report device range checks */
 #define MOE_FORCE_DECODE (1u << 2)  /* use the small-batch (weight-streaming) kernels at any T */
-#define MOE_FORCE_PREFILL (1u << 3) /* use the large-batch (grouped GEMM) kernels at any T */
+#define MOE_FORCE_PREFILL (1u << 3) /* use the grouped-GEMM kernels at any T (H a multiple of 256) */
 #define MOE_OUT_F32 (1u << 4)       /* out is f32 [T][H] (the f32 sum, no bf16 rounding): for
                                        checking the arithmetic apart from the output rounding */
 
@@ -139,8 +139,10 @@ size_t moe_layer_workspace_bytes(const moe_cfg_t* cfg, int32_t T);
  * Arithmetic.  Router logits, scores and routing weights are f32.  Two
  * kernel sequences compute the experts:
  *  - small batches (T <= moe_decode_max_tokens(), unless MOE_FORCE_PREFILL),
- *    and larger ones when H is not a multiple of 256 or under
- *    MOE_FORCE_DECODE: weight-streaming kernels.  An activation row (x of a
+ *    and larger ones when H is not a multiple of 256, when T*K < 32*E (fewer
+ *    than 32 picks per routed expert on average; not under
+ *    MOE_FORCE_PREFILL), or under MOE_FORCE_DECODE: weight-streaming
+ *    kernels (moe_layer_path tells which).  An activation row (x of a
  *    token, or a 512-wide slice of its SwiGLU intermediate h) is written as
  *    s * (q0 + q1/256) with int8 q0, q1 and a power of two s from the row's
  *    largest magnitude, so each element is represented to within 2^-15 of
@@ -200,14 +202,21 @@ const char* moe_status_str(int status);
 /* MOE_ABI_VERSION of the loaded library. */
 int moe_abi_version(void);
 
-/* Largest T for which moe_layer_forward takes the small-batch
- * (weight-streaming) path when neither MOE_FORCE_* flag is set. */
+/* Largest T for which moe_layer_forward takes the small-batch path when
+ * neither MOE_FORCE_* flag is set. */
 int32_t moe_decode_max_tokens(void);
 
 /* Number of kernels one moe_layer_forward call launches for T tokens under
  * cfg (the stage events are not kernels).  Returns 0 if T = 0 or the call
  * would be rejected for cfg or T (the pointers in cfg are not looked at). */
 int32_t moe_layer_kernel_launches(const moe_cfg_t* cfg, int32_t T);
+
+/* The kernel sequence moe_layer_forward takes for T tokens under cfg (see
+ * "Arithmetic" above), or 0 if T = 0 or the call would be rejected. */
+#define MOE_PATH_SMALL_BATCH 1     /* cluster router, weight-streaming experts */
+#define MOE_PATH_TENSOR_CORE 2     /* large router, tensor-core grouped GEMMs */
+#define MOE_PATH_LARGE_STREAMING 3 /* large router, weight-streaming experts */
+int32_t moe_layer_path(const moe_cfg_t* cfg, int32_t T);
 
 #ifdef __cplusplus
 }

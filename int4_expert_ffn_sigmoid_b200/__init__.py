@@ -19,7 +19,8 @@ import torch
 __all__ = [
     "MoeError", "moe_cfg_t", "moe_shared_weights_t", "lib", "EXPORTED_SYMBOLS",
     "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK", "MOE_FORCE_DECODE", "MOE_FORCE_PREFILL", "MOE_OUT_F32",
-    "workspace_bytes", "layer_forward", "MoELayer", "decode_max_tokens", "kernel_launches", "LIB_PATH",
+    "workspace_bytes", "layer_forward", "MoELayer", "decode_max_tokens", "kernel_launches", "layer_path",
+    "MOE_PATH_SMALL_BATCH", "MOE_PATH_TENSOR_CORE", "MOE_PATH_LARGE_STREAMING", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_int4.so")
@@ -36,6 +37,10 @@ MOE_DEBUG_CHECK = 1 << 1
 MOE_FORCE_DECODE = 1 << 2
 MOE_FORCE_PREFILL = 1 << 3
 MOE_OUT_F32 = 1 << 4
+# kernel sequences (moe_layer_path)
+MOE_PATH_SMALL_BATCH = 1
+MOE_PATH_TENSOR_CORE = 2
+MOE_PATH_LARGE_STREAMING = 3
 
 MOE_STAGE_ROUTE, MOE_STAGE_GATE_UP, MOE_STAGE_DOWN, MOE_STAGE_COMBINE = range(4)
 MOE_NUM_STAGES = 4
@@ -44,7 +49,7 @@ STAGE_NAMES = ("route", "gate_up", "down", "combine")
 # Every function declared in include/moe_int4.h.
 EXPORTED_SYMBOLS = ("moe_layer_workspace_bytes", "moe_layer_forward", "moe_status_str",
                     "moe_abi_version", "moe_decode_max_tokens", "moe_layer_forward_static_ws",
-                    "moe_layer_kernel_launches")
+                    "moe_layer_kernel_launches", "moe_layer_path")
 
 # Scratch capacity of moe_layer_forward_static_ws (the entry point for callers
 # that cannot allocate device memory).
@@ -91,6 +96,8 @@ def _load() -> ctypes.CDLL:
     L.moe_decode_max_tokens.restype = ctypes.c_int32
     L.moe_layer_kernel_launches.argtypes = [ctypes.POINTER(moe_cfg_t), ctypes.c_int32]
     L.moe_layer_kernel_launches.restype = ctypes.c_int32
+    L.moe_layer_path.argtypes = [ctypes.POINTER(moe_cfg_t), ctypes.c_int32]
+    L.moe_layer_path.restype = ctypes.c_int32
     if L.moe_abi_version() != 1:
         raise ImportError("libmoe_int4.so ABI version mismatch")
     return L
@@ -137,6 +144,12 @@ def kernel_launches(shape, T: int, flags: int = 0) -> int:
     """Kernels one layer_forward call launches for T tokens (0: invalid)."""
     c = make_cfg(shape, flags)
     return int(lib.moe_layer_kernel_launches(ctypes.byref(c), int(T)))
+
+
+def layer_path(shape, T: int, flags: int = 0) -> int:
+    """MOE_PATH_* of a layer_forward call for T tokens (0: invalid)."""
+    c = make_cfg(shape, flags)
+    return int(lib.moe_layer_path(ctypes.byref(c), int(T)))
 
 
 def workspace_bytes(shape, T: int, flags: int = 0) -> int:

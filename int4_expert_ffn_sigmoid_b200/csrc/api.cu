@@ -23,11 +23,18 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 // + weight-streaming experts (H not a multiple of 256, or MOE_FORCE_DECODE).
 enum class Path { kSmall, kTensorCore, kLargeStreaming };
 
+// Average (token, pick) slots per routed expert below which large batches
+// stream the weights instead of running the grouped GEMM: with fewer tokens
+// per expert the GEMM's 128-token tiles are mostly padding and the layer is
+// bound by reading the touched experts' weights.
+constexpr int kTcMinSlotsPerExpert = 32;
+
 Path choose_path(const moe_cfg_t& c, int32_t T) {
     if (T <= kDecodeMaxTokens && !(c.flags & MOE_FORCE_PREFILL)) return Path::kSmall;
     // GEMM-2 of the tensor-core path tiles 256 output columns
-    if (!(c.flags & MOE_FORCE_DECODE) && c.H % 256 == 0) return Path::kTensorCore;
-    return Path::kLargeStreaming;
+    if ((c.flags & MOE_FORCE_DECODE) || c.H % 256 != 0) return Path::kLargeStreaming;
+    if (c.flags & MOE_FORCE_PREFILL) return Path::kTensorCore;
+    return (long long)T * c.K >= (long long)kTcMinSlotsPerExpert * c.E ? Path::kTensorCore : Path::kLargeStreaming;
 }
 
 struct WsLayout {
@@ -126,9 +133,18 @@ int32_t moe_decode_max_tokens(void) { return kDecodeMaxTokens; }
 int32_t moe_layer_kernel_launches(const moe_cfg_t* cfg, int32_t T) {
     if (validate_cfg(cfg) != MOE_OK || T <= 0 || T > kMaxTokens) return 0;
     // small batch: [router logits,] cluster router, gate/up, down, combine;
-    // otherwise: router, finalize, scatter, gate/up, down, combine
-    if (choose_path(*cfg, T) == Path::kSmall) return router_split_slices(cfg->E, cfg->H, true) > 0 ? 5 : 4;
-    return 6;
+    // otherwise: [router logits,] router, finalize, scatter, gate/up, down, combine
+    const bool small = choose_path(*cfg, T) == Path::kSmall;
+    return (small ? 4 : 6) + (router_split_slices(cfg->E, cfg->H, small) > 0 ? 1 : 0);
+}
+
+int32_t moe_layer_path(const moe_cfg_t* cfg, int32_t T) {
+    if (validate_cfg(cfg) != MOE_OK || T <= 0 || T > kMaxTokens) return 0;
+    switch (choose_path(*cfg, T)) {
+        case Path::kSmall: return MOE_PATH_SMALL_BATCH;
+        case Path::kTensorCore: return MOE_PATH_TENSOR_CORE;
+        default: return MOE_PATH_LARGE_STREAMING;
+    }
 }
 
 const char* moe_status_str(int status) {
@@ -226,7 +242,7 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
         p.nsl_s = slices_of(cfg->Is);
     }
     p.decode_groups = small ? cdiv(T, kDecodeRouterTok) : 0;
-    p.lslices = router_split_slices(cfg->E, cfg->H, small);
+    p.lslices = router_split_slices(cfg->E, cfg->H, small);  // on either path
     p.lpart = p.lslices > 0 ? static_cast<float*>(at(L.lpart)) : nullptr;
     // down tasks of large hidden sizes cover several 128-row groups, so that a
     // task streams enough weight bytes to outweigh its per-task costs

@@ -315,18 +315,26 @@ __device__ __forceinline__ void reset_ctrl(const Params& p) {
 constexpr int kRouterXMaxH = 12288;
 constexpr int kRouterWarps = 16;
 constexpr int kRouterBatch = 8;  // router-weight blocks per batch of loads
-// When a warp of the cluster router would stream more than this many bytes of
-// router weights (its ceil(epc / kRouterWarps) rows of H f32 each), the
-// logits are computed by a separate kernel spread over many SMs
-// (router_logits_kernel) instead of by the clusters' 8 CTAs per token group.
+// The logits are computed by a separate kernel spread over many SMs
+// (router_logits_kernel) when a warp of the cluster router would stream more
+// than kRouterWarpMaxBytes of router weights (its ceil(epc / kRouterWarps)
+// rows of H f32 each), and on the large-batch path when the router weights
+// (E * H f32, which every CTA of router_large_kernel reads) exceed
+// kRouterLargeMaxBytes.
 constexpr size_t kRouterWarpMaxBytes = 8192;
+constexpr size_t kRouterLargeMaxBytes = (size_t)2 << 20;
 constexpr int kLogitSliceBlocks = 3;   // 128-element blocks of the hidden dimension per slice
 constexpr int kLogitCtaExperts = 32;   // experts per CTA (4 per warp)
+constexpr int kLogitTileTokens = 64;   // tokens per CTA
 
 int router_split_slices(int E, int H, bool small_path) {
-    const int epc = (E + kDecodeRouterCtas - 1) / kDecodeRouterCtas;
-    const size_t warp_bytes = (size_t)((epc + kRouterWarps - 1) / kRouterWarps) * H * 4;
-    if (!small_path || warp_bytes <= kRouterWarpMaxBytes) return 0;
+    if (small_path) {
+        const int epc = (E + kDecodeRouterCtas - 1) / kDecodeRouterCtas;
+        const size_t warp_bytes = (size_t)((epc + kRouterWarps - 1) / kRouterWarps) * H * 4;
+        if (warp_bytes <= kRouterWarpMaxBytes) return 0;
+    } else if ((size_t)E * H * 4 <= kRouterLargeMaxBytes) {
+        return 0;
+    }
     return (H / 128 + kLogitSliceBlocks - 1) / kLogitSliceBlocks;
 }
 
@@ -334,20 +342,22 @@ size_t router_decode_smem(int H) {
     return H <= kRouterXMaxH ? (size_t)kDecodeRouterTok * H * sizeof(__nv_bfloat16) : 0;
 }
 
-// Split small-batch router, first kernel: CTA (s, b) computes, for every
-// token, the partial logits over hidden slice s (blocks s*kLogitSliceBlocks
-// onwards, 128 elements each) of experts [32 b, 32 b + 32): warp w takes
-// experts 32 b + 4 w .. + 3 and holds their weights of the slice in
-// registers (loaded before waiting on the previous kernel); the tokens'
-// activations of the slice are staged in shared memory.  Lane l accumulates
-// the elements 128 i + 4 l + j of the slice (i ascending, then j) and the
-// lanes are summed by the xor-butterfly; the cluster kernel adds the slices
-// in ascending order.  The logit of a token therefore does not depend on the
-// other tokens of the batch.
+// Split router, first kernel: CTA (s, b, z) computes, for tokens [64 z,
+// 64 z + 64), the partial logits over hidden slice s (blocks
+// s*kLogitSliceBlocks onwards, 128 elements each) of experts [32 b, 32 b +
+// 32): warp w takes experts 32 b + 4 w .. + 3 and holds their weights of the
+// slice in registers (loaded before waiting on the previous kernel); the
+// tokens' activations of the slice are staged in shared memory.  Lane l
+// accumulates the elements 128 i + 4 l + j of the slice (i ascending, then j)
+// and the lanes are summed by the xor-butterfly; the selecting kernel (the
+// cluster router or router_large_kernel) adds the slices in ascending order.
+// The logit of a token therefore does not depend on the other tokens of the
+// batch.
 __global__ void __launch_bounds__(256) router_logits_kernel(Params p) {
-    extern __shared__ __align__(16) __nv_bfloat16 s_xl[];  // [T][kLogitSliceBlocks * 128]
+    extern __shared__ __align__(16) __nv_bfloat16 s_xl[];  // [tile tokens][kLogitSliceBlocks * 128]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int E = p.E, H = p.H, T = p.T;
+    const int t0 = blockIdx.z * kLogitTileTokens, nt = min(kLogitTileTokens, T - t0);
     const int s = blockIdx.x;
     const int b0 = s * kLogitSliceBlocks, nb = min(kLogitSliceBlocks, H / 128 - b0);
     const int e0 = blockIdx.y * kLogitCtaExperts + warp * 4;
@@ -363,18 +373,18 @@ __global__ void __launch_bounds__(256) router_logits_kernel(Params p) {
     pdl_wait();
     pdl_release();
     const int per = nb * 16;  // 16-byte chunks of a token's slice
-    for (int c = threadIdx.x; c < T * per; c += blockDim.x) {
+    for (int c = threadIdx.x; c < nt * per; c += blockDim.x) {
         const int t = c / per, k = c - t * per;
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(
                          __cvta_generic_to_shared(s_xl + (size_t)t * kW + k * 8))),
-                     "l"(p.x + (size_t)t * H + b0 * 128 + k * 8)
+                     "l"(p.x + (size_t)(t0 + t) * H + b0 * 128 + k * 8)
                      : "memory");
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
     if (e0 >= E) return;
-    for (int t = 0; t < T; ++t) {
+    for (int t = 0; t < nt; ++t) {
         uint2 xv[kLogitSliceBlocks];
 #pragma unroll
         for (int i = 0; i < kLogitSliceBlocks; ++i)
@@ -391,12 +401,14 @@ __global__ void __launch_bounds__(256) router_logits_kernel(Params p) {
         }
         if (lane < 4 && e0 + lane < E) {
             const float r = lane == 0 ? v[0] : lane == 1 ? v[1] : lane == 2 ? v[2] : v[3];
-            p.lpart[((size_t)s * T + t) * E + e0 + lane] = r;
+            p.lpart[((size_t)s * T + t0 + t) * E + e0 + lane] = r;
         }
     }
 }
 
-size_t router_logits_smem(int T) { return (size_t)T * kLogitSliceBlocks * 128 * sizeof(__nv_bfloat16); }
+size_t router_logits_smem(int T) {
+    return (size_t)min(T, kLogitTileTokens) * kLogitSliceBlocks * 128 * sizeof(__nv_bfloat16);
+}
 
 __global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(32 * kRouterWarps, 1)
     router_decode_kernel(Params p) {
@@ -596,6 +608,22 @@ __global__ void __launch_bounds__(256) router_large_kernel(Params p) {
         const int t0 = tile * kRouterTileTokens;
         const int nt = min(kRouterTileTokens, p.T - t0);
         for (int tt = warp; tt < nt; tt += 8) token_hexp(p, t0 + tt, lane);
+        if (p.lslices > 0) {  // logits from the split kernel's partials, slice 0 first
+            __syncthreads();  // s_logit is free (previous tile done)
+            for (int i = threadIdx.x; i < nt * E; i += blockDim.x) {
+                const int tt = i / E, e = i - tt * E;
+                const float* src = p.lpart + (size_t)(t0 + tt) * E + e;
+                float v = 0.f;
+                for (int sl = 0; sl < p.lslices; ++sl) v += __ldcg(src + (size_t)sl * p.T * E);
+                s_logit[tt][e] = v;
+            }
+            __syncthreads();
+            for (int tt = warp; tt < nt; tt += 8) {
+                const int sel = select_token(p, t0 + tt, s_logit[tt], lane);
+                if (lane < p.K && sel >= 0 && sel < E) atomicAdd(&s_cnt[sel], 1);
+            }
+            continue;
+        }
 
         auto stage_chunk = [&](int c, int buf) {
             for (int i = threadIdx.x; i < kRouterTileTokens * (kRouterKC / 8); i += blockDim.x) {
@@ -705,19 +733,27 @@ __global__ void __launch_bounds__(1024) router_finalize_kernel(Params p) {
     const int E = p.E, nblk = p.router_blocks;
     pdl_wait();
     pdl_release();
-    // hist[b][e] -> exclusive prefix over b (per expert), one warp per expert
+    // hist[b][e] -> exclusive prefix over b (per expert), one warp per expert;
+    // all of an expert's counts are loaded before the scan (one round trip)
+    constexpr int kPer = (kRouterMaxBlocks + 31) / 32;
     for (int e = warp; e < E; e += nwarp) {
+        int v[kPer];
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int b = 32 * j + lane;
+            v[j] = b < nblk ? p.hist[(size_t)b * E + e] : 0;
+        }
         int run = 0;
-        for (int b0 = 0; b0 < nblk; b0 += 32) {
-            const int b = b0 + lane;
-            const int v = b < nblk ? p.hist[(size_t)b * E + e] : 0;
-            int inc = v;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int b = 32 * j + lane;
+            int inc = v[j];
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int u = __shfl_up_sync(0xffffffffu, inc, o);
                 if (lane >= o) inc += u;
             }
-            if (b < nblk) p.hist[(size_t)b * E + e] = run + inc - v;
+            if (b < nblk) p.hist[(size_t)b * E + e] = run + inc - v[j];
             run += __shfl_sync(0xffffffffu, inc, 31);
         }
         if (lane == 0) s_cnt[e] = run;
@@ -793,6 +829,12 @@ __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
     }
 }
 
+cudaError_t launch_router_logits(const Params& p, cudaStream_t stream) {
+    const dim3 grid(p.lslices, (p.E + kLogitCtaExperts - 1) / kLogitCtaExperts,
+                    (p.T + kLogitTileTokens - 1) / kLogitTileTokens);
+    return launch_pdl(router_logits_kernel, grid, dim3(256), router_logits_smem(p.T), stream, p);
+}
+
 cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream) {
     cudaError_t err;
     if (small_path) {
@@ -806,12 +848,15 @@ cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream)
             attr_set[dev] = 1;
         }
         if (p.lslices > 0) {
-            const cudaError_t e = launch_pdl(router_logits_kernel, dim3(p.lslices, (p.E + kLogitCtaExperts - 1) / kLogitCtaExperts),
-                                             dim3(256), router_logits_smem(p.T), stream, p);
+            const cudaError_t e = launch_router_logits(p, stream);
             if (e != cudaSuccess) return e;
         }
         return launch_pdl(router_decode_kernel, dim3(p.decode_groups, kDecodeRouterCtas), dim3(32 * kRouterWarps),
                           smem, stream, p);
+    }
+    if (p.lslices > 0) {
+        err = launch_router_logits(p, stream);
+        if (err != cudaSuccess) return err;
     }
     err = launch_pdl(router_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
     if (err == cudaSuccess) err = launch_pdl(router_finalize_kernel, dim3(1), dim3(1024), 0, stream, p);

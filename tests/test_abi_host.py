@@ -56,7 +56,8 @@ def test_struct_layout_matches_c(moe, tmp_path):
 def test_header_constants_match_binding(moe):
     text = open(HEADER).read()
     for name in ("MOE_STATIC_WORKSPACE_BYTES", "MOE_OUT_F32", "MOE_FORCE_DECODE",
-                 "MOE_FORCE_PREFILL", "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK"):
+                 "MOE_FORCE_PREFILL", "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK",
+                 "MOE_PATH_SMALL_BATCH", "MOE_PATH_TENSOR_CORE", "MOE_PATH_LARGE_STREAMING"):
         m = re.search(rf"#define {name} (.+)", text)
         assert m, name
         expr = m.group(1).split("/*")[0].replace("(size_t)", "").replace("u", "")
@@ -99,9 +100,27 @@ def test_kernel_launch_count(moe):
     assert moe.kernel_launches(nano, 16, moe.MOE_FORCE_PREFILL) == 6
     assert moe.kernel_launches(nano, 4096, moe.MOE_FORCE_DECODE) == 6
     assert moe.kernel_launches(large, 1) == 5       # + the split router's logits kernel
-    assert moe.kernel_launches(large, 512) == 6
+    assert moe.kernel_launches(large, 512) == 7     # large router with the logits kernel
     assert moe.kernel_launches(_shape(H=1000), 16) == 0
     assert moe.kernel_launches(nano, (1 << 20) + 1) == 0
+
+
+def test_path_choice(moe):
+    nano = _shape()
+    large = _shape(H=6144, E=256, K=8, I=2048, Is=2048, routed_scaling=2.5)
+    S, TC, LS = moe.MOE_PATH_SMALL_BATCH, moe.MOE_PATH_TENSOR_CORE, moe.MOE_PATH_LARGE_STREAMING
+    assert moe.layer_path(nano, 0) == 0
+    assert moe.layer_path(nano, 64) == S
+    assert moe.layer_path(nano, 65) == LS             # 130 picks over 64 experts: streaming
+    assert moe.layer_path(nano, 1023) == LS           # T*K = 2046 < 32*E = 2048
+    assert moe.layer_path(nano, 1024) == TC
+    assert moe.layer_path(nano, 4096) == TC
+    assert moe.layer_path(nano, 4096, moe.MOE_FORCE_DECODE) == LS
+    assert moe.layer_path(nano, 16, moe.MOE_FORCE_PREFILL) == TC
+    assert moe.layer_path(nano, 100, moe.MOE_FORCE_PREFILL) == TC
+    assert moe.layer_path(_shape(H=1152), 4096) == LS  # H not a multiple of 256
+    assert moe.layer_path(large, 512) == LS            # 16 picks per expert
+    assert moe.layer_path(large, 1024) == TC
 
 
 # Fake device pointers: validation runs before any dereference or CUDA call.

@@ -173,6 +173,13 @@ def test_split_router(moe, cuda_device):
     for t0, sub in ((0, 1), (5, 9), (40, 24)):
         o1, _, _ = run(moe, x[t0:t0 + sub].contiguous(), layer, shape)
         assert torch.equal(o1, out[t0:t0 + sub])
+    # large batches: the logits kernel over token tiles of 64 (150 = 64 + 64 + 22)
+    # feeding the large router's selection
+    assert moe.kernel_launches(shape, 150) == 7
+    x = workloads.make_x(shape, 150, 250, batch=1, device=cuda_device)
+    out, _, _, _ = check(moe, x, layer, shape, layer_cpu=cpu, sample=sample_tokens(150, 40, 5))
+    o1, _, _ = run(moe, x[10:110].contiguous(), layer, shape)
+    assert torch.equal(o1, out[10:110])
 
 
 @pytest.mark.parametrize("H", [1152, 2176, 2304])
@@ -228,18 +235,23 @@ def test_nan_bias_never_selected(moe, cuda_device):
 
 def test_batch_independence_and_permutation(moe, cuda_device):
     """A token's output does not depend on the rest of the batch, bit for bit,
-    within each path: the small-batch path (T <= 64) and the large-batch path
-    (T > 64, tensor-core router and grouped GEMMs)."""
+    within each path: the small-batch path (T <= 64), the large-batch
+    weight-streaming path (T = 200 gives ~6 picks per expert) and the
+    tensor-core path (forced)."""
     wl = workloads.WORKLOADS["nano_layer_t16"]
     layer = workloads.make_layer(wl.shape, wl.wid, 0, cuda_device, wl.bias_mode)
-    for T, sub in ((16, 1), (200, 70)):
+    cases = ((16, 1, 0, moe.MOE_PATH_SMALL_BATCH), (200, 70, 0, moe.MOE_PATH_LARGE_STREAMING),
+             (200, 70, moe.MOE_FORCE_PREFILL, moe.MOE_PATH_TENSOR_CORE))
+    for T, sub, flags, path in cases:
+        assert moe.layer_path(wl.shape, T, flags) == path
+        assert moe.layer_path(wl.shape, sub, flags) == path
         x = workloads.make_x(wl.shape, T, wl.wid, batch=5, device=cuda_device)
-        out, _, _ = run(moe, x, layer, wl.shape)
+        out, _, _ = run(moe, x, layer, wl.shape, flags=flags)
         perm = torch.randperm(T, generator=torch.Generator().manual_seed(T)).to(cuda_device)
-        outp, _, _ = run(moe, x[perm].contiguous(), layer, wl.shape)
+        outp, _, _ = run(moe, x[perm].contiguous(), layer, wl.shape, flags=flags)
         assert torch.equal(outp, out[perm])
         for t0 in (0, T // 2, T - sub):
-            o1, _, _ = run(moe, x[t0:t0 + sub].contiguous(), layer, wl.shape)
+            o1, _, _ = run(moe, x[t0:t0 + sub].contiguous(), layer, wl.shape, flags=flags)
             assert torch.equal(o1, out[t0:t0 + sub])
 
 
