@@ -255,20 +255,23 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
     }
     const int ntiles = cdiv(T, kRouterTileTokens);
     p.router_blocks = ntiles < kRouterMaxBlocks ? ntiles : kRouterMaxBlocks;
+    // large batches whose expert kernels both take the TMA-ring kernels stream
+    // an expert's weights once for up to kMaxChunk of its tokens
+    const bool w2_tma = experts_w2_tma(cfg->H, cfg->I, cfg->Is);
+    p.chunk = path == Path::kLargeStreaming && experts_w13_tma(cfg->H) && w2_tma ? kMaxChunk : kChunkTokens;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const long long TK = (long long)T * cfg->K;
-    const long long routed_buckets = (cfg->E < TK ? cfg->E : TK) + cdiv(TK, kChunkTokens);
-    const long long shared_chunks = cfg->Is > 0 ? cdiv(T, kChunkTokens) : 0;
+    const long long routed_buckets = (cfg->E < TK ? cfg->E : TK) + cdiv(TK, p.chunk);
+    const long long shared_chunks = cfg->Is > 0 ? cdiv(T, p.chunk) : 0;
     // upper bounds of the weight-streaming kernels' CTA tasks
     const long long tasks13 = (long long)(cfg->I / 64) * routed_buckets + (long long)(cfg->Is / 64) * shared_chunks;
     const long long tasks2 = (long long)(cfg->H / p.rows2) *
                              (routed_buckets * slices_of(cfg->I) + shared_chunks * slices_of(cfg->Is));
     int grid13 = 0, grid2 = 0;
     if (!use_tc) {
-        const bool w2_tma = experts_w2_tma(cfg->H, cfg->I, cfg->Is);
-        const long long cap13 = experts_resident_ctas(0, cfg->H, w2_tma);
-        const long long cap2 = experts_resident_ctas(1, cfg->H, w2_tma);
+        const long long cap13 = experts_resident_ctas(0, cfg->H, w2_tma, p.chunk);
+        const long long cap2 = experts_resident_ctas(1, cfg->H, w2_tma, p.chunk);
         grid13 = (int)(tasks13 < cap13 ? tasks13 : cap13);
         grid2 = (int)(tasks2 < cap2 ? tasks2 : cap2);
     }

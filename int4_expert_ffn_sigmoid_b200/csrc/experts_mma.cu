@@ -102,9 +102,9 @@ struct Shm {
     TaskDesc td[kMaxCtaTasks];                    // the first tasks of this CTA, in its order
     int tok[kMaxSlots];                           // token of each routed slot (T*K <= kMaxSlots)
     float xsr[2][kChunkTokens];                   // gate/up: activation scale of each token (per buffer)
-    float hmr[kChunkTokens][kSliceK / kRows13];   // down: the slice's per-64-row maxima of |h|
-    float xsc[kChunkTokens];                      // down: activation scale / 16 of each token
-    QScale qs[kChunkTokens];                      // down: activation scale of each token
+    float hmr[kMaxChunk][kSliceK / kRows13];      // down: the slice's per-64-row maxima of |h|
+    float xsc[kMaxChunk];                         // down: activation scale / 16 of each token
+    QScale qs[kMaxChunk];                         // down: activation scale of each token
     float hm[8][kChunkTokens];                    // gate/up: per-warp max |h| of each token
 };
 constexpr size_t kShmBytes = (sizeof(Shm) + 127) & ~size_t(127);
@@ -197,8 +197,8 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
             c[j] = e < E ? s_cnt[e] : 0;
             v[0] += c[j];
             v[1] += c[j] > 0;
-            v[2] += R13 * chunks_of(c[j]);
-            v[3] += R2 * chunks_of(c[j]);
+            v[2] += R13 * chunks_of(c[j], p.chunk);
+            v[3] += R2 * chunks_of(c[j], p.chunk);
         }
         int inc[4] = {v[0], v[1], v[2], v[3]};
 #pragma unroll
@@ -228,8 +228,8 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
                     ++b;
                 }
                 off += c[j];
-                b13 += R13 * chunks_of(c[j]);
-                b2 += R2 * chunks_of(c[j]);
+                b13 += R13 * chunks_of(c[j], p.chunk);
+                b2 += R2 * chunks_of(c[j], p.chunk);
             }
         }
         const int total = __shfl_sync(0xffffffffu, inc[0], 31);
@@ -252,8 +252,8 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
                     p.bucket_off[nb] = TK;
                     p.ts2[nb] = t2;
                 }
-                t13 += (p.Is / kTaskRows13) * chunks_of(T);
-                t2 += (p.H / p.rows2) * slices_of(p.Is) * chunks_of(T);
+                t13 += (p.Is / kTaskRows13) * chunks_of(T, p.chunk);
+                t2 += (p.H / p.rows2) * slices_of(p.Is) * chunks_of(T, p.chunk);
                 ++nb;
             }
             tb.ts[nb] = t13;
@@ -438,8 +438,8 @@ __device__ __forceinline__ Task13 make13(const Params& p, int e, int n, int off,
     const int R = t.irow / kRows13;
     const int c = local / R;
     t.rbk = local - c * R;
-    t.tok0 = c * kChunkTokens;
-    t.nc = min(kChunkTokens, n - t.tok0);
+    t.tok0 = c * p.chunk;
+    t.nc = min(p.chunk, n - t.tok0);
     t.r0 = t.rbk * kRows13 + warp * 8;
     const int row_bytes = p.H / 2;
     const uint8_t* W = t.shared ? p.sh_w13 : p.w13 + (size_t)(t.ok ? e : 0) * 2 * p.I * row_bytes;
@@ -481,8 +481,8 @@ __device__ __forceinline__ TaskDesc decode_task(const Params& p, const Tables& t
     }
     d.e = e;
     d.off = tb.off[b];
-    d.tok0 = c * kChunkTokens;
-    d.nc = min(kChunkTokens, n - d.tok0);
+    d.tok0 = c * p.chunk;
+    d.nc = min(p.chunk, n - d.tok0);
     return d;
 }
 
@@ -603,7 +603,7 @@ __global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
     // depend on the routing: a CTA whose first task is one starts its weight
     // stream before the router has finished; the rest of the shared expert
     // is warmed in L2.
-    const int ns = p.Is > 0 ? (p.Is / kRows13) * chunks_of(p.T) : 0;
+    const int ns = p.Is > 0 ? (p.Is / kRows13) * chunks_of(p.T, p.chunk) : 0;
     bool primed = false;
     const uint8_t* primed_ra = nullptr;
     if ((int)blockIdx.x < ns) {
@@ -833,7 +833,7 @@ __global__ void __launch_bounds__(256, 1) experts_w13_bulk_kernel(Params p) {
     (void)wslot_bytes;
     // A CTA whose first task belongs to the shared expert fetches its weights
     // before the router has finished.
-    const int ns = p.Is > 0 ? (p.Is / kRows13) * chunks_of(p.T) : 0;
+    const int ns = p.Is > 0 ? (p.Is / kRows13) * chunks_of(p.T, p.chunk) : 0;
     bool pre = false;
     const uint8_t* pre_ra = nullptr;
     if ((int)blockIdx.x < ns) {
@@ -925,18 +925,23 @@ __global__ void __launch_bounds__(256, 1) experts_w13_bulk_kernel(Params p) {
 // stages hold, and the producer waits (bounded) for its last copies before
 // it exits.
 // ---------------------------------------------------------------------------
-constexpr int kTmaStages = 8;
 constexpr int kTmaChunk = 256;                                 // k elements per stage
 constexpr int kTmaRowBytes = kTmaChunk / 2;                    // 128 bytes of codes per row and stage
 constexpr int kTmaWBytes = 2 * kRows13 * kTmaRowBytes;         // gate + up tiles: 16 KB
 constexpr int kTmaXStride = kTmaChunk + kPadB;                 // staged activation row
-constexpr int kTmaXBytes = kStageRows * kTmaXStride;
 constexpr int kTmaThreads = 288;                               // 8 consumer warps + the producer warp
-constexpr size_t kTmaMiscBytes = 256 + 2 * 8 * kChunkTokens * 4;  // barriers, flag, per-warp maxima
-constexpr size_t kSmem13Tma = kShmBytes + kTmaMiscBytes + 1024 /* alignment */ +
-                              (size_t)kTmaStages * (kTmaWBytes + kTmaXBytes);
-static_assert(kSmem13Tma <= 227 * 1024, "TMA gate/up shared memory");
-static_assert((size_t)kTmaStages * kTmaXBytes >= kBuildBytes, "table build scratch fits the activation ring");
+// Ring geometry for tasks of kChunk tokens: the activation part of a stage
+// holds 2 kChunk rows, and the ring is as deep as shared memory allows
+// (8 stages for 16 tokens, 6 for 32).
+template <int kChunk>
+struct Tma13 {
+    static constexpr int kStages = kChunk == kChunkTokens ? 8 : 6;
+    static constexpr int kXBytes = 2 * kChunk * kTmaXStride;
+    static constexpr size_t kMisc = 256 + 2 * 8 * kChunk * 4;  // barriers, flag, per-warp maxima
+    static constexpr size_t kSmem = kShmBytes + kMisc + 1024 /* alignment */ + (size_t)kStages * (kTmaWBytes + kXBytes);
+    static_assert(kSmem <= 227 * 1024, "TMA gate/up shared memory");
+    static_assert((size_t)kStages * kXBytes >= kBuildBytes, "table build scratch fits the activation ring");
+};
 
 __device__ __forceinline__ void bar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar)))
@@ -965,7 +970,7 @@ __device__ __forceinline__ void issue_w13_chunk(const CUtensorMap* map, uint64_t
 }
 
 // Consumer main loop of one task: nch stages from stage counter n on.
-template <int NT>
+template <int NT, int kStages, int kXBytes>
 __device__ __forceinline__ void consume13(int nch, uint32_t& n, uint64_t* full, uint64_t* empty, const uint8_t* wring,
                                           const uint8_t* xring, volatile int* abort, unsigned* status,
                                           int (&acc)[NT][4]) {
@@ -979,13 +984,13 @@ __device__ __forceinline__ void consume13(int nch, uint32_t& n, uint64_t* full, 
     // row warp*8 + g of a 1024-byte aligned tile: its 16-byte chunk j sits at j ^ g
     const int wrow = (warp * 8 + g) * kTmaRowBytes;
     for (int c = 0; c < nch; ++c, ++n) {
-        const int s = n % kTmaStages;
-        if (!*abort && !bar_wait(full + s, (n / kTmaStages) & 1, kBulkWaitCycles)) {
+        const int s = n % kStages;
+        if (!*abort && !bar_wait(full + s, (n / kStages) & 1, kBulkWaitCycles)) {
             *abort = 1;
             if (lane == 0) atomicOr(status, ST_TIMEOUT);
         }
         const uint8_t* wt = wring + (size_t)s * kTmaWBytes + wrow;
-        const uint8_t* xt = xring + (size_t)s * kTmaXBytes + g * kTmaXStride + q * 32;
+        const uint8_t* xt = xring + (size_t)s * kXBytes + g * kTmaXStride + q * 32;
 #pragma unroll
         for (int kb = 0; kb < kTmaChunk / 128; ++kb) {
             const int off = ((kb * 4 + q) ^ g) << 4;
@@ -1002,24 +1007,27 @@ __device__ __forceinline__ void consume13(int nch, uint32_t& n, uint64_t* full, 
         for (int c = 0; c < 4; ++c) acc[i][c] = part[0][i][c] + part[kSets - 1][i][c] * (kSets - 1);
 }
 
+template <int kChunk>
 __global__ void __launch_bounds__(kTmaThreads, 1)
     experts_w13_tma_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_s, Params p) {
+    using Cfg = Tma13<kChunk>;
+    constexpr int kStages = Cfg::kStages, kXBytes = Cfg::kXBytes;
     extern __shared__ __align__(128) uint8_t dsm[];
     Shm& sh = *reinterpret_cast<Shm*>(dsm);
     uint64_t* full = reinterpret_cast<uint64_t*>(dsm + kShmBytes);
-    uint64_t* empty = full + kTmaStages;
-    volatile int* abort = reinterpret_cast<volatile int*>(empty + kTmaStages);
-    float(*hm2)[8][kChunkTokens] = reinterpret_cast<float(*)[8][kChunkTokens]>(dsm + kShmBytes + 256);
+    uint64_t* empty = full + kStages;
+    volatile int* abort = reinterpret_cast<volatile int*>(empty + kStages);
+    float(*hm2)[8][kChunk] = reinterpret_cast<float(*)[8][kChunk]>(dsm + kShmBytes + 256);
     const uint32_t base_s = static_cast<uint32_t>(__cvta_generic_to_shared(dsm));
-    const uint32_t ring_s = (base_s + (uint32_t)(kShmBytes + kTmaMiscBytes) + 1023u) & ~1023u;
+    const uint32_t ring_s = (base_s + (uint32_t)(kShmBytes + Cfg::kMisc) + 1023u) & ~1023u;
     uint8_t* wring = dsm + (ring_s - base_s);
-    uint8_t* xring = wring + (size_t)kTmaStages * kTmaWBytes;
+    uint8_t* xring = wring + (size_t)kStages * kTmaWBytes;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const bool producer = warp == 8;
     const int H = p.H, nch = H / kTmaChunk;
     unsigned* status = &p.ctrl->status;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kTmaStages; ++i) {
+        for (int i = 0; i < kStages; ++i) {
             bar_init(full + i, 1 + 32);  // the tile loads' arrival + one cp.async arrival per producer lane
             bar_init(empty + i, 8);      // one arrival per consumer warp
         }
@@ -1028,14 +1036,14 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     }
     __syncthreads();
     // the shared expert's first task of this CTA, if its first task is one
-    const int ns = p.Is > 0 ? (p.Is / kRows13) * chunks_of(p.T) : 0;
+    const int ns = p.Is > 0 ? (p.Is / kRows13) * chunks_of(p.T, p.chunk) : 0;
     const bool pre = (int)blockIdx.x < ns;
-    const int npre = pre ? min(kTmaStages, nch) : 0;
+    const int npre = pre ? min(kStages, nch) : 0;
     int pre_rbk = 0, pre_tok0 = 0;
     if (pre) {
         const int R = p.Is / kRows13, local = ns - 1 - (int)blockIdx.x;
         pre_rbk = local % R;
-        pre_tok0 = (local / R) * kChunkTokens;
+        pre_tok0 = (local / R) * p.chunk;
         if (producer && lane == 0)
             for (int c = 0; c < npre; ++c)
                 issue_w13_chunk(&tm_s, full + c, wring + (size_t)c * kTmaWBytes, c, pre_rbk * kRows13,
@@ -1059,24 +1067,29 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     if (!producer && *abort) return;
     if (producer) {
         uint32_t n = 0;
-        int last_round[kTmaStages];
+        int last_round[kStages];
 #pragma unroll
-        for (int s = 0; s < kTmaStages; ++s) last_round[s] = s < npre ? 0 : -1;
+        for (int s = 0; s < kStages; ++s) last_round[s] = s < npre ? 0 : -1;
         for (int r = 0; !*abort && snake(blockIdx.x, r) < ntask; ++r) {
             const TaskDesc d = task_desc(p, sh, 0, r);
             if (d.e < 0 || d.e > p.E || (d.e == p.E && p.Is == 0)) break;  // the consumers flag it
             const bool shared = d.e == p.E;
             const int irow = shared ? p.Is : p.I;
             const int rg = (shared ? 0 : d.e * 2 * p.I) + d.rbk * kRows13, ru = rg + irow;
-            // lane l < 2 nc copies activation row l (part l & 1 of the chunk's token l >> 1)
-            const int8_t* src = nullptr;
-            if (lane < 2 * d.nc) {
-                const int tok = slot_token(p, sh, shared, d.off, d.tok0 + (lane >> 1));
-                if (tok >= 0 && tok < p.T) src = p.xq + (size_t)tok * 2 * H + (lane & 1) * H;
+            // lane l copies activation rows l and l + 32 (row r: part r & 1 of the
+            // chunk's token r >> 1)
+            const int8_t* src[2] = {nullptr, nullptr};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int row = lane + 32 * h;
+                if (row < 2 * d.nc) {
+                    const int tok = slot_token(p, sh, shared, d.off, d.tok0 + (row >> 1));
+                    if (tok >= 0 && tok < p.T) src[h] = p.xq + (size_t)tok * 2 * H + (row & 1) * H;
+                }
             }
             for (int c = 0; c < nch; ++c, ++n) {
-                const int s = n % kTmaStages;
-                const int round = (int)(n / kTmaStages);
+                const int s = n % kStages;
+                const int round = (int)(n / kStages);
                 const bool issued = r == 0 && c < npre;  // weights issued before the wait
                 if (round > 0) {
                     bool ok = *abort == 0 && bar_wait(empty + s, (round - 1) & 1, kBulkWaitCycles);
@@ -1088,11 +1101,14 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
                 }
                 if (lane == 0 && !issued)
                     issue_w13_chunk(shared ? &tm_s : &tm_r, full + s, wring + (size_t)s * kTmaWBytes, c, rg, ru);
-                if (src) {
-                    uint8_t* dst = xring + (size_t)s * kTmaXBytes + lane * kTmaXStride;
 #pragma unroll
-                    for (int j = 0; j < kTmaChunk / 16; ++j) cp_async16(dst + j * 16, src + c * kTmaChunk + j * 16);
-                }
+                for (int h = 0; h < 2; ++h)
+                    if (src[h]) {
+                        uint8_t* dst = xring + (size_t)s * kXBytes + (lane + 32 * h) * kTmaXStride;
+#pragma unroll
+                        for (int j = 0; j < kTmaChunk / 16; ++j)
+                            cp_async16(dst + j * 16, src[h] + c * kTmaChunk + j * 16);
+                    }
                 cp_async_arrive(full + s);
                 last_round[s] = round;
             }
@@ -1102,7 +1118,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         if (*abort) {
             for (int s = 0; s < npre; ++s)
                 if (last_round[s] == 0 && n <= (uint32_t)s) cp_async_arrive(full + s);
-            for (int s = 0; s < kTmaStages; ++s)
+            for (int s = 0; s < kStages; ++s)
                 if (last_round[s] >= 0) bar_wait(full + s, last_round[s] & 1, kBulkWaitCycles);
         }
         cp_async_wait<0>();
@@ -1119,9 +1135,10 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         const float* S = t.shared ? p.sh_s13 : p.s13 + (size_t)t.e * 2 * p.I;
         const float gs = __ldg(S + t.r0 + g), us = __ldg(S + t.irow + t.r0 + g);
         const int NTt = (2 * t.nc + 7) >> 3;
-        float xsc[4];
+        constexpr int kMaxNT = kChunk / 4;
+        float xsc[kMaxNT];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kMaxNT; ++i) {
             const int j = 4 * i + q;
             xsc[i] = 0.f;
             if (i < NTt && j < t.nc) {
@@ -1129,18 +1146,26 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
                 xsc[i] = (tok >= 0 && tok < p.T) ? __ldcg(p.xs + tok) * 0.0625f : 0.f;
             }
         }
-        int acc[4][4];
+        int acc[kMaxNT][4];
+#define MOE_CONSUME13(N)                                                                                        \
+    consume13<N, kStages, kXBytes>(nch, n, full, empty, wring, xring, abort, status,                          \
+                                   reinterpret_cast<int(&)[N][4]>(acc))
         switch (NTt) {
-            case 1: consume13<1>(nch, n, full, empty, wring, xring, abort, status, reinterpret_cast<int(&)[1][4]>(acc)); break;
-            case 2: consume13<2>(nch, n, full, empty, wring, xring, abort, status, reinterpret_cast<int(&)[2][4]>(acc)); break;
-            case 3: consume13<3>(nch, n, full, empty, wring, xring, abort, status, reinterpret_cast<int(&)[3][4]>(acc)); break;
-            default: consume13<4>(nch, n, full, empty, wring, xring, abort, status, acc); break;
+            case 1: MOE_CONSUME13(1); break;
+            case 2: MOE_CONSUME13(2); break;
+            case 3: MOE_CONSUME13(3); break;
+            case 4: MOE_CONSUME13(4); break;
+            case 5: MOE_CONSUME13((kMaxNT > 4 ? 5 : 1)); break;
+            case 6: MOE_CONSUME13((kMaxNT > 4 ? 6 : 1)); break;
+            case 7: MOE_CONSUME13((kMaxNT > 4 ? 7 : 1)); break;
+            default: MOE_CONSUME13(kMaxNT); break;
         }
+#undef MOE_CONSUME13
         const int slot0 = (t.shared ? 0 : t.off) + t.tok0;
         float* hrow0 = (t.shared ? p.h32_s : p.h32_r) + (size_t)slot0 * t.irow + t.r0 + g;
-        float(*hm)[kChunkTokens] = hm2[r & 1];
+        float(*hm)[kChunk] = hm2[r & 1];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kMaxNT; ++i) {
             if (i >= NTt) break;
             const int j = 4 * i + q;
             float hmv = 0.f;
@@ -1191,8 +1216,8 @@ __device__ __forceinline__ Task2 make2(const Params& p, int e, int n, int off, i
     const int c = rest / nsl;
     t.k0 = t.sl * kSliceK;
     t.klen = min(kSliceK, t.irow - t.k0);
-    t.tok0 = c * kChunkTokens;
-    t.nc = min(kChunkTokens, n - t.tok0);
+    t.tok0 = c * p.chunk;
+    t.nc = min(p.chunk, n - t.tok0);
     t.row0 = rbk * p.rows2;
     t.ng = p.rows2 / kRows2;
     t.j0 = warp * 16;
@@ -1303,7 +1328,7 @@ __global__ void __launch_bounds__(256, 2) experts_w2_kernel(Params p) {
     float* rs2 = reinterpret_cast<float*>(xs + kRs2Off);  // [task parity][row of the task]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     Ring ring;
-    const int ns = p.Is > 0 ? (p.H / p.rows2) * chunks_of(p.T) * slices_of(p.Is) : 0;
+    const int ns = p.Is > 0 ? (p.H / p.rows2) * chunks_of(p.T, p.chunk) * slices_of(p.Is) : 0;
     bool primed = false;
     const uint8_t* primed_ra = nullptr;
     if ((int)blockIdx.x < ns) {
@@ -1377,11 +1402,16 @@ __global__ void __launch_bounds__(256, 2) experts_w2_kernel(Params p) {
 // ---------------------------------------------------------------------------
 constexpr int kW2Bytes = kRows2 * kTmaRowBytes;  // one stage: 16 KB
 constexpr size_t kW2MiscBytes = 256;
-constexpr size_t kW2XOff = (size_t)kTmaStages * kW2Bytes;           // from the ring's start
-constexpr size_t kW2RawOff = kW2XOff + (size_t)kStageRows * kStride2;
-constexpr size_t kW2RsOff = kW2RawOff + (size_t)kChunkTokens * kSliceK * 4;
-constexpr size_t kSmem2Tma = kShmBytes + kW2MiscBytes + 1024 /* alignment */ + kW2RsOff + (size_t)2 * kMaxRows2 * 4;
-static_assert(kSmem2Tma <= 227 * 1024, "TMA down shared memory");
+// Ring and staging for tasks of kChunk tokens (offsets from the ring's start).
+template <int kChunk>
+struct Tma2 {
+    static constexpr int kStages = kChunk == kChunkTokens ? 8 : 6;
+    static constexpr size_t kXOff = (size_t)kStages * kW2Bytes;
+    static constexpr size_t kRawOff = kXOff + (size_t)2 * kChunk * kStride2;
+    static constexpr size_t kRsOff = kRawOff + (size_t)kChunk * kSliceK * 4;
+    static constexpr size_t kSmem = kShmBytes + kW2MiscBytes + 1024 /* alignment */ + kRsOff + (size_t)2 * kMaxRows2 * 4;
+    static_assert(kSmem <= 227 * 1024, "TMA down shared memory");
+};
 
 __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
@@ -1407,7 +1437,7 @@ __device__ __forceinline__ void fetch2c(const Params& p, Shm& sh, const Task2& t
     cp_async_commit();
 }
 
-template <int NT>
+template <int NT, int kStages>
 __device__ __forceinline__ void consume2(const Task2& tk, uint32_t& n, uint64_t* full, uint64_t* empty,
                                          const uint8_t* wring, const uint8_t* xs, const float* rs, const Params& p,
                                          const Shm& sh, volatile int* abort, unsigned* status) {
@@ -1425,8 +1455,8 @@ __device__ __forceinline__ void consume2(const Task2& tk, uint32_t& n, uint64_t*
 #pragma unroll
             for (int i = 0; i < NT; ++i) part[s][i][0] = part[s][i][1] = part[s][i][2] = part[s][i][3] = 0;
         for (int c = 0; c < nkc; ++c, ++n) {
-            const int s = n % kTmaStages;
-            if (!*abort && !bar_wait(full + s, (n / kTmaStages) & 1, kBulkWaitCycles)) {
+            const int s = n % kStages;
+            if (!*abort && !bar_wait(full + s, (n / kStages) & 1, kBulkWaitCycles)) {
                 *abort = 1;
                 if (lane == 0) atomicOr(status, ST_TIMEOUT);
             }
@@ -1462,24 +1492,27 @@ __device__ __forceinline__ void consume2(const Task2& tk, uint32_t& n, uint64_t*
     }
 }
 
+template <int kChunk>
 __global__ void __launch_bounds__(kTmaThreads, 1)
     experts_w2_tma_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_s, Params p) {
+    using Cfg = Tma2<kChunk>;
+    constexpr int kStages = Cfg::kStages;
     extern __shared__ __align__(128) uint8_t dsm[];
     Shm& sh = *reinterpret_cast<Shm*>(dsm);
     uint64_t* full = reinterpret_cast<uint64_t*>(dsm + kShmBytes);
-    uint64_t* empty = full + kTmaStages;
-    volatile int* abort = reinterpret_cast<volatile int*>(empty + kTmaStages);
+    uint64_t* empty = full + kStages;
+    volatile int* abort = reinterpret_cast<volatile int*>(empty + kStages);
     const uint32_t base_s = static_cast<uint32_t>(__cvta_generic_to_shared(dsm));
     const uint32_t ring_s = (base_s + (uint32_t)(kShmBytes + kW2MiscBytes) + 1023u) & ~1023u;
     uint8_t* wring = dsm + (ring_s - base_s);
-    uint8_t* xs = wring + kW2XOff;
-    float* raw = reinterpret_cast<float*>(wring + kW2RawOff);
-    float* rs2 = reinterpret_cast<float*>(wring + kW2RsOff);  // [task parity][row of the task]
+    uint8_t* xs = wring + Cfg::kXOff;
+    float* raw = reinterpret_cast<float*>(wring + Cfg::kRawOff);
+    float* rs2 = reinterpret_cast<float*>(wring + Cfg::kRsOff);  // [task parity][row of the task]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool producer = warp == 8;
     unsigned* status = &p.ctrl->status;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kTmaStages; ++i) {
+        for (int i = 0; i < kStages; ++i) {
             bar_init(full + i, 1);   // the tile load's arrival
             bar_init(empty + i, 8);  // one arrival per consumer warp
         }
@@ -1490,16 +1523,16 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     const int R = p.H / p.rows2, ng = p.rows2 / kRows2;
     // the shared expert's first task of this CTA, if its first task is one
     const int nsl_s = p.Is > 0 ? slices_of(p.Is) : 0;
-    const int ns = p.Is > 0 ? R * chunks_of(p.T) * nsl_s : 0;
+    const int ns = p.Is > 0 ? R * chunks_of(p.T, p.chunk) * nsl_s : 0;
     const bool pre = (int)blockIdx.x < ns;
     int pre_rbk = 0, pre_sl = 0, pre_tok0 = 0, npre = 0;
     if (pre) {
         const int local = ns - 1 - (int)blockIdx.x, rest = local / R;
         pre_rbk = local % R;
         pre_sl = rest % nsl_s;
-        pre_tok0 = (rest / nsl_s) * kChunkTokens;
+        pre_tok0 = (rest / nsl_s) * p.chunk;
         const int k0 = pre_sl * kSliceK, nkc = min(kSliceK, p.Is - k0) / kTmaChunk;
-        npre = min(kTmaStages, ng * nkc);
+        npre = min(kStages, ng * nkc);
         if (producer && lane == 0)
             for (int i = 0; i < npre; ++i) {
                 const int m = i / nkc, c = i - m * nkc;
@@ -1526,9 +1559,9 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     if (!producer && *abort) return;
     if (producer) {
         uint32_t n = 0;
-        int last_round[kTmaStages];
+        int last_round[kStages];
 #pragma unroll
-        for (int s = 0; s < kTmaStages; ++s) last_round[s] = s < npre ? 0 : -1;
+        for (int s = 0; s < kStages; ++s) last_round[s] = s < npre ? 0 : -1;
         for (int r = 0; !*abort && snake(blockIdx.x, r) < ntask; ++r) {
             const TaskDesc d = task_desc(p, sh, 1, r);
             if (d.e < 0 || d.e > p.E || (d.e == p.E && p.Is == 0)) break;  // the consumers flag it
@@ -1540,8 +1573,8 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
             bool stop = false;
             for (int m = 0; m < ng && !stop; ++m)
                 for (int c = 0; c < nkc; ++c, ++n) {
-                    const int s = n % kTmaStages;
-                    const int round = (int)(n / kTmaStages);
+                    const int s = n % kStages;
+                    const int round = (int)(n / kStages);
                     if (round > 0) {
                         const bool ok = *abort == 0 && bar_wait(empty + s, (round - 1) & 1, kBulkWaitCycles);
                         if (__any_sync(0xffffffffu, !ok)) {
@@ -1560,7 +1593,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         }
         // copies nobody will consume land before the CTA exits
         if (*abort && lane == 0)
-            for (int s = 0; s < kTmaStages; ++s)
+            for (int s = 0; s < kStages; ++s)
                 if (last_round[s] >= 0) bar_wait(full + s, last_round[s] & 1, kBulkWaitCycles);
         __syncwarp();
         return;
@@ -1603,12 +1636,19 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         consumers_sync();  // staged; raw and hmr are free for the next task
         if (nx.ok) fetch2c(p, sh, nx, raw, rs2 + ((r + 1) & 1) * kMaxRows2);
         const float* rs = rs2 + (r & 1) * kMaxRows2;
+        constexpr int kMaxNT = kChunk / 4;
+#define MOE_CONSUME2(N) consume2<N, kStages>(cur, n, full, empty, wring, xs, rs, p, sh, abort, status)
         switch ((2 * nc + 7) >> 3) {
-            case 1: consume2<1>(cur, n, full, empty, wring, xs, rs, p, sh, abort, status); break;
-            case 2: consume2<2>(cur, n, full, empty, wring, xs, rs, p, sh, abort, status); break;
-            case 3: consume2<3>(cur, n, full, empty, wring, xs, rs, p, sh, abort, status); break;
-            default: consume2<4>(cur, n, full, empty, wring, xs, rs, p, sh, abort, status); break;
+            case 1: MOE_CONSUME2(1); break;
+            case 2: MOE_CONSUME2(2); break;
+            case 3: MOE_CONSUME2(3); break;
+            case 4: MOE_CONSUME2(4); break;
+            case 5: MOE_CONSUME2((kMaxNT > 4 ? 5 : 1)); break;
+            case 6: MOE_CONSUME2((kMaxNT > 4 ? 6 : 1)); break;
+            case 7: MOE_CONSUME2((kMaxNT > 4 ? 7 : 1)); break;
+            default: MOE_CONSUME2(kMaxNT); break;
         }
+#undef MOE_CONSUME2
         cur = nx;
     }
     cp_async_wait<0>();
@@ -1621,7 +1661,7 @@ bool w13_tma(int H) { return H >= kTmaMinH && H % kTmaChunk == 0; }
 
 template <typename Kern>
 int resident(Kern kern, size_t smem, int which, int threads = 256) {
-    static int cache[8][64];
+    static int cache[9][64];  // by kernel (`which`) and device
     static_assert(kSmem13Bulk <= 227 * 1024, "bulk gate/up shared memory");
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
@@ -1640,10 +1680,15 @@ int resident(Kern kern, size_t smem, int which, int threads = 256) {
 
 // Persistent grid of the weight-streaming kernels: the CTAs that fit at once
 // (which: 0 gate/up, 1 down).  Also sets the kernels' shared-memory limits.
-int experts_resident_ctas(int which, int H, bool w2_tma) {
-    if (which == 1) return w2_tma ? resident(experts_w2_tma_kernel, kSmem2Tma, 6, kTmaThreads)
-                                  : resident(experts_w2_kernel, kSmem2, 3);
-    if (w13_tma(H)) return resident(experts_w13_tma_kernel, kSmem13Tma, 5, kTmaThreads);
+int experts_resident_ctas(int which, int H, bool w2_tma, int chunk) {
+    if (which == 1) {
+        if (!w2_tma) return resident(experts_w2_kernel, kSmem2, 3);
+        return chunk == kMaxChunk ? resident(experts_w2_tma_kernel<kMaxChunk>, Tma2<kMaxChunk>::kSmem, 7, kTmaThreads)
+                                  : resident(experts_w2_tma_kernel<kChunkTokens>, Tma2<kChunkTokens>::kSmem, 6, kTmaThreads);
+    }
+    if (w13_tma(H))
+        return chunk == kMaxChunk ? resident(experts_w13_tma_kernel<kMaxChunk>, Tma13<kMaxChunk>::kSmem, 8, kTmaThreads)
+                                  : resident(experts_w13_tma_kernel<kChunkTokens>, Tma13<kChunkTokens>::kSmem, 5, kTmaThreads);
     if (H <= kBulkMaxK) return resident(experts_w13_bulk_kernel, kSmem13Bulk, 4);
     const int mode = H <= kDoubleMaxK ? 0 : H <= kWholeMaxK ? 1 : 2;
     switch (mode) {
@@ -1666,7 +1711,11 @@ cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
                                  p.H / 2, p.Is > 0 ? 2 * (uint64_t)p.Is : 2 * (uint64_t)kRows13, kTmaRowBytes, kRows13,
                                  CU_TENSOR_MAP_SWIZZLE_128B);
         if (!ok) return cudaErrorInvalidValue;
-        return launch_pdl(experts_w13_tma_kernel, g, dim3(kTmaThreads), kSmem13Tma, stream, tm_r, tm_s, p);
+        if (p.chunk == kMaxChunk)
+            return launch_pdl(experts_w13_tma_kernel<kMaxChunk>, g, dim3(kTmaThreads), Tma13<kMaxChunk>::kSmem, stream,
+                              tm_r, tm_s, p);
+        return launch_pdl(experts_w13_tma_kernel<kChunkTokens>, g, dim3(kTmaThreads), Tma13<kChunkTokens>::kSmem, stream,
+                          tm_r, tm_s, p);
     }
     if (p.H <= kBulkMaxK) return launch_pdl(experts_w13_bulk_kernel, g, b, kSmem13Bulk, stream, p);
     const int mode = p.H <= kDoubleMaxK ? 0 : p.H <= kWholeMaxK ? 1 : 2;
@@ -1676,6 +1725,8 @@ cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
         default: return launch_pdl(experts_w13_kernel<2>, g, b, kSmem13[2], stream, p);
     }
 }
+
+bool experts_w13_tma(int H) { return w13_tma(H); }
 
 bool experts_w2_tma(int H, int I, int Is) { return H >= kTmaMinH && I % kTmaChunk == 0 && Is % kTmaChunk == 0; }
 
@@ -1690,7 +1741,11 @@ cudaError_t launch_experts_w2(const Params& p, int grid, cudaStream_t stream) {
             encode_tensor_map_2d(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.Is > 0 ? (const void*)p.sh_w2 : (const void*)p.w2,
                                  p.Is > 0 ? p.Is / 2 : p.I / 2, p.H, kTmaRowBytes, kRows2, CU_TENSOR_MAP_SWIZZLE_128B);
         if (!ok) return cudaErrorInvalidValue;
-        return launch_pdl(experts_w2_tma_kernel, dim3(grid), dim3(kTmaThreads), kSmem2Tma, stream, tm_r, tm_s, p);
+        if (p.chunk == kMaxChunk)
+            return launch_pdl(experts_w2_tma_kernel<kMaxChunk>, dim3(grid), dim3(kTmaThreads), Tma2<kMaxChunk>::kSmem,
+                              stream, tm_r, tm_s, p);
+        return launch_pdl(experts_w2_tma_kernel<kChunkTokens>, dim3(grid), dim3(kTmaThreads), Tma2<kChunkTokens>::kSmem,
+                          stream, tm_r, tm_s, p);
     }
     return launch_pdl(experts_w2_kernel, dim3(grid), dim3(256), kSmem2, stream, p);
 }

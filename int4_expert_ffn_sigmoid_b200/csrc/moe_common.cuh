@@ -16,10 +16,13 @@ constexpr int kDecodeMaxTokens = 64;
 constexpr int kTaskRows13 = 64;
 constexpr int kTaskRows2 = 128;
 constexpr int kMaxRows2 = 1024;
-// Tokens of one bucket handled by one weight-streaming task: each token
-// takes two int8 columns (its two activation parts), so 16 tokens fill four
-// mma n-tiles of 8 columns.
+// Tokens of one bucket handled by one weight-streaming task (Params::chunk):
+// each token takes two int8 columns (its two activation parts), so 16 tokens
+// fill four mma n-tiles of 8 columns.  Large batches whose expert kernels
+// both take the TMA-ring kernels use chunks of kMaxChunk tokens, so that an
+// expert's weights are streamed once for up to 32 of its tokens.
 constexpr int kChunkTokens = 16;
+constexpr int kMaxChunk = 32;
 // Reduction slice of the weight-streaming down projection: its activations
 // are quantized per (token, slice) and every slice writes its own partial
 // output row, summed by the combine.
@@ -157,6 +160,7 @@ struct Params {
     float* hmax_s;        // [T][Is/64]
     int nsl_r, nsl_s;     // slices of the down projection's reduction (routed, shared)
     int rows2;            // output rows of one down task (kTaskRows2 times 1..8, dividing H)
+    int chunk;            // tokens per weight-streaming task: kChunkTokens or kMaxChunk
     int decode_groups;    // token groups of the small-batch router (0: tables come from the large router)
     float* lpart;         // [lslices][T][E] partial router logits of the split small-batch router
     int lslices;          // hidden-dimension slices of lpart (0: the small-batch router computes its logits)
@@ -232,7 +236,7 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
 }
 
 // Bucket geometry of the expert kernels.
-__device__ __host__ __forceinline__ int chunks_of(int n) { return (n + kChunkTokens - 1) / kChunkTokens; }
+__device__ __host__ __forceinline__ int chunks_of(int n, int chunk) { return (n + chunk - 1) / chunk; }
 __device__ __host__ __forceinline__ int slices_of(int k) { return (k + kSliceK - 1) / kSliceK; }
 
 // ---------------------------------------------------------------------------

@@ -19,8 +19,9 @@ cudaError_t launch_experts_w2(const Params& p, int grid, cudaStream_t stream);
 // CTAs of the weight-streaming kernel `which` (0: gate/up, 1: down) that fit
 // on the device at once (the persistent grid size) for hidden size H.  Also
 // sets the kernel's shared-memory attribute.
-int experts_resident_ctas(int which, int H, bool w2_tma);
-// Whether the down projection takes the TMA-ring kernel for this shape.
+int experts_resident_ctas(int which, int H, bool w2_tma, int chunk);
+// Whether the gate/up (down) projection takes the TMA-ring kernel for this shape.
+bool experts_w13_tma(int H);
 bool experts_w2_tma(int H, int I, int Is);
 // Weighted combine + shared expert (+ residual) -> bf16 out.
 cudaError_t launch_combine(const Params& p, cudaStream_t stream);

@@ -243,7 +243,7 @@ __device__ void finalize_buckets(const Params& p, const int* s_cnt, int* s_off) 
                 const int e = p.bucket_e[b];
                 const int irow = (e == E) ? p.Is : p.I;
                 const int n = p.bucket_n[b];
-                const int ch = chunks_of(n);
+                const int ch = chunks_of(n, p.chunk);
                 n13 = (irow / kTaskRows13) * ch;                    // gate/up rows x a token chunk
                 n2 = (p.H / p.rows2) * ch * slices_of(irow);        // down rows x a chunk x a slice
                 if (e != E) {  // tensor-core tiles: 128 tokens x 128 features / 256 columns
