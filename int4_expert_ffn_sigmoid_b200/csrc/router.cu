@@ -322,7 +322,7 @@ constexpr int kRouterBatch = 8;  // router-weight blocks per batch of loads
 // (E * H f32, which every CTA of router_large_kernel reads) exceed
 // kRouterLargeMaxBytes.
 constexpr size_t kRouterWarpMaxBytes = 8192;
-constexpr size_t kRouterLargeMaxBytes = (size_t)2 << 20;
+constexpr size_t kRouterLargeMaxBytes = (size_t)512 << 10;
 constexpr int kLogitSliceBlocks = 3;   // 128-element blocks of the hidden dimension per slice
 constexpr int kLogitCtaExperts = 32;   // experts per CTA (4 per warp)
 constexpr int kLogitTileTokens = 64;   // tokens per CTA
@@ -663,14 +663,17 @@ __global__ void __launch_bounds__(256) router_large_kernel(Params p) {
                 if (ntile < n_ntiles) {
                     const int e = ntile * 8 + g;
                     const float* wrow = p.rw + (size_t)min(e, E - 1) * H + c * kRouterKC;
-                    for (int ks = 0; ks < kRouterKC / 16; ks += 2) {
-                        // B fragments of two k steps: w[k + 2q, +1] and w[k + 2q + 8, +9]
-                        float2 wv[2][2];
+                    // B fragments of every k step of the chunk, loaded together (one
+                    // round trip): w[k + 2q, +1] and w[k + 2q + 8, +9]
+                    float2 wall[kRouterKC / 16][2];
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            wv[u][0] = __ldg(reinterpret_cast<const float2*>(wrow + (ks + u) * 16 + 2 * q));
-                            wv[u][1] = __ldg(reinterpret_cast<const float2*>(wrow + (ks + u) * 16 + 2 * q + 8));
-                        }
+                    for (int k = 0; k < kRouterKC / 16; ++k) {
+                        wall[k][0] = __ldg(reinterpret_cast<const float2*>(wrow + k * 16 + 2 * q));
+                        wall[k][1] = __ldg(reinterpret_cast<const float2*>(wrow + k * 16 + 2 * q + 8));
+                    }
+#pragma unroll
+                    for (int ks = 0; ks < kRouterKC / 16; ks += 2) {
+                        const float2(*wv)[2] = &wall[ks];
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
                             uint32_t bh[2], bm[2], bl[2];
