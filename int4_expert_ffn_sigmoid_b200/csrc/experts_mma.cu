@@ -7,15 +7,23 @@
 // nanocolibri-engine README, "Converting a checkpoint yourself": per-row
 // symmetric int4, f32 row scales.
 //
-// Design.  One CTA (8 warps) owns one task and walks the reduction dimension
-// in 128-wide k blocks.  Gate/up task = (bucket, chunk of up to 16 of its
-// tokens, 64 gate rows + the same 64 up rows); down task = (bucket, chunk,
-// 512-wide slice of the intermediate dimension, 128 down rows).  The grid is
-// persistent; CTA c takes tasks c, c + grid, ... counted from the heaviest
-// end of the task list (the shared expert's tasks are at that end).
-//  - Weights go HBM -> registers: every thread streams 16 contiguous bytes
+// Design.  One CTA (8 compute warps) owns one task and walks the reduction
+// dimension in 128-wide k blocks.  Gate/up task = (bucket, chunk of up to 16
+// of its tokens (32 on large batches), 64 gate rows + the same 64 up rows);
+// down task = (bucket, chunk, 512-wide slice of the intermediate dimension,
+// a group of 128-row blocks).  The grid is persistent; CTA c takes tasks in
+// snake order counted from the heaviest end of the task list (the shared
+// expert's tasks are at that end).  Three ways to bring the weights in:
+//  - TMA ring (H >= 1024, multiples of 256; experts_w13_tma_kernel,
+//    experts_w2_tma_kernel): a producer warp keeps 6-8 stages of 16 KB of
+//    swizzled weight tiles in flight per SM across task boundaries; the
+//    compute warps read their fragments from shared memory.
+//  - Bulk copies (H < 1024, experts_w13_bulk_kernel): each warp's 16 rows of
+//    a task are two contiguous blocks fetched with cp.async.bulk two tasks
+//    ahead.
+//  - Register ring (other shapes): every thread streams 16 contiguous bytes
 //    (32 codes) of two rows per k block with non-allocating 128-bit loads,
-//    kept 4 k blocks ahead in a register ring; they never touch shared memory.
+//    kept 4 k blocks ahead in registers.
 //  - The codes become int8 operands 16*c with three logic operations per
 //    eight weights (lo8 / hi8), and feed mma.sync m16n8k32 (s8 x s8 -> s32).
 //    Thread q's 16-byte chunk of a row is exactly its A fragments of four
