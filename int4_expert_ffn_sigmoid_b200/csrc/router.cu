@@ -568,6 +568,7 @@ __global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(32 *
 constexpr int kRouterKC = 128;                // hidden elements per staged chunk (H % 128 == 0)
 constexpr int kRouterXS = kRouterKC + 8;      // padded row (bf16 elements)
 constexpr int kRouterMT = kRouterTileTokens / 16;
+constexpr int kRouterXStages = 4;             // staged chunks in flight
 
 __device__ __forceinline__ void split3(float w, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
     const __nv_bfloat16 h = __float2bfloat16_rn(w);
@@ -587,7 +588,7 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* smem_r
 
 __global__ void __launch_bounds__(256) router_large_kernel(Params p) {
     // the staged activations and, after the k loop, the tile's logits share one buffer
-    constexpr int kXBytes = 2 * kRouterTileTokens * kRouterXS * 2;
+    constexpr int kXBytes = kRouterXStages * kRouterTileTokens * kRouterXS * 2;
     constexpr int kLBytes = kRouterTileTokens * kMaxE * 4;
     __shared__ __align__(16) uint8_t s_buf[kXBytes > kLBytes ? kXBytes : kLBytes];
     __shared__ int s_cnt[kMaxE];
@@ -597,6 +598,19 @@ __global__ void __launch_bounds__(256) router_large_kernel(Params p) {
     const int g = lane >> 2, q = lane & 3;
     const int E = p.E, H = p.H;
     const int n_ntiles = (E + 7) / 8;
+    // B fragments of this warp's first n-tile for one chunk: w[k + 2q, +1] and
+    // w[k + 2q + 8, +9] of every k step, loaded together one chunk ahead (the
+    // first before waiting on the previous kernel: they do not depend on it)
+    float2 wpre[kRouterKC / 16][2];
+    auto load_w0 = [&](int c) {
+        const float* wrow = p.rw + (size_t)min(warp * 8 + g, E - 1) * H + c * kRouterKC;
+#pragma unroll
+        for (int k = 0; k < kRouterKC / 16; ++k) {
+            wpre[k][0] = __ldg(reinterpret_cast<const float2*>(wrow + k * 16 + 2 * q));
+            wpre[k][1] = __ldg(reinterpret_cast<const float2*>(wrow + k * 16 + 2 * q + 8));
+        }
+    };
+    if (p.lslices == 0 && warp < n_ntiles) load_w0(0);
     pdl_wait();
     reset_ctrl(p);
     pdl_release();
@@ -607,8 +621,8 @@ __global__ void __launch_bounds__(256) router_large_kernel(Params p) {
     for (int tile = blockIdx.x; tile < ntiles_tok; tile += gridDim.x) {
         const int t0 = tile * kRouterTileTokens;
         const int nt = min(kRouterTileTokens, p.T - t0);
-        for (int tt = warp; tt < nt; tt += 8) token_hexp(p, t0 + tt, lane);
         if (p.lslices > 0) {  // logits from the split kernel's partials, slice 0 first
+            for (int tt = warp; tt < nt; tt += 8) token_hexp(p, t0 + tt, lane);
             __syncthreads();  // s_logit is free (previous tile done)
             for (int i = threadIdx.x; i < nt * E; i += blockDim.x) {
                 const int tt = i / E, e = i - tt * E;
@@ -649,27 +663,53 @@ __global__ void __launch_bounds__(256) router_large_kernel(Params p) {
 #pragma unroll
             for (int m = 0; m < kRouterMT; ++m) acc[j][m][0] = acc[j][m][1] = acc[j][m][2] = acc[j][m][3] = 0.f;
 
+        // sum of squares of the tile's tokens from the staged chunks (k_t of the
+        // h scale): thread 8 r + u takes elements 16 u .. 16 u + 15 of row r of
+        // every chunk, and the 8 partial sums are added by an xor-butterfly
+        float sq = 0.f;
+        const int sq_row = threadIdx.x >> 3, sq_col = (threadIdx.x & 7) * 16;
         __syncthreads();  // s_x is free (previous tile done)
-        stage_chunk(0, 0);
-        for (int c = 0; c < nchunks; ++c) {
-            if (c + 1 < nchunks) stage_chunk(c + 1, (c + 1) & 1);
+#pragma unroll
+        for (int i = 0; i < kRouterXStages - 1; ++i) {
+            if (i < nchunks) stage_chunk(i, i);
             else asm volatile("cp.async.commit_group;" ::: "memory");
-            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        }
+        for (int c = 0; c < nchunks; ++c) {
+            const int cn = c + kRouterXStages - 1;  // into the buffer chunk c - 1 used
+            if (cn < nchunks) stage_chunk(cn, cn % kRouterXStages);
+            else asm volatile("cp.async.commit_group;" ::: "memory");
+            asm volatile("cp.async.wait_group %0;" ::"n"(kRouterXStages - 1) : "memory");
             __syncthreads();
-            const uint16_t (*xs)[kRouterXS] = s_x[c & 1];
+            const uint16_t (*xs)[kRouterXS] = s_x[c % kRouterXStages];
+            {
+                const uint4 a = *reinterpret_cast<const uint4*>(&xs[sq_row][sq_col]);
+                const uint4 b = *reinterpret_cast<const uint4*>(&xs[sq_row][sq_col + 8]);
+                sq = sq_step(sq, make_uint2(a.x, a.y));
+                sq = sq_step(sq, make_uint2(a.z, a.w));
+                sq = sq_step(sq, make_uint2(b.x, b.y));
+                sq = sq_step(sq, make_uint2(b.z, b.w));
+            }
 #pragma unroll
             for (int j = 0; j < kMaxE / 64; ++j) {
                 const int ntile = warp + 8 * j;
                 if (ntile < n_ntiles) {
                     const int e = ntile * 8 + g;
-                    const float* wrow = p.rw + (size_t)min(e, E - 1) * H + c * kRouterKC;
-                    // B fragments of every k step of the chunk, loaded together (one
-                    // round trip): w[k + 2q, +1] and w[k + 2q + 8, +9]
                     float2 wall[kRouterKC / 16][2];
+                    if (j == 0) {  // prefetched; fetch the next chunk's (or the next tile's first)
 #pragma unroll
-                    for (int k = 0; k < kRouterKC / 16; ++k) {
-                        wall[k][0] = __ldg(reinterpret_cast<const float2*>(wrow + k * 16 + 2 * q));
-                        wall[k][1] = __ldg(reinterpret_cast<const float2*>(wrow + k * 16 + 2 * q + 8));
+                        for (int k = 0; k < kRouterKC / 16; ++k) {
+                            wall[k][0] = wpre[k][0];
+                            wall[k][1] = wpre[k][1];
+                        }
+                        if (c + 1 < nchunks) load_w0(c + 1);
+                        else if (tile + (int)gridDim.x < ntiles_tok) load_w0(0);
+                    } else {  // every k step of the chunk loaded together (one round trip)
+                        const float* wrow = p.rw + (size_t)min(e, E - 1) * H + c * kRouterKC;
+#pragma unroll
+                        for (int k = 0; k < kRouterKC / 16; ++k) {
+                            wall[k][0] = __ldg(reinterpret_cast<const float2*>(wrow + k * 16 + 2 * q));
+                            wall[k][1] = __ldg(reinterpret_cast<const float2*>(wrow + k * 16 + 2 * q + 8));
+                        }
                     }
 #pragma unroll
                     for (int ks = 0; ks < kRouterKC / 16; ks += 2) {
@@ -703,6 +743,14 @@ __global__ void __launch_bounds__(256) router_large_kernel(Params p) {
                 }
             }
             __syncthreads();  // chunk c's readers are done before it is overwritten
+        }
+        sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+        sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+        sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+        if ((threadIdx.x & 7) == 0 && sq_row < nt) {
+            const float ms = sq / (float)H;
+            const int ex = (ms > 0.f && isfinite(ms)) ? ilogbf(ms) : 0;
+            p.hexp[t0 + sq_row] = min(max(kHExpBase + ex, kHExpMin), kHExpMax);
         }
 #pragma unroll
         for (int j = 0; j < kMaxE / 64; ++j) {
@@ -772,6 +820,7 @@ __global__ void __launch_bounds__(1024) router_finalize_kernel(Params p) {
 __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
     __shared__ int s_base[kMaxE];
     __shared__ int s_idx[kRouterTileTokens * kMaxK];
+    __shared__ int s_slot[kRouterTileTokens * kMaxK];  // -1: not copied
     const int E = p.E, K = p.K;
     const int TK = p.T * K;
     pdl_wait();
@@ -802,8 +851,10 @@ __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
             if (slot < 0 || slot >= TK) {
                 atomicOr(&p.ctrl->status, ST_BAD_SLOT);
                 p.slot_of[(size_t)t0 * K + i] = 0;
+                s_slot[i] = -1;
                 continue;
             }
+            s_slot[i] = slot;
             p.slot_of[(size_t)t0 * K + i] = slot;
             p.tok_of_slot[slot] = t0 + i / K;
         }
@@ -811,8 +862,8 @@ __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
         if (p.x_perm) {  // copy each token row to its slots (one warp per slot)
             const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
             for (int i = warp; i < n; i += blockDim.x / 32) {
-                if (s_idx[i] < 0) continue;
-                const int slot = p.slot_of[(size_t)t0 * K + i];
+                const int slot = s_slot[i];
+                if (slot < 0) continue;
                 const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)(t0 + i / K) * p.H);
                 uint4* dst = reinterpret_cast<uint4*>(p.x_perm + (size_t)slot * p.H);
                 for (int c = lane; c < p.H / 8; c += 32) dst[c] = __ldg(src + c);
