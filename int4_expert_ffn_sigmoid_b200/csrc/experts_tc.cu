@@ -388,8 +388,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
                 const uint8_t* raw = raw_tile(s);
                 uint8_t* bt = b_tile(sb);
                 {
-                    const uint4 q0 = *reinterpret_cast<const uint4*>(raw + r * 32);
-                    const uint4 q1 = *reinterpret_cast<const uint4*>(raw + r * 32 + 16);
+                    // the two 16-byte halves of this row, the half (r ^ r >> 2) & 1 first:
+                    // each quarter-warp's 8 reads then fall on 8 different 16-byte bank
+                    // groups (rows are 32 bytes apart)
+                    const int h0 = (r ^ (r >> 2)) & 1;
+                    const uint4 qa = *reinterpret_cast<const uint4*>(raw + r * 32 + 16 * h0);
+                    const uint4 qb = *reinterpret_cast<const uint4*>(raw + r * 32 + 16 * (h0 ^ 1));
+                    const uint4 q0 = h0 ? qb : qa, q1 = h0 ? qa : qb;
                     const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
                     uint8_t* row = bt + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll

@@ -586,7 +586,7 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* smem_r
                  : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_row))));
 }
 
-__global__ void __launch_bounds__(256) router_large_kernel(Params p) {
+__global__ void __launch_bounds__(256, 2) router_large_kernel(Params p) {
     // the staged activations and, after the k loop, the tile's logits share one buffer
     constexpr int kXBytes = kRouterXStages * kRouterTileTokens * kRouterXS * 2;
     constexpr int kLBytes = kRouterTileTokens * kMaxE * 4;
