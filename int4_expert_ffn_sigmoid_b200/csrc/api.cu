@@ -133,9 +133,9 @@ int32_t moe_decode_max_tokens(void) { return kDecodeMaxTokens; }
 int32_t moe_layer_kernel_launches(const moe_cfg_t* cfg, int32_t T) {
     if (validate_cfg(cfg) != MOE_OK || T <= 0 || T > kMaxTokens) return 0;
     // small batch: [router logits,] cluster router, gate/up, down, combine;
-    // otherwise: [router logits,] router, finalize, scatter, gate/up, down, combine
+    // otherwise: [router logits,] router, scatter, gate/up, down, combine
     const bool small = choose_path(*cfg, T) == Path::kSmall;
-    return (small ? 4 : 6) + (router_split_slices(cfg->E, cfg->H, small) > 0 ? 1 : 0);
+    return (small ? 4 : 5) + (router_split_slices(cfg->E, cfg->H, small) > 0 ? 1 : 0);
 }
 
 int32_t moe_layer_path(const moe_cfg_t* cfg, int32_t T) {

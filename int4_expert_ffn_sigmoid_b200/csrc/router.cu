@@ -546,14 +546,15 @@ __global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(32 *
 }
 
 // ---------------------------------------------------------------------------
-// Large batch, three kernels.
-// router_large_kernel: router_blocks CTAs walk tiles of 16 tokens (tile =
-// block, block + grid, ...); each tile's logits stay in shared memory, one
-// warp per token selects, and every CTA records its per-expert slot counts.
-// router_finalize_kernel: one CTA sums the counts, scans and builds the
-// bucket and task lists.  scatter_large_kernel: slots, and the gathered
-// activation rows of the tensor-core path or the int8 activations of the
-// weight-streaming kernels.
+// Large batch, two kernels (after router_logits_kernel when the router
+// weights are large).
+// router_large_kernel: router_blocks CTAs walk tiles of kRouterTileTokens
+// tokens (tile = block, block + grid, ...); each tile's logits stay in shared
+// memory, one warp per token selects, and every CTA records its per-expert
+// pick counts.  scatter_large_kernel: every CTA derives the bucket offsets
+// and its own slot bases from those counts (CTA 0 also writes the bucket and
+// task lists), then the slots, and the gathered activation rows of the
+// tensor-core path or the int8 activations of the weight-streaming kernels.
 // ---------------------------------------------------------------------------
 // Tensor-core router logits for a tile of kRouterTileTokens tokens and every
 // expert.  x is exactly bf16; each f32 router weight w is split exactly into
@@ -777,55 +778,71 @@ __global__ void __launch_bounds__(256, 2) router_large_kernel(Params p) {
     for (int i = threadIdx.x; i < E; i += blockDim.x) p.hist[(size_t)blockIdx.x * E + i] = s_cnt[i];
 }
 
-__global__ void __launch_bounds__(1024) router_finalize_kernel(Params p) {
-    __shared__ int s_cnt[kMaxE];
-    __shared__ int s_off[kMaxE];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
-    const int E = p.E, nblk = p.router_blocks;
-    pdl_wait();
-    pdl_release();
-    // hist[b][e] -> exclusive prefix over b (per expert), one warp per expert;
-    // all of an expert's counts are loaded before the scan (one round trip)
-    constexpr int kPer = (kRouterMaxBlocks + 31) / 32;
-    for (int e = warp; e < E; e += nwarp) {
-        int v[kPer];
+// Exclusive prefix of s_tot[0..E) into s_off (warp 0; the caller synchronises).
+__device__ void expert_offsets(const int* s_tot, int* s_off, int E) {
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x >= 32) return;
+    constexpr int kPer = kMaxE / 32;
+    int c[kPer], sum = 0;
 #pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            const int b = 32 * j + lane;
-            v[j] = b < nblk ? p.hist[(size_t)b * E + e] : 0;
-        }
-        int run = 0;
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            const int b = 32 * j + lane;
-            int inc = v[j];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int u = __shfl_up_sync(0xffffffffu, inc, o);
-                if (lane >= o) inc += u;
-            }
-            if (b < nblk) p.hist[(size_t)b * E + e] = run + inc - v[j];
-            run += __shfl_sync(0xffffffffu, inc, 31);
-        }
-        if (lane == 0) s_cnt[e] = run;
+    for (int j = 0; j < kPer; ++j) {
+        const int e = lane * kPer + j;
+        c[j] = e < E ? s_tot[e] : 0;
+        sum += c[j];
     }
-    __syncthreads();
-    finalize_buckets(p, s_cnt, s_off);
-    // base of every (router CTA, expert) = bucket start + earlier CTAs' slots
-    for (int i = threadIdx.x; i < nblk * E; i += blockDim.x) p.hist[i] += s_off[i % E];
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += u;
+    }
+    int off = inc - sum;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int e = lane * kPer + j;
+        if (e < E) s_off[e] = off;
+        off += c[j];
+    }
 }
 
 // CTA c walks the same tiles as router CTA c and assigns slots in (tile,
-// token, k) order, after the slots of CTAs 0..c-1.
+// token, k) order, after the slots of CTAs 0..c-1: from the router CTAs'
+// per-expert counts it takes every expert's total (the bucket offsets) and
+// the picks of CTAs 0..c-1.  CTA 0 also builds the bucket and task lists.
 __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
     __shared__ int s_base[kMaxE];
+    __shared__ int s_tot[kMaxE];
+    __shared__ int s_off[kMaxE];
     __shared__ int s_idx[kRouterTileTokens * kMaxK];
     __shared__ int s_slot[kRouterTileTokens * kMaxK];  // -1: not copied
     const int E = p.E, K = p.K;
     const int TK = p.T * K;
+    const int nblk = p.router_blocks;
     pdl_wait();
     pdl_release();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) s_base[e] = p.hist[(size_t)blockIdx.x * E + e];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int before = 0, tot = 0;
+        for (int b0 = 0; b0 < nblk; b0 += 8) {
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = b0 + u < nblk ? __ldcg(p.hist + (size_t)(b0 + u) * E + e) : 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                tot += v[u];
+                if (b0 + u < (int)blockIdx.x) before += v[u];
+            }
+        }
+        s_tot[e] = tot;
+        s_base[e] = before;
+    }
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        finalize_buckets(p, s_tot, s_off);  // the tables (and s_off); synchronises the CTA
+    } else {
+        expert_offsets(s_tot, s_off, E);
+        __syncthreads();
+    }
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_base[e] += s_off[e];
     __syncthreads();
     const int ntiles = (p.T + kRouterTileTokens - 1) / kRouterTileTokens;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -913,7 +930,6 @@ cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream)
         if (err != cudaSuccess) return err;
     }
     err = launch_pdl(router_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
-    if (err == cudaSuccess) err = launch_pdl(router_finalize_kernel, dim3(1), dim3(1024), 0, stream, p);
     if (err == cudaSuccess) err = launch_pdl(scatter_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
     return err;
 }

@@ -96,11 +96,11 @@ def test_kernel_launch_count(moe):
     large = _shape(H=6144, E=256, K=8, I=2048, Is=2048, routed_scaling=2.5)
     assert moe.kernel_launches(nano, 0) == 0
     assert moe.kernel_launches(nano, 16) == 4       # cluster router, gate/up, down, combine
-    assert moe.kernel_launches(nano, 4096) == 6     # router, finalize, scatter, 2 GEMMs, combine
-    assert moe.kernel_launches(nano, 16, moe.MOE_FORCE_PREFILL) == 6
-    assert moe.kernel_launches(nano, 4096, moe.MOE_FORCE_DECODE) == 6
+    assert moe.kernel_launches(nano, 4096) == 5     # router, scatter, 2 GEMMs, combine
+    assert moe.kernel_launches(nano, 16, moe.MOE_FORCE_PREFILL) == 5
+    assert moe.kernel_launches(nano, 4096, moe.MOE_FORCE_DECODE) == 5
     assert moe.kernel_launches(large, 1) == 5       # + the split router's logits kernel
-    assert moe.kernel_launches(large, 512) == 7     # large router with the logits kernel
+    assert moe.kernel_launches(large, 512) == 6     # large router with the logits kernel
     assert moe.kernel_launches(_shape(H=1000), 16) == 0
     assert moe.kernel_launches(nano, (1 << 20) + 1) == 0
 
