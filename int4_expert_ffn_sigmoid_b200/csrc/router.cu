@@ -820,20 +820,27 @@ __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
     const int nblk = p.router_blocks;
     pdl_wait();
     pdl_release();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int before = 0, tot = 0;
-        for (int b0 = 0; b0 < nblk; b0 += 8) {
-            int v[8];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_tot[e] = s_base[e] = 0;
+    __syncthreads();
+    {  // the whole [nblk][E] count matrix, 16 loads in flight per thread
+        const int total = nblk * E;
+        for (int i0 = threadIdx.x; i0 < total; i0 += 16 * blockDim.x) {
+            int v[16];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = b0 + u < nblk ? __ldcg(p.hist + (size_t)(b0 + u) * E + e) : 0;
+            for (int u = 0; u < 16; ++u) {
+                const int i = i0 + u * blockDim.x;
+                v[u] = i < total ? __ldcg(p.hist + i) : 0;
+            }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                tot += v[u];
-                if (b0 + u < (int)blockIdx.x) before += v[u];
+            for (int u = 0; u < 16; ++u) {
+                const int i = i0 + u * blockDim.x;
+                if (i < total && v[u] != 0) {
+                    const int b = i / E, e = i - b * E;
+                    atomicAdd(&s_tot[e], v[u]);
+                    if (b < (int)blockIdx.x) atomicAdd(&s_base[e], v[u]);
+                }
             }
         }
-        s_tot[e] = tot;
-        s_base[e] = before;
     }
     __syncthreads();
     if (blockIdx.x == 0) {
