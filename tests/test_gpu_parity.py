@@ -199,6 +199,20 @@ def test_streaming_kernel_variants(moe, cuda_device, H):
         check(moe, x, layer, shape, layer_cpu=cpu, residual=True, flags=flags)
 
 
+def test_hot_expert_many_chunks(moe, cuda_device):
+    """Large-batch weight streaming with 32-token tasks: one expert picked by
+    every token (a bucket of 150 = 4 x 32 + 22 tokens), next to the shared
+    expert's chunks and the light buckets of the other experts."""
+    wl = workloads.WORKLOADS["nano_layer_t16"]
+    layer = workloads.make_layer(wl.shape, wl.wid, 0, cuda_device, wl.bias_mode)
+    layer["router_bias"][7] = 5.0
+    x = workloads.make_x(wl.shape, 150, wl.wid, batch=9, device=cuda_device)
+    assert moe.layer_path(wl.shape, 150, moe.MOE_FORCE_DECODE) == moe.MOE_PATH_LARGE_STREAMING
+    out, idx, _, _ = check(moe, x, layer, wl.shape, flags=moe.MOE_FORCE_DECODE,
+                           sample=sample_tokens(150, 40, 7))
+    assert idx[:, 0].eq(7).all()
+
+
 def test_large_intermediate_values(moe, cuda_device):
     """Inputs around +-300 drive the SwiGLU intermediate to ~1e5 (beyond fp16's
     65504 unless it is stored scaled); outputs stay finite and match."""
