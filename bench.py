@@ -80,17 +80,40 @@ def measured_peaks():
 # --------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """SM clock and clock-event reasons sampled during the timed region: through
+    NVML every 2 ms on the GPU this process uses (matched by PCI bus id), else
+    through nvidia-smi every 200 ms.  Reading only; no setting is changed."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40}
+    PERIOD_S = 0.002
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, pci_bus_id: str = None):
         self.index = index
+        self.pci_bus_id = pci_bus_id
         self.proc = None
+        self.nvml = None
         self.lines = []
+        self.samples = []  # (sm_mhz, max_mhz, reason bits)
+        self.stop = threading.Event()
 
     def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            if self.pci_bus_id:
+                h = pynvml.nvmlDeviceGetHandleByPciBusId(self.pci_bus_id.encode())
+            else:
+                h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.nvml = (pynvml, h)
+            self.t = threading.Thread(target=self._poll, daemon=True)
+            self.t.start()
+            return self
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
@@ -101,11 +124,31 @@ class ClockSampler:
             self.proc = None
         return self
 
+    def _poll(self):
+        nv, h = self.nvml
+        reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self.stop.is_set():
+            try:
+                self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                     float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)),
+                                     int(reasons(h))))
+            except Exception:
+                return
+            self.stop.wait(self.PERIOD_S)
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
     def __exit__(self, *a):
+        self.stop.set()
+        if self.nvml is not None:
+            self.t.join(timeout=5)
+            try:
+                self.nvml[0].nvmlShutdown()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -115,6 +158,10 @@ class ClockSampler:
 
     def summary(self):
         sm, mx, reasons = [], [], set()
+        for f, m, bits in self.samples:
+            sm.append(f)
+            mx.append(m)
+            reasons.update(n for n, b in self.REASON_BITS.items() if bits & b)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -132,6 +179,15 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def pci_bus_id(device) -> str:
+    """NVML-style PCI bus id of a torch CUDA device, or None."""
+    try:
+        pr = torch.cuda.get_device_properties(device)
+        return f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+    except Exception:
+        return None
 
 
 # --------------------------------------------------------------------------- work accounting
@@ -422,7 +478,7 @@ def run_ours(args, rank, world, device, dist):
 
     stack = Stack(moe, wl, T, device)
     uniq = stack.routing_unique()
-    with ClockSampler(device.index if device.index is not None else 0) as clk:
+    with ClockSampler(device.index if device.index is not None else 0, pci_bus_id(device)) as clk:
         step_ms, _ = timed_steps(stack, args.steps, args.warmup, use_graph, flush, dist_barrier=barrier)
     clocks = clk.summary()
     _, stage_ms = timed_steps(stack, args.steps, 2, use_graph, flush, instrumented=True)

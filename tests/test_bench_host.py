@@ -93,3 +93,13 @@ def test_streaming_kernel_names_follow_the_library_selection():
     assert bench.streaming_kernel_names(small) == ("experts_w13_bulk_kernel", "experts_w2_kernel")
     odd = workloads.LayerShape(H=1152, E=8, K=2, I=768, Is=256, routed_scaling=1.0)
     assert bench.streaming_kernel_names(odd) == ("experts_w13_kernel", "experts_w2_tma_kernel")
+
+
+def test_clock_sampler_summary_from_nvml_samples():
+    s = bench.ClockSampler(0)
+    s.samples = [(1965.0, 1965.0, 0), (1900.0, 1965.0, 0x4), (1950.0, 1965.0, 0)]
+    got = s.summary()
+    assert got == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    s.samples = [(1200.0, 1965.0, 0x8 | 0x40)]
+    assert s.summary()["reasons"] == ["hw_slowdown", "hw_thermal_slowdown"]
+    assert bench.ClockSampler(0).summary()["samples"] == 0
