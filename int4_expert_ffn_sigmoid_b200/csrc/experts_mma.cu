@@ -34,13 +34,14 @@
 //    thread's accumulators hold both parts of the same (row, token) and the
 //    products accumulate exactly in int32.  The chunk's activation rows are
 //    staged in shared memory, padded by 16 bytes so that the per-thread
-//    16-byte fragment reads are conflict-free: the gate/up kernel copies the
-//    router's quantized x (cp.async, whole rows; for H <= 1024 into a second
-//    buffer while the previous task computes; for H > 2048 through a 4-deep
-//    ring of 128-wide slices); the down kernel prefetches the next task's f32
-//    slice of h and its per-64-row maxima of |h| (from the gate/up epilogue)
-//    while the current task computes, then quantizes it with one scale per
-//    (token, slice).
+//    16-byte fragment reads are conflict-free: the gate/up kernels copy the
+//    router's quantized x with cp.async (the TMA-ring kernel into each stage,
+//    256-wide; the bulk kernel whole rows into a second buffer while the
+//    previous task computes; the register-ring kernel whole rows, or for
+//    H > 2048 a 4-deep ring of 128-wide slices); the down kernels prefetch
+//    the next task's f32 slice of h and its per-64-row maxima of |h| (from
+//    the gate/up epilogue) while the current task computes, then quantize it
+//    with one scale per (token, slice).
 //  - Latency: the weight ring runs on across task boundaries (the last
 //    blocks of a task are replaced by the first blocks of the CTA's next
 //    task), and a CTA whose first task belongs to the shared expert fills its
@@ -74,9 +75,8 @@ constexpr int kPadB = 16;     // bytes of padding per staged row
 constexpr int kStageRows = 2 * kChunkTokens;  // two int8 rows (parts) per token
 constexpr int kTab = kMaxE + 2;               // entries of each table
 constexpr int kMaxSlots = kDecodeMaxTokens * kMaxK;
-// Gate/up activation staging: two whole-row buffers up to kDoubleMaxK, one
-// up to kWholeMaxK, a ring of slices beyond.
-constexpr int kDoubleMaxK = 1024;
+// Register-ring gate/up activation staging: one whole-row buffer up to
+// kWholeMaxK, a ring of slices beyond.
 constexpr int kWholeMaxK = 2048;
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
@@ -117,14 +117,12 @@ struct Shm {
 };
 constexpr size_t kShmBytes = (sizeof(Shm) + 127) & ~size_t(127);
 
-// gate/up staging modes: 0 two whole-row buffers, 1 one whole-row buffer, 2 ring of slices
 // scratch of the small-batch table build, in the staging area
 constexpr size_t kBuildBytes = (size_t)(kDecodeGroups + 2) * kMaxE * 4;
 static_assert(kBuildBytes <= (size_t)kStageRows * (kXRing * 128 + kPadB), "table build scratch fits the staging area");
 // Mode 2 stages whole rows too when a task's rows fit in this many bytes.
 constexpr size_t kRingWholeBytes = 100 * 1024;
-constexpr size_t kSmem13[3] = {kShmBytes + (size_t)2 * kStageRows * (kDoubleMaxK + kPadB),
-                               kShmBytes + (size_t)kStageRows * (kWholeMaxK + kPadB),
+constexpr size_t kSmem13[3] = {0 /* no mode 0 */, kShmBytes + (size_t)kStageRows * (kWholeMaxK + kPadB),
                                kShmBytes + kRingWholeBytes};
 static_assert(kRingWholeBytes >= (size_t)kStageRows * (kXRing * 128 + kPadB), "ring staging fits");
 // down: int8 staging of one slice + the next task's f32 slice
@@ -593,10 +591,10 @@ __device__ __forceinline__ bool run13(Ring& ring, const Task13& tk, const WStrea
     return cont;
 }
 
-// kMode: 0 two whole-row staging buffers (the next task's activations load
-// while the current task computes), 1 one whole-row buffer, 2 (large H) one
+// kMode: 1 one whole-row buffer (H <= kWholeMaxK), 2 (larger H) one
 // whole-row buffer for tasks whose rows fit in kRingWholeBytes, else a ring of
-// 128-wide slices.
+// 128-wide slices.  Serves hidden sizes above 1024 that the TMA-ring kernel
+// does not (not a multiple of 256).
 template <int kMode>
 __global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
     extern __shared__ __align__(128) uint8_t dsm[];
@@ -604,8 +602,8 @@ __global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
     uint8_t* xs = dsm + kShmBytes;
     const int g = (threadIdx.x & 31) >> 2;
     const int H = p.H;
+    static_assert(kMode == 1 || kMode == 2, "staging mode");
     const int stride = (kMode == 2 ? kXRing * 128 : H) + kPadB;
-    const int bufbytes = kStageRows * stride;
     Ring ring;
     // The shared expert's tasks come first in every CTA's order and do not
     // depend on the routing: a CTA whose first task is one starts its weight
@@ -633,7 +631,6 @@ __global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
     if (kMode != 2 && cur.ok) stage13(p, sh, cur, xs, stride, sh.xsr[0]);
     const float* S = cur.shared ? p.sh_s13 : p.s13 + (size_t)cur.e * 2 * p.I;
     float gs = cur.ok ? __ldg(S + cur.r0 + g) : 0.f, us = cur.ok ? __ldg(S + cur.irow + cur.r0 + g) : 0.f;
-    int buf = 0;
     for (int r = 0, lin = blockIdx.x; lin < tb.ntask; lin = snake(blockIdx.x, ++r)) {
         const Task13 nx = task13_r(p, sh, r + 1);
         if (!cur.ok) {  // a table entry out of range: flag it and stop
@@ -654,7 +651,6 @@ __global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
         }
         if (kMode != 2) cp_async_wait<0>();
         __syncthreads();  // cur's activations are visible; the previous task is done with every buffer
-        if (kMode == 0 && nx.ok) stage13(p, sh, nx, xs + (buf ^ 1) * bufbytes, stride, sh.xsr[buf ^ 1]);
         float gs_n = 0.f, us_n = 0.f;
         if (nx.ok) {
             const float* Sn = nx.shared ? p.sh_s13 : p.s13 + (size_t)nx.e * 2 * p.I;
@@ -672,8 +668,8 @@ __global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
                                p.xq + (size_t)tok * 2 * H + (r & 1) * H + kb * 128 + part * 16);
             }
         };
-        const uint8_t* xb = xs + (kMode == 0 ? buf * bufbytes : 0);
-        const float* xsr = sh.xsr[kMode == 0 ? buf : 0];
+        const uint8_t* xb = xs;
+        const float* xsr = sh.xsr[0];
         if (kMode == 2 && whole2) {
             switch ((2 * nc + 7) >> 3) {
                 case 1: primed = run13<1, false>(ring, cur, nx.w, gs, us, p, xb, H + kPadB, sh, xsr, stage_slice); break;
@@ -693,7 +689,6 @@ __global__ void __launch_bounds__(256, 2) experts_w13_kernel(Params p) {
         cur = nx;
         gs = gs_n;
         us = us_n;
-        if (kMode == 0) buf ^= 1;
     }
 }
 
@@ -1698,12 +1693,8 @@ int experts_resident_ctas(int which, int H, bool w2_tma, int chunk) {
         return chunk == kMaxChunk ? resident(experts_w13_tma_kernel<kMaxChunk>, Tma13<kMaxChunk>::kSmem, 8, kTmaThreads)
                                   : resident(experts_w13_tma_kernel<kChunkTokens>, Tma13<kChunkTokens>::kSmem, 5, kTmaThreads);
     if (H <= kBulkMaxK) return resident(experts_w13_bulk_kernel, kSmem13Bulk, 4);
-    const int mode = H <= kDoubleMaxK ? 0 : H <= kWholeMaxK ? 1 : 2;
-    switch (mode) {
-        case 0: return resident(experts_w13_kernel<0>, kSmem13[0], 0);
-        case 1: return resident(experts_w13_kernel<1>, kSmem13[1], 1);
-        default: return resident(experts_w13_kernel<2>, kSmem13[2], 2);
-    }
+    return H <= kWholeMaxK ? resident(experts_w13_kernel<1>, kSmem13[1], 1)
+                           : resident(experts_w13_kernel<2>, kSmem13[2], 2);
 }
 
 cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
@@ -1726,12 +1717,8 @@ cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
                           tm_r, tm_s, p);
     }
     if (p.H <= kBulkMaxK) return launch_pdl(experts_w13_bulk_kernel, g, b, kSmem13Bulk, stream, p);
-    const int mode = p.H <= kDoubleMaxK ? 0 : p.H <= kWholeMaxK ? 1 : 2;
-    switch (mode) {
-        case 0: return launch_pdl(experts_w13_kernel<0>, g, b, kSmem13[0], stream, p);
-        case 1: return launch_pdl(experts_w13_kernel<1>, g, b, kSmem13[1], stream, p);
-        default: return launch_pdl(experts_w13_kernel<2>, g, b, kSmem13[2], stream, p);
-    }
+    if (p.H <= kWholeMaxK) return launch_pdl(experts_w13_kernel<1>, g, b, kSmem13[1], stream, p);
+    return launch_pdl(experts_w13_kernel<2>, g, b, kSmem13[2], stream, p);
 }
 
 bool experts_w13_tma(int H) { return w13_tma(H); }
