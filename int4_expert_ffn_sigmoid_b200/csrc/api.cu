@@ -244,21 +244,30 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
     p.decode_groups = small ? cdiv(T, kDecodeRouterTok) : 0;
     p.lslices = router_split_slices(cfg->E, cfg->H, small);  // on either path
     p.lpart = p.lslices > 0 ? static_cast<float*>(at(L.lpart)) : nullptr;
-    // down tasks of large hidden sizes cover several 128-row groups, so that a
-    // task streams enough weight bytes to outweigh its per-task costs
-    {
-        const int groups = cfg->H / kTaskRows2, want = cfg->H / 1024 > 1 ? cfg->H / 1024 : 1;
-        int rg = 1;
-        for (int c : {8, 6, 4, 3, 2})
-            if (c <= want && groups % c == 0) { rg = c; break; }
-        p.rows2 = kTaskRows2 * rg;
-    }
     const int ntiles = cdiv(T, kRouterTileTokens);
     p.router_blocks = ntiles < kRouterMaxBlocks ? ntiles : kRouterMaxBlocks;
     // large batches whose expert kernels both take the TMA-ring kernels stream
     // an expert's weights once for up to kMaxChunk of its tokens
     const bool w2_tma = experts_w2_tma(cfg->H, cfg->I, cfg->Is);
     p.chunk = path == Path::kLargeStreaming && experts_w13_tma(cfg->H) && w2_tma ? kMaxChunk : kChunkTokens;
+    // A down task covers rg 128-row groups (rg up to max(4, H/1024), dividing
+    // H/128): the task's h slice is quantized once for all of them and it
+    // streams enough weight bytes to outweigh its per-task costs.  rg stays
+    // small enough that the down tasks (counted from the upper bound of the
+    // routed buckets) still give every SM one.
+    {
+        const long long TKl = (long long)T * cfg->K;
+        const long long bucket_slices = (cfg->E < TKl ? cfg->E : TKl) * slices_of(cfg->I) +
+                                        (cfg->Is > 0 ? (long long)cdiv(T, p.chunk) * slices_of(cfg->Is) : 0);
+        const int groups = cfg->H / kTaskRows2, want = cfg->H / 1024 > 4 ? cfg->H / 1024 : 4;
+        int rg = 1;
+        for (int c : {8, 6, 4, 3, 2})
+            if (c <= want && groups % c == 0 && (long long)(groups / c) * bucket_slices >= sm_count()) {
+                rg = c;
+                break;
+            }
+        p.rows2 = kTaskRows2 * rg;
+    }
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const long long TK = (long long)T * cfg->K;
