@@ -118,10 +118,14 @@ typedef struct moe_cfg {
 /* Bytes of workspace moe_layer_forward needs for T tokens under `cfg`
  * (workspace, workspace_bytes and the output pointers are ignored; flags are
  * not: the size depends on the kernel sequence that T and the flags select,
- * so a workspace for up to N tokens must hold the largest of the sizes for
- * T = N and T = min(N, moe_decode_max_tokens())).
+ * and a smaller T can need more; see moe_layer_workspace_bytes_upto).
  * Returns 0 if cfg is NULL or the shape is invalid or unsupported. */
 size_t moe_layer_workspace_bytes(const moe_cfg_t* cfg, int32_t T);
+
+/* Bytes of workspace that serve every call of 0..N tokens under `cfg`: the
+ * largest moe_layer_workspace_bytes(cfg, T) over T <= N.  Returns 0 if cfg is
+ * NULL, the shape is invalid or unsupported, or N is out of range. */
+size_t moe_layer_workspace_bytes_upto(const moe_cfg_t* cfg, int32_t N);
 
 /* Forward pass of one MoE layer for T tokens.
  *   x          : bf16 [T][H]

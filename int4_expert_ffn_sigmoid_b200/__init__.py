@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "MoeError", "moe_cfg_t", "moe_shared_weights_t", "lib", "EXPORTED_SYMBOLS",
     "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK", "MOE_FORCE_DECODE", "MOE_FORCE_PREFILL", "MOE_OUT_F32",
-    "workspace_bytes", "layer_forward", "MoELayer", "decode_max_tokens", "kernel_launches", "layer_path",
+    "workspace_bytes", "workspace_bytes_upto", "layer_forward", "MoELayer", "decode_max_tokens", "kernel_launches", "layer_path",
     "MOE_PATH_SMALL_BATCH", "MOE_PATH_TENSOR_CORE", "MOE_PATH_LARGE_STREAMING", "LIB_PATH",
 ]
 
@@ -49,7 +49,7 @@ STAGE_NAMES = ("route", "gate_up", "down", "combine")
 # Every function declared in include/moe_int4.h.
 EXPORTED_SYMBOLS = ("moe_layer_workspace_bytes", "moe_layer_forward", "moe_status_str",
                     "moe_abi_version", "moe_decode_max_tokens", "moe_layer_forward_static_ws",
-                    "moe_layer_kernel_launches", "moe_layer_path")
+                    "moe_layer_kernel_launches", "moe_layer_path", "moe_layer_workspace_bytes_upto")
 
 # Scratch capacity of moe_layer_forward_static_ws (the entry point for callers
 # that cannot allocate device memory).
@@ -83,6 +83,8 @@ def _load() -> ctypes.CDLL:
     vp = ctypes.c_void_p
     L.moe_layer_workspace_bytes.argtypes = [ctypes.POINTER(moe_cfg_t), ctypes.c_int32]
     L.moe_layer_workspace_bytes.restype = ctypes.c_size_t
+    L.moe_layer_workspace_bytes_upto.argtypes = [ctypes.POINTER(moe_cfg_t), ctypes.c_int32]
+    L.moe_layer_workspace_bytes_upto.restype = ctypes.c_size_t
     L.moe_layer_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(moe_shared_weights_t),
                                     vp, ctypes.c_int32, ctypes.POINTER(moe_cfg_t), vp]
     L.moe_layer_forward.restype = ctypes.c_int
@@ -157,11 +159,14 @@ def workspace_bytes(shape, T: int, flags: int = 0) -> int:
     return int(lib.moe_layer_workspace_bytes(ctypes.byref(c), int(T)))
 
 
+def workspace_bytes_upto(shape, T: int, flags: int = 0) -> int:
+    c = make_cfg(shape, flags)
+    return int(lib.moe_layer_workspace_bytes_upto(ctypes.byref(c), int(T)))
+
+
 def new_workspace(shape, T: int, device, flags: int = 0) -> torch.Tensor:
-    """A workspace for any call of up to T tokens under `flags` (the sizes of
-    the two kernel sequences differ, so both sides of the small-batch limit
-    are asked)."""
-    n = max(workspace_bytes(shape, T, flags), workspace_bytes(shape, min(T, decode_max_tokens()), flags))
+    """A workspace for any call of up to T tokens under `flags`."""
+    n = workspace_bytes_upto(shape, T, flags)
     if n == 0:
         raise MoeError(MOE_ERR_UNSUPPORTED, "moe_layer_workspace_bytes")
     return torch.empty(n, dtype=torch.uint8, device=device)

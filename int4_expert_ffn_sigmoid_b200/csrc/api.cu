@@ -164,6 +164,23 @@ size_t moe_layer_workspace_bytes(const moe_cfg_t* cfg, int32_t T) {
     return ws_layout(*cfg, T).total;
 }
 
+size_t moe_layer_workspace_bytes_upto(const moe_cfg_t* cfg, int32_t N) {
+    if (validate_cfg(cfg) != MOE_OK || N < 0 || N > kMaxTokens) return 0;
+    // The size grows with T within each kernel sequence, so the largest T of
+    // each sequence up to N bounds it: N itself, the last small-batch T, and
+    // the last T below the tensor-core threshold (T*K < kTcMinSlotsPerExpert*E).
+    const long long t_stream = ((long long)kTcMinSlotsPerExpert * cfg->E - 1) / cfg->K;
+    const long long cands[3] = {N, kDecodeMaxTokens, t_stream};
+    size_t best = 0;
+    for (long long t : cands) {
+        const int32_t tt = (int32_t)(t < N ? t : N);
+        if (tt < 0) continue;
+        const size_t b = ws_layout(*cfg, tt).total;
+        if (b > best) best = b;
+    }
+    return best;
+}
+
 int moe_layer_forward(const void* x, const float* router_w, const float* router_bias,
                       const uint8_t* packed_w13, const float* scales13, const uint8_t* packed_w2,
                       const float* scales2, const moe_shared_weights_t* shared_w, void* out, int32_t T,

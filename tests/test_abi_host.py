@@ -105,6 +105,22 @@ def test_kernel_launch_count(moe):
     assert moe.kernel_launches(nano, (1 << 20) + 1) == 0
 
 
+def test_workspace_upto_covers_every_smaller_call(moe):
+    """A smaller T can need more workspace (the weight-streaming sequence keeps
+    f32 h and per-slice partial rows); the _upto query is the maximum over
+    every T up to N, checked here against all T."""
+    for shape in (_shape(), _shape(H=6144, E=256, K=8, I=2048, Is=2048, routed_scaling=2.5),
+                  _shape(H=1152, E=16, K=3, I=768, Is=256)):
+        for flags in (0, moe.MOE_FORCE_DECODE, moe.MOE_FORCE_PREFILL):
+            for N in (1, 64, 65, 700, 1100, 3000):
+                sizes = [moe.workspace_bytes(shape, t, flags) for t in range(N + 1)]
+                assert moe.workspace_bytes_upto(shape, N, flags) == max(sizes), (shape, flags, N)
+    nano = _shape()
+    # the example that needs it: a workspace for 1100 tokens sized at T = 1100 alone is too small
+    assert moe.workspace_bytes(nano, 1100) < moe.workspace_bytes(nano, 1000)
+    assert moe.workspace_bytes_upto(_shape(H=1000), 16) == 0
+
+
 def test_path_choice(moe):
     nano = _shape()
     large = _shape(H=6144, E=256, K=8, I=2048, Is=2048, routed_scaling=2.5)
