@@ -59,7 +59,7 @@ extern "C" {
 /* Flags of moe_cfg_t.flags. */
 #define MOE_ADD_RESIDUAL (1u << 0)  /* out = x + MoE(x) (one layer of a residual stack) */
 #define MOE_DEBUG_CHECK (1u << 1)   /* synchronise the stream and report device range checks */
-#define MOE_FORCE_DECODE (1u << 2)  /* use the small-batch (weight-streaming) kernels at any T */
+#define MOE_FORCE_DECODE (1u << 2)  /* use the weight-streaming expert kernels at any T */
 #define MOE_FORCE_PREFILL (1u << 3) /* use the grouped-GEMM kernels at any T (H a multiple of 256) */
 #define MOE_OUT_F32 (1u << 4)       /* out is f32 [T][H] (the f32 sum, no bf16 rounding): for
                                        checking the arithmetic apart from the output rounding */
