@@ -63,6 +63,23 @@ extern "C" {
 #define MOE_FORCE_PREFILL (1u << 3) /* use the grouped-GEMM kernels at any T (H a multiple of 256) */
 #define MOE_OUT_F32 (1u << 4)       /* out is f32 [T][H] (the f32 sum, no bf16 rounding): for
                                        checking the arithmetic apart from the output rounding */
+#define MOE_TEST_STALL (1u << 6)    /* test only: in the expert kernels that take part (the
+                                       tensor-core grouped GEMMs and the TMA-ring weight-streaming
+                                       kernels), one role first waits ~1 ms on a flag that nothing
+                                       sets, so that the kernel takes its timeout path while its
+                                       copies and MMAs are in flight: it stops, drains what it
+                                       issued and records MOE_DEVSTAT_TIMEOUT.  The output is then
+                                       undefined; with MOE_DEBUG_CHECK the call returns
+                                       MOE_ERR_DEVICE_CHECK.  The next call runs normally. */
+
+/* Device status word: the first 4 bytes of the workspace hold the OR of these
+ * bits after a call completes on the device (0 = no check failed).  Under
+ * MOE_DEBUG_CHECK a non-zero word makes the call return MOE_ERR_DEVICE_CHECK. */
+#define MOE_DEVSTAT_BAD_EXPERT (1u << 0) /* a routing index outside [0, E) */
+#define MOE_DEVSTAT_BAD_SLOT (1u << 1)   /* a bucket slot outside [0, T*K) */
+#define MOE_DEVSTAT_BAD_COUNT (1u << 2)  /* bucket counts do not sum to T*K */
+#define MOE_DEVSTAT_BAD_TASK (1u << 3)   /* a work item resolved outside the bucket list */
+#define MOE_DEVSTAT_TIMEOUT (1u << 4)    /* a bounded wait (about 2 s; MOE_TEST_STALL: ~1 ms) gave up */
 
 /* The always-resident shared expert (intermediate size Is).
  *   w13: uint8 [2*Is][H/2]  rows 0..Is-1 gate, rows Is..2*Is-1 up
@@ -185,7 +202,10 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
  *  - It allocates nothing and calls no allocating routine.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current.  Make that first call
- *    before any stream capture begins.
+ *    before any stream capture begins.  The address belongs to the device's
+ *    current driver context: after cudaDeviceReset, or under another
+ *    context, the next call looks it up again (so make that call, too,
+ *    outside a capture).
  *  - Every call on a device shares the one array, and the array keeps the
  *    last call's contents.  Calls that may run at the same time on the GPU
  *    (on different streams, with nothing ordering them) race on it and must

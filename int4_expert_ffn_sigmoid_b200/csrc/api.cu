@@ -13,7 +13,13 @@ namespace {
 using namespace moe;
 
 constexpr unsigned kKnownFlags =
-    MOE_ADD_RESIDUAL | MOE_DEBUG_CHECK | MOE_FORCE_DECODE | MOE_FORCE_PREFILL | MOE_OUT_F32;
+    MOE_ADD_RESIDUAL | MOE_DEBUG_CHECK | MOE_FORCE_DECODE | MOE_FORCE_PREFILL | MOE_OUT_F32 | MOE_TEST_STALL;
+static_assert(kFlagResidual == MOE_ADD_RESIDUAL && kFlagOutF32 == MOE_OUT_F32 && kFlagTestStall == MOE_TEST_STALL,
+              "kernel flag bits match the C ABI");
+static_assert(ST_BAD_EXPERT == MOE_DEVSTAT_BAD_EXPERT && ST_BAD_SLOT == MOE_DEVSTAT_BAD_SLOT &&
+                  ST_BAD_COUNT == MOE_DEVSTAT_BAD_COUNT && ST_BAD_TASK == MOE_DEVSTAT_BAD_TASK &&
+                  ST_TIMEOUT == MOE_DEVSTAT_TIMEOUT && offsetof(Ctrl, status) == 0,
+              "device status bits match the C ABI");
 constexpr int32_t kMaxTokens = 1 << 20;
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }

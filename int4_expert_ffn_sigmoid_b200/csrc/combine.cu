@@ -44,11 +44,11 @@ __global__ void __launch_bounds__(256) combine_kernel(Params p) {
         }
         a0 += v.x; a1 += v.y; a2 += v.z; a3 += v.w;
     }
-    if (p.flags & 1u) {  // MOE_ADD_RESIDUAL
+    if (p.flags & kFlagResidual) {
         const uint2 xv = __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)t * H + j));
         a0 += bf16lo(xv.x); a1 += bf16hi(xv.x); a2 += bf16lo(xv.y); a3 += bf16hi(xv.y);
     }
-    if (p.flags & (1u << 4)) {  // MOE_OUT_F32
+    if (p.flags & kFlagOutF32) {
         *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)t * H + j) = make_float4(a0, a1, a2, a3);
         return;
     }

@@ -62,6 +62,7 @@
 #include "moe_common.cuh"
 #include "moe_launch.h"
 #include "moe_tc.h"
+#include "stream_ops.cuh"
 
 namespace moe {
 
@@ -71,27 +72,12 @@ constexpr int kRows13 = kTaskRows13;  // gate (and up) rows per gate/up task
 constexpr int kRows2 = kTaskRows2;    // down rows per down task
 constexpr int kRing = 4;      // weight k blocks in flight per thread
 constexpr int kXRing = 4;     // staged activation slices (ring mode)
-constexpr int kPadB = 16;     // bytes of padding per staged row
 constexpr int kStageRows = 2 * kChunkTokens;  // two int8 rows (parts) per token
 constexpr int kTab = kMaxE + 2;               // entries of each table
 constexpr int kMaxSlots = kDecodeMaxTokens * kMaxK;
 // Register-ring gate/up activation staging: one whole-row buffer up to
 // kWholeMaxK, a ring of slices beyond.
 constexpr int kWholeMaxK = 2048;
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
-                 "l"(gmem)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
-                 "l"(gmem)
-                 : "memory");
-}
 
 struct Tables {
     int n_buckets, ntask;
@@ -314,30 +300,6 @@ __device__ __forceinline__ int slot_token(const Params& p, const Shm& sh, bool s
 // One k block: this thread's 16 bytes of weight rows a (mma row g) and b (mma
 // row g + 8) against NT n-tiles of staged activations; xrow points at staged
 // row g, byte q*32 of the k block, and n-tile i is 8*i rows further.
-template <int NT, int kSets>
-__device__ __forceinline__ void kblock8(const uint4& wa, const uint4& wb, const uint8_t* xrow, int tile_stride,
-                                        int (&part)[kSets][NT][4]) {
-    const uint32_t aw[4] = {wa.x, wa.y, wa.z, wa.w};
-    const uint32_t bw[4] = {wb.x, wb.y, wb.z, wb.w};
-    uint32_t A[4][4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        A[m][0] = lo8(aw[m]);
-        A[m][1] = lo8(bw[m]);
-        A[m][2] = hi8(aw[m]);
-        A[m][3] = hi8(bw[m]);
-    }
-#pragma unroll
-    for (int i = 0; i < NT; ++i) {
-        const uint4 b01 = *reinterpret_cast<const uint4*>(xrow + i * tile_stride);
-        const uint4 b23 = *reinterpret_cast<const uint4*>(xrow + i * tile_stride + 16);
-        mma_s8(part[0][i], A[0], b01.x, b01.y);
-        mma_s8(part[kSets - 1][i], A[1], b01.z, b01.w);
-        mma_s8(part[0][i], A[2], b23.x, b23.y);
-        mma_s8(part[kSets - 1][i], A[3], b23.z, b23.w);
-    }
-}
-
 // This thread's weight stream of one task: 16 bytes of rows a (mma row g)
 // and b (mma row g + 8) per k block, nkb blocks 64 bytes apart (nkb = 0: no
 // task).
@@ -419,10 +381,6 @@ __device__ __forceinline__ bool stream8(Ring& ring, const WStream& cur, const WS
         for (int c = 0; c < 4; ++c) acc[i][c] = part[0][i][c] + part[kSets - 1][i][c] * (kSets - 1);
     return cont;
 }
-
-// Both int8 parts of mma columns 2j, 2j+1 -> the value in units of the
-// activation scale times 16.
-__device__ __forceinline__ float join(int c0, int c1) { return (float)c0 + (float)c1 * (1.0f / 256.0f); }
 
 // One gate/up task as this thread sees it.
 struct Task13 {
@@ -709,44 +667,6 @@ constexpr size_t kBulkWarpSlot = 16 * (kBulkMaxK / 2);  // 8 gate + 8 up rows
 constexpr size_t kBulkBarBytes = 128;
 constexpr size_t kSmem13Bulk = kShmBytes + kBulkBarBytes + 8 * kBulkSlots * kBulkWarpSlot +
                                (size_t)2 * kStageRows * (kBulkMaxK + kPadB);
-constexpr long long kBulkWaitCycles = 4000000000LL;  // ~2 s
-
-__device__ __forceinline__ void bar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar))),
-                 "r"(count)
-                 : "memory");
-}
-__device__ __forceinline__ void bar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
-                     static_cast<uint32_t>(__cvta_generic_to_shared(bar))),
-                 "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool bar_try(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar))), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait for phase `parity` of bar.
-__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, long long limit) {
-    if (bar_try(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!bar_try(bar, parity))
-        if (clock64() - t0 > limit) return false;
-    return true;
-}
-// bytes (a multiple of 16, both addresses 16-byte aligned) global -> shared,
-// completion counted on bar.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-                 "l"(src), "r"(bytes), "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar)))
-                 : "memory");
-}
 
 // Lane 0 of the calling warp issues the warp's 8 gate + 8 up rows of task t
 // into `slot`.
@@ -928,10 +848,6 @@ __global__ void __launch_bounds__(256, 1) experts_w13_bulk_kernel(Params p) {
 // stages hold, and the producer waits (bounded) for its last copies before
 // it exits.
 // ---------------------------------------------------------------------------
-constexpr int kTmaChunk = 256;                                 // k elements per stage
-constexpr int kTmaRowBytes = kTmaChunk / 2;                    // 128 bytes of codes per row and stage
-constexpr int kTmaWBytes = 2 * kRows13 * kTmaRowBytes;         // gate + up tiles: 16 KB
-constexpr int kTmaXStride = kTmaChunk + kPadB;                 // staged activation row
 constexpr int kTmaThreads = 288;                               // 8 consumer warps + the producer warp
 // Ring geometry for tasks of kChunk tokens: the activation part of a stage
 // holds 2 kChunk rows, and the ring is as deep as shared memory allows
@@ -946,23 +862,6 @@ struct Tma13 {
     static_assert((size_t)kStages * kXBytes >= kBuildBytes, "table build scratch fits the activation ring");
 };
 
-__device__ __forceinline__ void bar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar)))
-                 : "memory");
-}
-// Arrives on bar once every cp.async this thread issued so far has landed.
-__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
-                     static_cast<uint32_t>(__cvta_generic_to_shared(bar)))
-                 : "memory");
-}
-__device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
-            static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar))), "r"(x), "r"(y)
-        : "memory");
-}
 // The weights of k chunk c of a task whose gate rows start at row rg and up
 // rows at ru of `map`: expect the bytes, then the two tile loads.
 __device__ __forceinline__ void issue_w13_chunk(const CUtensorMap* map, uint64_t* bar, uint8_t* dst, int c, int rg,
@@ -988,7 +887,7 @@ __device__ __forceinline__ void consume13(int nch, uint32_t& n, uint64_t* full, 
     const int wrow = (warp * 8 + g) * kTmaRowBytes;
     for (int c = 0; c < nch; ++c, ++n) {
         const int s = n % kStages;
-        if (!*abort && !bar_wait(full + s, (n / kStages) & 1, kBulkWaitCycles)) {
+        if (!*abort && !bar_wait_or_abort(full + s, (n / kStages) & 1, kBulkWaitCycles, abort)) {
             *abort = 1;
             if (lane == 0) atomicOr(status, ST_TIMEOUT);
         }
@@ -1020,6 +919,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     uint64_t* full = reinterpret_cast<uint64_t*>(dsm + kShmBytes);
     uint64_t* empty = full + kStages;
     volatile int* abort = reinterpret_cast<volatile int*>(empty + kStages);
+    volatile int* never = abort + 1;  // nothing sets it (MOE_TEST_STALL)
     float(*hm2)[8][kChunk] = reinterpret_cast<float(*)[8][kChunk]>(dsm + kShmBytes + 256);
     const uint32_t base_s = static_cast<uint32_t>(__cvta_generic_to_shared(dsm));
     const uint32_t ring_s = (base_s + (uint32_t)(kShmBytes + Cfg::kMisc) + 1023u) & ~1023u;
@@ -1035,6 +935,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
             bar_init(empty + i, 8);      // one arrival per consumer warp
         }
         *abort = 0;
+        *never = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -1095,7 +996,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
                 const int round = (int)(n / kStages);
                 const bool issued = r == 0 && c < npre;  // weights issued before the wait
                 if (round > 0) {
-                    bool ok = *abort == 0 && bar_wait(empty + s, (round - 1) & 1, kBulkWaitCycles);
+                    bool ok = *abort == 0 && bar_wait_or_abort(empty + s, (round - 1) & 1, kBulkWaitCycles, abort);
                     if (__any_sync(0xffffffffu, !ok)) {
                         if (lane == 0 && !*abort) atomicOr(status, ST_TIMEOUT);
                         *abort = 1;
@@ -1128,6 +1029,11 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         return;
     }
     // consumers
+    if ((p.flags & kFlagTestStall) && threadIdx.x == 0) {  // a wait that runs out: take the timeout path
+        stall_on_unset_flag(never, kStallCycles);
+        *abort = 1;
+        atomicOr(status, ST_TIMEOUT);
+    }
     uint32_t n = 0;
     for (int r = 0; snake(blockIdx.x, r) < ntask; ++r) {
         const Task13 t = task13_r(p, sh, r);
@@ -1403,7 +1309,6 @@ __global__ void __launch_bounds__(256, 2) experts_w2_kernel(Params p) {
 // cp.async and quantize the current task's slice in shared memory while the
 // producer keeps the ring full.
 // ---------------------------------------------------------------------------
-constexpr int kW2Bytes = kRows2 * kTmaRowBytes;  // one stage: 16 KB
 constexpr size_t kW2MiscBytes = 256;
 // Ring and staging for tasks of kChunk tokens (offsets from the ring's start).
 template <int kChunk>
@@ -1459,7 +1364,7 @@ __device__ __forceinline__ void consume2(const Task2& tk, uint32_t& n, uint64_t*
             for (int i = 0; i < NT; ++i) part[s][i][0] = part[s][i][1] = part[s][i][2] = part[s][i][3] = 0;
         for (int c = 0; c < nkc; ++c, ++n) {
             const int s = n % kStages;
-            if (!*abort && !bar_wait(full + s, (n / kStages) & 1, kBulkWaitCycles)) {
+            if (!*abort && !bar_wait_or_abort(full + s, (n / kStages) & 1, kBulkWaitCycles, abort)) {
                 *abort = 1;
                 if (lane == 0) atomicOr(status, ST_TIMEOUT);
             }
@@ -1505,6 +1410,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     uint64_t* full = reinterpret_cast<uint64_t*>(dsm + kShmBytes);
     uint64_t* empty = full + kStages;
     volatile int* abort = reinterpret_cast<volatile int*>(empty + kStages);
+    volatile int* never = abort + 1;  // nothing sets it (MOE_TEST_STALL)
     const uint32_t base_s = static_cast<uint32_t>(__cvta_generic_to_shared(dsm));
     const uint32_t ring_s = (base_s + (uint32_t)(kShmBytes + kW2MiscBytes) + 1023u) & ~1023u;
     uint8_t* wring = dsm + (ring_s - base_s);
@@ -1520,6 +1426,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
             bar_init(empty + i, 8);  // one arrival per consumer warp
         }
         *abort = 0;
+        *never = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -1579,7 +1486,8 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
                     const int s = n % kStages;
                     const int round = (int)(n / kStages);
                     if (round > 0) {
-                        const bool ok = *abort == 0 && bar_wait(empty + s, (round - 1) & 1, kBulkWaitCycles);
+                        const bool ok =
+                            *abort == 0 && bar_wait_or_abort(empty + s, (round - 1) & 1, kBulkWaitCycles, abort);
                         if (__any_sync(0xffffffffu, !ok)) {
                             if (lane == 0 && !*abort) atomicOr(status, ST_TIMEOUT);
                             *abort = 1;
@@ -1602,6 +1510,11 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         return;
     }
     // consumers
+    if ((p.flags & kFlagTestStall) && threadIdx.x == 0) {  // a wait that runs out: take the timeout path
+        stall_on_unset_flag(never, kStallCycles);
+        *abort = 1;
+        atomicOr(status, ST_TIMEOUT);
+    }
     uint32_t n = 0;
     Task2 cur = task2_r(p, sh, 0);
     if (cur.ok) fetch2c(p, sh, cur, raw, rs2);

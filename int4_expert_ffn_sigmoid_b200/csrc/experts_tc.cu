@@ -25,7 +25,10 @@
 //   warps 10-13 epilogue: tcgen05.ld of the accumulator, scales (staged in
 //               shared memory per tile), SwiGLU, stores
 // Every mbarrier wait is bounded (clock64); on timeout the CTA records
-// ST_TIMEOUT in the status word, drains what it issued and exits.
+// ST_TIMEOUT in the status word and stops.  The drains then ignore the abort
+// (each with its own bound): the producer waits until every TMA copy it issued
+// has landed and the MMA thread until every MMA it issued has completed, and
+// only then is tensor memory released and the CTA gone.
 #include <cuda.h>
 
 #include "moe_common.cuh"
@@ -51,6 +54,10 @@ constexpr int NUM_THREADS = 64 + 32 * DEQ_WARPS + 128;
 constexpr int TMEM_COLS = 512;          // two 256-column accumulators
 constexpr long long kTimeoutCycles = 4000000000LL;
 constexpr long long kDrainCycles = 200000000LL;
+// MOE_TEST_STALL: the epilogue first waits this long on a barrier nothing
+// arrives on (~1 ms), which makes the CTA take its timeout path while its
+// copies and MMAs are in flight.
+constexpr long long kStallCycles = 1LL << 21;
 constexpr int SMEM_BYTES = RING_BYTES + 1024 + 1280;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of the grouped GEMM");
 
@@ -62,6 +69,7 @@ struct Shared {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
+    uint64_t never;  // nothing arrives on it (MOE_TEST_STALL)
     uint32_t tmem_base;
     int abort_flag;
     float ep_scale[BN];  // the current tile's row scales (epilogue)
@@ -112,6 +120,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Shared
             return false;
         }
     }
+}
+
+// Bounded wait that ignores the abort flag: the drains after an abort, which
+// must see the CTA's own copies and MMAs complete before its shared memory
+// and tensor memory go away.  Returns false only when `limit` runs out.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, long long limit) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > limit) return false;
+    return true;
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
@@ -271,6 +290,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
             mbar_init(&sh->acc_empty[b], 4);
         }
         mbar_init(&sh->drain, 1);
+        mbar_init(&sh->never, 1);
         sh->abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -329,7 +349,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
             }
             // make sure no copy is still landing when the CTA leaves
             for (int i = 0; i < TSTAGES; ++i)
-                if (issued[i]) mbar_wait(&sh->full_tma[i], issued_par[i], sh, kDrainCycles);
+                if (issued[i]) mbar_wait_drain(&sh->full_tma[i], issued_par[i], kDrainCycles);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -368,9 +388,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
                 acc_ph[buf] ^= 1u;
                 buf ^= 1;
             }
-            if (!ok && any) {  // wait for the tensor cores before TMEM is released
+            // Before TMEM is released, every MMA this thread issued must be done:
+            // after an abort the epilogue may not wait for the accumulators.
+            if (any) {
                 mma_commit(&sh->drain);
-                mbar_wait(&sh->drain, 0, sh, kDrainCycles);
+                mbar_wait_drain(&sh->drain, 0, kDrainCycles);
             }
         }
     } else if (warp < 2 + DEQ_WARPS) {
@@ -440,7 +462,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
             const int tok = valid ? (t.shared ? t.slot0 + m : __ldg(a.tok_of_slot + t.slot0 + m)) : 0;
             const int hx = __ldg(a.hexp + tok);
             int got = 0;
-            if (lane == 0) got = mbar_wait(&sh->acc_full[buf], acc_ph[buf], sh);
+            if (lane == 0)
+                got = (!a.stall || mbar_wait(&sh->never, 0, sh, kStallCycles)) &&
+                      mbar_wait(&sh->acc_full[buf], acc_ph[buf], sh);
             if (lane == 0) sh->ep_ok[quarter] = got;
             epi_bar();  // scales visible; every warp's wait outcome known
             if (!(sh->ep_ok[0] && sh->ep_ok[1] && sh->ep_ok[2] && sh->ep_ok[3])) break;
@@ -578,6 +602,7 @@ cudaError_t launch_tc_gemm(const Params& p, int gemm, int grid, cudaStream_t str
     a.bucket_e = p.bucket_e; a.bucket_n = p.bucket_n; a.bucket_off = p.bucket_off;
     a.status = &p.ctrl->status;
     a.h_r = p.h_r; a.h_s = p.h_s; a.y = p.y;
+    a.stall = (p.flags & kFlagTestStall) != 0;
     a.tok_of_slot = p.tok_of_slot; a.hexp = p.hexp;
     bool ok;
     if (gemm == 1) {

@@ -47,13 +47,19 @@ constexpr int kHExpBase = 8;
 constexpr int kHExpMin = -40;
 constexpr int kHExpMax = 60;
 
+// Flag bits of Params::flags that the kernels read (the values of the
+// MOE_* flags of the C ABI).
+constexpr unsigned kFlagResidual = 1u << 0;   // MOE_ADD_RESIDUAL
+constexpr unsigned kFlagOutF32 = 1u << 4;     // MOE_OUT_F32
+constexpr unsigned kFlagTestStall = 1u << 6;  // MOE_TEST_STALL
+
 // Device status bits (set by range checks, read back under MOE_DEBUG_CHECK).
 enum : unsigned {
     ST_BAD_EXPERT = 1u,  // a routing index outside [0, E)
     ST_BAD_SLOT = 2u,    // a slot outside [0, T*K)
     ST_BAD_COUNT = 4u,   // bucket counts do not sum to T*K
     ST_BAD_TASK = 8u,    // a task resolved to a bucket outside the list
-    ST_TIMEOUT = 16u,    // a bounded pipeline wait of the tensor-core kernel gave up
+    ST_TIMEOUT = 16u,    // a bounded pipeline wait gave up
 };
 
 // First 256 bytes of the workspace.  The first kernel of every call zeroes

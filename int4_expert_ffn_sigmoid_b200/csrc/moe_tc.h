@@ -27,6 +27,7 @@ struct TcArgs {
     const int32_t* tok_of_slot;
     const int32_t* hexp;  // per-token exponent of the h storage scale
     unsigned* status;
+    int stall;            // MOE_TEST_STALL: the epilogue's first wait runs out
 };
 
 // Signature of cuTensorMapEncodeTiled (fetched from the driver at run time).
