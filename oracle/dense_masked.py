@@ -34,26 +34,34 @@ def _sigmoid(z):
     return 1.0 / (1.0 + np.exp(-z))
 
 
-def routing_matrix(x: np.ndarray, W: np.ndarray, bias: np.ndarray, K: int, scale: float):
-    """Dense routing weights R [T,E]: R[t,e] = w[t,k] if e = e_k, else 0."""
+def routing_matrix(x: np.ndarray, W: np.ndarray, bias: np.ndarray, K: int, scale: float, forced=None):
+    """Dense routing weights R [T,E]: R[t,e] = w[t,k] if e = e_k, else 0.
+
+    ``forced`` [T,K] (optional) replaces the selection by the given experts;
+    their weights still come from the unbiased scores, normalised over the
+    forced set."""
     s = _sigmoid(x @ W.T.astype(np.float64))
     key = s + bias.astype(np.float64)[None, :]
     key = np.where(np.isnan(key), -np.inf, key)
     T, E = s.shape
     R = np.zeros((T, E))
     for t in range(T):
-        order = np.argsort(-key[t], kind="stable")  # equal keys keep index order
-        sel = order[:K]
+        if forced is None:
+            order = np.argsort(-key[t], kind="stable")  # equal keys keep index order
+            sel = order[:K]
+        else:
+            sel = np.asarray(forced[t], np.int64)
         R[t, sel] = scale * s[t, sel] / s[t, sel].sum()
     return R
 
 
-def moe_dense(x, layer: dict, shape, residual: bool = False):
-    """Layer output [T,H] in float64.  x: bf16 [T,H] (torch) or bf16 bits."""
+def moe_dense(x, layer: dict, shape, residual: bool = False, forced=None):
+    """Layer output [T,H] in float64.  x: bf16 [T,H] (torch) or bf16 bits.
+    ``forced`` [T,K]: evaluate these experts instead of the router's choice."""
     xf = bf16_bits_to_f64(x)
     E, K, I, Is = shape.E, shape.K, shape.I, shape.Is
     R = routing_matrix(xf, _np(layer["router_w"], np.float64), _np(layer["router_bias"], np.float64),
-                       K, shape.routed_scaling)
+                       K, shape.routed_scaling, forced)
     W13 = decode_int4(_np(layer["w13"], np.uint8)) * _np(layer["s13"], np.float64)[..., None]
     W2 = decode_int4(_np(layer["w2"], np.uint8)) * _np(layer["s2"], np.float64)[..., None]
     G = np.einsum("th,eih->tei", xf, W13[:, :I])

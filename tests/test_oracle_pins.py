@@ -283,6 +283,34 @@ def test_override_with_own_choice_is_identity():
     np.testing.assert_array_equal(r2["out"], r["out"])
 
 
+def test_override_evaluates_the_forced_experts():
+    """idx_override replaces the selection: the oracle then evaluates exactly
+    the forced experts, weighted by their unbiased sigmoid scores normalised
+    over the forced set (the bias only ever decides a selection), which the
+    dense-masked formulation computes independently.  The forced experts are
+    each token's K lowest keys, so an override that were ignored, or that only
+    reordered the router's own choice, would fail."""
+    shape = workloads.LayerShape(H=32, E=8, K=3, I=16, Is=8, routed_scaling=2.5)
+    layer = workloads.make_layer(shape, 93, device="cpu")
+    x = workloads.make_x(shape, 6, 93)
+    own = oracle.moe_tokens(x, layer, shape)
+    rt = oracle.route(x, layer["router_w"], layer["router_bias"], shape.K, shape.routed_scaling)
+    keys = rt["scores"] + layer["router_bias"].double().numpy()[None, :]
+    forced = np.argsort(keys, axis=1, kind="stable")[:, :shape.K][:, ::-1].astype(np.int32).copy()
+    assert not np.any(np.isin(forced, own["idx"]).all(axis=1))
+    r = oracle.moe_tokens(x, layer, shape, residual=True, idx_override=forced)
+    np.testing.assert_array_equal(r["idx"], forced)
+    s = rt["scores"][np.arange(6)[:, None], forced]
+    np.testing.assert_allclose(r["weights"], 2.5 * s / s.sum(axis=1, keepdims=True), rtol=1e-14)
+    ref, R = dense_masked.moe_dense(x, layer, shape, residual=True, forced=forced)
+    np.testing.assert_allclose(r["out"], ref, rtol=0, atol=1e-12 * np.abs(ref).max())
+    assert np.abs(r["out"] - oracle.moe_tokens(x, layer, shape, residual=True)["out"]).max() > 1e-3
+    # a subset of tokens with their own overrides
+    tok = np.array([4, 1], np.int32)
+    r2 = oracle.moe_tokens(x, layer, shape, residual=True, tokens=tok, idx_override=forced[tok])
+    np.testing.assert_array_equal(r2["out"], r["out"][tok])
+
+
 def test_sigmoid_saturation_finite():
     shape = workloads.LayerShape(H=8, E=4, K=2, I=2, Is=0, routed_scaling=1.0)
     W = np.full((4, 8), 500.0, np.float32)
