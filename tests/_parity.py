@@ -65,6 +65,12 @@ def check_routing(idx_gpu: np.ndarray, w_gpu: np.ndarray, ref: dict, bias: np.nd
         assert len(set(sel.tolist())) == K, (t, sel)
         kth = np.sort(keys[t])[::-1][K - 1]
         assert np.all(keys[t, sel] >= kth - TIE_MARGIN), (t, sel, keys[t, sel], kth)
+    # the documented order of topk_idx_out: decreasing s + bias (two selected
+    # experts whose keys agree to within rounding may come in either order)
+    sel_keys = np.take_along_axis(keys, idx_gpu.astype(np.int64), axis=1)
+    drop = sel_keys[:, :-1] - sel_keys[:, 1:]
+    bad = np.nonzero(np.any(drop < -TIE_MARGIN, axis=1))[0]
+    assert bad.size == 0, f"selection not in decreasing key order at tokens {bad[:5]}: {sel_keys[bad[:3]]}"
     werr = 0.0
     if non.any():
         og = np.argsort(idx_gpu, axis=1)
@@ -89,6 +95,30 @@ def bf16_round(ref: np.ndarray) -> np.ndarray:
     return torch.from_numpy(ref).to(torch.bfloat16).double().numpy()
 
 
+def oracle_tokens(x, layer_cpu: dict, shape, residual: bool, tokens: np.ndarray, idx_override: np.ndarray,
+                  threads: int = 0) -> np.ndarray:
+    """The oracle's output for `tokens` (with the given selections), the
+    tokens split over host threads (the oracle is plain C called through
+    ctypes, which releases the interpreter lock; it keeps no state between
+    calls)."""
+    import concurrent.futures
+    import os
+    n = len(tokens)
+    threads = threads or max(1, min(16, os.cpu_count() or 1))
+    if n <= 8 or threads == 1:
+        return oracle.moe_tokens(x, layer_cpu, shape, residual=residual, tokens=tokens.astype(np.int32),
+                                 idx_override=idx_override)["out"]
+    parts = np.array_split(np.arange(n), min(threads, n))
+
+    def run(sel):
+        return oracle.moe_tokens(x, layer_cpu, shape, residual=residual, tokens=tokens[sel].astype(np.int32),
+                                 idx_override=idx_override[sel])["out"]
+
+    with concurrent.futures.ThreadPoolExecutor(len(parts)) as ex:
+        outs = list(ex.map(run, parts))
+    return np.concatenate(outs, axis=0)
+
+
 def compare_layer(x: torch.Tensor, out: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, layer_cpu: dict,
                   shape, residual: bool, sample=None, tol: float = OUT_TOL, rounded: bool = False) -> dict:
     """Full comparison.  Routing is checked on every token; outputs on
@@ -101,15 +131,63 @@ def compare_layer(x: torch.Tensor, out: torch.Tensor, idx: torch.Tensor, w: torc
     ties, werr = check_routing(idx_g, w_g, ref_r, layer_cpu["router_bias"].numpy(), shape.K)
     T = x.shape[0]
     tok = np.arange(T) if sample is None else np.unique(np.asarray(sample, np.int64))
-    ref = oracle.moe_tokens(xc, layer_cpu, shape, residual=residual, tokens=tok.astype(np.int32),
-                            idx_override=idx_g[tok])
+    ref = oracle_tokens(xc, layer_cpu, shape, residual, tok, np.ascontiguousarray(idx_g[tok]))
     o = out[torch.from_numpy(tok).to(out.device)]
-    err = rel_l2(o, ref["out"], bf16_round(ref["out"]) if rounded else None)
+    err = rel_l2(o, ref, bf16_round(ref) if rounded else None)
     assert np.all(np.isfinite(err)), "non-finite output"
     worst = int(tok[int(np.argmax(err))])
     assert err.max() <= tol, f"per-token rel L2 {err.max():.3e} > {tol} at token {worst}"
     return dict(ties=len(ties), max_rel_l2=float(err.max()), mean_rel_l2=float(err.mean()),
                 max_w_rel=werr, tokens_checked=len(tok))
+
+
+def tile_cover(idx: np.ndarray, E: int, tile: int, shared: bool) -> np.ndarray:
+    """Tokens that put at least one checked token into every work unit of the
+    expert kernels: every `tile`-slot piece of every routed bucket (buckets in
+    ascending expert order, each listing its tokens in (t, k) order, as the
+    kernels lay out their slots) and, with a shared expert, every `tile`-token
+    piece of the shared bucket (tokens in order).  Greedy: a unit not yet
+    covered adds its first token, which also covers the units of that token's
+    other picks and its shared piece.  The last token of every bucket (its
+    ragged tail) is added as well when the bucket spans several units."""
+    T, K = idx.shape
+    flat = idx.reshape(-1).astype(np.int64)
+    tok = np.repeat(np.arange(T), K)
+    order = np.argsort(flat, kind="stable")  # (t, k) order within each expert
+    se, st = flat[order], tok[order]
+    start = np.searchsorted(se, np.arange(E))
+    unit_of = np.empty(T * K, np.int64)  # unit id of each (t, k) pick
+    units_first = []
+    uid = 0
+    for e in range(E):
+        lo, hi = start[e], (start[e + 1] if e + 1 < E else se.size)
+        for m0 in range(lo, hi, tile):
+            m1 = min(hi, m0 + tile)
+            unit_of[order[m0:m1]] = uid
+            units_first.append(int(st[m0]))
+            uid += 1
+    n_routed = uid
+    covered = np.zeros(n_routed + (-(-T // tile) if shared else 0), bool)
+    picks_of = unit_of.reshape(T, K)
+    chosen = []
+
+    def take(t):
+        chosen.append(t)
+        covered[picks_of[t]] = True
+        if shared:
+            covered[n_routed + t // tile] = True
+
+    for u in range(n_routed):
+        if not covered[u]:
+            take(units_first[u])
+    if shared:
+        for m in range(-(-T // tile)):
+            if not covered[n_routed + m]:
+                take(m * tile)
+    assert covered.all()
+    ends = np.append(start[1:], se.size)
+    tails = [int(st[ends[e] - 1]) for e in range(E) if ends[e] - start[e] > tile]
+    return np.unique(np.asarray(chosen + tails + [T - 1], np.int64))
 
 
 def sample_tokens(T: int, n: int = 32, seed: int = 0, extra=()) -> np.ndarray:

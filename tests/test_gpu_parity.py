@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import workloads
-from tests._parity import OUT_F32_TOL, compare_layer, sample_tokens, to_cpu_layer
+from tests._parity import OUT_F32_TOL, compare_layer, sample_tokens, tile_cover, to_cpu_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -65,11 +65,26 @@ def test_nano_decode_stack(moe, cuda_device, T):
     assert not torch.equal(x, x0)
 
 
+def work_unit_sample(moe, shape, T, idx, n, seed, extra=()):
+    """Checked tokens of a full-size case: at least one token of every work
+    unit of the expert kernels that ran (every 128-token tile of every bucket
+    on the tensor-core path; every 16-token piece of every bucket, which
+    covers the 32-token tasks too, on the weight-streaming paths), every
+    multi-unit bucket's last token, head and tail tokens and a seeded draw."""
+    path = moe.layer_path(shape, T)
+    tile = 128 if path == moe.MOE_PATH_TENSOR_CORE else 16
+    cover = tile_cover(idx.cpu().numpy(), shape.E, tile, shape.Is > 0)
+    return np.union1d(cover, sample_tokens(T, n, seed, extra))
+
+
 def test_nano_prefill_t4096(moe, cuda_device):
     wl = workloads.WORKLOADS["nano_prefill_t4096"]
     layer = workloads.make_layer(wl.shape, wl.wid, 0, cuda_device, wl.bias_mode)
     x = workloads.make_x(wl.shape, 4096, wl.wid, device=cuda_device)
-    _, idx, _, _ = check(moe, x, layer, wl.shape, sample=sample_tokens(4096, 40, 1))
+    out, idx, w = run(moe, x, layer, wl.shape)
+    sample = work_unit_sample(moe, wl.shape, 4096, idx, 40, 1)
+    r = compare_layer(x, out, idx, w, to_cpu_layer(layer), wl.shape, False, sample)
+    print("prefill", r)
     loads = torch.bincount(idx.flatten().long(), minlength=64)
     assert int(loads.min()) > 0            # zero bias: every expert receives tokens
 
@@ -83,8 +98,8 @@ def test_nano_zipf_t16384(moe, cuda_device):
     loads = np.bincount(idx_np.reshape(-1), minlength=64)
     hot = np.nonzero(idx_np == np.argmax(loads))[0][:3]
     cold = np.nonzero(idx_np == np.argmin(loads))[0][:3]
-    r = compare_layer(x, out, idx, w, to_cpu_layer(layer), wl.shape, False,
-                      sample_tokens(16384, 32, 2, extra=np.concatenate([hot, cold])))
+    sample = work_unit_sample(moe, wl.shape, 16384, idx, 32, 2, extra=np.concatenate([hot, cold]))
+    r = compare_layer(x, out, idx, w, to_cpu_layer(layer), wl.shape, False, sample)
     print("zipf loads", sorted(loads.tolist(), reverse=True)[:5], "...", sorted(loads.tolist())[:3], r)
     assert loads.max() > 2000 and loads.min() < 200
 
@@ -94,7 +109,9 @@ def test_large_layer(moe, cuda_device, T, n):
     wl = workloads.WORKLOADS["large_layer"]
     layer = workloads.make_layer(wl.shape, wl.wid, 0, cuda_device, wl.bias_mode)
     x = workloads.make_x(wl.shape, T, wl.wid, device=cuda_device)
-    check(moe, x, layer, wl.shape, sample=sample_tokens(T, n, 3))
+    out, idx, w = run(moe, x, layer, wl.shape)
+    r = compare_layer(x, out, idx, w, to_cpu_layer(layer), wl.shape, False, work_unit_sample(moe, wl.shape, T, idx, n, 3))
+    print(f"large T={T}", r)
 
 
 # --- edge cases on small shapes -------------------------------------------------
@@ -208,8 +225,9 @@ def test_hot_expert_many_chunks(moe, cuda_device):
     layer["router_bias"][7] = 5.0
     x = workloads.make_x(wl.shape, 150, wl.wid, batch=9, device=cuda_device)
     assert moe.layer_path(wl.shape, 150, moe.MOE_FORCE_DECODE) == moe.MOE_PATH_LARGE_STREAMING
-    out, idx, _, _ = check(moe, x, layer, wl.shape, flags=moe.MOE_FORCE_DECODE,
-                           sample=sample_tokens(150, 40, 7))
+    out, idx, w = run(moe, x, layer, wl.shape, flags=moe.MOE_FORCE_DECODE)
+    sample = np.union1d(tile_cover(idx.cpu().numpy(), wl.shape.E, 16, True), sample_tokens(150, 40, 7))
+    compare_layer(x, out, idx, w, to_cpu_layer(layer), wl.shape, False, sample)
     assert idx[:, 0].eq(7).all()
 
 
