@@ -19,6 +19,7 @@ import torch
 __all__ = [
     "MoeError", "moe_cfg_t", "moe_shared_weights_t", "lib", "EXPORTED_SYMBOLS",
     "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK", "MOE_FORCE_DECODE", "MOE_FORCE_PREFILL", "MOE_OUT_F32",
+    "MOE_TEST_STALL", "MOE_DEVSTAT_TIMEOUT", "device_status",
     "workspace_bytes", "workspace_bytes_upto", "layer_forward", "MoELayer", "decode_max_tokens", "kernel_launches", "layer_path",
     "MOE_PATH_SMALL_BATCH", "MOE_PATH_TENSOR_CORE", "MOE_PATH_LARGE_STREAMING", "LIB_PATH",
 ]
@@ -37,6 +38,13 @@ MOE_DEBUG_CHECK = 1 << 1
 MOE_FORCE_DECODE = 1 << 2
 MOE_FORCE_PREFILL = 1 << 3
 MOE_OUT_F32 = 1 << 4
+MOE_TEST_STALL = 1 << 6
+# device status word (the first 4 bytes of the workspace)
+MOE_DEVSTAT_BAD_EXPERT = 1 << 0
+MOE_DEVSTAT_BAD_SLOT = 1 << 1
+MOE_DEVSTAT_BAD_COUNT = 1 << 2
+MOE_DEVSTAT_BAD_TASK = 1 << 3
+MOE_DEVSTAT_TIMEOUT = 1 << 4
 # kernel sequences (moe_layer_path)
 MOE_PATH_SMALL_BATCH = 1
 MOE_PATH_TENSOR_CORE = 2
@@ -228,15 +236,27 @@ def layer_forward(x: torch.Tensor, layer: dict, shape, out: Optional[torch.Tenso
     return out
 
 
+def device_status(workspace: torch.Tensor) -> int:
+    """The device status word (MOE_DEVSTAT_* bits) that the last call on
+    ``workspace`` left in its first 4 bytes (synchronises the stream)."""
+    return int(workspace[:4].view(torch.int32).item()) & 0xFFFFFFFF
+
+
 class MoELayer:
-    """One layer's device weights plus a workspace sized for up to ``max_tokens``."""
+    """One layer's device weights plus a workspace sized for every call of up
+    to ``max_tokens`` tokens under any per-call flags (the kernel sequence,
+    and so the workspace, depends on MOE_FORCE_DECODE / MOE_FORCE_PREFILL)."""
 
     def __init__(self, layer: dict, shape, max_tokens: int, device=None):
         self.layer = layer
         self.shape = shape
         self.device = torch.device(device) if device is not None else layer["w13"].device
         self.max_tokens = int(max_tokens)
-        self.workspace = new_workspace(shape, self.max_tokens, self.device)
+        n = max(workspace_bytes_upto(shape, self.max_tokens, f)
+                for f in (0, MOE_FORCE_DECODE, MOE_FORCE_PREFILL))
+        if n == 0:
+            raise MoeError(MOE_ERR_UNSUPPORTED, "moe_layer_workspace_bytes")
+        self.workspace = torch.empty(n, dtype=torch.uint8, device=self.device)
 
     def __call__(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, residual: bool = False,
                  flags: int = 0, topk_idx=None, topk_w=None, stage_events=None) -> torch.Tensor:

@@ -2,7 +2,10 @@
 // allocate device memory (see include/moe_int4.h).  The scratch memory the
 // kernels need comes from a fixed-size array in this file instead of a
 // caller-provided workspace; everything else is moe_layer_forward unchanged.
-#include <atomic>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
 
 #include "moe_int4.h"
 
@@ -15,11 +18,49 @@ constexpr size_t kStaticWorkspaceBytes = MOE_STATIC_WORKSPACE_BYTES;
 
 __device__ __align__(256) unsigned char g_static_ws[kStaticWorkspaceBytes];
 
-// Device address of g_static_ws per device.  In host code the symbol's name
-// is only a host-side stand-in; a kernel given it would fault (or, where the
-// GPU can reach host memory, silently use the wrong memory), so the address
-// is fetched from the runtime with the device current.
-std::atomic<void*> g_static_ws_ptr[64];
+// Device address of g_static_ws per device, with the driver context it
+// belongs to.  In host code the symbol's name is only a host-side stand-in; a
+// kernel given it would fault (or, where the GPU can reach host memory,
+// silently use the wrong memory), so the address is fetched from the runtime
+// with the device current.  The module, and so the address, is per context:
+// after cudaDeviceReset, or under another context on the same device, the
+// address is looked up again.
+struct StaticWs {
+    void* ctx = nullptr;
+    void* ptr = nullptr;
+};
+StaticWs g_static_ws_of[64];
+std::mutex g_static_ws_mu;
+
+typedef CUresult (*PFN_ctxGetCurrent)(CUcontext*);
+
+void* current_context() {
+    static PFN_ctxGetCurrent fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<PFN_ctxGetCurrent>(f);
+    }();
+    CUcontext c = nullptr;
+    if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
+// The array's device address on device `dev` (current) in the current
+// context, or nullptr if the runtime cannot give it.
+void* static_ws_address(int dev) {
+    std::lock_guard<std::mutex> lock(g_static_ws_mu);
+    StaticWs& w = g_static_ws_of[dev];
+    void* ctx = current_context();
+    if (w.ptr && ctx && ctx == w.ctx) return w.ptr;
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_ws) != cudaSuccess || !ptr) return nullptr;
+    w.ptr = ptr;
+    w.ctx = current_context();  // the lookup made the runtime's context current if none was
+    return ptr;
+}
 
 }  // namespace
 
@@ -43,11 +84,8 @@ int moe_layer_forward_static_ws(const void* x, const float* router_w, const floa
     if (need > kStaticWorkspaceBytes) return MOE_ERR_WORKSPACE;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
-    void* ws = g_static_ws_ptr[dev].load(std::memory_order_acquire);
-    if (!ws) {
-        if (cudaGetSymbolAddress(&ws, g_static_ws) != cudaSuccess || !ws) return MOE_ERR_CUDA;
-        g_static_ws_ptr[dev].store(ws, std::memory_order_release);
-    }
+    void* ws = static_ws_address(dev);
+    if (!ws) return MOE_ERR_CUDA;
     moe_cfg_t c = *cfg;
     c.workspace = ws;
     c.workspace_bytes = kStaticWorkspaceBytes;

@@ -53,6 +53,8 @@ def test_static_workspace_matches_regular_entry_point(moe, cuda_device, T):
         torch.cuda.synchronize()
         err = rel_l2(out, ref.double().cpu().numpy())
         assert np.all(np.isfinite(err)) and err.max() <= OUT_TOL
+        # the same kernels on the same inputs: the same result, bit for bit
+        assert torch.equal(out, ref)
 
 
 def test_static_workspace_rejects_oversized_calls(moe, cuda_device):
