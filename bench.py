@@ -4,18 +4,24 @@ top-k, int4 SwiGLU experts, shared expert, weighted combine) on B200.
 
 Default workload: the Nano decode stack -- 23 stacked MoE layers (hidden 1024,
 64 experts, top-2, routed intermediate 512, shared intermediate 2048), each
-layer adding its input (x_{l+1} = x_l + MoE_l(x_l)), at T=64 tokens, with the
-decode sweep T in {1,4,16,64} reported beside it.  One step = one pass of the
+layer adding its input (x_{l+1} = x_l + MoE_l(x_l)), at T=64 tokens, run as
+ONE moe_stack_forward call (the fused stack kernel), with the sweep over the
+decode and speculative-verify sizes T in {1,2,3,4,16,64} (fused kernel and
+per-layer kernel sequences) reported beside it.  One step = one pass of the
 whole layer stack over one batch of synthetic tokens.  The metric counts one
 token passing through one MoE layer as one token (tokens/s = T*layers/s).
+The line also carries the other workloads (one Nano layer at T=16, Nano
+prefill at T=4096, Zipf routing at T=16384, the large layer at T=1, 32 and
+512), each timed through the public API with its own clock record.
 
 Timing: W warm-up steps, then exactly K timed steps bracketed by a barrier
 and a device synchronize; each step is timed with CUDA events on the stream
 that runs it, and L2 is flushed (a 256 MiB write) between steps, outside the
 timed events.  Four different input batches rotate, so the routing changes
 from step to step.  The step is replayed as a CUDA graph of the library's
-C-ABI calls.  A second, instrumented pass records the library's per-stage
-events to time each kernel; the roofline uses that per-kernel time.
+C-ABI call(s).  The fused kernel is the whole step, so its roofline uses the
+step's median time; for the per-layer kernel sequences an instrumented eager
+pass records the library's per-stage events to time each kernel.
 
 --impl reference times the CPU oracle (plain C, double precision, one core)
 on a bounded sample of the same workload.
@@ -59,6 +65,10 @@ def parse_args():
     ap.add_argument("--tokens", type=int, default=None, help="T (default: the workload's largest)")
     ap.add_argument("--no-sweep", action="store_true", help="skip the per-T sweep of the decode stack")
     ap.add_argument("--no-graph", action="store_true", help="launch the C-ABI calls directly")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other workloads (prefill, Zipf, large layer) reported beside the decode stack")
+    ap.add_argument("--per-layer", action="store_true",
+                    help="time the stack as one moe_layer_forward call per layer instead of the fused kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -233,43 +243,54 @@ def stage_work(stage, shape, T, uniq):
 
 # --------------------------------------------------------------------------- our arm
 
-class Stack:
-    """Device weights of the workload's layers and the buffers of one T."""
+class Runner:
+    """A workload's weights and the buffers of one T, with one step = one pass
+    of every layer over one batch: either ONE moe_stack_forward call (the fused
+    stack kernel; mode "fused") or one moe_layer_forward call per layer (mode
+    "per_layer")."""
 
-    def __init__(self, moe, wl, T, device, layers=None):
-        self.moe, self.wl, self.T, self.device = moe, wl, T, device
+    def __init__(self, moe, wl, T, device, stacked, mode):
+        self.moe, self.wl, self.T, self.device, self.mode = moe, wl, T, device, mode
         self.shape = wl.shape
-        self.layers = layers if layers is not None else [
-            workloads.make_layer(wl.shape, wl.wid, l, device, wl.bias_mode) for l in range(wl.layers)]
+        self.L = wl.layers
+        self.stacked = stacked
+        self.layers = [{k: v[l] for k, v in stacked.items()} for l in range(self.L)]
         self.xs = [workloads.make_x(wl.shape, T, wl.wid, batch=b, device=device) for b in range(N_BATCHES)]
-        self.acts = [torch.empty((T, wl.shape.H), dtype=torch.bfloat16, device=device) for _ in range(wl.layers)]
-        self.ws = moe.new_workspace(wl.shape, T, device)
+        self.outs = torch.empty((self.L, T, wl.shape.H), dtype=torch.bfloat16, device=device)
         self.flags = moe.MOE_ADD_RESIDUAL if wl.residual else 0
+        if mode == "fused":
+            n = moe.stack_workspace_bytes(wl.shape, T, self.L, self.flags)
+            self.ws = torch.empty(n, dtype=torch.uint8, device=device)
+        else:
+            self.ws = moe.new_workspace(wl.shape, T, device)
 
-    def run(self, b, stage_events=None, x=None):
+    def run(self, b, x=None, stage_events=None, topk_idx=None):
         inp = self.xs[b] if x is None else x
-        for l, layer in enumerate(self.layers):
-            ev = None if stage_events is None else stage_events[l]
-            self.moe.layer_forward(inp, layer, self.shape, out=self.acts[l], workspace=self.ws,
-                                   flags=self.flags, stage_events=ev)
-            inp = self.acts[l]
-        return inp
+        if self.mode == "fused":
+            self.moe.stack_forward(inp, self.stacked, self.shape, outs=self.outs, workspace=self.ws, flags=self.flags,
+                                   topk_idx=topk_idx)
+        else:
+            for l, layer in enumerate(self.layers):
+                ev = None if stage_events is None else stage_events[l]
+                self.moe.layer_forward(inp, layer, self.shape, out=self.outs[l], workspace=self.ws, flags=self.flags,
+                                       stage_events=ev, topk_idx=None if topk_idx is None else topk_idx[l])
+                inp = self.outs[l]
+        return self.outs[self.L - 1]
 
     def routing_unique(self):
         """Touched routed experts per (batch, layer), from the library's top-k output."""
-        K = self.shape.K
-        idx = torch.empty((self.T, K), dtype=torch.int32, device=self.device)
+        idx = torch.empty((self.L, self.T, self.shape.K), dtype=torch.int32, device=self.device)
         out = []
         for b in range(N_BATCHES):
-            inp, per = self.xs[b], []
-            for l, layer in enumerate(self.layers):
-                self.moe.layer_forward(inp, layer, self.shape, out=self.acts[l], workspace=self.ws,
-                                       flags=self.flags, topk_idx=idx)
-                per.append(int(torch.unique(idx).numel()))
-                inp = self.acts[l]
-            out.append(per)
+            self.run(b, topk_idx=idx)
+            out.append([int(torch.unique(idx[l]).numel()) for l in range(self.L)])
         torch.cuda.synchronize()
         return out
+
+    def launches_per_step(self):
+        if self.mode == "fused":
+            return 1
+        return self.moe.kernel_launches(self.shape, self.T) * self.L
 
 
 def make_events(n):
@@ -279,15 +300,18 @@ def make_events(n):
     return evs
 
 
-def timed_steps(stack, steps, warmup, use_graph, flush, instrumented=False, dist_barrier=None):
+def timed_steps(runner, steps, warmup, use_graph, flush, instrumented=False, dist_barrier=None):
     """Returns (per-step ms list, per-stage ms sums per step).
 
-    instrumented=True: the library records its per-stage events around every
-    kernel.  Events recorded inside a captured graph cannot be timed, so this
+    Each step is timed with CUDA events on the stream that runs it; the L2
+    flush runs before each step, outside the events.  instrumented=True (per
+    layer mode only): the library records its per-stage events around every
+    kernel; events recorded inside a captured graph cannot be timed, so this
     pass launches the C-ABI calls directly, behind a GPU sleep long enough for
-    the whole step to be queued first: the stage brackets then hold device
-    time only, not host launch latency."""
-    L = len(stack.layers)
+    the whole step to be queued first, so that the brackets hold device time
+    and not host launch latency (but the kernels no longer overlap their
+    neighbours' tails, so a kernel's time there is an upper bound)."""
+    L = runner.L
     stage_ev = [make_events(8) for _ in range(L)] if instrumented else None
     if instrumented:
         use_graph = False
@@ -299,13 +323,13 @@ def timed_steps(stack, steps, warmup, use_graph, flush, instrumented=False, dist
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
             for b in range(N_BATCHES):  # eager warm-up before capture
-                stack.run(b, stage_ev)
+                runner.run(b)
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
         for b in range(N_BATCHES):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                stack.run(b, stage_ev)
+                runner.run(b)
             graphs.append(g)
         torch.cuda.synchronize()
 
@@ -313,7 +337,7 @@ def timed_steps(stack, steps, warmup, use_graph, flush, instrumented=False, dist
         if graphs is not None:
             graphs[b].replay()
         else:
-            stack.run(b, stage_ev)
+            runner.run(b, stage_events=stage_ev)
 
     for i in range(warmup):
         flush.zero_()
@@ -324,7 +348,7 @@ def timed_steps(stack, steps, warmup, use_graph, flush, instrumented=False, dist
     torch.cuda.synchronize()
     st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    step_ms, stage_ms = [], []
+    stage_ms = []
     for i in range(steps):
         flush.zero_()
         if instrumented:
@@ -345,21 +369,22 @@ def timed_steps(stack, steps, warmup, use_graph, flush, instrumented=False, dist
     return step_ms, stage_ms
 
 
-def e2e_steps(stack, steps, warmup, flush, dist_barrier=None):
+def e2e_steps(runner, steps, warmup, flush, dist_barrier=None):
     """Same step through the public API with host buffers: pinned host x ->
-    device, the layer stack (graph of C-ABI calls), device -> pinned host out."""
-    T, H = stack.T, stack.shape.H
-    host_x = [stack.xs[b].cpu().pin_memory() for b in range(N_BATCHES)]
+    device, the step (a CUDA graph of the C-ABI call(s)), the last layer's
+    output device -> pinned host."""
+    T, H = runner.T, runner.shape.H
+    host_x = [runner.xs[b].cpu().pin_memory() for b in range(N_BATCHES)]
     host_out = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(stack.xs[0])
+    x_dev = torch.empty_like(runner.xs[0])
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
-        stack.run(0, x=x_dev)
+        runner.run(0, x=x_dev)
     torch.cuda.current_stream().wait_stream(s)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        out_dev = stack.run(0, x=x_dev)
+        out_dev = runner.run(0, x=x_dev)
     torch.cuda.synchronize()
 
     def one(b):
@@ -388,30 +413,68 @@ def e2e_steps(stack, steps, warmup, flush, dist_barrier=None):
     return ms, T * H * 2, T * H * 2
 
 
-def cpu_baseline_sample(stack, budget_s=20.0):
+def host_cpu():
+    """CPU model and logical CPU count of the host (for the CPU baseline)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
+
+
+class pinned_to_one_core:
+    """Runs the block on one host core (the first this process may use), as the
+    CPU baseline plan asks (taskset -c <core>); restores the affinity after."""
+
+    def __enter__(self):
+        self.old = None
+        self.core = None
+        try:
+            self.old = os.sched_getaffinity(0)
+            self.core = min(self.old)
+            os.sched_setaffinity(0, {self.core})
+        except (AttributeError, OSError):
+            pass
+        return self
+
+    def __exit__(self, *a):
+        if self.old is not None:
+            try:
+                os.sched_setaffinity(0, self.old)
+            except OSError:
+                pass
+
+
+def cpu_baseline_sample(runner, budget_s=15.0):
     """The oracle (single-threaded C, f64) on a bounded sample of the step:
     the first tokens of batch 0 through every layer, each layer fed the GPU's
-    bf16 input of that layer.  Returns tokens/s (token-layers) and the sample."""
+    bf16 input of that layer, pinned to one host core.  Returns (tokens/s
+    counting token-layers, the sample, the core)."""
     import oracle
-    shape = stack.shape
+    shape = runner.shape
     with torch.no_grad():
-        inputs = [stack.xs[0]]
-        stack.run(0)
-        inputs += stack.acts[:-1]
+        runner.run(0)
+        torch.cuda.synchronize()
+        inputs = [runner.xs[0]] + [runner.outs[l] for l in range(runner.L - 1)]
         inputs = [t.cpu() for t in inputs]
-    layers_cpu = [{k: v.cpu() for k, v in layer.items()} for layer in stack.layers]
-    n_tok = stack.T
-    # calibrate on one token of layer 0, then size the sample to the budget
-    t0 = time.perf_counter()
-    oracle.moe_tokens(inputs[0], layers_cpu[0], shape, residual=stack.wl.residual, tokens=[0])
-    per = max(time.perf_counter() - t0, 1e-4)
-    n_tok = int(max(1, min(stack.T, budget_s / (per * len(layers_cpu)))))
-    toks = list(range(n_tok))
-    t0 = time.perf_counter()
-    for l, layer in enumerate(layers_cpu):
-        oracle.moe_tokens(inputs[l], layer, shape, residual=stack.wl.residual, tokens=toks)
-    dt = time.perf_counter() - t0
-    return n_tok * len(layers_cpu) / dt, f"{n_tok} of {stack.T} tokens of one batch through all {len(layers_cpu)} layers ({dt:.1f} s)"
+    layers_cpu = [{k: v.cpu() for k, v in layer.items()} for layer in runner.layers]
+    with pinned_to_one_core() as pin:
+        t0 = time.perf_counter()
+        oracle.moe_tokens(inputs[0], layers_cpu[0], shape, residual=runner.wl.residual, tokens=[0])
+        per = max(time.perf_counter() - t0, 1e-4)
+        n_tok = int(max(1, min(runner.T, budget_s / (per * len(layers_cpu)))))
+        toks = list(range(n_tok))
+        t0 = time.perf_counter()
+        for l, layer in enumerate(layers_cpu):
+            oracle.moe_tokens(inputs[l], layer, shape, residual=runner.wl.residual, tokens=toks)
+        dt = time.perf_counter() - t0
+    sample = f"{n_tok} of {runner.T} tokens of one batch through all {len(layers_cpu)} layers ({dt:.1f} s)"
+    return n_tok * len(layers_cpu) / dt, sample, pin.core
 
 
 def captured_traffic(workload: str, T: int, kernel: str):
@@ -467,6 +530,98 @@ def job_throughput(world, tokens_per_step, steps, total_ms):
     return world * tokens_per_step * steps / (total_ms / 1e3)
 
 
+def dist_or_none(world, dist):
+    return dist if world > 1 else None
+
+
+def percentiles(ms):
+    s = sorted(ms)
+    q = lambda f: s[min(len(s) - 1, int(f * (len(s) - 1) + 0.5))]
+    return {"median": round(statistics.median(s), 4), "p10": round(q(0.1), 4), "p90": round(q(0.9), 4),
+            "mean": round(statistics.mean(s), 4), "n": len(s)}
+
+
+def roofline_of(alg_b, alg_f, seconds, peaks, kernel, timing, traffic=None):
+    """Roofline object of one kernel (or step): bound from the arithmetic
+    intensity against the ridge of the measured peaks."""
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if alg_b > 0 and alg_f / alg_b >= ridge:
+        achieved = alg_f / seconds / 1e12
+        r = {"bound": "tensor", "kernel": kernel, "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
+             "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+             "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json bf16_tflops, burst)"}
+    else:
+        achieved = alg_b / seconds / 1e9
+        r = {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+             "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+             "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy)"}
+    r.update({"traffic": traffic, "alg_bytes_per_launch": int(alg_b), "alg_flops_per_launch": int(alg_f),
+              "avg_launch_us": round(seconds * 1e6, 3), "timing": timing})
+    return r
+
+
+def stacked_weights(moe, wl, device):
+    layers = [workloads.make_layer(wl.shape, wl.wid, l, device, wl.bias_mode) for l in range(wl.layers)]
+    st = moe.stack_layers(layers)
+    del layers
+    torch.cuda.empty_cache()
+    return st
+
+
+def measure(runner, steps, warmup, use_graph, flush, peaks, device, barrier=None):
+    """Timed steps of one runner with its clock record and work accounting."""
+    uniq = runner.routing_unique()
+    with ClockSampler(device.index if device.index is not None else 0, pci_bus_id(device)) as clk:
+        ms, _ = timed_steps(runner, steps, warmup, use_graph, flush, dist_barrier=barrier)
+    work = [step_bytes_flops(runner.shape, runner.T, uniq[i % N_BATCHES]) for i in range(steps)]
+    return {"ms": ms, "uniq": uniq, "clocks": clk.summary(), "bytes": statistics.mean(w[0] for w in work),
+            "flops": statistics.mean(w[1] for w in work)}
+
+
+def workload_entry(moe, wl, T, device, steps, warmup, use_graph, flush, peaks, stacked=None):
+    """One extra workload: its step (all its layers) timed through the public
+    API, median over the steps, with its own clock record; for the per-layer
+    kernel sequences the dominant expert kernel's rate from the instrumented
+    eager pass."""
+    stacked = stacked if stacked is not None else stacked_weights(moe, wl, device)
+    L = wl.layers
+    modes = ["per_layer"]
+    if moe.stack_path(wl.shape, T, L, moe.MOE_ADD_RESIDUAL if wl.residual else 0) == moe.MOE_PATH_FUSED_STACK:
+        modes.insert(0, "fused")
+    entry = {"workload": wl.name, "T": T, "layers": L}
+    for mode in modes:
+        r = Runner(moe, wl, T, device, stacked, mode)
+        m = measure(r, steps, warmup, use_graph, flush, peaks, device)
+        med = statistics.median(m["ms"]) / 1e3
+        d = {"ms_per_step": percentiles(m["ms"]), "tokens_per_s": round(T * L / med, 1),
+             "alg_bytes_per_step": int(m["bytes"]), "alg_flops_per_step": int(m["flops"]),
+             "step_roofline": roofline_of(m["bytes"], m["flops"], med, peaks, "whole step", "CUDA graph, median"),
+             "clocks": m["clocks"], "gpu_launches_per_step": r.launches_per_step(),
+             "path": "fused stack kernel" if mode == "fused" else
+                     {moe.MOE_PATH_SMALL_BATCH: "small-batch kernels", moe.MOE_PATH_TENSOR_CORE: "tensor-core kernels",
+                      moe.MOE_PATH_LARGE_STREAMING: "large-batch streaming kernels"}[moe.layer_path(wl.shape, T)]}
+        if mode == "per_layer":
+            _, stage_ms = timed_steps(r, max(3, steps // 2), 2, use_graph, flush, instrumented=True)
+            stage_mean = [statistics.mean(s[k] for s in stage_ms) for k in range(4)]
+            dom = 1 if stage_mean[1] >= stage_mean[2] else 2
+            names = moe.STAGE_NAMES
+            tc = moe.layer_path(wl.shape, T) == moe.MOE_PATH_TENSOR_CORE
+            w13, w2 = streaming_kernel_names(wl.shape)
+            kname = (f"grouped_gemm_kernel<{dom}>" if tc else (w13 if dom == 1 else w2))
+            u = m["uniq"]
+            kw = [[stage_work(names[dom], wl.shape, T, x) for x in u[i % N_BATCHES]] for i in range(len(stage_ms))]
+            kb = statistics.mean(sum(w[0] for w in ws) for ws in kw) / L
+            kf = statistics.mean(sum(w[1] for w in ws) for ws in kw) / L
+            d["stages_us_per_step"] = {names[k]: round(stage_mean[k] * 1e3, 2) for k in range(4)}
+            d["kernel_roofline"] = roofline_of(kb, kf, stage_mean[dom] / L / 1e3, peaks, kname,
+                                               "eager pass with per-stage events (no overlap with neighbours)",
+                                               captured_traffic(wl.name, T, kname))
+        entry[mode] = d
+        del r
+        torch.cuda.empty_cache()
+    return entry
+
+
 def run_ours(args, rank, world, device, dist):
     import int4_expert_ffn_sigmoid_b200 as moe
     wl = workloads.WORKLOADS[args.workload]
@@ -475,97 +630,109 @@ def run_ours(args, rank, world, device, dist):
     barrier = (lambda: dist.barrier()) if world > 1 else None
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     use_graph = not args.no_graph
-
-    stack = Stack(moe, wl, T, device)
-    uniq = stack.routing_unique()
-    with ClockSampler(device.index if device.index is not None else 0, pci_bus_id(device)) as clk:
-        step_ms, _ = timed_steps(stack, args.steps, args.warmup, use_graph, flush, dist_barrier=barrier)
-    clocks = clk.summary()
-    _, stage_ms = timed_steps(stack, args.steps, 2, use_graph, flush, instrumented=True)
-    e2e_ms, h2d, d2h = e2e_steps(stack, args.steps, args.warmup, flush, dist_barrier=barrier)
-
-    total_ms, e2e_total = max_over_ranks([sum(step_ms), sum(e2e_ms)], dist if world > 1 else None, device)
+    stacked = stacked_weights(moe, wl, device)
+    flags = moe.MOE_ADD_RESIDUAL if wl.residual else 0
+    fused = (not args.per_layer) and moe.stack_path(wl.shape, T, wl.layers, flags) == moe.MOE_PATH_FUSED_STACK
+    runner = Runner(moe, wl, T, device, stacked, "fused" if fused else "per_layer")
     L = wl.layers
+
+    m = measure(runner, args.steps, args.warmup, use_graph, flush, peaks, device, barrier)
+    step_ms = m["ms"]
+    e2e_ms, h2d, d2h = e2e_steps(runner, args.steps, args.warmup, flush, dist_barrier=barrier)
+    total_ms, e2e_total, med_ms = max_over_ranks([sum(step_ms), sum(e2e_ms), statistics.median(step_ms)],
+                                                 dist_or_none(world, dist), device)
     tokens_per_step = T * L
     value = job_throughput(world, tokens_per_step, args.steps, total_ms)
     e2e_value = job_throughput(world, tokens_per_step, args.steps, e2e_total)
-
-    # work accounting (batch i % 4 at step i)
-    step_b, step_f = [], []
-    for i in range(args.steps):
-        b, f = step_bytes_flops(wl.shape, T, uniq[i % N_BATCHES])
-        step_b.append(b)
-        step_f.append(f)
     ms_mean = total_ms / args.steps
-    step_gbs = statistics.mean(step_b) / (ms_mean / 1e3) / 1e9
-    step_tflops = statistics.mean(step_f) / (ms_mean / 1e3) / 1e12
+    step_gbs = m["bytes"] / (ms_mean / 1e3) / 1e9
 
-    # dominant kernel (largest per-step stage time) and its roofline
-    stage_mean = [statistics.mean(s[k] for s in stage_ms) for k in range(4)]
-    names = moe.STAGE_NAMES
-    dom = 1 if stage_mean[1] >= stage_mean[2] else 2  # the dominant expert kernel
-    tc_path = moe.layer_path(wl.shape, T) == moe.MOE_PATH_TENSOR_CORE
-    w13_name, w2_name = streaming_kernel_names(wl.shape)
-    kname = (("grouped_gemm_kernel<1>" if dom == 1 else "grouped_gemm_kernel<2>") if tc_path
-             else (w13_name if dom == 1 else w2_name))
-    work = [[stage_work(names[dom], wl.shape, T, u) for u in uniq[i % N_BATCHES]] for i in range(args.steps)]
-    alg_b = statistics.mean(sum(w[0] for w in ws) for ws in work) / L
-    alg_f = statistics.mean(sum(w[1] for w in ws) for ws in work) / L
-    per_launch_s = stage_mean[dom] / L / 1e3
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if alg_f / alg_b >= ridge:
-        achieved = alg_f / per_launch_s / 1e12
-        roofline = {"bound": "tensor", "kernel": kname, "achieved": round(achieved, 2),
-                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-                    "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json bf16_tflops, burst)"}
+    if fused:
+        # one kernel per step: the step's events bracket it (and the counters'
+        # memset that precedes it, about 1-2 us)
+        roofline = roofline_of(m["bytes"], m["flops"], med_ms / 1e3, peaks, "decode_stack_kernel",
+                               "CUDA graph step (memset + the one kernel), median over the timed steps",
+                               captured_traffic(wl.name, T, "decode_stack_kernel"))
+        stages = None
     else:
-        achieved = alg_b / per_launch_s / 1e9
-        roofline = {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                    "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                    "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy)"}
-    roofline.update({"traffic": captured_traffic(wl.name, T, kname), "alg_bytes_per_launch": int(alg_b), "alg_flops_per_launch": int(alg_f),
-                     "avg_launch_us": round(per_launch_s * 1e6, 3)})
+        _, stage_ms = timed_steps(runner, args.steps, 2, use_graph, flush, instrumented=True)
+        stage_mean = [statistics.mean(s[k] for s in stage_ms) for k in range(4)]
+        names = moe.STAGE_NAMES
+        dom = 1 if stage_mean[1] >= stage_mean[2] else 2
+        tc = moe.layer_path(wl.shape, T) == moe.MOE_PATH_TENSOR_CORE
+        w13, w2 = streaming_kernel_names(wl.shape)
+        kname = f"grouped_gemm_kernel<{dom}>" if tc else (w13 if dom == 1 else w2)
+        kw = [[stage_work(names[dom], wl.shape, T, u) for u in m["uniq"][i % N_BATCHES]] for i in range(len(stage_ms))]
+        roofline = roofline_of(statistics.mean(sum(w[0] for w in ws) for ws in kw) / L,
+                               statistics.mean(sum(w[1] for w in ws) for ws in kw) / L,
+                               stage_mean[dom] / L / 1e3, peaks, kname,
+                               "eager pass with per-stage events (no overlap with neighbours)",
+                               captured_traffic(wl.name, T, kname))
+        stages = {names[k]: round(stage_mean[k] * 1e3, 2) for k in range(4)}
 
     sweep = {}
     if wl.name == "nano_decode_stack" and not args.no_sweep:
         for Ts in wl.tokens:
-            st = stack if Ts == T else Stack(moe, wl, Ts, device, layers=stack.layers)
-            u = st.routing_unique()
-            ms, _ = timed_steps(st, max(5, args.steps // 2), 3, use_graph, flush)
-            b = statistics.mean(step_bytes_flops(wl.shape, Ts, u[i % N_BATCHES])[0] for i in range(len(ms)))
-            m = statistics.mean(ms)
-            sweep[str(Ts)] = {"tokens_per_s": round(Ts * L / (m / 1e3), 1), "ms_per_step": round(m, 4),
-                              "step_gbs": round(b / (m / 1e3) / 1e9, 1),
-                              "step_hbm_frac": round(b / (m / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
-            if st is not stack:
-                del st
-                torch.cuda.empty_cache()
+            row = {}
+            for mode in ("fused", "per_layer"):
+                if mode == "fused" and moe.stack_path(wl.shape, Ts, L, flags) != moe.MOE_PATH_FUSED_STACK:
+                    continue
+                r = runner if (Ts == T and mode == runner.mode) else Runner(moe, wl, Ts, device, stacked, mode)
+                ms = m if r is runner else measure(r, max(10, args.steps // 2), 3, use_graph, flush, peaks, device)
+                med = statistics.median(ms["ms"])
+                row[mode] = {"ms_per_step": round(med, 4), "tokens_per_s": round(Ts * L / (med / 1e3), 1),
+                             "step_gbs": round(ms["bytes"] / (med / 1e3) / 1e9, 1),
+                             "step_hbm_frac": round(ms["bytes"] / (med / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                             "sm_mhz": ms["clocks"]["sm_mhz"], "reasons": ms["clocks"]["reasons"]}
+                if r is not runner:
+                    del r
+                    torch.cuda.empty_cache()
+            sweep[str(Ts)] = row
+
+    extra = None
+    if world == 1 and not args.no_workloads and wl.name == "nano_decode_stack":
+        extra = []
+        steps = max(10, args.steps)
+        for name, Ts_list in (("nano_layer_t16", (16,)), ("nano_prefill_t4096", (4096,)),
+                              ("nano_zipf_t16384", (16384,)), ("large_layer", (1, 32, 512))):
+            w2l = workloads.WORKLOADS[name]
+            st = stacked_weights(moe, w2l, device)
+            for Ts in Ts_list:
+                extra.append(workload_entry(moe, w2l, Ts, device, steps, 3, use_graph, flush, peaks, st))
+            del st
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, sample = cpu_baseline_sample(stack)
-        cpu = {"value": round(v, 2), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
+        v, sample, core = cpu_baseline_sample(runner)
+        cpu = {"value": round(v, 2), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+               "pinned_core": core, **host_cpu()}
 
-    kernels_per_layer = moe.kernel_launches(wl.shape, T)
-    launches = args.steps * L
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "warmup": args.warmup, "ms_per_step": round(ms_mean, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8" if runner.mode == "fused" or moe.layer_path(wl.shape, T) != moe.MOE_PATH_TENSOR_CORE else "bf16",
+        "dtype_note": "weight-streaming arithmetic: int4 codes as int8, activations as two int8 parts, exact int32 "
+                      "products, f32 router, scales and sums, bf16 in and out",
+        "data": "synthetic",
         "config": {"workload": wl.name, "layers": L, "T": T, "H": wl.shape.H, "E": wl.shape.E,
                    "K": wl.shape.K, "I": wl.shape.I, "Is": wl.shape.Is, "tokens_counted": "T*layers per step",
+                   "path": "fused stack kernel (moe_stack_forward)" if fused else "one moe_layer_forward per layer",
                    "l2": "flushed between steps (256 MiB write, outside the timed events)",
                    "inputs": f"{N_BATCHES} rotating batches", "cuda_graph": use_graph,
                    "parallelism": "replicas" if world > 1 else "single"},
+        "timing": {"ms_per_step": percentiles(step_ms)},
         "step_hbm": {"achieved_gbs": round(step_gbs, 1), "frac": round(step_gbs / peaks["hbm_gbs"], 4),
-                     "alg_bytes_per_step": int(statistics.mean(step_b)), "tflops": round(step_tflops, 3)},
-        "stages_us_per_step": {names[k]: round(stage_mean[k] * 1e3, 2) for k in range(4)},
+                     "alg_bytes_per_step": int(m["bytes"]), "tflops": round(m["flops"] / (ms_mean / 1e3) / 1e12, 3)},
+        "stages_us_per_step": stages,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": kernels_per_layer * launches,
-        "clocks": clocks,
+        "gpu_launches": runner.launches_per_step() * args.steps,
+        "clocks": m["clocks"],
         "sweep": sweep or None,
+        "workloads": extra,
     }
     return line
 
@@ -575,7 +742,8 @@ def run_ours(args, rank, world, device, dist):
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm: each step is a bounded sample of
     the workload (the first tokens of a batch through every layer, the oracle
-    chaining its own outputs rounded to bf16 as the next layer's input)."""
+    chaining its own outputs rounded to bf16 as the next layer's input), on
+    one pinned host core."""
     import oracle
     if rank != 0:
         return None
@@ -591,19 +759,22 @@ def run_reference(args, rank, world):
             r = oracle.moe_tokens(x, layer, wl.shape, residual=wl.residual)
             x = torch.from_numpy(r["out"]).to(torch.bfloat16)
 
-    for i in range(args.warmup):
-        step(i)
-    t0 = time.perf_counter()
-    for i in range(args.steps):
-        step(i)
-    dt = time.perf_counter() - t0
+    with pinned_to_one_core() as pin:
+        for i in range(args.warmup):
+            step(i)
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            step(i)
+        dt = time.perf_counter() - t0
     value = n_tok * wl.layers * args.steps / dt
     sample = f"{n_tok} of {T} tokens per step through all {wl.layers} layers"
     return {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": wl.name, "layers": wl.layers, "T": T, "tokens_counted": "T*layers per step"},
-            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "config": {"workload": wl.name, "layers": wl.layers, "T": T, "H": wl.shape.H, "E": wl.shape.E,
+                       "K": wl.shape.K, "I": wl.shape.I, "Is": wl.shape.Is, "tokens_counted": "T*layers per step"},
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+                             "pinned_core": pin.core, **host_cpu()},
             "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 

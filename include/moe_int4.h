@@ -63,9 +63,13 @@ extern "C" {
 #define MOE_FORCE_PREFILL (1u << 3) /* use the grouped-GEMM kernels at any T (H a multiple of 256) */
 #define MOE_OUT_F32 (1u << 4)       /* out is f32 [T][H] (the f32 sum, no bf16 rounding): for
                                        checking the arithmetic apart from the output rounding */
+#define MOE_NO_LOOKAHEAD (1u << 5)  /* moe_stack_forward: no L2 prefetch hints (the next layer's
+                                       shared expert, routers and predicted experts); the output
+                                       is bit-identical either way */
 #define MOE_TEST_STALL (1u << 6)    /* test only: in the expert kernels that take part (the
-                                       tensor-core grouped GEMMs and the TMA-ring weight-streaming
-                                       kernels), one role first waits ~1 ms on a flag that nothing
+                                       tensor-core grouped GEMMs, the TMA-ring weight-streaming
+                                       kernels and the fused stack kernel), one role first waits
+                                       ~1 ms on a flag that nothing
                                        sets, so that the kernel takes its timeout path while its
                                        copies and MMAs are in flight: it stops, drains what it
                                        issued and records MOE_DEVSTAT_TIMEOUT.  The output is then
@@ -219,6 +223,72 @@ int moe_layer_forward_static_ws(const void* x, const float* router_w, const floa
                                 const uint8_t* packed_w2, const float* scales2,
                                 const moe_shared_weights_t* shared_w, void* out, int32_t T,
                                 const moe_cfg_t* cfg, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * A stack of L MoE layers: x_{l+1} = MoE_l(x_l) (+ x_l under MOE_ADD_RESIDUAL),
+ * each layer as moe_layer_forward defines it, x_0 = x.  (The Colibri-Nano
+ * decode runs 23 such MoE layers per token; attention between them is not
+ * part of this library.)
+ *
+ * The weights of all layers are stacked along a leading layer dimension, in
+ * the per-layer layouts of moe_layer_forward:
+ *   router_w [L][E][H] f32, router_bias [L][E] f32,
+ *   w13 [L][E][2I][H/2] uint8, s13 [L][E][2I] f32,
+ *   w2 [L][E][H][I/2] uint8, s2 [L][E][H] f32,
+ *   shared.w13 [L][2Is][H/2], shared.s13 [L][2Is], shared.w2 [L][H][Is/2],
+ *   shared.s2 [L][H].
+ * outs: bf16 [L][T][H]; layer l writes outs[l], which is layer l+1's input.
+ * cfg->topk_idx_out / topk_w_out (optional): [L][T][K].
+ *
+ * Small batches (1 <= T <= 64, H, I and Is multiples of 256, L <= 128, no
+ * MOE_FORCE_* flag) run the whole stack in ONE cooperative kernel with one
+ * CTA per SM (MOE_PATH_FUSED_STACK): per layer, router units combine the
+ * previous layer's expert outputs, compute the router logits on the tensor
+ * cores and select; every CTA then builds the layer's buckets and runs its
+ * share of the expert tasks, the down projection of an expert starting as
+ * soon as that expert's gate/up tasks are done.  Across layers it prefetches
+ * into L2 the next layer's shared expert and routers, and the experts that the
+ * next layer's router picks when run on the current layer's input (the
+ * cross-layer expert prediction of the nanocolibri-engine README, knobs
+ * table, PREDICT; colibri README, "How it works"); MOE_NO_LOOKAHEAD turns the
+ * hints off, which changes no output bit.  One cudaMemsetAsync of the
+ * workspace's counters precedes the kernel.  The arithmetic is the
+ * weight-streaming path's (see "Arithmetic" above); the router logits are
+ * summed per 128-column block of the hidden dimension, so they can differ
+ * from moe_layer_forward's in the last bits.  Other calls run one
+ * moe_layer_forward per layer (MOE_PATH_PER_LAYER).
+ *
+ * MOE_OUT_F32 is rejected (MOE_ERR_INVALID_ARG).  Under MOE_DEBUG_CHECK the
+ * call synchronises and reports the device status word (the first 4 bytes of
+ * the workspace).  A fused call waits, with bounded waits (~2 s), on counters
+ * that other CTAs of the same launch advance; a wait that runs out records
+ * MOE_DEVSTAT_TIMEOUT and every CTA stops.
+ * ------------------------------------------------------------------------- */
+typedef struct moe_stack_weights {
+    const float* router_w;
+    const float* router_bias;
+    const uint8_t* w13;
+    const float* s13;
+    const uint8_t* w2;
+    const float* s2;
+    moe_shared_weights_t shared;
+} moe_stack_weights_t;
+
+#define MOE_PATH_FUSED_STACK 4 /* moe_stack_forward: one fused kernel for the whole stack */
+#define MOE_PATH_PER_LAYER 5   /* moe_stack_forward: one moe_layer_forward per layer */
+
+/* Workspace bytes of moe_stack_forward for T tokens and L layers (0: invalid). */
+size_t moe_stack_workspace_bytes(const moe_cfg_t* cfg, int32_t T, int32_t L);
+
+/* MOE_PATH_FUSED_STACK or MOE_PATH_PER_LAYER for T tokens and L layers, or 0
+ * if T = 0 or the call would be rejected. */
+int32_t moe_stack_path(const moe_cfg_t* cfg, int32_t T, int32_t L);
+
+/* Forward of L stacked layers for T tokens (T = 0: MOE_OK, nothing launched).
+ * x: bf16 [T][H]; w: the stacked weights; outs: bf16 [L][T][H], not
+ * overlapping x.  Returns as moe_layer_forward. */
+int moe_stack_forward(const void* x, const moe_stack_weights_t* w, int32_t L, void* outs, int32_t T,
+                      const moe_cfg_t* cfg, void* stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* moe_status_str(int status);

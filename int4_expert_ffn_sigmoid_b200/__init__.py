@@ -19,7 +19,9 @@ import torch
 __all__ = [
     "MoeError", "moe_cfg_t", "moe_shared_weights_t", "lib", "EXPORTED_SYMBOLS",
     "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK", "MOE_FORCE_DECODE", "MOE_FORCE_PREFILL", "MOE_OUT_F32",
-    "MOE_TEST_STALL", "MOE_DEVSTAT_TIMEOUT", "device_status",
+    "MOE_TEST_STALL", "MOE_NO_LOOKAHEAD", "MOE_DEVSTAT_TIMEOUT", "device_status",
+    "moe_stack_weights_t", "stack_workspace_bytes", "stack_path", "stack_forward", "stack_layers",
+    "MOE_PATH_FUSED_STACK", "MOE_PATH_PER_LAYER",
     "workspace_bytes", "workspace_bytes_upto", "layer_forward", "MoELayer", "decode_max_tokens", "kernel_launches", "layer_path",
     "MOE_PATH_SMALL_BATCH", "MOE_PATH_TENSOR_CORE", "MOE_PATH_LARGE_STREAMING", "LIB_PATH",
 ]
@@ -38,6 +40,7 @@ MOE_DEBUG_CHECK = 1 << 1
 MOE_FORCE_DECODE = 1 << 2
 MOE_FORCE_PREFILL = 1 << 3
 MOE_OUT_F32 = 1 << 4
+MOE_NO_LOOKAHEAD = 1 << 5
 MOE_TEST_STALL = 1 << 6
 # device status word (the first 4 bytes of the workspace)
 MOE_DEVSTAT_BAD_EXPERT = 1 << 0
@@ -49,6 +52,8 @@ MOE_DEVSTAT_TIMEOUT = 1 << 4
 MOE_PATH_SMALL_BATCH = 1
 MOE_PATH_TENSOR_CORE = 2
 MOE_PATH_LARGE_STREAMING = 3
+MOE_PATH_FUSED_STACK = 4
+MOE_PATH_PER_LAYER = 5
 
 MOE_STAGE_ROUTE, MOE_STAGE_GATE_UP, MOE_STAGE_DOWN, MOE_STAGE_COMBINE = range(4)
 MOE_NUM_STAGES = 4
@@ -57,7 +62,8 @@ STAGE_NAMES = ("route", "gate_up", "down", "combine")
 # Every function declared in include/moe_int4.h.
 EXPORTED_SYMBOLS = ("moe_layer_workspace_bytes", "moe_layer_forward", "moe_status_str",
                     "moe_abi_version", "moe_decode_max_tokens", "moe_layer_forward_static_ws",
-                    "moe_layer_kernel_launches", "moe_layer_path", "moe_layer_workspace_bytes_upto")
+                    "moe_layer_kernel_launches", "moe_layer_path", "moe_layer_workspace_bytes_upto",
+                    "moe_stack_workspace_bytes", "moe_stack_path", "moe_stack_forward")
 
 # Scratch capacity of moe_layer_forward_static_ws (the entry point for callers
 # that cannot allocate device memory).
@@ -84,6 +90,13 @@ class moe_shared_weights_t(ctypes.Structure):
                 ("w2", ctypes.c_void_p), ("s2", ctypes.c_void_p)]
 
 
+class moe_stack_weights_t(ctypes.Structure):
+    _fields_ = [("router_w", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
+                ("w13", ctypes.c_void_p), ("s13", ctypes.c_void_p),
+                ("w2", ctypes.c_void_p), ("s2", ctypes.c_void_p),
+                ("shared", moe_shared_weights_t)]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is not built; run `python int4_expert_ffn_sigmoid_b200/_build.py`")
@@ -108,6 +121,13 @@ def _load() -> ctypes.CDLL:
     L.moe_layer_kernel_launches.restype = ctypes.c_int32
     L.moe_layer_path.argtypes = [ctypes.POINTER(moe_cfg_t), ctypes.c_int32]
     L.moe_layer_path.restype = ctypes.c_int32
+    L.moe_stack_workspace_bytes.argtypes = [ctypes.POINTER(moe_cfg_t), ctypes.c_int32, ctypes.c_int32]
+    L.moe_stack_workspace_bytes.restype = ctypes.c_size_t
+    L.moe_stack_path.argtypes = [ctypes.POINTER(moe_cfg_t), ctypes.c_int32, ctypes.c_int32]
+    L.moe_stack_path.restype = ctypes.c_int32
+    L.moe_stack_forward.argtypes = [vp, ctypes.POINTER(moe_stack_weights_t), ctypes.c_int32, vp, ctypes.c_int32,
+                                    ctypes.POINTER(moe_cfg_t), vp]
+    L.moe_stack_forward.restype = ctypes.c_int
     if L.moe_abi_version() != 1:
         raise ImportError("libmoe_int4.so ABI version mismatch")
     return L
@@ -234,6 +254,77 @@ def layer_forward(x: torch.Tensor, layer: dict, shape, out: Optional[torch.Tenso
     if st != MOE_OK:
         raise MoeError(st)
     return out
+
+
+STACK_KEYS = ("router_w", "router_bias", "w13", "s13", "w2", "s2", "sh_w13", "sh_s13", "sh_w2", "sh_s2")
+
+
+def stack_layers(layers) -> dict:
+    """Stacks per-layer weight dicts (``workloads.make_layer``'s layout) along a
+    new leading layer dimension: the layout moe_stack_forward reads."""
+    keys = [k for k in STACK_KEYS if k in layers[0]]
+    return {k: torch.stack([l[k] for l in layers]).contiguous() for k in keys}
+
+
+def stack_workspace_bytes(shape, T: int, L: int, flags: int = 0) -> int:
+    c = make_cfg(shape, flags)
+    return int(lib.moe_stack_workspace_bytes(ctypes.byref(c), int(T), int(L)))
+
+
+def stack_path(shape, T: int, L: int, flags: int = 0) -> int:
+    """MOE_PATH_FUSED_STACK or MOE_PATH_PER_LAYER of a stack_forward call (0: invalid)."""
+    c = make_cfg(shape, flags)
+    return int(lib.moe_stack_path(ctypes.byref(c), int(T), int(L)))
+
+
+def stack_forward(x: torch.Tensor, stacked: dict, shape, outs: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, flags: int = 0,
+                  topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Call ``moe_stack_forward`` on torch tensors: ``stacked`` holds the
+    weights of L layers stacked along dimension 0 (see ``stack_layers``).
+    Returns ``outs`` (bf16 [L, T, H]; outs[l] is layer l's output).
+    ``topk_idx`` / ``topk_w``: optional [L, T, K]."""
+    T = x.shape[0]
+    H, E, K, I, Is = shape.H, shape.E, shape.K, shape.I, shape.Is
+    L = stacked["router_w"].shape[0]
+    _check_dev("x", x, torch.bfloat16, (T, H))
+    _check_dev("router_w", stacked["router_w"], torch.float32, (L, E, H))
+    _check_dev("router_bias", stacked["router_bias"], torch.float32, (L, E))
+    _check_dev("w13", stacked["w13"], torch.uint8, (L, E, 2 * I, H // 2))
+    _check_dev("s13", stacked["s13"], torch.float32, (L, E, 2 * I))
+    _check_dev("w2", stacked["w2"], torch.uint8, (L, E, H, I // 2))
+    _check_dev("s2", stacked["s2"], torch.float32, (L, E, H))
+    w = moe_stack_weights_t()
+    w.router_w, w.router_bias = stacked["router_w"].data_ptr(), stacked["router_bias"].data_ptr()
+    w.w13, w.s13 = stacked["w13"].data_ptr(), stacked["s13"].data_ptr()
+    w.w2, w.s2 = stacked["w2"].data_ptr(), stacked["s2"].data_ptr()
+    if Is > 0:
+        _check_dev("sh_w13", stacked["sh_w13"], torch.uint8, (L, 2 * Is, H // 2))
+        _check_dev("sh_s13", stacked["sh_s13"], torch.float32, (L, 2 * Is))
+        _check_dev("sh_w2", stacked["sh_w2"], torch.uint8, (L, H, Is // 2))
+        _check_dev("sh_s2", stacked["sh_s2"], torch.float32, (L, H))
+        w.shared.w13, w.shared.s13 = stacked["sh_w13"].data_ptr(), stacked["sh_s13"].data_ptr()
+        w.shared.w2, w.shared.s2 = stacked["sh_w2"].data_ptr(), stacked["sh_s2"].data_ptr()
+    if outs is None:
+        outs = torch.empty((L, T, H), dtype=torch.bfloat16, device=x.device)
+    _check_dev("outs", outs, torch.bfloat16, (L, T, H))
+    if workspace is None:
+        n = stack_workspace_bytes(shape, T, L, flags)
+        if n == 0:
+            raise MoeError(MOE_ERR_UNSUPPORTED, "moe_stack_workspace_bytes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=x.device)
+    if topk_idx is not None:
+        _check_dev("topk_idx", topk_idx, torch.int32, (L, T, K))
+    if topk_w is not None:
+        _check_dev("topk_w", topk_w, torch.float32, (L, T, K))
+    cfg = make_cfg(shape, flags, workspace, topk_idx, topk_w)
+    s = stream if stream is not None else torch.cuda.current_stream(x.device)
+    st = lib.moe_stack_forward(_ptr(x), ctypes.byref(w), int(L), _ptr(outs), int(T), ctypes.byref(cfg),
+                               ctypes.c_void_p(s.cuda_stream))
+    if st != MOE_OK:
+        raise MoeError(st, "moe_stack_forward")
+    return outs
 
 
 def device_status(workspace: torch.Tensor) -> int:

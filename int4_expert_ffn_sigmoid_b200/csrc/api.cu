@@ -4,6 +4,7 @@
 #include <string.h>
 
 #include "moe_common.cuh"
+#include "moe_fused.h"
 #include "moe_int4.h"
 #include "moe_launch.h"
 #include "moe_tc.h"
@@ -13,8 +14,10 @@ namespace {
 using namespace moe;
 
 constexpr unsigned kKnownFlags =
-    MOE_ADD_RESIDUAL | MOE_DEBUG_CHECK | MOE_FORCE_DECODE | MOE_FORCE_PREFILL | MOE_OUT_F32 | MOE_TEST_STALL;
-static_assert(kFlagResidual == MOE_ADD_RESIDUAL && kFlagOutF32 == MOE_OUT_F32 && kFlagTestStall == MOE_TEST_STALL,
+    MOE_ADD_RESIDUAL | MOE_DEBUG_CHECK | MOE_FORCE_DECODE | MOE_FORCE_PREFILL | MOE_OUT_F32 | MOE_TEST_STALL |
+    MOE_NO_LOOKAHEAD;
+static_assert(kFlagResidual == MOE_ADD_RESIDUAL && kFlagOutF32 == MOE_OUT_F32 && kFlagTestStall == MOE_TEST_STALL &&
+                  kFlagNoLookahead == MOE_NO_LOOKAHEAD,
               "kernel flag bits match the C ABI");
 static_assert(ST_BAD_EXPERT == MOE_DEVSTAT_BAD_EXPERT && ST_BAD_SLOT == MOE_DEVSTAT_BAD_SLOT &&
                   ST_BAD_COUNT == MOE_DEVSTAT_BAD_COUNT && ST_BAD_TASK == MOE_DEVSTAT_BAD_TASK &&
@@ -127,6 +130,66 @@ int sm_count() {
 }
 
 inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// Whether a stack call takes the fused kernel.
+bool stack_fused(const moe_cfg_t& c, int32_t T, int32_t L) {
+    if (c.flags & (MOE_FORCE_DECODE | MOE_FORCE_PREFILL)) return false;
+    return fused_supported(c.H, c.E, c.K, c.I, c.Is, T, L) && fused_grid() > 0;
+}
+
+// Workspace of the fused kernel: a zeroed control block and counters, then
+// the data regions (see FArgs).
+struct FusedLayout {
+    size_t ctrl, grp_cnt, groups_done, down_done, ready, pred_bits, act_bits, counters_end;
+    size_t lp, lpn, idx, wts, xq, xs, h32_r, h32_s, hmax_r, hmax_s, y, total;
+};
+
+FusedLayout fused_layout(const moe_cfg_t& c, int32_t T, int32_t L) {
+    FusedLayout F{};
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t r = o;
+        o = align256(o + bytes);
+        return r;
+    };
+    auto take4 = [&](size_t n) {  // counters: packed, 4-byte aligned
+        const size_t r = o;
+        o += n * 4;
+        return r;
+    };
+    const size_t TK = (size_t)T * c.K, H = c.H, Ls = (size_t)L;
+    F.ctrl = take(256);
+    F.grp_cnt = take4(Ls * kMaxGroupsF);
+    F.groups_done = take4(Ls);
+    F.down_done = take4(Ls);
+    F.ready = take4(Ls * (kMaxE + 1));
+    F.pred_bits = take4(Ls * 8);
+    F.act_bits = take4(Ls * 8);
+    F.counters_end = o;
+    o = align256(o);
+    const size_t ncb = H / 128;
+    F.lp = take(ncb * T * c.E * 4);
+    F.lpn = take(ncb * T * c.E * 4);
+    F.idx = take(TK * 4);
+    F.wts = take(TK * 4);
+    F.xq = take((size_t)T * 2 * H);
+    F.xs = take((size_t)T * 4);
+    F.h32_r = take(TK * c.I * 4);
+    F.h32_s = take((size_t)T * c.Is * 4);
+    F.hmax_r = take(TK * (c.I / 64) * 4);
+    F.hmax_s = take((size_t)T * (c.Is / 64) * 4);
+    F.y = take((TK * slices_of(c.I) + (c.Is > 0 ? (size_t)T * slices_of(c.Is) : 0)) * H * 4);
+    F.total = o;
+    return F;
+}
+
+int validate_stack(const moe_cfg_t* cfg, int32_t T, int32_t L) {
+    const int st = validate_cfg(cfg);
+    if (st != MOE_OK) return st;
+    if (T < 0 || T > kMaxTokens || L < 1 || L > kMaxFusedLayers) return MOE_ERR_INVALID_ARG;
+    if (cfg->flags & MOE_OUT_F32) return MOE_ERR_INVALID_ARG;  // outputs feed the next layer: bf16
+    return MOE_OK;
+}
 
 }  // namespace
 
@@ -338,6 +401,118 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
     if (cfg->flags & MOE_DEBUG_CHECK) {
         unsigned status = 0;
         err = cudaMemcpyAsync(&status, &p.ctrl->status, sizeof status, cudaMemcpyDeviceToHost, s);
+        if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+        if (err != cudaSuccess) return MOE_ERR_CUDA;
+        if (status != 0) return MOE_ERR_DEVICE_CHECK;
+    }
+    return MOE_OK;
+}
+
+size_t moe_stack_workspace_bytes(const moe_cfg_t* cfg, int32_t T, int32_t L) {
+    if (validate_stack(cfg, T, L) != MOE_OK) return 0;
+    if (T > 0 && stack_fused(*cfg, T, L)) return fused_layout(*cfg, T, L).total;
+    return ws_layout(*cfg, T).total;
+}
+
+int32_t moe_stack_path(const moe_cfg_t* cfg, int32_t T, int32_t L) {
+    if (validate_stack(cfg, T, L) != MOE_OK || T <= 0) return 0;
+    return stack_fused(*cfg, T, L) ? MOE_PATH_FUSED_STACK : MOE_PATH_PER_LAYER;
+}
+
+int moe_stack_forward(const void* x, const moe_stack_weights_t* w, int32_t L, void* outs, int32_t T,
+                      const moe_cfg_t* cfg, void* stream) {
+    int st = validate_stack(cfg, T, L);
+    if (st != MOE_OK) return st;
+    if (!x || !w || !outs || !w->router_w || !w->router_bias || !w->w13 || !w->s13 || !w->w2 || !w->s2)
+        return MOE_ERR_INVALID_ARG;
+    const moe_shared_weights_t& shw = w->shared;
+    if (cfg->Is > 0 && (!shw.w13 || !shw.s13 || !shw.w2 || !shw.s2)) return MOE_ERR_INVALID_ARG;
+    const void* ptrs[] = {x, outs, w->router_w, w->router_bias, w->w13, w->s13, w->w2, w->s2,
+                          cfg->Is > 0 ? shw.w13 : nullptr, cfg->Is > 0 ? shw.s13 : nullptr,
+                          cfg->Is > 0 ? shw.w2 : nullptr, cfg->Is > 0 ? shw.s2 : nullptr,
+                          cfg->topk_idx_out, cfg->topk_w_out};
+    for (const void* ptr : ptrs)
+        if (ptr && !aligned(ptr, 16)) return MOE_ERR_INVALID_ARG;
+    const size_t H = cfg->H, E = cfg->E, I = cfg->I, Is = cfg->Is;
+    const size_t xbytes = (size_t)T * H * 2, obytes = xbytes * L;
+    const uintptr_t xa = (uintptr_t)x, oa = (uintptr_t)outs;
+    if (T > 0 && xa < oa + obytes && oa < xa + xbytes) return MOE_ERR_INVALID_ARG;
+    const size_t need = moe_stack_workspace_bytes(cfg, T, L);
+    if (!cfg->workspace || cfg->workspace_bytes < need) return MOE_ERR_WORKSPACE;
+    if (!aligned(cfg->workspace, 256)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t TK = (size_t)T * cfg->K;
+    if (!stack_fused(*cfg, T, L)) {
+        // one moe_layer_forward call per layer, each layer's output the next one's input
+        for (int32_t l = 0; l < L; ++l) {
+            moe_cfg_t c = *cfg;
+            c.flags &= ~(unsigned)MOE_NO_LOOKAHEAD;
+            c.topk_idx_out = cfg->topk_idx_out ? cfg->topk_idx_out + l * TK : nullptr;
+            c.topk_w_out = cfg->topk_w_out ? cfg->topk_w_out + l * TK : nullptr;
+            c.stage_events = nullptr;
+            moe_shared_weights_t sl{};
+            if (Is > 0) {
+                sl.w13 = shw.w13 + l * 2 * Is * (H / 2);
+                sl.s13 = shw.s13 + l * 2 * Is;
+                sl.w2 = shw.w2 + l * H * (Is / 2);
+                sl.s2 = shw.s2 + l * H;
+            }
+            const void* in = l == 0 ? x : static_cast<const char*>(outs) + (size_t)(l - 1) * xbytes;
+            void* out = static_cast<char*>(outs) + (size_t)l * xbytes;
+            st = moe_layer_forward(in, w->router_w + l * E * H, w->router_bias + l * E, w->w13 + l * E * 2 * I * (H / 2),
+                                   w->s13 + l * E * 2 * I, w->w2 + l * E * H * (I / 2), w->s2 + l * E * H, &sl, out, T,
+                                   &c, stream);
+            if (st != MOE_OK) return st;
+        }
+        return MOE_OK;
+    }
+    const FusedLayout F = fused_layout(*cfg, T, L);
+    char* ws = static_cast<char*>(cfg->workspace);
+    FArgs a;
+    memset(&a, 0, sizeof a);
+    a.T = T; a.H = cfg->H; a.E = cfg->E; a.K = cfg->K; a.I = cfg->I; a.Is = cfg->Is; a.L = L;
+    a.G = cdiv(T, 8);
+    a.NCB = cfg->H / 128;
+    a.rows2 = fused_rows2(cfg->H, cfg->E, cfg->K, cfg->I, cfg->Is, T, fused_grid());
+    a.nsl_r = slices_of(cfg->I);
+    a.nsl_s = cfg->Is > 0 ? slices_of(cfg->Is) : 0;
+    a.scale = cfg->routed_scaling;
+    a.flags = cfg->flags;
+    a.x = static_cast<const __nv_bfloat16*>(x);
+    a.outs = static_cast<__nv_bfloat16*>(outs);
+    a.rw = w->router_w; a.rb = w->router_bias;
+    a.w13 = w->w13; a.s13 = w->s13; a.w2 = w->w2; a.s2 = w->s2;
+    if (cfg->Is > 0) {
+        a.sh_w13 = shw.w13; a.sh_s13 = shw.s13; a.sh_w2 = shw.w2; a.sh_s2 = shw.s2;
+    }
+    a.topk_idx = cfg->topk_idx_out;
+    a.topk_w = cfg->topk_w_out;
+    a.status = reinterpret_cast<unsigned*>(ws + F.ctrl);
+    a.abort = reinterpret_cast<int*>(ws + F.ctrl + 4);
+    a.grp_cnt = reinterpret_cast<int*>(ws + F.grp_cnt);
+    a.groups_done = reinterpret_cast<int*>(ws + F.groups_done);
+    a.down_done = reinterpret_cast<int*>(ws + F.down_done);
+    a.ready = reinterpret_cast<int*>(ws + F.ready);
+    a.pred_bits = reinterpret_cast<unsigned*>(ws + F.pred_bits);
+    a.act_bits = reinterpret_cast<unsigned*>(ws + F.act_bits);
+    a.lp = reinterpret_cast<float*>(ws + F.lp);
+    a.lpn = reinterpret_cast<float*>(ws + F.lpn);
+    a.idx = reinterpret_cast<int32_t*>(ws + F.idx);
+    a.wts = reinterpret_cast<float*>(ws + F.wts);
+    a.xq = reinterpret_cast<int8_t*>(ws + F.xq);
+    a.xs = reinterpret_cast<float*>(ws + F.xs);
+    a.h32_r = reinterpret_cast<float*>(ws + F.h32_r);
+    a.h32_s = reinterpret_cast<float*>(ws + F.h32_s);
+    a.hmax_r = reinterpret_cast<float*>(ws + F.hmax_r);
+    a.hmax_s = reinterpret_cast<float*>(ws + F.hmax_s);
+    a.y = reinterpret_cast<float*>(ws + F.y);
+    cudaError_t err = cudaMemsetAsync(ws, 0, F.counters_end, s);
+    if (err == cudaSuccess) err = launch_decode_stack(a, fused_grid(), s);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    if (cfg->flags & MOE_DEBUG_CHECK) {
+        unsigned status = 0;
+        err = cudaMemcpyAsync(&status, a.status, sizeof status, cudaMemcpyDeviceToHost, s);
         if (err == cudaSuccess) err = cudaStreamSynchronize(s);
         if (err != cudaSuccess) return MOE_ERR_CUDA;
         if (status != 0) return MOE_ERR_DEVICE_CHECK;

@@ -91,8 +91,9 @@ WORKLOADS: Dict[str, Workload] = {
     w.name: w for w in [
         Workload("nano_layer_t16", 0, NANO, 1, (16,), "uniform", False,
                  "one Nano MoE layer, T=16"),
-        Workload("nano_decode_stack", 1, NANO, 23, (1, 4, 16, 64), "uniform", True,
-                 "23 stacked Nano MoE layers with residual, decode T in {1,4,16,64}"),
+        Workload("nano_decode_stack", 1, NANO, 23, (1, 2, 3, 4, 16, 64), "uniform", True,
+                 "23 stacked Nano MoE layers with residual, decode T in {1,4,16,64} and "
+                 "speculative-verify T in {2,3,4}"),
         Workload("nano_prefill_t4096", 2, NANO, 1, (4096,), "zero", False,
                  "one Nano MoE layer, T=4096, zero router bias (balanced loads)"),
         Workload("nano_zipf_t16384", 3, NANO, 1, (16384,), "zipf", False,
