@@ -70,6 +70,8 @@ def parse_args():
     ap.add_argument("--per-layer", action="store_true",
                     help="time the stack as one moe_layer_forward call per layer instead of the fused kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--trace", action="store_true",
+                    help="add the fused kernel's per-phase timeline (MOE_TRACE stamps) to the line")
     return ap.parse_args()
 
 
@@ -270,10 +272,14 @@ class Runner:
             self.moe.stack_forward(inp, self.stacked, self.shape, outs=self.outs, workspace=self.ws, flags=self.flags,
                                    topk_idx=topk_idx)
         else:
+            # a per-layer slice of [L][T][K] need not be 16-byte aligned: one [T][K] buffer per call
+            one = None if topk_idx is None else torch.empty_like(topk_idx[0])
             for l, layer in enumerate(self.layers):
                 ev = None if stage_events is None else stage_events[l]
                 self.moe.layer_forward(inp, layer, self.shape, out=self.outs[l], workspace=self.ws, flags=self.flags,
-                                       stage_events=ev, topk_idx=None if topk_idx is None else topk_idx[l])
+                                       stage_events=ev, topk_idx=one)
+                if one is not None:
+                    topk_idx[l].copy_(one)
                 inp = self.outs[l]
         return self.outs[self.L - 1]
 
@@ -530,6 +536,46 @@ def job_throughput(world, tokens_per_step, steps, total_ms):
     return world * tokens_per_step * steps / (total_ms / 1e3)
 
 
+def phase_trace(moe, runner):
+    """One traced call of the fused kernel: per layer, the critical path split
+    into the router part (the last CTA done with the previous layer's down
+    tasks -> every token group selected) and the expert part (selected -> the
+    last CTA done with this layer's down tasks), and per phase the median over
+    the CTAs of its duration; medians over the layers, in microseconds."""
+    T, L, shape = runner.T, runner.L, runner.shape
+    flags = runner.flags | moe.MOE_TRACE
+    ws = torch.empty(moe.stack_workspace_bytes(shape, T, L, flags), dtype=torch.uint8, device=runner.device)
+    moe.stack_forward(runner.xs[0], runner.stacked, shape, outs=runner.outs, workspace=ws, flags=flags)
+    torch.cuda.synchronize()
+    grid = torch.cuda.get_device_properties(runner.device).multi_processor_count
+    st = moe.stack_trace(ws, shape, T, L, flags, grid).double() / 1e3  # us
+    med = lambda v: float(torch.median(v))
+    rows = {k: [] for k in ("router_critical", "experts_critical", "layer", "units_wait", "units_work",
+                            "groups_wait", "tables", "gate_up", "down")}
+    G = -(-T // 8)
+    U = G * (shape.H // 128)
+    unit_ctas = torch.arange(grid - min(U, grid), grid)
+    for l in range(L):
+        s = st[:, l]
+        prev_end = st[:, l - 1, 6].max() if l > 0 else st[:, 0, 0].min()
+        sel = s[:, 3].min()
+        end = s[:, 6].max()
+        rows["router_critical"].append(float(sel - prev_end))
+        rows["experts_critical"].append(float(end - sel))
+        rows["layer"].append(float(end - prev_end))
+        u = s[unit_ctas]
+        rows["units_wait"].append(med(u[:, 1] - u[:, 0]))
+        rows["units_work"].append(med(u[:, 2] - u[:, 1]))
+        rows["groups_wait"].append(med(s[:, 3] - s[:, 2]))
+        rows["tables"].append(med(s[:, 4] - s[:, 3]))
+        rows["gate_up"].append(med(s[:, 5] - s[:, 4]))
+        rows["down"].append(med(s[:, 6] - s[:, 5]))
+    out = {k: round(statistics.median(v), 2) for k, v in rows.items()}
+    out["total_us"] = round(float(st[:, L, 2].max() - st[:, 0, 0].min()), 1)
+    out["note"] = "one traced call (L2 not flushed before it); medians over layers of per-layer spans, us"
+    return out
+
+
 def dist_or_none(world, dist):
     return dist if world > 1 else None
 
@@ -670,6 +716,8 @@ def run_ours(args, rank, world, device, dist):
                                captured_traffic(wl.name, T, kname))
         stages = {names[k]: round(stage_mean[k] * 1e3, 2) for k in range(4)}
 
+    trace = phase_trace(moe, runner) if (args.trace and fused) else None
+
     sweep = {}
     if wl.name == "nano_decode_stack" and not args.no_sweep:
         for Ts in wl.tokens:
@@ -732,6 +780,7 @@ def run_ours(args, rank, world, device, dist):
         "gpu_launches": runner.launches_per_step() * args.steps,
         "clocks": m["clocks"],
         "sweep": sweep or None,
+        "trace": trace,
         "workloads": extra,
     }
     return line

@@ -76,6 +76,18 @@ extern "C" {
                                        undefined; with MOE_DEBUG_CHECK the call returns
                                        MOE_ERR_DEVICE_CHECK.  The next call runs normally. */
 
+#define MOE_TEST_BAD_INDEX (1u << 7) /* test only: the router writes expert index E (out of range)
+                                       for token 0's first pick; the kernels' range checks must
+                                       catch it (MOE_DEVSTAT_BAD_EXPERT) without an out-of-range
+                                       access.  The output is then undefined. */
+#define MOE_TRACE (1u << 8)         /* moe_stack_forward, fused kernel: stamp each CTA's phases
+                                       with the GPU's nanosecond timer into the workspace (see
+                                       moe_stack_trace_offset); the output is unchanged */
+#define MOE_DEBUG_POISON (1u << 9)  /* fill the workspace (past the fused kernel's counters) with
+                                       0xFF bytes before the kernels run: a kernel that read scratch
+                                       it had not written would see NaN / -1; the output must not
+                                       change */
+
 /* Device status word: the first 4 bytes of the workspace hold the OR of these
  * bits after a call completes on the device (0 = no check failed).  Under
  * MOE_DEBUG_CHECK a non-zero word makes the call return MOE_ERR_DEVICE_CHECK. */
@@ -279,6 +291,15 @@ typedef struct moe_stack_weights {
 
 /* Workspace bytes of moe_stack_forward for T tokens and L layers (0: invalid). */
 size_t moe_stack_workspace_bytes(const moe_cfg_t* cfg, int32_t T, int32_t L);
+
+/* MOE_TRACE on the fused path: byte offset in the workspace of the trace,
+ * an array [grid][L+1][8] of uint64 %globaltimer stamps (ns) written by each
+ * CTA (grid = the number of SMs) at: 0 entering a layer's router phase, 1 the
+ * previous layer's down tasks all done, 2 its router units done, 3 every token
+ * group of the layer selected, 4 the layer's tables built, 5 its gate/up tasks
+ * done, 6 its down tasks done (7 unused; row L holds the final combine's 0-2).
+ * Returns 0 when the call would not trace (no MOE_TRACE, or not fused). */
+size_t moe_stack_trace_offset(const moe_cfg_t* cfg, int32_t T, int32_t L);
 
 /* MOE_PATH_FUSED_STACK or MOE_PATH_PER_LAYER for T tokens and L layers, or 0
  * if T = 0 or the call would be rejected. */

@@ -19,7 +19,8 @@ import torch
 __all__ = [
     "MoeError", "moe_cfg_t", "moe_shared_weights_t", "lib", "EXPORTED_SYMBOLS",
     "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK", "MOE_FORCE_DECODE", "MOE_FORCE_PREFILL", "MOE_OUT_F32",
-    "MOE_TEST_STALL", "MOE_NO_LOOKAHEAD", "MOE_DEVSTAT_TIMEOUT", "device_status",
+    "MOE_TEST_STALL", "MOE_NO_LOOKAHEAD", "MOE_TEST_BAD_INDEX", "MOE_TRACE", "MOE_DEBUG_POISON",
+    "MOE_DEVSTAT_TIMEOUT", "MOE_DEVSTAT_BAD_EXPERT", "device_status", "stack_trace",
     "moe_stack_weights_t", "stack_workspace_bytes", "stack_path", "stack_forward", "stack_layers",
     "MOE_PATH_FUSED_STACK", "MOE_PATH_PER_LAYER",
     "workspace_bytes", "workspace_bytes_upto", "layer_forward", "MoELayer", "decode_max_tokens", "kernel_launches", "layer_path",
@@ -42,6 +43,9 @@ MOE_FORCE_PREFILL = 1 << 3
 MOE_OUT_F32 = 1 << 4
 MOE_NO_LOOKAHEAD = 1 << 5
 MOE_TEST_STALL = 1 << 6
+MOE_TEST_BAD_INDEX = 1 << 7
+MOE_TRACE = 1 << 8
+MOE_DEBUG_POISON = 1 << 9
 # device status word (the first 4 bytes of the workspace)
 MOE_DEVSTAT_BAD_EXPERT = 1 << 0
 MOE_DEVSTAT_BAD_SLOT = 1 << 1
@@ -63,7 +67,7 @@ STAGE_NAMES = ("route", "gate_up", "down", "combine")
 EXPORTED_SYMBOLS = ("moe_layer_workspace_bytes", "moe_layer_forward", "moe_status_str",
                     "moe_abi_version", "moe_decode_max_tokens", "moe_layer_forward_static_ws",
                     "moe_layer_kernel_launches", "moe_layer_path", "moe_layer_workspace_bytes_upto",
-                    "moe_stack_workspace_bytes", "moe_stack_path", "moe_stack_forward")
+                    "moe_stack_workspace_bytes", "moe_stack_path", "moe_stack_forward", "moe_stack_trace_offset")
 
 # Scratch capacity of moe_layer_forward_static_ws (the entry point for callers
 # that cannot allocate device memory).
@@ -128,6 +132,8 @@ def _load() -> ctypes.CDLL:
     L.moe_stack_forward.argtypes = [vp, ctypes.POINTER(moe_stack_weights_t), ctypes.c_int32, vp, ctypes.c_int32,
                                     ctypes.POINTER(moe_cfg_t), vp]
     L.moe_stack_forward.restype = ctypes.c_int
+    L.moe_stack_trace_offset.argtypes = [ctypes.POINTER(moe_cfg_t), ctypes.c_int32, ctypes.c_int32]
+    L.moe_stack_trace_offset.restype = ctypes.c_size_t
     if L.moe_abi_version() != 1:
         raise ImportError("libmoe_int4.so ABI version mismatch")
     return L
@@ -325,6 +331,18 @@ def stack_forward(x: torch.Tensor, stacked: dict, shape, outs: Optional[torch.Te
     if st != MOE_OK:
         raise MoeError(st, "moe_stack_forward")
     return outs
+
+
+def stack_trace(workspace: torch.Tensor, shape, T: int, L: int, flags: int, grid: int) -> torch.Tensor:
+    """The MOE_TRACE stamps of the last fused call on ``workspace``: int64
+    [grid, L + 1, 8] nanosecond timer values (see moe_stack_trace_offset).
+    Synchronises the stream."""
+    c = make_cfg(shape, flags | MOE_TRACE)
+    off = int(lib.moe_stack_trace_offset(ctypes.byref(c), int(T), int(L)))
+    if off == 0:
+        raise ValueError("this call does not trace (not the fused kernel, or no MOE_TRACE)")
+    n = grid * (L + 1) * 8
+    return workspace[off:off + 8 * n].view(torch.int64).view(grid, L + 1, 8).cpu()
 
 
 def device_status(workspace: torch.Tensor) -> int:

@@ -13,11 +13,14 @@ namespace {
 
 using namespace moe;
 
-constexpr unsigned kKnownFlags =
-    MOE_ADD_RESIDUAL | MOE_DEBUG_CHECK | MOE_FORCE_DECODE | MOE_FORCE_PREFILL | MOE_OUT_F32 | MOE_TEST_STALL |
-    MOE_NO_LOOKAHEAD;
+constexpr unsigned kKnownFlags = MOE_ADD_RESIDUAL | MOE_DEBUG_CHECK | MOE_FORCE_DECODE | MOE_FORCE_PREFILL |
+                                 MOE_OUT_F32 | MOE_TEST_STALL | MOE_NO_LOOKAHEAD | MOE_TEST_BAD_INDEX |
+                                 MOE_TRACE | MOE_DEBUG_POISON;
+// Traced CTAs at most (the fused kernel runs one CTA per SM).
+constexpr int kMaxGridF = 256;
 static_assert(kFlagResidual == MOE_ADD_RESIDUAL && kFlagOutF32 == MOE_OUT_F32 && kFlagTestStall == MOE_TEST_STALL &&
-                  kFlagNoLookahead == MOE_NO_LOOKAHEAD,
+                  kFlagNoLookahead == MOE_NO_LOOKAHEAD && kFlagTestBadIndex == MOE_TEST_BAD_INDEX &&
+                  kFlagTrace == MOE_TRACE,
               "kernel flag bits match the C ABI");
 static_assert(ST_BAD_EXPERT == MOE_DEVSTAT_BAD_EXPERT && ST_BAD_SLOT == MOE_DEVSTAT_BAD_SLOT &&
                   ST_BAD_COUNT == MOE_DEVSTAT_BAD_COUNT && ST_BAD_TASK == MOE_DEVSTAT_BAD_TASK &&
@@ -140,8 +143,8 @@ bool stack_fused(const moe_cfg_t& c, int32_t T, int32_t L) {
 // Workspace of the fused kernel: a zeroed control block and counters, then
 // the data regions (see FArgs).
 struct FusedLayout {
-    size_t ctrl, grp_cnt, groups_done, down_done, ready, pred_bits, act_bits, counters_end;
-    size_t lp, lpn, idx, wts, xq, xs, h32_r, h32_s, hmax_r, hmax_s, y, total;
+    size_t ctrl, grp_cnt, groups_done, down_done, ready, pred_bits, counters_end;
+    size_t lp, lpn, idx, wts, xq, xs, h32_r, h32_s, hmax_r, hmax_s, y, trace, total;
 };
 
 FusedLayout fused_layout(const moe_cfg_t& c, int32_t T, int32_t L) {
@@ -164,7 +167,6 @@ FusedLayout fused_layout(const moe_cfg_t& c, int32_t T, int32_t L) {
     F.down_done = take4(Ls);
     F.ready = take4(Ls * (kMaxE + 1));
     F.pred_bits = take4(Ls * 8);
-    F.act_bits = take4(Ls * 8);
     F.counters_end = o;
     o = align256(o);
     const size_t ncb = H / 128;
@@ -179,6 +181,7 @@ FusedLayout fused_layout(const moe_cfg_t& c, int32_t T, int32_t L) {
     F.hmax_r = take(TK * (c.I / 64) * 4);
     F.hmax_s = take((size_t)T * (c.Is / 64) * 4);
     F.y = take((TK * slices_of(c.I) + (c.Is > 0 ? (size_t)T * slices_of(c.Is) : 0)) * H * 4);
+    F.trace = (c.flags & MOE_TRACE) ? take((size_t)kMaxGridF * (Ls + 1) * kTraceSlots * 8) : 0;
     F.total = o;
     return F;
 }
@@ -375,7 +378,10 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
     auto mark = [&](int idx) -> cudaError_t {
         return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[idx]), s) : cudaSuccess;
     };
-    cudaError_t err = mark(2 * MOE_STAGE_ROUTE);
+    cudaError_t err = cudaSuccess;
+    if (cfg->flags & MOE_DEBUG_POISON)  // every byte a kernel reads must have been written first
+        err = cudaMemsetAsync(ws, 0xFF, L.total, s);
+    if (err == cudaSuccess) err = mark(2 * MOE_STAGE_ROUTE);
     if (err == cudaSuccess) err = launch_router(p, small, s);
     if (err == cudaSuccess) err = mark(2 * MOE_STAGE_ROUTE + 1);
     int tc_grid1 = 0, tc_grid2 = 0;
@@ -412,6 +418,12 @@ size_t moe_stack_workspace_bytes(const moe_cfg_t* cfg, int32_t T, int32_t L) {
     if (validate_stack(cfg, T, L) != MOE_OK) return 0;
     if (T > 0 && stack_fused(*cfg, T, L)) return fused_layout(*cfg, T, L).total;
     return ws_layout(*cfg, T).total;
+}
+
+size_t moe_stack_trace_offset(const moe_cfg_t* cfg, int32_t T, int32_t L) {
+    if (validate_stack(cfg, T, L) != MOE_OK || T <= 0 || !(cfg->flags & MOE_TRACE) || !stack_fused(*cfg, T, L))
+        return 0;
+    return fused_layout(*cfg, T, L).trace;
 }
 
 int32_t moe_stack_path(const moe_cfg_t* cfg, int32_t T, int32_t L) {
@@ -495,7 +507,7 @@ int moe_stack_forward(const void* x, const moe_stack_weights_t* w, int32_t L, vo
     a.down_done = reinterpret_cast<int*>(ws + F.down_done);
     a.ready = reinterpret_cast<int*>(ws + F.ready);
     a.pred_bits = reinterpret_cast<unsigned*>(ws + F.pred_bits);
-    a.act_bits = reinterpret_cast<unsigned*>(ws + F.act_bits);
+    a.trace = (cfg->flags & MOE_TRACE) ? reinterpret_cast<unsigned long long*>(ws + F.trace) : nullptr;
     a.lp = reinterpret_cast<float*>(ws + F.lp);
     a.lpn = reinterpret_cast<float*>(ws + F.lpn);
     a.idx = reinterpret_cast<int32_t*>(ws + F.idx);
@@ -507,7 +519,11 @@ int moe_stack_forward(const void* x, const moe_stack_weights_t* w, int32_t L, vo
     a.hmax_r = reinterpret_cast<float*>(ws + F.hmax_r);
     a.hmax_s = reinterpret_cast<float*>(ws + F.hmax_s);
     a.y = reinterpret_cast<float*>(ws + F.y);
-    cudaError_t err = cudaMemsetAsync(ws, 0, F.counters_end, s);
+    if (fused_grid() > kMaxGridF && (cfg->flags & MOE_TRACE)) return MOE_ERR_UNSUPPORTED;
+    cudaError_t err = cudaSuccess;
+    if (cfg->flags & MOE_DEBUG_POISON)  // every byte a kernel reads must have been written first
+        err = cudaMemsetAsync(ws + F.counters_end, 0xFF, F.total - F.counters_end, s);
+    if (err == cudaSuccess) err = cudaMemsetAsync(ws, 0, F.counters_end, s);
     if (err == cudaSuccess) err = launch_decode_stack(a, fused_grid(), s);
     if (err != cudaSuccess) return MOE_ERR_CUDA;
     if (cfg->flags & MOE_DEBUG_CHECK) {

@@ -72,9 +72,15 @@ constexpr int kRawBytes = kChunk * kSliceK * 4;    // f32 h slice of a down task
 constexpr int kRsBytes = kMaxRows2 * 4;            // row scales of a down task
 constexpr int kXbStride = kColBlk + 8;             // staged x row of a router unit (bf16)
 constexpr long long kDrainCycles = 200000000LL;
-constexpr size_t kPrefetchPiece = 64 << 10;
 
-static_assert(16 * kXbStride * 2 + kMaxSlots / 32 * kMaxE <= kRawBytes, "phase A/B scratch fits the h staging");
+// Scratch of phases A and B inside the h staging area of the down tasks:
+// the staged x block of a router unit, the table build's per-chunk counts,
+// and the summed logits of a token group (this layer's and the lookahead's).
+constexpr int kScrXb = 0;
+constexpr int kScrCnt = kScrXb + 16 * kXbStride * 2;
+constexpr int kScrLog = kScrCnt + kMaxSlots / 32 * kMaxE;
+constexpr int kScrEnd = kScrLog + 2 * kGroupTok * kMaxE * 4;
+static_assert(kScrEnd <= kRawBytes, "phase A/B scratch fits the h staging");
 
 struct TaskD {
     int e, n, off, rbk, sl, tok0, nc;  // e < 0: none; e == E: the shared expert
@@ -109,30 +115,31 @@ static_assert(kSmem <= 227 * 1024, "fused decode shared memory");
 
 __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
+// MOE_TRACE: thread 0 of the consumers stamps event `slot` of layer l.
+__device__ __forceinline__ void stamp(const FArgs& a, int l, int slot) {
+    if (a.trace && threadIdx.x == 0) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        a.trace[((size_t)blockIdx.x * (a.L + 1) + l) * kTraceSlots + slot] = t;
+    }
+}
+
 __device__ __forceinline__ int ld_acquire(const int* p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
 
-__device__ __forceinline__ void prefetch_bulk_l2(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-// Prefetches bytes [0, n) of p into L2 (n a multiple of 16), pieces spread
-// over the calling lanes [lane0, lane0 + lanes).
-__device__ __forceinline__ void prefetch_range(const void* p, size_t n, int lane, int lanes) {
+// This CTA's 1/grid share of the 128-byte lines of bytes [0, n) of p, one
+// prefetch.global.L2 per line over `threads` threads (thread `tid`).  Spread
+// over every SM, the prefetches of a region cost each SM a few instructions.
+__device__ __forceinline__ void prefetch_share(const void* p, size_t n, int tid, int threads) {
+    const size_t lines = (n + 127) / 128;
+    const size_t per = (lines + gridDim.x - 1) / gridDim.x;
+    const size_t first = (size_t)blockIdx.x * per;
     const char* c = static_cast<const char*>(p);
-    for (size_t o = (size_t)lane * kPrefetchPiece; o < n; o += (size_t)lanes * kPrefetchPiece)
-        prefetch_bulk_l2(c + o, (uint32_t)(n - o < kPrefetchPiece ? n - o : kPrefetchPiece));
-}
-
-// This CTA's 1/grid share (16-byte granules) of bytes [0, n) of p.
-__device__ __forceinline__ void prefetch_share(const void* p, size_t n) {
-    const size_t per = ((n + gridDim.x - 1) / gridDim.x + 15) & ~size_t(15);
-    const size_t o = (size_t)blockIdx.x * per;
-    if (o >= n) return;
-    prefetch_range(static_cast<const char*>(p) + o, (n - o < per ? n - o : per), threadIdx.x & 31, 32);
+    for (size_t l = first + tid; l < first + per && l < lines; l += threads)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(c + l * 128));
 }
 
 // Bounded wait of thread 0 for *ctr >= target.  Gives up when the global
@@ -229,31 +236,36 @@ __device__ __forceinline__ void select_warp(const float (&L)[kMaxE / 32], const 
     my_w = lane < K ? scale * my_s / ssum : 0.f;
 }
 
-// Sum of the partial logits of token t over the hidden blocks, block 0 first.
-__device__ __forceinline__ void sum_logits(const FArgs& a, const float* part, int t, int lane,
-                                           float (&L)[kMaxE / 32]) {
+// Logits of the group's tokens t0 .. t0+nt-1 (all 256 consumer threads):
+// dst[tt * kMaxE + e] = the partial logits of (t0 + tt, e) summed over the
+// hidden blocks, block 0 first.  Loads are issued eight blocks at a time.
+__device__ __forceinline__ void sum_logits(const FArgs& a, const float* part, int t0, int nt, float* dst) {
+    const int n = nt * a.E;
+    for (int i = threadIdx.x; i < n; i += 256) {
+        const int tt = i / a.E, e = i - tt * a.E;
+        const float* src = part + (size_t)(t0 + tt) * a.E + e;
+        const size_t step = (size_t)a.T * a.E;
+        float acc = 0.f;
+        int cb = 0;
+        for (; cb + 8 <= a.NCB; cb += 8) {
+            float v[8];
 #pragma unroll
-    for (int j = 0; j < kMaxE / 32; ++j) L[j] = 0.f;
-    for (int cb = 0; cb < a.NCB; ++cb) {
-        const float* src = part + ((size_t)cb * a.T + t) * a.E;
+            for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (cb + u) * step);
 #pragma unroll
-        for (int j = 0; j < kMaxE / 32; ++j) {
-            const int e = lane + 32 * j;
-            if (e < a.E) L[j] += __ldcg(src + e);
+            for (int u = 0; u < 8; ++u) acc += v[u];
         }
+        for (; cb < a.NCB; ++cb) acc += __ldcg(src + cb * step);
+        dst[tt * kMaxE + e] = acc;
     }
 }
 
-// Starts the L2 prefetch of expert e of layer l (codes and scales), over the
-// lanes of the calling group.
-__device__ __forceinline__ void prefetch_expert(const FArgs& a, int l, int e, int lane, int lanes) {
+// This CTA's share of the L2 prefetch of expert e of layer l (codes and scales).
+__device__ __forceinline__ void prefetch_expert_share(const FArgs& a, int l, int e, int tid, int threads) {
     const size_t le = (size_t)l * a.E + e;
-    prefetch_range(a.w13 + le * (size_t)a.I * a.H, (size_t)a.I * a.H, lane, lanes);
-    prefetch_range(a.w2 + le * (size_t)a.H * (a.I / 2), (size_t)a.H * (a.I / 2), lane, lanes);
-    if (lane == 0) {
-        prefetch_bulk_l2(a.s13 + le * 2 * a.I, (uint32_t)(2 * a.I * 4));
-        prefetch_bulk_l2(a.s2 + le * a.H, (uint32_t)(a.H * 4));
-    }
+    prefetch_share(a.w13 + le * (size_t)a.I * a.H, (size_t)a.I * a.H, tid, threads);
+    prefetch_share(a.w2 + le * (size_t)a.H * (a.I / 2), (size_t)a.H * (a.I / 2), tid, threads);
+    prefetch_share(a.s13 + le * 2 * a.I, (size_t)2 * a.I * 4, tid, threads);
+    prefetch_share(a.s2 + le * a.H, (size_t)a.H * 4, tid, threads);
 }
 
 // x_l of token t as the input of layer l (the stack's input, or layer l-1's output).
@@ -266,6 +278,7 @@ __device__ void quantize_token(const FArgs& a, int l, int t, int lane) {
     const uint4* xr = reinterpret_cast<const uint4*>(layer_input(a, l) + (size_t)t * a.H);
     const int ng = a.H / 8;
     float m = 0.f;
+#pragma unroll 4
     for (int gi = lane; gi < ng; gi += 32) {
         const uint4 v = __ldcg(xr + gi);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -277,6 +290,7 @@ __device__ void quantize_token(const FArgs& a, int l, int t, int lane) {
     const QScale qs = qscale(m);
     uint2* q0 = reinterpret_cast<uint2*>(a.xq + (size_t)t * 2 * a.H);
     uint2* q1 = reinterpret_cast<uint2*>(a.xq + (size_t)t * 2 * a.H + a.H);
+#pragma unroll 4
     for (int gi = lane; gi < ng; gi += 32) {
         const uint4 v = __ldcg(xr + gi);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -868,7 +882,11 @@ __device__ bool phase_units(const FArgs& a, Sh& sh, const Smem& m, int l) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = a.G, U = G * a.NCB;
     const int first = (int)gridDim.x - 1 - (int)blockIdx.x;
-    if (first >= U) return true;
+    stamp(a, l, 0);
+    if (first >= U) {
+        stamp(a, l, 2);
+        return true;
+    }
     const bool final = l == a.L;
     const bool look = !final && l + 1 < a.L && !(a.flags & kFlagNoLookahead);
     uint16_t* xb = reinterpret_cast<uint16_t*>(m.raw);
@@ -888,6 +906,7 @@ __device__ bool phase_units(const FArgs& a, Sh& sh, const Smem& m, int l) {
         consumers_sync();
         if (!sh.bcast) return false;
     }
+    stamp(a, l, 1);
     for (int u = first; u < U; u += gridDim.x) {
         const int g = u / a.NCB, cb = u - g * a.NCB;
         const int t0 = g * kGroupTok, nt = min(kGroupTok, a.T - t0), col0 = cb * kColBlk;
@@ -914,13 +933,19 @@ __device__ bool phase_units(const FArgs& a, Sh& sh, const Smem& m, int l) {
         consumers_sync();
         if (!sh.last) continue;
         // the last unit of group g: select its tokens and quantize their rows
+        float* lg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(m.raw) + kScrLog);
+        sum_logits(a, a.lp, t0, nt, lg);
+        if (look) sum_logits(a, a.lpn, t0, nt, lg + kGroupTok * kMaxE);
+        consumers_sync();
         if (warp < nt) {
             const int t = t0 + warp;
             float L[kMaxE / 32];
-            sum_logits(a, a.lp, t, lane, L);
+#pragma unroll
+            for (int j = 0; j < kMaxE / 32; ++j) L[j] = lg[warp * kMaxE + lane + 32 * j];
             int e;
             float w;
             select_warp(L, a.rb + (size_t)l * a.E, a.E, a.K, a.scale, lane, e, w);
+            if ((a.flags & kFlagTestBadIndex) && t == 0 && lane == 0) e = a.E;  // test hook: an out-of-range pick
             if (lane < a.K) {
                 const size_t o = (size_t)t * a.K + lane;
                 a.idx[o] = e;
@@ -928,36 +953,15 @@ __device__ bool phase_units(const FArgs& a, Sh& sh, const Smem& m, int l) {
                 if (a.topk_idx) a.topk_idx[(size_t)l * a.T * a.K + o] = e;
                 if (a.topk_w) a.topk_w[(size_t)l * a.T * a.K + o] = w;
             }
-            if (!(a.flags & kFlagNoLookahead)) {
-                // this layer's experts, unless the previous layer's lookahead predicted them
-                const unsigned bit = 1u << (e & 31);
-                bool fetch = false;
-                if (lane < a.K && e >= 0 && e < a.E) {
-                    const bool predicted = l > 0 && (__ldcg(a.pred_bits + l * 8 + (e >> 5)) & bit);
-                    fetch = !predicted && !(atomicOr(a.act_bits + l * 8 + (e >> 5), bit) & bit);
-                }
-                unsigned todo = __ballot_sync(0xffffffffu, fetch);
-                while (todo) {
-                    const int k = __ffs(todo) - 1;
-                    todo &= todo - 1;
-                    prefetch_expert(a, l, __shfl_sync(0xffffffffu, e, k), lane, 32);
-                }
-            }
             if (look) {
-                // the next layer's router on this layer's input: its predicted experts
-                sum_logits(a, a.lpn, t, lane, L);
+                // the next layer's router on this layer's input: the experts it
+                // predicts are prefetched (by every CTA, its share) in the tables phase
+#pragma unroll
+                for (int j = 0; j < kMaxE / 32; ++j) L[j] = lg[(kGroupTok + warp) * kMaxE + lane + 32 * j];
                 int pe;
                 float pw;
                 select_warp(L, a.rb + (size_t)(l + 1) * a.E, a.E, a.K, a.scale, lane, pe, pw);
-                const unsigned bit = 1u << (pe & 31);
-                const bool fetch = lane < a.K && pe >= 0 && pe < a.E &&
-                                   !(atomicOr(a.pred_bits + (l + 1) * 8 + (pe >> 5), bit) & bit);
-                unsigned todo = __ballot_sync(0xffffffffu, fetch);
-                while (todo) {
-                    const int k = __ffs(todo) - 1;
-                    todo &= todo - 1;
-                    prefetch_expert(a, l + 1, __shfl_sync(0xffffffffu, pe, k), lane, 32);
-                }
+                if (lane < a.K && pe >= 0 && pe < a.E) atomicOr(a.pred_bits + (l + 1) * 8 + (pe >> 5), 1u << (pe & 31));
             }
             quantize_token(a, l, t, lane);
         }
@@ -967,6 +971,7 @@ __device__ bool phase_units(const FArgs& a, Sh& sh, const Smem& m, int l) {
             atomicAdd(a.groups_done + l, 1);
         }
     }
+    stamp(a, l, 2);
     return !aborted(sh);
 }
 
@@ -981,17 +986,41 @@ __device__ bool phase_tables(const FArgs& a, Sh& sh, const Smem& m, int l) {
     }
     consumers_sync();
     if (!sh.bcast) return false;
-    build_tables(a, sh, reinterpret_cast<uint8_t*>(m.raw) + 16 * kXbStride * 2);
-    // the next layer's shared expert and routers (this CTA's share) into L2
-    if (!(a.flags & kFlagNoLookahead) && l + 1 < a.L && threadIdx.x < 32) {
-        const int n1 = l + 1;
-        if (a.Is > 0) {
-            prefetch_share(a.sh_w13 + (size_t)n1 * a.Is * a.H, (size_t)a.Is * a.H);
-            prefetch_share(a.sh_w2 + (size_t)n1 * a.H * (a.Is / 2), (size_t)a.H * (a.Is / 2));
+    stamp(a, l, 3);
+    build_tables(a, sh, reinterpret_cast<uint8_t*>(m.raw) + kScrCnt);
+    if (threadIdx.x == 0) bar_arrive(&sh.tready);  // the producer may start
+    stamp(a, l, 4);
+    if (!(a.flags & kFlagNoLookahead)) {
+        // L2 prefetch, every CTA its share: this layer's selected experts that
+        // the previous layer's lookahead did not predict; the next layer's
+        // predicted experts, shared expert and router (and the router after it,
+        // which the next lookahead reads)
+        const int tid = threadIdx.x;
+        for (int b = 0; b < sh.nb; ++b) {
+            const int e = sh.be[b];
+            if (e < a.E && !(l > 0 && (__ldcg(a.pred_bits + l * 8 + (e >> 5)) >> (e & 31)) & 1u))
+                prefetch_expert_share(a, l, e, tid, 256);
         }
-        if (l + 2 < a.L) prefetch_share(a.rw + (size_t)(l + 2) * a.E * a.H, (size_t)a.E * a.H * 4);
+        if (l + 1 < a.L) {
+            const int n1 = l + 1;
+            for (int w = 0; w < (a.E + 31) / 32; ++w) {
+                unsigned bits = __ldcg(a.pred_bits + n1 * 8 + w);
+                while (bits) {
+                    const int e = 32 * w + __ffs(bits) - 1;
+                    bits &= bits - 1;
+                    prefetch_expert_share(a, n1, e, tid, 256);
+                }
+            }
+            if (a.Is > 0) {
+                prefetch_share(a.sh_w13 + (size_t)n1 * a.Is * a.H, (size_t)a.Is * a.H, tid, 256);
+                prefetch_share(a.sh_w2 + (size_t)n1 * a.H * (a.Is / 2), (size_t)a.H * (a.Is / 2), tid, 256);
+                prefetch_share(a.sh_s13 + (size_t)n1 * 2 * a.Is, (size_t)2 * a.Is * 4, tid, 256);
+                prefetch_share(a.sh_s2 + (size_t)n1 * a.H, (size_t)a.H * 4, tid, 256);
+            }
+            prefetch_share(a.rw + (size_t)n1 * a.E * a.H, (size_t)a.E * a.H * 4, tid, 256);
+            if (l + 2 < a.L) prefetch_share(a.rw + (size_t)(l + 2) * a.E * a.H, (size_t)a.E * a.H * 4, tid, 256);
+        }
     }
-    if (threadIdx.x == 0) bar_arrive(&sh.tready);
     return true;
 }
 
@@ -1064,6 +1093,7 @@ __device__ bool phase_gate_up(const FArgs& a, Sh& sh, const Smem& m, int l, uint
         }
         if (aborted(sh)) return false;
     }
+    stamp(a, l, 5);
     return true;
 }
 
@@ -1136,6 +1166,7 @@ __device__ bool phase_down(const FArgs& a, Sh& sh, const Smem& m, int l, uint32_
         if (aborted(sh)) return false;
     }
     consumers_sync();
+    stamp(a, l, 6);
     if (tid == 0) {
         __threadfence();
         atomicAdd(a.down_done + l, 1);
@@ -1180,12 +1211,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicOr(a.status, ST_TIMEOUT);
         atomicExch(a.abort, 1);
     }
-    if (!(a.flags & kFlagNoLookahead) && threadIdx.x < 32) {
+    if (!(a.flags & kFlagNoLookahead)) {
         if (a.Is > 0) {
-            prefetch_share(a.sh_w13, (size_t)a.Is * a.H);
-            prefetch_share(a.sh_w2, (size_t)a.H * (a.Is / 2));
+            prefetch_share(a.sh_w13, (size_t)a.Is * a.H, threadIdx.x, 256);
+            prefetch_share(a.sh_w2, (size_t)a.H * (a.Is / 2), threadIdx.x, 256);
         }
-        if (a.L > 1) prefetch_share(a.rw + (size_t)a.E * a.H, (size_t)a.E * a.H * 4);
+        if (a.L > 1) prefetch_share(a.rw + (size_t)a.E * a.H, (size_t)a.E * a.H * 4, threadIdx.x, 256);
     }
     uint32_t n = 0;
     bool ok = true;

@@ -53,6 +53,8 @@ constexpr unsigned kFlagResidual = 1u << 0;   // MOE_ADD_RESIDUAL
 constexpr unsigned kFlagOutF32 = 1u << 4;     // MOE_OUT_F32
 constexpr unsigned kFlagNoLookahead = 1u << 5;  // MOE_NO_LOOKAHEAD
 constexpr unsigned kFlagTestStall = 1u << 6;  // MOE_TEST_STALL
+constexpr unsigned kFlagTestBadIndex = 1u << 7;  // MOE_TEST_BAD_INDEX
+constexpr unsigned kFlagTrace = 1u << 8;      // MOE_TRACE
 
 // Device status bits (set by range checks, read back under MOE_DEBUG_CHECK).
 enum : unsigned {

@@ -11,6 +11,10 @@ namespace moe {
 // Layers of one fused call, and the token groups of its router units.
 constexpr int kMaxFusedLayers = 128;
 constexpr int kMaxGroupsF = kDecodeMaxTokens / 8;
+// MOE_TRACE: stamps per (CTA, layer): 0 phase A entered, 1 the previous
+// layer's down tasks all done, 2 phase A done, 3 every token group selected,
+// 4 tables built, 5 gate/up tasks done, 6 down tasks done, 7 unused.
+constexpr int kTraceSlots = 8;
 
 // Everything the fused kernel reads and writes.  Weights of all L layers are
 // stacked along a leading layer dimension (layer l of router_w is at
@@ -43,8 +47,8 @@ struct FArgs {
     int* groups_done;   // [L]               token groups selected
     int* down_done;     // [L]               CTAs done with the layer's down tasks
     int* ready;         // [L][kMaxE + 1]    gate/up tasks done per expert (E: the shared expert)
-    unsigned* pred_bits;  // [L][8]          experts prefetched by the lookahead (bit e)
-    unsigned* act_bits;   // [L][8]          experts prefetched after their selection
+    unsigned* pred_bits;  // [L][8]          experts predicted by the lookahead (bit e)
+    unsigned long long* trace;  // MOE_TRACE: [grid][L + 1][kTraceSlots] %globaltimer stamps, or null
     // workspace: data
     float* lp;          // [NCB][T][E] partial router logits of the current layer
     float* lpn;         // [NCB][T][E] partial logits of the next layer's router on the current input

@@ -122,6 +122,7 @@ __device__ int select_from_logits(const Params& p, int t, const float (&L)[kMaxE
         if (lane == k) { my_e = be; my_s = bs; }
         ssum += bs;
     }
+    if ((p.flags & kFlagTestBadIndex) && t == 0 && lane == 0) my_e = E;  // test hook: an out-of-range pick
     if (lane < K) {
         const float w = p.scale * my_s / ssum;
         const size_t o = (size_t)t * K + lane;

@@ -43,13 +43,17 @@ def test_struct_layout_matches_c(moe, tmp_path):
         "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(moe_cfg_t),"
         " offsetof(moe_cfg_t, routed_scaling), offsetof(moe_cfg_t, flags),"
         " offsetof(moe_cfg_t, workspace), offsetof(moe_cfg_t, workspace_bytes),"
-        " offsetof(moe_cfg_t, topk_w_out), sizeof(moe_shared_weights_t)); return 0;}\n")
+        " offsetof(moe_cfg_t, topk_w_out), sizeof(moe_shared_weights_t));"
+        " printf(\"%zu %zu %zu\\n\", sizeof(moe_stack_weights_t), offsetof(moe_stack_weights_t, s2),"
+        " offsetof(moe_stack_weights_t, shared)); return 0;}\n")
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)])
     c_vals = [int(v) for v in subprocess.check_output([str(exe)]).split()]
     cfg = moe.moe_cfg_t
     py_vals = [ctypes.sizeof(cfg), cfg.routed_scaling.offset, cfg.flags.offset, cfg.workspace.offset,
-               cfg.workspace_bytes.offset, cfg.topk_w_out.offset, ctypes.sizeof(moe.moe_shared_weights_t)]
+               cfg.workspace_bytes.offset, cfg.topk_w_out.offset, ctypes.sizeof(moe.moe_shared_weights_t),
+               ctypes.sizeof(moe.moe_stack_weights_t), moe.moe_stack_weights_t.s2.offset,
+               moe.moe_stack_weights_t.shared.offset]
     assert c_vals == py_vals
 
 
@@ -57,7 +61,9 @@ def test_header_constants_match_binding(moe):
     text = open(HEADER).read()
     for name in ("MOE_STATIC_WORKSPACE_BYTES", "MOE_OUT_F32", "MOE_FORCE_DECODE",
                  "MOE_FORCE_PREFILL", "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK",
-                 "MOE_PATH_SMALL_BATCH", "MOE_PATH_TENSOR_CORE", "MOE_PATH_LARGE_STREAMING"):
+                 "MOE_PATH_SMALL_BATCH", "MOE_PATH_TENSOR_CORE", "MOE_PATH_LARGE_STREAMING",
+                 "MOE_NO_LOOKAHEAD", "MOE_TEST_STALL", "MOE_TEST_BAD_INDEX", "MOE_TRACE", "MOE_DEBUG_POISON",
+                 "MOE_DEVSTAT_TIMEOUT", "MOE_DEVSTAT_BAD_EXPERT", "MOE_PATH_FUSED_STACK", "MOE_PATH_PER_LAYER"):
         m = re.search(rf"#define {name} (.+)", text)
         assert m, name
         expr = m.group(1).split("/*")[0].replace("(size_t)", "").replace("u", "")
@@ -174,7 +180,7 @@ def test_forward_validation_codes(moe):
     assert _call(moe, _shape(K=9, E=64)) == moe.MOE_ERR_UNSUPPORTED
     assert _call(moe, _shape(K=5, E=4)) == moe.MOE_ERR_INVALID_ARG
     assert _call(moe, _shape(routed_scaling=0.0)) == moe.MOE_ERR_INVALID_ARG
-    assert _call(moe, s, flags=1 << 7) == moe.MOE_ERR_INVALID_ARG
+    assert _call(moe, s, flags=1 << 12) == moe.MOE_ERR_INVALID_ARG  # an unknown flag
     assert _call(moe, s, flags=moe.MOE_FORCE_DECODE | moe.MOE_FORCE_PREFILL) == moe.MOE_ERR_INVALID_ARG
 
     def bad_size(c):
@@ -182,3 +188,40 @@ def test_forward_validation_codes(moe):
     assert _call(moe, s, cfg_patch=bad_size) == moe.MOE_ERR_INVALID_ARG
     assert moe.lib.moe_layer_forward(None, None, None, None, None, None, None, None, None, 0, None,
                                      None) == moe.MOE_ERR_INVALID_ARG
+
+
+def _stack_call(moe, shape, T=0, L=2, x=None, outs=None, ws=None, ws_bytes=1 << 30, flags=0, null_field=None):
+    w = moe.moe_stack_weights_t()
+    for f in ("router_w", "router_bias", "w13", "s13", "w2", "s2"):
+        setattr(w, f, FAKE)
+    w.shared.w13 = w.shared.s13 = w.shared.w2 = w.shared.s2 = FAKE
+    if null_field:
+        setattr(w, null_field, None)
+    cfg = moe.make_cfg(shape, flags)
+    cfg.workspace = FAKE * 256 if ws is None else ws
+    cfg.workspace_bytes = ws_bytes
+    vp = ctypes.c_void_p
+    return moe.lib.moe_stack_forward(vp(FAKE * 2 if x is None else x), ctypes.byref(w), L,
+                                     vp(FAKE * 64 if outs is None else outs), T, ctypes.byref(cfg), None)
+
+
+def test_stack_validation_codes(moe):
+    """moe_stack_forward checks its arguments before launching anything."""
+    s = _shape()
+    assert _stack_call(moe, s) == 0                                               # T = 0: no-op
+    assert _stack_call(moe, s, L=0) == moe.MOE_ERR_INVALID_ARG
+    assert _stack_call(moe, s, L=129) == moe.MOE_ERR_INVALID_ARG                  # more layers than supported
+    assert _stack_call(moe, s, T=-1) == moe.MOE_ERR_INVALID_ARG
+    assert _stack_call(moe, s, flags=moe.MOE_OUT_F32) == moe.MOE_ERR_INVALID_ARG  # outputs feed the next layer
+    assert _stack_call(moe, s, null_field="w2") == moe.MOE_ERR_INVALID_ARG
+    assert _stack_call(moe, s, x=FAKE * 2 + 8) == moe.MOE_ERR_INVALID_ARG         # misaligned
+    assert _stack_call(moe, s, T=4, outs=FAKE * 2) == moe.MOE_ERR_INVALID_ARG     # outs overlaps x
+    assert _stack_call(moe, s, T=4, ws_bytes=100) == moe.MOE_ERR_WORKSPACE
+    assert _stack_call(moe, s, flags=1 << 12) == moe.MOE_ERR_INVALID_ARG
+    assert moe.stack_workspace_bytes(s, 64, 23) > 0
+    assert moe.stack_workspace_bytes(s, 64, 0) == 0
+    # without a GPU the fused kernel cannot be resident: every call takes the per-layer path
+    assert moe.stack_path(s, 0, 23) == 0
+    assert moe.stack_path(s, 16, 23) in (moe.MOE_PATH_FUSED_STACK, moe.MOE_PATH_PER_LAYER)
+    assert moe.stack_path(s, 100, 23) == moe.MOE_PATH_PER_LAYER                   # beyond 64 tokens
+    assert moe.stack_path(s, 16, 23, moe.MOE_FORCE_DECODE) == moe.MOE_PATH_PER_LAYER

@@ -1,4 +1,5 @@
-"""Failure detection on the device: a bounded wait that runs out.
+"""Failure detection on the device: a bounded wait that runs out, a
+corrupted routing index, and a poisoned workspace.
 
 MOE_TEST_STALL makes one role of each expert kernel that takes part wait ~1 ms
 on a flag that nothing sets.  The kernel then takes its timeout path while its
@@ -52,3 +53,69 @@ def test_stalled_wait_reports_timeout_then_recovers(moe, cuda_device, case):
     torch.cuda.synchronize()
     assert moe.device_status(ws) == 0
     assert torch.equal(again, good), what
+
+
+# --- a corrupted routing index and a poisoned workspace --------------------------
+
+PATHS = [
+    # (description, shape, T, flags)
+    ("small-batch kernels", workloads.LayerShape(1024, 64, 2, 512, 2048, 1.0), 16, 0),
+    ("tensor-core kernels", workloads.LayerShape(512, 16, 8, 256, 384, 2.5), 130, "prefill"),
+    ("large-batch streaming kernels", workloads.LayerShape(1024, 64, 2, 512, 2048, 1.0), 150, "decode"),
+]
+
+
+def _flags(moe, f):
+    return {0: 0, "prefill": moe.MOE_FORCE_PREFILL, "decode": moe.MOE_FORCE_DECODE}[f]
+
+
+@pytest.mark.parametrize("case", range(len(PATHS)))
+def test_bad_routing_index_is_caught(moe, cuda_device, case):
+    """The router hands an out-of-range expert index to the kernels that
+    follow (MOE_TEST_BAD_INDEX); their range checks report it and nothing
+    reads or writes out of bounds: the next normal call is bit-identical."""
+    what, shape, T, f = PATHS[case]
+    base = _flags(moe, f)
+    layer = workloads.make_layer(shape, 320 + case, 0, cuda_device)
+    x = workloads.make_x(shape, T, 320 + case, device=cuda_device)
+    ws = moe.new_workspace(shape, T, cuda_device, base)
+    good = moe.layer_forward(x, layer, shape, workspace=ws, flags=base | moe.MOE_DEBUG_CHECK).clone()
+    with pytest.raises(moe.MoeError) as err:
+        moe.layer_forward(x, layer, shape, workspace=ws, flags=base | moe.MOE_TEST_BAD_INDEX | moe.MOE_DEBUG_CHECK)
+    assert err.value.status == moe.MOE_ERR_DEVICE_CHECK, what
+    assert moe.device_status(ws) & moe.MOE_DEVSTAT_BAD_EXPERT, what
+    again = moe.layer_forward(x, layer, shape, workspace=ws, flags=base | moe.MOE_DEBUG_CHECK)
+    torch.cuda.synchronize()
+    assert torch.equal(again, good), what
+
+
+@pytest.mark.parametrize("case", range(len(PATHS)))
+def test_poisoned_workspace_changes_nothing(moe, cuda_device, case):
+    """Every scratch byte the kernels read was written first in the same call:
+    filling the workspace with 0xFF (NaN / -1) beforehand changes no output bit."""
+    what, shape, T, f = PATHS[case]
+    base = _flags(moe, f)
+    layer = workloads.make_layer(shape, 330 + case, 0, cuda_device)
+    x = workloads.make_x(shape, T, 330 + case, device=cuda_device)
+    a = moe.layer_forward(x, layer, shape, flags=base | moe.MOE_DEBUG_CHECK)
+    b = moe.layer_forward(x, layer, shape, flags=base | moe.MOE_DEBUG_POISON | moe.MOE_DEBUG_CHECK)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b), what
+
+
+def test_fused_stack_bad_index_and_poison(moe, cuda_device):
+    shape = workloads.LayerShape(1024, 64, 2, 512, 2048, 1.0)
+    layers = [workloads.make_layer(shape, 340, l, cuda_device) for l in range(3)]
+    stacked = moe.stack_layers(layers)
+    x = workloads.make_x(shape, 24, 340, device=cuda_device)
+    f = moe.MOE_ADD_RESIDUAL | moe.MOE_DEBUG_CHECK
+    assert moe.stack_path(shape, 24, 3, f) == moe.MOE_PATH_FUSED_STACK
+    ws = torch.empty(moe.stack_workspace_bytes(shape, 24, 3, f), dtype=torch.uint8, device=cuda_device)
+    good = moe.stack_forward(x, stacked, shape, workspace=ws, flags=f).clone()
+    with pytest.raises(moe.MoeError) as err:
+        moe.stack_forward(x, stacked, shape, workspace=ws, flags=f | moe.MOE_TEST_BAD_INDEX)
+    assert err.value.status == moe.MOE_ERR_DEVICE_CHECK
+    assert moe.device_status(ws) & moe.MOE_DEVSTAT_BAD_EXPERT
+    poisoned = moe.stack_forward(x, stacked, shape, workspace=ws, flags=f | moe.MOE_DEBUG_POISON)
+    torch.cuda.synchronize()
+    assert torch.equal(poisoned, good)
