@@ -70,6 +70,8 @@ def parse_args():
     ap.add_argument("--per-layer", action="store_true",
                     help="time the stack as one moe_layer_forward call per layer instead of the fused kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lookahead", action="store_true",
+                    help="fused kernel with its L2 prefetch hints (MOE_LOOKAHEAD; the output is the same)")
     ap.add_argument("--trace", action="store_true",
                     help="add the fused kernel's per-phase timeline (MOE_TRACE stamps) to the line")
     return ap.parse_args()
@@ -251,7 +253,7 @@ class Runner:
     stack kernel; mode "fused") or one moe_layer_forward call per layer (mode
     "per_layer")."""
 
-    def __init__(self, moe, wl, T, device, stacked, mode):
+    def __init__(self, moe, wl, T, device, stacked, mode, extra_flags=0):
         self.moe, self.wl, self.T, self.device, self.mode = moe, wl, T, device, mode
         self.shape = wl.shape
         self.L = wl.layers
@@ -259,7 +261,7 @@ class Runner:
         self.layers = [{k: v[l] for k, v in stacked.items()} for l in range(self.L)]
         self.xs = [workloads.make_x(wl.shape, T, wl.wid, batch=b, device=device) for b in range(N_BATCHES)]
         self.outs = torch.empty((self.L, T, wl.shape.H), dtype=torch.bfloat16, device=device)
-        self.flags = moe.MOE_ADD_RESIDUAL if wl.residual else 0
+        self.flags = (moe.MOE_ADD_RESIDUAL if wl.residual else 0) | extra_flags
         if mode == "fused":
             n = moe.stack_workspace_bytes(wl.shape, T, self.L, self.flags)
             self.ws = torch.empty(n, dtype=torch.uint8, device=device)
@@ -537,42 +539,49 @@ def job_throughput(world, tokens_per_step, steps, total_ms):
 
 
 def phase_trace(moe, runner):
-    """One traced call of the fused kernel: per layer, the critical path split
-    into the router part (the last CTA done with the previous layer's down
-    tasks -> every token group selected) and the expert part (selected -> the
-    last CTA done with this layer's down tasks), and per phase the median over
-    the CTAs of its duration; medians over the layers, in microseconds."""
+    """One traced call of the fused kernel (MOE_TRACE stamps, see
+    moe_stack_trace_offset).  Per layer: the critical path split into the
+    router part (the last CTA done with the previous layer's down tasks ->
+    every token group selected) and the expert part (selected -> the last CTA
+    done with this layer's down tasks); and the steps inside them, each the
+    median over the CTAs that took both of its stamps.  Medians over the
+    layers, in microseconds."""
     T, L, shape = runner.T, runner.L, runner.shape
     flags = runner.flags | moe.MOE_TRACE
     ws = torch.empty(moe.stack_workspace_bytes(shape, T, L, flags), dtype=torch.uint8, device=runner.device)
     moe.stack_forward(runner.xs[0], runner.stacked, shape, outs=runner.outs, workspace=ws, flags=flags)
     torch.cuda.synchronize()
     grid = torch.cuda.get_device_properties(runner.device).multi_processor_count
-    st = moe.stack_trace(ws, shape, T, L, flags, grid).double() / 1e3  # us
-    med = lambda v: float(torch.median(v))
-    rows = {k: [] for k in ("router_critical", "experts_critical", "layer", "units_wait", "units_work",
-                            "groups_wait", "tables", "gate_up", "down")}
-    G = -(-T // 8)
-    U = G * (shape.H // 128)
-    unit_ctas = torch.arange(grid - min(U, grid), grid)
+    st = moe.stack_trace(ws, shape, T, L, flags, grid).double() / 1e3  # us, 0 = not taken
+
+    def span(s, a, b):
+        ok = (s[:, a] > 0) & (s[:, b] > 0)
+        return float(torch.median(s[ok, b] - s[ok, a])) if bool(ok.any()) else None
+
+    steps = {"wait_prev_down": (0, 1), "combine": (1, 7), "router_mma": (7, 8), "count": (8, 9),
+             "select": (9, 10), "quantize": (10, 11), "units_to_selected": (2, 3), "tables": (3, 4),
+             "prefetch": (4, 12), "first_stage": (12, 13), "gate_up": (4, 5), "down_ready": (5, 14),
+             "down_stage_h": (14, 15), "down": (5, 6)}
+    rows = {k: [] for k in ["router_critical", "experts_critical", "layer", "selected_seen"] + list(steps)}
     for l in range(L):
         s = st[:, l]
-        prev_end = st[:, l - 1, 6].max() if l > 0 else st[:, 0, 0].min()
-        sel = s[:, 3].min()
+        prev_end = st[:, l - 1, 6].max() if l > 0 else st[:, 0, 0][st[:, 0, 0] > 0].min()
+        sel = s[:, 3][s[:, 3] > 0].min()
         end = s[:, 6].max()
         rows["router_critical"].append(float(sel - prev_end))
         rows["experts_critical"].append(float(end - sel))
         rows["layer"].append(float(end - prev_end))
-        u = s[unit_ctas]
-        rows["units_wait"].append(med(u[:, 1] - u[:, 0]))
-        rows["units_work"].append(med(u[:, 2] - u[:, 1]))
-        rows["groups_wait"].append(med(s[:, 3] - s[:, 2]))
-        rows["tables"].append(med(s[:, 4] - s[:, 3]))
-        rows["gate_up"].append(med(s[:, 5] - s[:, 4]))
-        rows["down"].append(med(s[:, 6] - s[:, 5]))
-    out = {k: round(statistics.median(v), 2) for k, v in rows.items()}
-    out["total_us"] = round(float(st[:, L, 2].max() - st[:, 0, 0].min()), 1)
-    out["note"] = "one traced call (L2 not flushed before it); medians over layers of per-layer spans, us"
+        q = s[:, 11][s[:, 11] > 0]
+        if q.numel():
+            rows["selected_seen"].append(float(sel - q.max()))
+        for k, (a_, b_) in steps.items():
+            v = span(s, a_, b_)
+            if v is not None:
+                rows[k].append(v)
+    out = {k: round(statistics.median(v), 2) for k, v in rows.items() if v}
+    out["total_us"] = round(float(st[:, L, 2].max() - st[:, 0, 0][st[:, 0, 0] > 0].min()), 1)
+    out["note"] = ("one traced call (L2 not flushed before it); per layer, medians over the CTAs of each step's "
+                   "duration, then medians over the layers, us")
     return out
 
 
@@ -679,7 +688,8 @@ def run_ours(args, rank, world, device, dist):
     stacked = stacked_weights(moe, wl, device)
     flags = moe.MOE_ADD_RESIDUAL if wl.residual else 0
     fused = (not args.per_layer) and moe.stack_path(wl.shape, T, wl.layers, flags) == moe.MOE_PATH_FUSED_STACK
-    runner = Runner(moe, wl, T, device, stacked, "fused" if fused else "per_layer")
+    runner = Runner(moe, wl, T, device, stacked, "fused" if fused else "per_layer",
+                    moe.MOE_LOOKAHEAD if (args.lookahead and fused) else 0)
     L = wl.layers
 
     m = measure(runner, args.steps, args.warmup, use_graph, flush, peaks, device, barrier)

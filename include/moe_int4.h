@@ -63,9 +63,11 @@ extern "C" {
 #define MOE_FORCE_PREFILL (1u << 3) /* use the grouped-GEMM kernels at any T (H a multiple of 256) */
 #define MOE_OUT_F32 (1u << 4)       /* out is f32 [T][H] (the f32 sum, no bf16 rounding): for
                                        checking the arithmetic apart from the output rounding */
-#define MOE_NO_LOOKAHEAD (1u << 5)  /* moe_stack_forward: no L2 prefetch hints (the next layer's
-                                       shared expert, routers and predicted experts); the output
-                                       is bit-identical either way */
+#define MOE_LOOKAHEAD (1u << 5)     /* moe_stack_forward, fused kernel: L2 prefetch hints (the
+                                       next layer's shared expert, routers and the experts its
+                                       router picks on the current input); the output is
+                                       bit-identical either way.  Off by default: measured slower
+                                       here, the prefetches competing with the demand loads */
 #define MOE_TEST_STALL (1u << 6)    /* test only: in the expert kernels that take part (the
                                        tensor-core grouped GEMMs, the TMA-ring weight-streaming
                                        kernels and the fused stack kernel), one role first waits
@@ -262,8 +264,8 @@ int moe_layer_forward_static_ws(const void* x, const float* router_w, const floa
  * into L2 the next layer's shared expert and routers, and the experts that the
  * next layer's router picks when run on the current layer's input (the
  * cross-layer expert prediction of the nanocolibri-engine README, knobs
- * table, PREDICT; colibri README, "How it works"); MOE_NO_LOOKAHEAD turns the
- * hints off, which changes no output bit.  One cudaMemsetAsync of the
+ * table, PREDICT; colibri README, "How it works") when MOE_LOOKAHEAD is set;
+ * the hints change no output bit.  One cudaMemsetAsync of the
  * workspace's counters precedes the kernel.  The arithmetic is the
  * weight-streaming path's (see "Arithmetic" above); the router logits are
  * summed per 128-column block of the hidden dimension, so they can differ
@@ -293,11 +295,16 @@ typedef struct moe_stack_weights {
 size_t moe_stack_workspace_bytes(const moe_cfg_t* cfg, int32_t T, int32_t L);
 
 /* MOE_TRACE on the fused path: byte offset in the workspace of the trace,
- * an array [grid][L+1][8] of uint64 %globaltimer stamps (ns) written by each
- * CTA (grid = the number of SMs) at: 0 entering a layer's router phase, 1 the
- * previous layer's down tasks all done, 2 its router units done, 3 every token
- * group of the layer selected, 4 the layer's tables built, 5 its gate/up tasks
- * done, 6 its down tasks done (7 unused; row L holds the final combine's 0-2).
+ * an array [grid][L+1][16] of uint64 %globaltimer stamps (ns) written by each
+ * CTA (grid = the number of SMs; a stamp a CTA does not take stays 0) at:
+ *  0 entering a layer's router phase, 1 the previous layer's down tasks all
+ *  done, 2 its router units done, 3 every token group of the layer selected,
+ *  4 the layer's tables built, 5 its gate/up tasks done, 6 its down tasks
+ *  done; the CTA's first router unit: 7 combined, 8 partial logits written,
+ *  9 counted; the unit that completed a token group: 10 selected, 11 rows
+ *  quantized; 12 this layer's prefetches issued; 13 the first gate/up stage
+ *  landed; the first down task: 14 its expert ready, 15 its activations
+ *  staged.  Row L holds the final combine's stamps 0-2.
  * Returns 0 when the call would not trace (no MOE_TRACE, or not fused). */
 size_t moe_stack_trace_offset(const moe_cfg_t* cfg, int32_t T, int32_t L);
 

@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "MoeError", "moe_cfg_t", "moe_shared_weights_t", "lib", "EXPORTED_SYMBOLS",
     "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK", "MOE_FORCE_DECODE", "MOE_FORCE_PREFILL", "MOE_OUT_F32",
-    "MOE_TEST_STALL", "MOE_NO_LOOKAHEAD", "MOE_TEST_BAD_INDEX", "MOE_TRACE", "MOE_DEBUG_POISON",
+    "MOE_TEST_STALL", "MOE_LOOKAHEAD", "MOE_TEST_BAD_INDEX", "MOE_TRACE", "MOE_DEBUG_POISON",
     "MOE_DEVSTAT_TIMEOUT", "MOE_DEVSTAT_BAD_EXPERT", "device_status", "stack_trace",
     "moe_stack_weights_t", "stack_workspace_bytes", "stack_path", "stack_forward", "stack_layers",
     "MOE_PATH_FUSED_STACK", "MOE_PATH_PER_LAYER",
@@ -41,11 +41,12 @@ MOE_DEBUG_CHECK = 1 << 1
 MOE_FORCE_DECODE = 1 << 2
 MOE_FORCE_PREFILL = 1 << 3
 MOE_OUT_F32 = 1 << 4
-MOE_NO_LOOKAHEAD = 1 << 5
+MOE_LOOKAHEAD = 1 << 5
 MOE_TEST_STALL = 1 << 6
 MOE_TEST_BAD_INDEX = 1 << 7
 MOE_TRACE = 1 << 8
 MOE_DEBUG_POISON = 1 << 9
+TRACE_SLOTS = 16  # MOE_TRACE stamps per (CTA, layer)
 # device status word (the first 4 bytes of the workspace)
 MOE_DEVSTAT_BAD_EXPERT = 1 << 0
 MOE_DEVSTAT_BAD_SLOT = 1 << 1
@@ -335,14 +336,14 @@ def stack_forward(x: torch.Tensor, stacked: dict, shape, outs: Optional[torch.Te
 
 def stack_trace(workspace: torch.Tensor, shape, T: int, L: int, flags: int, grid: int) -> torch.Tensor:
     """The MOE_TRACE stamps of the last fused call on ``workspace``: int64
-    [grid, L + 1, 8] nanosecond timer values (see moe_stack_trace_offset).
-    Synchronises the stream."""
+    [grid, L + 1, 16] nanosecond timer values, 0 where a CTA took no stamp
+    (see moe_stack_trace_offset).  Synchronises the stream."""
     c = make_cfg(shape, flags | MOE_TRACE)
     off = int(lib.moe_stack_trace_offset(ctypes.byref(c), int(T), int(L)))
     if off == 0:
         raise ValueError("this call does not trace (not the fused kernel, or no MOE_TRACE)")
-    n = grid * (L + 1) * 8
-    return workspace[off:off + 8 * n].view(torch.int64).view(grid, L + 1, 8).cpu()
+    n = grid * (L + 1) * TRACE_SLOTS
+    return workspace[off:off + 8 * n].view(torch.int64).view(grid, L + 1, TRACE_SLOTS).cpu()
 
 
 def device_status(workspace: torch.Tensor) -> int:

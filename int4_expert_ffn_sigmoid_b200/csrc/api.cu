@@ -14,12 +14,12 @@ namespace {
 using namespace moe;
 
 constexpr unsigned kKnownFlags = MOE_ADD_RESIDUAL | MOE_DEBUG_CHECK | MOE_FORCE_DECODE | MOE_FORCE_PREFILL |
-                                 MOE_OUT_F32 | MOE_TEST_STALL | MOE_NO_LOOKAHEAD | MOE_TEST_BAD_INDEX |
+                                 MOE_OUT_F32 | MOE_TEST_STALL | MOE_LOOKAHEAD | MOE_TEST_BAD_INDEX |
                                  MOE_TRACE | MOE_DEBUG_POISON;
 // Traced CTAs at most (the fused kernel runs one CTA per SM).
 constexpr int kMaxGridF = 256;
 static_assert(kFlagResidual == MOE_ADD_RESIDUAL && kFlagOutF32 == MOE_OUT_F32 && kFlagTestStall == MOE_TEST_STALL &&
-                  kFlagNoLookahead == MOE_NO_LOOKAHEAD && kFlagTestBadIndex == MOE_TEST_BAD_INDEX &&
+                  kFlagLookahead == MOE_LOOKAHEAD && kFlagTestBadIndex == MOE_TEST_BAD_INDEX &&
                   kFlagTrace == MOE_TRACE,
               "kernel flag bits match the C ABI");
 static_assert(ST_BAD_EXPERT == MOE_DEVSTAT_BAD_EXPERT && ST_BAD_SLOT == MOE_DEVSTAT_BAD_SLOT &&
@@ -459,7 +459,7 @@ int moe_stack_forward(const void* x, const moe_stack_weights_t* w, int32_t L, vo
         // one moe_layer_forward call per layer, each layer's output the next one's input
         for (int32_t l = 0; l < L; ++l) {
             moe_cfg_t c = *cfg;
-            c.flags &= ~(unsigned)MOE_NO_LOOKAHEAD;
+            c.flags &= ~(unsigned)MOE_LOOKAHEAD;
             c.topk_idx_out = cfg->topk_idx_out ? cfg->topk_idx_out + l * TK : nullptr;
             c.topk_w_out = cfg->topk_w_out ? cfg->topk_w_out + l * TK : nullptr;
             c.stage_events = nullptr;
@@ -489,6 +489,10 @@ int moe_stack_forward(const void* x, const moe_stack_weights_t* w, int32_t L, vo
     a.rows2 = fused_rows2(cfg->H, cfg->E, cfg->K, cfg->I, cfg->Is, T, fused_grid());
     a.nsl_r = slices_of(cfg->I);
     a.nsl_s = cfg->Is > 0 ? slices_of(cfg->Is) : 0;
+    a.r13_r = cfg->I / kTaskRows13;
+    a.r13_s = cfg->Is / kTaskRows13;
+    a.r2_r = (cfg->H / a.rows2) * a.nsl_r;
+    a.r2_s = (cfg->H / a.rows2) * a.nsl_s;
     a.scale = cfg->routed_scaling;
     a.flags = cfg->flags;
     a.x = static_cast<const __nv_bfloat16*>(x);
@@ -524,6 +528,8 @@ int moe_stack_forward(const void* x, const moe_stack_weights_t* w, int32_t L, vo
     if (cfg->flags & MOE_DEBUG_POISON)  // every byte a kernel reads must have been written first
         err = cudaMemsetAsync(ws + F.counters_end, 0xFF, F.total - F.counters_end, s);
     if (err == cudaSuccess) err = cudaMemsetAsync(ws, 0, F.counters_end, s);
+    if (err == cudaSuccess && (cfg->flags & MOE_TRACE))  // stamps a CTA does not take stay 0
+        err = cudaMemsetAsync(ws + F.trace, 0, F.total - F.trace, s);
     if (err == cudaSuccess) err = launch_decode_stack(a, fused_grid(), s);
     if (err != cudaSuccess) return MOE_ERR_CUDA;
     if (cfg->flags & MOE_DEBUG_CHECK) {

@@ -70,15 +70,13 @@ constexpr int kStride2 = kSliceK + kPadB;          // quantized h row of a down 
 constexpr int kXs2Bytes = 2 * kChunk * kStride2;
 constexpr int kRawBytes = kChunk * kSliceK * 4;    // f32 h slice of a down task
 constexpr int kRsBytes = kMaxRows2 * 4;            // row scales of a down task
-constexpr int kXbStride = kColBlk + 8;             // staged x row of a router unit (bf16)
 constexpr long long kDrainCycles = 200000000LL;
 
-// Scratch of phases A and B inside the h staging area of the down tasks:
-// the staged x block of a router unit, the table build's per-chunk counts,
-// and the summed logits of a token group (this layer's and the lookahead's).
+// Scratch of phase A inside the h staging area of the down tasks: the staged
+// x block of a router unit, and the summed logits of a token group (this
+// layer's and the lookahead's).
 constexpr int kScrXb = 0;
-constexpr int kScrCnt = kScrXb + 16 * kXbStride * 2;
-constexpr int kScrLog = kScrCnt + kMaxSlots / 32 * kMaxE;
+constexpr int kScrLog = kScrXb + kGroupTok * kColBlk * 4;
 constexpr int kScrEnd = kScrLog + 2 * kGroupTok * kMaxE * 4;
 static_assert(kScrEnd <= kRawBytes, "phase A/B scratch fits the h staging");
 
@@ -107,6 +105,8 @@ struct Sh {
     alignas(16) float hmr[kChunk][kSliceK / kTaskRows13];
     float xsc[kChunk];
     QScale qs[kChunk];
+    float bias[2][kMaxE];  // router bias of layer l and l + 1 (router units)
+    alignas(8) uint8_t cnt8[kMaxSlots / 32][kMaxE];  // table build: picks of each expert per 32-pick chunk
 };
 
 constexpr size_t kSmem = ((sizeof(Sh) + 1023) & ~size_t(1023)) + 1024 /* alignment slack */ +
@@ -116,8 +116,8 @@ static_assert(kSmem <= 227 * 1024, "fused decode shared memory");
 __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // MOE_TRACE: thread 0 of the consumers stamps event `slot` of layer l.
-__device__ __forceinline__ void stamp(const FArgs& a, int l, int slot) {
-    if (a.trace && threadIdx.x == 0) {
+__device__ __forceinline__ void stamp(const FArgs& a, int l, int slot, bool when = true) {
+    if (a.trace && when && threadIdx.x == 0) {
         unsigned long long t;
         asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
         a.trace[((size_t)blockIdx.x * (a.L + 1) + l) * kTraceSlots + slot] = t;
@@ -128,18 +128,6 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
-}
-
-// This CTA's 1/grid share of the 128-byte lines of bytes [0, n) of p, one
-// prefetch.global.L2 per line over `threads` threads (thread `tid`).  Spread
-// over every SM, the prefetches of a region cost each SM a few instructions.
-__device__ __forceinline__ void prefetch_share(const void* p, size_t n, int tid, int threads) {
-    const size_t lines = (n + 127) / 128;
-    const size_t per = (lines + gridDim.x - 1) / gridDim.x;
-    const size_t first = (size_t)blockIdx.x * per;
-    const char* c = static_cast<const char*>(p);
-    for (size_t l = first + tid; l < first + per && l < lines; l += threads)
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(c + l * 128));
 }
 
 // Bounded wait of thread 0 for *ctr >= target.  Gives up when the global
@@ -202,7 +190,7 @@ __device__ __forceinline__ void select_warp(const float (&L)[kMaxE / 32], const 
         sc[j] = 0.f;
         if (e < E) {
             const float s = 1.0f / (1.0f + expf(-L[j]));
-            const float kk = s + __ldg(bias + e);
+            const float kk = s + bias[e];
             key[j] = isnan(kk) ? -INFINITY : kk;
             sc[j] = s;
         }
@@ -210,9 +198,8 @@ __device__ __forceinline__ void select_warp(const float (&L)[kMaxE / 32], const 
     unsigned taken = 0;
     my_e = -1;
     float my_s = 0.f, ssum = 0.f;
-#pragma unroll
-    for (int k = 0; k < kMaxK; ++k) {
-        if (k >= K) break;
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
         float bk = -INFINITY, bs = 0.f;
         int be = 0x7fffffff;
 #pragma unroll
@@ -238,34 +225,38 @@ __device__ __forceinline__ void select_warp(const float (&L)[kMaxE / 32], const 
 
 // Logits of the group's tokens t0 .. t0+nt-1 (all 256 consumer threads):
 // dst[tt * kMaxE + e] = the partial logits of (t0 + tt, e) summed over the
-// hidden blocks, block 0 first.  Loads are issued eight blocks at a time.
-__device__ __forceinline__ void sum_logits(const FArgs& a, const float* part, int t0, int nt, float* dst) {
+// hidden blocks, block 0 first; with `look`, the lookahead's too, into
+// dst[(kGroupTok + tt) * kMaxE + e].  Loads are issued eight blocks at a time,
+// both routers' together.
+__device__ __forceinline__ void sum_logits(const FArgs& a, int t0, int nt, bool look, float* dst) {
     const int n = nt * a.E;
+    const size_t step = (size_t)a.T * a.E;
     for (int i = threadIdx.x; i < n; i += 256) {
         const int tt = i / a.E, e = i - tt * a.E;
-        const float* src = part + (size_t)(t0 + tt) * a.E + e;
-        const size_t step = (size_t)a.T * a.E;
-        float acc = 0.f;
+        const float* src = a.lp + (size_t)(t0 + tt) * a.E + e;
+        const float* srn = a.lpn + (size_t)(t0 + tt) * a.E + e;
+        float acc = 0.f, acn = 0.f;
         int cb = 0;
         for (; cb + 8 <= a.NCB; cb += 8) {
-            float v[8];
+            float v[8], w[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (cb + u) * step);
+            for (int u = 0; u < 8; ++u) {
+                v[u] = __ldcg(src + (cb + u) * step);
+                w[u] = look ? __ldcg(srn + (cb + u) * step) : 0.f;
+            }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) acc += v[u];
+            for (int u = 0; u < 8; ++u) {
+                acc += v[u];
+                acn += w[u];
+            }
         }
-        for (; cb < a.NCB; ++cb) acc += __ldcg(src + cb * step);
+        for (; cb < a.NCB; ++cb) {
+            acc += __ldcg(src + cb * step);
+            if (look) acn += __ldcg(srn + cb * step);
+        }
         dst[tt * kMaxE + e] = acc;
+        if (look) dst[(kGroupTok + tt) * kMaxE + e] = acn;
     }
-}
-
-// This CTA's share of the L2 prefetch of expert e of layer l (codes and scales).
-__device__ __forceinline__ void prefetch_expert_share(const FArgs& a, int l, int e, int tid, int threads) {
-    const size_t le = (size_t)l * a.E + e;
-    prefetch_share(a.w13 + le * (size_t)a.I * a.H, (size_t)a.I * a.H, tid, threads);
-    prefetch_share(a.w2 + le * (size_t)a.H * (a.I / 2), (size_t)a.H * (a.I / 2), tid, threads);
-    prefetch_share(a.s13 + le * 2 * a.I, (size_t)2 * a.I * 4, tid, threads);
-    prefetch_share(a.s2 + le * a.H, (size_t)a.H * 4, tid, threads);
 }
 
 // x_l of token t as the input of layer l (the stack's input, or layer l-1's output).
@@ -277,6 +268,45 @@ __device__ __forceinline__ const __nv_bfloat16* layer_input(const FArgs& a, int 
 __device__ void quantize_token(const FArgs& a, int l, int t, int lane) {
     const uint4* xr = reinterpret_cast<const uint4*>(layer_input(a, l) + (size_t)t * a.H);
     const int ng = a.H / 8;
+    constexpr int kRegGroups = 8;  // rows up to 32 * 8 * 8 = 2048 elements stay in registers
+    if (ng <= 32 * kRegGroups) {
+        uint4 v[kRegGroups];
+        float m = 0.f;
+#pragma unroll
+        for (int i = 0; i < kRegGroups; ++i) {
+            const int gi = lane + 32 * i;
+            v[i] = gi < ng ? __ldcg(xr + gi) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < kRegGroups; ++i) {
+            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) m = nanmax(nanmax(m, fabsf(bf16lo(w[k]))), fabsf(bf16hi(w[k])));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = nanmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const QScale qs = qscale(m);
+        uint2* q0 = reinterpret_cast<uint2*>(a.xq + (size_t)t * 2 * a.H);
+        uint2* q1 = reinterpret_cast<uint2*>(a.xq + (size_t)t * 2 * a.H + a.H);
+#pragma unroll
+        for (int i = 0; i < kRegGroups; ++i) {
+            const int gi = lane + 32 * i;
+            if (gi >= ng) break;
+            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+            float f[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                f[2 * k] = bf16lo(w[k]);
+                f[2 * k + 1] = bf16hi(w[k]);
+            }
+            uint2 p0, p1;
+            quant2x8(f, qs, p0, p1);
+            q0[gi] = p0;
+            q1[gi] = p1;
+        }
+        if (lane == 0) a.xs[t] = qs.s;
+        return;
+    }
     float m = 0.f;
 #pragma unroll 4
     for (int gi = lane; gi < ng; gi += 32) {
@@ -309,73 +339,55 @@ __device__ void quantize_token(const FArgs& a, int l, int t, int lane) {
 }
 
 // ---------------------------------------------------------------------------
-// Router unit on the tensor cores.  A job is (router, n-tile of 8 experts):
-// the B fragments of its 8 k steps of the unit's 128 columns.
-struct WFrag {
-    float2 w[kColBlk / 16][2];
+// Router unit: partial logits of a block of 128 hidden columns for the
+// group's tokens.  Thread (expert e = 64 b + tid / 4, quarter q = tid % 4)
+// accumulates, for each token, the columns 16 i + 4 q .. 16 i + 4 q + 3 for
+// i = 0..7 in that order with fused multiply-adds (the four quarters read
+// neighbouring 16-byte chunks of a staged row: no bank conflict); the four
+// quarters are then summed by an xor-butterfly (1, 2).  A job is (router,
+// block b of 64 experts): this thread's 32 router weights of it.  A token's
+// logit never depends on the other tokens of the batch.
+struct WRow {
+    float4 w[kColBlk / 4 / 4];
 };
 
-__device__ __forceinline__ void load_wfrag(const FArgs& a, int layer, int ntile, int col0, int lane, WFrag& f) {
-    const int g = lane >> 2, q = lane & 3;
-    const int e = ntile * 8 + g;
-    const float* wrow = a.rw + ((size_t)layer * a.E + (e < a.E ? e : a.E - 1)) * a.H + col0;
+// Coherent (L2) loads, so that the compiler keeps them where they are: they
+// are issued before the unit waits for the previous layer.
+__device__ __forceinline__ void load_wrow(const FArgs& a, int layer, int eb, int col0, WRow& f) {
+    const int e = eb * 64 + (threadIdx.x >> 2), q = threadIdx.x & 3;
+    const float4* src = reinterpret_cast<const float4*>(a.rw + ((size_t)layer * a.E + min(e, a.E - 1)) * a.H + col0) + q;
 #pragma unroll
-    for (int k = 0; k < kColBlk / 16; ++k) {
-        f.w[k][0] = __ldg(reinterpret_cast<const float2*>(wrow + k * 16 + 2 * q));
-        f.w[k][1] = __ldg(reinterpret_cast<const float2*>(wrow + k * 16 + 2 * q + 8));
-    }
+    for (int i = 0; i < kColBlk / 16; ++i) f.w[i] = __ldcg(src + 4 * i);
 }
 
-__device__ __forceinline__ void split3(float w, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(w);
-    const float r1 = w - __bfloat162float(h);
-    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(m);
-    hi = __bfloat16_as_ushort(h);
-    mid = __bfloat16_as_ushort(m);
-    lo = __bfloat16_as_ushort(__float2bfloat16_rn(r2));
-}
-
-__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* smem_row) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(smem_addr(smem_row)));
-}
-
-// Partial logits of the staged block (xb: 16 rows, tokens in rows 0..nt-1)
-// against the job's experts -> part[(cb * T + t0 + row) * E + e].
-__device__ __forceinline__ void router_job(const FArgs& a, const uint16_t* xb, const WFrag& f, int ntile, int cb,
-                                           int t0, int nt, float* part, int lane) {
-    const int g = lane >> 2, q = lane & 3;
-    const bool valid_e = ntile * 8 + g < a.E;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+// xf: the staged block, [kGroupTok][kColBlk] f32.
+__device__ __forceinline__ void router_job(const FArgs& a, const float* xf, const WRow& f, int eb, int cb, int t0,
+                                           int nt, float* part) {
+    const int e = eb * 64 + (threadIdx.x >> 2), q = threadIdx.x & 3;
+    float acc[kGroupTok];
 #pragma unroll
-    for (int ks = 0; ks < kColBlk / 16; ++ks) {
-        uint32_t bh[2], bm[2], bl[2];
+    for (int t = 0; t < kGroupTok; ++t) acc[t] = 0.f;
+#pragma unroll 1
+    for (int i = 0; i < kColBlk / 16; ++i) {
 #pragma unroll
-        for (int v = 0; v < 2; ++v) {
-            const float w0 = valid_e ? f.w[ks][v].x : 0.f, w1 = valid_e ? f.w[ks][v].y : 0.f;
-            uint16_t h0, m0, l0, h1, m1, l1;
-            split3(w0, h0, m0, l0);
-            split3(w1, h1, m1, l1);
-            bh[v] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-            bm[v] = (uint32_t)m0 | ((uint32_t)m1 << 16);
-            bl[v] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+        for (int t = 0; t < kGroupTok; ++t) {
+            const float4 xv = *reinterpret_cast<const float4*>(xf + t * kColBlk + 16 * i + 4 * q);
+            acc[t] = fmaf(xv.x, f.w[i].x, acc[t]);
+            acc[t] = fmaf(xv.y, f.w[i].y, acc[t]);
+            acc[t] = fmaf(xv.z, f.w[i].z, acc[t]);
+            acc[t] = fmaf(xv.w, f.w[i].w, acc[t]);
         }
-        uint32_t af[4];
-        ldmatrix_x4(af, xb + (lane & 15) * kXbStride + ks * 16 + (lane >> 4) * 8);
-        float t[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_bf16(t, af, bl[0], bl[1]);
-        mma_bf16(t, af, bm[0], bm[1]);
-        mma_bf16(t, af, bh[0], bh[1]);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[v] += t[v];
     }
-    const int e = ntile * 8 + 2 * q;
-    if (g < nt) {
-        float* dst = part + ((size_t)cb * a.T + t0 + g) * a.E;
-        if (e < a.E) dst[e] = acc[0];
-        if (e + 1 < a.E) dst[e + 1] = acc[1];
+#pragma unroll
+    for (int t = 0; t < kGroupTok; ++t) {
+        acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 1);
+        acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 2);
+    }
+    // lane quarter q stores tokens q and q + 4
+    if (e < a.E) {
+#pragma unroll
+        for (int t = 0; t < kGroupTok; ++t)
+            if ((t & 3) == q && t < nt) part[((size_t)cb * a.T + t0 + t) * a.E + e] = acc[t];
     }
 }
 
@@ -386,7 +398,7 @@ __device__ __forceinline__ void router_job(const FArgs& a, const uint16_t* xb, c
 // ascending), then the shared expert's slices, then the residual, rounded
 // once.
 __device__ __forceinline__ void combine_block(const FArgs& a, const Sh& sh, int l, int t0, int nt, int col0,
-                                              uint16_t* xb) {
+                                              float* xf) {
     const int t = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (t >= nt) return;
     const int tok = t0 + t, j = col0 + 4 * lane;
@@ -428,7 +440,9 @@ __device__ __forceinline__ void combine_block(const FArgs& a, const Sh& sh, int 
         xv.y = *reinterpret_cast<uint32_t*>(&o23);
         *reinterpret_cast<uint2*>(a.outs + ((size_t)(l - 1) * a.T + tok) * H + j) = xv;
     }
-    if (xb) *reinterpret_cast<uint2*>(xb + t * kXbStride + 4 * lane) = xv;
+    if (xf)
+        *reinterpret_cast<float4*>(xf + t * kColBlk + 4 * lane) =
+            make_float4(bf16lo(xv.x), bf16hi(xv.x), bf16lo(xv.y), bf16hi(xv.y));
 }
 
 // ---------------------------------------------------------------------------
@@ -437,10 +451,7 @@ __device__ __forceinline__ void combine_block(const FArgs& a, const Sh& sh, int 
 // the last bucket.  Slots are expert-contiguous and in (t, k) order within an
 // expert; the shared bucket's slots are T*K + t.
 __device__ __forceinline__ int tasks13_of(const FArgs& a, int e, int n) {
-    return ((e == a.E ? a.Is : a.I) / kTaskRows13) * chunks_of(n, kChunk);
-}
-__device__ __forceinline__ int tasks2_of(const FArgs& a, int e, int n) {
-    return (a.H / a.rows2) * slices_of(e == a.E ? a.Is : a.I) * chunks_of(n, kChunk);
+    return (e == a.E ? a.r13_s : a.r13_r) * chunks_of(n, kChunk);
 }
 
 __device__ __forceinline__ int snake(int c, int r) {
@@ -497,13 +508,13 @@ __device__ __forceinline__ int my_task_count(int ntask) {
 // Builds layer l's tables in shared memory from the selections (all 256
 // consumer threads; the same result in every CTA).  cnt8: scratch of
 // kMaxSlots / 32 x kMaxE bytes.
-__device__ void build_tables(const FArgs& a, Sh& sh, uint8_t* cnt8) {
+__device__ void build_tables(const FArgs& a, Sh& sh) {
     const int tid = threadIdx.x, lane = tid & 31;
     const int E = a.E, K = a.K, T = a.T, TK = T * K;
     constexpr int kChunks = kMaxSlots / 32;
     int my_e[2], my_rank[2];
-    for (int i = tid; i < kChunks * kMaxE / 4; i += 256) reinterpret_cast<int*>(cnt8)[i] = 0;
-    consumers_sync();
+    bool leader[2];
+    // sh.cnt8 is all zero here (zeroed at the start, and after every use)
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
         const int i = tid + 256 * u;
@@ -520,28 +531,34 @@ __device__ void build_tables(const FArgs& a, Sh& sh, uint8_t* cnt8) {
         const unsigned m = __match_any_sync(0xffffffffu, i < TK ? e : -2 - lane);
         my_e[u] = e;
         my_rank[u] = __popc(m & ((1u << lane) - 1u));
-        if (e >= 0 && lane == __ffs(m) - 1) cnt8[(i >> 5) * kMaxE + e] = (uint8_t)__popc(m);
-    }
-    consumers_sync();
-    if (tid < E) {
-        int c = 0;
-        for (int ch = 0; ch < kChunks; ++ch) c += cnt8[ch * kMaxE + tid];
-        sh.cnt[tid] = c;
+        leader[u] = e >= 0 && lane == __ffs(m) - 1;
+        if (leader[u]) sh.cnt8[i >> 5][e] = (uint8_t)__popc(m);
     }
     consumers_sync();
     if (tid < 32) {
         // lane l owns experts 8l .. 8l+7: counts, buckets, gate/up and down tasks
         constexpr int kPer = kMaxE / 32;
         int c[kPer];
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) c[j] = 0;
+        for (int ch = 0; ch < (TK + 31) / 32; ++ch) {
+            const uint2 w = *reinterpret_cast<const uint2*>(&sh.cnt8[ch][lane * kPer]);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                c[j] += (w.x >> (8 * j)) & 0xFF;
+                c[4 + j] += (w.y >> (8 * j)) & 0xFF;
+            }
+        }
         int v[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
             const int e = lane * kPer + j;
-            c[j] = e < E ? sh.cnt[e] : 0;
+            if (e >= E) c[j] = 0;
+            const int ch = (c[j] + kChunk - 1) / kChunk;
             v[0] += c[j];
             v[1] += c[j] > 0;
-            v[2] += c[j] > 0 ? tasks13_of(a, e, c[j]) : 0;
-            v[3] += c[j] > 0 ? tasks2_of(a, e, c[j]) : 0;
+            v[2] += a.r13_r * ch;
+            v[3] += a.r2_r * ch;
         }
         int inc[4] = {v[0], v[1], v[2], v[3]};
 #pragma unroll
@@ -558,14 +575,15 @@ __device__ void build_tables(const FArgs& a, Sh& sh, uint8_t* cnt8) {
             if (e < E) {
                 sh.off[e] = off;
                 if (c[j] > 0) {
+                    const int ch = (c[j] + kChunk - 1) / kChunk;
                     sh.be[b] = e;
                     sh.bn[b] = c[j];
                     sh.boff[b] = off;
                     sh.ts13[b] = b13;
                     sh.ts2[b] = b2;
                     ++b;
-                    b13 += tasks13_of(a, e, c[j]);
-                    b2 += tasks2_of(a, e, c[j]);
+                    b13 += a.r13_r * ch;
+                    b2 += a.r2_r * ch;
                 }
                 off += c[j];
             }
@@ -579,13 +597,14 @@ __device__ void build_tables(const FArgs& a, Sh& sh, uint8_t* cnt8) {
                 nb = t13 = t2 = 0;
             }
             if (a.Is > 0) {
+                const int ch = (T + kChunk - 1) / kChunk;
                 sh.be[nb] = E;
                 sh.bn[nb] = T;
                 sh.boff[nb] = TK;
                 sh.ts13[nb] = t13;
                 sh.ts2[nb] = t2;
-                t13 += tasks13_of(a, E, T);
-                t2 += tasks2_of(a, E, T);
+                t13 += a.r13_s * ch;
+                t2 += a.r2_s * ch;
                 ++nb;
             }
             sh.ts13[nb] = t13;
@@ -596,6 +615,7 @@ __device__ void build_tables(const FArgs& a, Sh& sh, uint8_t* cnt8) {
         }
     }
     consumers_sync();
+    // slots; this CTA's task count and first task descriptors
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
         const int i = tid + 256 * u;
@@ -604,7 +624,7 @@ __device__ void build_tables(const FArgs& a, Sh& sh, uint8_t* cnt8) {
         int slot = -1;
         if (e >= 0) {
             int base = 0;
-            for (int ch = 0; ch < (i >> 5); ++ch) base += cnt8[ch * kMaxE + e];
+            for (int ch = 0; ch < (i >> 5); ++ch) base += sh.cnt8[ch][e];
             slot = sh.off[e] + base + my_rank[u];
         }
         if (slot < 0 || slot >= TK) {
@@ -619,10 +639,14 @@ __device__ void build_tables(const FArgs& a, Sh& sh, uint8_t* cnt8) {
         sh.my13 = my_task_count(sh.ntask13);
         sh.my2 = my_task_count(sh.ntask2);
     }
+    if (tid >= 64 && tid < 64 + kMaxTasks) sh.td13[tid - 64] = decode_task(a, sh, 0, snake(blockIdx.x, tid - 64));
+    else if (tid >= 64 + kMaxTasks && tid < 64 + 2 * kMaxTasks)
+        sh.td2[tid - 64 - kMaxTasks] = decode_task(a, sh, 1, snake(blockIdx.x, tid - 64 - kMaxTasks));
     consumers_sync();
-    if (tid < kMaxTasks) sh.td13[tid] = decode_task(a, sh, 0, snake(blockIdx.x, tid));
-    else if (tid < 2 * kMaxTasks) sh.td2[tid - kMaxTasks] = decode_task(a, sh, 1, snake(blockIdx.x, tid - kMaxTasks));
-    consumers_sync();
+    // back to zero for the next layer (only the leaders' entries are set)
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+        if (leader[u]) sh.cnt8[(tid + 256 * u) >> 5][my_e[u]] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -719,6 +743,54 @@ __device__ __forceinline__ bool task_ok(const FArgs& a, const TaskD& d) {
     return d.e >= 0 && d.e <= a.E && !(d.e == a.E && a.Is == 0) && d.nc > 0;
 }
 
+// L2 prefetch by the producer warp (bulk prefetches through the CTA's copy
+// engine, lanes in parallel), every CTA its 1/grid share of each region: what
+// layer `n1` reads first -- the experts its router picked when run on the
+// previous layer's input (the lookahead), its shared expert and router, and
+// the router after it (which the next lookahead reads).
+__device__ __forceinline__ void prefetch_bulk_share(const void* p, size_t n) {
+    const size_t per = ((n + gridDim.x - 1) / gridDim.x + 15) & ~size_t(15);
+    const size_t o = (size_t)blockIdx.x * per;
+    if (o >= n) return;
+    const size_t len = n - o < per ? n - o : per;
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(static_cast<const char*>(p) + o), "r"((uint32_t)len)
+                 : "memory");
+}
+
+__device__ void prefetch_layer(const FArgs& a, int n1, bool experts, int lane) {
+    if (!(a.flags & kFlagLookahead) || n1 >= a.L) return;
+    if (experts) {
+        unsigned pred[kMaxE / 32];
+#pragma unroll
+        for (int w = 0; w < kMaxE / 32; ++w) pred[w] = __ldcg(a.pred_bits + n1 * 8 + w);
+        // lane j takes the j-th, (j+32)-th, ... predicted expert
+        int k = 0;
+#pragma unroll
+        for (int w = 0; w < kMaxE / 32; ++w) {
+            unsigned bits = pred[w];
+            while (bits) {
+                const int e = 32 * w + __ffs(bits) - 1;
+                bits &= bits - 1;
+                if ((k++ & 31) == lane) {
+                    const size_t le = (size_t)n1 * a.E + e;
+                    prefetch_bulk_share(a.w13 + le * (size_t)a.I * a.H, (size_t)a.I * a.H);
+                    prefetch_bulk_share(a.w2 + le * (size_t)a.H * (a.I / 2), (size_t)a.H * (a.I / 2));
+                    prefetch_bulk_share(a.s13 + le * 2 * a.I, (size_t)2 * a.I * 4);
+                    prefetch_bulk_share(a.s2 + le * a.H, (size_t)a.H * 4);
+                }
+            }
+        }
+    }
+    if (a.Is > 0) {
+        if (lane == 0) prefetch_bulk_share(a.sh_w13 + (size_t)n1 * a.Is * a.H, (size_t)a.Is * a.H);
+        if (lane == 1) prefetch_bulk_share(a.sh_w2 + (size_t)n1 * a.H * (a.Is / 2), (size_t)a.H * (a.Is / 2));
+        if (lane == 2) prefetch_bulk_share(a.sh_s13 + (size_t)n1 * 2 * a.Is, (size_t)2 * a.Is * 4);
+        if (lane == 3) prefetch_bulk_share(a.sh_s2 + (size_t)n1 * a.H, (size_t)a.H * 4);
+    }
+    if (lane == 4) prefetch_bulk_share(a.rw + (size_t)n1 * a.E * a.H, (size_t)a.E * a.H * 4);
+    if (lane == 5 && n1 + 1 < a.L) prefetch_bulk_share(a.rw + (size_t)(n1 + 1) * a.E * a.H, (size_t)a.E * a.H * 4);
+}
+
 // ---------------------------------------------------------------------------
 // Producer warp.
 __device__ void producer(const FArgs& a, Sh& sh, uint8_t* wring, uint8_t* xring, const CUtensorMap* tm13,
@@ -740,6 +812,7 @@ __device__ void producer(const FArgs& a, Sh& sh, uint8_t* wring, uint8_t* xring,
     const int Rs = a.Is / kTaskRows13;
     const int ns = a.Is > 0 ? Rs * chunks_of(a.T, kChunk) : 0;
     bool ok = true;
+    prefetch_layer(a, 0, false, lane);
     // next free stage: waits for its slot (round > 0); false on abort / timeout
     auto acquire = [&](int& s, int& round) -> bool {
         s = (int)(n % kStages);
@@ -774,6 +847,9 @@ __device__ void producer(const FArgs& a, Sh& sh, uint8_t* wring, uint8_t* xring,
             }
             if (!ok) break;
         }
+        // the layer's predicted experts, shared expert and routers (MOE_LOOKAHEAD),
+        // behind its first weights and ahead of its routing
+        if (l > 0) prefetch_layer(a, l, true, lane);
         // (b) the layer's tables
         const bool got = ring_wait(a, sh, &sh.tready, l & 1);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -888,19 +964,24 @@ __device__ bool phase_units(const FArgs& a, Sh& sh, const Smem& m, int l) {
         return true;
     }
     const bool final = l == a.L;
-    const bool look = !final && l + 1 < a.L && !(a.flags & kFlagNoLookahead);
-    uint16_t* xb = reinterpret_cast<uint16_t*>(m.raw);
-    const int n_e = (a.E + 7) / 8;  // expert n-tiles per router
-    const int jobs = final ? 0 : ((n_e + 7 - warp) / 8) * (look ? 2 : 1);  // this warp's jobs per unit
-    // job k of this warp: router k / per (0 = layer l, 1 = layer l + 1), n-tile warp + 8 (k % per)
-    const int per = (n_e + 7 - warp) / 8;
-    WFrag wf[2];
-    auto load_job = [&](int k, int col0, WFrag& f) {
-        if (k < jobs) load_wfrag(a, l + k / per, warp + 8 * (k % per), col0, lane, f);
+    const bool look = !final && l + 1 < a.L && (a.flags & kFlagLookahead);
+    float* xf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(m.raw) + kScrXb);
+    const int per = (a.E + 63) / 64;  // expert blocks per router
+    const int jobs = final ? 0 : per * (look ? 2 : 1);
+    // job k: router k / per (0 = layer l, 1 = layer l + 1), expert block k % per
+    WRow wr[2];
+    auto load_job = [&](int k, int col0, WRow& f) {
+        if (k < jobs) load_wrow(a, l + k / per, k % per, col0, f);
     };
-    // the first unit's first two jobs are loaded before the wait (they do not depend on it)
-    load_job(0, (first % a.NCB) * kColBlk, wf[0]);
-    load_job(1, (first % a.NCB) * kColBlk, wf[1]);
+    // nothing of this depends on the wait below: the first unit's first two
+    // jobs' router weights, and the routers' biases
+    load_job(0, (first % a.NCB) * kColBlk, wr[0]);
+    load_job(1, (first % a.NCB) * kColBlk, wr[1]);
+    if (!final)
+        for (int i = tid; i < 2 * a.E; i += 256) {
+            const int r = i / a.E, e = i - r * a.E;
+            if (r == 0 || look) sh.bias[r][e] = __ldcg(a.rb + (size_t)(l + r) * a.E + e);
+        }
     if (l > 0) {
         if (tid == 0) sh.bcast = wait_count(a, a.down_done + (l - 1), (int)gridDim.x);
         consumers_sync();
@@ -911,19 +992,24 @@ __device__ bool phase_units(const FArgs& a, Sh& sh, const Smem& m, int l) {
         const int g = u / a.NCB, cb = u - g * a.NCB;
         const int t0 = g * kGroupTok, nt = min(kGroupTok, a.T - t0), col0 = cb * kColBlk;
         if (u != first) {
-            consumers_sync();  // the previous unit is done with xb
-            load_job(0, col0, wf[0]);
-            load_job(1, col0, wf[1]);
+            consumers_sync();  // the previous unit is done with xf
+            load_job(0, col0, wr[0]);
+            load_job(1, col0, wr[1]);
         }
-        combine_block(a, sh, l, t0, nt, col0, final ? nullptr : xb);
+        combine_block(a, sh, l, t0, nt, col0, final ? nullptr : xf);
         if (final) continue;
-        consumers_sync();  // xb staged
-        for (int k = 0; k < jobs; ++k) {
-            const int r = k / per, ntile = warp + 8 * (k % per);
-            router_job(a, xb, wf[k & 1], ntile, cb, t0, nt, r == 0 ? a.lp : a.lpn, lane);
-            load_job(k + 2, col0, wf[k & 1]);
+        consumers_sync();  // xf staged
+        stamp(a, l, 7, u == first);
+        for (int k = 0; k < jobs; k += 2) {  // two jobs per round: wr is indexed statically
+            router_job(a, xf, wr[0], k % per, cb, t0, nt, k / per == 0 ? a.lp : a.lpn);
+            load_job(k + 2, col0, wr[0]);
+            if (k + 1 < jobs) {
+                router_job(a, xf, wr[1], (k + 1) % per, cb, t0, nt, (k + 1) / per == 0 ? a.lp : a.lpn);
+                load_job(k + 3, col0, wr[1]);
+            }
         }
         consumers_sync();  // every partial logit and output of the unit written
+        stamp(a, l, 8, u == first);
         if (tid == 0) {
             __threadfence();  // this unit's writes before its count
             const int old = atomicAdd(a.grp_cnt + l * kMaxGroupsF + g, 1);
@@ -931,11 +1017,11 @@ __device__ bool phase_units(const FArgs& a, Sh& sh, const Smem& m, int l) {
             sh.last = old == a.NCB - 1;
         }
         consumers_sync();
+        stamp(a, l, 9, u == first);
         if (!sh.last) continue;
         // the last unit of group g: select its tokens and quantize their rows
         float* lg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(m.raw) + kScrLog);
-        sum_logits(a, a.lp, t0, nt, lg);
-        if (look) sum_logits(a, a.lpn, t0, nt, lg + kGroupTok * kMaxE);
+        sum_logits(a, t0, nt, look, lg);
         consumers_sync();
         if (warp < nt) {
             const int t = t0 + warp;
@@ -944,7 +1030,7 @@ __device__ bool phase_units(const FArgs& a, Sh& sh, const Smem& m, int l) {
             for (int j = 0; j < kMaxE / 32; ++j) L[j] = lg[warp * kMaxE + lane + 32 * j];
             int e;
             float w;
-            select_warp(L, a.rb + (size_t)l * a.E, a.E, a.K, a.scale, lane, e, w);
+            select_warp(L, sh.bias[0], a.E, a.K, a.scale, lane, e, w);
             if ((a.flags & kFlagTestBadIndex) && t == 0 && lane == 0) e = a.E;  // test hook: an out-of-range pick
             if (lane < a.K) {
                 const size_t o = (size_t)t * a.K + lane;
@@ -960,12 +1046,14 @@ __device__ bool phase_units(const FArgs& a, Sh& sh, const Smem& m, int l) {
                 for (int j = 0; j < kMaxE / 32; ++j) L[j] = lg[(kGroupTok + warp) * kMaxE + lane + 32 * j];
                 int pe;
                 float pw;
-                select_warp(L, a.rb + (size_t)(l + 1) * a.E, a.E, a.K, a.scale, lane, pe, pw);
+                select_warp(L, sh.bias[1], a.E, a.K, a.scale, lane, pe, pw);
                 if (lane < a.K && pe >= 0 && pe < a.E) atomicOr(a.pred_bits + (l + 1) * 8 + (pe >> 5), 1u << (pe & 31));
             }
+            if (warp == 0) stamp(a, l, 10);
             quantize_token(a, l, t, lane);
         }
         consumers_sync();
+        stamp(a, l, 11);
         if (tid == 0) {
             __threadfence();
             atomicAdd(a.groups_done + l, 1);
@@ -987,40 +1075,10 @@ __device__ bool phase_tables(const FArgs& a, Sh& sh, const Smem& m, int l) {
     consumers_sync();
     if (!sh.bcast) return false;
     stamp(a, l, 3);
-    build_tables(a, sh, reinterpret_cast<uint8_t*>(m.raw) + kScrCnt);
+    build_tables(a, sh);
     if (threadIdx.x == 0) bar_arrive(&sh.tready);  // the producer may start
     stamp(a, l, 4);
-    if (!(a.flags & kFlagNoLookahead)) {
-        // L2 prefetch, every CTA its share: this layer's selected experts that
-        // the previous layer's lookahead did not predict; the next layer's
-        // predicted experts, shared expert and router (and the router after it,
-        // which the next lookahead reads)
-        const int tid = threadIdx.x;
-        for (int b = 0; b < sh.nb; ++b) {
-            const int e = sh.be[b];
-            if (e < a.E && !(l > 0 && (__ldcg(a.pred_bits + l * 8 + (e >> 5)) >> (e & 31)) & 1u))
-                prefetch_expert_share(a, l, e, tid, 256);
-        }
-        if (l + 1 < a.L) {
-            const int n1 = l + 1;
-            for (int w = 0; w < (a.E + 31) / 32; ++w) {
-                unsigned bits = __ldcg(a.pred_bits + n1 * 8 + w);
-                while (bits) {
-                    const int e = 32 * w + __ffs(bits) - 1;
-                    bits &= bits - 1;
-                    prefetch_expert_share(a, n1, e, tid, 256);
-                }
-            }
-            if (a.Is > 0) {
-                prefetch_share(a.sh_w13 + (size_t)n1 * a.Is * a.H, (size_t)a.Is * a.H, tid, 256);
-                prefetch_share(a.sh_w2 + (size_t)n1 * a.H * (a.Is / 2), (size_t)a.H * (a.Is / 2), tid, 256);
-                prefetch_share(a.sh_s13 + (size_t)n1 * 2 * a.Is, (size_t)2 * a.Is * 4, tid, 256);
-                prefetch_share(a.sh_s2 + (size_t)n1 * a.H, (size_t)a.H * 4, tid, 256);
-            }
-            prefetch_share(a.rw + (size_t)n1 * a.E * a.H, (size_t)a.E * a.H * 4, tid, 256);
-            if (l + 2 < a.L) prefetch_share(a.rw + (size_t)(l + 2) * a.E * a.H, (size_t)a.E * a.H * 4, tid, 256);
-        }
-    }
+    stamp(a, l, 12);
     return true;
 }
 
@@ -1052,6 +1110,10 @@ __device__ bool phase_gate_up(const FArgs& a, Sh& sh, const Smem& m, int l, uint
             }
         }
         int acc[4][4];
+        if (r == 0 && a.trace) {  // MOE_TRACE: when the first stage lands
+            ring_wait(a, sh, &sh.full[n % kStages], (n / kStages) & 1);
+            stamp(a, l, 13);
+        }
         switch (NTt) {
             case 1: consume13<1>(a, sh, nch, n, m.wring, m.xring, acc); break;
             case 2: consume13<2>(a, sh, nch, n, m.wring, m.xring, acc); break;
@@ -1114,6 +1176,7 @@ __device__ bool phase_down(const FArgs& a, Sh& sh, const Smem& m, int l, uint32_
         if (tid == 0) sh.bcast = wait_count(a, a.ready + l * (kMaxE + 1) + d.e, tasks13_of(a, d.e, d.n));
         consumers_sync();
         if (!sh.bcast) return false;
+        stamp(a, l, 14, r == 0);
         // the slice of h, its per-64-row maxima and the task's row scales
         const float* S = (shd ? a.sh_s2 + (size_t)l * a.H : a.s2 + ((size_t)l * a.E + d.e) * a.H) + d.rbk * a.rows2;
         for (int c = tid; c < a.rows2 / 4; c += 256) cp_async16(m.rs + 4 * c, S + 4 * c);
@@ -1156,6 +1219,7 @@ __device__ bool phase_down(const FArgs& a, Sh& sh, const Smem& m, int l, uint32_
             }
         }
         consumers_sync();  // staged
+        stamp(a, l, 15, r == 0);
         switch ((2 * d.nc + 7) >> 3) {
             case 1: consume2<1>(a, sh, d, l, n, m.wring, m.xs2, m.rs); break;
             case 2: consume2<2>(a, sh, d, l, n, m.wring, m.xs2, m.rs); break;
@@ -1211,13 +1275,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicOr(a.status, ST_TIMEOUT);
         atomicExch(a.abort, 1);
     }
-    if (!(a.flags & kFlagNoLookahead)) {
-        if (a.Is > 0) {
-            prefetch_share(a.sh_w13, (size_t)a.Is * a.H, threadIdx.x, 256);
-            prefetch_share(a.sh_w2, (size_t)a.H * (a.Is / 2), threadIdx.x, 256);
-        }
-        if (a.L > 1) prefetch_share(a.rw + (size_t)a.E * a.H, (size_t)a.E * a.H * 4, threadIdx.x, 256);
-    }
+    for (int i = threadIdx.x; i < (int)sizeof(sh.cnt8) / 4; i += 256) reinterpret_cast<int*>(sh.cnt8)[i] = 0;
+    consumers_sync();
     uint32_t n = 0;
     bool ok = true;
     for (int l = 0; ok && l < a.L; ++l) {

@@ -51,7 +51,7 @@ constexpr int kHExpMax = 60;
 // MOE_* flags of the C ABI).
 constexpr unsigned kFlagResidual = 1u << 0;   // MOE_ADD_RESIDUAL
 constexpr unsigned kFlagOutF32 = 1u << 4;     // MOE_OUT_F32
-constexpr unsigned kFlagNoLookahead = 1u << 5;  // MOE_NO_LOOKAHEAD
+constexpr unsigned kFlagLookahead = 1u << 5;  // MOE_LOOKAHEAD
 constexpr unsigned kFlagTestStall = 1u << 6;  // MOE_TEST_STALL
 constexpr unsigned kFlagTestBadIndex = 1u << 7;  // MOE_TEST_BAD_INDEX
 constexpr unsigned kFlagTrace = 1u << 8;      // MOE_TRACE

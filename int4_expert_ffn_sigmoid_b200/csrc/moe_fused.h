@@ -13,8 +13,12 @@ constexpr int kMaxFusedLayers = 128;
 constexpr int kMaxGroupsF = kDecodeMaxTokens / 8;
 // MOE_TRACE: stamps per (CTA, layer): 0 phase A entered, 1 the previous
 // layer's down tasks all done, 2 phase A done, 3 every token group selected,
-// 4 tables built, 5 gate/up tasks done, 6 down tasks done, 7 unused.
-constexpr int kTraceSlots = 8;
+// 4 tables built, 5 gate/up tasks done, 6 down tasks done; first router unit
+// of the CTA: 7 combined, 8 partial logits written, 9 counted; the unit that
+// completed a group: 10 selected, 11 rows quantized; 12 prefetches issued;
+// 13 the first gate/up stage landed; first down task: 14 its expert ready,
+// 15 its activations staged.
+constexpr int kTraceSlots = 16;
 
 // Everything the fused kernel reads and writes.  Weights of all L layers are
 // stacked along a leading layer dimension (layer l of router_w is at
@@ -24,6 +28,8 @@ struct FArgs {
     int T, H, E, K, I, Is, L;
     int G, NCB;            // token groups of 8, hidden blocks of 128
     int rows2, nsl_r, nsl_s;
+    int r13_r, r13_s;      // gate/up tasks per 16-token chunk of a routed / the shared bucket
+    int r2_r, r2_s;        // down tasks per 16-token chunk of a routed / the shared bucket
     float scale;
     unsigned flags;
     const __nv_bfloat16* x;  // [T][H], layer 0's input

@@ -62,7 +62,7 @@ def test_header_constants_match_binding(moe):
     for name in ("MOE_STATIC_WORKSPACE_BYTES", "MOE_OUT_F32", "MOE_FORCE_DECODE",
                  "MOE_FORCE_PREFILL", "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK",
                  "MOE_PATH_SMALL_BATCH", "MOE_PATH_TENSOR_CORE", "MOE_PATH_LARGE_STREAMING",
-                 "MOE_NO_LOOKAHEAD", "MOE_TEST_STALL", "MOE_TEST_BAD_INDEX", "MOE_TRACE", "MOE_DEBUG_POISON",
+                 "MOE_LOOKAHEAD", "MOE_TEST_STALL", "MOE_TEST_BAD_INDEX", "MOE_TRACE", "MOE_DEBUG_POISON",
                  "MOE_DEVSTAT_TIMEOUT", "MOE_DEVSTAT_BAD_EXPERT", "MOE_PATH_FUSED_STACK", "MOE_PATH_PER_LAYER"):
         m = re.search(rf"#define {name} (.+)", text)
         assert m, name

@@ -79,7 +79,7 @@ def test_lookahead_changes_no_bit(moe, cuda_device, nano_stack):
     for T in (1, 64):
         x = workloads.make_x(wl.shape, T, wl.wid, batch=3, device=cuda_device)
         a, ia, wa = run_stack(moe, x, stacked, wl.shape, f)
-        b, ib, wb = run_stack(moe, x, stacked, wl.shape, f | moe.MOE_NO_LOOKAHEAD)
+        b, ib, wb = run_stack(moe, x, stacked, wl.shape, f | moe.MOE_LOOKAHEAD)
         assert torch.equal(a, b) and torch.equal(ia, ib) and torch.equal(wa, wb)
 
 
