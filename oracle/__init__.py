@@ -55,14 +55,14 @@ def _load():
             lib = ctypes.CDLL(build())
             lib.oracle_unpack_int4.argtypes = [_u8p, ctypes.c_int64, _i32p]
             lib.oracle_route.argtypes = [_u16p, _f32p, _f32p, ctypes.c_int32, ctypes.c_int32,
-                                         ctypes.c_int32, ctypes.c_int32, ctypes.c_double,
-                                         _f64p, _f64p, _i32p, _f64p, _f64p]
+                                         ctypes.c_int32, ctypes.c_int32, ctypes.c_double, ctypes.c_double,
+                                         _f64p, _f64p, _i32p, _f64p, _f64p, _f64p]
             lib.oracle_select_topk.argtypes = [_f64p, _f32p, ctypes.c_int32, ctypes.c_int32,
                                                ctypes.c_int32, _i32p, _f64p]
             lib.oracle_expert_ffn.argtypes = [_f64p, ctypes.c_int32, ctypes.c_int32, _u8p, _f32p,
                                               _u8p, _f32p, _f64p, _f64p]
             lib.oracle_moe_tokens.argtypes = (
-                [_u16p] + [ctypes.c_int32] * 6 + [ctypes.c_double, ctypes.c_int32]
+                [_u16p] + [ctypes.c_int32] * 6 + [ctypes.c_double, ctypes.c_double, ctypes.c_int32]
                 + [_f32p, _f32p, _u8p, _f32p, _u8p, _f32p, _u8p, _f32p, _u8p, _f32p]
                 + [_i32p, ctypes.c_int32, _i32p, _f64p, _i32p, _f64p, _f64p])
             for fn in ("oracle_unpack_int4", "oracle_route", "oracle_select_topk",
@@ -102,19 +102,23 @@ def unpack_int4(row, n: int) -> np.ndarray:
     return out
 
 
-def route(x, router_w, router_bias, K: int, scale: float) -> dict:
-    """Router of every token.  x: bf16 [T,H] (torch) or uint16 bf16 bits."""
+def route(x, router_w, router_bias, K: int, scale: float, topp: float = 0.0) -> dict:
+    """Router of every token.  x: bf16 [T,H] (torch) or uint16 bf16 bits.
+    topp: 0 = plain top-K, 0 < topp < 1 = adaptive expert top-p (dropped picks
+    are -1, after the kept ones; ``topp_margin`` tells how close each token's
+    top-p decision came to going the other way, relative to its score sum)."""
     xb = _np(x, np.uint16)
     W = _np(router_w, np.float32)
     b = _np(router_bias, np.float32)
     T, H = xb.shape
     E = W.shape[0]
     logits = np.empty((T, E)); scores = np.empty((T, E))
-    idx = np.empty((T, K), np.int32); w = np.empty((T, K)); margin = np.empty(T)
+    idx = np.empty((T, K), np.int32); w = np.empty((T, K)); margin = np.empty(T); pm = np.empty(T)
     _check(_load().oracle_route(_ptr(xb, _u16p), _ptr(W, _f32p), _ptr(b, _f32p), T, H, E, K,
-                                float(scale), _ptr(logits, _f64p), _ptr(scores, _f64p),
-                                _ptr(idx, _i32p), _ptr(w, _f64p), _ptr(margin, _f64p)), "route")
-    return dict(logits=logits, scores=scores, idx=idx, weights=w, margin=margin)
+                                float(scale), float(topp), _ptr(logits, _f64p), _ptr(scores, _f64p),
+                                _ptr(idx, _i32p), _ptr(w, _f64p), _ptr(margin, _f64p), _ptr(pm, _f64p)),
+           "route")
+    return dict(logits=logits, scores=scores, idx=idx, weights=w, margin=margin, topp_margin=pm)
 
 
 def select_topk(scores, bias, K: int):
@@ -143,12 +147,13 @@ def expert_ffn(xvec, w13, s13, w2, s2):
 
 
 def moe_tokens(x, layer: dict, shape, residual: bool = False, tokens=None,
-               idx_override=None) -> dict:
+               idx_override=None, topp: float = 0.0) -> dict:
     """Layer output (float64) for ``tokens`` (default: all tokens).
 
     ``layer`` is the dict produced by ``workloads.make_layer``; ``shape`` a
     ``workloads.LayerShape``.  ``idx_override`` [n,K] evaluates the given
-    experts instead of the router's choice.
+    experts instead of the router's choice (with ``topp``, -1 entries are
+    dropped picks).  ``topp``: 0 = plain top-K, else the adaptive top-p.
     """
     xb = _np(x, np.uint16)
     T, H = xb.shape
@@ -165,7 +170,7 @@ def moe_tokens(x, layer: dict, shape, residual: bool = False, tokens=None,
                     sw2=_np(layer["sh_w2"], np.uint8), ss2=_np(layer["sh_s2"], np.float32))
     out = np.empty((n, H)); idx = np.empty((n, K), np.int32); w = np.empty((n, K)); m = np.empty(n)
     _check(_load().oracle_moe_tokens(
-        _ptr(xb, _u16p), T, H, E, K, I, Is, float(shape.routed_scaling), int(bool(residual)),
+        _ptr(xb, _u16p), T, H, E, K, I, Is, float(shape.routed_scaling), float(topp), int(bool(residual)),
         _ptr(arrs["rw"], _f32p), _ptr(arrs["rb"], _f32p), _ptr(arrs["w13"], _u8p),
         _ptr(arrs["s13"], _f32p), _ptr(arrs["w2"], _u8p), _ptr(arrs["s2"], _f32p),
         _ptr(arrs.get("sw13"), _u8p), _ptr(arrs.get("ss13"), _f32p),

@@ -34,12 +34,32 @@ def _sigmoid(z):
     return 1.0 / (1.0 + np.exp(-z))
 
 
-def routing_matrix(x: np.ndarray, W: np.ndarray, bias: np.ndarray, K: int, scale: float, forced=None):
+def topp_keep(s_sel: np.ndarray, e_sel: np.ndarray, p: float) -> np.ndarray:
+    """Adaptive expert top-p over one token's K picks (scores s_sel, experts
+    e_sel): a boolean mask of the picks kept -- the fewest of the
+    highest-scoring ones (ties: lower expert index) whose scores reach p of the
+    K picks' total.  Written as a search over prefix lengths: the smallest n
+    such that the n best picks carry at least p of the total (a pick is needed
+    while the mass before it is still below p)."""
+    order = sorted(range(len(s_sel)), key=lambda k: (-s_sel[k], e_sel[k]))
+    total = float(np.sum(s_sel))
+    keep = np.zeros(len(s_sel), bool)
+    for n in range(1, len(order) + 1):
+        if sum(s_sel[order[j]] for j in range(n - 1)) >= p * total:
+            break
+        keep[order[n - 1]] = True
+    return keep
+
+
+def routing_matrix(x: np.ndarray, W: np.ndarray, bias: np.ndarray, K: int, scale: float, forced=None,
+                   topp: float = 0.0):
     """Dense routing weights R [T,E]: R[t,e] = w[t,k] if e = e_k, else 0.
 
-    ``forced`` [T,K] (optional) replaces the selection by the given experts;
-    their weights still come from the unbiased scores, normalised over the
-    forced set."""
+    ``forced`` [T,K] (optional) replaces the selection by the given experts
+    (-1 entries: none); their weights still come from the unbiased scores,
+    normalised over the forced set.  ``topp`` (0 < p < 1): the adaptive expert
+    top-p drops picks (``topp_keep``) and the kept ones are normalised over the
+    kept set."""
     s = _sigmoid(x @ W.T.astype(np.float64))
     key = s + bias.astype(np.float64)[None, :]
     key = np.where(np.isnan(key), -np.inf, key)
@@ -49,19 +69,22 @@ def routing_matrix(x: np.ndarray, W: np.ndarray, bias: np.ndarray, K: int, scale
         if forced is None:
             order = np.argsort(-key[t], kind="stable")  # equal keys keep index order
             sel = order[:K]
+            if 0.0 < topp < 1.0:
+                sel = sel[topp_keep(s[t, sel], sel, topp)]
         else:
-            sel = np.asarray(forced[t], np.int64)
+            sel = np.asarray([e for e in forced[t] if e >= 0], np.int64)
         R[t, sel] = scale * s[t, sel] / s[t, sel].sum()
     return R
 
 
-def moe_dense(x, layer: dict, shape, residual: bool = False, forced=None):
+def moe_dense(x, layer: dict, shape, residual: bool = False, forced=None, topp: float = 0.0):
     """Layer output [T,H] in float64.  x: bf16 [T,H] (torch) or bf16 bits.
-    ``forced`` [T,K]: evaluate these experts instead of the router's choice."""
+    ``forced`` [T,K]: evaluate these experts instead of the router's choice.
+    ``topp``: the adaptive expert top-p (0 = off)."""
     xf = bf16_bits_to_f64(x)
     E, K, I, Is = shape.E, shape.K, shape.I, shape.Is
     R = routing_matrix(xf, _np(layer["router_w"], np.float64), _np(layer["router_bias"], np.float64),
-                       K, shape.routed_scaling, forced)
+                       K, shape.routed_scaling, forced, topp)
     W13 = decode_int4(_np(layer["w13"], np.uint8)) * _np(layer["s13"], np.float64)[..., None]
     W2 = decode_int4(_np(layer["w2"], np.uint8)) * _np(layer["s2"], np.float64)[..., None]
     G = np.einsum("th,eih->tei", xf, W13[:, :I])

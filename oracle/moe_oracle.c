@@ -35,6 +35,14 @@
  *             every weight dequantised as code * row_scale
  *   out[t]  = sum_k w[t,k] * FFN_{e_k}(x_t) + FFN_shared(x_t) [+ x_t]
  *   (the shared expert has weight 1 and is not multiplied by `scale`).
+ * Adaptive expert top-p (opt-in; colibri README, "Quick start" knobs: "--topp
+ * 0.7 adaptive expert top-p"), 0 < p < 1: of the K selected experts, taken in
+ * decreasing score order (ties: lower expert index), an expert is kept while
+ * the scores of the experts kept before it sum to less than p times the
+ * scores of all K: the fewest highest-weight experts whose normalised weight
+ * reaches p.  Kept experts keep their selection order and are re-weighted
+ * over the kept set, w[t,k] = scale * s[t,e_k] / sum_{j kept} s[t,j]; the
+ * dropped picks become index -1 with weight 0, after the kept ones.
  * Int4 code layout: byte j of a row holds element 2j in bits 0..3 and element
  * 2j+1 in bits 4..7, each a 4-bit two's-complement value in [-8, 7].
  */
@@ -90,11 +98,58 @@ static int sel_cmp(const void* a, const void* b) {
     return (x->e < y->e) ? -1 : (x->e > y->e);
 }
 
+/* Adaptive top-p over the K picks idx[0..K) with the given scores (see the
+ * header): compacts the kept picks to the front, in their order, and writes
+ * their re-normalised weights; the rest become -1 / 0.  topp_margin (nullable)
+ * receives min over the picks of |cum_before - p * total| / total, how close
+ * the decision came to going the other way. */
+static void apply_topp(double topp, double scale, const double* scores, int K, int32_t* idx, double* wts,
+                       double* topp_margin) {
+    int ord[64], keep[64];
+    double total = 0.0;
+    for (int k = 0; k < K; ++k) {
+        ord[k] = k;
+        keep[k] = 0;
+        total += scores[idx[k]];
+    }
+    /* insertion sort of the picks by (score desc, expert index asc) */
+    for (int i = 1; i < K; ++i) {
+        int v = ord[i], j = i - 1;
+        while (j >= 0 && (scores[idx[ord[j]]] < scores[idx[v]] ||
+                          (scores[idx[ord[j]]] == scores[idx[v]] && idx[ord[j]] > idx[v]))) {
+            ord[j + 1] = ord[j];
+            --j;
+        }
+        ord[j + 1] = v;
+    }
+    double cum = 0.0, mm = INFINITY;
+    for (int j = 0; j < K; ++j) {
+        double d = fabs(cum - topp * total) / total;
+        if (d < mm) mm = d;
+        if (cum < topp * total) {
+            keep[ord[j]] = 1;
+            cum += scores[idx[ord[j]]];
+        }
+    }
+    int32_t kept_idx[64];
+    int n = 0;
+    for (int k = 0; k < K; ++k)
+        if (keep[k]) kept_idx[n++] = idx[k];
+    double denom = 0.0;
+    for (int k = 0; k < n; ++k) denom += scores[kept_idx[k]];
+    for (int k = 0; k < K; ++k) {
+        idx[k] = k < n ? kept_idx[k] : -1;
+        wts[k] = k < n ? scale * scores[kept_idx[k]] / denom : 0.0;
+    }
+    if (topp_margin) *topp_margin = mm;
+}
+
 /* Router of one token: logits, sigmoid scores, biased keys, top-K by a full
- * sort of (key desc, index asc), margin = key_(K) - key_(K+1), weights. */
+ * sort of (key desc, index asc), margin = key_(K) - key_(K+1), weights; then
+ * the adaptive top-p when 0 < topp < 1. */
 static int route_one(const double* xt, const float* W, const float* bias, int H, int E, int K,
-                     double scale, const int32_t* forced, double* logits, double* scores,
-                     int32_t* idx, double* wts, double* margin, sel_item* items) {
+                     double scale, double topp, const int32_t* forced, double* logits, double* scores,
+                     int32_t* idx, double* wts, double* margin, double* topp_margin, sel_item* items) {
     for (int e = 0; e < E; ++e) {
         double L = 0.0;
         const float* We = W + (int64_t)e * H;
@@ -109,14 +164,32 @@ static int route_one(const double* xt, const float* W, const float* bias, int H,
     }
     qsort(items, (size_t)E, sizeof(sel_item), sel_cmp);
     if (margin) *margin = (K < E) ? (items[K - 1].key - items[K].key) : INFINITY;
-    for (int k = 0; k < K; ++k) {
-        int32_t e = forced ? forced[k] : items[k].e;
-        if (e < 0 || e >= E) return ORC_EINVAL;
-        idx[k] = e;
+    if (topp_margin) *topp_margin = INFINITY;
+    if (forced) {
+        /* a forced selection as given (with -1 for picks the top-p dropped) */
+        int n = 0;
+        for (int k = 0; k < K; ++k) {
+            int32_t e = forced[k];
+            if (e == -1 && topp > 0.0 && topp < 1.0) {
+                idx[k] = -1;
+                continue;
+            }
+            if (e < 0 || e >= E) return ORC_EINVAL;
+            idx[k] = e;
+            ++n;
+        }
+        if (n == 0) return ORC_EINVAL;
+        double denom = 0.0;
+        for (int k = 0; k < K; ++k)
+            if (idx[k] >= 0) denom += scores[idx[k]];
+        for (int k = 0; k < K; ++k) wts[k] = idx[k] >= 0 ? scale * scores[idx[k]] / denom : 0.0;
+        return ORC_OK;
     }
+    for (int k = 0; k < K; ++k) idx[k] = items[k].e;
     double denom = 0.0;
     for (int k = 0; k < K; ++k) denom += scores[idx[k]];
     for (int k = 0; k < K; ++k) wts[k] = scale * scores[idx[k]] / denom;
+    if (topp > 0.0 && topp < 1.0) apply_topp(topp, scale, scores, K, idx, wts, topp_margin);
     return ORC_OK;
 }
 
@@ -141,12 +214,13 @@ int oracle_select_topk(const double* scores, const float* bias, int32_t T, int32
     return ORC_OK;
 }
 
-/* Router for T tokens.  x: bf16 bits [T,H]; W: f32 [E,H]; bias: f32 [E].
- * Outputs (row-major): logits/scores [T,E] (nullable), idx [T,K], weights
- * [T,K], margin [T] (nullable). */
+/* Router for T tokens.  x: bf16 bits [T,H]; W: f32 [E,H]; bias: f32 [E];
+ * topp: 0 = plain top-K, else the adaptive top-p.  Outputs (row-major):
+ * logits/scores [T,E] (nullable), idx [T,K], weights [T,K], margin [T] and
+ * topp_margin [T] (nullable). */
 int oracle_route(const uint16_t* x, const float* W, const float* bias, int32_t T, int32_t H,
-                 int32_t E, int32_t K, double scale, double* logits, double* scores,
-                 int32_t* idx, double* weights, double* margin) {
+                 int32_t E, int32_t K, double scale, double topp, double* logits, double* scores,
+                 int32_t* idx, double* weights, double* margin, double* topp_margin) {
     if (!x || !W || !bias || !idx || !weights || T < 0 || H <= 0 || E <= 0 || K <= 0 || K > E)
         return ORC_EINVAL;
     double* xt = (double*)malloc(sizeof(double) * (size_t)H);
@@ -155,9 +229,9 @@ int oracle_route(const uint16_t* x, const float* W, const float* bias, int32_t T
     int rc = (xt && sc && items) ? ORC_OK : ORC_ENOMEM;
     for (int32_t t = 0; rc == ORC_OK && t < T; ++t) {
         for (int h = 0; h < H; ++h) xt[h] = bf16_bits_to_double(x[(int64_t)t * H + h]);
-        rc = route_one(xt, W, bias, H, E, K, scale, NULL, logits ? logits + (int64_t)t * E : NULL,
+        rc = route_one(xt, W, bias, H, E, K, scale, topp, NULL, logits ? logits + (int64_t)t * E : NULL,
                        sc, idx + (int64_t)t * K, weights + (int64_t)t * K,
-                       margin ? margin + t : NULL, items);
+                       margin ? margin + t : NULL, topp_margin ? topp_margin + t : NULL, items);
         if (scores) memcpy(scores + (int64_t)t * E, sc, sizeof(double) * (size_t)E);
     }
     free(xt); free(sc); free(items);
@@ -192,11 +266,12 @@ int oracle_expert_ffn(const double* x, int32_t H, int32_t I, const uint8_t* w13,
  * w13 packed [E,2I,H/2]; s13 f32 [E,2I]; w2 packed [E,H,I/2]; s2 f32 [E,H];
  * sh_* the shared expert with intermediate Is (Is = 0: no shared expert).
  * idx_override [n,K] (nullable): evaluate with these experts instead of the
- * router's choice (weights still come from the router's scores).
- * Outputs: out double [n,H]; idx_out [n,K], w_out [n,K], margin_out [n]
- * (each nullable). */
+ * router's choice (weights still come from the router's scores; with top-p,
+ * -1 entries are dropped picks).  topp: 0 = plain top-K, else the adaptive
+ * top-p.  Outputs: out double [n,H]; idx_out [n,K], w_out [n,K], margin_out
+ * [n] (each nullable). */
 int oracle_moe_tokens(const uint16_t* x, int32_t T, int32_t H, int32_t E, int32_t K, int32_t I,
-                      int32_t Is, double scale, int32_t residual, const float* router_w,
+                      int32_t Is, double scale, double topp, int32_t residual, const float* router_w,
                       const float* router_bias, const uint8_t* w13, const float* s13,
                       const uint8_t* w2, const float* s2, const uint8_t* sh_w13,
                       const float* sh_s13, const uint8_t* sh_w2, const float* sh_s2,
@@ -221,14 +296,15 @@ int oracle_moe_tokens(const uint16_t* x, int32_t T, int32_t H, int32_t E, int32_
         if (t < 0 || t >= T) { rc = ORC_EINVAL; break; }
         for (int h = 0; h < H; ++h) xt[h] = bf16_bits_to_double(x[(int64_t)t * H + h]);
         double margin;
-        rc = route_one(xt, router_w, router_bias, H, E, K, scale,
+        rc = route_one(xt, router_w, router_bias, H, E, K, scale, topp,
                        idx_override ? idx_override + (int64_t)i * K : NULL, NULL, sc, idx, wts,
-                       &margin, items);
+                       &margin, NULL, items);
         if (rc != ORC_OK) break;
         double* o = out + (int64_t)i * H;
         for (int h = 0; h < H; ++h) o[h] = 0.0;
         for (int k = 0; k < K && rc == ORC_OK; ++k) {
             int32_t e = idx[k];
+            if (e < 0) continue; /* dropped by the top-p */
             rc = oracle_expert_ffn(xt, H, I, w13 + e * e13, s13 + (int64_t)e * 2 * I, w2 + e * e2,
                                    s2 + (int64_t)e * H, NULL, y);
             for (int h = 0; h < H; ++h) o[h] += wts[k] * y[h];

@@ -319,3 +319,72 @@ def test_sigmoid_saturation_finite():
     r = oracle.route(x, W, np.zeros(4, np.float32), 2, 1.0)
     assert np.all(np.isfinite(r["weights"]))
     assert r["idx"][0].tolist() == [0, 2]
+
+
+# --- adaptive expert top-p (opt-in) ---------------------------------------------
+
+def _route_with_scores(scores, K, scale=1.0, topp=0.0):
+    """oracle.route on one token whose sigmoid scores are (close to) `scores`:
+    x = [1, 0], router row e = [logit(s_e), 0], bias 0."""
+    s = np.asarray(scores, np.float64)
+    W = np.zeros((len(s), 2), np.float32)
+    W[:, 0] = np.log(s / (1.0 - s))
+    x = torch.tensor([[1.0, 0.0]]).to(torch.bfloat16)
+    return oracle.route(x, W, np.zeros(len(s), np.float32), K, scale, topp)
+
+
+def test_topp_hand_worked():
+    """Scores 0.5, 0.3, 0.2 (all three picked, K = 3): with p = 0.7 the two
+    best carry 0.8 >= 0.7 of the mass, so the third is dropped and the weights
+    become scale * (0.5, 0.3) / 0.8; with p = 0.45 the best alone reaches it;
+    with p = 0.81 all three are needed; p = 1 (or 0) is plain top-K."""
+    for p, kept, w in ((0.7, [0, 1], [0.625, 0.375]), (0.45, [0], [1.0]), (0.81, [0, 1, 2], [0.5, 0.3, 0.2]),
+                       (1.0, [0, 1, 2], [0.5, 0.3, 0.2]), (0.0, [0, 1, 2], [0.5, 0.3, 0.2])):
+        r = _route_with_scores([0.5, 0.3, 0.2], 3, scale=2.5, topp=p)
+        n = len(kept)
+        assert r["idx"][0, :n].tolist() == kept, (p, r["idx"])
+        assert np.all(r["idx"][0, n:] == -1) and np.all(r["weights"][0, n:] == 0.0)
+        np.testing.assert_allclose(r["weights"][0, :n], 2.5 * np.array(w), rtol=2e-6)
+
+
+def test_topp_brute_force_over_subsets():
+    """The kept picks are the smallest subset of the K picks whose scores reach
+    p of their total, the highest-mass one among subsets of that size (checked
+    against every subset), kept in selection order; their weights are
+    normalised over the kept set."""
+    rng = np.random.default_rng(11)
+    for trial in range(200):
+        E, K = 7, int(rng.integers(1, 6))
+        s = rng.uniform(0.05, 0.95, E)
+        p = float(rng.uniform(0.05, 0.99))
+        r = _route_with_scores(s, K, scale=1.3, topp=p)
+        sc = r["scores"][0]
+        picks = np.argsort(-sc, kind="stable")[:K]  # zero bias: the K best scores
+        total = sc[picks].sum()
+        best = None
+        for size in range(1, K + 1):
+            cands = [c for c in itertools.combinations(picks.tolist(), size) if sc[list(c)].sum() >= p * total]
+            if cands:
+                best = max(cands, key=lambda c: sc[list(c)].sum())
+                break
+        got = [e for e in r["idx"][0] if e >= 0]
+        assert set(got) == set(best), (trial, got, best)
+        assert got == [e for e in picks if e in set(best)]  # selection order kept
+        np.testing.assert_allclose(r["weights"][0, :len(got)], 1.3 * sc[got] / sc[got].sum(), rtol=1e-12)
+
+
+def test_topp_layer_matches_dense_formulation():
+    shape = workloads.LayerShape(H=32, E=8, K=4, I=16, Is=8, routed_scaling=2.5)
+    layer = workloads.make_layer(shape, 94, device="cpu")
+    layer["router_w"].mul_(20)  # a wide spread of scores, so the top-p drops picks
+    x = workloads.make_x(shape, 9, 94)
+    for p in (0.3, 0.6, 0.9):
+        r = oracle.moe_tokens(x, layer, shape, residual=True, topp=p)
+        assert np.any(r["idx"] == -1)
+        ref, R = dense_masked.moe_dense(x, layer, shape, residual=True, topp=p)
+        np.testing.assert_allclose(r["out"], ref, rtol=0, atol=1e-12 * np.abs(ref).max())
+        # the override path evaluates the same kept picks (-1 = dropped)
+        r2 = oracle.moe_tokens(x, layer, shape, residual=True, topp=p, idx_override=r["idx"])
+        np.testing.assert_array_equal(r2["out"], r["out"])
+    plain = oracle.moe_tokens(x, layer, shape, residual=True)
+    np.testing.assert_array_equal(oracle.moe_tokens(x, layer, shape, residual=True, topp=1.0)["out"], plain["out"])
