@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 /* Status codes. */
 #define MOE_OK 0
@@ -137,7 +137,16 @@ typedef struct moe_shared_weights {
  *   stage_events   : optional array of 2*MOE_NUM_STAGES cudaEvent_t handles
  *                    (created by the caller, e.g. with cudaEventCreate);
  *                    events [2s] and [2s+1] are recorded on `stream` before
- *                    and after stage s.  NULL = no recording. */
+ *                    and after stage s.  NULL = no recording.
+ *   topp           : adaptive expert top-p (colibri README, "Quick start"
+ *                    knobs, "--topp 0.7"): 0 (or >= 1) = plain top-K; for
+ *                    0 < topp < 1, of each token's K selected experts the
+ *                    fewest highest-scoring ones whose sigmoid scores reach
+ *                    topp of the K's total are kept (in selection order, at
+ *                    least one), re-weighted as routed_scaling * s /
+ *                    (sum of the kept s); the dropped picks are not computed
+ *                    and appear in topk_idx_out as -1 (weight 0) after the
+ *                    kept ones.  The keep decision is taken in f32. */
 typedef struct moe_cfg {
     uint32_t struct_size;
     int32_t H, E, K, I, Is;
@@ -148,6 +157,7 @@ typedef struct moe_cfg {
     int32_t* topk_idx_out;
     float* topk_w_out;
     void* const* stage_events;
+    float topp;
 } moe_cfg_t;
 
 /* Bytes of workspace moe_layer_forward needs for T tokens under `cfg`

@@ -87,7 +87,7 @@ class moe_cfg_t(ctypes.Structure):
                 ("routed_scaling", ctypes.c_float), ("flags", ctypes.c_uint32),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
                 ("topk_idx_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p),
-                ("stage_events", ctypes.c_void_p)]
+                ("stage_events", ctypes.c_void_p), ("topp", ctypes.c_float)]
 
 
 class moe_shared_weights_t(ctypes.Structure):
@@ -135,7 +135,7 @@ def _load() -> ctypes.CDLL:
     L.moe_stack_forward.restype = ctypes.c_int
     L.moe_stack_trace_offset.argtypes = [ctypes.POINTER(moe_cfg_t), ctypes.c_int32, ctypes.c_int32]
     L.moe_stack_trace_offset.restype = ctypes.c_size_t
-    if L.moe_abi_version() != 1:
+    if L.moe_abi_version() != 2:
         raise ImportError("libmoe_int4.so ABI version mismatch")
     return L
 
@@ -157,8 +157,9 @@ def _ptr(t: Optional[torch.Tensor]):
 
 def make_cfg(shape, flags: int = 0, workspace: Optional[torch.Tensor] = None,
              topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
-             stage_events=None) -> moe_cfg_t:
+             stage_events=None, topp: float = 0.0) -> moe_cfg_t:
     c = moe_cfg_t()
+    c.topp = float(topp)
     c.struct_size = ctypes.sizeof(moe_cfg_t)
     c.H, c.E, c.K, c.I, c.Is = shape.H, shape.E, shape.K, shape.I, shape.Is
     c.routed_scaling = float(shape.routed_scaling)
@@ -217,7 +218,7 @@ def _check_dev(name, t, dtype, shape=None):
 def layer_forward(x: torch.Tensor, layer: dict, shape, out: Optional[torch.Tensor] = None,
                   workspace: Optional[torch.Tensor] = None, flags: int = 0,
                   topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
-                  stream: Optional[torch.cuda.Stream] = None, stage_events=None) -> torch.Tensor:
+                  stream: Optional[torch.cuda.Stream] = None, stage_events=None, topp: float = 0.0) -> torch.Tensor:
     """Call ``moe_layer_forward`` on torch tensors (see include/moe_int4.h).
 
     ``layer`` holds router_w, router_bias, w13, s13, w2, s2 and, when
@@ -252,7 +253,7 @@ def layer_forward(x: torch.Tensor, layer: dict, shape, out: Optional[torch.Tenso
         _check_dev("topk_idx", topk_idx, torch.int32, (T, shape.K))
     if topk_w is not None:
         _check_dev("topk_w", topk_w, torch.float32, (T, shape.K))
-    cfg = make_cfg(shape, flags, workspace, topk_idx, topk_w, stage_events)
+    cfg = make_cfg(shape, flags, workspace, topk_idx, topk_w, stage_events, topp)
     s = stream if stream is not None else torch.cuda.current_stream(x.device)
     st = lib.moe_layer_forward(_ptr(x), _ptr(layer["router_w"]), _ptr(layer["router_bias"]),
                                _ptr(layer["w13"]), _ptr(layer["s13"]), _ptr(layer["w2"]),
@@ -287,7 +288,7 @@ def stack_path(shape, T: int, L: int, flags: int = 0) -> int:
 def stack_forward(x: torch.Tensor, stacked: dict, shape, outs: Optional[torch.Tensor] = None,
                   workspace: Optional[torch.Tensor] = None, flags: int = 0,
                   topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
-                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+                  stream: Optional[torch.cuda.Stream] = None, topp: float = 0.0) -> torch.Tensor:
     """Call ``moe_stack_forward`` on torch tensors: ``stacked`` holds the
     weights of L layers stacked along dimension 0 (see ``stack_layers``).
     Returns ``outs`` (bf16 [L, T, H]; outs[l] is layer l's output).
@@ -325,7 +326,7 @@ def stack_forward(x: torch.Tensor, stacked: dict, shape, outs: Optional[torch.Te
         _check_dev("topk_idx", topk_idx, torch.int32, (L, T, K))
     if topk_w is not None:
         _check_dev("topk_w", topk_w, torch.float32, (L, T, K))
-    cfg = make_cfg(shape, flags, workspace, topk_idx, topk_w)
+    cfg = make_cfg(shape, flags, workspace, topk_idx, topk_w, topp=topp)
     s = stream if stream is not None else torch.cuda.current_stream(x.device)
     st = lib.moe_stack_forward(_ptr(x), ctypes.byref(w), int(L), _ptr(outs), int(T), ctypes.byref(cfg),
                                ctypes.c_void_p(s.cuda_stream))

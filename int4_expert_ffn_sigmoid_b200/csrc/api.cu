@@ -108,6 +108,7 @@ int validate_cfg(const moe_cfg_t* c) {
     if (!c || c->struct_size != sizeof(moe_cfg_t)) return MOE_ERR_INVALID_ARG;
     if (c->H <= 0 || c->E <= 0 || c->K <= 0 || c->I <= 0 || c->Is < 0 || c->K > c->E) return MOE_ERR_INVALID_ARG;
     if (!(c->routed_scaling > 0.0f) || !isfinite(c->routed_scaling)) return MOE_ERR_INVALID_ARG;
+    if (!(c->topp >= 0.0f) || !isfinite(c->topp)) return MOE_ERR_INVALID_ARG;
     if (c->flags & ~kKnownFlags) return MOE_ERR_INVALID_ARG;
     if ((c->flags & MOE_FORCE_DECODE) && (c->flags & MOE_FORCE_PREFILL)) return MOE_ERR_INVALID_ARG;
     if (c->H % 128 || c->H > 16384) return MOE_ERR_UNSUPPORTED;
@@ -287,6 +288,7 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
     memset(&p, 0, sizeof p);
     p.T = T; p.H = cfg->H; p.E = cfg->E; p.K = cfg->K; p.I = cfg->I; p.Is = cfg->Is;
     p.scale = cfg->routed_scaling;
+    p.topp = cfg->topp;
     p.flags = cfg->flags;
     p.x = static_cast<const __nv_bfloat16*>(x);
     p.rw = router_w; p.rb = router_bias;
@@ -494,6 +496,7 @@ int moe_stack_forward(const void* x, const moe_stack_weights_t* w, int32_t L, vo
     a.r2_r = (cfg->H / a.rows2) * a.nsl_r;
     a.r2_s = (cfg->H / a.rows2) * a.nsl_s;
     a.scale = cfg->routed_scaling;
+    a.topp = cfg->topp;
     a.flags = cfg->flags;
     a.x = static_cast<const __nv_bfloat16*>(x);
     a.outs = static_cast<__nv_bfloat16*>(outs);

@@ -24,6 +24,7 @@ __global__ void __launch_bounds__(256) combine_kernel(Params p) {
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     for (int k = 0; k < K; ++k) {
         const int s = __ldcg(p.slot_of + (size_t)t * K + k);
+        if (s < 0) continue;  // a pick the top-p dropped
         const float w = __ldcg(p.wts + (size_t)t * K + k);
         float4 v = __ldcg(reinterpret_cast<const float4*>(p.y + (size_t)s * H + j));
         for (int sl = 1; sl < p.nsl_r; ++sl) {

@@ -181,7 +181,7 @@ __device__ __forceinline__ bool aborted(const Sh& sh) { return *reinterpret_cast
 // the lower index); the k-th pick's weight is scale * s_k / (s_0 + ... +
 // s_{K-1}), the sum taken in pick order.  Lanes k < K return pick k.
 __device__ __forceinline__ void select_warp(const float (&L)[kMaxE / 32], const float* bias, int E, int K, float scale,
-                                            int lane, int& my_e, float& my_w) {
+                                            float topp, int lane, int& my_e, float& my_w) {
     float key[kMaxE / 32], sc[kMaxE / 32];
 #pragma unroll
     for (int j = 0; j < kMaxE / 32; ++j) {
@@ -220,7 +220,8 @@ __device__ __forceinline__ void select_warp(const float (&L)[kMaxE / 32], const 
         if (lane == k) { my_e = be; my_s = bs; }
         ssum += bs;
     }
-    my_w = lane < K ? scale * my_s / ssum : 0.f;
+    const int e_k = my_e;
+    topp_picks(K, topp, scale, lane, e_k, my_s, ssum, my_e, my_w);
 }
 
 // Logits of the group's tokens t0 .. t0+nt-1 (all 256 consumer threads):
@@ -410,6 +411,7 @@ __device__ __forceinline__ void combine_block(const FArgs& a, const Sh& sh, int 
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
         for (int k = 0; k < a.K; ++k) {
             const int s = sh.slot_of[tok * a.K + k];
+            if (s < 0) continue;  // a pick the top-p dropped
             const float w = sh.wts[tok * a.K + k];
             float4 v = __ldcg(reinterpret_cast<const float4*>(a.y + (size_t)s * H + j));
             for (int sl = 1; sl < a.nsl_r; ++sl) {
@@ -522,7 +524,9 @@ __device__ void build_tables(const FArgs& a, Sh& sh) {
         if (i < TK) {
             e = __ldcg(a.idx + i);
             sh.wts[i] = __ldcg(a.wts + i);
-            if (e < 0 || e >= E) {
+            if (e == -1 && a.topp > 0.f && a.topp < 1.f) {
+                // dropped by the top-p: no slot
+            } else if (e < 0 || e >= E) {
                 atomicOr(a.status, ST_BAD_EXPERT);
                 e = -1;
             }
@@ -592,7 +596,8 @@ __device__ void build_tables(const FArgs& a, Sh& sh) {
         int nb = __shfl_sync(0xffffffffu, inc[1], 31);
         int t13 = __shfl_sync(0xffffffffu, inc[2], 31), t2 = __shfl_sync(0xffffffffu, inc[3], 31);
         if (lane == 0) {
-            if (total != TK) {  // inconsistent selections: flag them and run no routed task
+            const bool topp = a.topp > 0.f && a.topp < 1.f;  // dropped picks: fewer slots than T*K
+            if (total != TK && !(topp && total < TK)) {  // inconsistent selections: flag them and run no routed task
                 atomicOr(a.status, ST_BAD_COUNT);
                 nb = t13 = t2 = 0;
             }
@@ -629,7 +634,7 @@ __device__ void build_tables(const FArgs& a, Sh& sh) {
         }
         if (slot < 0 || slot >= TK) {
             if (e >= 0) atomicOr(a.status, ST_BAD_SLOT);
-            sh.slot_of[i] = 0;
+            sh.slot_of[i] = e == -1 && a.topp > 0.f && a.topp < 1.f ? -1 : 0;
         } else {
             sh.slot_of[i] = (short)slot;
             sh.tok_of_slot[slot] = (short)(i / K);
@@ -1030,7 +1035,7 @@ __device__ bool phase_units(const FArgs& a, Sh& sh, const Smem& m, int l) {
             for (int j = 0; j < kMaxE / 32; ++j) L[j] = lg[warp * kMaxE + lane + 32 * j];
             int e;
             float w;
-            select_warp(L, sh.bias[0], a.E, a.K, a.scale, lane, e, w);
+            select_warp(L, sh.bias[0], a.E, a.K, a.scale, a.topp, lane, e, w);
             if ((a.flags & kFlagTestBadIndex) && t == 0 && lane == 0) e = a.E;  // test hook: an out-of-range pick
             if (lane < a.K) {
                 const size_t o = (size_t)t * a.K + lane;
@@ -1046,7 +1051,7 @@ __device__ bool phase_units(const FArgs& a, Sh& sh, const Smem& m, int l) {
                 for (int j = 0; j < kMaxE / 32; ++j) L[j] = lg[(kGroupTok + warp) * kMaxE + lane + 32 * j];
                 int pe;
                 float pw;
-                select_warp(L, sh.bias[1], a.E, a.K, a.scale, lane, pe, pw);
+                select_warp(L, sh.bias[1], a.E, a.K, a.scale, a.topp, lane, pe, pw);
                 if (lane < a.K && pe >= 0 && pe < a.E) atomicOr(a.pred_bits + (l + 1) * 8 + (pe >> 5), 1u << (pe & 31));
             }
             if (warp == 0) stamp(a, l, 10);

@@ -229,7 +229,8 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
         int t13 = __shfl_sync(0xffffffffu, inc[2], 31), t2 = __shfl_sync(0xffffffffu, inc[3], 31);
         __syncwarp();
         if (lane == 0) {
-            if (total != TK) {  // inconsistent counts: flag them and run no routed task
+            const bool topp = p.topp > 0.f && p.topp < 1.f;  // dropped picks: fewer slots than T*K
+            if (total != TK && !(topp && total < TK)) {  // inconsistent counts: flag them and run no routed task
                 atomicOr(&p.ctrl->status, ST_BAD_COUNT);
                 nb = t13 = t2 = 0;
             }
@@ -264,6 +265,10 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
         const int i = tid < 256 ? tid + 256 * u : TK;
         if (i >= TK) continue;
         const int e = my_e[u], t = i / K;
+        if (e == -1 && p.topp > 0.f && p.topp < 1.f) {  // dropped by the top-p: no slot
+            if (writer) p.slot_of[i] = -1;
+            continue;
+        }
         int slot = -1;
         if (e >= 0 && e < E) slot = s_off[e] + s_base[(t / kDecodeRouterTok) * kMaxE + e] + my_rank[u];
         else atomicOr(&p.ctrl->status, ST_BAD_EXPERT);

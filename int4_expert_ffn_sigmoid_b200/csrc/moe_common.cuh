@@ -56,6 +56,48 @@ constexpr unsigned kFlagTestStall = 1u << 6;  // MOE_TEST_STALL
 constexpr unsigned kFlagTestBadIndex = 1u << 7;  // MOE_TEST_BAD_INDEX
 constexpr unsigned kFlagTrace = 1u << 8;      // MOE_TRACE
 
+// Adaptive expert top-p over the K picks of one token (one warp; lanes k < K
+// hold pick k: expert e_k and sigmoid score s_k; ssum is the K scores' sum).
+// A pick is kept when the scores of the picks ordered before it (score
+// descending, ties to the lower expert index) sum to less than p * ssum.
+// Returns on lane o < K the o-th kept pick (in pick order) with weight
+// scale * s / (sum of the kept s, added in pick order), and e = -1, w = 0 past
+// the kept ones.  p outside (0, 1): every pick, with weight scale * s / ssum.
+__device__ __forceinline__ void topp_picks(int K, float p, float scale, int lane, int my_e, float my_s, float ssum,
+                                           int& out_e, float& out_w) {
+    if (!(p > 0.f && p < 1.f)) {
+        out_e = lane < K ? my_e : -1;
+        out_w = lane < K ? scale * my_s / ssum : 0.f;
+        return;
+    }
+    float before = 0.f;
+    for (int j = 0; j < K; ++j) {
+        const float sj = __shfl_sync(0xffffffffu, my_s, j);
+        const int ej = __shfl_sync(0xffffffffu, my_e, j);
+        if (j != lane && (sj > my_s || (sj == my_s && ej < my_e))) before += sj;
+    }
+    const unsigned km = __ballot_sync(0xffffffffu, lane < K && before < p * ssum);
+    float kept = 0.f;
+    out_e = -1;
+    out_w = 0.f;
+    int pos = 0;
+    for (int j = 0; j < K; ++j) {
+        const float sj = __shfl_sync(0xffffffffu, my_s, j);
+        if ((km >> j) & 1u) kept += sj;
+    }
+    for (int j = 0; j < K; ++j) {
+        const float sj = __shfl_sync(0xffffffffu, my_s, j);
+        const int ej = __shfl_sync(0xffffffffu, my_e, j);
+        if ((km >> j) & 1u) {
+            if (pos == lane) {
+                out_e = ej;
+                out_w = scale * sj / kept;
+            }
+            ++pos;
+        }
+    }
+}
+
 // Device status bits (set by range checks, read back under MOE_DEBUG_CHECK).
 enum : unsigned {
     ST_BAD_EXPERT = 1u,  // a routing index outside [0, E)
@@ -122,6 +164,7 @@ static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
 struct Params {
     int T, H, E, K, I, Is;
     float scale;
+    float topp;  // adaptive expert top-p (0: off); dropped picks are index -1
     unsigned flags;
     const __nv_bfloat16* x;
     const float* rw;

@@ -31,6 +31,7 @@ struct FArgs {
     int r13_r, r13_s;      // gate/up tasks per 16-token chunk of a routed / the shared bucket
     int r2_r, r2_s;        // down tasks per 16-token chunk of a routed / the shared bucket
     float scale;
+    float topp;            // adaptive expert top-p (0: off); dropped picks are index -1
     unsigned flags;
     const __nv_bfloat16* x;  // [T][H], layer 0's input
     __nv_bfloat16* outs;     // [L][T][H]

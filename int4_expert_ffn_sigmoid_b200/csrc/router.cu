@@ -122,16 +122,18 @@ __device__ int select_from_logits(const Params& p, int t, const float (&L)[kMaxE
         if (lane == k) { my_e = be; my_s = bs; }
         ssum += bs;
     }
-    if ((p.flags & kFlagTestBadIndex) && t == 0 && lane == 0) my_e = E;  // test hook: an out-of-range pick
+    int out_e;
+    float w;
+    topp_picks(K, p.topp, p.scale, lane, my_e, my_s, ssum, out_e, w);
+    if ((p.flags & kFlagTestBadIndex) && t == 0 && lane == 0) out_e = E;  // test hook: an out-of-range pick
     if (lane < K) {
-        const float w = p.scale * my_s / ssum;
         const size_t o = (size_t)t * K + lane;
-        p.idx[o] = my_e;
+        p.idx[o] = out_e;
         p.wts[o] = w;
-        if (p.topk_idx_out) p.topk_idx_out[o] = my_e;
+        if (p.topk_idx_out) p.topk_idx_out[o] = out_e;
         if (p.topk_w_out) p.topk_w_out[o] = w;
     }
-    return lane < K ? my_e : -1;
+    return lane < K ? out_e : -1;
 }
 
 // select_from_logits with the token's logits in shared memory.
@@ -223,7 +225,9 @@ __device__ void finalize_buckets(const Params& p, const int* s_cnt, int* s_off) 
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        if (s_total != p.T * p.K) atomicOr(&p.ctrl->status, ST_BAD_COUNT);
+        // (under the top-p, dropped picks make fewer slots than T*K)
+        const bool topp = p.topp > 0.f && p.topp < 1.f;
+        if (s_total != p.T * p.K && !(topp && s_total < p.T * p.K)) atomicOr(&p.ctrl->status, ST_BAD_COUNT);
         int nb = s_nb;
         if (p.Is > 0) {
             p.bucket_e[nb] = E;
@@ -856,9 +860,12 @@ __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int t0 = tile * kRouterTileTokens;
         const int n = min(kRouterTileTokens, p.T - t0) * K;
+        const bool topp = p.topp > 0.f && p.topp < 1.f;
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
             int e = p.idx[(size_t)t0 * K + i];
-            if (e < 0 || e >= E) {
+            if (e == -1 && topp) {
+                e = -2;  // dropped by the top-p: no slot
+            } else if (e < 0 || e >= E) {
                 atomicOr(&p.ctrl->status, ST_BAD_EXPERT);
                 e = -1;
             }
@@ -872,6 +879,11 @@ __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
                 int rank = 0;
                 for (int j = 0; j < i; ++j) rank += (s_idx[j] == e);
                 slot = s_base[e] + rank;
+            }
+            if (e == -2) {  // dropped by the top-p
+                p.slot_of[(size_t)t0 * K + i] = -1;
+                s_slot[i] = -1;
+                continue;
             }
             if (slot < 0 || slot >= TK) {
                 atomicOr(&p.ctrl->status, ST_BAD_SLOT);

@@ -47,37 +47,57 @@ def to_cpu_layer(layer: dict) -> dict:
     return {k: v.detach().cpu() for k, v in layer.items()}
 
 
-def check_routing(idx_gpu: np.ndarray, w_gpu: np.ndarray, ref: dict, bias: np.ndarray, K: int):
-    """Returns (tie token indices, max weight rel error over non-tie tokens)."""
+def check_routing(idx_gpu: np.ndarray, w_gpu: np.ndarray, ref: dict, bias: np.ndarray, K: int,
+                  topp: float = 0.0):
+    """Returns (tie token indices, max weight rel error over non-tie tokens).
+
+    With the adaptive top-p (0 < topp < 1) each row holds the kept picks and
+    then -1 entries (weight 0).  A token is also a tie when its top-p decision
+    came within 1e-6 of the score sum of going the other way (the kernels take
+    it in f32); for such tokens the kept picks must be the oracle's kept ones,
+    possibly plus or minus the one at the boundary."""
     T = idx_gpu.shape[0]
     margin = ref["margin"]
     keys = ref["scores"] + bias.astype(np.float64)[None, :]
-    ties = np.nonzero(margin < TIE_MARGIN)[0]
-    non = np.ones(T, bool)
-    non[ties] = False
-    sg = np.sort(idx_gpu, axis=1)
-    so = np.sort(ref["idx"], axis=1)
+    use_topp = 0.0 < topp < 1.0
+    tie = margin < TIE_MARGIN
+    if use_topp:
+        tie |= ref["topp_margin"] < TIE_MARGIN
+    ties = np.nonzero(tie)[0]
+    non = ~tie
+    # dropped picks (-1) come after the kept ones
+    kept = idx_gpu >= 0
+    assert np.all(kept[:, 0]), "a token with no expert"
+    assert np.all(kept[:, :-1] | ~kept[:, 1:]), "a dropped pick before a kept one"
+    if not use_topp:
+        assert np.all(kept), "-1 entries without the top-p"
+    assert np.all(w_gpu[~kept] == 0.0)
+    big = np.iinfo(np.int32).max
+    sg = np.sort(np.where(kept, idx_gpu, big), axis=1)
+    so = np.sort(np.where(ref["idx"] >= 0, ref["idx"], big), axis=1)
     bad = np.nonzero(non & np.any(sg != so, axis=1))[0]
     assert bad.size == 0, (f"{bad.size} non-tie tokens select different experts; first {bad[:5]}: "
                            f"gpu {idx_gpu[bad[:3]]} oracle {ref['idx'][bad[:3]]} margin {margin[bad[:3]]}")
     for t in ties:
-        sel = idx_gpu[t]
-        assert len(set(sel.tolist())) == K, (t, sel)
+        sel = idx_gpu[t][kept[t]]
+        assert len(set(sel.tolist())) == len(sel), (t, sel)
         kth = np.sort(keys[t])[::-1][K - 1]
         assert np.all(keys[t, sel] >= kth - TIE_MARGIN), (t, sel, keys[t, sel], kth)
-    # the documented order of topk_idx_out: decreasing s + bias (two selected
-    # experts whose keys agree to within rounding may come in either order)
-    sel_keys = np.take_along_axis(keys, idx_gpu.astype(np.int64), axis=1)
+    # the documented order of topk_idx_out: decreasing s + bias over the kept
+    # picks (two selected experts whose keys agree to within rounding may come
+    # in either order)
+    sel_keys = np.where(kept, np.take_along_axis(keys, np.maximum(idx_gpu, 0).astype(np.int64), axis=1), -1e300)
     drop = sel_keys[:, :-1] - sel_keys[:, 1:]
-    bad = np.nonzero(np.any(drop < -TIE_MARGIN, axis=1))[0]
+    bad = np.nonzero(np.any((drop < -TIE_MARGIN) & kept[:, 1:], axis=1))[0]
     assert bad.size == 0, f"selection not in decreasing key order at tokens {bad[:5]}: {sel_keys[bad[:3]]}"
     werr = 0.0
     if non.any():
-        og = np.argsort(idx_gpu, axis=1)
-        oo = np.argsort(ref["idx"], axis=1)
+        og = np.argsort(np.where(kept, idx_gpu, big), axis=1)
+        oo = np.argsort(np.where(ref["idx"] >= 0, ref["idx"], big), axis=1)
         wg = np.take_along_axis(w_gpu, og, axis=1)[non]
         wo = np.take_along_axis(ref["weights"], oo, axis=1)[non]
-        werr = float(np.max(np.abs(wg - wo) / np.abs(wo)))
+        m = wo > 0
+        werr = float(np.max(np.abs(wg[m] - wo[m]) / np.abs(wo[m])))
         assert werr <= W_RTOL, f"routing weight relative error {werr:.3e} > {W_RTOL}"
     return ties, werr
 
@@ -96,7 +116,7 @@ def bf16_round(ref: np.ndarray) -> np.ndarray:
 
 
 def oracle_tokens(x, layer_cpu: dict, shape, residual: bool, tokens: np.ndarray, idx_override: np.ndarray,
-                  threads: int = 0) -> np.ndarray:
+                  threads: int = 0, topp: float = 0.0) -> np.ndarray:
     """The oracle's output for `tokens` (with the given selections), the
     tokens split over host threads (the oracle is plain C called through
     ctypes, which releases the interpreter lock; it keeps no state between
@@ -107,12 +127,12 @@ def oracle_tokens(x, layer_cpu: dict, shape, residual: bool, tokens: np.ndarray,
     threads = threads or max(1, min(16, os.cpu_count() or 1))
     if n <= 8 or threads == 1:
         return oracle.moe_tokens(x, layer_cpu, shape, residual=residual, tokens=tokens.astype(np.int32),
-                                 idx_override=idx_override)["out"]
+                                 idx_override=idx_override, topp=topp)["out"]
     parts = np.array_split(np.arange(n), min(threads, n))
 
     def run(sel):
         return oracle.moe_tokens(x, layer_cpu, shape, residual=residual, tokens=tokens[sel].astype(np.int32),
-                                 idx_override=idx_override[sel])["out"]
+                                 idx_override=idx_override[sel], topp=topp)["out"]
 
     with concurrent.futures.ThreadPoolExecutor(len(parts)) as ex:
         outs = list(ex.map(run, parts))
@@ -120,18 +140,19 @@ def oracle_tokens(x, layer_cpu: dict, shape, residual: bool, tokens: np.ndarray,
 
 
 def compare_layer(x: torch.Tensor, out: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, layer_cpu: dict,
-                  shape, residual: bool, sample=None, tol: float = OUT_TOL, rounded: bool = False) -> dict:
+                  shape, residual: bool, sample=None, tol: float = OUT_TOL, rounded: bool = False,
+                  topp: float = 0.0) -> dict:
     """Full comparison.  Routing is checked on every token; outputs on
     ``sample`` (token indices; default all).  ``rounded``: compare with the
     correctly rounded bf16 result instead of the exact one."""
     xc = x.detach().cpu()
-    ref_r = oracle.route(xc, layer_cpu["router_w"], layer_cpu["router_bias"], shape.K, shape.routed_scaling)
+    ref_r = oracle.route(xc, layer_cpu["router_w"], layer_cpu["router_bias"], shape.K, shape.routed_scaling, topp)
     idx_g = idx.detach().cpu().numpy()
     w_g = w.detach().cpu().numpy().astype(np.float64)
-    ties, werr = check_routing(idx_g, w_g, ref_r, layer_cpu["router_bias"].numpy(), shape.K)
+    ties, werr = check_routing(idx_g, w_g, ref_r, layer_cpu["router_bias"].numpy(), shape.K, topp)
     T = x.shape[0]
     tok = np.arange(T) if sample is None else np.unique(np.asarray(sample, np.int64))
-    ref = oracle_tokens(xc, layer_cpu, shape, residual, tok, np.ascontiguousarray(idx_g[tok]))
+    ref = oracle_tokens(xc, layer_cpu, shape, residual, tok, np.ascontiguousarray(idx_g[tok]), topp=topp)
     o = out[torch.from_numpy(tok).to(out.device)]
     err = rel_l2(o, ref, bf16_round(ref) if rounded else None)
     assert np.all(np.isfinite(err)), "non-finite output"
@@ -156,7 +177,7 @@ def tile_cover(idx: np.ndarray, E: int, tile: int, shared: bool) -> np.ndarray:
     order = np.argsort(flat, kind="stable")  # (t, k) order within each expert
     se, st = flat[order], tok[order]
     start = np.searchsorted(se, np.arange(E))
-    unit_of = np.empty(T * K, np.int64)  # unit id of each (t, k) pick
+    unit_of = np.full(T * K, -1, np.int64)  # unit id of each (t, k) pick (-1: a pick the top-p dropped)
     units_first = []
     uid = 0
     for e in range(E):
@@ -173,7 +194,8 @@ def tile_cover(idx: np.ndarray, E: int, tile: int, shared: bool) -> np.ndarray:
 
     def take(t):
         chosen.append(t)
-        covered[picks_of[t]] = True
+        u = picks_of[t]
+        covered[u[u >= 0]] = True
         if shared:
             covered[n_routed + t // tile] = True
 

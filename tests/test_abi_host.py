@@ -44,6 +44,7 @@ def test_struct_layout_matches_c(moe, tmp_path):
         " offsetof(moe_cfg_t, routed_scaling), offsetof(moe_cfg_t, flags),"
         " offsetof(moe_cfg_t, workspace), offsetof(moe_cfg_t, workspace_bytes),"
         " offsetof(moe_cfg_t, topk_w_out), sizeof(moe_shared_weights_t));"
+        " printf(\"%zu \", offsetof(moe_cfg_t, topp));"
         " printf(\"%zu %zu %zu\\n\", sizeof(moe_stack_weights_t), offsetof(moe_stack_weights_t, s2),"
         " offsetof(moe_stack_weights_t, shared)); return 0;}\n")
     exe = tmp_path / "layout"
@@ -52,6 +53,7 @@ def test_struct_layout_matches_c(moe, tmp_path):
     cfg = moe.moe_cfg_t
     py_vals = [ctypes.sizeof(cfg), cfg.routed_scaling.offset, cfg.flags.offset, cfg.workspace.offset,
                cfg.workspace_bytes.offset, cfg.topk_w_out.offset, ctypes.sizeof(moe.moe_shared_weights_t),
+               cfg.topp.offset,
                ctypes.sizeof(moe.moe_stack_weights_t), moe.moe_stack_weights_t.s2.offset,
                moe.moe_stack_weights_t.shared.offset]
     assert c_vals == py_vals
@@ -71,7 +73,7 @@ def test_header_constants_match_binding(moe):
 
 
 def test_version_and_strings(moe):
-    assert moe.lib.moe_abi_version() == 1
+    assert moe.lib.moe_abi_version() == 2
     assert moe.status_str(0) == "MOE_OK"
     assert moe.status_str(3) == "MOE_ERR_WORKSPACE"
     assert moe.status_str(99) == "MOE_ERR_UNKNOWN"
@@ -181,6 +183,14 @@ def test_forward_validation_codes(moe):
     assert _call(moe, _shape(K=5, E=4)) == moe.MOE_ERR_INVALID_ARG
     assert _call(moe, _shape(routed_scaling=0.0)) == moe.MOE_ERR_INVALID_ARG
     assert _call(moe, s, flags=1 << 12) == moe.MOE_ERR_INVALID_ARG  # an unknown flag
+
+    def topp(v):
+        def patch(c):
+            c.topp = v
+        return patch
+    assert _call(moe, s, cfg_patch=topp(float("nan"))) == moe.MOE_ERR_INVALID_ARG
+    assert _call(moe, s, cfg_patch=topp(-0.5)) == moe.MOE_ERR_INVALID_ARG
+    assert _call(moe, s, cfg_patch=topp(0.7)) == 0
     assert _call(moe, s, flags=moe.MOE_FORCE_DECODE | moe.MOE_FORCE_PREFILL) == moe.MOE_ERR_INVALID_ARG
 
     def bad_size(c):
