@@ -388,10 +388,10 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
     if (err == cudaSuccess) err = mark(2 * MOE_STAGE_ROUTE + 1);
     int tc_grid1 = 0, tc_grid2 = 0;
     if (use_tc) {
-        const long long mt_routed = (cfg->E < TK ? cfg->E : TK) + cdiv(TK, 128);
-        const long long mt_shared = cfg->Is > 0 ? cdiv(T, 128) : 0;
-        const long long t1 = mt_routed * (cfg->I / 128) + mt_shared * (cfg->Is / 128);
-        const long long t2 = (mt_routed + mt_shared) * (cfg->H / 256);
+        const long long mt_routed = (cfg->E < TK ? cfg->E : TK) + cdiv(TK, kTcTokens);
+        const long long mt_shared = cfg->Is > 0 ? cdiv(T, kTcTokens) : 0;
+        const long long t1 = mt_routed * (cfg->I / kTcFeat1) + mt_shared * (cfg->Is / kTcFeat1);
+        const long long t2 = (mt_routed + mt_shared) * (cfg->H / kTcFeat2);
         const int sms = sm_count();
         tc_grid1 = (int)(t1 < sms ? t1 : sms);
         tc_grid2 = (int)(t2 < sms ? t2 : sms);

@@ -10,20 +10,29 @@
 // batch is read once and applied to all of its tokens); nanocolibri-engine
 // README, "Converting a checkpoint yourself": per-row symmetric int4, f32 scales.
 //
-// Tile: 128 tokens (MMA M, one TMEM lane per token) x 256 output columns (MMA
-// N) x 64 reduction elements per pipeline stage.  Two rings: TMA stages hold
-// the activation and raw int4 tiles of 6 k blocks; 2 slots hold the
-// dequantised B operand between the dequantisers and the MMA.  GEMM-1's 256 columns are 128
-// gate rows and the 128 up rows of the same features, so one thread of the
-// epilogue holds gate and up of one (token, feature) pair.
-// Roles (448 threads):
-//   warp 0      TMA producer (activation tile, raw int4 weight tile) and TMEM owner
-//   warp 1      MMA issuer (one thread, tcgen05.mma kind::f16, M=128 N=256 K=16)
-//   warps 2-9   dequantisers, one B row per thread: raw int4 -> exact 16-bit
-//               integers in the 128-byte swizzled K-major layout of the B
-//               operand (the row scale is applied in the epilogue)
-//   warps 10-13 epilogue: tcgen05.ld of the accumulator, scales (staged in
-//               shared memory per tile), SwiGLU, stores
+// Tile: 128 tokens (MMA M, one TMEM lane per token) x 256 weight rows (MMA N)
+// x 64 reduction elements per pipeline stage.  Tokens are the A operand and
+// the dequantised weights the B operand, both in shared memory (128-byte
+// swizzle).  A tile spans 256 weight rows because the loads from L2 bound the
+// kernel: per k block it moves 16 KiB of tokens and 8 KiB of raw int4 for
+// 128 x 256 x 64 multiply-adds, twice the weight rows per token byte of a
+// 128-row tile.  GEMM-1's 256 rows are 128 gate rows and the 128 up rows of
+// the same features, so one epilogue thread holds gate and up of a (token,
+// feature) pair.  Two rings: TMA stages hold the token and raw int4 tiles of
+// TSTAGES k blocks; BSTAGES slots hold the dequantised B operand.
+// Roles (864 threads):
+//   warp 0       TMA producer (token tile, raw int4 tile) and TMEM owner
+//   warp 1       MMA issuer (one thread, tcgen05.mma kind::f16, M=128 N=256 K=16)
+//   warps 2-17   dequantisers, two groups of eight warps: group g takes the k
+//                blocks n = g mod 2 of the CTA's sequence (B slot n mod 3),
+//                one B row per thread: raw int4 -> exact 16-bit integers in
+//                the swizzled K-major layout (the row scale is applied in the
+//                epilogue)
+//   warp 18      staging: each tile's token rows, h-scale factors and weight
+//                row scales into shared memory, a tile or two ahead
+//   warps 19-26  epilogue: the warp of lane quarter q and column half c reads
+//                tokens 32q..32q+31 and half c of the tile's columns
+//                (tcgen05.ld), scales, SwiGLU, stores
 // Every mbarrier wait is bounded (clock64); on timeout the CTA records
 // ST_TIMEOUT in the status word and stops.  The drains then ignore the abort
 // (each with its own bound): the producer waits until every TMA copy it issued
@@ -38,50 +47,80 @@
 namespace moe {
 namespace tc {
 
-constexpr int BM = 128, BN = 256, BK = 64;
-// Two rings: TMA stages (activation tile + raw int4 tile) run TSTAGES k
-// blocks ahead to cover load latency; the dequantised B operand needs only
-// BSTAGES slots between the dequantisers and the MMA.
-constexpr int TSTAGES = 6;
-constexpr int BSTAGES = 2;
-constexpr int A_BYTES = BM * BK * 2;    // 16 KiB, bf16/fp16 activations
+constexpr int BM = 128;  // tokens per tile (A rows, TMEM lanes)
+constexpr int BN = 256;  // weight rows per tile (B rows, accumulator columns)
+constexpr int BK = 64;   // reduction elements per stage
+static_assert(BM == kTcTokens && BN == 2 * kTcFeat1 && BN == kTcFeat2, "tile geometry");
+constexpr int TSTAGES = 5;
+constexpr int BSTAGES = 3;
+constexpr int A_BYTES = BM * BK * 2;    // 16 KiB, bf16/fp16 tokens
 constexpr int B_BYTES = BN * BK * 2;    // 32 KiB, dequantised weights
 constexpr int RAW_BYTES = BN * BK / 2;  // 8 KiB, packed int4 weights
 constexpr int TSTAGE_BYTES = A_BYTES + RAW_BYTES;
 constexpr int RING_BYTES = TSTAGES * TSTAGE_BYTES + BSTAGES * B_BYTES;
-constexpr int DEQ_WARPS = 8;
-constexpr int NUM_THREADS = 64 + 32 * DEQ_WARPS + 128;
-constexpr int TMEM_COLS = 512;          // two 256-column accumulators
+constexpr int DEQ_GROUPS = 2;
+constexpr int DEQ_WARPS = 8 * DEQ_GROUPS;
+constexpr int EPI_WARPS = 8;
+constexpr int WARP_STAGE = 2 + DEQ_WARPS;
+constexpr int WARP_EPI0 = WARP_STAGE + 1;
+constexpr int NUM_THREADS = 32 * (WARP_EPI0 + EPI_WARPS);
+constexpr int TMEM_COLS = 512;  // two 256-column accumulators
 constexpr long long kTimeoutCycles = 4000000000LL;
 constexpr long long kDrainCycles = 200000000LL;
 // MOE_TEST_STALL: the epilogue first waits this long on a barrier nothing
 // arrives on (~1 ms), which makes the CTA take its timeout path while its
 // copies and MMAs are in flight.
 constexpr long long kStallCycles = 1LL << 21;
-constexpr int SMEM_BYTES = RING_BYTES + 1024 + 1280;
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of the grouped GEMM");
+
+// Per-tile data of the epilogue, written by the staging warp.
+struct Stage {
+    int slot[BM];   // output row of each token (h row / y slot), -1 past the tile
+    float fac[BM];  // per-token factor of the h storage scale (2^-k for GEMM-1, 2^k for GEMM-2)
+    float sc[BN];   // scale of each weight row of the tile
+};
 
 struct Shared {
-    uint64_t full_tma[TSTAGES];  // activation + raw tiles landed (TMA transaction count)
-    uint64_t empty_t[TSTAGES];   // MMA done with the activation tile, dequantisers with the raw tile
-    uint64_t full_deq[BSTAGES];  // B operand dequantised (one arrival per dequant warp)
-    uint64_t empty_b[BSTAGES];   // MMA done with the B operand
+    uint64_t full_tma[TSTAGES];  // token + raw tiles landed (TMA transaction count)
+    uint64_t empty_t[TSTAGES];   // MMA done with the token tile, a dequantiser group with the raw tile
+    uint64_t full_b[BSTAGES];    // B slot written (one arrival per warp of its group)
+    uint64_t empty_b[BSTAGES];   // MMA done with the B slot
     uint64_t acc_full[2];
-    uint64_t acc_empty[2];
+    uint64_t acc_empty[2];       // one arrival per epilogue warp
+    uint64_t stage_full[2];      // one arrival per staging lane
+    uint64_t stage_empty[2];     // one arrival per epilogue warp
     uint64_t drain;
     uint64_t never;  // nothing arrives on it (MOE_TEST_STALL)
     uint32_t tmem_base;
     int abort_flag;
-    float ep_scale[BN];  // the current tile's row scales (epilogue)
-    int ep_ok[4];        // per epilogue warp: its accumulator wait succeeded
+    alignas(16) Stage stage[2];
 };
-static_assert(sizeof(Shared) <= 1280, "shared control block");
-
-// Barrier among the 4 epilogue warps only.
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+constexpr int SMEM_BYTES = RING_BYTES + 1024 + (int)((sizeof(Shared) + 127) / 128 * 128);
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of the grouped GEMM");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Shared-memory accesses by 32-bit shared address (the tiles sit behind a
+// runtime 1024-byte alignment, which generic pointers would not let the
+// compiler see as shared).
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float4 lds128f(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ int lds32(uint32_t a) {
+    int v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -122,6 +161,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Shared
     }
 }
 
+// Every lane of the warp waits (each then observes the phase and what it
+// releases); the warp goes on only if every lane's wait succeeded.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Shared* sh) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, sh)) != 0;
+}
+
 // Bounded wait that ignores the abort flag: the drains after an abort, which
 // must see the CTA's own copies and MMAs complete before its shared memory
 // and tensor memory go away.  Returns false only when `limit` runs out.
@@ -155,6 +200,8 @@ __host__ __device__ constexpr uint32_t idesc_f16(int fmt, int M, int N) {
            ((uint32_t)(M >> 4) << 24);
 }
 
+// D (tensor memory) += A (shared memory descriptor, 128 x 16) * B (shared
+// memory descriptor, N x 16).
 __device__ __forceinline__ void mma_f16_ss(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                            uint32_t accumulate) {
     asm volatile(
@@ -188,22 +235,23 @@ __device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, uint32_t (&r)[16]
 // in natural order: out[j] = (element 2j, element 2j+1), by the exponent-bias
 // technique of Kim et al. (2022): (c + 8) in the low mantissa bits of 2^m,
 // minus 2^m + 8.  magic = 2^m in both halves, bias = 2^m + 8 in both halves.
+// The code c + 8 is the nibble with its top bit flipped, so one AND-XOR gives
+// the biased code and the exponent together.
 template <bool kBf16>
-__device__ __forceinline__ void int4x8_natural(uint32_t w, uint32_t (&o)[4]) {
-    const uint32_t v = w ^ 0x88888888u;
-    const uint32_t v4 = v >> 4;
+__device__ __forceinline__ void int4x8_natural(uint32_t w, uint32_t* o) {
+    const uint32_t w4 = w >> 4;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        // byte j of v (low nibble = element 2j) into half 0, byte j of v>>4
+        // byte j of w (low nibble = element 2j) into half 0, byte j of w>>4
         // (low nibble = element 2j+1) into half 1
-        const uint32_t t = __byte_perm(v, v4, j | ((4 + j) << 8)) & 0x000F000Fu;
+        const uint32_t t = __byte_perm(w, w4, j | ((4 + j) << 8));
         if (kBf16) {
-            uint32_t u = t | 0x43004300u;
+            uint32_t u = (t & 0x000F000Fu) ^ 0x43084308u;
             __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&u),
                                        __halves2bfloat162(__ushort_as_bfloat16(0x4308), __ushort_as_bfloat16(0x4308)));
             o[j] = *reinterpret_cast<uint32_t*>(&r);
         } else {
-            uint32_t u = t | 0x64006400u;
+            uint32_t u = (t & 0x000F000Fu) ^ 0x64086408u;
             __half2 r = __hsub2(*reinterpret_cast<__half2*>(&u),
                                 __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408)));
             o[j] = *reinterpret_cast<uint32_t*>(&r);
@@ -215,14 +263,17 @@ struct Tile {
     int shared;   // 1: shared expert
     int e;        // expert id (E for shared)
     int n_valid;  // valid tokens in this tile
-    int a_row;    // first activation row (TMA y coordinate)
-    int slot0;    // first output row of the tile (h row / y slot)
-    int col0;     // first output column (GEMM-1: feature j0; GEMM-2: feature n0)
+    int slot0;    // first token row of the tile (TMA y coordinate of the token map; h row / y slot)
+    int col0;     // GEMM-1: first feature of the tile (128 of them); GEMM-2: first output feature (256)
     int nkb;      // k blocks
 };
 
+// Tiles of a launch: the shared expert's first (token tile mt, feature block
+// ft: index ft * mt_s + mt), then every routed bucket's (local index
+// ft * mtiles + mt, buckets in order, tstart the prefix of their counts).
 __device__ __forceinline__ Tile decode_tile(const TcArgs& a, int tile) {
     Tile t;
+    const int fw = a.gemm == 1 ? kTcFeat1 : kTcFeat2;
     const int mt_s = a.Is > 0 ? (a.T + BM - 1) / BM : 0;
     const int n_sh = mt_s * a.ntile_s;
     if (tile < n_sh) {
@@ -230,9 +281,8 @@ __device__ __forceinline__ Tile decode_tile(const TcArgs& a, int tile) {
         t.shared = 1;
         t.e = a.E;
         t.n_valid = min(BM, a.T - mt * BM);
-        t.a_row = mt * BM;
         t.slot0 = mt * BM;
-        t.col0 = nt * (a.gemm == 1 ? BN / 2 : BN);
+        t.col0 = nt * fw;
         t.nkb = a.kdim_s / BK;
         return t;
     }
@@ -251,9 +301,8 @@ __device__ __forceinline__ Tile decode_tile(const TcArgs& a, int tile) {
     t.shared = 0;
     t.e = __ldg(a.bucket_e + lo);
     t.n_valid = min(BM, n - mt * BM);
-    t.a_row = off + mt * BM;
     t.slot0 = off + mt * BM;
-    t.col0 = nt * (a.gemm == 1 ? BN / 2 : BN);
+    t.col0 = nt * fw;
     t.nkb = a.kdim_r / BK;
     return t;
 }
@@ -265,13 +314,13 @@ __device__ __forceinline__ int total_tiles(const TcArgs& a) {
 
 template <int GEMM>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
-                    const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_constant__ CUtensorMap tmX_s,
+                    const __grid_constant__ CUtensorMap tmW_r, const __grid_constant__ CUtensorMap tmW_s,
                     const TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Shared* sh = reinterpret_cast<Shared*>(smem + RING_BYTES);
-    auto a_tile = [&](int s) { return smem + s * TSTAGE_BYTES; };
+    auto x_tile = [&](int s) { return smem + s * TSTAGE_BYTES; };
     auto raw_tile = [&](int s) { return smem + s * TSTAGE_BYTES + A_BYTES; };
     auto b_tile = [&](int s) { return smem + TSTAGES * TSTAGE_BYTES + s * B_BYTES; };
 
@@ -279,15 +328,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
     if (threadIdx.x == 0) {
         for (int s = 0; s < TSTAGES; ++s) {
             mbar_init(&sh->full_tma[s], 1);
-            mbar_init(&sh->empty_t[s], 1 + DEQ_WARPS);
+            mbar_init(&sh->empty_t[s], 1 + 8);
         }
         for (int s = 0; s < BSTAGES; ++s) {
-            mbar_init(&sh->full_deq[s], DEQ_WARPS);
+            mbar_init(&sh->full_b[s], 8);
             mbar_init(&sh->empty_b[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sh->acc_full[b], 1);
-            mbar_init(&sh->acc_empty[b], 4);
+            mbar_init(&sh->acc_empty[b], EPI_WARPS);
+            mbar_init(&sh->stage_full[b], 32);
+            mbar_init(&sh->stage_empty[b], EPI_WARPS);
         }
         mbar_init(&sh->drain, 1);
         mbar_init(&sh->never, 1);
@@ -311,10 +362,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA_r)) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA_s)) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB_r)) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB_s)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX_r)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX_s)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW_r)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW_s)) : "memory");
             int s = 0;
             uint32_t ph = 0;
             uint32_t issued_par[TSTAGES];
@@ -323,25 +374,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
                 const Tile t = decode_tile(a, tile);
-                const CUtensorMap* mA = t.shared ? &tmA_s : &tmA_r;
-                const CUtensorMap* mB = t.shared ? &tmB_s : &tmB_r;
-                int brow0, brow1;
+                const CUtensorMap* mX = t.shared ? &tmX_s : &tmX_r;
+                const CUtensorMap* mW = t.shared ? &tmW_s : &tmW_r;
+                int wrow0, wrow1;  // raw rows of B rows 0..127 and 128..255
                 if (GEMM == 1) {
                     const int irow = t.shared ? a.Is : a.I;
                     const int base = t.shared ? 0 : t.e * 2 * a.I;
-                    brow0 = base + t.col0;
-                    brow1 = base + irow + t.col0;
+                    wrow0 = base + t.col0;         // gate rows
+                    wrow1 = base + irow + t.col0;  // up rows of the same features
                 } else {
-                    const int base = t.shared ? 0 : t.e * a.H;
-                    brow0 = base + t.col0;
-                    brow1 = base + t.col0 + BN / 2;
+                    wrow0 = (t.shared ? 0 : t.e * a.H) + t.col0;
+                    wrow1 = wrow0 + BN / 2;
                 }
                 for (int kb = 0; kb < t.nkb; ++kb) {
                     if (!mbar_wait(&sh->empty_t[s], ph ^ 1u, sh)) { ok = false; break; }
                     mbar_expect_tx(&sh->full_tma[s], A_BYTES + RAW_BYTES);
-                    tma_load_2d(a_tile(s), mA, &sh->full_tma[s], kb * BK, t.a_row);
-                    tma_load_2d(raw_tile(s), mB, &sh->full_tma[s], kb * (BK / 2), brow0);
-                    tma_load_2d(raw_tile(s) + RAW_BYTES / 2, mB, &sh->full_tma[s], kb * (BK / 2), brow1);
+                    tma_load_2d(x_tile(s), mX, &sh->full_tma[s], kb * BK, t.slot0);
+                    tma_load_2d(raw_tile(s), mW, &sh->full_tma[s], kb * (BK / 2), wrow0);
+                    tma_load_2d(raw_tile(s) + RAW_BYTES / 2, mW, &sh->full_tma[s], kb * (BK / 2), wrow1);
                     issued[s] = true;
                     issued_par[s] = ph;
                     if (++s == TSTAGES) { s = 0; ph ^= 1u; }
@@ -366,17 +416,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
                 tc_fence_after();
                 const uint32_t d = tmem + buf * BN;
                 for (int kb = 0; kb < t.nkb; ++kb) {
-                    if (!mbar_wait(&sh->full_tma[s], ph, sh) || !mbar_wait(&sh->full_deq[sb], phb, sh)) {
+                    if (!mbar_wait(&sh->full_tma[s], ph, sh) || !mbar_wait(&sh->full_b[sb], phb, sh)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t aaddr = smem_u32(a_tile(s)), baddr = smem_u32(b_tile(sb));
+                    const uint32_t xaddr = smem_u32(x_tile(s)), baddr = smem_u32(b_tile(sb));
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        mma_f16_ss(d, smem_desc_sw128(aaddr + kk * 32), smem_desc_sw128(baddr + kk * 32), idesc,
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_f16_ss(d, smem_desc_sw128(xaddr + kk * 32), smem_desc_sw128(baddr + kk * 32), idesc,
                                    (kb | kk) != 0);
-                    }
                     any = true;
                     mma_commit(&sh->empty_t[s]);
                     mma_commit(&sh->empty_b[sb]);
@@ -395,131 +444,157 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
                 mbar_wait_drain(&sh->drain, 0, kDrainCycles);
             }
         }
-    } else if (warp < 2 + DEQ_WARPS) {
-        // ---------------- dequantisers (one B row per thread) ----------------
-        const int r = threadIdx.x - 64;  // B row = output column of the tile
-        int s = 0, sb = 0;
-        uint32_t ph = 0, phb = 0;
+    } else if (warp < WARP_STAGE) {
+        // ---------------- dequantisers: one B row per thread ----------------
+        // Group g handles the k blocks n = g (mod 2) of the CTA's sequence, which
+        // use B slot n mod BSTAGES and TMA stage n mod TSTAGES.
+        const int g = (warp - 2) >> 3;
+        const int r = ((warp - 2) & 7) * 32 + lane;  // B row = accumulator column
+        // the 16-byte half read first: a quarter-warp's eight reads then fall on
+        // eight different 16-byte bank groups (raw rows are 32 bytes apart)
+        const int h0 = (r ^ (r >> 2)) & 1;
+        const uint32_t brow_off = (r >> 3) * 1024 + (r & 7) * 128;
+        const uint32_t ring = smem_u32(smem);
+        uint32_t n = 0;  // k blocks of the CTA so far
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
             const Tile t = decode_tile(a, tile);
-            for (int kb = 0; kb < t.nkb; ++kb) {
-                int got = 0;
-                if (lane == 0) got = mbar_wait(&sh->full_tma[s], ph, sh) && mbar_wait(&sh->empty_b[sb], phb ^ 1u, sh);
-                if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
-                const uint8_t* raw = raw_tile(s);
-                uint8_t* bt = b_tile(sb);
-                {
-                    // the two 16-byte halves of this row, the half (r ^ r >> 2) & 1 first:
-                    // each quarter-warp's 8 reads then fall on 8 different 16-byte bank
-                    // groups (rows are 32 bytes apart)
-                    const int h0 = (r ^ (r >> 2)) & 1;
-                    const uint4 qa = *reinterpret_cast<const uint4*>(raw + r * 32 + 16 * h0);
-                    const uint4 qb = *reinterpret_cast<const uint4*>(raw + r * 32 + 16 * (h0 ^ 1));
-                    const uint4 q0 = h0 ? qb : qa, q1 = h0 ? qa : qb;
-                    const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-                    uint8_t* row = bt + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {  // 16-byte chunk c = elements 8c..8c+7
-                        uint32_t o[4];
-                        int4x8_natural<GEMM == 1>(words[c], o);
-                        *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                    }
+            for (int kb = 0; kb < t.nkb; ++kb, ++n) {
+                if ((int)(n & (DEQ_GROUPS - 1)) != g) continue;
+                const int s = (int)(n % TSTAGES), sb = (int)(n % BSTAGES);
+                const uint32_t ph = (n / TSTAGES) & 1u, phb = (n / BSTAGES) & 1u;
+                if (!warp_wait(&sh->full_tma[s], ph, sh) || !warp_wait(&sh->empty_b[sb], phb ^ 1u, sh)) {
+                    ok = false;
+                    break;
                 }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                const uint32_t rrow = ring + s * TSTAGE_BYTES + A_BYTES + r * (BK / 2);
+                const uint4 qa = lds128(rrow + 16 * h0);
+                const uint4 qb = lds128(rrow + 16 * (h0 ^ 1));
+                const uint4 q0 = h0 ? qb : qa, q1 = h0 ? qa : qb;
+                const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                const uint32_t brow = ring + TSTAGES * TSTAGE_BYTES + sb * B_BYTES + brow_off;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {  // 16-byte chunk c = elements 8c..8c+7
+                    uint32_t o[4];
+                    int4x8_natural<GEMM == 1>(words[c], o);
+                    sts128(brow + ((c ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the MMA reads through the async proxy
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(&sh->full_deq[sb]);
+                    mbar_arrive(&sh->full_b[sb]);
                     mbar_arrive(&sh->empty_t[s]);  // this warp is done with the raw tile
                 }
-                if (++s == TSTAGES) { s = 0; ph ^= 1u; }
-                if (++sb == BSTAGES) { sb = 0; phb ^= 1u; }
             }
         }
-    } else {
-        // ---------------- epilogue (128 threads, one TMEM lane each) ----------------
-        const int quarter = warp & 3;
-        const int m = quarter * 32 + lane;  // token row of the tile
-        uint32_t acc_ph[2] = {0, 0};
-        int buf = 0;
-        const int et = threadIdx.x - 64 - 32 * DEQ_WARPS;  // 0..127
+    } else if (warp == WARP_STAGE) {
+        // ---------------- staging: per-tile token rows, factors and row scales ----------------
+        uint32_t st_ph[2] = {0, 0};
+        int b = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
             const Tile t = decode_tile(a, tile);
-            const bool valid = m < t.n_valid;
-            // this tile's row scales and this thread's token, loaded while the
-            // tensor cores still work on the tile
+            if (!warp_wait(&sh->stage_empty[b], st_ph[b] ^ 1u, sh)) break;
+            Stage& st = sh->stage[b];
             const int irow = t.shared ? a.Is : a.I;
-            epi_bar();  // every epilogue warp is done with the previous tile's scales
-            if (GEMM == 1) {
-                const float* sc = t.shared ? a.s_s : a.s_r + (size_t)t.e * 2 * a.I;
-                sh->ep_scale[et] = __ldg(sc + t.col0 + et);
-                sh->ep_scale[BN / 2 + et] = __ldg(sc + irow + t.col0 + et);
-            } else {
-                const float* sc = t.shared ? a.s_s : a.s_r + (size_t)t.e * a.H;
-                sh->ep_scale[et] = __ldg(sc + t.col0 + et);
-                sh->ep_scale[BN / 2 + et] = __ldg(sc + t.col0 + BN / 2 + et);
+            const float* S = GEMM == 1 ? (t.shared ? a.s_s : a.s_r + (size_t)t.e * 2 * a.I)
+                                       : (t.shared ? a.s_s : a.s_r + (size_t)t.e * a.H);
+#pragma unroll
+            for (int j = lane; j < BM; j += 32) {
+                if (j < t.n_valid) {
+                    const int tok = t.shared ? t.slot0 + j : __ldg(a.tok_of_slot + t.slot0 + j);
+                    const int hx = __ldg(a.hexp + tok);
+                    st.slot[j] = GEMM == 1 ? t.slot0 + j : (t.shared ? a.T * a.K + t.slot0 + j : t.slot0 + j);
+                    st.fac[j] = ldexpf(1.0f, GEMM == 1 ? -hx : hx);
+                } else {
+                    st.slot[j] = -1;
+                    st.fac[j] = 0.f;
+                }
             }
-            const int tok = valid ? (t.shared ? t.slot0 + m : __ldg(a.tok_of_slot + t.slot0 + m)) : 0;
-            const int hx = __ldg(a.hexp + tok);
-            int got = 0;
-            if (lane == 0)
-                got = (!a.stall || mbar_wait(&sh->never, 0, sh, kStallCycles)) &&
-                      mbar_wait(&sh->acc_full[buf], acc_ph[buf], sh);
-            if (lane == 0) sh->ep_ok[quarter] = got;
-            epi_bar();  // scales visible; every warp's wait outcome known
-            if (!(sh->ep_ok[0] && sh->ep_ok[1] && sh->ep_ok[2] && sh->ep_ok[3])) break;
+#pragma unroll
+            for (int j = lane; j < BN; j += 32)
+                st.sc[j] = GEMM == 1 ? __ldg(S + (j < BN / 2 ? 0 : irow) + t.col0 + (j & (BN / 2 - 1)))
+                                     : __ldg(S + t.col0 + j);
+            mbar_arrive(&sh->stage_full[b]);  // every lane: its writes are released with the arrival
+            st_ph[b] ^= 1u;
+            b ^= 1;
+        }
+    } else {
+        // ---------------- epilogue: tokens of lane quarter q, column half c ----------------
+        const int quarter = warp & 3, chalf = (warp - WARP_EPI0) >> 2;
+        const int m = quarter * 32 + lane;  // token row of the tile = TMEM lane
+        uint32_t acc_ph[2] = {0, 0};
+        int buf = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            const Tile t = decode_tile(a, tile);
+            const bool got = (!a.stall || mbar_wait(&sh->never, 0, sh, kStallCycles)) &&
+                             mbar_wait(&sh->stage_full[buf], acc_ph[buf], sh) &&
+                             mbar_wait(&sh->acc_full[buf], acc_ph[buf], sh);
+            if (!__all_sync(0xffffffffu, got)) break;
             tc_fence_after();
+            const Stage& st = sh->stage[buf];
+            const uint32_t st_sc = smem_u32(&st.sc[0]);
+            const int row = lds32(smem_u32(&st.slot[m]));
+            const float fac = __int_as_float(lds32(smem_u32(&st.fac[m])));
             const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;
-            const float* scs = sh->ep_scale;
             if (GEMM == 1) {
-                __half* hrow = (t.shared ? a.h_s : a.h_r) + (size_t)(t.slot0 + m) * irow + t.col0;
-                const float hsc = ldexpf(1.0f, -hx);
+                // features 64c .. 64c + 63 of the tile: gate in column j, up in column 128 + j
+                const int irow = t.shared ? a.Is : a.I;
+                __half* hrow = (t.shared ? a.h_s : a.h_r) + (size_t)(row < 0 ? 0 : row) * irow + t.col0;
 #pragma unroll 1
-                for (int c0 = 0; c0 < BN / 2; c0 += 16) {
-                    uint32_t g[16], u[16];
-                    tmem_ld16_wait(tbase + c0, g);
-                    tmem_ld16_wait(tbase + BN / 2 + c0, u);
+                for (int c0 = 64 * chalf; c0 < 64 * chalf + 64; c0 += 16) {
+                    uint32_t gv[16], uv[16];
+                    tmem_ld16_wait(tbase + c0, gv);
+                    tmem_ld16_wait(tbase + BN / 2 + c0, uv);
+                    float sg[16], su[16];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 a4 = lds128f(st_sc + 4 * (c0 + 4 * q));
+                        const float4 b4 = lds128f(st_sc + 4 * (BN / 2 + c0 + 4 * q));
+                        sg[4 * q] = a4.x; sg[4 * q + 1] = a4.y; sg[4 * q + 2] = a4.z; sg[4 * q + 3] = a4.w;
+                        su[4 * q] = b4.x; su[4 * q + 1] = b4.y; su[4 * q + 2] = b4.z; su[4 * q + 3] = b4.w;
+                    }
                     uint32_t packed[8];
 #pragma unroll
                     for (int i = 0; i < 16; i += 2) {
-                        const int j = c0 + i;
-                        const float g0 = __uint_as_float(g[i]) * scs[j];
-                        const float g1 = __uint_as_float(g[i + 1]) * scs[j + 1];
-                        const float u0 = __uint_as_float(u[i]) * scs[BN / 2 + j];
-                        const float u1 = __uint_as_float(u[i + 1]) * scs[BN / 2 + j + 1];
-                        __half2 hv = __floats2half2_rn(silu_mul(g0, u0) * hsc, silu_mul(g1, u1) * hsc);
+                        const float h0v = silu_mul(__uint_as_float(gv[i]) * sg[i], __uint_as_float(uv[i]) * su[i]) * fac;
+                        const float h1v =
+                            silu_mul(__uint_as_float(gv[i + 1]) * sg[i + 1], __uint_as_float(uv[i + 1]) * su[i + 1]) * fac;
+                        __half2 hv = __floats2half2_rn(h0v, h1v);
                         packed[i >> 1] = *reinterpret_cast<uint32_t*>(&hv);
                     }
-                    if (valid) {
+                    if (row >= 0) {
                         uint4* dst = reinterpret_cast<uint4*>(hrow + c0);
                         dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
                         dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
                     }
                 }
             } else {
-                const size_t slot = t.shared ? (size_t)a.T * a.K + t.slot0 + m : (size_t)(t.slot0 + m);
-                float* yrow = a.y + slot * a.H + t.col0;
-                const float inv = ldexpf(1.0f, hx);
+                // output columns 128c .. 128c + 127 of the tile
+                float* yrow = a.y + (size_t)(row < 0 ? 0 : row) * a.H + t.col0;
 #pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 16) {
+                for (int c0 = 128 * chalf; c0 < 128 * chalf + 128; c0 += 16) {
                     uint32_t v[16];
                     tmem_ld16_wait(tbase + c0, v);
-                    if (valid) {
-                        float4* dst = reinterpret_cast<float4*>(yrow + c0);
+                    float4 o[4];
 #pragma unroll
-                        for (int i = 0; i < 16; i += 4) {
-                            const int j = c0 + i;
-                            dst[i >> 2] = make_float4(__uint_as_float(v[i]) * (scs[j] * inv),
-                                                      __uint_as_float(v[i + 1]) * (scs[j + 1] * inv),
-                                                      __uint_as_float(v[i + 2]) * (scs[j + 2] * inv),
-                                                      __uint_as_float(v[i + 3]) * (scs[j + 3] * inv));
-                        }
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 s4 = lds128f(st_sc + 4 * (c0 + 4 * q));
+                        o[q] = make_float4(__uint_as_float(v[4 * q]) * (s4.x * fac), __uint_as_float(v[4 * q + 1]) * (s4.y * fac),
+                                           __uint_as_float(v[4 * q + 2]) * (s4.z * fac),
+                                           __uint_as_float(v[4 * q + 3]) * (s4.w * fac));
+                    }
+                    if (row >= 0) {
+                        float4* dst = reinterpret_cast<float4*>(yrow + c0);
+                        dst[0] = o[0]; dst[1] = o[1]; dst[2] = o[2]; dst[3] = o[3];
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sh->acc_empty[buf]);
+            if (lane == 0) {
+                mbar_arrive(&sh->acc_empty[buf]);
+                mbar_arrive(&sh->stage_empty[buf]);
+            }
             acc_ph[buf] ^= 1u;
             buf ^= 1;
         }
@@ -593,7 +668,7 @@ cudaError_t launch_tc_gemm(const Params& p, int gemm, int grid, cudaStream_t str
     }
     const int TK = p.T * p.K;
     const int Is = p.Is > 0 ? p.Is : 128;  // any valid map when there is no shared expert
-    CUtensorMap mA_r, mA_s, mB_r, mB_s;
+    CUtensorMap mX_r, mX_s, mW_r, mW_s;
     TcArgs a;
     memset(&a, 0, sizeof a);
     a.T = p.T; a.H = p.H; a.E = p.E; a.K = p.K; a.I = p.I; a.Is = p.Is;
@@ -607,37 +682,37 @@ cudaError_t launch_tc_gemm(const Params& p, int gemm, int grid, cudaStream_t str
     bool ok;
     if (gemm == 1) {
         a.kdim_r = p.H; a.kdim_s = p.H;
-        a.ntile_r = p.I / 128; a.ntile_s = p.Is / 128;
+        a.ntile_r = p.I / kTcFeat1; a.ntile_s = p.Is / kTcFeat1;
         a.tstart = p.tcs1;
         a.s_r = p.s13; a.s_s = p.sh_s13;
-        ok = make_map(&mA_r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.x_perm, p.H, TK, 64, 128,
+        ok = make_map(&mX_r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.x_perm, p.H, TK, 64, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
-             make_map(&mA_s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.x, p.H, p.T, 64, 128,
+             make_map(&mX_s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.x, p.H, p.T, 64, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
-             make_map(&mB_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.w13, p.H / 2, (uint64_t)p.E * 2 * p.I, 32, 128,
+             make_map(&mW_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.w13, p.H / 2, (uint64_t)p.E * 2 * p.I, 32, tc::BN / 2,
                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
-             make_map(&mB_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.Is > 0 ? (const void*)p.sh_w13 : (const void*)p.w13,
-                      p.H / 2, 2 * (uint64_t)Is, 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+             make_map(&mW_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.Is > 0 ? (const void*)p.sh_w13 : (const void*)p.w13,
+                      p.H / 2, 2 * (uint64_t)Is, 32, tc::BN / 2, CU_TENSOR_MAP_SWIZZLE_NONE);
     } else {
         a.kdim_r = p.I; a.kdim_s = p.Is;
-        a.ntile_r = p.H / 256; a.ntile_s = p.H / 256;
+        a.ntile_r = p.H / kTcFeat2; a.ntile_s = p.H / kTcFeat2;
         a.tstart = p.tcs2;
         a.s_r = p.s2; a.s_s = p.sh_s2;
-        ok = make_map(&mA_r, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.h_r, p.I, TK, 64, 128,
+        ok = make_map(&mX_r, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.h_r, p.I, TK, 64, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
-             make_map(&mA_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.Is > 0 ? (const void*)p.h_s : (const void*)p.h_r,
+             make_map(&mX_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.Is > 0 ? (const void*)p.h_s : (const void*)p.h_r,
                       Is, p.T, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
-             make_map(&mB_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.w2, p.I / 2, (uint64_t)p.E * p.H, 32, 128,
+             make_map(&mW_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.w2, p.I / 2, (uint64_t)p.E * p.H, 32, tc::BN / 2,
                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
-             make_map(&mB_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.Is > 0 ? (const void*)p.sh_w2 : (const void*)p.w2,
-                      Is / 2, p.H, 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+             make_map(&mW_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.Is > 0 ? (const void*)p.sh_w2 : (const void*)p.w2,
+                      Is / 2, p.H, 32, tc::BN / 2, CU_TENSOR_MAP_SWIZZLE_NONE);
     }
     if (!ok) return cudaErrorInvalidValue;
     if (gemm == 1)
-        return launch_pdl(tc::grouped_gemm_kernel<1>, dim3(grid), dim3(tc::NUM_THREADS), tc::SMEM_BYTES, stream, mA_r,
-                          mA_s, mB_r, mB_s, a);
-    return launch_pdl(tc::grouped_gemm_kernel<2>, dim3(grid), dim3(tc::NUM_THREADS), tc::SMEM_BYTES, stream, mA_r,
-                      mA_s, mB_r, mB_s, a);
+        return launch_pdl(tc::grouped_gemm_kernel<1>, dim3(grid), dim3(tc::NUM_THREADS), tc::SMEM_BYTES, stream, mX_r,
+                          mX_s, mW_r, mW_s, a);
+    return launch_pdl(tc::grouped_gemm_kernel<2>, dim3(grid), dim3(tc::NUM_THREADS), tc::SMEM_BYTES, stream, mX_r,
+                      mX_s, mW_r, mW_s, a);
 }
 
 }  // namespace moe

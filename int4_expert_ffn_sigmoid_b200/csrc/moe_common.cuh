@@ -11,6 +11,11 @@ namespace moe {
 
 // Largest T that takes the weight-streaming (small-batch) path by default.
 constexpr int kDecodeMaxTokens = 64;
+// Tensor-core grouped GEMM tiles: 128 tokens x 128 features (GEMM-1: their
+// gate and up rows, 256 weight rows) or x 256 output features (GEMM-2).
+constexpr int kTcTokens = 128;
+constexpr int kTcFeat1 = 128;
+constexpr int kTcFeat2 = 256;
 // Rows of one weight-streaming task: gate/up (each with its up row); one
 // row group of a down task (a down task has Params::rows2 rows, a multiple).
 constexpr int kTaskRows13 = 64;

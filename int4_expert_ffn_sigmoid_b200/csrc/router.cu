@@ -251,10 +251,10 @@ __device__ void finalize_buckets(const Params& p, const int* s_cnt, int* s_off) 
                 const int ch = chunks_of(n, p.chunk);
                 n13 = (irow / kTaskRows13) * ch;                    // gate/up rows x a token chunk
                 n2 = (p.H / p.rows2) * ch * slices_of(irow);        // down rows x a chunk x a slice
-                if (e != E) {  // tensor-core tiles: 128 tokens x 128 features / 256 columns
-                    const int mt = (n + 127) / 128;
-                    nt1 = mt * (p.I / 128);
-                    nt2 = mt * (p.H / 256);
+                if (e != E) {  // tensor-core tiles: 128 tokens x 128 features / 256 output features
+                    const int mt = (n + kTcTokens - 1) / kTcTokens;
+                    nt1 = mt * (p.I / kTcFeat1);
+                    nt2 = mt * (p.H / kTcFeat2);
                 }
             }
             int i13 = n13, i2 = n2, it1 = nt1, it2 = nt2;
