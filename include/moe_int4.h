@@ -185,8 +185,11 @@ size_t moe_layer_workspace_bytes_upto(const moe_cfg_t* cfg, int32_t N);
  *                or f32 [T][H] under MOE_OUT_F32
  *   T          : tokens, 0..2^20 (T = 0 returns MOE_OK and launches nothing)
  *   cfg, stream: see above.
- * Arithmetic.  Router logits, scores and routing weights are f32.  Two
- * kernel sequences compute the experts:
+ * Arithmetic.  Router logits, scores and routing weights are f32 (on the
+ * large-batch sequences the logits are summed on the tensor cores from an
+ * exact three-term bf16 split of each f32 router weight, 16 products per
+ * step, with f32 adds between steps).  Two kernel sequences compute the
+ * experts:
  *  - small batches (T <= moe_decode_max_tokens(), unless MOE_FORCE_PREFILL),
  *    and larger ones when H is not a multiple of 256, when T*K < 32*E (fewer
  *    than 32 picks per routed expert on average; not under

@@ -51,7 +51,7 @@ Path choose_path(const moe_cfg_t& c, int32_t T) {
 
 struct WsLayout {
     size_t ctrl, idx, wts, counts, offsets, bucket_e, bucket_n, bucket_off, ts13, ts2, tcs1, tcs2;
-    size_t tok_of_slot, slot_of, hist, rank, hexp, y, lpart;
+    size_t tok_of_slot, slot_of, hist, rank, hexp, y, lpart, wsplit;
     size_t h_r, h_s, x_perm;                            // tensor-core path
     size_t xq, xs, h32_r, h32_s, hmax_r, hmax_s;        // weight-streaming paths
     size_t total;
@@ -84,7 +84,12 @@ WsLayout ws_layout(const moe_cfg_t& c, int32_t T) {
     L.hist = take((size_t)kRouterMaxBlocks * E * 4);
     L.rank = take(TK * 4);
     L.hexp = take((size_t)T * 4);
-    L.lpart = take((size_t)router_split_slices(c.E, c.H, path == Path::kSmall) * T * E * 4);
+    if (path == Path::kSmall) {
+        L.lpart = take((size_t)router_split_slices(c.E, c.H) * T * E * 4);
+    } else if (router_large_uses_tc(c.E, c.H)) {  // the tensor-core router's partial logits and split weights
+        L.lpart = take((size_t)tc_router_slices(c.E, c.H) * T * E * 4);
+        L.wsplit = take(3 * E * H * 2);
+    }
     const size_t shared_rows = c.Is > 0 ? (size_t)T : 0;
     if (path == Path::kTensorCore) {
         L.h_r = take(TK * (size_t)c.I * 2);
@@ -206,9 +211,11 @@ int32_t moe_decode_max_tokens(void) { return kDecodeMaxTokens; }
 int32_t moe_layer_kernel_launches(const moe_cfg_t* cfg, int32_t T) {
     if (validate_cfg(cfg) != MOE_OK || T <= 0 || T > kMaxTokens) return 0;
     // small batch: [router logits,] cluster router, gate/up, down, combine;
-    // otherwise: [router logits,] router, scatter, gate/up, down, combine
-    const bool small = choose_path(*cfg, T) == Path::kSmall;
-    return (small ? 4 : 5) + (router_split_slices(cfg->E, cfg->H, small) > 0 ? 1 : 0);
+    // otherwise: router (or, with large router weights, the weight split, the
+    // tensor-core router logits and the selection), scatter, gate/up, down,
+    // combine
+    if (choose_path(*cfg, T) != Path::kSmall) return router_large_uses_tc(cfg->E, cfg->H) ? 7 : 5;
+    return 4 + (router_split_slices(cfg->E, cfg->H) > 0 ? 1 : 0);
 }
 
 int32_t moe_layer_path(const moe_cfg_t* cfg, int32_t T) {
@@ -333,7 +340,13 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
         p.nsl_s = slices_of(cfg->Is);
     }
     p.decode_groups = small ? cdiv(T, kDecodeRouterTok) : 0;
-    p.lslices = router_split_slices(cfg->E, cfg->H, small);  // on either path
+    if (small) {
+        p.lslices = router_split_slices(cfg->E, cfg->H);
+    } else if (router_large_uses_tc(cfg->E, cfg->H)) {  // large router weights: logits on the tensor cores
+        p.tc_router = 1;
+        p.lslices = tc_router_slices(cfg->E, cfg->H);
+        p.wsplit = static_cast<__nv_bfloat16*>(at(L.wsplit));
+    }
     p.lpart = p.lslices > 0 ? static_cast<float*>(at(L.lpart)) : nullptr;
     const int ntiles = cdiv(T, kRouterTileTokens);
     p.router_blocks = ntiles < kRouterMaxBlocks ? ntiles : kRouterMaxBlocks;

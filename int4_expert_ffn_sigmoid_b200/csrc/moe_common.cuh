@@ -219,9 +219,31 @@ struct Params {
     int rows2;            // output rows of one down task (kTaskRows2 times 1..8, dividing H)
     int chunk;            // tokens per weight-streaming task: kChunkTokens or kMaxChunk
     int decode_groups;    // token groups of the small-batch router (0: tables come from the large router)
-    float* lpart;         // [lslices][T][E] partial router logits of the split small-batch router
-    int lslices;          // hidden-dimension slices of lpart (0: the small-batch router computes its logits)
+    float* lpart;         // [lslices][T][E] partial router logits (split router or tensor-core router)
+    int lslices;          // hidden-dimension slices of lpart (0: the selecting router computes its logits)
+    __nv_bfloat16* wsplit;  // [3][E][H] router weights as exact bf16 terms hi, mid, lo (tensor-core router)
+    int tc_router;        // 1: the tensor-core router logits run first on the large-batch path
 };
+
+// Zeroes the per-call status word (first kernel of a call, one thread,
+// after pdl_wait: every kernel of the previous call has completed).
+__device__ __forceinline__ void reset_ctrl(const Params& p) {
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) p.ctrl->status = 0;
+}
+
+// An f32 weight as three bf16 terms with w = hi + mid + lo exactly (hi =
+// bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid): the three 8-bit
+// significands cover w's 24 bits), as raw bf16 bits.
+__device__ __forceinline__ void split3(float w, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(m);
+    hi = __bfloat16_as_ushort(h);
+    mid = __bfloat16_as_ushort(m);
+    lo = __bfloat16_as_ushort(__float2bfloat16_rn(r2));
+}
+
 
 // ---------------------------------------------------------------------------
 // int4 -> 16-bit float by the exponent-bias ("magic number") technique of

@@ -11,7 +11,15 @@ namespace moe {
 cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream);
 // Hidden-dimension slices of the split small-batch router's partial logits
 // (0: the cluster router computes the logits itself).
-int router_split_slices(int E, int H, bool small_path);
+int router_split_slices(int E, int H);
+// Tensor-core router logits of the large-batch path: the weight split and
+// the logits kernel (slices of the hidden dimension, partials in lpart).
+cudaError_t launch_router_tc(const Params& p, cudaStream_t stream);
+// Whether the large-batch path computes the router logits on the tensor cores
+// (router_tc.cu; router weights above 512 KB) rather than in router_large_kernel.
+bool router_large_uses_tc(int E, int H);
+// Hidden slices of the tensor-core router (a function of E and H only).
+int tc_router_slices(int E, int H);
 // Expert gate/up + SwiGLU (weight-streaming mma.sync kernel).
 cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream);
 // Expert down projection (weight-streaming mma.sync kernel).

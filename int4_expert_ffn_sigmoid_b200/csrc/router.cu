@@ -13,8 +13,8 @@
 // whatever it is batched with (within one path).  The small-batch router
 // accumulates, in lane l of a warp, the elements 128*i + 4*l + j (i ascending,
 // then j = 0..3) with fused multiply-adds and sums the 32 lane partials by an
-// xor-butterfly (16, 8, 4, 2, 1); the large-batch router is described above
-// router_large_kernel.
+// xor-butterfly (16, 8, 4, 2, 1); the large-batch routers are described above
+// router_large_kernel and in router_tc.cu.
 #include <cooperative_groups.h>
 
 #include "moe_common.cuh"
@@ -57,22 +57,34 @@ __device__ __forceinline__ void store_hexp(const Params& p, int t, float lane_sq
     if (lane == 0) p.hexp[t] = min(max(kHExpBase + e, kHExpMin), kHExpMax);
 }
 
-// k_t of one token (one warp), loads issued four 128-blocks at a time.
-__device__ __forceinline__ void token_hexp(const Params& p, int t, int lane) {
-    const __nv_bfloat16* xr = p.x + (size_t)t * p.H;
+// k_t of the tokens warp, warp + 8, warp + 16, warp + 24 of a tile (nt
+// tokens from t0): lane l sums the squares of elements 128 i + 4 l .. + 3 of
+// each 128-block i in ascending order, with the four tokens' loads of four
+// 128-blocks in flight together.
+__device__ __forceinline__ void tile_hexp(const Params& p, int t0, int nt, int warp, int lane) {
     const int nblk = p.H / 128;
-    float acc = 0.f;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int i0 = 0; i0 < nblk; i0 += 4) {
-        uint2 xv[4];
+        uint2 xv[4][4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            xv[u] = i0 + u < nblk ? __ldg(reinterpret_cast<const uint2*>(xr + (i0 + u) * 128 + lane * 4))
-                                  : make_uint2(0u, 0u);
+        for (int j = 0; j < 4; ++j) {
+            const int tt = warp + 8 * j;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (i0 + u < nblk) acc = sq_step(acc, xv[u]);
+            for (int u = 0; u < 4; ++u)
+                xv[j][u] = (tt < nt && i0 + u < nblk)
+                               ? __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)(t0 + tt) * p.H + (i0 + u) * 128 +
+                                                                      lane * 4))
+                               : make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (i0 + u < nblk) acc[j] = sq_step(acc[j], xv[j][u]);
     }
-    store_hexp(p, t, acc, lane);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        if (warp + 8 * j < nt) store_hexp(p, t0 + warp + 8 * j, acc[j], lane);
 }
 
 // Top-K of one token (one warp).  Lane l holds the logits L[j] of experts
@@ -292,11 +304,6 @@ __device__ void finalize_buckets(const Params& p, const int* s_cnt, int* s_off) 
     __syncthreads();
 }
 
-// Zeroes the per-call status word (first kernel of a call, one thread,
-// after pdl_wait: every kernel of the previous call has completed).
-__device__ __forceinline__ void reset_ctrl(const Params& p) {
-    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) p.ctrl->status = 0;
-}
 
 // ---------------------------------------------------------------------------
 // Small batch (T <= kDecodeMaxTokens): one kernel, a cluster of
@@ -320,26 +327,25 @@ __device__ __forceinline__ void reset_ctrl(const Params& p) {
 constexpr int kRouterXMaxH = 12288;
 constexpr int kRouterWarps = 16;
 constexpr int kRouterBatch = 8;  // router-weight blocks per batch of loads
-// The logits are computed by a separate kernel spread over many SMs
-// (router_logits_kernel) when a warp of the cluster router would stream more
-// than kRouterWarpMaxBytes of router weights (its ceil(epc / kRouterWarps)
-// rows of H f32 each), and on the large-batch path when the router weights
-// (E * H f32, which every CTA of router_large_kernel reads) exceed
-// kRouterLargeMaxBytes.
+// The small-batch logits are computed by a separate kernel spread over many
+// SMs (router_logits_kernel) when a warp of the cluster router would stream
+// more than kRouterWarpMaxBytes of router weights (its ceil(epc /
+// kRouterWarps) rows of H f32 each).  On the large-batch path the router
+// weights (E * H f32) are read by every CTA of router_large_kernel up to
+// kRouterLargeMaxBytes; above that the tensor-core logits of router_tc.cu
+// compute the logits in hidden slices.
 constexpr size_t kRouterWarpMaxBytes = 8192;
 constexpr size_t kRouterLargeMaxBytes = (size_t)512 << 10;
+
+bool router_large_uses_tc(int E, int H) { return (size_t)E * H * 4 > kRouterLargeMaxBytes; }
 constexpr int kLogitSliceBlocks = 3;   // 128-element blocks of the hidden dimension per slice
 constexpr int kLogitCtaExperts = 32;   // experts per CTA (4 per warp)
 constexpr int kLogitTileTokens = 64;   // tokens per CTA
 
-int router_split_slices(int E, int H, bool small_path) {
-    if (small_path) {
-        const int epc = (E + kDecodeRouterCtas - 1) / kDecodeRouterCtas;
-        const size_t warp_bytes = (size_t)((epc + kRouterWarps - 1) / kRouterWarps) * H * 4;
-        if (warp_bytes <= kRouterWarpMaxBytes) return 0;
-    } else if ((size_t)E * H * 4 <= kRouterLargeMaxBytes) {
-        return 0;
-    }
+int router_split_slices(int E, int H) {
+    const int epc = (E + kDecodeRouterCtas - 1) / kDecodeRouterCtas;
+    const size_t warp_bytes = (size_t)((epc + kRouterWarps - 1) / kRouterWarps) * H * 4;
+    if (warp_bytes <= kRouterWarpMaxBytes) return 0;
     return (H / 128 + kLogitSliceBlocks - 1) / kLogitSliceBlocks;
 }
 
@@ -355,7 +361,7 @@ size_t router_decode_smem(int H) {
 // tokens' activations of the slice are staged in shared memory.  Lane l
 // accumulates the elements 128 i + 4 l + j of the slice (i ascending, then j)
 // and the lanes are summed by the xor-butterfly; the selecting kernel (the
-// cluster router or router_large_kernel) adds the slices in ascending order.
+// cluster router) adds the slices in ascending order.
 // The logit of a token therefore does not depend on the other tokens of the
 // batch.
 __global__ void __launch_bounds__(256) router_logits_kernel(Params p) {
@@ -551,15 +557,18 @@ __global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(32 *
 }
 
 // ---------------------------------------------------------------------------
-// Large batch, two kernels (after router_logits_kernel when the router
-// weights are large).
-// router_large_kernel: router_blocks CTAs walk tiles of kRouterTileTokens
+// Large batch, two kernels.
+// router_large_kernel (router weights up to kRouterLargeMaxBytes) or, after
+// the tensor-core router logits of router_tc.cu (larger router weights),
+// router_select_kernel: router_blocks CTAs walk tiles of kRouterTileTokens
 // tokens (tile = block, block + grid, ...); each tile's logits stay in shared
-// memory, one warp per token selects, and every CTA records its per-expert
-// pick counts.  scatter_large_kernel: every CTA derives the bucket offsets
-// and its own slot bases from those counts (CTA 0 also writes the bucket and
-// task lists), then the slots, and the gathered activation rows of the
-// tensor-core path or the int8 activations of the weight-streaming kernels.
+// memory (router_select_kernel: the hidden slices' partial logits added in
+// ascending order), one warp per token selects, and every CTA records its
+// per-expert pick counts.  scatter_large_kernel: every CTA derives the bucket
+// offsets and its own slot bases from those counts (CTA 0 also writes the
+// bucket and task lists), then the slots, and the gathered activation rows of
+// the tensor-core path or the int8 activations of the weight-streaming
+// kernels.
 // ---------------------------------------------------------------------------
 // Tensor-core router logits for a tile of kRouterTileTokens tokens and every
 // expert.  x is exactly bf16; each f32 router weight w is split exactly into
@@ -576,15 +585,6 @@ constexpr int kRouterXS = kRouterKC + 8;      // padded row (bf16 elements)
 constexpr int kRouterMT = kRouterTileTokens / 16;
 constexpr int kRouterXStages = 4;             // staged chunks in flight
 
-__device__ __forceinline__ void split3(float w, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(w);
-    const float r1 = w - __bfloat162float(h);
-    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(m);
-    hi = __bfloat16_as_ushort(h);
-    mid = __bfloat16_as_ushort(m);
-    lo = __bfloat16_as_ushort(__float2bfloat16_rn(r2));
-}
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* smem_row) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -616,7 +616,7 @@ __global__ void __launch_bounds__(256, 2) router_large_kernel(Params p) {
             wpre[k][1] = __ldg(reinterpret_cast<const float2*>(wrow + k * 16 + 2 * q + 8));
         }
     };
-    if (p.lslices == 0 && warp < n_ntiles) load_w0(0);
+    if (warp < n_ntiles) load_w0(0);
     pdl_wait();
     reset_ctrl(p);
     pdl_release();
@@ -627,24 +627,6 @@ __global__ void __launch_bounds__(256, 2) router_large_kernel(Params p) {
     for (int tile = blockIdx.x; tile < ntiles_tok; tile += gridDim.x) {
         const int t0 = tile * kRouterTileTokens;
         const int nt = min(kRouterTileTokens, p.T - t0);
-        if (p.lslices > 0) {  // logits from the split kernel's partials, slice 0 first
-            for (int tt = warp; tt < nt; tt += 8) token_hexp(p, t0 + tt, lane);
-            __syncthreads();  // s_logit is free (previous tile done)
-            for (int i = threadIdx.x; i < nt * E; i += blockDim.x) {
-                const int tt = i / E, e = i - tt * E;
-                const float* src = p.lpart + (size_t)(t0 + tt) * E + e;
-                float v = 0.f;
-                for (int sl = 0; sl < p.lslices; ++sl) v += __ldcg(src + (size_t)sl * p.T * E);
-                s_logit[tt][e] = v;
-            }
-            __syncthreads();
-            for (int tt = warp; tt < nt; tt += 8) {
-                const int sel = select_token(p, t0 + tt, s_logit[tt], lane);
-                if (lane < p.K && sel >= 0 && sel < E) atomicAdd(&s_cnt[sel], 1);
-            }
-            continue;
-        }
-
         auto stage_chunk = [&](int c, int buf) {
             for (int i = threadIdx.x; i < kRouterTileTokens * (kRouterKC / 8); i += blockDim.x) {
                 const int r = i / (kRouterKC / 8), part = i % (kRouterKC / 8);
@@ -769,6 +751,61 @@ __global__ void __launch_bounds__(256, 2) router_large_kernel(Params p) {
                     if (e < E) { s_logit[r][e] = acc[j][m][0]; s_logit[r + 8][e] = acc[j][m][2]; }
                     if (e + 1 < E) { s_logit[r][e + 1] = acc[j][m][1]; s_logit[r + 8][e + 1] = acc[j][m][3]; }
                 }
+            }
+        }
+        __syncthreads();
+        for (int tt = warp; tt < nt; tt += 8) {
+            const int sel = select_token(p, t0 + tt, s_logit[tt], lane);
+            // an index outside [0, E) cannot occur; it is counted nowhere and
+            // reported by the scatter kernel's range check
+            if (lane < p.K && sel >= 0 && sel < E) atomicAdd(&s_cnt[sel], 1);
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < E; i += blockDim.x) p.hist[(size_t)blockIdx.x * E + i] = s_cnt[i];
+}
+
+__global__ void __launch_bounds__(256) router_select_kernel(Params p) {
+    __shared__ __align__(16) float s_logit[kRouterTileTokens][kMaxE];
+    __shared__ int s_cnt[kMaxE];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int E = p.E;
+    pdl_wait();  // the weight split, the call's first kernel, zeroed the status word
+    pdl_release();
+    for (int i = threadIdx.x; i < E; i += blockDim.x) s_cnt[i] = 0;
+    __syncthreads();
+    const int ntiles_tok = (p.T + kRouterTileTokens - 1) / kRouterTileTokens;
+    for (int tile = blockIdx.x; tile < ntiles_tok; tile += gridDim.x) {
+        const int t0 = tile * kRouterTileTokens;
+        const int nt = min(kRouterTileTokens, p.T - t0);
+        static_assert(kRouterTileTokens == 32, "four tokens per warp in tile_hexp");
+        tile_hexp(p, t0, nt, warp, lane);
+        __syncthreads();  // s_logit is free (previous tile done)
+        // four elements per thread, each summed over the slices in ascending
+        // order, with up to eight slices' loads of all four in flight
+        for (int i0 = threadIdx.x; i0 < nt * E; i0 += 4 * blockDim.x) {
+            float v[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int sl0 = 0; sl0 < p.lslices; sl0 += 8) {
+                float part[8][4];
+#pragma unroll
+                for (int sl = 0; sl < 8; ++sl)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = i0 + u * blockDim.x;
+                        part[sl][u] = (sl0 + sl < p.lslices && i < nt * E)
+                                          ? __ldcg(p.lpart + ((size_t)(sl0 + sl) * p.T + t0 + i / E) * E + i % E)
+                                          : 0.f;
+                    }
+#pragma unroll
+                for (int sl = 0; sl < 8; ++sl)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (sl0 + sl < p.lslices) v[u] += part[sl][u];
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * blockDim.x;
+                if (i < nt * E) s_logit[i / E][i % E] = v[u];
             }
         }
         __syncthreads();
@@ -945,11 +982,14 @@ cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream)
         return launch_pdl(router_decode_kernel, dim3(p.decode_groups, kDecodeRouterCtas), dim3(32 * kRouterWarps),
                           smem, stream, p);
     }
-    if (p.lslices > 0) {
-        err = launch_router_logits(p, stream);
-        if (err != cudaSuccess) return err;
+    if (p.tc_router) {
+        if (p.lslices <= 0) return cudaErrorInvalidValue;
+        err = launch_router_tc(p, stream);
+        if (err == cudaSuccess) err = launch_pdl(router_select_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
+    } else {
+        err = launch_pdl(router_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
     }
-    err = launch_pdl(router_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
+    if (err != cudaSuccess) return err;
     if (err == cudaSuccess) err = launch_pdl(scatter_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
     return err;
 }

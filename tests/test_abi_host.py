@@ -108,7 +108,8 @@ def test_kernel_launch_count(moe):
     assert moe.kernel_launches(nano, 16, moe.MOE_FORCE_PREFILL) == 5
     assert moe.kernel_launches(nano, 4096, moe.MOE_FORCE_DECODE) == 5
     assert moe.kernel_launches(large, 1) == 5       # + the split router's logits kernel
-    assert moe.kernel_launches(large, 512) == 6     # large router with the logits kernel
+    # weight split, tensor-core router logits, selection, scatter, 2 expert kernels, combine
+    assert moe.kernel_launches(large, 512) == 7
     assert moe.kernel_launches(_shape(H=1000), 16) == 0
     assert moe.kernel_launches(nano, (1 << 20) + 1) == 0
 

@@ -190,9 +190,10 @@ def test_split_router(moe, cuda_device):
     for t0, sub in ((0, 1), (5, 9), (40, 24)):
         o1, _, _ = run(moe, x[t0:t0 + sub].contiguous(), layer, shape)
         assert torch.equal(o1, out[t0:t0 + sub])
-    # large batches: the logits kernel over token tiles of 64 (150 = 64 + 64 + 22)
-    # feeding the large router's selection
-    assert moe.kernel_launches(shape, 150) == 6
+    # large batches: the tensor-core router logits (a 128-token tile and a
+    # ragged one of 22; expert tiles of 128 and 72) feeding the large router's
+    # selection
+    assert moe.kernel_launches(shape, 150) == 7
     x = workloads.make_x(shape, 150, 250, batch=1, device=cuda_device)
     out, _, _, _ = check(moe, x, layer, shape, layer_cpu=cpu, sample=sample_tokens(150, 40, 5))
     o1, _, _ = run(moe, x[10:110].contiguous(), layer, shape)
