@@ -1107,6 +1107,437 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Gate/up on the 5th-generation tensor cores (tcgen05.mma kind::i8), for H a
+// multiple of 256 on the large-batch weight-streaming sequence.  Two rings
+// per 256-wide k chunk of a task: a weight ring (two 64-row TMA tiles of the
+// codes, issued by one producer thread) and an activation ring (both int8
+// parts of every token of the task, copied with cp.async by a second
+// producer warp into the 128-byte swizzled K-major layout of the MMA's B
+// operand: N = 2 * chunk rows, token j's parts are rows 2j and 2j+1).  The 8 converter warps turn a
+// weight stage's int4 codes into int8 16*c (lo8 / hi8, the activations' byte
+// order) and write them into a tensor-memory A stage (row 2i is gate row i
+// of the task, row 2i + 1 up row i), which frees the weight stage at once:
+// the weight ring refills without waiting for the MMAs.  One thread issues the
+// MMAs (M = 128, N, K = 32; int32 accumulators in tensor memory), and 4
+// epilogue warps join the two parts of each token, apply the row and
+// activation scales and SwiGLU (a lane and its neighbour hold gate and up of
+// one feature), store h in f32 and the per-(token, 64-row block) maxima of
+// |h|.  Every wait is bounded and gives up when the CTA aborts; the producer
+// waits for its copies and the MMA thread for its MMAs before the CTA exits.
+// ---------------------------------------------------------------------------
+constexpr int kTc8Threads = 480;  // converters 0-7, weight producer 8, MMA 9, epilogue 10-13, activations 14
+constexpr int kTc8AStages = 4;    // int8 A stages in tensor memory (64 columns each)
+constexpr int kTc8ACols = kTmaChunk / 4;
+
+template <int kChunk>
+struct Tc8 {
+    static constexpr int kN = 2 * kChunk;      // MMA N
+    static constexpr int kStages = 5;          // weight stages
+    static constexpr int kXStages = 8;         // activation stages
+    static constexpr int kXBytes = 2 * kN * 128;  // two 128-byte K blocks of kN rows
+    static constexpr int kTmemCols = 512;         // accumulators at 0 and kN, A stages from 128
+    static constexpr int kACol0 = 128;
+    static constexpr size_t kMisc = 512 + 4 * kChunk * 4;  // barriers, flags, per-warp maxima
+    static constexpr size_t kSmem = kShmBytes + kMisc + 1024 + (size_t)kStages * kTmaWBytes + (size_t)kXStages * kXBytes;
+    static_assert(2 * kN <= kACol0 && kACol0 + kTc8AStages * kTc8ACols <= kTmemCols, "tensor memory layout");
+    static_assert(kSmem <= 227 * 1024, "tcgen05 gate/up shared memory");
+    static_assert((size_t)kXStages * kXBytes >= kBuildBytes, "table build scratch fits the activation ring");
+};
+
+__device__ __forceinline__ uint64_t tc8_desc_sw128(uint32_t addr) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// kind::i8: signed 8-bit A and B, s32 accumulate, both K-major.
+__host__ __device__ constexpr uint32_t tc8_idesc(int M, int N) {
+    return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void tc8_mma(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void tc8_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc8_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc8_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Every lane waits; the warp goes on only if every lane's wait succeeded.
+__device__ __forceinline__ bool tc8_warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    const bool ok = *abort == 0 && bar_wait_or_abort(bar, parity, kBulkWaitCycles, abort);
+    return __all_sync(0xffffffffu, ok) != 0;
+}
+
+template <int kChunk>
+__global__ void __launch_bounds__(kTc8Threads, 1)
+    experts_w13_tc8_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_s, Params p) {
+    using Cfg = Tc8<kChunk>;
+    constexpr int kStages = Cfg::kStages, kXStages = Cfg::kXStages, kXBytes = Cfg::kXBytes, kN = Cfg::kN;
+    extern __shared__ __align__(128) uint8_t dsm[];
+    Shm& sh = *reinterpret_cast<Shm*>(dsm);
+    uint64_t* full = reinterpret_cast<uint64_t*>(dsm + kShmBytes);  // weight stage landed
+    uint64_t* empty = full + kStages;                                // weight stage converted
+    uint64_t* xfull = empty + kStages;                               // activation stage landed
+    uint64_t* xempty = xfull + kXStages;                             // activation stage consumed by the MMAs
+    uint64_t* a_full = xempty + kXStages;
+    uint64_t* a_empty = a_full + kTc8AStages;
+    uint64_t* acc_full = a_empty + kTc8AStages;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drain = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* never = abort + 1;  // nothing sets it (MOE_TEST_STALL)
+    volatile int* ep_ok = abort + 2;  // [4] per epilogue warp: its accumulator wait succeeded
+    float(*hmx)[kChunk] = reinterpret_cast<float(*)[kChunk]>(dsm + kShmBytes + 512);
+    static_assert((2 * kStages + 2 * kXStages + 2 * kTc8AStages + 5) * 8 + 4 * 7 <= 512, "barrier area");
+    const uint32_t base_s = smem_addr(dsm);
+    const uint32_t ring_s = (base_s + (uint32_t)(kShmBytes + Cfg::kMisc) + 1023u) & ~1023u;
+    uint8_t* wring = dsm + (ring_s - base_s);
+    uint8_t* xring = wring + (size_t)kStages * kTmaWBytes;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int H = p.H, nch = H / kTmaChunk;
+    unsigned* status = &p.ctrl->status;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            bar_init(full + i, 1);   // the tile loads' arrival
+            bar_init(empty + i, 8);  // one arrival per converter warp
+        }
+        for (int i = 0; i < kXStages; ++i) {
+            bar_init(xfull + i, 32);  // one cp.async arrival per lane of the activation warp
+            bar_init(xempty + i, 1);  // the MMAs' commit
+        }
+        for (int i = 0; i < kTc8AStages; ++i) {
+            bar_init(a_full + i, 8);
+            bar_init(a_empty + i, 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            bar_init(acc_full + i, 1);
+            bar_init(acc_empty + i, 4);
+        }
+        bar_init(drain, 1);
+        *abort = 0;
+        *never = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 9) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                     "r"(Cfg::kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc8_fence_before();
+    __syncthreads();
+    tc8_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // the shared expert's first task of this CTA, if its first task is one
+    const int ns = p.Is > 0 ? (p.Is / kRows13) * chunks_of(p.T, p.chunk) : 0;
+    const bool pre = (int)blockIdx.x < ns;
+    const int npre = pre ? min(kStages, nch) : 0;
+    int pre_rbk = 0, pre_tok0 = 0;
+    if (pre) {
+        const int R = p.Is / kRows13, local = ns - 1 - (int)blockIdx.x;
+        pre_rbk = local % R;
+        pre_tok0 = (local / R) * p.chunk;
+        if (warp == 8 && lane == 0)
+            for (int c = 0; c < npre; ++c)
+                issue_w13_chunk(&tm_s, full + c, wring + (size_t)c * kTmaWBytes, c, pre_rbk * kRows13,
+                                p.Is + pre_rbk * kRows13);
+    }
+    if (p.Is > 0) prefetch_l2_slice(p.sh_w13, (size_t)p.Is * p.H);
+    pdl_wait();
+    pdl_release();
+    if (p.decode_groups > 0) build_tables_small(p, sh, reinterpret_cast<int*>(xring));
+    else load_tables(p, p.ts13, &p.ctrl->tasks13, sh.tb, sh.tok);
+    precompute_tasks(p, sh, 0);
+    if (threadIdx.x == 0 && pre) {  // cannot fail with consistent tables
+        const TaskDesc d = sh.td[0];
+        if (!(d.e == p.E && d.rbk == pre_rbk && d.tok0 == pre_tok0 && sh.tb.ntask > (int)blockIdx.x)) {
+            *abort = 1;
+            atomicOr(status, ST_BAD_TASK);
+        }
+    }
+    __syncthreads();
+    const int ntask = sh.tb.ntask;
+    auto task_ok = [&](const TaskDesc& d) { return !(d.e < 0 || d.e > p.E || (d.e == p.E && p.Is == 0)); };
+
+    if (warp == 8) {
+        // ---------------- weight producer: two TMA tiles per k chunk ----------------
+        if (lane == 0) {
+            uint32_t n = 0;
+            int last_round[kStages];
+#pragma unroll
+            for (int s = 0; s < kStages; ++s) last_round[s] = s < npre ? 0 : -1;
+            for (int r = 0; !*abort && snake(blockIdx.x, r) < ntask; ++r) {
+                const TaskDesc d = task_desc(p, sh, 0, r);
+                if (!task_ok(d)) break;  // the epilogue flags it
+                const bool shared = d.e == p.E;
+                const int irow = shared ? p.Is : p.I;
+                const int rg = (shared ? 0 : d.e * 2 * p.I) + d.rbk * kRows13, ru = rg + irow;
+                bool ok = true;
+                for (int c = 0; c < nch; ++c, ++n) {
+                    const int s = n % kStages;
+                    const int round = (int)(n / kStages);
+                    if (round > 0 && !(*abort == 0 && bar_wait_or_abort(empty + s, (round - 1) & 1, kBulkWaitCycles, abort))) {
+                        if (!*abort) atomicOr(status, ST_TIMEOUT);
+                        *abort = 1;
+                        ok = false;
+                        break;
+                    }
+                    if (!(r == 0 && c < npre))  // else issued before the tables were read
+                        issue_w13_chunk(shared ? &tm_s : &tm_r, full + s, wring + (size_t)s * kTmaWBytes, c, rg, ru);
+                    last_round[s] = round;
+                }
+                if (!ok) break;
+            }
+            // every tile load issued lands before the CTA exits
+            for (int s = 0; s < kStages; ++s)
+                if (last_round[s] >= 0) bar_wait(full + s, last_round[s] & 1, kBulkWaitCycles);
+        }
+    } else if (warp == 14) {
+        // ---------------- activation producer: both int8 parts of the task's tokens ----------------
+        uint32_t n = 0;
+        for (int r = 0; !*abort && snake(blockIdx.x, r) < ntask; ++r) {
+            const TaskDesc d = task_desc(p, sh, 0, r);
+            if (!task_ok(d)) break;
+            const bool shared = d.e == p.E;
+            // lane l copies rows l and l + 32 (row r: part r & 1 of the task's token
+            // r >> 1) into the swizzled B layout
+            const int8_t* src[2] = {nullptr, nullptr};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int row = lane + 32 * h;
+                if (row < 2 * d.nc) {
+                    const int tok = slot_token(p, sh, shared, d.off, d.tok0 + (row >> 1));
+                    if (tok >= 0 && tok < p.T) src[h] = p.xq + (size_t)tok * 2 * H + (row & 1) * H;
+                }
+            }
+            bool ok = true;
+            for (int c = 0; c < nch; ++c, ++n) {
+                const int s = n % kXStages;
+                const int round = (int)(n / kXStages);
+                if (round > 0) {
+                    const bool w = *abort == 0 && bar_wait_or_abort(xempty + s, (round - 1) & 1, kBulkWaitCycles, abort);
+                    if (__any_sync(0xffffffffu, !w)) {
+                        if (lane == 0 && !*abort) atomicOr(status, ST_TIMEOUT);
+                        *abort = 1;
+                        ok = false;
+                        break;
+                    }
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    if (src[h]) {
+                        const int row = lane + 32 * h;
+                        uint8_t* dst = xring + (size_t)s * kXBytes + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+                        for (int j = 0; j < kTmaChunk / 16; ++j)
+                            cp_async16(dst + (j >> 3) * (kN * 128) + (((j & 7) ^ (row & 7)) << 4),
+                                       src[h] + c * kTmaChunk + j * 16);
+                    }
+                cp_async_arrive(xfull + s);
+            }
+            if (!ok) break;
+        }
+        cp_async_wait<0>();  // every copy issued lands before the CTA exits
+    } else if (warp == 9) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = tc8_idesc(128, kN);
+            uint32_t n = 0, acc_ph[2] = {0, 0};
+            int buf = 0;
+            bool any = false, ok = true;
+            for (int r = 0; ok && snake(blockIdx.x, r) < ntask; ++r) {
+                if (!task_ok(task_desc(p, sh, 0, r))) break;
+                if (!(*abort == 0 && bar_wait_or_abort(acc_empty + buf, acc_ph[buf] ^ 1u, kBulkWaitCycles, abort))) {
+                    ok = false;
+                    break;
+                }
+                tc8_fence_after();
+                const uint32_t d = tmem + buf * kN;
+                for (int c = 0; c < nch; ++c, ++n) {
+                    const int s = n % kXStages, sa = n % kTc8AStages;
+                    if (!(*abort == 0 && bar_wait_or_abort(xfull + s, (n / kXStages) & 1, kBulkWaitCycles, abort) &&
+                          bar_wait_or_abort(a_full + sa, (n / kTc8AStages) & 1, kBulkWaitCycles, abort))) {
+                        ok = false;
+                        break;
+                    }
+                    tc8_fence_after();
+                    const uint32_t xs = smem_addr(xring + (size_t)s * kXBytes);
+                    const uint32_t acol = tmem + Cfg::kACol0 + sa * kTc8ACols;
+#pragma unroll
+                    for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc8_mma(d, acol + kb * 32 + kk * 8, tc8_desc_sw128(xs + kb * (kN * 128) + kk * 32), idesc,
+                                    (c | kb | kk) != 0);
+                    any = true;
+                    tc8_commit(xempty + s);
+                    tc8_commit(a_empty + sa);
+                }
+                if (!ok) break;
+                tc8_commit(acc_full + buf);
+                acc_ph[buf] ^= 1u;
+                buf ^= 1;
+            }
+            if (!ok && !*abort) *abort = 1;
+            if (any) {  // every MMA issued is complete before tensor memory is freed
+                tc8_commit(drain);
+                bar_wait(drain, 0, kBulkWaitCycles);
+            }
+        }
+    } else if (warp < 8) {
+        // ---------------- converters: int4 codes -> int8 A rows in tensor memory ----------------
+        // warp w writes TMEM lanes 32 (w % 4) .. + 31, the K half w / 4 of the
+        // 256-wide chunk (32 columns of 4 bytes); lane l's row m = 32 (w % 4) + l
+        // is gate row m / 2 (m even) or up row m / 2 (m odd) of the task
+        const int quarter = warp & 3, kh = warp >> 2;
+        const int m = quarter * 32 + lane, i = m >> 1;
+        const uint32_t roff = (uint32_t)((m & 1) ? kTmaWBytes / 2 : 0) + (uint32_t)i * kTmaRowBytes;
+        const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16) + Cfg::kACol0 + kh * 32;
+        uint32_t n = 0;
+        for (int r = 0; snake(blockIdx.x, r) < ntask; ++r) {
+            if (!task_ok(task_desc(p, sh, 0, r))) break;
+            bool ok = true;
+            for (int c = 0; c < nch; ++c, ++n) {
+                const int s = n % kStages, sa = n % kTc8AStages;
+                if (!tc8_warp_wait(full + s, (n / kStages) & 1, abort) ||
+                    !tc8_warp_wait(a_empty + sa, ((n / kTc8AStages) & 1) ^ 1u, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc8_fence_after();
+                const uint32_t wrow = smem_addr(wring + (size_t)s * kTmaWBytes) + roff;
+                uint32_t o[32];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {  // 16-byte chunk 4 kh + j of the row (swizzled)
+                    uint4 w;
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
+                                 : "r"(wrow + ((((uint32_t)(4 * kh + j)) ^ (uint32_t)(i & 7)) << 4)));
+                    o[8 * j + 0] = lo8(w.x); o[8 * j + 1] = hi8(w.x);
+                    o[8 * j + 2] = lo8(w.y); o[8 * j + 3] = hi8(w.y);
+                    o[8 * j + 4] = lo8(w.z); o[8 * j + 5] = hi8(w.z);
+                    o[8 * j + 6] = lo8(w.w); o[8 * j + 7] = hi8(w.w);
+                }
+                asm volatile(
+                    "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+                    "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n"
+                    "tcgen05.wait::st.sync.aligned;\n" ::"r"(tlane + sa * kTc8ACols),
+                    "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7]), "r"(o[8]),
+                    "r"(o[9]), "r"(o[10]), "r"(o[11]), "r"(o[12]), "r"(o[13]), "r"(o[14]), "r"(o[15]), "r"(o[16]),
+                    "r"(o[17]), "r"(o[18]), "r"(o[19]), "r"(o[20]), "r"(o[21]), "r"(o[22]), "r"(o[23]), "r"(o[24]),
+                    "r"(o[25]), "r"(o[26]), "r"(o[27]), "r"(o[28]), "r"(o[29]), "r"(o[30]), "r"(o[31])
+                    : "memory");
+                tc8_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    bar_arrive(a_full + sa);
+                    bar_arrive(empty + s);  // this warp is done with the stage's weights
+                }
+            }
+            if (!ok) break;
+        }
+    } else {
+        // ---------------- epilogue: a lane quarter each (rows 32 q .. 32 q + 31) ----------------
+        const int quarter = warp & 3;
+        const int m = quarter * 32 + lane, i = m >> 1;
+        const bool up = m & 1;
+        if ((p.flags & kFlagTestStall) && warp == 10 && lane == 0) {  // a wait that runs out: the timeout path
+            stall_on_unset_flag(never, kStallCycles);
+            *abort = 1;
+            atomicOr(status, ST_TIMEOUT);
+        }
+        uint32_t acc_ph[2] = {0, 0};
+        int buf = 0;
+        for (int r = 0; snake(blockIdx.x, r) < ntask; ++r) {
+            const TaskDesc d = task_desc(p, sh, 0, r);
+            if (!task_ok(d)) {
+                if (warp == 10 && lane == 0) atomicOr(status, ST_BAD_TASK);
+                break;
+            }
+            const bool shared = d.e == p.E;
+            const int irow = shared ? p.Is : p.I;
+            const float* S = shared ? p.sh_s13 : p.s13 + (size_t)d.e * 2 * p.I;
+            const float rs = __ldg(S + (up ? irow : 0) + d.rbk * kRows13 + i);
+            // token j's activation scale / 16 (the weights are 16 c), on lane j
+            float xsc_l = 0.f;
+            if (lane < d.nc) {
+                const int tok = slot_token(p, sh, shared, d.off, d.tok0 + lane);
+                xsc_l = (tok >= 0 && tok < p.T) ? __ldcg(p.xs + tok) * 0.0625f : 0.f;
+            }
+            const bool got = tc8_warp_wait(acc_full + buf, acc_ph[buf], abort);
+            if (lane == 0) ep_ok[quarter] = got;
+            asm volatile("bar.sync 2, 128;" ::: "memory");  // every epilogue warp's outcome is known
+            if (!(ep_ok[0] && ep_ok[1] && ep_ok[2] && ep_ok[3])) break;
+            tc8_fence_after();
+            const int slot0 = (shared ? 0 : d.off) + d.tok0;
+            float* hcol = (shared ? p.h32_s : p.h32_r) + (size_t)slot0 * irow + d.rbk * kRows13 + i;
+            const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * kN;
+#pragma unroll
+            for (int c0 = 0; c0 < kN; c0 += 32) {  // tokens c0 / 2 .. c0 / 2 + 15
+                uint32_t v[32];
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                    "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+                    "tcgen05.wait::ld.sync.aligned;\n"
+                    : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                      "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+                      "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+                      "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+                      "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                    : "r"(tbase + c0)
+                    : "memory");
+#pragma unroll
+                for (int jj = 0; jj < 16; jj += 2) {  // tokens j0 = c0/2 + jj and j0 + 1
+                    const int j0 = c0 / 2 + jj;
+                    const float x0 = __shfl_sync(0xffffffffu, xsc_l, j0 & 31);
+                    const float x1 = __shfl_sync(0xffffffffu, xsc_l, (j0 + 1) & 31);
+                    const float e0 = join((int)v[2 * jj], (int)v[2 * jj + 1]) * (rs * x0);
+                    const float e1 = join((int)v[2 * jj + 2], (int)v[2 * jj + 3]) * (rs * x1);
+                    // the gate lane takes token j0, the up lane token j0 + 1
+                    const float recv = __shfl_xor_sync(0xffffffffu, up ? e0 : e1, 1);
+                    const float gv = up ? recv : e0, uv = up ? e1 : recv;
+                    const int j = up ? j0 + 1 : j0;
+                    const float h = silu_mul(gv, uv);
+                    float hm = 0.f;
+                    if (j < d.nc) {
+                        hcol[(size_t)j * irow] = h;
+                        hm = fabsf(h);
+                    }
+                    // max over the warp's 16 features (lanes of the same parity)
+                    hm = nanmax(hm, __shfl_xor_sync(0xffffffffu, hm, 2));
+                    hm = nanmax(hm, __shfl_xor_sync(0xffffffffu, hm, 4));
+                    hm = nanmax(hm, __shfl_xor_sync(0xffffffffu, hm, 8));
+                    hm = nanmax(hm, __shfl_xor_sync(0xffffffffu, hm, 16));
+                    if (lane < 2 && j < d.nc) hmx[quarter][j] = hm;
+                }
+            }
+            tc8_fence_before();
+            asm volatile("bar.sync 2, 128;" ::: "memory");  // the four warps' maxima are in
+            if (warp == 10 && lane < d.nc) {
+                const int nrb = irow / kRows13;
+                const float mx = nanmax(nanmax(hmx[0][lane], hmx[1][lane]), nanmax(hmx[2][lane], hmx[3][lane]));
+                (shared ? p.hmax_s : p.hmax_r)[(size_t)(slot0 + lane) * nrb + d.rbk] = mx;
+            }
+            __syncwarp();
+            if (lane == 0) bar_arrive(acc_empty + buf);
+            asm volatile("bar.sync 2, 128;" ::: "memory");  // hmx and ep_ok are read before the next task writes them
+            acc_ph[buf] ^= 1u;
+            buf ^= 1;
+        }
+    }
+    __syncthreads();
+    if (warp == 9) {
+        tc8_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(Cfg::kTmemCols) : "memory");
+    }
+}
+
 // One down task as this thread sees it: ng row groups of 128 rows starting
 // at row0; in group m this thread streams rows row0 + 128 m + j0 + g and + 8.
 struct Task2 {
@@ -1582,7 +2013,7 @@ bool w13_tma(int H) { return H >= kTmaMinH && H % kTmaChunk == 0; }
 
 template <typename Kern>
 int resident(Kern kern, size_t smem, int which, int threads = 256) {
-    static int cache[9][64];  // by kernel (`which`) and device
+    static int cache[10][64];  // by kernel (`which`) and device
     static_assert(kSmem13Bulk <= 227 * 1024, "bulk gate/up shared memory");
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
@@ -1628,6 +2059,14 @@ cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
                                  p.H / 2, p.Is > 0 ? 2 * (uint64_t)p.Is : 2 * (uint64_t)kRows13, kTmaRowBytes, kRows13,
                                  CU_TENSOR_MAP_SWIZZLE_128B);
         if (!ok) return cudaErrorInvalidValue;
+        if (p.chunk == kMaxChunk && experts_w13_tc8(p.H, p.I, p.Is, p.T, p.K, p.E)) {
+            // one CTA per SM, like the mma.sync kernel whose residency sized the grid
+            // (this call also sets the kernel's shared-memory limit)
+            if (resident(experts_w13_tc8_kernel<kMaxChunk>, Tc8<kMaxChunk>::kSmem, 9, kTc8Threads) < grid)
+                return cudaErrorInvalidConfiguration;
+            return launch_pdl(experts_w13_tc8_kernel<kMaxChunk>, g, dim3(kTc8Threads), Tc8<kMaxChunk>::kSmem, stream,
+                              tm_r, tm_s, p);
+        }
         if (p.chunk == kMaxChunk)
             return launch_pdl(experts_w13_tma_kernel<kMaxChunk>, g, dim3(kTmaThreads), Tma13<kMaxChunk>::kSmem, stream,
                               tm_r, tm_s, p);
@@ -1640,6 +2079,17 @@ cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
 }
 
 bool experts_w13_tma(int H) { return w13_tma(H); }
+
+// Picks per routed expert (T*K/E, on average) from which the tcgen05 gate/up
+// kernel runs on the large-batch streaming sequence: measured on the
+// 6144-hidden 256-expert layer, it takes 1.06-1.10 ms at 16 picks per expert
+// against 1.22 ms for the mma.sync kernel, and 0.72 / 0.61 ms at 6 and 2.5
+// (against 0.64 / 0.38 ms).
+constexpr int kTc8MinPicksPerExpert = 12;
+
+bool experts_w13_tc8(int H, int I, int Is, int T, int K, int E) {
+    return w13_tma(H) && experts_w2_tma(H, I, Is) && (long long)T * K >= (long long)kTc8MinPicksPerExpert * E;
+}
 
 bool experts_w2_tma(int H, int I, int Is) { return H >= kTmaMinH && I % kTmaChunk == 0 && Is % kTmaChunk == 0; }
 

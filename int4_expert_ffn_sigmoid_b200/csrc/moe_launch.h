@@ -30,6 +30,10 @@ cudaError_t launch_experts_w2(const Params& p, int grid, cudaStream_t stream);
 int experts_resident_ctas(int which, int H, bool w2_tma, int chunk);
 // Whether the gate/up (down) projection takes the TMA-ring kernel for this shape.
 bool experts_w13_tma(int H);
+// Whether the large-batch streaming sequence runs gate/up on the tcgen05
+// kernel: TMA-ring shapes with at least kTc8MinPicksPerExpert picks per
+// routed expert on average (T*K/E), where it outruns the mma.sync kernel.
+bool experts_w13_tc8(int H, int I, int Is, int T, int K, int E);
 bool experts_w2_tma(int H, int I, int Is);
 // Weighted combine + shared expert (+ residual) -> bf16 out.
 cudaError_t launch_combine(const Params& p, cudaStream_t stream);

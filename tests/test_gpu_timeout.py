@@ -30,14 +30,17 @@ CASES = [
      "prefill"),
     ("TMA-ring weight-streaming kernels", workloads.LayerShape(H=1024, E=64, K=2, I=512, Is=2048, routed_scaling=1.0),
      16, "decode"),
+    ("tcgen05 streaming gate/up kernel", workloads.LayerShape(H=1024, E=64, K=2, I=512, Is=2048, routed_scaling=1.0),
+     400, "decode"),
 ]
 
 
 @pytest.mark.parametrize("case", range(len(CASES)))
 def test_stalled_wait_reports_timeout_then_recovers(moe, cuda_device, case):
     what, shape, T, mode = CASES[case]
-    base = moe.MOE_FORCE_PREFILL if mode == "prefill" else 0
-    path = moe.MOE_PATH_TENSOR_CORE if mode == "prefill" else moe.MOE_PATH_SMALL_BATCH
+    base = moe.MOE_FORCE_PREFILL if mode == "prefill" else (moe.MOE_FORCE_DECODE if T > 64 else 0)
+    path = moe.MOE_PATH_TENSOR_CORE if mode == "prefill" else (moe.MOE_PATH_LARGE_STREAMING if T > 64 else
+                                                                  moe.MOE_PATH_SMALL_BATCH)
     assert moe.layer_path(shape, T, base) == path, what
     layer = workloads.make_layer(shape, 300 + case, 0, cuda_device)
     x = workloads.make_x(shape, T, 300 + case, device=cuda_device)
@@ -62,6 +65,7 @@ PATHS = [
     ("small-batch kernels", workloads.LayerShape(1024, 64, 2, 512, 2048, 1.0), 16, 0),
     ("tensor-core kernels", workloads.LayerShape(512, 16, 8, 256, 384, 2.5), 130, "prefill"),
     ("large-batch streaming kernels", workloads.LayerShape(1024, 64, 2, 512, 2048, 1.0), 150, "decode"),
+    ("large-batch streaming, tcgen05 gate/up", workloads.LayerShape(1024, 64, 2, 512, 2048, 1.0), 400, "decode"),
 ]
 
 
