@@ -262,7 +262,8 @@ class Runner:
         self.xs = [workloads.make_x(wl.shape, T, wl.wid, batch=b, device=device) for b in range(N_BATCHES)]
         self.outs = torch.empty((self.L, T, wl.shape.H), dtype=torch.bfloat16, device=device)
         self.flags = (moe.MOE_ADD_RESIDUAL if wl.residual else 0) | extra_flags
-        if mode == "fused":
+        if mode == "fused":  # the fused kernel wherever it serves the call (not the library's default choice)
+            self.flags |= moe.MOE_STACK_FUSED
             n = moe.stack_workspace_bytes(wl.shape, T, self.L, self.flags)
             self.ws = torch.empty(n, dtype=torch.uint8, device=device)
         else:
@@ -641,7 +642,8 @@ def workload_entry(moe, wl, T, device, steps, warmup, use_graph, flush, peaks, s
     stacked = stacked if stacked is not None else stacked_weights(moe, wl, device)
     L = wl.layers
     modes = ["per_layer"]
-    if moe.stack_path(wl.shape, T, L, moe.MOE_ADD_RESIDUAL if wl.residual else 0) == moe.MOE_PATH_FUSED_STACK:
+    if moe.stack_path(wl.shape, T, L, (moe.MOE_ADD_RESIDUAL if wl.residual else 0) | moe.MOE_STACK_FUSED) == \
+            moe.MOE_PATH_FUSED_STACK:
         modes.insert(0, "fused")
     entry = {"workload": wl.name, "T": T, "layers": L}
     for mode in modes:
@@ -687,7 +689,8 @@ def run_ours(args, rank, world, device, dist):
     use_graph = not args.no_graph
     stacked = stacked_weights(moe, wl, device)
     flags = moe.MOE_ADD_RESIDUAL if wl.residual else 0
-    fused = (not args.per_layer) and moe.stack_path(wl.shape, T, wl.layers, flags) == moe.MOE_PATH_FUSED_STACK
+    fused = (not args.per_layer) and \
+        moe.stack_path(wl.shape, T, wl.layers, flags | moe.MOE_STACK_FUSED) == moe.MOE_PATH_FUSED_STACK
     runner = Runner(moe, wl, T, device, stacked, "fused" if fused else "per_layer",
                     moe.MOE_LOOKAHEAD if (args.lookahead and fused) else 0)
     L = wl.layers
@@ -733,7 +736,8 @@ def run_ours(args, rank, world, device, dist):
         for Ts in wl.tokens:
             row = {}
             for mode in ("fused", "per_layer"):
-                if mode == "fused" and moe.stack_path(wl.shape, Ts, L, flags) != moe.MOE_PATH_FUSED_STACK:
+                if mode == "fused" and \
+                        moe.stack_path(wl.shape, Ts, L, flags | moe.MOE_STACK_FUSED) != moe.MOE_PATH_FUSED_STACK:
                     continue
                 r = runner if (Ts == T and mode == runner.mode) else Runner(moe, wl, Ts, device, stacked, mode)
                 ms = m if r is runner else measure(r, max(10, args.steps // 2), 3, use_graph, flush, peaks, device)

@@ -89,6 +89,10 @@ extern "C" {
                                        0xFF bytes before the kernels run: a kernel that read scratch
                                        it had not written would see NaN / -1; the output must not
                                        change */
+#define MOE_STACK_FUSED (1u << 10)  /* moe_stack_forward: take the fused stack kernel wherever it
+                                       serves the call (by default only where it was measured
+                                       faster than one moe_layer_forward per layer: L >= 2,
+                                       T <= 4, H <= 2048) */
 
 /* Device status word: the first 4 bytes of the workspace hold the OR of these
  * bits after a call completes on the device (0 = no check failed).  Under
@@ -268,8 +272,12 @@ int moe_layer_forward_static_ws(const void* x, const float* router_w, const floa
  * cfg->topk_idx_out / topk_w_out (optional): [L][T][K].
  *
  * Small batches (1 <= T <= 64, H, I and Is multiples of 256, L <= 128, no
- * MOE_FORCE_* flag) run the whole stack in ONE cooperative kernel with one
- * CTA per SM (MOE_PATH_FUSED_STACK): per layer, router units combine the
+ * MOE_FORCE_* flag) can run the whole stack in ONE cooperative kernel with
+ * one CTA per SM (MOE_PATH_FUSED_STACK): by default when L >= 2, T <= 4 and
+ * H <= 2048 (where it was measured faster than the per-layer kernels; at
+ * T = 16 and for the 6144-hidden layer they are faster, at T = 64 the two
+ * are equal), under MOE_STACK_FUSED whenever it serves the call.  The fused
+ * kernel: per layer, router units combine the
  * previous layer's expert outputs, compute the router logits on the tensor
  * cores and select; every CTA then builds the layer's buckets and runs its
  * share of the expert tasks, the down projection of an expert starting as

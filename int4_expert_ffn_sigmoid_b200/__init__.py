@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "MoeError", "moe_cfg_t", "moe_shared_weights_t", "lib", "EXPORTED_SYMBOLS",
     "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK", "MOE_FORCE_DECODE", "MOE_FORCE_PREFILL", "MOE_OUT_F32",
-    "MOE_TEST_STALL", "MOE_LOOKAHEAD", "MOE_TEST_BAD_INDEX", "MOE_TRACE", "MOE_DEBUG_POISON",
+    "MOE_TEST_STALL", "MOE_LOOKAHEAD", "MOE_TEST_BAD_INDEX", "MOE_TRACE", "MOE_DEBUG_POISON", "MOE_STACK_FUSED",
     "MOE_DEVSTAT_TIMEOUT", "MOE_DEVSTAT_BAD_EXPERT", "device_status", "stack_trace",
     "moe_stack_weights_t", "stack_workspace_bytes", "stack_path", "stack_forward", "stack_layers",
     "MOE_PATH_FUSED_STACK", "MOE_PATH_PER_LAYER",
@@ -46,6 +46,7 @@ MOE_TEST_STALL = 1 << 6
 MOE_TEST_BAD_INDEX = 1 << 7
 MOE_TRACE = 1 << 8
 MOE_DEBUG_POISON = 1 << 9
+MOE_STACK_FUSED = 1 << 10
 TRACE_SLOTS = 16  # MOE_TRACE stamps per (CTA, layer)
 # device status word (the first 4 bytes of the workspace)
 MOE_DEVSTAT_BAD_EXPERT = 1 << 0

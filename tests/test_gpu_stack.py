@@ -31,7 +31,9 @@ def run_stack(moe, x, stacked, shape, flags=0):
     T = x.shape[0]
     idx = torch.empty((L, T, shape.K), dtype=torch.int32, device=x.device)
     w = torch.empty((L, T, shape.K), dtype=torch.float32, device=x.device)
-    outs = moe.stack_forward(x, stacked, shape, flags=flags | moe.MOE_DEBUG_CHECK, topk_idx=idx, topk_w=w)
+    # the fused kernel wherever it serves the call (the default takes it only at T <= 4)
+    outs = moe.stack_forward(x, stacked, shape, flags=flags | moe.MOE_DEBUG_CHECK | moe.MOE_STACK_FUSED, topk_idx=idx,
+                             topk_w=w)
     torch.cuda.synchronize()
     return outs, idx, w
 
@@ -43,7 +45,7 @@ def layer_of(stacked, l):
 def check_stack(moe, x, stacked, shape, residual, flags=0, rounded=False, layers_cpu=None, sample=None):
     f = flags | (moe.MOE_ADD_RESIDUAL if residual else 0)
     L = stacked["router_w"].shape[0]
-    assert moe.stack_path(shape, x.shape[0], L, f) == moe.MOE_PATH_FUSED_STACK
+    assert moe.stack_path(shape, x.shape[0], L, f | moe.MOE_STACK_FUSED) == moe.MOE_PATH_FUSED_STACK
     outs, idx, w = run_stack(moe, x, stacked, shape, f)
     worst = 0.0
     for l in range(L):
@@ -149,7 +151,7 @@ def test_fused_stall_reports_timeout_then_recovers(moe, cuda_device, nano_stack)
     wl, stacked, _ = nano_stack
     sub = {k: v[:4].contiguous() for k, v in stacked.items()}
     x = workloads.make_x(wl.shape, 16, wl.wid, batch=8, device=cuda_device)
-    f = moe.MOE_ADD_RESIDUAL | moe.MOE_DEBUG_CHECK
+    f = moe.MOE_ADD_RESIDUAL | moe.MOE_DEBUG_CHECK | moe.MOE_STACK_FUSED
     ws = torch.empty(moe.stack_workspace_bytes(wl.shape, 16, 4, f), dtype=torch.uint8, device=cuda_device)
     good = moe.stack_forward(x, sub, wl.shape, workspace=ws, flags=f).clone()
     assert moe.device_status(ws) == 0

@@ -112,7 +112,7 @@ def test_fused_stack_bad_index_and_poison(moe, cuda_device):
     layers = [workloads.make_layer(shape, 340, l, cuda_device) for l in range(3)]
     stacked = moe.stack_layers(layers)
     x = workloads.make_x(shape, 24, 340, device=cuda_device)
-    f = moe.MOE_ADD_RESIDUAL | moe.MOE_DEBUG_CHECK
+    f = moe.MOE_ADD_RESIDUAL | moe.MOE_DEBUG_CHECK | moe.MOE_STACK_FUSED
     assert moe.stack_path(shape, 24, 3, f) == moe.MOE_PATH_FUSED_STACK
     ws = torch.empty(moe.stack_workspace_bytes(shape, 24, 3, f), dtype=torch.uint8, device=cuda_device)
     good = moe.stack_forward(x, stacked, shape, workspace=ws, flags=f).clone()

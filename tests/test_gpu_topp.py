@@ -84,7 +84,7 @@ def test_topp_fused_stack(moe, cuda_device):
     stacked = moe.stack_layers(layers)
     T = 24
     x = workloads.make_x(shape, T, 370, device=cuda_device)
-    f = moe.MOE_ADD_RESIDUAL | moe.MOE_DEBUG_CHECK
+    f = moe.MOE_ADD_RESIDUAL | moe.MOE_DEBUG_CHECK | moe.MOE_STACK_FUSED
     assert moe.stack_path(shape, T, 3, f) == moe.MOE_PATH_FUSED_STACK
     idx = torch.empty((3, T, shape.K), dtype=torch.int32, device=cuda_device)
     w = torch.empty((3, T, shape.K), dtype=torch.float32, device=cuda_device)
