@@ -510,16 +510,18 @@ def captured_traffic(workload: str, T: int, kernel: str):
     return None
 
 
-def streaming_kernel_names(shape):
+def streaming_kernel_names(shape, T):
     """Gate/up and down kernels of the weight-streaming path for this shape
-    (the library's selection: TMA-ring kernels from H = 1024 on when H, I and
-    Is are multiples of 256; bulk-copy gate/up below; register-ring kernels
-    otherwise)."""
+    and T (the library's selection: TMA-ring kernels from H = 1024 on when H,
+    I and Is are multiples of 256, the tcgen05 gate/up kernel among them on
+    the large-batch sequence at 12 or more picks per routed expert; bulk-copy
+    gate/up below; register-ring kernels otherwise)."""
+    tma2 = shape.H >= 1024 and shape.I % 256 == 0 and shape.Is % 256 == 0
     if shape.H >= 1024 and shape.H % 256 == 0:
-        w13 = "experts_w13_tma_kernel"
+        tc8 = tma2 and T > 64 and T * shape.K >= 12 * shape.E
+        w13 = "experts_w13_tc8_kernel" if tc8 else "experts_w13_tma_kernel"
     else:
         w13 = "experts_w13_bulk_kernel" if shape.H <= 1024 else "experts_w13_kernel"
-    tma2 = shape.H >= 1024 and shape.I % 256 == 0 and shape.Is % 256 == 0
     return w13, "experts_w2_tma_kernel" if tma2 else "experts_w2_kernel"
 
 
@@ -663,7 +665,7 @@ def workload_entry(moe, wl, T, device, steps, warmup, use_graph, flush, peaks, s
             dom = 1 if stage_mean[1] >= stage_mean[2] else 2
             names = moe.STAGE_NAMES
             tc = moe.layer_path(wl.shape, T) == moe.MOE_PATH_TENSOR_CORE
-            w13, w2 = streaming_kernel_names(wl.shape)
+            w13, w2 = streaming_kernel_names(wl.shape, T)
             kname = (f"grouped_gemm_kernel<{dom}>" if tc else (w13 if dom == 1 else w2))
             u = m["uniq"]
             kw = [[stage_work(names[dom], wl.shape, T, x) for x in u[i % N_BATCHES]] for i in range(len(stage_ms))]
@@ -719,7 +721,7 @@ def run_ours(args, rank, world, device, dist):
         names = moe.STAGE_NAMES
         dom = 1 if stage_mean[1] >= stage_mean[2] else 2
         tc = moe.layer_path(wl.shape, T) == moe.MOE_PATH_TENSOR_CORE
-        w13, w2 = streaming_kernel_names(wl.shape)
+        w13, w2 = streaming_kernel_names(wl.shape, T)
         kname = f"grouped_gemm_kernel<{dom}>" if tc else (w13 if dom == 1 else w2)
         kw = [[stage_work(names[dom], wl.shape, T, u) for u in m["uniq"][i % N_BATCHES]] for i in range(len(stage_ms))]
         roofline = roofline_of(statistics.mean(sum(w[0] for w in ws) for ws in kw) / L,
