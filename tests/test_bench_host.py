@@ -87,12 +87,15 @@ def test_captured_traffic_lookup():
 
 def test_streaming_kernel_names_follow_the_library_selection():
     import workloads
-    assert bench.streaming_kernel_names(workloads.NANO) == ("experts_w13_tma_kernel", "experts_w2_tma_kernel")
-    assert bench.streaming_kernel_names(workloads.LARGE) == ("experts_w13_tma_kernel", "experts_w2_tma_kernel")
+    assert bench.streaming_kernel_names(workloads.NANO, 64) == ("experts_w13_tma_kernel", "experts_w2_tma_kernel")
+    assert bench.streaming_kernel_names(workloads.LARGE, 32) == ("experts_w13_tma_kernel", "experts_w2_tma_kernel")
+    # the tcgen05 gate/up kernel from 12 picks per routed expert on the large-batch sequence
+    assert bench.streaming_kernel_names(workloads.LARGE, 200) == ("experts_w13_tma_kernel", "experts_w2_tma_kernel")
+    assert bench.streaming_kernel_names(workloads.LARGE, 512) == ("experts_w13_tc8_kernel", "experts_w2_tma_kernel")
     small = workloads.LayerShape(H=384, E=8, K=2, I=128, Is=128, routed_scaling=1.0)
-    assert bench.streaming_kernel_names(small) == ("experts_w13_bulk_kernel", "experts_w2_kernel")
+    assert bench.streaming_kernel_names(small, 100) == ("experts_w13_bulk_kernel", "experts_w2_kernel")
     odd = workloads.LayerShape(H=1152, E=8, K=2, I=768, Is=256, routed_scaling=1.0)
-    assert bench.streaming_kernel_names(odd) == ("experts_w13_kernel", "experts_w2_tma_kernel")
+    assert bench.streaming_kernel_names(odd, 100) == ("experts_w13_kernel", "experts_w2_tma_kernel")
 
 
 def test_clock_sampler_summary_from_nvml_samples():
