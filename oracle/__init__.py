@@ -60,10 +60,10 @@ def _load():
             lib.oracle_select_topk.argtypes = [_f64p, _f32p, ctypes.c_int32, ctypes.c_int32,
                                                ctypes.c_int32, _i32p, _f64p]
             lib.oracle_expert_ffn.argtypes = [_f64p, ctypes.c_int32, ctypes.c_int32, _u8p, _f32p,
-                                              _u8p, _f32p, _f64p, _f64p]
+                                              _u8p, _f32p, ctypes.c_int32, _f64p, _f64p]
             lib.oracle_moe_tokens.argtypes = (
                 [_u16p] + [ctypes.c_int32] * 6 + [ctypes.c_double, ctypes.c_double, ctypes.c_int32]
-                + [_f32p, _f32p, _u8p, _f32p, _u8p, _f32p, _u8p, _f32p, _u8p, _f32p]
+                + [_f32p, _f32p, _u8p, _f32p, _u8p, _f32p, _u8p, _f32p, _u8p, _f32p, ctypes.c_int32]
                 + [_i32p, ctypes.c_int32, _i32p, _f64p, _i32p, _f64p, _f64p])
             for fn in ("oracle_unpack_int4", "oracle_route", "oracle_select_topk",
                        "oracle_expert_ffn", "oracle_moe_tokens"):
@@ -132,16 +132,28 @@ def select_topk(scores, bias, K: int):
     return idx, margin
 
 
+def weight_bits(w13, H: int) -> int:
+    """Code width of expert weights from their row bytes: H/2 (packed int4) or H (int8)."""
+    n = _np(w13, np.uint8).shape[-1]
+    if n * 2 == H:
+        return 4
+    if n == H:
+        return 8
+    raise ValueError(f"expert rows of {n} bytes fit neither int4 nor int8 codes of {H} elements")
+
+
 def expert_ffn(xvec, w13, s13, w2, s2):
-    """One expert on one token (x given as float64 [H]).  Returns (h, y)."""
+    """One expert on one token (x given as float64 [H]).  Returns (h, y).
+    The code width (int4 or int8) follows from the rows' byte counts."""
     xv = _np(xvec, np.float64)
     a13 = _np(w13, np.uint8); a2 = _np(w2, np.uint8)
     f13 = _np(s13, np.float32); f2 = _np(s2, np.float32)
     H = xv.shape[0]
     I = f13.shape[0] // 2
+    wb = weight_bits(a13, H)
     h = np.empty(I); y = np.empty(H)
     _check(_load().oracle_expert_ffn(_ptr(xv, _f64p), H, I, _ptr(a13, _u8p), _ptr(f13, _f32p),
-                                     _ptr(a2, _u8p), _ptr(f2, _f32p), _ptr(h, _f64p),
+                                     _ptr(a2, _u8p), _ptr(f2, _f32p), wb, _ptr(h, _f64p),
                                      _ptr(y, _f64p)), "expert_ffn")
     return h, y
 
@@ -168,13 +180,14 @@ def moe_tokens(x, layer: dict, shape, residual: bool = False, tokens=None,
     if Is > 0:
         arrs.update(sw13=_np(layer["sh_w13"], np.uint8), ss13=_np(layer["sh_s13"], np.float32),
                     sw2=_np(layer["sh_w2"], np.uint8), ss2=_np(layer["sh_s2"], np.float32))
+    wb = weight_bits(arrs["w13"], H)
     out = np.empty((n, H)); idx = np.empty((n, K), np.int32); w = np.empty((n, K)); m = np.empty(n)
     _check(_load().oracle_moe_tokens(
         _ptr(xb, _u16p), T, H, E, K, I, Is, float(shape.routed_scaling), float(topp), int(bool(residual)),
         _ptr(arrs["rw"], _f32p), _ptr(arrs["rb"], _f32p), _ptr(arrs["w13"], _u8p),
         _ptr(arrs["s13"], _f32p), _ptr(arrs["w2"], _u8p), _ptr(arrs["s2"], _f32p),
         _ptr(arrs.get("sw13"), _u8p), _ptr(arrs.get("ss13"), _f32p),
-        _ptr(arrs.get("sw2"), _u8p), _ptr(arrs.get("ss2"), _f32p),
+        _ptr(arrs.get("sw2"), _u8p), _ptr(arrs.get("ss2"), _f32p), wb,
         _ptr(tok, _i32p), n, _ptr(ov, _i32p), _ptr(out, _f64p), _ptr(idx, _i32p),
         _ptr(w, _f64p), _ptr(m, _f64p)), "moe_tokens")
     return dict(out=out, idx=idx, weights=w, margin=m)

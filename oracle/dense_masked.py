@@ -30,6 +30,16 @@ def decode_int4(packed: np.ndarray) -> np.ndarray:
     return codes
 
 
+def decode_codes(raw: np.ndarray, n: int) -> np.ndarray:
+    """Expert weight bytes [..., n/2] (packed int4) or [..., n] (int8, byte j
+    = element j, two's complement) -> int codes [..., n]."""
+    if raw.shape[-1] * 2 == n:
+        return decode_int4(raw)
+    if raw.shape[-1] == n:
+        return raw.view(np.int8).astype(np.int16)
+    raise ValueError(f"rows of {raw.shape[-1]} bytes fit neither int4 nor int8 codes of {n} elements")
+
+
 def _sigmoid(z):
     return 1.0 / (1.0 + np.exp(-z))
 
@@ -85,16 +95,17 @@ def moe_dense(x, layer: dict, shape, residual: bool = False, forced=None, topp: 
     E, K, I, Is = shape.E, shape.K, shape.I, shape.Is
     R = routing_matrix(xf, _np(layer["router_w"], np.float64), _np(layer["router_bias"], np.float64),
                        K, shape.routed_scaling, forced, topp)
-    W13 = decode_int4(_np(layer["w13"], np.uint8)) * _np(layer["s13"], np.float64)[..., None]
-    W2 = decode_int4(_np(layer["w2"], np.uint8)) * _np(layer["s2"], np.float64)[..., None]
+    H = xf.shape[1]
+    W13 = decode_codes(_np(layer["w13"], np.uint8), H) * _np(layer["s13"], np.float64)[..., None]
+    W2 = decode_codes(_np(layer["w2"], np.uint8), I) * _np(layer["s2"], np.float64)[..., None]
     G = np.einsum("th,eih->tei", xf, W13[:, :I])
     U = np.einsum("th,eih->tei", xf, W13[:, I:])
     Hh = G * _sigmoid(G) * U
     Y = np.einsum("tei,eji->tej", Hh, W2)
     out = np.einsum("te,tej->tj", R, Y)
     if Is > 0:
-        S13 = decode_int4(_np(layer["sh_w13"], np.uint8)) * _np(layer["sh_s13"], np.float64)[:, None]
-        S2 = decode_int4(_np(layer["sh_w2"], np.uint8)) * _np(layer["sh_s2"], np.float64)[:, None]
+        S13 = decode_codes(_np(layer["sh_w13"], np.uint8), H) * _np(layer["sh_s13"], np.float64)[:, None]
+        S2 = decode_codes(_np(layer["sh_w2"], np.uint8), Is) * _np(layer["sh_s2"], np.float64)[:, None]
         g = xf @ S13[:Is].T
         u = xf @ S13[Is:].T
         out = out + (g * _sigmoid(g) * u) @ S2.T

@@ -45,6 +45,12 @@
  * dropped picks become index -1 with weight 0, after the kept ones.
  * Int4 code layout: byte j of a row holds element 2j in bits 0..3 and element
  * 2j+1 in bits 4..7, each a 4-bit two's-complement value in [-8, 7].
+ * Int8 experts (opt-in; nanocolibri-engine README, "Converting a checkpoint
+ * yourself": --ebits sets the expert bits, per-row symmetric with f32 scales;
+ * colibri README, "What's implemented": int8 / packed int4 quantisation
+ * kernels with per-row scales): byte j of a row is element j, an 8-bit
+ * two's-complement value in [-128, 127]; every weight is still code *
+ * row_scale.  `wbits` (4 or 8) tells which layout the expert weights use.
  */
 #include <math.h>
 #include <stdint.h>
@@ -81,10 +87,12 @@ int oracle_unpack_int4(const uint8_t* row, int64_t n, int32_t* codes) {
 
 /* Dot product of a dequantised packed row (code * scale, in double) with a
  * double vector of length n. */
-static double dequant_row_dot(const uint8_t* row, float scale, const double* v, int64_t n) {
+static int int8_code(const uint8_t* row, int64_t j) { return (int)(int8_t)row[j]; }
+
+static double dequant_row_dot(const uint8_t* row, float scale, const double* v, int64_t n, int wbits) {
     double acc = 0.0;
     double s = (double)scale;
-    for (int64_t j = 0; j < n; ++j) acc += ((double)int4_code(row, j) * s) * v[j];
+    for (int64_t j = 0; j < n; ++j) acc += ((double)(wbits == 8 ? int8_code(row, j) : int4_code(row, j)) * s) * v[j];
     return acc;
 }
 
@@ -239,22 +247,23 @@ int oracle_route(const uint16_t* x, const float* W, const float* bias, int32_t T
 }
 
 /* One SwiGLU expert applied to one token.
- * x: double [H]; w13: packed [2I, H/2] (rows 0..I-1 gate, I..2I-1 up);
- * s13: f32 [2I]; w2: packed [H, I/2]; s2: f32 [H].
+ * x: double [H]; w13: [2I, H*wbits/8] (rows 0..I-1 gate, I..2I-1 up);
+ * s13: f32 [2I]; w2: [H, I*wbits/8]; s2: f32 [H]; wbits: 4 (packed int4) or 8.
  * h_out: double [I] (nullable), y: double [H]. */
 int oracle_expert_ffn(const double* x, int32_t H, int32_t I, const uint8_t* w13, const float* s13,
-                      const uint8_t* w2, const float* s2, double* h_out, double* y) {
-    if (!x || !w13 || !s13 || !w2 || !s2 || !y || H <= 0 || I <= 0 || (H & 1) || (I & 1))
+                      const uint8_t* w2, const float* s2, int32_t wbits, double* h_out, double* y) {
+    if (!x || !w13 || !s13 || !w2 || !s2 || !y || H <= 0 || I <= 0 || (H & 1) || (I & 1) ||
+        (wbits != 4 && wbits != 8))
         return ORC_EINVAL;
     double* h = (double*)malloc(sizeof(double) * (size_t)I);
     if (!h) return ORC_ENOMEM;
-    const int64_t row13 = H / 2, row2 = I / 2;
+    const int64_t row13 = (int64_t)H * wbits / 8, row2 = (int64_t)I * wbits / 8;
     for (int32_t r = 0; r < I; ++r) {
-        double g = dequant_row_dot(w13 + (int64_t)r * row13, s13[r], x, H);
-        double u = dequant_row_dot(w13 + (int64_t)(I + r) * row13, s13[I + r], x, H);
+        double g = dequant_row_dot(w13 + (int64_t)r * row13, s13[r], x, H, wbits);
+        double u = dequant_row_dot(w13 + (int64_t)(I + r) * row13, s13[I + r], x, H, wbits);
         h[r] = (g * sigmoid(g)) * u;
     }
-    for (int32_t j = 0; j < H; ++j) y[j] = dequant_row_dot(w2 + (int64_t)j * row2, s2[j], h, I);
+    for (int32_t j = 0; j < H; ++j) y[j] = dequant_row_dot(w2 + (int64_t)j * row2, s2[j], h, I, wbits);
     if (h_out) memcpy(h_out, h, sizeof(double) * (size_t)I);
     free(h);
     return ORC_OK;
@@ -263,8 +272,9 @@ int oracle_expert_ffn(const double* x, int32_t H, int32_t I, const uint8_t* w13,
 /* The layer output for a list of tokens (NULL list = all T tokens, in order).
  *
  * x: bf16 bits [T,H]; router_w f32 [E,H]; router_bias f32 [E];
- * w13 packed [E,2I,H/2]; s13 f32 [E,2I]; w2 packed [E,H,I/2]; s2 f32 [E,H];
- * sh_* the shared expert with intermediate Is (Is = 0: no shared expert).
+ * w13 [E,2I,H*wbits/8]; s13 f32 [E,2I]; w2 [E,H,I*wbits/8]; s2 f32 [E,H];
+ * sh_* the shared expert with intermediate Is (Is = 0: no shared expert), in
+ * the same code layout; wbits: 4 (packed int4) or 8.
  * idx_override [n,K] (nullable): evaluate with these experts instead of the
  * router's choice (weights still come from the router's scores; with top-p,
  * -1 entries are dropped picks).  topp: 0 = plain top-K, else the adaptive
@@ -274,7 +284,7 @@ int oracle_moe_tokens(const uint16_t* x, int32_t T, int32_t H, int32_t E, int32_
                       int32_t Is, double scale, double topp, int32_t residual, const float* router_w,
                       const float* router_bias, const uint8_t* w13, const float* s13,
                       const uint8_t* w2, const float* s2, const uint8_t* sh_w13,
-                      const float* sh_s13, const uint8_t* sh_w2, const float* sh_s2,
+                      const float* sh_s13, const uint8_t* sh_w2, const float* sh_s2, int32_t wbits,
                       const int32_t* tokens, int32_t n_tokens, const int32_t* idx_override,
                       double* out, int32_t* idx_out, double* w_out, double* margin_out) {
     if (!x || !router_w || !router_bias || !w13 || !s13 || !w2 || !s2 || !out) return ORC_EINVAL;
@@ -290,7 +300,8 @@ int oracle_moe_tokens(const uint16_t* x, int32_t T, int32_t H, int32_t E, int32_
     double wts[64];
     int rc = (xt && y && sc && items) ? ORC_OK : ORC_ENOMEM;
     if (K > 64) rc = ORC_EINVAL;
-    const int64_t e13 = (int64_t)2 * I * (H / 2), e2 = (int64_t)H * (I / 2);
+    if (wbits != 4 && wbits != 8) rc = ORC_EINVAL;
+    const int64_t e13 = (int64_t)2 * I * H * wbits / 8, e2 = (int64_t)H * I * wbits / 8;
     for (int32_t i = 0; rc == ORC_OK && i < n; ++i) {
         int32_t t = tokens ? tokens[i] : i;
         if (t < 0 || t >= T) { rc = ORC_EINVAL; break; }
@@ -306,11 +317,11 @@ int oracle_moe_tokens(const uint16_t* x, int32_t T, int32_t H, int32_t E, int32_
             int32_t e = idx[k];
             if (e < 0) continue; /* dropped by the top-p */
             rc = oracle_expert_ffn(xt, H, I, w13 + e * e13, s13 + (int64_t)e * 2 * I, w2 + e * e2,
-                                   s2 + (int64_t)e * H, NULL, y);
+                                   s2 + (int64_t)e * H, wbits, NULL, y);
             for (int h = 0; h < H; ++h) o[h] += wts[k] * y[h];
         }
         if (rc == ORC_OK && Is > 0) {
-            rc = oracle_expert_ffn(xt, H, Is, sh_w13, sh_s13, sh_w2, sh_s2, NULL, y);
+            rc = oracle_expert_ffn(xt, H, Is, sh_w13, sh_s13, sh_w2, sh_s2, wbits, NULL, y);
             for (int h = 0; h < H; ++h) o[h] += y[h];
         }
         if (residual)

@@ -73,6 +73,75 @@ def test_quantiser_bounds_and_roundtrip():
         assert np.isclose(s[r], np.abs(w[r].numpy()).max() / 7, rtol=1e-6)
 
 
+def test_quantiser_int8_bounds_and_roundtrip():
+    g = torch.Generator().manual_seed(6)
+    w = torch.randn(29, 80, generator=g) * 0.02
+    w[5] = 0.0
+    codes8, scale = workloads.quantize_rows_int8(w)
+    assert codes8.shape == (29, 80) and codes8.dtype == torch.uint8
+    codes = codes8.numpy().view(np.int8).astype(np.int64)
+    assert codes.min() >= -127 and codes.max() <= 127
+    s = scale.numpy().astype(np.float64)
+    err = np.abs(w.numpy().astype(np.float64) - codes * s[:, None])
+    assert np.all(err <= s[:, None] / 2 * (1 + 1e-6) + 1e-12)
+    for r in range(29):
+        if r == 5:
+            assert s[r] == 0 and np.all(codes[r] == 0)
+            continue
+        j = int(np.argmax(np.abs(w[r].numpy())))
+        assert abs(codes[r, j]) == 127
+        assert np.isclose(s[r], np.abs(w[r].numpy()).max() / 127, rtol=1e-6)
+
+
+# --- int8 code layout ---------------------------------------------------------
+
+def test_int8_decode_literal():
+    """Byte j of an int8 row is element j in two's complement."""
+    raw = np.array([[0x00, 0x7F, 0x80, 0xFF, 0x01, 0xFE]], np.uint8)
+    assert dense_masked.decode_codes(raw, 6)[0].tolist() == [0, 127, -128, -1, 1, -2]
+    assert dense_masked.decode_codes(np.array([[0x8F]], np.uint8), 2)[0].tolist() == [-1, -8]
+
+
+def test_int8_expert_hand_example():
+    """One int8 expert at x = (1, -2), power-of-two scales, extreme codes:
+    gate (127/128, 2), up (-1, -254/128), h = (-silu(127/128), silu(2) * -254/128),
+    y = (127 h0 - 128 h1, (h0 - h1) / 2)."""
+    silu = lambda z: z / (1 + math.exp(-z))
+    b = lambda v: v & 0xFF
+    w13 = np.array([[b(127), 0], [0, b(-128)], [b(-128), 0], [0, b(127)]], np.uint8)
+    s13 = np.array([2.0 ** -7, 2.0 ** -7, 2.0 ** -7, 2.0 ** -7], np.float32)
+    w2 = np.array([[b(127), b(-128)], [1, b(-1)]], np.uint8)
+    s2 = np.array([1.0, 0.5], np.float32)
+    h, y = oracle.expert_ffn(np.array([1.0, -2.0]), w13, s13, w2, s2)
+    h_exp = [silu(127 / 128) * -1.0, silu(2.0) * (-254 / 128)]
+    np.testing.assert_allclose(h, h_exp, rtol=1e-15)
+    np.testing.assert_allclose(y, [127 * h_exp[0] - 128 * h_exp[1], 0.5 * (h_exp[0] - h_exp[1])], rtol=1e-14)
+
+
+def test_int8_layer_equals_int4_recoded():
+    """An int4 layer re-encoded one code per byte gives the same outputs, bit
+    for bit: the int8 path only changes how codes are read."""
+    shape = workloads.LayerShape(H=32, E=6, K=3, I=16, Is=8, routed_scaling=2.5)
+    layer4 = workloads.make_layer(shape, 91, device="cpu", raw_codes=True)
+    table = np.array([CODE_OF_NIBBLE[v] for v in range(16)], np.int16)
+
+    def recode(packed):
+        p = packed.numpy()
+        codes = np.stack([table[p & 0xF], table[p >> 4]], axis=-1).reshape(*p.shape[:-1], 2 * p.shape[-1])
+        return torch.from_numpy((codes & 0xFF).astype(np.uint8))
+    layer8 = dict(layer4)
+    for k in ("w13", "w2", "sh_w13", "sh_w2"):
+        layer8[k] = recode(layer4[k])
+    assert oracle.weight_bits(layer8["w13"], shape.H) == 8
+    x = workloads.make_x(shape, 6, 91)
+    r4 = oracle.moe_tokens(x, layer4, shape)
+    r8 = oracle.moe_tokens(x, layer8, shape)
+    np.testing.assert_array_equal(r8["out"], r4["out"])
+    np.testing.assert_array_equal(r8["idx"], r4["idx"])
+    d8, _ = dense_masked.moe_dense(x, layer8, shape)
+    np.testing.assert_allclose(d8, r4["out"], rtol=1e-12, atol=1e-13)
+
+
 # --- selection --------------------------------------------------------------
 
 @pytest.mark.parametrize("K", [1, 2, 3])
@@ -204,10 +273,12 @@ def test_hand_example_expert_h():
     dict(H=64, E=16, K=4, I=32, Is=0, scale=2.5, T=5, residual=True, raw=False),
     dict(H=32, E=6, K=6, I=8, Is=8, scale=1.5, T=3, residual=False, raw=True),
     dict(H=16, E=5, K=1, I=4, Is=6, scale=1.0, T=9, residual=True, raw=True),
+    dict(H=32, E=8, K=2, I=16, Is=24, scale=1.0, T=7, residual=False, raw=False, wbits=8),
+    dict(H=16, E=5, K=3, I=6, Is=10, scale=2.5, T=6, residual=True, raw=True, wbits=8),
 ])
 def test_dense_masked_equals_per_token(case):
     shape = workloads.LayerShape(case["H"], case["E"], case["K"], case["I"], case["Is"], case["scale"])
-    layer = workloads.make_layer(shape, 90, device="cpu", raw_codes=case["raw"])
+    layer = workloads.make_layer(shape, 90, device="cpu", raw_codes=case["raw"], wbits=case.get("wbits", 4))
     x = workloads.make_x(shape, case["T"], 90)
     r = oracle.moe_tokens(x, layer, shape, residual=case["residual"])
     dense, R = dense_masked.moe_dense(x, layer, shape, case["residual"])

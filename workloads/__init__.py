@@ -20,6 +20,12 @@ Quantisation rule (per output row r of a [rows, cols] matrix, computed in f32):
 Packing: byte j of a row holds element 2j in bits 0..3 and element 2j+1 in
 bits 4..7, each a 4-bit two's-complement code.
 
+The int8 expert weights (the engine's ``--ebits 8`` conversion, nanocolibri-engine
+README "Converting a checkpoint yourself") use the same per-row rule with 127:
+    scale_r = max_c |w[r, c]| / 127
+    q[r, c] = clamp(round_half_even(w[r, c] / scale_r), -128, 127)
+one byte per element, two's complement, in column order.
+
 Randomness: every tensor is drawn from its own ``torch.Generator`` seeded with
 a fixed integer derived from (workload id, layer, tensor id, chunk), on the
 device the caller asks for.  The CPU and CUDA generators are different
@@ -35,7 +41,7 @@ import torch
 
 __all__ = [
     "LayerShape", "NANO", "LARGE", "LARGE_E32", "Workload", "WORKLOADS",
-    "quantize_rows_int4", "pack_int4", "random_int4_codes",
+    "quantize_rows_int4", "quantize_rows_int8", "pack_int4", "random_int4_codes",
     "make_layer", "make_x", "zipf_bias_path", "load_zipf_bias",
     "layer_weight_bytes", "expert_bytes",
 ]
@@ -147,6 +153,20 @@ def quantize_rows_int4(w: torch.Tensor):
     return pack_int4(q), scale.contiguous()
 
 
+def quantize_rows_int8(w: torch.Tensor):
+    """Per-row symmetric int8 quantisation of an f32 tensor [..., cols].
+
+    Returns (codes uint8 [..., cols], the int8 two's-complement bytes, and
+    scales f32 [...]).  Same rounding and zero-row rule as the int4 quantiser.
+    """
+    w = w.to(torch.float32)
+    scale = w.abs().amax(dim=-1) / 127.0
+    safe = torch.where(scale > 0, scale, torch.ones_like(scale))
+    q = torch.round(w / safe.unsqueeze(-1)).clamp_(-128, 127)
+    q = torch.where(scale.unsqueeze(-1) > 0, q, torch.zeros_like(q)).to(torch.int8)
+    return q.view(torch.uint8).contiguous(), scale.contiguous()
+
+
 def random_int4_codes(shape, generator: torch.Generator, device) -> torch.Tensor:
     """Uniformly random packed bytes: every one of the 16 codes (including -8,
     which the quantiser never emits) appears in both nibbles."""
@@ -180,7 +200,7 @@ def _normal(shape, g, device, std=_WEIGHT_STD):
 
 def make_layer(shape: LayerShape, wid: int, layer: int = 0, device="cpu",
                bias_mode: str = "uniform", raw_codes: bool = False,
-               experts: Optional[Iterable[int]] = None) -> Dict[str, torch.Tensor]:
+               experts: Optional[Iterable[int]] = None, wbits: int = 4) -> Dict[str, torch.Tensor]:
     """Materialise one layer's weights on ``device``.
 
     Returns a dict with router_w f32 [E,H], router_bias f32 [E],
@@ -192,8 +212,15 @@ def make_layer(shape: LayerShape, wid: int, layer: int = 0, device="cpu",
     packed codes with random positive scales (exercises code -8).
     ``experts`` restricts the routed experts that are generated (the others
     stay zero): only used to keep CPU tests small.
+    wbits=8 gives int8 expert and shared weights instead (one byte per
+    element: w13 u8 [E,2I,H], w2 u8 [E,H,I], sh_w13 [2Is,H], sh_w2 [H,Is]);
+    raw_codes then draws every byte value, -128 included.
     """
+    if wbits not in (4, 8):
+        raise ValueError("wbits must be 4 or 8")
     H, E, I, Is = shape.H, shape.E, shape.I, shape.Is
+    per = 2 if wbits == 4 else 1          # elements per byte
+    quant = quantize_rows_int4 if wbits == 4 else quantize_rows_int8
     dev = torch.device(device)
     out: Dict[str, torch.Tensor] = {}
     out["router_w"] = _normal((E, H), _gen(dev, _seed(wid, layer, _TID_RW)), dev)
@@ -207,9 +234,9 @@ def make_layer(shape: LayerShape, wid: int, layer: int = 0, device="cpu",
     else:
         raise ValueError(bias_mode)
 
-    w13 = torch.zeros((E, 2 * I, H // 2), dtype=torch.uint8, device=dev)
+    w13 = torch.zeros((E, 2 * I, H // per), dtype=torch.uint8, device=dev)
     s13 = torch.zeros((E, 2 * I), dtype=torch.float32, device=dev)
-    w2 = torch.zeros((E, H, I // 2), dtype=torch.uint8, device=dev)
+    w2 = torch.zeros((E, H, I // per), dtype=torch.uint8, device=dev)
     s2 = torch.zeros((E, H), dtype=torch.float32, device=dev)
     wanted = set(range(E)) if experts is None else set(int(e) for e in experts)
     for c0 in range(0, E, _EXPERT_CHUNK):
@@ -221,14 +248,14 @@ def make_layer(shape: LayerShape, wid: int, layer: int = 0, device="cpu",
         g2 = _gen(dev, _seed(wid, layer, _TID_W2, chunk))
         n = c1 - c0
         if raw_codes:
-            w13[c0:c1] = random_int4_codes((n, 2 * I, H // 2), g13, dev)
+            w13[c0:c1] = random_int4_codes((n, 2 * I, H // per), g13, dev)
             s13[c0:c1] = torch.rand((n, 2 * I), generator=g13, device=dev).mul_(0.01).add_(0.001)
-            w2[c0:c1] = random_int4_codes((n, H, I // 2), g2, dev)
+            w2[c0:c1] = random_int4_codes((n, H, I // per), g2, dev)
             s2[c0:c1] = torch.rand((n, H), generator=g2, device=dev).mul_(0.01).add_(0.001)
         else:
-            p, s = quantize_rows_int4(_normal((n, 2 * I, H), g13, dev))
+            p, s = quant(_normal((n, 2 * I, H), g13, dev))
             w13[c0:c1], s13[c0:c1] = p, s
-            p, s = quantize_rows_int4(_normal((n, H, I), g2, dev))
+            p, s = quant(_normal((n, H, I), g2, dev))
             w2[c0:c1], s2[c0:c1] = p, s
     if experts is not None:
         keep = torch.zeros(E, dtype=torch.bool, device=dev)
@@ -242,13 +269,13 @@ def make_layer(shape: LayerShape, wid: int, layer: int = 0, device="cpu",
         g13 = _gen(dev, _seed(wid, layer, _TID_SW13))
         g2 = _gen(dev, _seed(wid, layer, _TID_SW2))
         if raw_codes:
-            out["sh_w13"] = random_int4_codes((2 * Is, H // 2), g13, dev)
+            out["sh_w13"] = random_int4_codes((2 * Is, H // per), g13, dev)
             out["sh_s13"] = torch.rand((2 * Is,), generator=g13, device=dev).mul_(0.01).add_(0.001)
-            out["sh_w2"] = random_int4_codes((H, Is // 2), g2, dev)
+            out["sh_w2"] = random_int4_codes((H, Is // per), g2, dev)
             out["sh_s2"] = torch.rand((H,), generator=g2, device=dev).mul_(0.01).add_(0.001)
         else:
-            out["sh_w13"], out["sh_s13"] = quantize_rows_int4(_normal((2 * Is, H), g13, dev))
-            out["sh_w2"], out["sh_s2"] = quantize_rows_int4(_normal((H, Is), g2, dev))
+            out["sh_w13"], out["sh_s13"] = quant(_normal((2 * Is, H), g13, dev))
+            out["sh_w2"], out["sh_s2"] = quant(_normal((H, Is), g2, dev))
     return out
 
 
@@ -260,18 +287,18 @@ def make_x(shape: LayerShape, T: int, wid: int, batch: int = 0, device="cpu",
     return torch.randn((T, shape.H), generator=g, device=device, dtype=torch.float32).mul_(std).to(torch.bfloat16)
 
 
-def expert_bytes(shape: LayerShape) -> int:
-    """Bytes of one routed expert at int4 plus its f32 row scales."""
+def expert_bytes(shape: LayerShape, wbits: int = 4) -> int:
+    """Bytes of one routed expert at int4 (or int8) plus its f32 row scales."""
     H, I = shape.H, shape.I
-    return 3 * H * I // 2 + (2 * I + H) * 4
+    return 3 * H * I * wbits // 8 + (2 * I + H) * 4
 
 
-def layer_weight_bytes(shape: LayerShape) -> Dict[str, int]:
+def layer_weight_bytes(shape: LayerShape, wbits: int = 4) -> Dict[str, int]:
     H, E, I, Is = shape.H, shape.E, shape.I, shape.Is
-    shared = (3 * H * Is // 2 + (2 * Is + H) * 4) if Is else 0
+    shared = (3 * H * Is * wbits // 8 + (2 * Is + H) * 4) if Is else 0
     return {
         "router": E * H * 4 + E * 4,
-        "expert": expert_bytes(shape),
-        "experts_total": E * expert_bytes(shape),
+        "expert": expert_bytes(shape, wbits),
+        "experts_total": E * expert_bytes(shape, wbits),
         "shared": shared,
     }
