@@ -206,13 +206,13 @@ def pci_bus_id(device) -> str:
 
 # --------------------------------------------------------------------------- work accounting
 
-def step_bytes_flops(shape, T, uniq_per_layer):
+def step_bytes_flops(shape, T, uniq_per_layer, wbits=4):
     """Algorithmic bytes and flops of one pass over the layers.
 
     bytes: router W + bias, shared-expert weights + scales, every touched
     routed expert's weights + scales, x in and out (bf16).  Scratch excluded.
     flops: 2*T*E*H + 6*T*K*H*I + 6*T*H*Is per layer."""
-    lb = workloads.layer_weight_bytes(shape)
+    lb = workloads.layer_weight_bytes(shape, wbits)
     H, E, K, I, Is = shape.H, shape.E, shape.K, shape.I, shape.Is
     nbytes = 0
     for u in uniq_per_layer:
@@ -221,7 +221,7 @@ def step_bytes_flops(shape, T, uniq_per_layer):
     return nbytes, flops
 
 
-def stage_work(stage, shape, T, uniq):
+def stage_work(stage, shape, T, uniq, wbits=4):
     """Algorithmic (bytes, flops) of one launch of a layer stage.
 
     gate_up: the w13 codes + scales of every touched routed expert and of the
@@ -230,14 +230,15 @@ def stage_work(stage, shape, T, uniq):
     real tokens count (no tile padding), scratch traffic beyond that is not
     algorithmic."""
     H, K, I, Is = shape.H, shape.K, shape.I, shape.Is
+    cb = 8 // wbits  # code elements per byte
     if stage == "gate_up":
-        per_expert = 2 * I * H // 2 + 2 * I * 4
-        shared = (2 * Is * H // 2 + 2 * Is * 4) if Is else 0
+        per_expert = 2 * I * H // cb + 2 * I * 4
+        shared = (2 * Is * H // cb + 2 * Is * 4) if Is else 0
         nbytes = uniq * per_expert + shared + T * H * 2 + T * K * I * 2 + T * Is * 2
         flops = 4 * T * K * H * I + 4 * T * H * Is
     elif stage == "down":
-        per_expert = H * I // 2 + H * 4
-        shared = (H * Is // 2 + H * 4) if Is else 0
+        per_expert = H * I // cb + H * 4
+        shared = (H * Is // cb + H * 4) if Is else 0
         nbytes = uniq * per_expert + shared + T * K * I * 2 + T * Is * 2 + (T * K + (T if Is else 0)) * H * 4
         flops = 2 * T * K * H * I + 2 * T * H * Is
     else:
@@ -262,12 +263,13 @@ class Runner:
         self.xs = [workloads.make_x(wl.shape, T, wl.wid, batch=b, device=device) for b in range(N_BATCHES)]
         self.outs = torch.empty((self.L, T, wl.shape.H), dtype=torch.bfloat16, device=device)
         self.flags = (moe.MOE_ADD_RESIDUAL if wl.residual else 0) | extra_flags
+        self.flags |= moe.MOE_WEIGHTS_INT8 if wl.wbits == 8 else 0
         if mode == "fused":  # the fused kernel wherever it serves the call (not the library's default choice)
             self.flags |= moe.MOE_STACK_FUSED
             n = moe.stack_workspace_bytes(wl.shape, T, self.L, self.flags)
             self.ws = torch.empty(n, dtype=torch.uint8, device=device)
         else:
-            self.ws = moe.new_workspace(wl.shape, T, device)
+            self.ws = moe.new_workspace(wl.shape, T, device, self.flags)
 
     def run(self, b, x=None, stage_events=None, topk_idx=None):
         inp = self.xs[b] if x is None else x
@@ -299,7 +301,10 @@ class Runner:
     def launches_per_step(self):
         if self.mode == "fused":
             return 1
-        return self.moe.kernel_launches(self.shape, self.T) * self.L
+        return self.moe.kernel_launches(self.shape, self.T, self.flags) * self.L
+
+    def path(self):
+        return self.moe.layer_path(self.shape, self.T, self.flags)
 
 
 def make_events(n):
@@ -619,7 +624,7 @@ def roofline_of(alg_b, alg_f, seconds, peaks, kernel, timing, traffic=None):
 
 
 def stacked_weights(moe, wl, device):
-    layers = [workloads.make_layer(wl.shape, wl.wid, l, device, wl.bias_mode) for l in range(wl.layers)]
+    layers = [workloads.make_layer(wl.shape, wl.wid, l, device, wl.bias_mode, wbits=wl.wbits) for l in range(wl.layers)]
     st = moe.stack_layers(layers)
     del layers
     torch.cuda.empty_cache()
@@ -631,7 +636,7 @@ def measure(runner, steps, warmup, use_graph, flush, peaks, device, barrier=None
     uniq = runner.routing_unique()
     with ClockSampler(device.index if device.index is not None else 0, pci_bus_id(device)) as clk:
         ms, _ = timed_steps(runner, steps, warmup, use_graph, flush, dist_barrier=barrier)
-    work = [step_bytes_flops(runner.shape, runner.T, uniq[i % N_BATCHES]) for i in range(steps)]
+    work = [step_bytes_flops(runner.shape, runner.T, uniq[i % N_BATCHES], runner.wl.wbits) for i in range(steps)]
     return {"ms": ms, "uniq": uniq, "clocks": clk.summary(), "bytes": statistics.mean(w[0] for w in work),
             "flops": statistics.mean(w[1] for w in work)}
 
@@ -647,7 +652,7 @@ def workload_entry(moe, wl, T, device, steps, warmup, use_graph, flush, peaks, s
     if moe.stack_path(wl.shape, T, L, (moe.MOE_ADD_RESIDUAL if wl.residual else 0) | moe.MOE_STACK_FUSED) == \
             moe.MOE_PATH_FUSED_STACK:
         modes.insert(0, "fused")
-    entry = {"workload": wl.name, "T": T, "layers": L}
+    entry = {"workload": wl.name, "T": T, "layers": L, "expert_bits": wl.wbits}
     for mode in modes:
         r = Runner(moe, wl, T, device, stacked, mode)
         m = measure(r, steps, warmup, use_graph, flush, peaks, device)
@@ -658,17 +663,18 @@ def workload_entry(moe, wl, T, device, steps, warmup, use_graph, flush, peaks, s
              "clocks": m["clocks"], "gpu_launches_per_step": r.launches_per_step(),
              "path": "fused stack kernel" if mode == "fused" else
                      {moe.MOE_PATH_SMALL_BATCH: "small-batch kernels", moe.MOE_PATH_TENSOR_CORE: "tensor-core kernels",
-                      moe.MOE_PATH_LARGE_STREAMING: "large-batch streaming kernels"}[moe.layer_path(wl.shape, T)]}
+                      moe.MOE_PATH_LARGE_STREAMING: "large-batch streaming kernels"}[r.path()]}
         if mode == "per_layer":
             _, stage_ms = timed_steps(r, max(3, steps // 2), 2, use_graph, flush, instrumented=True)
             stage_mean = [statistics.mean(s[k] for s in stage_ms) for k in range(4)]
             dom = 1 if stage_mean[1] >= stage_mean[2] else 2
             names = moe.STAGE_NAMES
-            tc = moe.layer_path(wl.shape, T) == moe.MOE_PATH_TENSOR_CORE
+            tc = r.path() == moe.MOE_PATH_TENSOR_CORE
             w13, w2 = streaming_kernel_names(wl.shape, T)
-            kname = (f"grouped_gemm_kernel<{dom}>" if tc else (w13 if dom == 1 else w2))
+            kname = (f"grouped_gemm_kernel<{dom}, {wl.wbits}>" if tc else (w13 if dom == 1 else w2))
             u = m["uniq"]
-            kw = [[stage_work(names[dom], wl.shape, T, x) for x in u[i % N_BATCHES]] for i in range(len(stage_ms))]
+            kw = [[stage_work(names[dom], wl.shape, T, x, wl.wbits) for x in u[i % N_BATCHES]]
+                  for i in range(len(stage_ms))]
             kb = statistics.mean(sum(w[0] for w in ws) for ws in kw) / L
             kf = statistics.mean(sum(w[1] for w in ws) for ws in kw) / L
             d["stages_us_per_step"] = {names[k]: round(stage_mean[k] * 1e3, 2) for k in range(4)}
@@ -720,10 +726,11 @@ def run_ours(args, rank, world, device, dist):
         stage_mean = [statistics.mean(s[k] for s in stage_ms) for k in range(4)]
         names = moe.STAGE_NAMES
         dom = 1 if stage_mean[1] >= stage_mean[2] else 2
-        tc = moe.layer_path(wl.shape, T) == moe.MOE_PATH_TENSOR_CORE
+        tc = runner.path() == moe.MOE_PATH_TENSOR_CORE
         w13, w2 = streaming_kernel_names(wl.shape, T)
-        kname = f"grouped_gemm_kernel<{dom}>" if tc else (w13 if dom == 1 else w2)
-        kw = [[stage_work(names[dom], wl.shape, T, u) for u in m["uniq"][i % N_BATCHES]] for i in range(len(stage_ms))]
+        kname = f"grouped_gemm_kernel<{dom}, {wl.wbits}>" if tc else (w13 if dom == 1 else w2)
+        kw = [[stage_work(names[dom], wl.shape, T, u, wl.wbits) for u in m["uniq"][i % N_BATCHES]]
+              for i in range(len(stage_ms))]
         roofline = roofline_of(statistics.mean(sum(w[0] for w in ws) for ws in kw) / L,
                                statistics.mean(sum(w[1] for w in ws) for ws in kw) / L,
                                stage_mean[dom] / L / 1e3, peaks, kname,
@@ -758,7 +765,8 @@ def run_ours(args, rank, world, device, dist):
         extra = []
         steps = max(10, args.steps)
         for name, Ts_list in (("nano_layer_t16", (16,)), ("nano_prefill_t4096", (4096,)),
-                              ("nano_zipf_t16384", (16384,)), ("large_layer", (1, 32, 512))):
+                              ("nano_prefill_t4096_int8", (4096,)), ("nano_zipf_t16384", (16384,)),
+                              ("large_layer", (1, 32, 512))):
             w2l = workloads.WORKLOADS[name]
             st = stacked_weights(moe, w2l, device)
             for Ts in Ts_list:
@@ -776,7 +784,7 @@ def run_ours(args, rank, world, device, dist):
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_mean, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "int8" if runner.mode == "fused" or moe.layer_path(wl.shape, T) != moe.MOE_PATH_TENSOR_CORE else "bf16",
+        "dtype": "int8" if runner.mode == "fused" or runner.path() != moe.MOE_PATH_TENSOR_CORE else "bf16",
         "dtype_note": "weight-streaming arithmetic: int4 codes as int8, activations as two int8 parts, exact int32 "
                       "products, f32 router, scales and sums, bf16 in and out",
         "data": "synthetic",
@@ -814,7 +822,7 @@ def run_reference(args, rank, world):
         return None
     wl = workloads.WORKLOADS[args.workload]
     T = args.tokens or max(wl.tokens)
-    layers = [workloads.make_layer(wl.shape, wl.wid, l, "cpu", wl.bias_mode) for l in range(wl.layers)]
+    layers = [workloads.make_layer(wl.shape, wl.wid, l, "cpu", wl.bias_mode, wbits=wl.wbits) for l in range(wl.layers)]
     xs = [workloads.make_x(wl.shape, T, wl.wid, batch=b, device="cpu") for b in range(N_BATCHES)]
     n_tok = min(T, 4)
 

@@ -93,6 +93,15 @@ extern "C" {
                                        serves the call (by default only where it was measured
                                        faster than one moe_layer_forward per layer: L >= 2,
                                        T <= 4, H <= 2048) */
+#define MOE_WEIGHTS_INT8 (1u << 11) /* the expert weights (routed and shared) are int8 codes, one
+                                       byte per element: w13 [E][2I][H], w2 [E][H][I], shared
+                                       w13 [2Is][H], w2 [H][Is] (byte j of a row = element j, two's
+                                       complement; weight = code * row scale).  Every T takes the
+                                       tensor-core sequence (H a multiple of 256, else
+                                       MOE_ERR_UNSUPPORTED; MOE_FORCE_DECODE is MOE_ERR_INVALID_ARG).
+                                       Expert bit width of the checkpoint converter:
+                                       nanocolibri-engine README, "Converting a checkpoint
+                                       yourself" */
 
 /* Device status word: the first 4 bytes of the workspace hold the OR of these
  * bits after a call completes on the device (0 = no check failed).  Under
@@ -107,7 +116,8 @@ extern "C" {
  *   w13: uint8 [2*Is][H/2]  rows 0..Is-1 gate, rows Is..2*Is-1 up
  *   s13: f32   [2*Is]       one scale per w13 row
  *   w2 : uint8 [H][Is/2]
- *   s2 : f32   [H] */
+ *   s2 : f32   [H]
+ * (under MOE_WEIGHTS_INT8: w13 [2*Is][H], w2 [H][Is]) */
 typedef struct moe_shared_weights {
     const uint8_t* w13;
     const float* s13;
@@ -184,6 +194,7 @@ size_t moe_layer_workspace_bytes_upto(const moe_cfg_t* cfg, int32_t N);
  *   scales13   : f32  [E][2I]
  *   packed_w2  : uint8 [E][H][I/2]
  *   scales2    : f32  [E][H]
+ *                (under MOE_WEIGHTS_INT8: packed_w13 [E][2I][H], packed_w2 [E][H][I])
  *   shared_w   : the shared expert (required when cfg->Is > 0, else ignored)
  *   out        : bf16 [T][H]  (written; one round-to-nearest-even of the f32 sum),
  *                or f32 [T][H] under MOE_OUT_F32
@@ -205,9 +216,11 @@ size_t moe_layer_workspace_bytes_upto(const moe_cfg_t* cfg, int32_t N);
  *    that magnitude (rows whose largest magnitude is below 2^-113 become
  *    zero; a row holding NaN or infinity gives NaN outputs).  Weight codes
  *    times activation parts accumulate exactly in int32; h is kept in f32.
- *  - otherwise: tensor-core kernels with bf16 x, f32 accumulation, and h
- *    kept in fp16 as h * 2^-k_t with a per-token power of two 2^-k_t that
- *    keeps it in fp16's normal range.
+ *  - otherwise (and at every T under MOE_WEIGHTS_INT8): tensor-core kernels
+ *    with bf16 x, f32 accumulation, and h kept in fp16 as h * 2^-k_t with a
+ *    per-token power of two 2^-k_t that keeps it in fp16's normal range.
+ *    Weight codes (int4 or int8) enter the MMAs exactly as 16-bit values;
+ *    the row scales are applied to the f32 accumulators.
  * Expert outputs and their weighted sum are f32 until the output rounding.
  * Returns MOE_OK or an MOE_ERR_* code; on an error nothing is launched
  * (except MOE_ERR_CUDA / MOE_ERR_DEVICE_CHECK, raised after launching). */
@@ -267,7 +280,9 @@ int moe_layer_forward_static_ws(const void* x, const float* router_w, const floa
  *   w13 [L][E][2I][H/2] uint8, s13 [L][E][2I] f32,
  *   w2 [L][E][H][I/2] uint8, s2 [L][E][H] f32,
  *   shared.w13 [L][2Is][H/2], shared.s13 [L][2Is], shared.w2 [L][H][Is/2],
- *   shared.s2 [L][H].
+ *   shared.s2 [L][H]
+ * (under MOE_WEIGHTS_INT8 the code rows are H, I and Is bytes long, and every
+ * layer takes its own moe_layer_forward call).
  * outs: bf16 [L][T][H]; layer l writes outs[l], which is layer l+1's input.
  * cfg->topk_idx_out / topk_w_out (optional): [L][T][K].
  *

@@ -20,6 +20,7 @@ __all__ = [
     "MoeError", "moe_cfg_t", "moe_shared_weights_t", "lib", "EXPORTED_SYMBOLS",
     "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK", "MOE_FORCE_DECODE", "MOE_FORCE_PREFILL", "MOE_OUT_F32",
     "MOE_TEST_STALL", "MOE_LOOKAHEAD", "MOE_TEST_BAD_INDEX", "MOE_TRACE", "MOE_DEBUG_POISON", "MOE_STACK_FUSED",
+    "MOE_WEIGHTS_INT8", "weight_flags",
     "MOE_DEVSTAT_TIMEOUT", "MOE_DEVSTAT_BAD_EXPERT", "device_status", "stack_trace",
     "moe_stack_weights_t", "stack_workspace_bytes", "stack_path", "stack_forward", "stack_layers",
     "MOE_PATH_FUSED_STACK", "MOE_PATH_PER_LAYER",
@@ -47,6 +48,7 @@ MOE_TEST_BAD_INDEX = 1 << 7
 MOE_TRACE = 1 << 8
 MOE_DEBUG_POISON = 1 << 9
 MOE_STACK_FUSED = 1 << 10
+MOE_WEIGHTS_INT8 = 1 << 11
 TRACE_SLOTS = 16  # MOE_TRACE stamps per (CTA, layer)
 # device status word (the first 4 bytes of the workspace)
 MOE_DEVSTAT_BAD_EXPERT = 1 << 0
@@ -216,6 +218,17 @@ def _check_dev(name, t, dtype, shape=None):
         raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
+def weight_flags(layer: dict, shape) -> int:
+    """MOE_WEIGHTS_INT8 when ``layer``'s expert codes are one byte per element
+    (w13 rows of H bytes), 0 for packed int4 (H/2 bytes)."""
+    n = layer["w13"].shape[-1]
+    if n == shape.H:
+        return MOE_WEIGHTS_INT8
+    if 2 * n == shape.H:
+        return 0
+    raise ValueError(f"w13 rows of {n} bytes fit neither int4 nor int8 codes of H={shape.H}")
+
+
 def layer_forward(x: torch.Tensor, layer: dict, shape, out: Optional[torch.Tensor] = None,
                   workspace: Optional[torch.Tensor] = None, flags: int = 0,
                   topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
@@ -224,23 +237,25 @@ def layer_forward(x: torch.Tensor, layer: dict, shape, out: Optional[torch.Tenso
 
     ``layer`` holds router_w, router_bias, w13, s13, w2, s2 and, when
     shape.Is > 0, sh_w13, sh_s13, sh_w2, sh_s2 (the layout of
-    ``workloads.make_layer``).  Returns ``out`` (bf16 [T, H]).  ``stage_events``:
+    ``workloads.make_layer``).  With int8 expert weights (one byte per element)
+    ``flags`` must hold MOE_WEIGHTS_INT8.  Returns ``out`` (bf16 [T, H]).  ``stage_events``:
     optional sequence of 2*MOE_NUM_STAGES ``torch.cuda.Event`` already recorded
     once (so that they exist); the library records them around each stage."""
     T = x.shape[0]
     H, E, I, Is = shape.H, shape.E, shape.I, shape.Is
+    per = 1 if flags & MOE_WEIGHTS_INT8 else 2  # code elements per byte
     _check_dev("x", x, torch.bfloat16, (T, H))
     _check_dev("router_w", layer["router_w"], torch.float32, (E, H))
     _check_dev("router_bias", layer["router_bias"], torch.float32, (E,))
-    _check_dev("w13", layer["w13"], torch.uint8, (E, 2 * I, H // 2))
+    _check_dev("w13", layer["w13"], torch.uint8, (E, 2 * I, H // per))
     _check_dev("s13", layer["s13"], torch.float32, (E, 2 * I))
-    _check_dev("w2", layer["w2"], torch.uint8, (E, H, I // 2))
+    _check_dev("w2", layer["w2"], torch.uint8, (E, H, I // per))
     _check_dev("s2", layer["s2"], torch.float32, (E, H))
     sh = moe_shared_weights_t()
     if Is > 0:
-        _check_dev("sh_w13", layer["sh_w13"], torch.uint8, (2 * Is, H // 2))
+        _check_dev("sh_w13", layer["sh_w13"], torch.uint8, (2 * Is, H // per))
         _check_dev("sh_s13", layer["sh_s13"], torch.float32, (2 * Is,))
-        _check_dev("sh_w2", layer["sh_w2"], torch.uint8, (H, Is // 2))
+        _check_dev("sh_w2", layer["sh_w2"], torch.uint8, (H, Is // per))
         _check_dev("sh_s2", layer["sh_s2"], torch.float32, (H,))
         sh.w13, sh.s13 = layer["sh_w13"].data_ptr(), layer["sh_s13"].data_ptr()
         sh.w2, sh.s2 = layer["sh_w2"].data_ptr(), layer["sh_s2"].data_ptr()
@@ -297,21 +312,22 @@ def stack_forward(x: torch.Tensor, stacked: dict, shape, outs: Optional[torch.Te
     T = x.shape[0]
     H, E, K, I, Is = shape.H, shape.E, shape.K, shape.I, shape.Is
     L = stacked["router_w"].shape[0]
+    per = 1 if flags & MOE_WEIGHTS_INT8 else 2  # code elements per byte
     _check_dev("x", x, torch.bfloat16, (T, H))
     _check_dev("router_w", stacked["router_w"], torch.float32, (L, E, H))
     _check_dev("router_bias", stacked["router_bias"], torch.float32, (L, E))
-    _check_dev("w13", stacked["w13"], torch.uint8, (L, E, 2 * I, H // 2))
+    _check_dev("w13", stacked["w13"], torch.uint8, (L, E, 2 * I, H // per))
     _check_dev("s13", stacked["s13"], torch.float32, (L, E, 2 * I))
-    _check_dev("w2", stacked["w2"], torch.uint8, (L, E, H, I // 2))
+    _check_dev("w2", stacked["w2"], torch.uint8, (L, E, H, I // per))
     _check_dev("s2", stacked["s2"], torch.float32, (L, E, H))
     w = moe_stack_weights_t()
     w.router_w, w.router_bias = stacked["router_w"].data_ptr(), stacked["router_bias"].data_ptr()
     w.w13, w.s13 = stacked["w13"].data_ptr(), stacked["s13"].data_ptr()
     w.w2, w.s2 = stacked["w2"].data_ptr(), stacked["s2"].data_ptr()
     if Is > 0:
-        _check_dev("sh_w13", stacked["sh_w13"], torch.uint8, (L, 2 * Is, H // 2))
+        _check_dev("sh_w13", stacked["sh_w13"], torch.uint8, (L, 2 * Is, H // per))
         _check_dev("sh_s13", stacked["sh_s13"], torch.float32, (L, 2 * Is))
-        _check_dev("sh_w2", stacked["sh_w2"], torch.uint8, (L, H, Is // 2))
+        _check_dev("sh_w2", stacked["sh_w2"], torch.uint8, (L, H, Is // per))
         _check_dev("sh_s2", stacked["sh_s2"], torch.float32, (L, H))
         w.shared.w13, w.shared.s13 = stacked["sh_w13"].data_ptr(), stacked["sh_s13"].data_ptr()
         w.shared.w2, w.shared.s2 = stacked["sh_w2"].data_ptr(), stacked["sh_s2"].data_ptr()
@@ -357,14 +373,17 @@ def device_status(workspace: torch.Tensor) -> int:
 class MoELayer:
     """One layer's device weights plus a workspace sized for every call of up
     to ``max_tokens`` tokens under any per-call flags (the kernel sequence,
-    and so the workspace, depends on MOE_FORCE_DECODE / MOE_FORCE_PREFILL)."""
+    and so the workspace, depends on MOE_FORCE_DECODE / MOE_FORCE_PREFILL).
+    The code width of the expert weights (int4 or int8) is read from their
+    shapes and its flag added to every call."""
 
     def __init__(self, layer: dict, shape, max_tokens: int, device=None):
         self.layer = layer
         self.shape = shape
         self.device = torch.device(device) if device is not None else layer["w13"].device
         self.max_tokens = int(max_tokens)
-        n = max(workspace_bytes_upto(shape, self.max_tokens, f)
+        self.weight_flags = weight_flags(layer, shape)
+        n = max(workspace_bytes_upto(shape, self.max_tokens, f | self.weight_flags)
                 for f in (0, MOE_FORCE_DECODE, MOE_FORCE_PREFILL))
         if n == 0:
             raise MoeError(MOE_ERR_UNSUPPORTED, "moe_layer_workspace_bytes")
@@ -374,6 +393,6 @@ class MoELayer:
                  flags: int = 0, topk_idx=None, topk_w=None, stage_events=None) -> torch.Tensor:
         if x.shape[0] > self.max_tokens:
             raise ValueError(f"T={x.shape[0]} exceeds max_tokens={self.max_tokens}")
-        f = flags | (MOE_ADD_RESIDUAL if residual else 0)
+        f = flags | self.weight_flags | (MOE_ADD_RESIDUAL if residual else 0)
         return layer_forward(x, self.layer, self.shape, out=out, workspace=self.workspace, flags=f,
                              topk_idx=topk_idx, topk_w=topk_w, stage_events=stage_events)

@@ -15,12 +15,12 @@ using namespace moe;
 
 constexpr unsigned kKnownFlags = MOE_ADD_RESIDUAL | MOE_DEBUG_CHECK | MOE_FORCE_DECODE | MOE_FORCE_PREFILL |
                                  MOE_OUT_F32 | MOE_TEST_STALL | MOE_LOOKAHEAD | MOE_TEST_BAD_INDEX |
-                                 MOE_TRACE | MOE_DEBUG_POISON | MOE_STACK_FUSED;
+                                 MOE_TRACE | MOE_DEBUG_POISON | MOE_STACK_FUSED | MOE_WEIGHTS_INT8;
 // Traced CTAs at most (the fused kernel runs one CTA per SM).
 constexpr int kMaxGridF = 256;
 static_assert(kFlagResidual == MOE_ADD_RESIDUAL && kFlagOutF32 == MOE_OUT_F32 && kFlagTestStall == MOE_TEST_STALL &&
                   kFlagLookahead == MOE_LOOKAHEAD && kFlagTestBadIndex == MOE_TEST_BAD_INDEX &&
-                  kFlagTrace == MOE_TRACE,
+                  kFlagTrace == MOE_TRACE && kFlagWeightsInt8 == MOE_WEIGHTS_INT8,
               "kernel flag bits match the C ABI");
 static_assert(ST_BAD_EXPERT == MOE_DEVSTAT_BAD_EXPERT && ST_BAD_SLOT == MOE_DEVSTAT_BAD_SLOT &&
                   ST_BAD_COUNT == MOE_DEVSTAT_BAD_COUNT && ST_BAD_TASK == MOE_DEVSTAT_BAD_TASK &&
@@ -31,8 +31,9 @@ constexpr int32_t kMaxTokens = 1 << 20;
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Kernel sequence of a call: the small-batch router + weight-streaming
-// experts; the large router + tensor-core grouped GEMMs; or the large router
-// + weight-streaming experts (H not a multiple of 256, or MOE_FORCE_DECODE).
+// experts; the large router + tensor-core grouped GEMMs (every T with int8
+// expert weights); or the large router + weight-streaming experts (H not a
+// multiple of 256, or MOE_FORCE_DECODE).
 enum class Path { kSmall, kTensorCore, kLargeStreaming };
 
 // Average (token, pick) slots per routed expert below which large batches
@@ -42,6 +43,7 @@ enum class Path { kSmall, kTensorCore, kLargeStreaming };
 constexpr int kTcMinSlotsPerExpert = 32;
 
 Path choose_path(const moe_cfg_t& c, int32_t T) {
+    if (c.flags & MOE_WEIGHTS_INT8) return Path::kTensorCore;
     if (T <= kDecodeMaxTokens && !(c.flags & MOE_FORCE_PREFILL)) return Path::kSmall;
     // GEMM-2 of the tensor-core path tiles 256 output columns
     if ((c.flags & MOE_FORCE_DECODE) || c.H % 256 != 0) return Path::kLargeStreaming;
@@ -116,7 +118,11 @@ int validate_cfg(const moe_cfg_t* c) {
     if (!(c->topp >= 0.0f) || !isfinite(c->topp)) return MOE_ERR_INVALID_ARG;
     if (c->flags & ~kKnownFlags) return MOE_ERR_INVALID_ARG;
     if ((c->flags & MOE_FORCE_DECODE) && (c->flags & MOE_FORCE_PREFILL)) return MOE_ERR_INVALID_ARG;
+    if ((c->flags & MOE_WEIGHTS_INT8) && (c->flags & MOE_FORCE_DECODE)) return MOE_ERR_INVALID_ARG;
     if (c->H % 128 || c->H > 16384) return MOE_ERR_UNSUPPORTED;
+    // int8 expert weights are served by the tensor-core sequence alone, whose
+    // down projection tiles 256 output columns
+    if ((c->flags & MOE_WEIGHTS_INT8) && c->H % 256) return MOE_ERR_UNSUPPORTED;
     if (c->E > kMaxE || c->K > kMaxK) return MOE_ERR_UNSUPPORTED;
     if (c->I % 128 || c->I > 8192) return MOE_ERR_UNSUPPORTED;
     if (c->Is % 128 || c->Is > 8192) return MOE_ERR_UNSUPPORTED;
@@ -149,7 +155,7 @@ constexpr int kFusedDefaultMaxH = 2048;
 
 // Whether a stack call takes the fused kernel.
 bool stack_fused(const moe_cfg_t& c, int32_t T, int32_t L) {
-    if (c.flags & (MOE_FORCE_DECODE | MOE_FORCE_PREFILL)) return false;
+    if (c.flags & (MOE_FORCE_DECODE | MOE_FORCE_PREFILL | MOE_WEIGHTS_INT8)) return false;
     if (!(fused_supported(c.H, c.E, c.K, c.I, c.Is, T, L) && fused_grid() > 0)) return false;
     if (c.flags & MOE_STACK_FUSED) return true;
     return L >= 2 && T <= kFusedDefaultMaxT && c.H <= kFusedDefaultMaxH;
@@ -480,7 +486,9 @@ int moe_stack_forward(const void* x, const moe_stack_weights_t* w, int32_t L, vo
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t TK = (size_t)T * cfg->K;
     if (!stack_fused(*cfg, T, L)) {
-        // one moe_layer_forward call per layer, each layer's output the next one's input
+        // one moe_layer_forward call per layer, each layer's output the next one's input;
+        // a code row of n elements is n/2 bytes (int4) or n bytes (int8)
+        const size_t per = (cfg->flags & MOE_WEIGHTS_INT8) ? 1 : 2;
         for (int32_t l = 0; l < L; ++l) {
             moe_cfg_t c = *cfg;
             c.flags &= ~(unsigned)MOE_LOOKAHEAD;
@@ -489,15 +497,15 @@ int moe_stack_forward(const void* x, const moe_stack_weights_t* w, int32_t L, vo
             c.stage_events = nullptr;
             moe_shared_weights_t sl{};
             if (Is > 0) {
-                sl.w13 = shw.w13 + l * 2 * Is * (H / 2);
+                sl.w13 = shw.w13 + l * 2 * Is * (H / per);
                 sl.s13 = shw.s13 + l * 2 * Is;
-                sl.w2 = shw.w2 + l * H * (Is / 2);
+                sl.w2 = shw.w2 + l * H * (Is / per);
                 sl.s2 = shw.s2 + l * H;
             }
             const void* in = l == 0 ? x : static_cast<const char*>(outs) + (size_t)(l - 1) * xbytes;
             void* out = static_cast<char*>(outs) + (size_t)l * xbytes;
-            st = moe_layer_forward(in, w->router_w + l * E * H, w->router_bias + l * E, w->w13 + l * E * 2 * I * (H / 2),
-                                   w->s13 + l * E * 2 * I, w->w2 + l * E * H * (I / 2), w->s2 + l * E * H, &sl, out, T,
+            st = moe_layer_forward(in, w->router_w + l * E * H, w->router_bias + l * E, w->w13 + l * E * 2 * I * (H / per),
+                                   w->s13 + l * E * 2 * I, w->w2 + l * E * H * (I / per), w->s2 + l * E * H, &sl, out, T,
                                    &c, stream);
             if (st != MOE_OK) return st;
         }

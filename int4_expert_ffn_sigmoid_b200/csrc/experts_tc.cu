@@ -9,6 +9,9 @@
 // per-row scales, dequant-on-use; batch-union MoE (each expert touched by the
 // batch is read once and applied to all of its tokens); nanocolibri-engine
 // README, "Converting a checkpoint yourself": per-row symmetric int4, f32 scales.
+// The same kernels serve int8 expert weights (the converter's 8-bit expert
+// setting): template parameter WB = 4 or 8 sets the raw tile (8 or 16 KiB per
+// k block), the ring depths and the code conversion; everything else is shared.
 //
 // Tile: 128 tokens (MMA M, one TMEM lane per token) x 256 weight rows (MMA N)
 // x 64 reduction elements per pipeline stage.  Tokens are the A operand and
@@ -51,13 +54,22 @@ constexpr int BM = 128;  // tokens per tile (A rows, TMEM lanes)
 constexpr int BN = 256;  // weight rows per tile (B rows, accumulator columns)
 constexpr int BK = 64;   // reduction elements per stage
 static_assert(BM == kTcTokens && BN == 2 * kTcFeat1 && BN == kTcFeat2, "tile geometry");
-constexpr int TSTAGES = 5;
-constexpr int BSTAGES = 3;
 constexpr int A_BYTES = BM * BK * 2;    // 16 KiB, bf16/fp16 tokens
 constexpr int B_BYTES = BN * BK * 2;    // 32 KiB, dequantised weights
-constexpr int RAW_BYTES = BN * BK / 2;  // 8 KiB, packed int4 weights
-constexpr int TSTAGE_BYTES = A_BYTES + RAW_BYTES;
-constexpr int RING_BYTES = TSTAGES * TSTAGE_BYTES + BSTAGES * B_BYTES;
+// Ring geometry per code width: WB = 4 (packed int4, 32 raw bytes per B row
+// and k block) or 8 (int8, 64 bytes).  The int8 raw tile is twice as large,
+// so its rings are one TMA stage and one B slot shallower (shared memory).
+template <int WB>
+struct Geo {
+    static_assert(WB == 4 || WB == 8, "int4 or int8 codes");
+    static constexpr int TSTAGES = WB == 4 ? 5 : 4;
+    static constexpr int BSTAGES = WB == 4 ? 3 : 2;
+    static constexpr int RAW_ROW = BK * WB / 8;      // bytes of one raw B row per k block
+    static constexpr int RAW_BYTES = BN * RAW_ROW;   // 8 or 16 KiB
+    static constexpr int TSTAGE_BYTES = A_BYTES + RAW_BYTES;
+    static constexpr int RING_BYTES = TSTAGES * TSTAGE_BYTES + BSTAGES * B_BYTES;
+};
+constexpr int MAX_TSTAGES = 5, MAX_BSTAGES = 3;
 constexpr int DEQ_GROUPS = 2;
 constexpr int DEQ_WARPS = 8 * DEQ_GROUPS;
 constexpr int EPI_WARPS = 8;
@@ -80,10 +92,10 @@ struct Stage {
 };
 
 struct Shared {
-    uint64_t full_tma[TSTAGES];  // token + raw tiles landed (TMA transaction count)
-    uint64_t empty_t[TSTAGES];   // MMA done with the token tile, a dequantiser group with the raw tile
-    uint64_t full_b[BSTAGES];    // B slot written (one arrival per warp of its group)
-    uint64_t empty_b[BSTAGES];   // MMA done with the B slot
+    uint64_t full_tma[MAX_TSTAGES];  // token + raw tiles landed (TMA transaction count)
+    uint64_t empty_t[MAX_TSTAGES];   // MMA done with the token tile, a dequantiser group with the raw tile
+    uint64_t full_b[MAX_BSTAGES];    // B slot written (one arrival per warp of its group)
+    uint64_t empty_b[MAX_BSTAGES];   // MMA done with the B slot
     uint64_t acc_full[2];
     uint64_t acc_empty[2];       // one arrival per epilogue warp
     uint64_t stage_full[2];      // one arrival per staging lane
@@ -94,8 +106,11 @@ struct Shared {
     int abort_flag;
     alignas(16) Stage stage[2];
 };
-constexpr int SMEM_BYTES = RING_BYTES + 1024 + (int)((sizeof(Shared) + 127) / 128 * 128);
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of the grouped GEMM");
+template <int WB>
+constexpr int smem_bytes() {
+    return Geo<WB>::RING_BYTES + 1024 + (int)((sizeof(Shared) + 127) / 128 * 128);
+}
+static_assert(smem_bytes<4>() <= 227 * 1024 && smem_bytes<8>() <= 227 * 1024, "shared memory of the grouped GEMM");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -259,6 +274,36 @@ __device__ __forceinline__ void int4x8_natural(uint32_t w, uint32_t* o) {
     }
 }
 
+// Four int8 codes (a 32-bit word, element j in byte j) -> two 16-bit pairs
+// in natural order: o[0] = (element 0, element 1), o[1] = (element 2, 3).
+// The same exponent-bias technique: c + 128 (the byte with its top bit
+// flipped) in the low mantissa bits of 2^m, minus 2^m + 128.  fp16 has ten
+// mantissa bits, so m = 10 works in 16 bits (0x6400 = 1024, 1152 = 0x6480).
+// bf16 has seven, too few for eight-bit codes: the value is formed in f32
+// (2^23 = 0x4B000000, minus 2^23 + 128), where the integer c is exact, and
+// its upper 16 bits, the bf16 encoding of c (the lower 16 are zero), kept.
+template <bool kBf16>
+__device__ __forceinline__ void int8x4_natural(uint32_t w, uint32_t* o) {
+    if (kBf16) {
+        const uint32_t u = w ^ 0x80808080u;
+        float f[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)  // bytes (u_j, 0, 0, 0x4B): 2^23 + c_j + 128
+            f[j] = __uint_as_float(__byte_perm(u, 0x4B000000u, j | 0x7440)) - 8388736.0f;
+        o[0] = __byte_perm(__float_as_uint(f[0]), __float_as_uint(f[1]), 0x7632);
+        o[1] = __byte_perm(__float_as_uint(f[2]), __float_as_uint(f[3]), 0x7632);
+    } else {
+        // bytes 0, 1 (then 2, 3) into the low byte of each half, top bit flipped, exponent of 1024
+        uint32_t u0 = __byte_perm(w, 0u, 0x4140) ^ 0x64806480u;
+        uint32_t u1 = __byte_perm(w, 0u, 0x4342) ^ 0x64806480u;
+        const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+        __half2 r0 = __hsub2(*reinterpret_cast<__half2*>(&u0), bias);
+        __half2 r1 = __hsub2(*reinterpret_cast<__half2*>(&u1), bias);
+        o[0] = *reinterpret_cast<uint32_t*>(&r0);
+        o[1] = *reinterpret_cast<uint32_t*>(&r1);
+    }
+}
+
 struct Tile {
     int shared;   // 1: shared expert
     int e;        // expert id (E for shared)
@@ -312,11 +357,14 @@ __device__ __forceinline__ int total_tiles(const TcArgs& a) {
     return mt_s * a.ntile_s + (a.gemm == 1 ? a.ctrl->tc_tiles1 : a.ctrl->tc_tiles2);
 }
 
-template <int GEMM>
+template <int GEMM, int WB>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_constant__ CUtensorMap tmX_s,
                     const __grid_constant__ CUtensorMap tmW_r, const __grid_constant__ CUtensorMap tmW_s,
                     const TcArgs a) {
+    constexpr int TSTAGES = Geo<WB>::TSTAGES, BSTAGES = Geo<WB>::BSTAGES;
+    constexpr int RAW_ROW = Geo<WB>::RAW_ROW, RAW_BYTES = Geo<WB>::RAW_BYTES;
+    constexpr int TSTAGE_BYTES = Geo<WB>::TSTAGE_BYTES, RING_BYTES = Geo<WB>::RING_BYTES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Shared* sh = reinterpret_cast<Shared*>(smem + RING_BYTES);
@@ -390,8 +438,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
                     if (!mbar_wait(&sh->empty_t[s], ph ^ 1u, sh)) { ok = false; break; }
                     mbar_expect_tx(&sh->full_tma[s], A_BYTES + RAW_BYTES);
                     tma_load_2d(x_tile(s), mX, &sh->full_tma[s], kb * BK, t.slot0);
-                    tma_load_2d(raw_tile(s), mW, &sh->full_tma[s], kb * (BK / 2), wrow0);
-                    tma_load_2d(raw_tile(s) + RAW_BYTES / 2, mW, &sh->full_tma[s], kb * (BK / 2), wrow1);
+                    tma_load_2d(raw_tile(s), mW, &sh->full_tma[s], kb * RAW_ROW, wrow0);
+                    tma_load_2d(raw_tile(s) + RAW_BYTES / 2, mW, &sh->full_tma[s], kb * RAW_ROW, wrow1);
                     issued[s] = true;
                     issued_par[s] = ph;
                     if (++s == TSTAGES) { s = 0; ph ^= 1u; }
@@ -450,9 +498,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
         // use B slot n mod BSTAGES and TMA stage n mod TSTAGES.
         const int g = (warp - 2) >> 3;
         const int r = ((warp - 2) & 7) * 32 + lane;  // B row = accumulator column
-        // the 16-byte half read first: a quarter-warp's eight reads then fall on
-        // eight different 16-byte bank groups (raw rows are 32 bytes apart)
+        // int4: the 16-byte half read first; a quarter-warp's eight reads then
+        // fall on eight different 16-byte bank groups (raw rows 32 bytes apart).
+        // int8: the raw tile lands with the 64-byte swizzle (16-byte chunk q of
+        // row r at q ^ ((r >> 1) & 3)), so that every lane reads the same
+        // logical quarter at once without bank conflicts and then stores the
+        // same B chunks (the B layout's own swizzle keeps those conflict-free).
         const int h0 = (r ^ (r >> 2)) & 1;
+        const int rot = (r >> 1) & 3;
         const uint32_t brow_off = (r >> 3) * 1024 + (r & 7) * 128;
         const uint32_t ring = smem_u32(smem);
         uint32_t n = 0;  // k blocks of the CTA so far
@@ -467,17 +520,31 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
                     ok = false;
                     break;
                 }
-                const uint32_t rrow = ring + s * TSTAGE_BYTES + A_BYTES + r * (BK / 2);
-                const uint4 qa = lds128(rrow + 16 * h0);
-                const uint4 qb = lds128(rrow + 16 * (h0 ^ 1));
-                const uint4 q0 = h0 ? qb : qa, q1 = h0 ? qa : qb;
-                const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                const uint32_t rrow = ring + s * TSTAGE_BYTES + A_BYTES + r * RAW_ROW;
                 const uint32_t brow = ring + TSTAGES * TSTAGE_BYTES + sb * B_BYTES + brow_off;
+                if (WB == 4) {
+                    const uint4 qa = lds128(rrow + 16 * h0);
+                    const uint4 qb = lds128(rrow + 16 * (h0 ^ 1));
+                    const uint4 q0 = h0 ? qb : qa, q1 = h0 ? qa : qb;
+                    const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {  // 16-byte chunk c = elements 8c..8c+7
-                    uint32_t o[4];
-                    int4x8_natural<GEMM == 1>(words[c], o);
-                    sts128(brow + ((c ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
+                    for (int c = 0; c < 8; ++c) {  // 16-byte chunk c = elements 8c..8c+7
+                        uint32_t o[4];
+                        int4x8_natural<GEMM == 1>(words[c], o);
+                        sts128(brow + ((c ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {  // raw quarter q = elements 16q..16q+15 = chunks 2q, 2q+1
+                        const uint4 v = lds128(rrow + 16 * (q ^ rot));
+                        uint32_t o[8];
+                        int8x4_natural<GEMM == 1>(v.x, o);
+                        int8x4_natural<GEMM == 1>(v.y, o + 2);
+                        int8x4_natural<GEMM == 1>(v.z, o + 4);
+                        int8x4_natural<GEMM == 1>(v.w, o + 6);
+                        sts128(brow + (((2 * q) ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
+                        sts128(brow + (((2 * q + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
+                    }
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the MMA reads through the async proxy
                 __syncwarp();
@@ -644,6 +711,16 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* bas
 
 int g_smem_set[64];
 
+template <int WB>
+cudaError_t set_smem_attrs() {
+    cudaError_t e = cudaFuncSetAttribute(tc::grouped_gemm_kernel<1, WB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         tc::smem_bytes<WB>());
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc::grouped_gemm_kernel<2, WB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::smem_bytes<WB>());
+    return e;
+}
+
 }  // namespace
 
 bool encode_tensor_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t inner,
@@ -651,21 +728,24 @@ bool encode_tensor_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int esize, con
     return get_encode() && make_map(m, dt, esize, base, inner, rows, box_inner, box_rows, sw);
 }
 
-int tc_smem_bytes() { return tc::SMEM_BYTES; }
+int tc_smem_bytes() { return tc::smem_bytes<4>(); }
 
 cudaError_t launch_tc_gemm(const Params& p, int gemm, int grid, cudaStream_t stream) {
     if (!get_encode()) return cudaErrorNotSupported;
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !g_smem_set[dev]) {
-        cudaError_t e1 = cudaFuncSetAttribute(tc::grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              tc::SMEM_BYTES);
-        cudaError_t e2 = cudaFuncSetAttribute(tc::grouped_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              tc::SMEM_BYTES);
-        if (e1 != cudaSuccess) return e1;
-        if (e2 != cudaSuccess) return e2;
+        cudaError_t e = set_smem_attrs<4>();
+        if (e == cudaSuccess) e = set_smem_attrs<8>();
+        if (e != cudaSuccess) return e;
         g_smem_set[dev] = 1;
     }
+    // code width: a row of n elements is n/2 bytes (int4) or n bytes (int8)
+    const bool int8w = (p.flags & kFlagWeightsInt8) != 0;
+    const int per = int8w ? 1 : 2;
+    const uint32_t raw_box = int8w ? tc::Geo<8>::RAW_ROW : tc::Geo<4>::RAW_ROW;
+    // int8 raw rows are one 64-byte swizzle span each (the dequantisers undo it)
+    const CUtensorMapSwizzle raw_sw = int8w ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE;
     const int TK = p.T * p.K;
     const int Is = p.Is > 0 ? p.Is : 128;  // any valid map when there is no shared expert
     CUtensorMap mX_r, mX_s, mW_r, mW_s;
@@ -689,10 +769,10 @@ cudaError_t launch_tc_gemm(const Params& p, int gemm, int grid, cudaStream_t str
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
              make_map(&mX_s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.x, p.H, p.T, 64, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
-             make_map(&mW_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.w13, p.H / 2, (uint64_t)p.E * 2 * p.I, 32, tc::BN / 2,
-                      CU_TENSOR_MAP_SWIZZLE_NONE) &&
+             make_map(&mW_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.w13, p.H / per, (uint64_t)p.E * 2 * p.I, raw_box,
+                      tc::BN / 2, raw_sw) &&
              make_map(&mW_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.Is > 0 ? (const void*)p.sh_w13 : (const void*)p.w13,
-                      p.H / 2, 2 * (uint64_t)Is, 32, tc::BN / 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+                      p.H / per, 2 * (uint64_t)Is, raw_box, tc::BN / 2, raw_sw);
     } else {
         a.kdim_r = p.I; a.kdim_s = p.Is;
         a.ntile_r = p.H / kTcFeat2; a.ntile_s = p.H / kTcFeat2;
@@ -702,17 +782,22 @@ cudaError_t launch_tc_gemm(const Params& p, int gemm, int grid, cudaStream_t str
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
              make_map(&mX_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.Is > 0 ? (const void*)p.h_s : (const void*)p.h_r,
                       Is, p.T, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
-             make_map(&mW_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.w2, p.I / 2, (uint64_t)p.E * p.H, 32, tc::BN / 2,
-                      CU_TENSOR_MAP_SWIZZLE_NONE) &&
+             make_map(&mW_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.w2, p.I / per, (uint64_t)p.E * p.H, raw_box,
+                      tc::BN / 2, raw_sw) &&
              make_map(&mW_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.Is > 0 ? (const void*)p.sh_w2 : (const void*)p.w2,
-                      Is / 2, p.H, 32, tc::BN / 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+                      Is / per, p.H, raw_box, tc::BN / 2, raw_sw);
     }
     if (!ok) return cudaErrorInvalidValue;
-    if (gemm == 1)
-        return launch_pdl(tc::grouped_gemm_kernel<1>, dim3(grid), dim3(tc::NUM_THREADS), tc::SMEM_BYTES, stream, mX_r,
-                          mX_s, mW_r, mW_s, a);
-    return launch_pdl(tc::grouped_gemm_kernel<2>, dim3(grid), dim3(tc::NUM_THREADS), tc::SMEM_BYTES, stream, mX_r,
-                      mX_s, mW_r, mW_s, a);
+    const dim3 g(grid), b(tc::NUM_THREADS);
+    if (int8w)
+        return gemm == 1 ? launch_pdl(tc::grouped_gemm_kernel<1, 8>, g, b, tc::smem_bytes<8>(), stream, mX_r, mX_s,
+                                      mW_r, mW_s, a)
+                         : launch_pdl(tc::grouped_gemm_kernel<2, 8>, g, b, tc::smem_bytes<8>(), stream, mX_r, mX_s,
+                                      mW_r, mW_s, a);
+    return gemm == 1 ? launch_pdl(tc::grouped_gemm_kernel<1, 4>, g, b, tc::smem_bytes<4>(), stream, mX_r, mX_s, mW_r,
+                                  mW_s, a)
+                     : launch_pdl(tc::grouped_gemm_kernel<2, 4>, g, b, tc::smem_bytes<4>(), stream, mX_r, mX_s, mW_r,
+                                  mW_s, a);
 }
 
 }  // namespace moe

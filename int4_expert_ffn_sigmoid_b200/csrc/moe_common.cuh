@@ -60,6 +60,7 @@ constexpr unsigned kFlagLookahead = 1u << 5;  // MOE_LOOKAHEAD
 constexpr unsigned kFlagTestStall = 1u << 6;  // MOE_TEST_STALL
 constexpr unsigned kFlagTestBadIndex = 1u << 7;  // MOE_TEST_BAD_INDEX
 constexpr unsigned kFlagTrace = 1u << 8;      // MOE_TRACE
+constexpr unsigned kFlagWeightsInt8 = 1u << 11;  // MOE_WEIGHTS_INT8
 
 // Adaptive expert top-p over the K picks of one token (one warp; lanes k < K
 // hold pick k: expert e_k and sigmoid score s_k; ssum is the K scores' sum).

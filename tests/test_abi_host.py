@@ -7,6 +7,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "moe_int4.h")
@@ -65,7 +66,8 @@ def test_header_constants_match_binding(moe):
                  "MOE_FORCE_PREFILL", "MOE_ADD_RESIDUAL", "MOE_DEBUG_CHECK",
                  "MOE_PATH_SMALL_BATCH", "MOE_PATH_TENSOR_CORE", "MOE_PATH_LARGE_STREAMING",
                  "MOE_LOOKAHEAD", "MOE_TEST_STALL", "MOE_TEST_BAD_INDEX", "MOE_TRACE", "MOE_DEBUG_POISON",
-                 "MOE_DEVSTAT_TIMEOUT", "MOE_DEVSTAT_BAD_EXPERT", "MOE_PATH_FUSED_STACK", "MOE_PATH_PER_LAYER"):
+                 "MOE_DEVSTAT_TIMEOUT", "MOE_DEVSTAT_BAD_EXPERT", "MOE_PATH_FUSED_STACK", "MOE_PATH_PER_LAYER",
+                 "MOE_STACK_FUSED", "MOE_WEIGHTS_INT8"):
         m = re.search(rf"#define {name} (.+)", text)
         assert m, name
         expr = m.group(1).split("/*")[0].replace("(size_t)", "").replace("u", "")
@@ -146,6 +148,34 @@ def test_path_choice(moe):
     assert moe.layer_path(_shape(H=1152), 4096) == LS  # H not a multiple of 256
     assert moe.layer_path(large, 512) == LS            # 16 picks per expert
     assert moe.layer_path(large, 1024) == TC
+
+
+def test_int8_weights_flag(moe):
+    """int8 expert weights take the tensor-core sequence at every T; the
+    weight-streaming sequence (MOE_FORCE_DECODE), a hidden size that is not a
+    multiple of 256 and the fused stack kernel are refused."""
+    nano = _shape()
+    I8 = moe.MOE_WEIGHTS_INT8
+    for T in (1, 16, 64, 65, 1023, 4096):
+        assert moe.layer_path(nano, T, I8) == moe.MOE_PATH_TENSOR_CORE, T
+        assert moe.layer_path(nano, T, I8 | moe.MOE_FORCE_PREFILL) == moe.MOE_PATH_TENSOR_CORE, T
+        assert moe.kernel_launches(nano, T, I8) == 5, T
+    assert moe.layer_path(nano, 16, I8 | moe.MOE_FORCE_DECODE) == 0
+    assert moe.workspace_bytes(nano, 16, I8 | moe.MOE_FORCE_DECODE) == 0
+    assert _call(moe, nano, T=4, flags=I8 | moe.MOE_FORCE_DECODE) == moe.MOE_ERR_INVALID_ARG
+    assert moe.layer_path(_shape(H=1152), 4096, I8) == 0
+    assert _call(moe, _shape(H=1152), T=4, flags=I8) == moe.MOE_ERR_UNSUPPORTED
+    # the tensor-core workspace at every T, largest at N itself
+    assert moe.workspace_bytes(nano, 16, I8) == moe.workspace_bytes(nano, 16, moe.MOE_FORCE_PREFILL)
+    assert moe.workspace_bytes_upto(nano, 300, I8) == moe.workspace_bytes(nano, 300, I8)
+    for T in (1, 4, 16):
+        assert moe.stack_path(nano, T, 23, I8) == moe.MOE_PATH_PER_LAYER
+        assert moe.stack_path(nano, T, 23, I8 | moe.MOE_STACK_FUSED) == moe.MOE_PATH_PER_LAYER
+    # the binding reads the code width from the weight shapes
+    assert moe.weight_flags({"w13": torch.empty(2, 4, 1024, dtype=torch.uint8)}, nano) == I8
+    assert moe.weight_flags({"w13": torch.empty(2, 4, 512, dtype=torch.uint8)}, nano) == 0
+    with pytest.raises(ValueError):
+        moe.weight_flags({"w13": torch.empty(2, 4, 100, dtype=torch.uint8)}, nano)
 
 
 # Fake device pointers: validation runs before any dereference or CUDA call.

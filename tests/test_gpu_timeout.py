@@ -32,17 +32,26 @@ CASES = [
      16, "decode"),
     ("tcgen05 streaming gate/up kernel", workloads.LayerShape(H=1024, E=64, K=2, I=512, Is=2048, routed_scaling=1.0),
      400, "decode"),
+    ("tensor-core grouped GEMMs, int8 weights", workloads.LayerShape(H=512, E=16, K=8, I=256, Is=384, routed_scaling=2.5),
+     130, "int8"),
 ]
+
+
+def _wbits(mode):
+    return 8 if mode == "int8" else 4
 
 
 @pytest.mark.parametrize("case", range(len(CASES)))
 def test_stalled_wait_reports_timeout_then_recovers(moe, cuda_device, case):
     what, shape, T, mode = CASES[case]
-    base = moe.MOE_FORCE_PREFILL if mode == "prefill" else (moe.MOE_FORCE_DECODE if T > 64 else 0)
-    path = moe.MOE_PATH_TENSOR_CORE if mode == "prefill" else (moe.MOE_PATH_LARGE_STREAMING if T > 64 else
-                                                                  moe.MOE_PATH_SMALL_BATCH)
+    if mode == "int8":
+        base, path = moe.MOE_WEIGHTS_INT8, moe.MOE_PATH_TENSOR_CORE
+    else:
+        base = moe.MOE_FORCE_PREFILL if mode == "prefill" else (moe.MOE_FORCE_DECODE if T > 64 else 0)
+        path = moe.MOE_PATH_TENSOR_CORE if mode == "prefill" else (moe.MOE_PATH_LARGE_STREAMING if T > 64 else
+                                                                      moe.MOE_PATH_SMALL_BATCH)
     assert moe.layer_path(shape, T, base) == path, what
-    layer = workloads.make_layer(shape, 300 + case, 0, cuda_device)
+    layer = workloads.make_layer(shape, 300 + case, 0, cuda_device, wbits=_wbits(mode))
     x = workloads.make_x(shape, T, 300 + case, device=cuda_device)
     ws = moe.new_workspace(shape, T, cuda_device, base)
     good = moe.layer_forward(x, layer, shape, workspace=ws, flags=base | moe.MOE_DEBUG_CHECK).clone()
@@ -66,11 +75,12 @@ PATHS = [
     ("tensor-core kernels", workloads.LayerShape(512, 16, 8, 256, 384, 2.5), 130, "prefill"),
     ("large-batch streaming kernels", workloads.LayerShape(1024, 64, 2, 512, 2048, 1.0), 150, "decode"),
     ("large-batch streaming, tcgen05 gate/up", workloads.LayerShape(1024, 64, 2, 512, 2048, 1.0), 400, "decode"),
+    ("tensor-core kernels, int8 weights", workloads.LayerShape(512, 16, 8, 256, 384, 2.5), 130, "int8"),
 ]
 
 
 def _flags(moe, f):
-    return {0: 0, "prefill": moe.MOE_FORCE_PREFILL, "decode": moe.MOE_FORCE_DECODE}[f]
+    return {0: 0, "prefill": moe.MOE_FORCE_PREFILL, "decode": moe.MOE_FORCE_DECODE, "int8": moe.MOE_WEIGHTS_INT8}[f]
 
 
 @pytest.mark.parametrize("case", range(len(PATHS)))
@@ -80,7 +90,7 @@ def test_bad_routing_index_is_caught(moe, cuda_device, case):
     reads or writes out of bounds: the next normal call is bit-identical."""
     what, shape, T, f = PATHS[case]
     base = _flags(moe, f)
-    layer = workloads.make_layer(shape, 320 + case, 0, cuda_device)
+    layer = workloads.make_layer(shape, 320 + case, 0, cuda_device, wbits=_wbits(f))
     x = workloads.make_x(shape, T, 320 + case, device=cuda_device)
     ws = moe.new_workspace(shape, T, cuda_device, base)
     good = moe.layer_forward(x, layer, shape, workspace=ws, flags=base | moe.MOE_DEBUG_CHECK).clone()
@@ -99,7 +109,7 @@ def test_poisoned_workspace_changes_nothing(moe, cuda_device, case):
     filling the workspace with 0xFF (NaN / -1) beforehand changes no output bit."""
     what, shape, T, f = PATHS[case]
     base = _flags(moe, f)
-    layer = workloads.make_layer(shape, 330 + case, 0, cuda_device)
+    layer = workloads.make_layer(shape, 330 + case, 0, cuda_device, wbits=_wbits(f))
     x = workloads.make_x(shape, T, 330 + case, device=cuda_device)
     a = moe.layer_forward(x, layer, shape, flags=base | moe.MOE_DEBUG_CHECK)
     b = moe.layer_forward(x, layer, shape, flags=base | moe.MOE_DEBUG_POISON | moe.MOE_DEBUG_CHECK)

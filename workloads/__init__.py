@@ -81,7 +81,7 @@ class Workload:
     own weights); tokens: the token counts the workload is run at;
     bias_mode: "uniform" (U(-0.1, 0.1)), "zero", or "zipf" (calibrated
     popularity bias read from a data file); residual: whether each layer adds
-    its input (x_{l+1} = x_l + MoE_l(x_l)).
+    its input (x_{l+1} = x_l + MoE_l(x_l)); wbits: expert code width (4 or 8).
     """
     name: str
     wid: int
@@ -91,6 +91,7 @@ class Workload:
     bias_mode: str
     residual: bool
     description: str
+    wbits: int = 4
 
 
 WORKLOADS: Dict[str, Workload] = {
@@ -104,6 +105,9 @@ WORKLOADS: Dict[str, Workload] = {
                  "one Nano MoE layer, T=4096, zero router bias (balanced loads)"),
         Workload("nano_zipf_t16384", 3, NANO, 1, (16384,), "zipf", False,
                  "one Nano MoE layer, T=16384, Zipf(1.2) expert popularity via router bias"),
+        Workload("nano_prefill_t4096_int8", 6, NANO, 1, (4096,), "zero", False,
+                 "one Nano MoE layer with int8 expert weights (the converter's 8-bit expert setting), "
+                 "T=4096, zero router bias", wbits=8),
         Workload("large_layer", 4, LARGE, 1, (1, 32, 512), "uniform", False,
                  "one 6144-hidden 256-expert top-8 layer, T in {1,32,512}"),
         Workload("large_layer_e32", 5, LARGE_E32, 1, (4,), "uniform", False,
