@@ -58,18 +58,20 @@ constexpr int A_BYTES = BM * BK * 2;    // 16 KiB, bf16/fp16 tokens
 constexpr int B_BYTES = BN * BK * 2;    // 32 KiB, dequantised weights
 // Ring geometry per code width: WB = 4 (packed int4, 32 raw bytes per B row
 // and k block) or 8 (int8, 64 bytes).  The int8 raw tile is twice as large,
-// so its rings are one TMA stage and one B slot shallower (shared memory).
+// so its B ring is one slot shallower (shared memory).  (Deeper TMA rings,
+// 5 and 6 stages for int4, measured no faster.)
 template <int WB>
 struct Geo {
     static_assert(WB == 4 || WB == 8, "int4 or int8 codes");
-    static constexpr int TSTAGES = WB == 4 ? 5 : 4;
+    static constexpr int TSTAGES = 4;
     static constexpr int BSTAGES = WB == 4 ? 3 : 2;
     static constexpr int RAW_ROW = BK * WB / 8;      // bytes of one raw B row per k block
     static constexpr int RAW_BYTES = BN * RAW_ROW;   // 8 or 16 KiB
     static constexpr int TSTAGE_BYTES = A_BYTES + RAW_BYTES;
     static constexpr int RING_BYTES = TSTAGES * TSTAGE_BYTES + BSTAGES * B_BYTES;
 };
-constexpr int MAX_TSTAGES = 5, MAX_BSTAGES = 3;
+constexpr int MAX_TSTAGES = 4, MAX_BSTAGES = 3;
+constexpr int EPI_STAGE_BYTES = 2048;  // per epilogue warp: 32 token rows x 64 bytes
 constexpr int DEQ_GROUPS = 2;
 constexpr int DEQ_WARPS = 8 * DEQ_GROUPS;
 constexpr int EPI_WARPS = 8;
@@ -105,6 +107,9 @@ struct Shared {
     uint32_t tmem_base;
     int abort_flag;
     alignas(16) Stage stage[2];
+    // epilogue transpose: each warp's 32 rows x 16 columns pass through here so
+    // that every global store instruction writes whole row segments
+    alignas(128) uint8_t epi[EPI_WARPS][EPI_STAGE_BYTES];
 };
 template <int WB>
 constexpr int smem_bytes() {
@@ -600,13 +605,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
             tc_fence_after();
             const Stage& st = sh->stage[buf];
             const uint32_t st_sc = smem_u32(&st.sc[0]);
-            const int row = lds32(smem_u32(&st.slot[m]));
             const float fac = __int_as_float(lds32(smem_u32(&st.fac[m])));
+            const uint32_t stg = smem_u32(&sh->epi[warp - WARP_EPI0][0]);
             const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;
             if (GEMM == 1) {
                 // features 64c .. 64c + 63 of the tile: gate in column j, up in column 128 + j
                 const int irow = t.shared ? a.Is : a.I;
-                __half* hrow = (t.shared ? a.h_s : a.h_r) + (size_t)(row < 0 ? 0 : row) * irow + t.col0;
+                __half* hbase = (t.shared ? a.h_s : a.h_r) + t.col0;
+                int rows[2];  // the token rows this lane stores: 16 i + lane / 2
+#pragma unroll
+                for (int i = 0; i < 2; ++i) rows[i] = lds32(smem_u32(&st.slot[quarter * 32 + 16 * i + (lane >> 1)]));
 #pragma unroll 1
                 for (int c0 = 64 * chalf; c0 < 64 * chalf + 64; c0 += 16) {
                     uint32_t gv[16], uv[16];
@@ -629,15 +637,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
                         __half2 hv = __floats2half2_rn(h0v, h1v);
                         packed[i >> 1] = *reinterpret_cast<uint32_t*>(&hv);
                     }
-                    if (row >= 0) {
-                        uint4* dst = reinterpret_cast<uint4*>(hrow + c0);
-                        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                    // this lane's 32 bytes (row `lane`) into the warp's stage, 16-byte
+                    // chunk c at c ^ ((lane >> 2) & 1); then two lanes per row, 16 rows
+                    // per store instruction
+                    const int sw = (lane >> 2) & 1;
+                    sts128(stg + lane * 32 + 16 * sw, packed[0], packed[1], packed[2], packed[3]);
+                    sts128(stg + lane * 32 + 16 * (sw ^ 1), packed[4], packed[5], packed[6], packed[7]);
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const int rr = 16 * i + (lane >> 1), cc = lane & 1;
+                        const uint4 val = lds128(stg + rr * 32 + 16 * (cc ^ ((rr >> 2) & 1)));
+                        if (rows[i] >= 0)
+                            *reinterpret_cast<uint4*>(hbase + (size_t)rows[i] * irow + c0 + 8 * cc) = val;
                     }
+                    __syncwarp();  // the stage is read before the next columns overwrite it
                 }
             } else {
                 // output columns 128c .. 128c + 127 of the tile
-                float* yrow = a.y + (size_t)(row < 0 ? 0 : row) * a.H + t.col0;
+                float* ybase = a.y + t.col0;
+                int rows[4];  // the token rows this lane stores: 8 i + lane / 4
+#pragma unroll
+                for (int i = 0; i < 4; ++i) rows[i] = lds32(smem_u32(&st.slot[quarter * 32 + 8 * i + (lane >> 2)]));
 #pragma unroll 1
                 for (int c0 = 128 * chalf; c0 < 128 * chalf + 128; c0 += 16) {
                     uint32_t v[16];
@@ -650,10 +671,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
                                            __uint_as_float(v[4 * q + 2]) * (s4.z * fac),
                                            __uint_as_float(v[4 * q + 3]) * (s4.w * fac));
                     }
-                    if (row >= 0) {
-                        float4* dst = reinterpret_cast<float4*>(yrow + c0);
-                        dst[0] = o[0]; dst[1] = o[1]; dst[2] = o[2]; dst[3] = o[3];
+                    // this lane's 64 bytes (row `lane`) into the warp's stage, 16-byte
+                    // chunk c at c ^ ((lane >> 1) & 3); then four lanes per row, 8 rows
+                    // per store instruction
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        sts128(stg + lane * 64 + 16 * (q ^ ((lane >> 1) & 3)), __float_as_uint(o[q].x),
+                               __float_as_uint(o[q].y), __float_as_uint(o[q].z), __float_as_uint(o[q].w));
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int rr = 8 * i + (lane >> 2), cc = lane & 3;
+                        const float4 val = lds128f(stg + rr * 64 + 16 * (cc ^ ((rr >> 1) & 3)));
+                        if (rows[i] >= 0) *reinterpret_cast<float4*>(ybase + (size_t)rows[i] * a.H + c0 + 4 * cc) = val;
                     }
+                    __syncwarp();  // the stage is read before the next columns overwrite it
                 }
             }
             tc_fence_before();
