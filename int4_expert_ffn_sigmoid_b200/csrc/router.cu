@@ -567,8 +567,9 @@ __global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(32 *
 // per-expert pick counts.  scatter_large_kernel: every CTA derives the bucket
 // offsets and its own slot bases from those counts (CTA 0 also writes the
 // bucket and task lists), then the slots, and the gathered activation rows of
-// the tensor-core path or the int8 activations of the weight-streaming
-// kernels.
+// the tensor-core path.  The int8 activations of the weight-streaming kernels
+// come from extra CTAs past the router's (one warp per token, every token in
+// flight at once), or, when the grid has no room for them, from the router's.
 // ---------------------------------------------------------------------------
 // Tensor-core router logits for a tile of kRouterTileTokens tokens and every
 // expert.  x is exactly bf16; each f32 router weight w is split exactly into
@@ -862,6 +863,15 @@ __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
     const int nblk = p.router_blocks;
     pdl_wait();
     pdl_release();
+    if ((int)blockIdx.x >= nblk) {
+        // quantizer CTAs (weight-streaming sequence, launched past the router's
+        // CTAs): the int8 activations, one warp per token, all tokens in flight
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+        const int nq = (int)gridDim.x - nblk;
+        for (int t = ((int)blockIdx.x - nblk) * nw + warp; t < p.T; t += nq * nw)
+            quantize_x_row(p, t, p.x + (size_t)t * p.H, lane);
+        return;
+    }
     for (int e = threadIdx.x; e < E; e += blockDim.x) s_tot[e] = s_base[e] = 0;
     __syncthreads();
     {  // the whole [nblk][E] count matrix, 16 loads in flight per thread
@@ -943,7 +953,7 @@ __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
                 for (int c = lane; c < p.H / 8; c += 32) dst[c] = __ldg(src + c);
             }
         }
-        if (p.xq) {  // int8 activations of the weight-streaming kernels (one warp per token)
+        if (p.xq && (int)gridDim.x == nblk) {  // int8 activations (no quantizer CTAs): one warp per token
             const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
             for (int tt = warp; tt < n / K; tt += blockDim.x / 32)
                 quantize_x_row(p, t0 + tt, p.x + (size_t)(t0 + tt) * p.H, lane);
@@ -990,7 +1000,15 @@ cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream)
         err = launch_pdl(router_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
     }
     if (err != cudaSuccess) return err;
-    if (err == cudaSuccess) err = launch_pdl(scatter_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
+    // the weight-streaming sequence's int8 activations: quantizer CTAs past the
+    // router's, one warp per token (up to kRouterMaxBlocks CTAs in all)
+    int quant_ctas = 0;
+    if (p.xq) {
+        const int want = (p.T + 7) / 8, room = kRouterMaxBlocks - p.router_blocks;
+        quant_ctas = want < room ? want : room;
+    }
+    if (err == cudaSuccess)
+        err = launch_pdl(scatter_large_kernel, dim3(p.router_blocks + quant_ctas), dim3(256), 0, stream, p);
     return err;
 }
 
