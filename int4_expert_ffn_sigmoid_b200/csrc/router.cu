@@ -874,24 +874,27 @@ __global__ void __launch_bounds__(256) scatter_large_kernel(Params p) {
     }
     for (int e = threadIdx.x; e < E; e += blockDim.x) s_tot[e] = s_base[e] = 0;
     __syncthreads();
-    {  // the whole [nblk][E] count matrix, 16 loads in flight per thread
-        const int total = nblk * E;
-        for (int i0 = threadIdx.x; i0 < total; i0 += 16 * blockDim.x) {
-            int v[16];
+    {  // the whole [nblk][E] count matrix: G = blockDim / E threads per expert
+       // (E <= kMaxE = blockDim) sum the blocks g, g + G, ... of their expert
+       // with eight loads in flight, then add their partial sums
+        const int G = (int)blockDim.x / E, e = (int)threadIdx.x % E, g = (int)threadIdx.x / E;
+        if (g < G) {
+            int tot = 0, base = 0;
+            for (int b0 = g; b0 < nblk; b0 += 8 * G) {
+                int v[8];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int i = i0 + u * blockDim.x;
-                v[u] = i < total ? __ldcg(p.hist + i) : 0;
-            }
+                for (int u = 0; u < 8; ++u) {
+                    const int b = b0 + u * G;
+                    v[u] = b < nblk ? __ldcg(p.hist + (size_t)b * E + e) : 0;
+                }
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int i = i0 + u * blockDim.x;
-                if (i < total && v[u] != 0) {
-                    const int b = i / E, e = i - b * E;
-                    atomicAdd(&s_tot[e], v[u]);
-                    if (b < (int)blockIdx.x) atomicAdd(&s_base[e], v[u]);
+                for (int u = 0; u < 8; ++u) {
+                    tot += v[u];
+                    if (b0 + u * G < (int)blockIdx.x) base += v[u];
                 }
             }
+            atomicAdd(&s_tot[e], tot);
+            atomicAdd(&s_base[e], base);
         }
     }
     __syncthreads();
