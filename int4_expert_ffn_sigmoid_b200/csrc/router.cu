@@ -148,15 +148,17 @@ __device__ int select_from_logits(const Params& p, int t, const float (&L)[kMaxE
     return lane < K ? out_e : -1;
 }
 
-// select_from_logits with the token's logits in shared memory.
-__device__ int select_token(const Params& p, int t, const float* lg, int lane) {
+// select_from_logits with the token's logits and the router bias in shared
+// memory (a bias read from global memory per token put a round trip on every
+// selection).
+__device__ int select_token(const Params& p, int t, const float* lg, const float* s_bias, int lane) {
     float L[kMaxE / 32];
 #pragma unroll
     for (int j = 0; j < kMaxE / 32; ++j) {
         const int e = lane + 32 * j;
         L[j] = e < p.E ? lg[e] : 0.f;
     }
-    return select_from_logits(p, t, L, p.rb, lane);
+    return select_from_logits(p, t, L, s_bias, lane);
 }
 
 // Writes xq (both int8 parts, see quant2) and xs of token t (one warp) from
@@ -599,6 +601,7 @@ __global__ void __launch_bounds__(256, 2) router_large_kernel(Params p) {
     constexpr int kLBytes = kRouterTileTokens * kMaxE * 4;
     __shared__ __align__(16) uint8_t s_buf[kXBytes > kLBytes ? kXBytes : kLBytes];
     __shared__ int s_cnt[kMaxE];
+    __shared__ float s_bias[kMaxE];
     auto s_x = reinterpret_cast<uint16_t (*)[kRouterTileTokens][kRouterXS]>(s_buf);
     auto s_logit = reinterpret_cast<float (*)[kMaxE]>(s_buf);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -621,7 +624,10 @@ __global__ void __launch_bounds__(256, 2) router_large_kernel(Params p) {
     pdl_wait();
     reset_ctrl(p);
     pdl_release();
-    for (int i = threadIdx.x; i < E; i += blockDim.x) s_cnt[i] = 0;
+    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+        s_cnt[i] = 0;
+        s_bias[i] = __ldg(p.rb + i);
+    }
     __syncthreads();
     const int ntiles_tok = (p.T + kRouterTileTokens - 1) / kRouterTileTokens;
     const int nchunks = H / kRouterKC;
@@ -756,7 +762,7 @@ __global__ void __launch_bounds__(256, 2) router_large_kernel(Params p) {
         }
         __syncthreads();
         for (int tt = warp; tt < nt; tt += 8) {
-            const int sel = select_token(p, t0 + tt, s_logit[tt], lane);
+            const int sel = select_token(p, t0 + tt, s_logit[tt], s_bias, lane);
             // an index outside [0, E) cannot occur; it is counted nowhere and
             // reported by the scatter kernel's range check
             if (lane < p.K && sel >= 0 && sel < E) atomicAdd(&s_cnt[sel], 1);
@@ -769,11 +775,15 @@ __global__ void __launch_bounds__(256, 2) router_large_kernel(Params p) {
 __global__ void __launch_bounds__(256) router_select_kernel(Params p) {
     __shared__ __align__(16) float s_logit[kRouterTileTokens][kMaxE];
     __shared__ int s_cnt[kMaxE];
+    __shared__ float s_bias[kMaxE];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int E = p.E;
     pdl_wait();  // the weight split, the call's first kernel, zeroed the status word
     pdl_release();
-    for (int i = threadIdx.x; i < E; i += blockDim.x) s_cnt[i] = 0;
+    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+        s_cnt[i] = 0;
+        s_bias[i] = __ldg(p.rb + i);
+    }
     __syncthreads();
     const int ntiles_tok = (p.T + kRouterTileTokens - 1) / kRouterTileTokens;
     for (int tile = blockIdx.x; tile < ntiles_tok; tile += gridDim.x) {
@@ -811,7 +821,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(Params p) {
         }
         __syncthreads();
         for (int tt = warp; tt < nt; tt += 8) {
-            const int sel = select_token(p, t0 + tt, s_logit[tt], lane);
+            const int sel = select_token(p, t0 + tt, s_logit[tt], s_bias, lane);
             // an index outside [0, E) cannot occur; it is counted nowhere and
             // reported by the scatter kernel's range check
             if (lane < p.K && sel >= 0 && sel < E) atomicAdd(&s_cnt[sel], 1);
