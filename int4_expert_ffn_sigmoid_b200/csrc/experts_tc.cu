@@ -314,7 +314,9 @@ struct Tile {
     int e;        // expert id (E for shared)
     int n_valid;  // valid tokens in this tile
     int slot0;    // first token row of the tile (TMA y coordinate of the token map; h row / y slot)
-    int col0;     // GEMM-1: first feature of the tile (128 of them); GEMM-2: first output feature (256)
+    int col0;     // GEMM-1: first feature of the unit; GEMM-2: first output feature
+    int ncol;     // weight rows (B rows, accumulator columns) of the unit: 256, 128 or 64;
+                  // GEMM-1: ncol / 2 features, gate rows then up rows
     int nkb;      // k blocks
 };
 
@@ -326,6 +328,7 @@ __device__ __forceinline__ Tile decode_tile(const TcArgs& a, int tile) {
     const int fw = a.gemm == 1 ? kTcFeat1 : kTcFeat2;
     const int mt_s = a.Is > 0 ? (a.T + BM - 1) / BM : 0;
     const int n_sh = mt_s * a.ntile_s;
+    t.ncol = BN;
     if (tile < n_sh) {
         const int mt = tile % mt_s, nt = tile / mt_s;
         t.shared = 1;
@@ -360,6 +363,35 @@ __device__ __forceinline__ Tile decode_tile(const TcArgs& a, int tile) {
 __device__ __forceinline__ int total_tiles(const TcArgs& a) {
     const int mt_s = a.Is > 0 ? (a.T + BM - 1) / BM : 0;
     return mt_s * a.ntile_s + (a.gemm == 1 ? a.ctrl->tc_tiles1 : a.ctrl->tc_tiles2);
+}
+
+// Work units of a launch.  CTA b takes units b, b + grid, ...  The tiles of
+// the full waves are units of their own; the tiles of the last, partial wave
+// are split by columns into f equal units (f = 1, 2 or 4, as many as the grid
+// holds), so that it spreads over more CTAs instead of leaving most of them
+// idle while a few finish whole tiles.  A unit covers all of its tile's k
+// blocks: every output element is summed exactly as in the unsplit tile.
+struct Units {
+    int full;   // units that are whole tiles
+    int f;      // units per tile of the last wave
+    int total;
+};
+__device__ __forceinline__ Units units_of(int ntiles, int grid) {
+    Units u;
+    const int rem = ntiles % grid;
+    u.full = ntiles - rem;
+    u.f = 1;
+    while (rem > 0 && u.f < 4 && rem * u.f * 2 <= grid) u.f *= 2;
+    u.total = u.full + rem * u.f;
+    return u;
+}
+__device__ __forceinline__ Tile decode_unit(const TcArgs& a, const Units& us, int unit) {
+    if (unit < us.full) return decode_tile(a, unit);
+    const int i = unit - us.full, part = i % us.f;
+    Tile t = decode_tile(a, us.full + i / us.f);
+    t.ncol = BN / us.f;
+    t.col0 += part * (a.gemm == 1 ? t.ncol / 2 : t.ncol);
+    return t;
 }
 
 template <int GEMM, int WB>
@@ -411,6 +443,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
     pdl_wait();  // barriers and TMEM were set up while the previous kernel finished
     pdl_release();
     const int ntiles = total_tiles(a);
+    const Units us = units_of(ntiles, gridDim.x);
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -425,11 +458,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
             bool issued[TSTAGES];
             for (int i = 0; i < TSTAGES; ++i) issued[i] = false, issued_par[i] = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-                const Tile t = decode_tile(a, tile);
+            for (int unit = blockIdx.x; ok && unit < us.total; unit += gridDim.x) {
+                const Tile t = decode_unit(a, us, unit);
                 const CUtensorMap* mX = t.shared ? &tmX_s : &tmX_r;
                 const CUtensorMap* mW = t.shared ? &tmW_s : &tmW_r;
-                int wrow0, wrow1;  // raw rows of B rows 0..127 and 128..255
+                int wrow0, wrow1;  // raw rows of the two 128-row boxes (a narrower unit uses the first rows of each)
                 if (GEMM == 1) {
                     const int irow = t.shared ? a.Is : a.I;
                     const int base = t.shared ? 0 : t.e * 2 * a.I;
@@ -457,17 +490,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_f16(GEMM == 1 ? 1 : 0, BM, BN);
+            constexpr int kFmt = GEMM == 1 ? 1 : 0;
             int s = 0, sb = 0;
             uint32_t ph = 0, phb = 0;
             uint32_t acc_ph[2] = {0, 0};
             int buf = 0;
             bool ok = true, any = false;
-            for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-                const Tile t = decode_tile(a, tile);
+            for (int unit = blockIdx.x; ok && unit < us.total; unit += gridDim.x) {
+                const Tile t = decode_unit(a, us, unit);
                 if (!mbar_wait(&sh->acc_empty[buf], acc_ph[buf] ^ 1u, sh)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem + buf * BN;
+                const uint32_t idesc = idesc_f16(kFmt, BM, t.ncol);
                 for (int kb = 0; kb < t.nkb; ++kb) {
                     if (!mbar_wait(&sh->full_tma[s], ph, sh) || !mbar_wait(&sh->full_b[sb], phb, sh)) {
                         ok = false;
@@ -509,14 +543,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
         // row r at q ^ ((r >> 1) & 3)), so that every lane reads the same
         // logical quarter at once without bank conflicts and then stores the
         // same B chunks (the B layout's own swizzle keeps those conflict-free).
-        const int h0 = (r ^ (r >> 2)) & 1;
-        const int rot = (r >> 1) & 3;
         const uint32_t brow_off = (r >> 3) * 1024 + (r & 7) * 128;
         const uint32_t ring = smem_u32(smem);
         uint32_t n = 0;  // k blocks of the CTA so far
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-            const Tile t = decode_tile(a, tile);
+        for (int unit = blockIdx.x; ok && unit < us.total; unit += gridDim.x) {
+            const Tile t = decode_unit(a, us, unit);
+            // raw row of this thread's B row: GEMM-1's up rows sit in the second
+            // 128-row box, whatever the unit's width; rows past the unit are idle
+            const int nf = t.ncol / 2;
+            const int rr = (GEMM == 1 && r >= nf) ? BN / 2 + (r - nf) : r;
+            const bool active = r < t.ncol;
+            const int h0 = (rr ^ (rr >> 2)) & 1;
+            const int rot = (rr >> 1) & 3;
             for (int kb = 0; kb < t.nkb; ++kb, ++n) {
                 if ((int)(n & (DEQ_GROUPS - 1)) != g) continue;
                 const int s = (int)(n % TSTAGES), sb = (int)(n % BSTAGES);
@@ -525,9 +564,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
                     ok = false;
                     break;
                 }
-                const uint32_t rrow = ring + s * TSTAGE_BYTES + A_BYTES + r * RAW_ROW;
+                const uint32_t rrow = ring + s * TSTAGE_BYTES + A_BYTES + rr * RAW_ROW;
                 const uint32_t brow = ring + TSTAGES * TSTAGE_BYTES + sb * B_BYTES + brow_off;
-                if (WB == 4) {
+                if (!active) {
+                } else if (WB == 4) {
                     const uint4 qa = lds128(rrow + 16 * h0);
                     const uint4 qb = lds128(rrow + 16 * (h0 ^ 1));
                     const uint4 q0 = h0 ? qb : qa, q1 = h0 ? qa : qb;
@@ -563,8 +603,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
         // ---------------- staging: per-tile token rows, factors and row scales ----------------
         uint32_t st_ph[2] = {0, 0};
         int b = 0;
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            const Tile t = decode_tile(a, tile);
+        for (int unit = blockIdx.x; unit < us.total; unit += gridDim.x) {
+            const Tile t = decode_unit(a, us, unit);
             if (!warp_wait(&sh->stage_empty[b], st_ph[b] ^ 1u, sh)) break;
             Stage& st = sh->stage[b];
             const int irow = t.shared ? a.Is : a.I;
@@ -582,10 +622,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
                     st.fac[j] = 0.f;
                 }
             }
+            const int nf = t.ncol / 2;  // GEMM-1: features of the unit
 #pragma unroll
             for (int j = lane; j < BN; j += 32)
-                st.sc[j] = GEMM == 1 ? __ldg(S + (j < BN / 2 ? 0 : irow) + t.col0 + (j & (BN / 2 - 1)))
-                                     : __ldg(S + t.col0 + j);
+                st.sc[j] = j >= t.ncol ? 0.f
+                           : GEMM == 1 ? __ldg(S + (j < nf ? t.col0 + j : irow + t.col0 + (j - nf)))
+                                       : __ldg(S + t.col0 + j);
             mbar_arrive(&sh->stage_full[b]);  // every lane: its writes are released with the arrival
             st_ph[b] ^= 1u;
             b ^= 1;
@@ -596,8 +638,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
         const int m = quarter * 32 + lane;  // token row of the tile = TMEM lane
         uint32_t acc_ph[2] = {0, 0};
         int buf = 0;
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            const Tile t = decode_tile(a, tile);
+        for (int unit = blockIdx.x; unit < us.total; unit += gridDim.x) {
+            const Tile t = decode_unit(a, us, unit);
             const bool got = (!a.stall || mbar_wait(&sh->never, 0, sh, kStallCycles)) &&
                              mbar_wait(&sh->stage_full[buf], acc_ph[buf], sh) &&
                              mbar_wait(&sh->acc_full[buf], acc_ph[buf], sh);
@@ -609,22 +651,23 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
             const uint32_t stg = smem_u32(&sh->epi[warp - WARP_EPI0][0]);
             const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;
             if (GEMM == 1) {
-                // features 64c .. 64c + 63 of the tile: gate in column j, up in column 128 + j
+                // features of column half c of the unit: gate in column j, up in column nf + j
                 const int irow = t.shared ? a.Is : a.I;
                 __half* hbase = (t.shared ? a.h_s : a.h_r) + t.col0;
                 int rows[2];  // the token rows this lane stores: 16 i + lane / 2
 #pragma unroll
                 for (int i = 0; i < 2; ++i) rows[i] = lds32(smem_u32(&st.slot[quarter * 32 + 16 * i + (lane >> 1)]));
+                const int nf = t.ncol / 2, hw = nf / 2;  // features of the unit, of this warp's half
 #pragma unroll 1
-                for (int c0 = 64 * chalf; c0 < 64 * chalf + 64; c0 += 16) {
+                for (int c0 = hw * chalf; c0 < hw * chalf + hw; c0 += 16) {
                     uint32_t gv[16], uv[16];
                     tmem_ld16_wait(tbase + c0, gv);
-                    tmem_ld16_wait(tbase + BN / 2 + c0, uv);
+                    tmem_ld16_wait(tbase + nf + c0, uv);
                     float sg[16], su[16];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const float4 a4 = lds128f(st_sc + 4 * (c0 + 4 * q));
-                        const float4 b4 = lds128f(st_sc + 4 * (BN / 2 + c0 + 4 * q));
+                        const float4 b4 = lds128f(st_sc + 4 * (nf + c0 + 4 * q));
                         sg[4 * q] = a4.x; sg[4 * q + 1] = a4.y; sg[4 * q + 2] = a4.z; sg[4 * q + 3] = a4.w;
                         su[4 * q] = b4.x; su[4 * q + 1] = b4.y; su[4 * q + 2] = b4.z; su[4 * q + 3] = b4.w;
                     }
@@ -654,13 +697,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX_r, const __grid_cons
                     __syncwarp();  // the stage is read before the next columns overwrite it
                 }
             } else {
-                // output columns 128c .. 128c + 127 of the tile
+                // output columns of column half c of the unit
                 float* ybase = a.y + t.col0;
                 int rows[4];  // the token rows this lane stores: 8 i + lane / 4
 #pragma unroll
                 for (int i = 0; i < 4; ++i) rows[i] = lds32(smem_u32(&st.slot[quarter * 32 + 8 * i + (lane >> 2)]));
+                const int hw = t.ncol / 2;
 #pragma unroll 1
-                for (int c0 = 128 * chalf; c0 < 128 * chalf + 128; c0 += 16) {
+                for (int c0 = hw * chalf; c0 < hw * chalf + hw; c0 += 16) {
                     uint32_t v[16];
                     tmem_ld16_wait(tbase + c0, v);
                     float4 o[4];
