@@ -96,12 +96,15 @@ extern "C" {
 #define MOE_WEIGHTS_INT8 (1u << 11) /* the expert weights (routed and shared) are int8 codes, one
                                        byte per element: w13 [E][2I][H], w2 [E][H][I], shared
                                        w13 [2Is][H], w2 [H][Is] (byte j of a row = element j, two's
-                                       complement; weight = code * row scale).  Every T takes the
-                                       tensor-core sequence (H a multiple of 256, else
-                                       MOE_ERR_UNSUPPORTED; MOE_FORCE_DECODE is MOE_ERR_INVALID_ARG).
-                                       Expert bit width of the checkpoint converter:
-                                       nanocolibri-engine README, "Converting a checkpoint
-                                       yourself" */
+                                       complement; weight = code * row scale).  H must be a
+                                       multiple of 256 (else MOE_ERR_UNSUPPORTED).  With H >= 1024
+                                       and I, Is multiples of 256 the kernel sequences are int4's
+                                       (weight-streaming kernels read the codes as int8 directly;
+                                       no fused stack kernel, no tcgen05 streaming gate/up); other
+                                       shapes take the tensor-core sequence at every T, and
+                                       MOE_FORCE_DECODE on them is MOE_ERR_UNSUPPORTED.  Expert bit
+                                       width of the checkpoint converter: nanocolibri-engine
+                                       README, "Converting a checkpoint yourself" */
 
 /* Device status word: the first 4 bytes of the workspace hold the OR of these
  * bits after a call completes on the device (0 = no check failed).  Under
@@ -216,7 +219,7 @@ size_t moe_layer_workspace_bytes_upto(const moe_cfg_t* cfg, int32_t N);
  *    that magnitude (rows whose largest magnitude is below 2^-113 become
  *    zero; a row holding NaN or infinity gives NaN outputs).  Weight codes
  *    times activation parts accumulate exactly in int32; h is kept in f32.
- *  - otherwise (and at every T under MOE_WEIGHTS_INT8): tensor-core kernels
+ *  - otherwise: tensor-core kernels
  *    with bf16 x, f32 accumulation, and h kept in fp16 as h * 2^-k_t with a
  *    per-token power of two 2^-k_t that keeps it in fp16's normal range.
  *    Weight codes (int4 or int8) enter the MMAs exactly as 16-bit values;

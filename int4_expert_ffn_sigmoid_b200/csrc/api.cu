@@ -31,9 +31,10 @@ constexpr int32_t kMaxTokens = 1 << 20;
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Kernel sequence of a call: the small-batch router + weight-streaming
-// experts; the large router + tensor-core grouped GEMMs (every T with int8
-// expert weights); or the large router + weight-streaming experts (H not a
-// multiple of 256, or MOE_FORCE_DECODE).
+// experts; the large router + tensor-core grouped GEMMs; or the large router
+// + weight-streaming experts (H not a multiple of 256, or MOE_FORCE_DECODE).
+// int8 expert weights stream through the TMA-ring kernels only: shapes those
+// do not serve take the tensor-core sequence at every T.
 enum class Path { kSmall, kTensorCore, kLargeStreaming };
 
 // Average (token, pick) slots per routed expert below which large batches
@@ -42,8 +43,10 @@ enum class Path { kSmall, kTensorCore, kLargeStreaming };
 // bound by reading the touched experts' weights.
 constexpr int kTcMinSlotsPerExpert = 32;
 
+bool int8_streams(const moe_cfg_t& c) { return experts_w13_tma(c.H) && experts_w2_tma(c.H, c.I, c.Is); }
+
 Path choose_path(const moe_cfg_t& c, int32_t T) {
-    if (c.flags & MOE_WEIGHTS_INT8) return Path::kTensorCore;
+    if ((c.flags & MOE_WEIGHTS_INT8) && !int8_streams(c)) return Path::kTensorCore;
     if (T <= kDecodeMaxTokens && !(c.flags & MOE_FORCE_PREFILL)) return Path::kSmall;
     // GEMM-2 of the tensor-core path tiles 256 output columns
     if ((c.flags & MOE_FORCE_DECODE) || c.H % 256 != 0) return Path::kLargeStreaming;
@@ -118,11 +121,11 @@ int validate_cfg(const moe_cfg_t* c) {
     if (!(c->topp >= 0.0f) || !isfinite(c->topp)) return MOE_ERR_INVALID_ARG;
     if (c->flags & ~kKnownFlags) return MOE_ERR_INVALID_ARG;
     if ((c->flags & MOE_FORCE_DECODE) && (c->flags & MOE_FORCE_PREFILL)) return MOE_ERR_INVALID_ARG;
-    if ((c->flags & MOE_WEIGHTS_INT8) && (c->flags & MOE_FORCE_DECODE)) return MOE_ERR_INVALID_ARG;
     if (c->H % 128 || c->H > 16384) return MOE_ERR_UNSUPPORTED;
-    // int8 expert weights are served by the tensor-core sequence alone, whose
-    // down projection tiles 256 output columns
+    // int8 expert weights: the tensor-core sequence (its down projection tiles
+    // 256 output columns) or the TMA-ring streaming kernels
     if ((c->flags & MOE_WEIGHTS_INT8) && c->H % 256) return MOE_ERR_UNSUPPORTED;
+    if ((c->flags & MOE_WEIGHTS_INT8) && (c->flags & MOE_FORCE_DECODE) && !int8_streams(*c)) return MOE_ERR_UNSUPPORTED;
     if (c->E > kMaxE || c->K > kMaxK) return MOE_ERR_UNSUPPORTED;
     if (c->I % 128 || c->I > 8192) return MOE_ERR_UNSUPPORTED;
     if (c->Is % 128 || c->Is > 8192) return MOE_ERR_UNSUPPORTED;
@@ -398,8 +401,9 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
                              (routed_buckets * slices_of(cfg->I) + shared_chunks * slices_of(cfg->Is));
     int grid13 = 0, grid2 = 0;
     if (!use_tc) {
-        const long long cap13 = experts_resident_ctas(0, cfg->H, w2_tma, p.chunk);
-        const long long cap2 = experts_resident_ctas(1, cfg->H, w2_tma, p.chunk);
+        const bool int8w = (cfg->flags & MOE_WEIGHTS_INT8) != 0;
+        const long long cap13 = experts_resident_ctas(0, cfg->H, w2_tma, p.chunk, int8w);
+        const long long cap2 = experts_resident_ctas(1, cfg->H, w2_tma, p.chunk, int8w);
         grid13 = (int)(tasks13 < cap13 ? tasks13 : cap13);
         grid2 = (int)(tasks2 < cap2 ? tasks2 : cap2);
     }

@@ -854,33 +854,48 @@ __global__ void __launch_bounds__(256, 1) experts_w13_bulk_kernel(Params p) {
 // it exits.
 // ---------------------------------------------------------------------------
 constexpr int kTmaThreads = 288;                               // 8 consumer warps + the producer warp
-// Ring geometry for tasks of kChunk tokens: the activation part of a stage
-// holds 2 kChunk rows, and the ring is as deep as shared memory allows
-// (8 stages for 16 tokens, 6 for 32).
-template <int kChunk>
+// Ring geometry for tasks of kChunk tokens and WB-bit codes: the activation
+// part of a stage holds 2 kChunk rows, the weight part the 256-wide k chunk of
+// 64 gate and 64 up rows (16 KiB of int4, 32 KiB of int8: the 128-byte rows
+// of four tiles, gate k 0..127, gate k 128..255, then up), and the ring is
+// as deep as shared memory allows (int4: 8 stages for 16 tokens, 6 for 32;
+// int8: 5 and 4).
+template <int kChunk, int WB>
 struct Tma13 {
-    static constexpr int kStages = kChunk == kChunkTokens ? 8 : 6;
+    static constexpr int kWBytes = kTmaWBytes * WB / 4;
+    static constexpr int kStages = WB == 4 ? (kChunk == kChunkTokens ? 8 : 6) : (kChunk == kChunkTokens ? 5 : 4);
     static constexpr int kXBytes = 2 * kChunk * kTmaXStride;
     static constexpr size_t kMisc = 256 + 2 * 8 * kChunk * 4;  // barriers, flag, per-warp maxima
-    static constexpr size_t kSmem = kShmBytes + kMisc + 1024 /* alignment */ + (size_t)kStages * (kTmaWBytes + kXBytes);
+    static constexpr size_t kSmem = kShmBytes + kMisc + 1024 /* alignment */ + (size_t)kStages * (kWBytes + kXBytes);
     static_assert(kSmem <= 227 * 1024, "TMA gate/up shared memory");
     static_assert((size_t)kStages * kXBytes >= kBuildBytes, "table build scratch fits the activation ring");
 };
 
 // The weights of k chunk c of a task whose gate rows start at row rg and up
-// rows at ru of `map`: expect the bytes, then the two tile loads.
+// rows at ru of `map`: expect the bytes, then the tile loads (64 rows x 128
+// bytes each: two for int4, four for int8).
+template <int WB>
 __device__ __forceinline__ void issue_w13_chunk(const CUtensorMap* map, uint64_t* bar, uint8_t* dst, int c, int rg,
                                                 int ru) {
-    bar_expect_tx(bar, kTmaWBytes);
-    tma_tile(dst, map, bar, c * kTmaRowBytes, rg);
-    tma_tile(dst + kTmaWBytes / 2, map, bar, c * kTmaRowBytes, ru);
+    constexpr int kTile = kRows13 * kTmaRowBytes;
+    bar_expect_tx(bar, kTmaWBytes * WB / 4);
+    if (WB == 4) {
+        tma_tile(dst, map, bar, c * kTmaRowBytes, rg);
+        tma_tile(dst + kTile, map, bar, c * kTmaRowBytes, ru);
+    } else {
+        tma_tile(dst, map, bar, c * kTmaChunk, rg);
+        tma_tile(dst + kTile, map, bar, c * kTmaChunk + kTmaRowBytes, rg);
+        tma_tile(dst + 2 * kTile, map, bar, c * kTmaChunk, ru);
+        tma_tile(dst + 3 * kTile, map, bar, c * kTmaChunk + kTmaRowBytes, ru);
+    }
 }
 
 // Consumer main loop of one task: nch stages from stage counter n on.
-template <int NT, int kStages, int kXBytes>
+template <int NT, int kStages, int kXBytes, int WB>
 __device__ __forceinline__ void consume13(int nch, uint32_t& n, uint64_t* full, uint64_t* empty, const uint8_t* wring,
                                           const uint8_t* xring, volatile int* abort, unsigned* status,
                                           int (&acc)[NT][4]) {
+    constexpr int kWBytes = kTmaWBytes * WB / 4, kTile = kRows13 * kTmaRowBytes;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, q = lane & 3;
     constexpr int kSets = NT == 1 ? 2 : 1;
     int part[kSets][NT][4];
@@ -896,14 +911,23 @@ __device__ __forceinline__ void consume13(int nch, uint32_t& n, uint64_t* full, 
             *abort = 1;
             if (lane == 0) atomicOr(status, ST_TIMEOUT);
         }
-        const uint8_t* wt = wring + (size_t)s * kTmaWBytes + wrow;
+        const uint8_t* wt = wring + (size_t)s * kWBytes + wrow;
         const uint8_t* xt = xring + (size_t)s * kXBytes + g * kTmaXStride + q * 32;
 #pragma unroll
         for (int kb = 0; kb < kTmaChunk / 128; ++kb) {
-            const int off = ((kb * 4 + q) ^ g) << 4;
-            const uint4 wa = *reinterpret_cast<const uint4*>(wt + off);
-            const uint4 wb = *reinterpret_cast<const uint4*>(wt + kTmaWBytes / 2 + off);
-            kblock8<NT, kSets>(wa, wb, xt + kb * 128, 8 * kTmaXStride, part);
+            if (WB == 4) {
+                const int off = ((kb * 4 + q) ^ g) << 4;
+                const uint4 wa = *reinterpret_cast<const uint4*>(wt + off);
+                const uint4 wb = *reinterpret_cast<const uint4*>(wt + kTile + off);
+                kblock8<NT, kSets>(wa, wb, xt + kb * 128, 8 * kTmaXStride, part);
+            } else {  // codes 32q .. 32q + 31 of block kb: 16-byte chunks 2q, 2q + 1 of tile kb
+                const uint8_t* ga = wt + kb * kTile;
+                const uint8_t* ub = wt + (2 + kb) * kTile;
+                const int o0 = ((2 * q) ^ g) << 4, o1 = ((2 * q + 1) ^ g) << 4;
+                kblock8_i8<NT, kSets>(*reinterpret_cast<const uint4*>(ga + o0), *reinterpret_cast<const uint4*>(ga + o1),
+                                      *reinterpret_cast<const uint4*>(ub + o0), *reinterpret_cast<const uint4*>(ub + o1),
+                                      xt + kb * 128, 8 * kTmaXStride, part);
+            }
         }
         __syncwarp();
         if (lane == 0) bar_arrive(empty + s);
@@ -914,11 +938,11 @@ __device__ __forceinline__ void consume13(int nch, uint32_t& n, uint64_t* full, 
         for (int c = 0; c < 4; ++c) acc[i][c] = part[0][i][c] + part[kSets - 1][i][c] * (kSets - 1);
 }
 
-template <int kChunk>
+template <int kChunk, int WB>
 __global__ void __launch_bounds__(kTmaThreads, 1)
     experts_w13_tma_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_s, Params p) {
-    using Cfg = Tma13<kChunk>;
-    constexpr int kStages = Cfg::kStages, kXBytes = Cfg::kXBytes;
+    using Cfg = Tma13<kChunk, WB>;
+    constexpr int kStages = Cfg::kStages, kXBytes = Cfg::kXBytes, kWBytes = Cfg::kWBytes;
     extern __shared__ __align__(128) uint8_t dsm[];
     Shm& sh = *reinterpret_cast<Shm*>(dsm);
     uint64_t* full = reinterpret_cast<uint64_t*>(dsm + kShmBytes);
@@ -929,7 +953,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     const uint32_t base_s = static_cast<uint32_t>(__cvta_generic_to_shared(dsm));
     const uint32_t ring_s = (base_s + (uint32_t)(kShmBytes + Cfg::kMisc) + 1023u) & ~1023u;
     uint8_t* wring = dsm + (ring_s - base_s);
-    uint8_t* xring = wring + (size_t)kStages * kTmaWBytes;
+    uint8_t* xring = wring + (size_t)kStages * kWBytes;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const bool producer = warp == 8;
     const int H = p.H, nch = H / kTmaChunk;
@@ -955,10 +979,10 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         pre_tok0 = (local / R) * p.chunk;
         if (producer && lane == 0)
             for (int c = 0; c < npre; ++c)
-                issue_w13_chunk(&tm_s, full + c, wring + (size_t)c * kTmaWBytes, c, pre_rbk * kRows13,
-                                p.Is + pre_rbk * kRows13);
+                issue_w13_chunk<WB>(&tm_s, full + c, wring + (size_t)c * kWBytes, c, pre_rbk * kRows13,
+                                    p.Is + pre_rbk * kRows13);
     }
-    if (p.Is > 0) prefetch_l2_slice(p.sh_w13, (size_t)p.Is * p.H);
+    if (p.Is > 0) prefetch_l2_slice(p.sh_w13, (size_t)p.Is * p.H * WB / 4);
     pdl_wait();
     pdl_release();
     if (p.decode_groups > 0) build_tables_small(p, sh, reinterpret_cast<int*>(xring));
@@ -1009,7 +1033,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
                     }
                 }
                 if (lane == 0 && !issued)
-                    issue_w13_chunk(shared ? &tm_s : &tm_r, full + s, wring + (size_t)s * kTmaWBytes, c, rg, ru);
+                    issue_w13_chunk<WB>(shared ? &tm_s : &tm_r, full + s, wring + (size_t)s * kWBytes, c, rg, ru);
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
                     if (src[h]) {
@@ -1057,12 +1081,12 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
             xsc[i] = 0.f;
             if (i < NTt && j < t.nc) {
                 const int tok = slot_token(p, sh, t.shared, t.off, t.tok0 + j);
-                xsc[i] = (tok >= 0 && tok < p.T) ? __ldcg(p.xs + tok) * 0.0625f : 0.f;
+                xsc[i] = (tok >= 0 && tok < p.T) ? __ldcg(p.xs + tok) * code_unit<WB>() : 0.f;
             }
         }
         int acc[kMaxNT][4];
 #define MOE_CONSUME13(N)                                                                                        \
-    consume13<N, kStages, kXBytes>(nch, n, full, empty, wring, xring, abort, status,                          \
+    consume13<N, kStages, kXBytes, WB>(nch, n, full, empty, wring, xring, abort, status,                      \
                                    reinterpret_cast<int(&)[N][4]>(acc))
         switch (NTt) {
             case 1: MOE_CONSUME13(1); break;
@@ -1245,8 +1269,8 @@ __global__ void __launch_bounds__(kTc8Threads, 1)
         pre_tok0 = (local / R) * p.chunk;
         if (warp == 8 && lane == 0)
             for (int c = 0; c < npre; ++c)
-                issue_w13_chunk(&tm_s, full + c, wring + (size_t)c * kTmaWBytes, c, pre_rbk * kRows13,
-                                p.Is + pre_rbk * kRows13);
+                issue_w13_chunk<4>(&tm_s, full + c, wring + (size_t)c * kTmaWBytes, c, pre_rbk * kRows13,
+                                   p.Is + pre_rbk * kRows13);
     }
     if (p.Is > 0) prefetch_l2_slice(p.sh_w13, (size_t)p.Is * p.H);
     pdl_wait();
@@ -1289,7 +1313,7 @@ __global__ void __launch_bounds__(kTc8Threads, 1)
                         break;
                     }
                     if (!(r == 0 && c < npre))  // else issued before the tables were read
-                        issue_w13_chunk(shared ? &tm_s : &tm_r, full + s, wring + (size_t)s * kTmaWBytes, c, rg, ru);
+                        issue_w13_chunk<4>(shared ? &tm_s : &tm_r, full + s, wring + (size_t)s * kTmaWBytes, c, rg, ru);
                     last_round[s] = round;
                 }
                 if (!ok) break;
@@ -1747,10 +1771,14 @@ __global__ void __launch_bounds__(256, 2) experts_w2_kernel(Params p) {
 // ---------------------------------------------------------------------------
 constexpr size_t kW2MiscBytes = 256;
 // Ring and staging for tasks of kChunk tokens (offsets from the ring's start).
-template <int kChunk>
+// Down ring geometry for tasks of kChunk tokens and WB-bit codes: a stage is
+// the 256-wide k chunk of 128 down rows (16 KiB of int4; 32 KiB of int8, two
+// 128-byte-row tiles for k 0..127 and 128..255).
+template <int kChunk, int WB>
 struct Tma2 {
-    static constexpr int kStages = kChunk == kChunkTokens ? 8 : 6;
-    static constexpr size_t kXOff = (size_t)kStages * kW2Bytes;
+    static constexpr int kWBytes = kW2Bytes * WB / 4;
+    static constexpr int kStages = WB == 4 ? (kChunk == kChunkTokens ? 8 : 6) : (kChunk == kChunkTokens ? 4 : 3);
+    static constexpr size_t kXOff = (size_t)kStages * kWBytes;
     static constexpr size_t kRawOff = kXOff + (size_t)2 * kChunk * kStride2;
     static constexpr size_t kRsOff = kRawOff + (size_t)kChunk * kSliceK * 4;
     static constexpr size_t kSmem = kShmBytes + kW2MiscBytes + 1024 /* alignment */ + kRsOff + (size_t)2 * kMaxRows2 * 4;
@@ -1781,10 +1809,11 @@ __device__ __forceinline__ void fetch2c(const Params& p, Shm& sh, const Task2& t
     cp_async_commit();
 }
 
-template <int NT, int kStages>
+template <int NT, int kStages, int WB>
 __device__ __forceinline__ void consume2(const Task2& tk, uint32_t& n, uint64_t* full, uint64_t* empty,
                                          const uint8_t* wring, const uint8_t* xs, const float* rs, const Params& p,
                                          const Shm& sh, volatile int* abort, unsigned* status) {
+    constexpr int kWBytes = kW2Bytes * WB / 4;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, q = lane & 3;
     constexpr int kSets = NT == 1 ? 2 : 1;
     const size_t TK = (size_t)p.T * p.K;
@@ -1804,14 +1833,24 @@ __device__ __forceinline__ void consume2(const Task2& tk, uint32_t& n, uint64_t*
                 *abort = 1;
                 if (lane == 0) atomicOr(status, ST_TIMEOUT);
             }
-            const uint8_t* wt = wring + (size_t)s * kW2Bytes;
+            const uint8_t* wt = wring + (size_t)s * kWBytes;
             const uint8_t* xt = xs + g * kStride2 + q * 32 + c * kTmaChunk;
 #pragma unroll
             for (int kb = 0; kb < kTmaChunk / 128; ++kb) {
-                const int off = ((kb * 4 + q) ^ g) << 4;
-                const uint4 wa = *reinterpret_cast<const uint4*>(wt + wa_row + off);
-                const uint4 wb = *reinterpret_cast<const uint4*>(wt + wb_row + off);
-                kblock8<NT, kSets>(wa, wb, xt + kb * 128, 8 * kStride2, part);
+                if (WB == 4) {
+                    const int off = ((kb * 4 + q) ^ g) << 4;
+                    const uint4 wa = *reinterpret_cast<const uint4*>(wt + wa_row + off);
+                    const uint4 wb = *reinterpret_cast<const uint4*>(wt + wb_row + off);
+                    kblock8<NT, kSets>(wa, wb, xt + kb * 128, 8 * kStride2, part);
+                } else {  // codes 32q .. 32q + 31 of block kb: 16-byte chunks 2q, 2q + 1 of tile kb
+                    const uint8_t* tb = wt + kb * kW2Bytes;
+                    const int o0 = ((2 * q) ^ g) << 4, o1 = ((2 * q + 1) ^ g) << 4;
+                    kblock8_i8<NT, kSets>(*reinterpret_cast<const uint4*>(tb + wa_row + o0),
+                                          *reinterpret_cast<const uint4*>(tb + wa_row + o1),
+                                          *reinterpret_cast<const uint4*>(tb + wb_row + o0),
+                                          *reinterpret_cast<const uint4*>(tb + wb_row + o1), xt + kb * 128, 8 * kStride2,
+                                          part);
+                }
             }
             __syncwarp();
             if (lane == 0) bar_arrive(empty + s);
@@ -1836,11 +1875,25 @@ __device__ __forceinline__ void consume2(const Task2& tk, uint32_t& n, uint64_t*
     }
 }
 
-template <int kChunk>
+// The down weights of k chunk c (k0 the chunk's first code) of the 128 rows from
+// `row` of `map`: expect the bytes, then the tile load(s): one 128 x 128-byte
+// tile of int4, two of int8.
+template <int WB>
+__device__ __forceinline__ void issue_w2_chunk(const CUtensorMap* map, uint64_t* bar, uint8_t* dst, int k0, int row) {
+    bar_expect_tx(bar, kW2Bytes * WB / 4);
+    if (WB == 4) {
+        tma_tile(dst, map, bar, k0 / 2, row);
+    } else {
+        tma_tile(dst, map, bar, k0, row);
+        tma_tile(dst + kW2Bytes, map, bar, k0 + kTmaRowBytes, row);
+    }
+}
+
+template <int kChunk, int WB>
 __global__ void __launch_bounds__(kTmaThreads, 1)
     experts_w2_tma_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_s, Params p) {
-    using Cfg = Tma2<kChunk>;
-    constexpr int kStages = Cfg::kStages;
+    using Cfg = Tma2<kChunk, WB>;
+    constexpr int kStages = Cfg::kStages, kWBytes = Cfg::kWBytes;
     extern __shared__ __align__(128) uint8_t dsm[];
     Shm& sh = *reinterpret_cast<Shm*>(dsm);
     uint64_t* full = reinterpret_cast<uint64_t*>(dsm + kShmBytes);
@@ -1882,12 +1935,11 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         if (producer && lane == 0)
             for (int i = 0; i < npre; ++i) {
                 const int m = i / nkc, c = i - m * nkc;
-                bar_expect_tx(full + i, kW2Bytes);
-                tma_tile(wring + (size_t)i * kW2Bytes, &tm_s, full + i, (k0 + c * kTmaChunk) / 2,
-                         pre_rbk * p.rows2 + m * kRows2);
+                issue_w2_chunk<WB>(&tm_s, full + i, wring + (size_t)i * kWBytes, k0 + c * kTmaChunk,
+                                   pre_rbk * p.rows2 + m * kRows2);
             }
     }
-    if (p.Is > 0) prefetch_l2_slice(p.sh_w2, (size_t)p.H * p.Is / 2);
+    if (p.Is > 0) prefetch_l2_slice(p.sh_w2, (size_t)p.H * p.Is * WB / 8);
     pdl_wait();
     pdl_release();
     load_tables(p, p.ts2, &p.ctrl->tasks2, sh.tb, nullptr);
@@ -1931,10 +1983,8 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
                             break;
                         }
                     }
-                    if (lane == 0 && !(r == 0 && (int)n < npre)) {
-                        bar_expect_tx(full + s, kW2Bytes);
-                        tma_tile(wring + (size_t)s * kW2Bytes, map, full + s, (k0 + c * kTmaChunk) / 2, row0 + m * kRows2);
-                    }
+                    if (lane == 0 && !(r == 0 && (int)n < npre))
+                        issue_w2_chunk<WB>(map, full + s, wring + (size_t)s * kWBytes, k0 + c * kTmaChunk, row0 + m * kRows2);
                     last_round[s] = round;
                 }
         }
@@ -1969,7 +2019,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
             for (int b = 0; b < klen / kRows13; ++b) m = nanmax(m, sh.hmr[j][b]);
             const QScale qs = qscale(m);
             sh.qs[j] = qs;
-            sh.xsc[j] = qs.s * 0.0625f;
+            sh.xsc[j] = qs.s * code_unit<WB>();
         }
         consumers_sync();
         for (int j = warp; j < nc; j += 8) {
@@ -1989,7 +2039,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         if (nx.ok) fetch2c(p, sh, nx, raw, rs2 + ((r + 1) & 1) * kMaxRows2);
         const float* rs = rs2 + (r & 1) * kMaxRows2;
         constexpr int kMaxNT = kChunk / 4;
-#define MOE_CONSUME2(N) consume2<N, kStages>(cur, n, full, empty, wring, xs, rs, p, sh, abort, status)
+#define MOE_CONSUME2(N) consume2<N, kStages, WB>(cur, n, full, empty, wring, xs, rs, p, sh, abort, status)
         switch ((2 * nc + 7) >> 3) {
             case 1: MOE_CONSUME2(1); break;
             case 2: MOE_CONSUME2(2); break;
@@ -2013,7 +2063,7 @@ bool w13_tma(int H) { return H >= kTmaMinH && H % kTmaChunk == 0; }
 
 template <typename Kern>
 int resident(Kern kern, size_t smem, int which, int threads = 256) {
-    static int cache[10][64];  // by kernel (`which`) and device
+    static int cache[16][64];  // by kernel (`which`) and device
     static_assert(kSmem13Bulk <= 227 * 1024, "bulk gate/up shared memory");
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
@@ -2031,16 +2081,28 @@ int resident(Kern kern, size_t smem, int which, int threads = 256) {
 }  // namespace
 
 // Persistent grid of the weight-streaming kernels: the CTAs that fit at once
-// (which: 0 gate/up, 1 down).  Also sets the kernels' shared-memory limits.
-int experts_resident_ctas(int which, int H, bool w2_tma, int chunk) {
+// (which: 0 gate/up, 1 down; int8w: int8 codes, TMA-ring kernels only).  Also
+// sets the kernels' shared-memory limits.
+int experts_resident_ctas(int which, int H, bool w2_tma, int chunk, bool int8w) {
+    if (int8w) {
+        if (which == 1)
+            return chunk == kMaxChunk
+                       ? resident(experts_w2_tma_kernel<kMaxChunk, 8>, Tma2<kMaxChunk, 8>::kSmem, 13, kTmaThreads)
+                       : resident(experts_w2_tma_kernel<kChunkTokens, 8>, Tma2<kChunkTokens, 8>::kSmem, 12, kTmaThreads);
+        return chunk == kMaxChunk
+                   ? resident(experts_w13_tma_kernel<kMaxChunk, 8>, Tma13<kMaxChunk, 8>::kSmem, 11, kTmaThreads)
+                   : resident(experts_w13_tma_kernel<kChunkTokens, 8>, Tma13<kChunkTokens, 8>::kSmem, 10, kTmaThreads);
+    }
     if (which == 1) {
         if (!w2_tma) return resident(experts_w2_kernel, kSmem2, 3);
-        return chunk == kMaxChunk ? resident(experts_w2_tma_kernel<kMaxChunk>, Tma2<kMaxChunk>::kSmem, 7, kTmaThreads)
-                                  : resident(experts_w2_tma_kernel<kChunkTokens>, Tma2<kChunkTokens>::kSmem, 6, kTmaThreads);
+        return chunk == kMaxChunk ? resident(experts_w2_tma_kernel<kMaxChunk, 4>, Tma2<kMaxChunk, 4>::kSmem, 7, kTmaThreads)
+                                  : resident(experts_w2_tma_kernel<kChunkTokens, 4>, Tma2<kChunkTokens, 4>::kSmem, 6,
+                                             kTmaThreads);
     }
     if (w13_tma(H))
-        return chunk == kMaxChunk ? resident(experts_w13_tma_kernel<kMaxChunk>, Tma13<kMaxChunk>::kSmem, 8, kTmaThreads)
-                                  : resident(experts_w13_tma_kernel<kChunkTokens>, Tma13<kChunkTokens>::kSmem, 5, kTmaThreads);
+        return chunk == kMaxChunk
+                   ? resident(experts_w13_tma_kernel<kMaxChunk, 4>, Tma13<kMaxChunk, 4>::kSmem, 8, kTmaThreads)
+                   : resident(experts_w13_tma_kernel<kChunkTokens, 4>, Tma13<kChunkTokens, 4>::kSmem, 5, kTmaThreads);
     if (H <= kBulkMaxK) return resident(experts_w13_bulk_kernel, kSmem13Bulk, 4);
     return H <= kWholeMaxK ? resident(experts_w13_kernel<1>, kSmem13[1], 1)
                            : resident(experts_w13_kernel<2>, kSmem13[2], 2);
@@ -2048,17 +2110,28 @@ int experts_resident_ctas(int which, int H, bool w2_tma, int chunk) {
 
 cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
     const dim3 g(grid), b(256);
+    const bool int8w = (p.flags & kFlagWeightsInt8) != 0;
+    if (int8w && !w13_tma(p.H)) return cudaErrorInvalidValue;  // the host routes such shapes elsewhere
     if (w13_tma(p.H)) {
-        // routed gate/up rows [E*2I][H/2] and the shared expert's [2Is][H/2],
-        // tiles of 64 rows x 128 bytes (any valid map when there is no shared expert)
+        // routed gate/up rows [E*2I][H/2] (int8: [H]) and the shared expert's
+        // [2Is][H/2] ([H]), tiles of 64 rows x 128 bytes (any valid map when
+        // there is no shared expert)
+        const int per = int8w ? 1 : 2;  // code elements per byte
         CUtensorMap tm_r, tm_s;
         const bool ok =
-            encode_tensor_map_2d(&tm_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.w13, p.H / 2, (uint64_t)p.E * 2 * p.I,
+            encode_tensor_map_2d(&tm_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.w13, p.H / per, (uint64_t)p.E * 2 * p.I,
                                  kTmaRowBytes, kRows13, CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_tensor_map_2d(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.Is > 0 ? (const void*)p.sh_w13 : (const void*)p.w13,
-                                 p.H / 2, p.Is > 0 ? 2 * (uint64_t)p.Is : 2 * (uint64_t)kRows13, kTmaRowBytes, kRows13,
+                                 p.H / per, p.Is > 0 ? 2 * (uint64_t)p.Is : 2 * (uint64_t)kRows13, kTmaRowBytes, kRows13,
                                  CU_TENSOR_MAP_SWIZZLE_128B);
         if (!ok) return cudaErrorInvalidValue;
+        if (int8w) {
+            if (p.chunk == kMaxChunk)
+                return launch_pdl(experts_w13_tma_kernel<kMaxChunk, 8>, g, dim3(kTmaThreads), Tma13<kMaxChunk, 8>::kSmem,
+                                  stream, tm_r, tm_s, p);
+            return launch_pdl(experts_w13_tma_kernel<kChunkTokens, 8>, g, dim3(kTmaThreads),
+                              Tma13<kChunkTokens, 8>::kSmem, stream, tm_r, tm_s, p);
+        }
         if (p.chunk == kMaxChunk && experts_w13_tc8(p.H, p.I, p.Is, p.T, p.K, p.E)) {
             // one CTA per SM, like the mma.sync kernel whose residency sized the grid
             // (this call also sets the kernel's shared-memory limit)
@@ -2068,10 +2141,10 @@ cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
                               tm_r, tm_s, p);
         }
         if (p.chunk == kMaxChunk)
-            return launch_pdl(experts_w13_tma_kernel<kMaxChunk>, g, dim3(kTmaThreads), Tma13<kMaxChunk>::kSmem, stream,
-                              tm_r, tm_s, p);
-        return launch_pdl(experts_w13_tma_kernel<kChunkTokens>, g, dim3(kTmaThreads), Tma13<kChunkTokens>::kSmem, stream,
-                          tm_r, tm_s, p);
+            return launch_pdl(experts_w13_tma_kernel<kMaxChunk, 4>, g, dim3(kTmaThreads), Tma13<kMaxChunk, 4>::kSmem,
+                              stream, tm_r, tm_s, p);
+        return launch_pdl(experts_w13_tma_kernel<kChunkTokens, 4>, g, dim3(kTmaThreads), Tma13<kChunkTokens, 4>::kSmem,
+                          stream, tm_r, tm_s, p);
     }
     if (p.H <= kBulkMaxK) return launch_pdl(experts_w13_bulk_kernel, g, b, kSmem13Bulk, stream, p);
     if (p.H <= kWholeMaxK) return launch_pdl(experts_w13_kernel<1>, g, b, kSmem13[1], stream, p);
@@ -2094,21 +2167,30 @@ bool experts_w13_tc8(int H, int I, int Is, int T, int K, int E) {
 bool experts_w2_tma(int H, int I, int Is) { return H >= kTmaMinH && I % kTmaChunk == 0 && Is % kTmaChunk == 0; }
 
 cudaError_t launch_experts_w2(const Params& p, int grid, cudaStream_t stream) {
+    const bool int8w = (p.flags & kFlagWeightsInt8) != 0;
+    if (int8w && !experts_w2_tma(p.H, p.I, p.Is)) return cudaErrorInvalidValue;  // routed elsewhere by the host
     if (experts_w2_tma(p.H, p.I, p.Is)) {
-        // routed down rows [E*H][I/2] and the shared expert's [H][Is/2], tiles
-        // of 128 rows x 128 bytes (any valid map when there is no shared expert)
+        // routed down rows [E*H][I/2] (int8: [I]) and the shared expert's
+        // [H][Is/2] ([Is]), tiles of 128 rows x 128 bytes (any valid map when
+        // there is no shared expert)
+        const int per = int8w ? 1 : 2;  // code elements per byte
         CUtensorMap tm_r, tm_s;
         const bool ok =
-            encode_tensor_map_2d(&tm_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.w2, p.I / 2, (uint64_t)p.E * p.H,
+            encode_tensor_map_2d(&tm_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.w2, p.I / per, (uint64_t)p.E * p.H,
                                  kTmaRowBytes, kRows2, CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_tensor_map_2d(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.Is > 0 ? (const void*)p.sh_w2 : (const void*)p.w2,
-                                 p.Is > 0 ? p.Is / 2 : p.I / 2, p.H, kTmaRowBytes, kRows2, CU_TENSOR_MAP_SWIZZLE_128B);
+                                 p.Is > 0 ? p.Is / per : p.I / per, p.H, kTmaRowBytes, kRows2, CU_TENSOR_MAP_SWIZZLE_128B);
         if (!ok) return cudaErrorInvalidValue;
-        if (p.chunk == kMaxChunk)
-            return launch_pdl(experts_w2_tma_kernel<kMaxChunk>, dim3(grid), dim3(kTmaThreads), Tma2<kMaxChunk>::kSmem,
-                              stream, tm_r, tm_s, p);
-        return launch_pdl(experts_w2_tma_kernel<kChunkTokens>, dim3(grid), dim3(kTmaThreads), Tma2<kChunkTokens>::kSmem,
-                          stream, tm_r, tm_s, p);
+        const dim3 g(grid), b(kTmaThreads);
+        if (int8w)
+            return p.chunk == kMaxChunk
+                       ? launch_pdl(experts_w2_tma_kernel<kMaxChunk, 8>, g, b, Tma2<kMaxChunk, 8>::kSmem, stream, tm_r, tm_s, p)
+                       : launch_pdl(experts_w2_tma_kernel<kChunkTokens, 8>, g, b, Tma2<kChunkTokens, 8>::kSmem, stream,
+                                    tm_r, tm_s, p);
+        return p.chunk == kMaxChunk
+                   ? launch_pdl(experts_w2_tma_kernel<kMaxChunk, 4>, g, b, Tma2<kMaxChunk, 4>::kSmem, stream, tm_r, tm_s, p)
+                   : launch_pdl(experts_w2_tma_kernel<kChunkTokens, 4>, g, b, Tma2<kChunkTokens, 4>::kSmem, stream, tm_r,
+                                tm_s, p);
     }
     return launch_pdl(experts_w2_kernel, dim3(grid), dim3(256), kSmem2, stream, p);
 }

@@ -136,6 +136,41 @@ __device__ __forceinline__ void kblock8(const uint4& wa, const uint4& wb, const 
     }
 }
 
+// kblock8 for int8 weight codes (one byte per element): wa0, wa1 hold the 32
+// consecutive codes of row g of the block and wb0, wb1 those of row g + 8.
+// The MMA k slots take, of every group of eight codes, the even ones and then
+// the odd ones (two byte permutes per register), the order in which the
+// activations are stored.  The products are c * q (the int4 path's are
+// 16 c * q).
+template <int NT, int kSets>
+__device__ __forceinline__ void kblock8_i8(const uint4& wa0, const uint4& wa1, const uint4& wb0, const uint4& wb1,
+                                           const uint8_t* xrow, int tile_stride, int (&part)[kSets][NT][4]) {
+    const uint32_t aw[8] = {wa0.x, wa0.y, wa0.z, wa0.w, wa1.x, wa1.y, wa1.z, wa1.w};
+    const uint32_t bw[8] = {wb0.x, wb0.y, wb0.z, wb0.w, wb1.x, wb1.y, wb1.z, wb1.w};
+    uint32_t A[4][4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        A[m][0] = __byte_perm(aw[2 * m], aw[2 * m + 1], 0x6420);
+        A[m][1] = __byte_perm(bw[2 * m], bw[2 * m + 1], 0x6420);
+        A[m][2] = __byte_perm(aw[2 * m], aw[2 * m + 1], 0x7531);
+        A[m][3] = __byte_perm(bw[2 * m], bw[2 * m + 1], 0x7531);
+    }
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+        const uint4 b01 = *reinterpret_cast<const uint4*>(xrow + i * tile_stride);
+        const uint4 b23 = *reinterpret_cast<const uint4*>(xrow + i * tile_stride + 16);
+        mma_s8(part[0][i], A[0], b01.x, b01.y);
+        mma_s8(part[kSets - 1][i], A[1], b01.z, b01.w);
+        mma_s8(part[0][i], A[2], b23.x, b23.y);
+        mma_s8(part[kSets - 1][i], A[3], b23.z, b23.w);
+    }
+}
+
+// Scale of the int32 sums into activation-scale units: the int4 codes enter
+// the MMAs as 16 c, the int8 codes as c.
+template <int WB>
+constexpr float code_unit() { return WB == 4 ? 0.0625f : 1.0f; }
+
 // Both int8 parts of mma columns 2j, 2j+1 -> the value in units of the
 // activation scale times 16.
 __device__ __forceinline__ float join(int c0, int c1) { return (float)c0 + (float)c1 * (1.0f / 256.0f); }

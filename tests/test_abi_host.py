@@ -151,23 +151,27 @@ def test_path_choice(moe):
 
 
 def test_int8_weights_flag(moe):
-    """int8 expert weights take the tensor-core sequence at every T; the
-    weight-streaming sequence (MOE_FORCE_DECODE), a hidden size that is not a
-    multiple of 256 and the fused stack kernel are refused."""
+    """int8 expert weights take int4's kernel sequences where the TMA-ring
+    streaming kernels serve the shape (H >= 1024, H, I, Is multiples of 256),
+    else the tensor-core sequence at every T; never the fused stack kernel."""
     nano = _shape()
     I8 = moe.MOE_WEIGHTS_INT8
-    for T in (1, 16, 64, 65, 1023, 4096):
-        assert moe.layer_path(nano, T, I8) == moe.MOE_PATH_TENSOR_CORE, T
-        assert moe.layer_path(nano, T, I8 | moe.MOE_FORCE_PREFILL) == moe.MOE_PATH_TENSOR_CORE, T
-        assert moe.kernel_launches(nano, T, I8) == 5, T
-    assert moe.layer_path(nano, 16, I8 | moe.MOE_FORCE_DECODE) == 0
-    assert moe.workspace_bytes(nano, 16, I8 | moe.MOE_FORCE_DECODE) == 0
-    assert _call(moe, nano, T=4, flags=I8 | moe.MOE_FORCE_DECODE) == moe.MOE_ERR_INVALID_ARG
+    S, TC, LS = moe.MOE_PATH_SMALL_BATCH, moe.MOE_PATH_TENSOR_CORE, moe.MOE_PATH_LARGE_STREAMING
+    for T, path in ((1, S), (16, S), (64, S), (65, LS), (1023, LS), (4096, TC)):
+        assert moe.layer_path(nano, T, I8) == path == moe.layer_path(nano, T), T
+        assert moe.kernel_launches(nano, T, I8) == moe.kernel_launches(nano, T), T
+        assert moe.workspace_bytes(nano, T, I8) == moe.workspace_bytes(nano, T), T
+    assert moe.layer_path(nano, 16, I8 | moe.MOE_FORCE_PREFILL) == TC
+    assert moe.layer_path(nano, 4096, I8 | moe.MOE_FORCE_DECODE) == LS
+    # shapes without int8 streaming kernels: the tensor-core sequence at every T
+    small = _shape(H=512, I=256, Is=256)
+    for T in (1, 16, 300):
+        assert moe.layer_path(small, T, I8) == TC, T
+    assert moe.layer_path(small, 16, I8 | moe.MOE_FORCE_DECODE) == 0
+    assert _call(moe, small, T=4, flags=I8 | moe.MOE_FORCE_DECODE) == moe.MOE_ERR_UNSUPPORTED
     assert moe.layer_path(_shape(H=1152), 4096, I8) == 0
     assert _call(moe, _shape(H=1152), T=4, flags=I8) == moe.MOE_ERR_UNSUPPORTED
-    # the tensor-core workspace at every T, largest at N itself
-    assert moe.workspace_bytes(nano, 16, I8) == moe.workspace_bytes(nano, 16, moe.MOE_FORCE_PREFILL)
-    assert moe.workspace_bytes_upto(nano, 300, I8) == moe.workspace_bytes(nano, 300, I8)
+    assert moe.workspace_bytes_upto(small, 300, I8) == moe.workspace_bytes(small, 300, I8)
     for T in (1, 4, 16):
         assert moe.stack_path(nano, T, 23, I8) == moe.MOE_PATH_PER_LAYER
         assert moe.stack_path(nano, T, 23, I8 | moe.MOE_STACK_FUSED) == moe.MOE_PATH_PER_LAYER

@@ -34,6 +34,8 @@ CASES = [
      400, "decode"),
     ("tensor-core grouped GEMMs, int8 weights", workloads.LayerShape(H=512, E=16, K=8, I=256, Is=384, routed_scaling=2.5),
      130, "int8"),
+    ("TMA-ring weight-streaming kernels, int8 weights",
+     workloads.LayerShape(H=1024, E=64, K=2, I=512, Is=2048, routed_scaling=1.0), 16, "int8"),
 ]
 
 
@@ -45,7 +47,8 @@ def _wbits(mode):
 def test_stalled_wait_reports_timeout_then_recovers(moe, cuda_device, case):
     what, shape, T, mode = CASES[case]
     if mode == "int8":
-        base, path = moe.MOE_WEIGHTS_INT8, moe.MOE_PATH_TENSOR_CORE
+        base = moe.MOE_WEIGHTS_INT8
+        path = moe.MOE_PATH_TENSOR_CORE if shape.H < 1024 else moe.MOE_PATH_SMALL_BATCH
     else:
         base = moe.MOE_FORCE_PREFILL if mode == "prefill" else (moe.MOE_FORCE_DECODE if T > 64 else 0)
         path = moe.MOE_PATH_TENSOR_CORE if mode == "prefill" else (moe.MOE_PATH_LARGE_STREAMING if T > 64 else
@@ -76,6 +79,7 @@ PATHS = [
     ("large-batch streaming kernels", workloads.LayerShape(1024, 64, 2, 512, 2048, 1.0), 150, "decode"),
     ("large-batch streaming, tcgen05 gate/up", workloads.LayerShape(1024, 64, 2, 512, 2048, 1.0), 400, "decode"),
     ("tensor-core kernels, int8 weights", workloads.LayerShape(512, 16, 8, 256, 384, 2.5), 130, "int8"),
+    ("large-batch streaming kernels, int8 weights", workloads.LayerShape(1024, 64, 2, 512, 2048, 1.0), 150, "int8"),
 ]
 
 
