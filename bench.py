@@ -515,15 +515,15 @@ def captured_traffic(workload: str, T: int, kernel: str):
     return None
 
 
-def streaming_kernel_names(shape, T):
+def streaming_kernel_names(shape, T, wbits=4):
     """Gate/up and down kernels of the weight-streaming path for this shape
     and T (the library's selection: TMA-ring kernels from H = 1024 on when H,
     I and Is are multiples of 256, the tcgen05 gate/up kernel among them on
-    the large-batch sequence at 12 or more picks per routed expert; bulk-copy
-    gate/up below; register-ring kernels otherwise)."""
+    the large-batch sequence at 12 or more picks per routed expert with int4
+    codes; bulk-copy gate/up below; register-ring kernels otherwise)."""
     tma2 = shape.H >= 1024 and shape.I % 256 == 0 and shape.Is % 256 == 0
     if shape.H >= 1024 and shape.H % 256 == 0:
-        tc8 = tma2 and T > 64 and T * shape.K >= 12 * shape.E
+        tc8 = wbits == 4 and tma2 and T > 64 and T * shape.K >= 12 * shape.E
         w13 = "experts_w13_tc8_kernel" if tc8 else "experts_w13_tma_kernel"
     else:
         w13 = "experts_w13_bulk_kernel" if shape.H <= 1024 else "experts_w13_kernel"
@@ -670,7 +670,7 @@ def workload_entry(moe, wl, T, device, steps, warmup, use_graph, flush, peaks, s
             dom = 1 if stage_mean[1] >= stage_mean[2] else 2
             names = moe.STAGE_NAMES
             tc = r.path() == moe.MOE_PATH_TENSOR_CORE
-            w13, w2 = streaming_kernel_names(wl.shape, T)
+            w13, w2 = streaming_kernel_names(wl.shape, T, wl.wbits)
             kname = (f"grouped_gemm_kernel<{dom}, {wl.wbits}>" if tc else (w13 if dom == 1 else w2))
             u = m["uniq"]
             kw = [[stage_work(names[dom], wl.shape, T, x, wl.wbits) for x in u[i % N_BATCHES]]
@@ -727,7 +727,7 @@ def run_ours(args, rank, world, device, dist):
         names = moe.STAGE_NAMES
         dom = 1 if stage_mean[1] >= stage_mean[2] else 2
         tc = runner.path() == moe.MOE_PATH_TENSOR_CORE
-        w13, w2 = streaming_kernel_names(wl.shape, T)
+        w13, w2 = streaming_kernel_names(wl.shape, T, wl.wbits)
         kname = f"grouped_gemm_kernel<{dom}, {wl.wbits}>" if tc else (w13 if dom == 1 else w2)
         kw = [[stage_work(names[dom], wl.shape, T, u, wl.wbits) for u in m["uniq"][i % N_BATCHES]]
               for i in range(len(stage_ms))]
