@@ -772,7 +772,9 @@ __global__ void __launch_bounds__(256, 2) router_large_kernel(Params p) {
     for (int i = threadIdx.x; i < E; i += blockDim.x) p.hist[(size_t)blockIdx.x * E + i] = s_cnt[i];
 }
 
-__global__ void __launch_bounds__(256) router_select_kernel(Params p) {
+// 512 threads: the selections of a tile's 32 tokens run two per warp.
+constexpr int kSelectThreads = 512;
+__global__ void __launch_bounds__(kSelectThreads) router_select_kernel(Params p) {
     __shared__ __align__(16) float s_logit[kRouterTileTokens][kMaxE];
     __shared__ int s_cnt[kMaxE];
     __shared__ float s_bias[kMaxE];
@@ -790,7 +792,9 @@ __global__ void __launch_bounds__(256) router_select_kernel(Params p) {
         const int t0 = tile * kRouterTileTokens;
         const int nt = min(kRouterTileTokens, p.T - t0);
         static_assert(kRouterTileTokens == 32, "four tokens per warp in tile_hexp");
-        tile_hexp(p, t0, nt, warp, lane);
+        // the h-scale exponents serve the tensor-core sequence's fp16 h only
+        // (the streaming sequences keep h in f32): a pass over x skipped there
+        if (p.x_perm && warp < 8) tile_hexp(p, t0, nt, warp, lane);
         __syncthreads();  // s_logit is free (previous tile done)
         // four elements per thread, each summed over the slices in ascending
         // order, with up to eight slices' loads of all four in flight
@@ -820,7 +824,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(Params p) {
             }
         }
         __syncthreads();
-        for (int tt = warp; tt < nt; tt += 8) {
+        for (int tt = warp; tt < nt; tt += (int)blockDim.x / 32) {
             const int sel = select_token(p, t0 + tt, s_logit[tt], s_bias, lane);
             // an index outside [0, E) cannot occur; it is counted nowhere and
             // reported by the scatter kernel's range check
@@ -1008,7 +1012,8 @@ cudaError_t launch_router(const Params& p, bool small_path, cudaStream_t stream)
     if (p.tc_router) {
         if (p.lslices <= 0) return cudaErrorInvalidValue;
         err = launch_router_tc(p, stream);
-        if (err == cudaSuccess) err = launch_pdl(router_select_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
+        if (err == cudaSuccess)
+            err = launch_pdl(router_select_kernel, dim3(p.router_blocks), dim3(kSelectThreads), 0, stream, p);
     } else {
         err = launch_pdl(router_large_kernel, dim3(p.router_blocks), dim3(256), 0, stream, p);
     }
