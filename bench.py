@@ -68,7 +68,10 @@ def parse_args():
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the other workloads (prefill, Zipf, large layer) reported beside the decode stack")
     ap.add_argument("--per-layer", action="store_true",
-                    help="time the stack as one moe_layer_forward call per layer instead of the fused kernel")
+                    help="time the stack as one moe_layer_forward call per layer, whatever the library's choice")
+    ap.add_argument("--fused", action="store_true",
+                    help="time the fused stack kernel wherever it serves the call (MOE_STACK_FUSED), whatever the "
+                         "library's choice")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--lookahead", action="store_true",
                     help="fused kernel with its L2 prefetch hints (MOE_LOOKAHEAD; the output is the same)")
@@ -649,8 +652,8 @@ def workload_entry(moe, wl, T, device, steps, warmup, use_graph, flush, peaks, s
     stacked = stacked if stacked is not None else stacked_weights(moe, wl, device)
     L = wl.layers
     modes = ["per_layer"]
-    if moe.stack_path(wl.shape, T, L, (moe.MOE_ADD_RESIDUAL if wl.residual else 0) | moe.MOE_STACK_FUSED) == \
-            moe.MOE_PATH_FUSED_STACK:
+    wflags = (moe.MOE_ADD_RESIDUAL if wl.residual else 0) | (moe.MOE_WEIGHTS_INT8 if wl.wbits == 8 else 0)
+    if moe.stack_path(wl.shape, T, L, wflags | moe.MOE_STACK_FUSED) == moe.MOE_PATH_FUSED_STACK:
         modes.insert(0, "fused")
     entry = {"workload": wl.name, "T": T, "layers": L, "expert_bits": wl.wbits}
     for mode in modes:
@@ -696,9 +699,10 @@ def run_ours(args, rank, world, device, dist):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     use_graph = not args.no_graph
     stacked = stacked_weights(moe, wl, device)
-    flags = moe.MOE_ADD_RESIDUAL if wl.residual else 0
-    fused = (not args.per_layer) and \
-        moe.stack_path(wl.shape, T, wl.layers, flags | moe.MOE_STACK_FUSED) == moe.MOE_PATH_FUSED_STACK
+    flags = (moe.MOE_ADD_RESIDUAL if wl.residual else 0) | (moe.MOE_WEIGHTS_INT8 if wl.wbits == 8 else 0)
+    # the library's own choice for the call (moe_stack_path), unless a flag forces one
+    choice = flags | (moe.MOE_STACK_FUSED if args.fused else 0)
+    fused = (not args.per_layer) and moe.stack_path(wl.shape, T, wl.layers, choice) == moe.MOE_PATH_FUSED_STACK
     runner = Runner(moe, wl, T, device, stacked, "fused" if fused else "per_layer",
                     moe.MOE_LOOKAHEAD if (args.lookahead and fused) else 0)
     L = wl.layers
