@@ -494,10 +494,10 @@ def cpu_baseline_sample(runner, budget_s=15.0):
     return n_tok * len(layers_cpu) / dt, sample, pin.core
 
 
-def captured_traffic(workload: str, T: int, kernel: str):
-    """DRAM bytes per launch of `kernel` on this workload and T from the
-    committed ncu capture (profiles/traffic.json), or None when there is none
-    or the kernel's sources have changed since it was taken."""
+def captured_entry(workload: str, T: int, kernel: str):
+    """The committed ncu capture of `kernel` on this workload and T
+    (profiles/traffic.json), or None when there is none or the kernel's
+    sources have changed since it was taken."""
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
@@ -514,8 +514,14 @@ def captured_traffic(workload: str, T: int, kernel: str):
                     h.update(f.read())
         except OSError:
             return None
-        return int(e["read"]) + int(e["write"]) if h.hexdigest() == e["sha256"] else None
+        return e if h.hexdigest() == e["sha256"] else None
     return None
+
+
+def captured_traffic(workload: str, T: int, kernel: str):
+    """DRAM bytes (read + written) per launch from the committed capture, or None."""
+    e = captured_entry(workload, T, kernel)
+    return int(e["read"]) + int(e["write"]) if e else None
 
 
 def streaming_kernel_names(shape, T, wbits=4):
@@ -626,6 +632,14 @@ def roofline_of(alg_b, alg_f, seconds, peaks, kernel, timing, traffic=None):
     return r
 
 
+def with_ncu_time(r, workload, T, kernel):
+    """Adds the committed ncu launch time (cold cache, serialised) of the same
+    kernel, workload and T beside the live one, as a cross-check."""
+    e = captured_entry(workload, T, kernel)
+    r["ncu_launch_us"] = e.get("ncu_us") if e else None
+    return r
+
+
 def stacked_weights(moe, wl, device):
     layers = [workloads.make_layer(wl.shape, wl.wid, l, device, wl.bias_mode, wbits=wl.wbits) for l in range(wl.layers)]
     st = moe.stack_layers(layers)
@@ -681,9 +695,10 @@ def workload_entry(moe, wl, T, device, steps, warmup, use_graph, flush, peaks, s
             kb = statistics.mean(sum(w[0] for w in ws) for ws in kw) / L
             kf = statistics.mean(sum(w[1] for w in ws) for ws in kw) / L
             d["stages_us_per_step"] = {names[k]: round(stage_mean[k] * 1e3, 2) for k in range(4)}
-            d["kernel_roofline"] = roofline_of(kb, kf, stage_mean[dom] / L / 1e3, peaks, kname,
-                                               "eager pass with per-stage events (no overlap with neighbours)",
-                                               captured_traffic(wl.name, T, kname))
+            d["kernel_roofline"] = with_ncu_time(
+                roofline_of(kb, kf, stage_mean[dom] / L / 1e3, peaks, kname,
+                            "eager pass with per-stage events (no overlap with neighbours)",
+                            captured_traffic(wl.name, T, kname)), wl.name, T, kname)
         entry[mode] = d
         del r
         torch.cuda.empty_cache()
@@ -721,9 +736,10 @@ def run_ours(args, rank, world, device, dist):
     if fused:
         # one kernel per step: the step's events bracket it (and the counters'
         # memset that precedes it, about 1-2 us)
-        roofline = roofline_of(m["bytes"], m["flops"], med_ms / 1e3, peaks, "decode_stack_kernel",
-                               "CUDA graph step (memset + the one kernel), median over the timed steps",
-                               captured_traffic(wl.name, T, "decode_stack_kernel"))
+        roofline = with_ncu_time(
+            roofline_of(m["bytes"], m["flops"], med_ms / 1e3, peaks, "decode_stack_kernel",
+                        "CUDA graph step (memset + the one kernel), median over the timed steps",
+                        captured_traffic(wl.name, T, "decode_stack_kernel")), wl.name, T, "decode_stack_kernel")
         stages = None
     else:
         _, stage_ms = timed_steps(runner, args.steps, 2, use_graph, flush, instrumented=True)
@@ -735,11 +751,12 @@ def run_ours(args, rank, world, device, dist):
         kname = f"grouped_gemm_kernel<{dom}, {wl.wbits}>" if tc else (w13 if dom == 1 else w2)
         kw = [[stage_work(names[dom], wl.shape, T, u, wl.wbits) for u in m["uniq"][i % N_BATCHES]]
               for i in range(len(stage_ms))]
-        roofline = roofline_of(statistics.mean(sum(w[0] for w in ws) for ws in kw) / L,
-                               statistics.mean(sum(w[1] for w in ws) for ws in kw) / L,
-                               stage_mean[dom] / L / 1e3, peaks, kname,
-                               "eager pass with per-stage events (no overlap with neighbours)",
-                               captured_traffic(wl.name, T, kname))
+        roofline = with_ncu_time(
+            roofline_of(statistics.mean(sum(w[0] for w in ws) for ws in kw) / L,
+                        statistics.mean(sum(w[1] for w in ws) for ws in kw) / L,
+                        stage_mean[dom] / L / 1e3, peaks, kname,
+                        "eager pass with per-stage events (no overlap with neighbours)",
+                        captured_traffic(wl.name, T, kname)), wl.name, T, kname)
         stages = {names[k]: round(stage_mean[k] * 1e3, 2) for k in range(4)}
 
     trace = phase_trace(moe, runner) if (args.trace and fused) else None
