@@ -859,15 +859,17 @@ constexpr int kTmaThreads = 288;                               // 8 consumer war
 // 64 gate and 64 up rows (16 KiB of int4, 32 KiB of int8: the 128-byte rows
 // of four tiles, gate k 0..127, gate k 128..255, then up), and the ring is
 // as deep as shared memory allows (int4: 8 stages for 16 tokens, 6 for 32;
-// int8: 5 and 4).
-template <int kChunk, int WB>
+// int8: 5 and 4), or, for two CTAs per SM (kOcc = 2: int4, 16-token tasks),
+// 4 stages each.
+template <int kChunk, int WB, int kOcc = 1>
 struct Tma13 {
+    static_assert(kOcc == 1 || (kOcc == 2 && WB == 4 && kChunk == kChunkTokens), "two CTAs per SM: int4, 16 tokens");
     static constexpr int kWBytes = kTmaWBytes * WB / 4;
-    static constexpr int kStages = WB == 4 ? (kChunk == kChunkTokens ? 8 : 6) : (kChunk == kChunkTokens ? 5 : 4);
+    static constexpr int kStages = kOcc == 2 ? 4 : WB == 4 ? (kChunk == kChunkTokens ? 8 : 6) : (kChunk == kChunkTokens ? 5 : 4);
     static constexpr int kXBytes = 2 * kChunk * kTmaXStride;
     static constexpr size_t kMisc = 256 + 2 * 8 * kChunk * 4;  // barriers, flag, per-warp maxima
     static constexpr size_t kSmem = kShmBytes + kMisc + 1024 /* alignment */ + (size_t)kStages * (kWBytes + kXBytes);
-    static_assert(kSmem <= 227 * 1024, "TMA gate/up shared memory");
+    static_assert(kSmem <= 227 * 1024 / kOcc, "TMA gate/up shared memory");
     static_assert((size_t)kStages * kXBytes >= kBuildBytes, "table build scratch fits the activation ring");
 };
 
@@ -938,10 +940,10 @@ __device__ __forceinline__ void consume13(int nch, uint32_t& n, uint64_t* full, 
         for (int c = 0; c < 4; ++c) acc[i][c] = part[0][i][c] + part[kSets - 1][i][c] * (kSets - 1);
 }
 
-template <int kChunk, int WB>
-__global__ void __launch_bounds__(kTmaThreads, 1)
+template <int kChunk, int WB, int kOcc = 1>
+__global__ void __launch_bounds__(kTmaThreads, kOcc)
     experts_w13_tma_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_s, Params p) {
-    using Cfg = Tma13<kChunk, WB>;
+    using Cfg = Tma13<kChunk, WB, kOcc>;
     constexpr int kStages = Cfg::kStages, kXBytes = Cfg::kXBytes, kWBytes = Cfg::kWBytes;
     extern __shared__ __align__(128) uint8_t dsm[];
     Shm& sh = *reinterpret_cast<Shm*>(dsm);
@@ -2083,7 +2085,7 @@ int resident(Kern kern, size_t smem, int which, int threads = 256) {
 // Persistent grid of the weight-streaming kernels: the CTAs that fit at once
 // (which: 0 gate/up, 1 down; int8w: int8 codes, TMA-ring kernels only).  Also
 // sets the kernels' shared-memory limits.
-int experts_resident_ctas(int which, int H, bool w2_tma, int chunk, bool int8w) {
+int experts_resident_ctas(int which, int H, bool w2_tma, int chunk, bool int8w, bool occ2) {
     if (int8w) {
         if (which == 1)
             return chunk == kMaxChunk
@@ -2099,6 +2101,8 @@ int experts_resident_ctas(int which, int H, bool w2_tma, int chunk, bool int8w) 
                                   : resident(experts_w2_tma_kernel<kChunkTokens, 4>, Tma2<kChunkTokens, 4>::kSmem, 6,
                                              kTmaThreads);
     }
+    if (w13_tma(H) && occ2 && chunk == kChunkTokens)
+        return resident(experts_w13_tma_kernel<kChunkTokens, 4, 2>, Tma13<kChunkTokens, 4, 2>::kSmem, 14, kTmaThreads);
     if (w13_tma(H))
         return chunk == kMaxChunk
                    ? resident(experts_w13_tma_kernel<kMaxChunk, 4>, Tma13<kMaxChunk, 4>::kSmem, 8, kTmaThreads)
@@ -2143,6 +2147,9 @@ cudaError_t launch_experts_w13(const Params& p, int grid, cudaStream_t stream) {
         if (p.chunk == kMaxChunk)
             return launch_pdl(experts_w13_tma_kernel<kMaxChunk, 4>, g, dim3(kTmaThreads), Tma13<kMaxChunk, 4>::kSmem,
                               stream, tm_r, tm_s, p);
+        if (p.w13_occ2)
+            return launch_pdl(experts_w13_tma_kernel<kChunkTokens, 4, 2>, g, dim3(kTmaThreads),
+                              Tma13<kChunkTokens, 4, 2>::kSmem, stream, tm_r, tm_s, p);
         return launch_pdl(experts_w13_tma_kernel<kChunkTokens, 4>, g, dim3(kTmaThreads), Tma13<kChunkTokens, 4>::kSmem,
                           stream, tm_r, tm_s, p);
     }

@@ -219,6 +219,7 @@ struct Params {
     int nsl_r, nsl_s;     // slices of the down projection's reduction (routed, shared)
     int rows2;            // output rows of one down task (kTaskRows2 times 1..8, dividing H)
     int chunk;            // tokens per weight-streaming task: kChunkTokens or kMaxChunk
+    int w13_occ2;         // gate/up on the two-CTAs-per-SM TMA-ring kernel (16-token tasks, int4)
     int decode_groups;    // token groups of the small-batch router (0: tables come from the large router)
     float* lpart;         // [lslices][T][E] partial router logits (split router or tensor-core router)
     int lslices;          // hidden-dimension slices of lpart (0: the selecting router computes its logits)

@@ -27,7 +27,7 @@ cudaError_t launch_experts_w2(const Params& p, int grid, cudaStream_t stream);
 // CTAs of the weight-streaming kernel `which` (0: gate/up, 1: down) that fit
 // on the device at once (the persistent grid size) for hidden size H.  Also
 // sets the kernel's shared-memory attribute.
-int experts_resident_ctas(int which, int H, bool w2_tma, int chunk, bool int8w);
+int experts_resident_ctas(int which, int H, bool w2_tma, int chunk, bool int8w, bool occ2 = false);
 // Whether the gate/up (down) projection takes the TMA-ring kernel for this shape.
 bool experts_w13_tma(int H);
 // Whether the large-batch streaming sequence runs gate/up on the tcgen05
