@@ -490,7 +490,27 @@ __global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(32 *
             s_logit[tt][e - e_lo] = v;
         }
     }
-    for (int e = e_lo + warp, j = 0; !split && e < e_hi; e += kRouterWarps, ++j) {
+    // Each warp's one expert row in registers (wpre): a rolled loop over the
+    // group's tokens, each in the block order of the general loop below.  The
+    // kernel runs once per layer with its code cold in the instruction cache;
+    // the rolled loop is a short stretch of code, fetched once (measured:
+    // Nano stack T = 16 0.760 -> 0.741 ms, T = 64 0.955 -> 0.944 ms).
+    const bool w_in_regs = !split && nblk <= kRouterBatch && epc <= kRouterWarps;
+    if (w_in_regs) {
+        const int e = e_lo + warp;
+        if (e < e_hi) {
+#pragma unroll 1
+            for (int tt = 0; tt < nt; ++tt) {
+                float acc = 0.f;
+#pragma unroll
+                for (int i = 0; i < kRouterBatch; ++i)
+                    if (i < nblk) acc = dot_step(acc, xblock(tt, i), wpre[i]);
+                const float v = warp_sum_tree(acc);
+                if (lane == 0) s_logit[tt][e - e_lo] = v;
+            }
+        }
+    }
+    for (int e = e_lo + warp, j = 0; !split && !w_in_regs && e < e_hi; e += kRouterWarps, ++j) {
         float acc[kDecodeRouterTok];
 #pragma unroll
         for (int tt = 0; tt < kDecodeRouterTok; ++tt) acc[tt] = 0.f;
