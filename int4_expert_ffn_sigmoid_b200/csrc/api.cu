@@ -153,19 +153,15 @@ int sm_count() {
 
 inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
 
-// Default choice of the fused kernel: where it was measured faster than one
-// moe_layer_forward per layer (the 23-layer Nano stack: 0.56 against 0.58 ms
-// at T = 1, 0.58 against 0.59 at T = 4, 0.79 against 0.73 at T = 16, equal
-// at T = 64; one 6144-hidden layer: slower at T = 1 and 32).
-constexpr int kFusedDefaultMaxT = 4;
-constexpr int kFusedDefaultMaxH = 2048;
-
-// Whether a stack call takes the fused kernel.
+// Whether a stack call takes the fused kernel: only under MOE_STACK_FUSED.
+// One moe_layer_forward per layer was measured faster at every T (the
+// 23-layer Nano stack: 0.507 against 0.561 ms at T = 1, 0.543 against 0.574
+// at T = 4, 0.725 against 0.790 at T = 16, 0.926 against 1.008 at T = 64;
+// one 6144-hidden layer: 0.084 against 0.123 ms at T = 1).
 bool stack_fused(const moe_cfg_t& c, int32_t T, int32_t L) {
     if (c.flags & (MOE_FORCE_DECODE | MOE_FORCE_PREFILL | MOE_WEIGHTS_INT8)) return false;
     if (!(fused_supported(c.H, c.E, c.K, c.I, c.Is, T, L) && fused_grid() > 0)) return false;
-    if (c.flags & MOE_STACK_FUSED) return true;
-    return L >= 2 && T <= kFusedDefaultMaxT && c.H <= kFusedDefaultMaxH;
+    return (c.flags & MOE_STACK_FUSED) != 0;
 }
 
 // Workspace of the fused kernel: a zeroed control block and counters, then

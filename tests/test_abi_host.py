@@ -267,10 +267,10 @@ def test_stack_validation_codes(moe):
     assert moe.stack_workspace_bytes(s, 64, 0) == 0
     # without a GPU the fused kernel cannot be resident: every call takes the per-layer path
     assert moe.stack_path(s, 0, 23) == 0
-    assert moe.stack_path(s, 4, 23) in (moe.MOE_PATH_FUSED_STACK, moe.MOE_PATH_PER_LAYER)
     assert moe.stack_path(s, 16, 23, moe.MOE_STACK_FUSED) in (moe.MOE_PATH_FUSED_STACK, moe.MOE_PATH_PER_LAYER)
-    # the default takes the fused kernel only for L >= 2, T <= 4, H <= 2048 (measured faster there)
-    assert moe.stack_path(s, 16, 23) == moe.MOE_PATH_PER_LAYER
+    # without MOE_STACK_FUSED every stack runs one layer call per layer (measured faster at every T)
+    for T in (1, 4, 16, 64):
+        assert moe.stack_path(s, T, 23) == moe.MOE_PATH_PER_LAYER
     assert moe.stack_path(s, 4, 1) == moe.MOE_PATH_PER_LAYER
     assert moe.stack_path(s, 100, 23, moe.MOE_STACK_FUSED) == moe.MOE_PATH_PER_LAYER  # beyond 64 tokens
     assert moe.stack_path(s, 16, 23, moe.MOE_FORCE_DECODE) == moe.MOE_PATH_PER_LAYER

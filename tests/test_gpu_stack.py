@@ -31,7 +31,7 @@ def run_stack(moe, x, stacked, shape, flags=0):
     T = x.shape[0]
     idx = torch.empty((L, T, shape.K), dtype=torch.int32, device=x.device)
     w = torch.empty((L, T, shape.K), dtype=torch.float32, device=x.device)
-    # the fused kernel wherever it serves the call (the default takes it only at T <= 4)
+    # the fused kernel wherever it serves the call (opt-in: the default runs one layer call per layer)
     outs = moe.stack_forward(x, stacked, shape, flags=flags | moe.MOE_DEBUG_CHECK | moe.MOE_STACK_FUSED, topk_idx=idx,
                              topk_w=w)
     torch.cuda.synchronize()
