@@ -93,6 +93,10 @@ __device__ __forceinline__ void tile_hexp(const Params& p, int t0, int nt, int w
 // k-th pick is scale * s_k / (s_0 + ... + s_{K-1}).  Writes idx / wts (and
 // the optional user outputs) of token t; returns, on lanes k < K, the k-th
 // selected expert (else -1).
+// kKUnroll: unrolling of the loop over the K picks (1 where the selection
+// runs once per launch, its code cold in the instruction cache: a short
+// rolled loop is fetched once).
+template <int kKUnroll = kMaxK>
 __device__ int select_from_logits(const Params& p, int t, const float (&L)[kMaxE / 32], const float* bias, int lane) {
     const int E = p.E, K = p.K;
     float key[kMaxE / 32], sc[kMaxE / 32];
@@ -111,7 +115,7 @@ __device__ int select_from_logits(const Params& p, int t, const float (&L)[kMaxE
     unsigned taken = 0;
     int my_e = -1;
     float my_s = 0.f, ssum = 0.f;
-#pragma unroll
+#pragma unroll kKUnroll
     for (int k = 0; k < kMaxK; ++k) {
         if (k >= K) break;
         float bk = -INFINITY, bs = 0.f;
@@ -553,7 +557,7 @@ __global__ void __cluster_dims__(1, kDecodeRouterCtas, 1) __launch_bounds__(32 *
                     L[jj] = *cluster.map_shared_rank(&s_logit[warp][e - src * epc], src);
                 }
             }
-            const int sel = select_from_logits(p, t0 + warp, L, s_bias, lane);
+            const int sel = select_from_logits<1>(p, t0 + warp, L, s_bias, lane);
             if (lane < K) s_pick[warp * K + lane] = sel;
         }
         __syncthreads();
