@@ -253,9 +253,10 @@ def stage_work(stage, shape, T, uniq, wbits=4):
 
 class Runner:
     """A workload's weights and the buffers of one T, with one step = one pass
-    of every layer over one batch: either ONE moe_stack_forward call (the fused
-    stack kernel; mode "fused") or one moe_layer_forward call per layer (mode
-    "per_layer")."""
+    of every layer over one batch: ONE moe_stack_forward call, either the
+    fused stack kernel (mode "fused") or one layer call per layer inside the
+    library (mode "per_layer"; the instrumented pass and the routing count
+    call moe_layer_forward per layer themselves)."""
 
     def __init__(self, moe, wl, T, device, stacked, mode, extra_flags=0):
         self.moe, self.wl, self.T, self.device, self.mode = moe, wl, T, device, mode
@@ -279,6 +280,8 @@ class Runner:
         if self.mode == "fused":
             self.moe.stack_forward(inp, self.stacked, self.shape, outs=self.outs, workspace=self.ws, flags=self.flags,
                                    topk_idx=topk_idx)
+        elif stage_events is None and topk_idx is None:
+            self.moe.stack_forward(inp, self.stacked, self.shape, outs=self.outs, workspace=self.ws, flags=self.flags)
         else:
             # a per-layer slice of [L][T][K] need not be 16-byte aligned: one [T][K] buffer per call
             one = None if topk_idx is None else torch.empty_like(topk_idx[0])
