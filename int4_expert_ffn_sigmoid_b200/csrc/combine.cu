@@ -14,18 +14,32 @@
 namespace moe {
 
 __global__ void __launch_bounds__(256) combine_kernel(Params p) {
+    __shared__ int s_slot[kMaxK];
+    __shared__ float s_w[kMaxK];
     const int t = blockIdx.x;
     const int j = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
+    const int K = p.K, H = p.H;
+    // The token's slots and routing weights, and its residual row, are final
+    // before this kernel starts: the kernel it waits for (the down
+    // projection) started only after the one before it had completed, and
+    // those were written there or earlier (the bucket tables, the router, the
+    // caller).  Only the expert outputs need the wait.
+    if (threadIdx.x < K) {
+        s_slot[threadIdx.x] = __ldcg(p.slot_of + (size_t)t * K + threadIdx.x);
+        s_w[threadIdx.x] = __ldcg(p.wts + (size_t)t * K + threadIdx.x);
+    }
+    const bool res = (p.flags & kFlagResidual) && j < H;
+    const uint2 xv = res ? __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)t * H + j)) : make_uint2(0u, 0u);
     pdl_wait();
     pdl_release();
-    if (j >= p.H) return;
-    const int K = p.K, H = p.H;
+    __syncthreads();
+    if (j >= H) return;
     const size_t TK = (size_t)p.T * K;
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     for (int k = 0; k < K; ++k) {
-        const int s = __ldcg(p.slot_of + (size_t)t * K + k);
+        const int s = s_slot[k];
         if (s < 0) continue;  // a pick the top-p dropped
-        const float w = __ldcg(p.wts + (size_t)t * K + k);
+        const float w = s_w[k];
         float4 v = __ldcg(reinterpret_cast<const float4*>(p.y + (size_t)s * H + j));
         for (int sl = 1; sl < p.nsl_r; ++sl) {
             const float4 u = __ldcg(reinterpret_cast<const float4*>(p.y + (sl * TK + s) * H + j));
@@ -45,8 +59,7 @@ __global__ void __launch_bounds__(256) combine_kernel(Params p) {
         }
         a0 += v.x; a1 += v.y; a2 += v.z; a3 += v.w;
     }
-    if (p.flags & kFlagResidual) {
-        const uint2 xv = __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)t * H + j));
+    if (res) {
         a0 += bf16lo(xv.x); a1 += bf16hi(xv.x); a2 += bf16lo(xv.y); a3 += bf16hi(xv.y);
     }
     if (p.flags & kFlagOutF32) {
