@@ -412,6 +412,12 @@ int moe_layer_forward(const void* x, const float* router_w, const float* router_
         const long long cap2 = experts_resident_ctas(1, cfg->H, w2_tma, p.chunk, int8w);
         grid13 = (int)(tasks13 < cap13 ? tasks13 : cap13);
         grid2 = (int)(tasks2 < cap2 ? tasks2 : cap2);
+        // The TMA down kernel builds its tables before its wait where its CTAs
+        // can start while the gate/up kernel still runs: SMs the gate/up grid
+        // leaves free, or the two-CTAs-per-SM gate/up's uneven finish
+        // (measured on the Nano stack: T = 1 0.481 -> 0.444 ms, T = 64 0.905
+        // -> 0.871 ms; with one gate/up CTA on every SM, T = 16, 1.8% slower)
+        p.w2_tables_early = small && w2_tma && (grid13 < sm_count() || p.w13_occ2);
     }
 
     void* const* ev = cfg->stage_events;

@@ -141,24 +141,25 @@ __device__ __forceinline__ void load_tables(const Params& p, const int32_t* ts, 
     __syncthreads();
 }
 
-// Small-batch path, gate/up kernel: the bucket list, the gate/up task prefix
-// and the token of every routed slot, from the router's per-group pick
-// counts (hist), picks (idx) and ranks.  The slot of pick (t, k) of expert e
-// is offset[e] + (picks of e in the groups before t's) + rank[t, k].  CTA 0
-// also writes the bucket list, the down-task prefix, slot_of and tok_of_slot
-// to the workspace.
-__device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
+// Small-batch path, from the router's per-group pick counts (hist), picks
+// (idx) and ranks.  kind 0 (gate/up kernel): the bucket list, the gate/up
+// task prefix and the token of every routed slot; the slot of pick (t, k) of
+// expert e is offset[e] + (picks of e in the groups before t's) + rank[t, k],
+// and CTA 0 also writes the bucket list, the down-task prefix, slot_of and
+// tok_of_slot to the workspace.  kind 1 (down kernel): the bucket list and
+// the down-task prefix only, with no write to global memory.
+__device__ void build_tables_small(const Params& p, Shm& sh, int* scratch, int kind = 0) {
     int* s_base = scratch;  // [kDecodeGroups][kMaxE]
     int* s_cnt = scratch + kDecodeGroups * kMaxE;
     int* s_off = s_cnt + kMaxE;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = p.E, K = p.K, T = p.T, TK = T * K, G = p.decode_groups;
-    const bool writer = blockIdx.x == 0;
+    const bool writer = kind == 0 && blockIdx.x == 0;
     Tables& tb = sh.tb;
     int my_e[2], my_rank[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {  // threads 0..255 cover the T*K <= 512 picks
-        const int i = tid < 256 ? tid + 256 * u : TK;
+        const int i = tid < 256 && kind == 0 ? tid + 256 * u : TK;
         my_e[u] = i < TK ? __ldcg(p.idx + i) : -1;
         my_rank[u] = i < TK ? __ldcg(p.rank + i) : 0;
     }
@@ -174,7 +175,8 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
         }
         s_cnt[tid] = run;
     }
-    for (int i = tid; i < kMaxSlots; i += blockDim.x) sh.tok[i] = -1;
+    if (kind == 0)
+        for (int i = tid; i < kMaxSlots; i += blockDim.x) sh.tok[i] = -1;
     __syncthreads();
     if (warp == 0) {
         // lane l owns experts 8l .. 8l+7: counts, non-empty buckets, gate/up
@@ -210,7 +212,7 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
                     tb.e[b] = e;
                     tb.n[b] = c[j];
                     tb.off[b] = off;
-                    tb.ts[b] = b13;
+                    tb.ts[b] = kind == 0 ? b13 : b2;
                     if (writer) {
                         p.bucket_e[b] = e;
                         p.bucket_n[b] = c[j];
@@ -238,7 +240,7 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
                 tb.e[nb] = E;
                 tb.n[nb] = T;
                 tb.off[nb] = TK;
-                tb.ts[nb] = t13;
+                tb.ts[nb] = kind == 0 ? t13 : t2;
                 if (writer) {
                     p.bucket_e[nb] = E;
                     p.bucket_n[nb] = T;
@@ -249,9 +251,9 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
                 t2 += (p.H / p.rows2) * slices_of(p.Is) * chunks_of(T, p.chunk);
                 ++nb;
             }
-            tb.ts[nb] = t13;
+            tb.ts[nb] = kind == 0 ? t13 : t2;
             tb.n_buckets = nb;
-            tb.ntask = t13;
+            tb.ntask = kind == 0 ? t13 : t2;
             if (writer) {
                 p.ts2[nb] = t2;
                 p.ctrl->n_buckets = nb;
@@ -261,8 +263,8 @@ __device__ void build_tables_small(const Params& p, Shm& sh, int* scratch) {
     }
     __syncthreads();
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const int i = tid < 256 ? tid + 256 * u : TK;
+    for (int u = 0; u < 2; ++u) {  // the slots (kind 0)
+        const int i = tid < 256 && kind == 0 ? tid + 256 * u : TK;
         if (i >= TK) continue;
         const int e = my_e[u], t = i / K;
         if (e == -1 && p.topp > 0.f && p.topp < 1.f) {  // dropped by the top-p: no slot
@@ -1785,6 +1787,7 @@ struct Tma2 {
     static constexpr size_t kRsOff = kRawOff + (size_t)kChunk * kSliceK * 4;
     static constexpr size_t kSmem = kShmBytes + kW2MiscBytes + 1024 /* alignment */ + kRsOff + (size_t)2 * kMaxRows2 * 4;
     static_assert(kSmem <= 227 * 1024, "TMA down shared memory");
+    static_assert(kRsOff - kXOff >= kBuildBytes, "table build scratch fits the activation and h staging");
 };
 
 __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
@@ -1942,10 +1945,21 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
             }
     }
     if (p.Is > 0) prefetch_l2_slice(p.sh_w2, (size_t)p.H * p.Is * WB / 8);
+    // Small batches can build the down tables from the router's outputs before
+    // the wait: the router completed before the gate/up kernel that this one
+    // waits for released it (scratch: the activation and h staging areas,
+    // unused until the first task).
+    const bool early = p.decode_groups > 0 && p.w2_tables_early;
+    if (early) {
+        build_tables_small(p, sh, reinterpret_cast<int*>(xs), 1);
+        precompute_tasks(p, sh, 1);
+    }
     pdl_wait();
     pdl_release();
-    load_tables(p, p.ts2, &p.ctrl->tasks2, sh.tb, nullptr);
-    precompute_tasks(p, sh, 1);
+    if (!early) {
+        load_tables(p, p.ts2, &p.ctrl->tasks2, sh.tb, nullptr);
+        precompute_tasks(p, sh, 1);
+    }
     if (threadIdx.x == 0 && pre) {  // cannot fail with consistent tables
         const TaskDesc d = sh.td[0];
         if (!(d.e == p.E && d.rbk == pre_rbk && d.sl == pre_sl && d.tok0 == pre_tok0 &&

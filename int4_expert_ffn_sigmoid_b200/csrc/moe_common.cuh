@@ -221,6 +221,7 @@ struct Params {
     int chunk;            // tokens per weight-streaming task: kChunkTokens or kMaxChunk
     int w13_occ2;         // gate/up on the two-CTAs-per-SM TMA-ring kernel (16-token tasks, int4)
     int decode_groups;    // token groups of the small-batch router (0: tables come from the large router)
+    int w2_tables_early;  // small batch: the down kernel builds its tables before its wait
     float* lpart;         // [lslices][T][E] partial router logits (split router or tensor-core router)
     int lslices;          // hidden-dimension slices of lpart (0: the selecting router computes its logits)
     __nv_bfloat16* wsplit;  // [3][E][H] router weights as exact bf16 terms hi, mid, lo (tensor-core router)
