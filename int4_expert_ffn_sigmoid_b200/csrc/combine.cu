@@ -23,23 +23,28 @@ __global__ void __launch_bounds__(256) combine_kernel(Params p) {
     // before this kernel starts: the kernel it waits for (the down
     // projection) started only after the one before it had completed, and
     // those were written there or earlier (the bucket tables, the router, the
-    // caller).  Only the expert outputs need the wait.
-    if (threadIdx.x < K) {
+    // caller).  Small batches, bound by the latency of this chain, read them
+    // before the wait (measured: Nano stack T = 64 0.924 -> 0.907 ms); large
+    // ones, with thousands of CTAs in flight, read them in the loop (the
+    // staging barrier made the T = 16384 combine 72 -> 86 us).
+    const bool early = p.decode_groups > 0;
+    if (early && threadIdx.x < K) {
         s_slot[threadIdx.x] = __ldcg(p.slot_of + (size_t)t * K + threadIdx.x);
         s_w[threadIdx.x] = __ldcg(p.wts + (size_t)t * K + threadIdx.x);
     }
     const bool res = (p.flags & kFlagResidual) && j < H;
-    const uint2 xv = res ? __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)t * H + j)) : make_uint2(0u, 0u);
+    uint2 xv = early && res ? __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)t * H + j)) : make_uint2(0u, 0u);
     pdl_wait();
     pdl_release();
-    __syncthreads();
+    if (early) __syncthreads();
     if (j >= H) return;
+    if (!early && res) xv = __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)t * H + j));
     const size_t TK = (size_t)p.T * K;
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     for (int k = 0; k < K; ++k) {
-        const int s = s_slot[k];
+        const int s = early ? s_slot[k] : __ldcg(p.slot_of + (size_t)t * K + k);
         if (s < 0) continue;  // a pick the top-p dropped
-        const float w = s_w[k];
+        const float w = early ? s_w[k] : __ldcg(p.wts + (size_t)t * K + k);
         float4 v = __ldcg(reinterpret_cast<const float4*>(p.y + (size_t)s * H + j));
         for (int sl = 1; sl < p.nsl_r; ++sl) {
             const float4 u = __ldcg(reinterpret_cast<const float4*>(p.y + (sl * TK + s) * H + j));
